@@ -1,0 +1,441 @@
+"""CPU oracle for the weight-only-quantized decode path.
+
+TEST INFRASTRUCTURE ONLY. Only the tests, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this module. It shares no code
+with the CUDA library and never imports it; the product path never calls it.
+
+Everything is plain numpy in float64, written from the definitions on the
+source pages, one step after another in the order the pages run them. Library
+primitives (a dot product, a matmul) stand in for single steps only. Where
+the GPU stores a value in bf16, the oracle rounds the float64 value to bf16
+(round to nearest even) at the same point; everything else stays float64.
+
+Sources (cited per function):
+  [TS] turbospark-runtime 0.3.0, src/qwen3_asr_metal.rs -- resident packed
+       affine-INT8 (group 64) Qwen3 text decoder.
+  [FT] fuel-transformers 0.19.1, src/models/lazy_quantized_whisper.rs --
+       GGUF Q4_0 Whisper (Q4_0 bake and forward).
+  [MK] makima commit eabd130 "Add Qwen3-TTS streaming endpoint",
+       src/tts/qwen3/model.rs and src/tts/qwen3/config.rs -- unquantized
+       candle Qwen3 decoder (RoPE, attention, MLP, layer order, defaults).
+
+Every function is pinned by a ``-m "not gpu"`` test in tests/test_oracle_*.py
+against something other than itself (closed forms, a worked example, a
+library routine, brute force, invariants). No function here is parity
+unpinned.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+GROUP = 64
+QK4_0 = 32
+Q4_0_BLOCK_BYTES = 18
+
+# ---------------------------------------------------------------------------
+# Number formats
+# ---------------------------------------------------------------------------
+
+_BF16_MIN_EXP = -125      # frexp exponent of the smallest normal bf16 (2**-126)
+_BF16_SIG_BITS = 8        # significant bits of bf16 (7 stored + 1 implicit)
+
+
+def _bf16_quantize(v, how):
+    """Round float64 values onto the bf16 grid with the integer rounding
+    function ``how`` (np.rint = nearest-even, np.floor, np.ceil)."""
+    v = np.asarray(v, dtype=np.float64)
+    out = v.copy()
+    fin = np.isfinite(v) & (v != 0)
+    _, e = np.frexp(v[fin])                       # v = m * 2**e, 0.5 <= |m| < 1
+    e = np.maximum(e, _BF16_MIN_EXP)              # fixed quantum below the normal range
+    r = np.ldexp(how(np.ldexp(v[fin], _BF16_SIG_BITS - e)), e - _BF16_SIG_BITS)
+    r = np.where(np.abs(r) >= 2.0 ** 128, np.copysign(np.inf, r), r)
+    out[fin] = r
+    return out
+
+
+def round_bf16(v):
+    """float64 -> nearest bf16 value (ties to even), returned as float64."""
+    return _bf16_quantize(v, np.rint)
+
+
+def round_bf16_down(v):
+    """float64 -> largest bf16 value <= v."""
+    return _bf16_quantize(v, np.floor)
+
+
+def round_bf16_up(v):
+    """float64 -> smallest bf16 value >= v."""
+    return _bf16_quantize(v, np.ceil)
+
+
+def bf16_bits_to_f64(bits):
+    """bf16 bit patterns (uint16) -> float64 values (exact)."""
+    b = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16
+    with np.errstate(invalid="ignore"):
+        return b.view(np.float32).astype(np.float64)
+
+
+def bf16_value_to_bits(v):
+    """bf16-representable float64 values -> uint16 bit patterns."""
+    f = np.asarray(v, dtype=np.float64).astype(np.float32)
+    return (f.view(np.uint32) >> 16).astype(np.uint16)
+
+
+def f16_bits_to_f64(bits):
+    """IEEE binary16 bit patterns -> float64 (exact)."""
+    return np.asarray(bits, dtype=np.uint16).view(np.float16).astype(np.float64)
+
+
+# ---------------------------------------------------------------------------
+# Affine-INT8, group 64  [TS: PackedLinear, load_packed_linear, embed_row_bytes]
+# ---------------------------------------------------------------------------
+
+def affine8_quantize(w):
+    """Quantize float weights ``w [N, K]`` to the affine-INT8 g64 format.
+
+    The pages only read checkpoints that arrive already packed ([TS]
+    ``open`` checks ``quantization_config {bits 8, group_size 64, mode
+    affine}``), so the quantizer is this library's reading: per group of 64,
+    bias = bf16 rounded down from the group minimum, scale = bf16 rounded up
+    from (max - bias) / 255, code = nearest integer of (w - bias) / scale
+    clamped to [0, 255]. The directed roundings keep every weight inside
+    [bias, bias + 255 * scale], so |w - dequant| <= scale / 2.
+
+    Returns (words uint32 [N, K/4], scales uint16 [N, K/64], biases uint16).
+    """
+    w = np.asarray(w, dtype=np.float64)
+    N, K = w.shape
+    assert K % GROUP == 0
+    g = w.reshape(N, K // GROUP, GROUP)
+    lo = g.min(axis=2)
+    hi = g.max(axis=2)
+    bias = round_bf16_down(lo)
+    scale = round_bf16_up((hi - bias) / 255.0)
+    scale = np.where(scale > 0, scale, 2.0 ** -126)
+    q = np.rint((g - bias[:, :, None]) / scale[:, :, None])
+    q = np.clip(q, 0, 255).astype(np.uint8).reshape(N, K)
+    return affine8_pack(q), bf16_value_to_bits(scale), bf16_value_to_bits(bias)
+
+
+def affine8_pack(q):
+    """Pack byte codes ``q [N, K]`` into u32 words ``[N, K/4]``: column
+    ``4*j + i`` is byte ``i`` (bits 8i..8i+7) of word ``j`` -- the U32
+    ``[rows, cols/4]`` tensor holding ``rows * cols`` bytes of [TS]
+    ``load_packed_linear``, read byte-per-column by ``embed_row_bytes``."""
+    q = np.asarray(q, dtype=np.uint8)
+    N, K = q.shape
+    words = np.zeros((N, K // 4), dtype=np.uint64)
+    for i in range(4):
+        words |= q[:, i::4].astype(np.uint64) << np.uint64(8 * i)
+    return words.astype(np.uint32)
+
+
+def affine8_unpack(words):
+    """Inverse of ``affine8_pack``: u32 words ``[N, K/4]`` -> byte codes ``[N, K]``."""
+    words = np.asarray(words, dtype=np.uint32).astype(np.uint64)
+    N, W = words.shape
+    q = np.zeros((N, 4 * W), dtype=np.uint8)
+    for i in range(4):
+        q[:, i::4] = ((words >> np.uint64(8 * i)) & np.uint64(0xFF)).astype(np.uint8)
+    return q
+
+
+def affine8_dequant_exact(words, scales, biases):
+    """Exact dequantized weights in float64: ``w = q * scale + bias`` with
+    the group of column c being c // 64 ([TS] ``embed_row_bytes``). The
+    product and sum are exact in float64 (8-bit code times 8-bit bf16
+    significand, then one add)."""
+    q = affine8_unpack(words).astype(np.float64)
+    N, K = q.shape
+    s = np.repeat(bf16_bits_to_f64(scales), GROUP, axis=1)
+    b = np.repeat(bf16_bits_to_f64(biases), GROUP, axis=1)
+    assert s.shape == (N, K)
+    return q * s + b
+
+
+def affine8_dequant_f32(words, scales, biases):
+    """Dequantized weights as float32 values: the exact value rounded once
+    to float32 (what a float32 ``q * s + b`` gives, since ``q * s`` is
+    exact in float32)."""
+    return affine8_dequant_exact(words, scales, biases).astype(np.float32)
+
+
+def gemv_affine8(words, scales, biases, x, residual=None):
+    """``y[b, r] = sum_c (q[r,c] * s[r, c//64] + beta[r, c//64]) * x[b, c]``
+    (+ ``residual[b, r]``). The GEMV of [TS] ``step`` (every packed linear,
+    no linear bias), accumulated in float64. ``x`` is ``[B, K]`` float64."""
+    w = affine8_dequant_exact(words, scales, biases)
+    y = np.asarray(x, dtype=np.float64) @ w.T
+    if residual is not None:
+        y = y + np.asarray(residual, dtype=np.float64)
+    return y
+
+
+def embed_rows(words, scales, biases, token_ids):
+    """Tied-embedding lookup: dequantize one packed row per token ([TS]
+    ``embed_row_bytes``; the same table is the LM head). Returns the float32
+    residual-stream rows as float64 values."""
+    ids = np.asarray(token_ids, dtype=np.int64)
+    return affine8_dequant_f32(words[ids], scales[ids], biases[ids]).astype(np.float64)
+
+
+# ---------------------------------------------------------------------------
+# GGUF Q4_0  [FT: quantize_in_out_to_q4_0, q_linear]
+# ---------------------------------------------------------------------------
+
+def q4_0_quantize(x):
+    """Quantize float32 rows ``x [N, K]`` into Q4_0 blocks as ggml's
+    ``BlockQ4_0::from_float`` does (named by [FT]
+    ``quantize_in_out_to_q4_0``): per block of 32, ``m`` = the element of
+    largest magnitude (first one on ties, sign kept), ``d = m / -8``,
+    ``id = 1/d`` (0 when d == 0), code ``n = min(15, trunc(x * id + 8.5))``;
+    stored as fp16 ``d`` followed by 16 bytes, byte j holding code j in its
+    low nibble and code j+16 in its high nibble. All arithmetic in float32
+    as ggml runs it. Returns uint8 ``[N, (K/32) * 18]``."""
+    x = np.asarray(x, dtype=np.float32)
+    N, K = x.shape
+    assert K % QK4_0 == 0
+    blk = x.reshape(N, K // QK4_0, QK4_0)
+    idx = np.argmax(np.abs(blk), axis=2)                     # first index of max |x|
+    m = np.take_along_axis(blk, idx[:, :, None], axis=2)[:, :, 0]
+    m = np.where(np.abs(m) > 0, m, np.float32(0.0))   # the running max starts at +0
+    d = (m / np.float32(-8.0)).astype(np.float32)
+    with np.errstate(divide="ignore"):
+        inv = np.where(d != 0, np.float32(1.0) / d, np.float32(0.0)).astype(np.float32)
+    v = (blk * inv[:, :, None]).astype(np.float32) + np.float32(8.5)
+    n = np.minimum(15, np.trunc(v.astype(np.float32))).astype(np.uint8)
+    out = np.empty((N, K // QK4_0, Q4_0_BLOCK_BYTES), dtype=np.uint8)
+    out[:, :, 0:2] = d.astype(np.float16).view(np.uint8).reshape(N, K // QK4_0, 2)
+    out[:, :, 2:] = n[:, :, :16] | (n[:, :, 16:] << 4)
+    return out.reshape(N, (K // QK4_0) * Q4_0_BLOCK_BYTES)
+
+
+def q4_0_unpack(blocks, K):
+    """Q4_0 bytes ``[N, (K/32)*18]`` -> (fp16 ``d`` as float64 ``[N, K/32]``,
+    codes ``n`` uint8 ``[N, K]``), codes in column order."""
+    b = np.asarray(blocks, dtype=np.uint8)
+    N = b.shape[0]
+    nb = K // QK4_0
+    b = b.reshape(N, nb, Q4_0_BLOCK_BYTES)
+    d = f16_bits_to_f64(b[:, :, 0:2].copy().view(np.uint16)[:, :, 0])
+    lo = b[:, :, 2:] & 0x0F
+    hi = b[:, :, 2:] >> 4
+    n = np.concatenate([lo, hi], axis=2).reshape(N, K)
+    return d, n
+
+
+def q4_0_dequant_exact(blocks, K):
+    """``w = d * (n - 8)`` (exact in float64 and in float32)."""
+    d, n = q4_0_unpack(blocks, K)
+    return np.repeat(d, QK4_0, axis=1) * (n.astype(np.float64) - 8.0)
+
+
+def gemv_q4_0(blocks, x, bias=None):
+    """Q4_0 linear of [FT] ``q_linear``: ``y = x @ W^T (+ bias)``, float64
+    accumulation. ``x`` is ``[B, K]``."""
+    x = np.asarray(x, dtype=np.float64)
+    w = q4_0_dequant_exact(blocks, x.shape[1])
+    y = x @ w.T
+    if bias is not None:
+        y = y + np.asarray(bias, dtype=np.float64)[None, :]
+    return y
+
+
+def gemm_q4_0_bf16(blocks, A, bias=None):
+    """The M-row Q4_0 matmul of the Whisper encoder ([FT] ``encoder_layer``
+    -> ``q_linear``) under this library's tensor-core operand contract: the
+    float32 activations and the dequantized weights are each rounded to bf16
+    (nearest even) before the product; accumulation is float64."""
+    A = round_bf16(np.asarray(A, dtype=np.float64))
+    w = round_bf16(q4_0_dequant_exact(blocks, A.shape[1]))
+    C = A @ w.T
+    if bias is not None:
+        C = C + np.asarray(bias, dtype=np.float64)[None, :]
+    return C
+
+
+# ---------------------------------------------------------------------------
+# Elementwise pieces  [TS: step; MK: model.rs]
+# ---------------------------------------------------------------------------
+
+def rmsnorm(x, w_bits, eps):
+    """``y = x / sqrt(mean(x^2) + eps) * w`` over the last axis; ``w`` bf16
+    ([TS] ``encode_rms_norm_bf16w`` calls; [MK] ``rms_norm`` layers)."""
+    x = np.asarray(x, dtype=np.float64)
+    w = bf16_bits_to_f64(w_bits)
+    ms = np.mean(x * x, axis=-1, keepdims=True)
+    return x / np.sqrt(ms + eps) * w
+
+
+def rmsnorm_perhead(x, w_bits, eps, D):
+    """Per-head RMSNorm (Qwen3 q_norm / k_norm): the norm of ``rmsnorm``
+    applied to every ``D``-wide head slice with one shared ``[D]`` weight
+    ([TS] ``encode_rms_norm_bf16w_perhead``; [MK] ``apply_head_norm``)."""
+    x = np.asarray(x, dtype=np.float64)
+    shp = x.shape
+    return rmsnorm(x.reshape(shp[:-1] + (shp[-1] // D, D)), w_bits, eps).reshape(shp)
+
+
+def rope_inv_freq(theta, rotary_dim):
+    """``inv_freq_i = theta^(-2i / rotary_dim)`` for ``i < rotary_dim/2``
+    ([MK] ``RotaryEmbedding::new``)."""
+    i = np.arange(rotary_dim // 2, dtype=np.float64)
+    return theta ** (-2.0 * i / rotary_dim)
+
+
+def rope_neox(x, pos, theta, D, rotary_dim=None):
+    """NeoX (rotate-half) RoPE on each ``D``-wide head of ``x [..., heads*D]``
+    at integer position ``pos`` ([MK] ``RotaryEmbedding::apply`` /
+    ``rotate_half``; [TS] ``encode_rope_neox_subdim`` with rotary_dim =
+    head_dim). With angle ``a_i = pos * inv_freq_i`` and half = rotary_dim/2:
+    ``out_i = x_i cos a_i - x_{i+half} sin a_i`` and
+    ``out_{i+half} = x_{i+half} cos a_i + x_i sin a_i``; dims at or beyond
+    ``rotary_dim`` pass through."""
+    rd = D if rotary_dim is None else rotary_dim
+    x = np.asarray(x, dtype=np.float64)
+    shp = x.shape
+    h = x.reshape(shp[:-1] + (shp[-1] // D, D)).copy()
+    half = rd // 2
+    a = float(pos) * rope_inv_freq(theta, rd)
+    c, s = np.cos(a), np.sin(a)
+    x1 = h[..., :half].copy()
+    x2 = h[..., half:rd].copy()
+    h[..., :half] = x1 * c - x2 * s
+    h[..., half:rd] = x2 * c + x1 * s
+    return h.reshape(shp)
+
+
+def silu_mul(gate, up):
+    """``silu(gate) * up`` with ``silu(z) = z / (1 + exp(-z))`` ([TS]
+    ``encode_silu_mul``; [MK] ``Qwen3Mlp::forward``)."""
+    g = np.asarray(gate, dtype=np.float64)
+    return g / (1.0 + np.exp(-g)) * np.asarray(up, dtype=np.float64)
+
+
+def decode_attention(q, k_cache, v_cache, kv_len, H, Hkv, D, scale=None):
+    """Decode attention of one query row per sequence over the first
+    ``kv_len`` cached rows ([TS] ``encode_attention_decode`` with
+    ``kv_start = 0``; [MK] ``Qwen3Attention::forward``). Query head h reads
+    KV head ``h // (H / Hkv)`` ([MK] ``repeat_kv``); scores are
+    ``q . k_t * scale`` with ``scale = 1/sqrt(D)``; softmax over all
+    ``kv_len`` scores in float64 (no splitting).
+
+    q ``[H*D]``; k_cache, v_cache ``[Hkv, >= kv_len, D]`` float64 values.
+    Returns ``[H*D]``.
+    """
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    q = np.asarray(q, dtype=np.float64).reshape(H, D)
+    g = H // Hkv
+    out = np.zeros((H, D))
+    for h in range(H):
+        kh = h // g
+        K_ = k_cache[kh, :kv_len, :]
+        V_ = v_cache[kh, :kv_len, :]
+        s = (K_ @ q[h]) * scale
+        p = np.exp(s - s.max())
+        p = p / p.sum()
+        out[h] = p @ V_
+    return out.reshape(H * D)
+
+
+def argmax_first(logits):
+    """Index of the first strict maximum, NaNs skipped (fold from -inf,
+    replace only on ``>``) -- [TS] ``argmax``. 0 when nothing beats -inf."""
+    best_i, best_v = 0, -math.inf
+    for i, v in enumerate(np.asarray(logits, dtype=np.float64).tolist()):
+        if v > best_v:
+            best_i, best_v = i, v
+    return best_i
+
+
+# ---------------------------------------------------------------------------
+# The decode step  [TS: step]
+# ---------------------------------------------------------------------------
+
+def decode_step(cfg, weights, k_cache, v_cache, token, pos):
+    """One token of one sequence through every layer, in the op order of
+    [TS] ``step``: input norm -> q, k, v GEMVs -> per-head q/k norm -> NeoX
+    RoPE on q and on k -> K/V written at cache row ``pos`` -> attention over
+    rows ``[0, pos]`` -> o_proj -> residual add -> post-attention norm ->
+    gate, up -> SiLU-mul -> down -> residual add; then the final norm and
+    the tied LM head. The embedding row is the dequantized packed row of
+    [TS] ``embed_row_bytes``.
+
+    Precision points (where the GPU stores bf16, rounded here as well):
+    norm outputs feeding a GEMV, K and V written to the cache, the attention
+    output, and the SiLU-mul output. The residual stream, q/k/v GEMV
+    outputs and logits are float64 here (float32 on the GPU).
+
+    ``k_cache``/``v_cache`` are float64 arrays ``[layers, Hkv, cap, D]``
+    holding bf16 values; row ``pos`` of every layer is overwritten.
+    Returns the logits ``[vocab]`` (float64).
+    """
+    H, Hkv, D = cfg["heads"], cfg["kv_heads"], cfg["head_dim"]
+    eps, theta = cfg["eps"], cfg["theta"]
+    ew, es, eb = weights["embed"]
+    x = embed_rows(ew, es, eb, [token])[0]
+    for l, lw in enumerate(weights["layers"]):
+        xn = round_bf16(rmsnorm(x, lw["input_norm"], eps))
+        q = gemv_affine8(*lw["q"], xn[None])[0]
+        k = gemv_affine8(*lw["k"], xn[None])[0]
+        v = gemv_affine8(*lw["v"], xn[None])[0]
+        q = rope_neox(rmsnorm_perhead(q, lw["q_norm"], eps, D), pos, theta, D)
+        k = rope_neox(rmsnorm_perhead(k, lw["k_norm"], eps, D), pos, theta, D)
+        k_cache[l, :, pos, :] = round_bf16(k).reshape(Hkv, D)
+        v_cache[l, :, pos, :] = round_bf16(v).reshape(Hkv, D)
+        att = round_bf16(decode_attention(q, k_cache[l], v_cache[l], pos + 1, H, Hkv, D))
+        x = x + gemv_affine8(*lw["o"], att[None])[0]
+        xn = round_bf16(rmsnorm(x, lw["post_norm"], eps))
+        gate = gemv_affine8(*lw["gate"], xn[None])[0]
+        up = gemv_affine8(*lw["up"], xn[None])[0]
+        hmid = round_bf16(silu_mul(gate, up))
+        x = x + gemv_affine8(*lw["down"], hmid[None])[0]
+    xn = round_bf16(rmsnorm(x, weights["final_norm"], eps))
+    return gemv_affine8(ew, es, eb, xn[None])[0]
+
+
+def new_kv_cache(cfg, cap):
+    return (np.zeros((cfg["layers"], cfg["kv_heads"], cap, cfg["head_dim"])),
+            np.zeros((cfg["layers"], cfg["kv_heads"], cap, cfg["head_dim"])))
+
+
+def prefix_forward(cfg, weights, token_ids):
+    """Whole-prefix forward with a causal mask ([MK] ``Qwen3Model::forward``
+    with the mask of ``causal_mask`` and ``Qwen3Attention::forward``): all
+    rows at once, no cache, the same precision points as ``decode_step``.
+    Returns logits ``[T, vocab]``. Used to pin ``decode_step``: the
+    incremental cache must give the same last-row logits."""
+    H, Hkv, D = cfg["heads"], cfg["kv_heads"], cfg["head_dim"]
+    eps, theta = cfg["eps"], cfg["theta"]
+    T = len(token_ids)
+    ew, es, eb = weights["embed"]
+    x = embed_rows(ew, es, eb, token_ids)
+    mask = np.triu(np.full((T, T), -np.inf), k=1)
+    g = H // Hkv
+    for lw in weights["layers"]:
+        xn = round_bf16(rmsnorm(x, lw["input_norm"], eps))
+        q = gemv_affine8(*lw["q"], xn)
+        k = gemv_affine8(*lw["k"], xn)
+        v = gemv_affine8(*lw["v"], xn)
+        q = np.stack([rope_neox(rmsnorm_perhead(q[t], lw["q_norm"], eps, D), t, theta, D) for t in range(T)])
+        k = np.stack([rope_neox(rmsnorm_perhead(k[t], lw["k_norm"], eps, D), t, theta, D) for t in range(T)])
+        k = round_bf16(k).reshape(T, Hkv, D)
+        v = round_bf16(v).reshape(T, Hkv, D)
+        q = q.reshape(T, H, D)
+        att = np.zeros((T, H, D))
+        for h in range(H):
+            s = q[:, h, :] @ k[:, h // g, :].T / math.sqrt(D) + mask
+            p = np.exp(s - s.max(axis=1, keepdims=True))
+            p = p / p.sum(axis=1, keepdims=True)
+            att[:, h, :] = p @ v[:, h // g, :]
+        att = round_bf16(att.reshape(T, H * D))
+        x = x + gemv_affine8(*lw["o"], att)
+        xn = round_bf16(rmsnorm(x, lw["post_norm"], eps))
+        hmid = round_bf16(silu_mul(gemv_affine8(*lw["gate"], xn), gemv_affine8(*lw["up"], xn)))
+        x = x + gemv_affine8(*lw["down"], hmid)
+    xn = round_bf16(rmsnorm(x, weights["final_norm"], eps))
+    return gemv_affine8(ew, es, eb, xn)

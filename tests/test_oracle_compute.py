@@ -1,0 +1,280 @@
+"""Pins for the oracle's arithmetic (CPU only).
+
+GEMVs against pure-Python brute force (bytes pulled out of the words with
+shifts, one multiply-add at a time), identity and one-hot matrices; norms,
+SiLU and attention against torch's own routines in float64; RoPE against a
+complex-number formulation and its group law; the decode step against a
+whole-prefix causal forward and a zero-weight closed form.
+"""
+import cmath
+import math
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import qg_synth
+from oracle import qg_oracle as O
+
+
+def _bf16(bits):
+    return torch.from_numpy(np.asarray(bits, np.uint16).view(np.int16)).view(torch.bfloat16).double().numpy()
+
+
+# ---------------------------------------------------------------- GEMV ----
+
+def _brute_gemv_affine8(words, scales, biases, x):
+    N, W = words.shape
+    K = 4 * W
+    B = x.shape[0]
+    s = _bf16(scales)
+    b = _bf16(biases)
+    y = [[0.0] * N for _ in range(B)]
+    for bb in range(B):
+        for r in range(N):
+            acc = 0.0
+            for c in range(K):
+                q = (int(words[r, c // 4]) >> (8 * (c % 4))) & 0xFF
+                acc += (q * s[r, c // 64] + b[r, c // 64]) * float(x[bb, c])
+            y[bb][r] = acc
+    return np.array(y)
+
+
+def test_gemv_affine8_brute_force():
+    words, s, b = qg_synth.affine8_packed(5, 128, seed=11)
+    x = _bf16(qg_synth.gaussian_bf16_bits((3, 128), 1.0, seed=12))
+    np.testing.assert_allclose(O.gemv_affine8(words, s, b, x),
+                               _brute_gemv_affine8(words, s, b, x), rtol=1e-12, atol=1e-14)
+
+
+def test_gemv_affine8_identity_and_one_hot():
+    K = 128
+    q = np.eye(K, dtype=np.uint8)
+    one = qg_synth.f32_to_bf16_bits(np.ones((K, K // 64), np.float32))
+    zero = np.zeros((K, K // 64), np.uint16)
+    x = _bf16(qg_synth.gaussian_bf16_bits((2, K), 1.0, seed=13))
+    np.testing.assert_array_equal(O.gemv_affine8(O.affine8_pack(q), one, zero, x), x)
+    words, s, b = qg_synth.affine8_packed(7, K, seed=14)
+    e = np.zeros((1, K))
+    e[0, 77] = 1.0
+    np.testing.assert_array_equal(O.gemv_affine8(words, s, b, e)[0],
+                                  O.affine8_dequant_exact(words, s, b)[:, 77])
+
+
+def test_gemv_affine8_factorisation():
+    # sum_g s_g * (sum_c q_c x_c) + beta_g * (sum_c x_c) equals the plain sum
+    words, s, b = qg_synth.affine8_packed(9, 256, seed=15)
+    x = _bf16(qg_synth.gaussian_bf16_bits((2, 256), 1.0, seed=16))
+    q = O.affine8_unpack(words).astype(np.float64).reshape(9, 4, 64)
+    xs = x.reshape(2, 4, 64)
+    y = np.einsum("rg,brg->br", _bf16(s), np.einsum("rgc,bgc->brg", q, xs)) \
+        + np.einsum("rg,bg->br", _bf16(b), xs.sum(axis=2))
+    np.testing.assert_allclose(O.gemv_affine8(words, s, b, x), y, rtol=1e-12)
+
+
+def test_gemv_affine8_residual():
+    words, s, b = qg_synth.affine8_packed(6, 64, seed=17)
+    x = np.ones((1, 64))
+    r = np.arange(6.0)[None]
+    np.testing.assert_allclose(O.gemv_affine8(words, s, b, x, residual=r),
+                               O.gemv_affine8(words, s, b, x) + r, rtol=0, atol=0)
+
+
+def _brute_gemv_q4_0(blocks, x, bias):
+    N = blocks.shape[0]
+    K = x.shape[1]
+    y = np.zeros((x.shape[0], N))
+    for bb in range(x.shape[0]):
+        for r in range(N):
+            acc = 0.0
+            for blk in range(K // 32):
+                base = blk * 18
+                d = float(np.frombuffer(bytes(blocks[r, base:base + 2]), dtype="<f2")[0])
+                for j in range(32):
+                    byte = int(blocks[r, base + 2 + (j % 16)])
+                    n = (byte & 0xF) if j < 16 else (byte >> 4)
+                    acc += d * (n - 8) * float(x[bb, blk * 32 + j])
+            y[bb, r] = acc + (bias[r] if bias is not None else 0.0)
+    return y
+
+
+def test_gemv_q4_0_brute_force():
+    blocks = qg_synth.q4_0_packed(4, 96, seed=18)
+    x = qg_synth.gaussian((2, 96), 1.0, seed=19).astype(np.float64)
+    bias = qg_synth.gaussian((4,), 1.0, seed=20).astype(np.float64)
+    np.testing.assert_allclose(O.gemv_q4_0(blocks, x, bias), _brute_gemv_q4_0(blocks, x, bias),
+                               rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(O.gemv_q4_0(blocks, x), _brute_gemv_q4_0(blocks, x, None),
+                               rtol=1e-12, atol=1e-14)
+
+
+def test_gemv_q4_0_identity():
+    K = 64
+    blk = np.zeros((K, K // 32, 18), np.uint8)
+    blk[:, :, 0:2] = np.array([1.0], np.float16).view(np.uint8)
+    n = np.full((K, K), 8, np.uint8)
+    n[np.arange(K), np.arange(K)] = 9
+    n = n.reshape(K, K // 32, 32)
+    blk[:, :, 2:] = n[:, :, :16] | (n[:, :, 16:] << 4)
+    x = qg_synth.gaussian((3, K), 1.0, seed=21).astype(np.float64)
+    np.testing.assert_array_equal(O.gemv_q4_0(blk.reshape(K, -1), x), x)
+
+
+def test_gemm_q4_0_bf16_contract_brute_force():
+    blocks = qg_synth.q4_0_packed(4, 64, seed=22)
+    A = qg_synth.gaussian((3, 64), 1.0, seed=23)
+    bias = qg_synth.gaussian((4,), 1.0, seed=24)
+    Ab = torch.from_numpy(A).to(torch.bfloat16).double()
+    # dequantize with the brute-force reader (identity x), cast with torch
+    W = _brute_gemv_q4_0(blocks, np.eye(64), None).T
+    Wb = torch.from_numpy(W.astype(np.float32)).to(torch.bfloat16).double()
+    want = (Ab @ Wb.T).numpy() + bias
+    np.testing.assert_allclose(O.gemm_q4_0_bf16(blocks, A, bias), want, rtol=1e-12, atol=1e-12)
+
+
+# ----------------------------------------------------------- elementwise --
+
+def test_rmsnorm_closed_form_and_torch():
+    w = qg_synth.f32_to_bf16_bits(np.linspace(0.5, 1.5, 64).astype(np.float32))
+    c, eps = 0.3, 1e-6
+    np.testing.assert_allclose(O.rmsnorm(np.full(64, c), w, eps), c / math.sqrt(c * c + eps) * _bf16(w),
+                               rtol=1e-14)
+    x = qg_synth.gaussian((5, 64), 3.0, seed=25).astype(np.float64)
+    want = F.rms_norm(torch.from_numpy(x), (64,), torch.from_numpy(_bf16(w)), eps=eps).numpy()
+    np.testing.assert_allclose(O.rmsnorm(x, w, eps), want, rtol=1e-13)
+    # scale invariance with eps = 0
+    np.testing.assert_allclose(O.rmsnorm(7.0 * x, w, 0.0), O.rmsnorm(x, w, 0.0), rtol=1e-13)
+
+
+def test_rmsnorm_perhead_is_rmsnorm_per_slice():
+    D = 32
+    w = qg_synth.f32_to_bf16_bits((1 + 0.1 * qg_synth.gaussian((D,), 1.0, seed=26)).astype(np.float32))
+    x = qg_synth.gaussian((3, 4 * D), 2.0, seed=27).astype(np.float64)
+    want = F.rms_norm(torch.from_numpy(x).reshape(3, 4, D), (D,), torch.from_numpy(_bf16(w)),
+                      eps=1e-5).reshape(3, 4 * D).numpy()
+    np.testing.assert_allclose(O.rmsnorm_perhead(x, w, 1e-5, D), want, rtol=1e-13)
+
+
+def test_rope_complex_form():
+    # NeoX pairs (i, i+half) rotate like the complex number x_i + 1j*x_{i+half}
+    D, theta, pos = 8, 10000.0, 37
+    x = qg_synth.gaussian((3 * D,), 1.0, seed=28).astype(np.float64)
+    got = O.rope_neox(x, pos, theta, D).reshape(3, D)
+    xh = x.reshape(3, D)
+    for h in range(3):
+        for i in range(D // 2):
+            z = complex(xh[h, i], xh[h, i + D // 2]) * cmath.exp(1j * pos * theta ** (-2 * i / D))
+            assert abs(got[h, i] - z.real) < 1e-12 and abs(got[h, i + D // 2] - z.imag) < 1e-12
+
+
+def test_rope_invariants():
+    D = 128
+    x = qg_synth.gaussian((4 * D,), 1.0, seed=29).astype(np.float64)
+    np.testing.assert_array_equal(O.rope_neox(x, 0, 1e6, D), x)
+    y = O.rope_neox(x, 511, 1e6, D).reshape(4, 2, D // 2)
+    xr = x.reshape(4, 2, D // 2)
+    np.testing.assert_allclose((y ** 2).sum(axis=1), (xr ** 2).sum(axis=1), rtol=1e-12)
+    np.testing.assert_allclose(O.rope_neox(O.rope_neox(x, 200, 1e6, D), 311, 1e6, D),
+                               O.rope_neox(x, 511, 1e6, D), rtol=1e-9, atol=1e-12)
+
+
+def test_rope_partial_rotary_dim_passes_tail_through():
+    D, rd = 64, 32
+    x = qg_synth.gaussian((2 * D,), 1.0, seed=30).astype(np.float64)
+    y = O.rope_neox(x, 9, 1e4, D, rotary_dim=rd).reshape(2, D)
+    np.testing.assert_array_equal(y[:, rd:], x.reshape(2, D)[:, rd:])
+    np.testing.assert_allclose(y[:, :rd], O.rope_neox(x.reshape(2, D)[:, :rd].reshape(-1), 9, 1e4, rd).reshape(2, rd))
+
+
+def test_silu_mul_against_torch():
+    g = qg_synth.gaussian((1000,), 4.0, seed=31).astype(np.float64)
+    u = qg_synth.gaussian((1000,), 1.0, seed=32).astype(np.float64)
+    want = (F.silu(torch.from_numpy(g)) * torch.from_numpy(u)).numpy()
+    np.testing.assert_allclose(O.silu_mul(g, u), want, rtol=1e-14)
+
+
+# ------------------------------------------------------------ attention --
+
+def _cache(Hkv, L, D, seed):
+    return (_bf16(qg_synth.gaussian_bf16_bits((Hkv, L, D), 1.0, seed)),
+            _bf16(qg_synth.gaussian_bf16_bits((Hkv, L, D), 1.0, seed + 1)))
+
+
+def test_attention_matches_torch_sdpa_with_repeat_kv():
+    H, Hkv, D, L = 16, 8, 128, 77
+    k, v = _cache(Hkv, 100, D, 33)
+    q = qg_synth.gaussian((H * D,), 1.0, seed=35).astype(np.float64)
+    got = O.decode_attention(q, k, v, L, H, Hkv, D)
+    kk = torch.from_numpy(k[:, :L]).repeat_interleave(H // Hkv, dim=0)   # explicit repeat_kv
+    vv = torch.from_numpy(v[:, :L]).repeat_interleave(H // Hkv, dim=0)
+    want = F.scaled_dot_product_attention(torch.from_numpy(q).reshape(H, 1, D), kk, vv).reshape(-1).numpy()
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-13)
+
+
+def test_attention_special_cases():
+    H, Hkv, D = 4, 2, 16
+    k, v = _cache(Hkv, 8, D, 36)
+    q = qg_synth.gaussian((H * D,), 1.0, seed=38).astype(np.float64)
+    # L = 1: the only value row comes back exactly
+    out = O.decode_attention(q, k, v, 1, H, Hkv, D).reshape(H, D)
+    for h in range(H):
+        np.testing.assert_array_equal(out[h], v[h // 2, 0])
+    # identical keys: the mean of the values
+    k2 = np.repeat(k[:, :1], 8, axis=1)
+    out = O.decode_attention(q, k2, v, 8, H, Hkv, D).reshape(H, D)
+    for h in range(H):
+        np.testing.assert_allclose(out[h], v[h // 2].mean(axis=0), rtol=1e-12, atol=1e-14)
+    # one dominant key: its value row
+    k3 = np.zeros_like(k)
+    qh = q.reshape(H, D)
+    for h in range(H):
+        k3[h // 2, 5] += 200.0 * qh[h] / np.linalg.norm(qh[h])
+    out = O.decode_attention(q, k3, v, 8, H, Hkv, D).reshape(H, D)
+    for h in range(H):
+        np.testing.assert_allclose(out[h], v[h // 2, 5], rtol=1e-9, atol=1e-12)
+
+
+def test_argmax_first_strict_max_skips_nan():
+    assert O.argmax_first([1.0, 3.0, 3.0, 2.0]) == 1
+    assert O.argmax_first([float("nan"), 0.5, float("nan"), 0.7, 0.7]) == 3
+    assert O.argmax_first([float("-inf")] * 3) == 0
+    x = qg_synth.gaussian((5000,), 1.0, seed=39)
+    assert O.argmax_first(x) == int(np.argmax(x))
+
+
+# --------------------------------------------------------- decode step ---
+
+def _tiny(seed, fixture=True):
+    cfg = dict(qg_synth.QWEN3_TINY)
+    return cfg, qg_synth.qwen3_weights(cfg, seed, fixture=fixture)
+
+
+@pytest.mark.parametrize("fixture", [True, False])
+def test_decode_step_matches_causal_prefix_forward(fixture):
+    cfg, w = _tiny(3, fixture)
+    toks = [5, 200, 17, 17, 260, 0]
+    kc, vc = O.new_kv_cache(cfg, 16)
+    for p, t in enumerate(toks):
+        logits = O.decode_step(cfg, w, kc, vc, t, p)
+    full = O.prefix_forward(cfg, w, toks)
+    np.testing.assert_allclose(logits, full[-1], rtol=1e-9, atol=1e-9 * np.abs(full[-1]).max())
+    assert np.isfinite(logits).all()
+
+
+def test_decode_step_zero_weights_closed_form():
+    # With every linear zero, attention and MLP add nothing: the logits are
+    # the LM head applied to the normed embedding row.
+    cfg, w = _tiny(4, fixture=False)
+    for lw in w["layers"]:
+        for name in qg_synth.LINEARS:
+            words, s, b = lw[name]
+            lw[name] = (np.zeros_like(words), s, np.zeros_like(b))
+    ew, es, eb = w["embed"]
+    t = 42
+    kc, vc = O.new_kv_cache(cfg, 4)
+    logits = O.decode_step(cfg, w, kc, vc, t, 0)
+    e = O.affine8_dequant_exact(ew, es, eb)
+    row = e[t].astype(np.float32).astype(np.float64)
+    xn = torch.from_numpy(row / np.sqrt(np.mean(row ** 2) + cfg["eps"])).to(torch.bfloat16).double().numpy()
+    np.testing.assert_allclose(logits, e @ xn, rtol=1e-12, atol=1e-12)
