@@ -1,0 +1,402 @@
+#!/usr/bin/env python
+"""Benchmark of the weight-only-quantized decode path on B200.
+
+One step = one decode step of a random-init Qwen3-0.6B-shaped text decoder
+(28 layers, hidden 1024, 16 Q / 8 KV heads, head_dim 128, FFN 3072, tied
+vocab 151936; affine-INT8 group-64 packed weights) for B sequences at KV
+length 512 (position 511, attending 512 cached rows): every hot-path stage
+(embedding dequant, RMSNorms, q/k/v, q/k norm + RoPE + KV append, split-KV
+attention, o-proj + residual, gate/up + SiLU-mul, down + residual, final norm
+and the tied LM head). The step is captured once into a CUDA graph and
+replayed. Inputs are seeded synthetic data; the weights of one step total
+~692 MB, larger than L2 (126 MB), so nothing survives in L2 between steps.
+
+Multi-GPU: replicas only -- every rank decodes its own sequences with its own
+weight copy; no data-path collective. ``value`` is the total steps/s of all
+ranks (weak scaling), timed as the max over ranks.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--batch B]
+       python bench.py --impl reference   (the CPU oracle on the host cores)
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import qg_synth  # noqa: E402
+
+METRIC = "quantized GEMV HBM GB/s & % of peak; decode steps/s (Qwen3-0.6B shape, b=1)"
+FALLBACK_HBM_GBS = 6650.0
+KV_LEN = 512
+
+
+# ------------------------------------------------------------ byte model ----
+
+def affine8_bytes(N, K, B, x_bytes=2, y_bytes=4):
+    """Algorithmic bytes of one affine-INT8 g64 GEMV: codes, bf16 scales and
+    biases, the activations read and the outputs written."""
+    return N * K + N * (K // 64) * 4 + B * K * x_bytes + B * N * y_bytes
+
+
+def step_bytes(cfg, B, L):
+    """Algorithmic bytes of one decode step: every packed weight byte once,
+    the norm weights, the embedding row, the K/V rows attended (L per layer
+    and sequence, read) and appended (one per layer and sequence)."""
+    h, H, Hk, D, F, V = (cfg["hidden"], cfg["heads"], cfg["kv_heads"], cfg["head_dim"],
+                         cfg["ffn"], cfg["vocab"])
+    sh = qg_synth.linear_shapes(cfg)
+    w = sum(affine8_bytes(n, k, 0) for n, k in sh.values()) * cfg["layers"]
+    head = affine8_bytes(V, h, 0)
+    norms = cfg["layers"] * (2 * h + 2 * D) * 2 + h * 2
+    emb = B * (h + (h // 64) * 4)
+    kv_read = B * cfg["layers"] * 2 * L * Hk * D * 2
+    kv_write = B * cfg["layers"] * 2 * Hk * D * 2
+    acts = B * V * 4
+    return w + head + norms + emb + kv_read + kv_write + acts
+
+
+# ------------------------------------------------------------- plumbing -----
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def traffic_from_profile(kernel_file):
+    """DRAM bytes per launch of the LM-head GEMV from the committed ncu
+    summary, or None when that summary is missing or was taken on a different
+    version of the kernel source (its sha256 must match)."""
+    path = os.path.join(ROOT, "profiles", "gemv_affine8_lm_head_151936x1024_b1.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m = re.search(r"traffic_bytes_per_launch:\s*(\d+)", text)
+    h = re.search(r"kernel_source_sha256:\s*([0-9a-f]{64})", text)
+    if not m or not h:
+        return None
+    cur = hashlib.sha256(open(kernel_file, "rb").read()).hexdigest()
+    return int(m.group(1)) if cur == h.group(1) else None
+
+
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons while running."""
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.rows = []
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) == 6:
+                self.rows.append(parts)
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[0]) for r in self.rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4) if r[2 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(self.rows)}
+
+
+def cpu_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n and n[0]:
+            return int(n[0])
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+# ------------------------------------------------------ oracle (CPU) legs ---
+
+def oracle_sample(cfg, weights, budget_steps=None, layers_only=None):
+    """Time the CPU oracle on a bounded sample of the decode step: whole
+    steps (28 layers + LM head) or, with ``layers_only``, that many single
+    layers plus one LM head, scaled to a whole step. Returns (steps/s,
+    description)."""
+    from oracle import qg_oracle as O
+    Hk, D = cfg["kv_heads"], cfg["head_dim"]
+    cap = KV_LEN + 1
+    kc = O.bf16_bits_to_f64(qg_synth.gaussian_bf16_bits((cfg["layers"], Hk, cap, D), 1.0, 70))
+    vc = O.bf16_bits_to_f64(qg_synth.gaussian_bf16_bits((cfg["layers"], Hk, cap, D), 1.0, 71))
+    tok = int(qg_synth.tokens(1, cfg["vocab"], 72)[0])
+    if layers_only is None:
+        t0 = time.perf_counter()
+        for _ in range(budget_steps):
+            O.decode_step(cfg, weights, kc, vc, tok, KV_LEN - 1)
+        dt = (time.perf_counter() - t0) / budget_steps
+        return 1.0 / dt, f"{budget_steps} full decode step(s) at position {KV_LEN - 1}, batch 1"
+    ew, es, eb = weights["embed"]
+    x = O.embed_rows(ew, es, eb, [tok])[0]
+    t0 = time.perf_counter()
+    for i in range(layers_only):
+        l = i % cfg["layers"]
+        x = O.decode_layer(cfg, weights["layers"][l], x, kc[l], vc[l], KV_LEN - 1)
+    t_layer = (time.perf_counter() - t0) / layers_only
+    t0 = time.perf_counter()
+    O.lm_head(cfg, weights, x)
+    t_head = time.perf_counter() - t0
+    return 1.0 / (cfg["layers"] * t_layer + t_head), (
+        f"{layers_only} single decoder layers at position {KV_LEN - 1} plus one LM head, "
+        f"scaled to 28 layers + head, batch 1")
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    cfg = dict(qg_synth.QWEN3_0_6B)
+    weights = qg_synth.qwen3_weights(cfg, 11)
+    # warm-up: W single layers; timed: K single layers (each a bounded sample)
+    oracle_sample(cfg, weights, layers_only=max(1, args.warmup))
+    v, desc = oracle_sample(cfg, weights, layers_only=max(1, args.steps))
+    cores = cpu_cores()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "steps/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 / v, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"Qwen3-0.6B-shaped affine-INT8 g64 decode step, batch 1, KV {KV_LEN}"},
+        "cpu_baseline": {"value": v, "unit": "steps/s", "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": v, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------ GPU arm -------
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    import weight_only_quantized_03_b200 as qg
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    cfg = dict(qg_synth.QWEN3_0_6B)
+    B = args.batch
+    weights = qg_synth.qwen3_weights(cfg, 11)
+    model = qg.Qwen3Model(cfg, weights, device=f"cuda:{local}")
+    cap = KV_LEN + 1
+    st = model.new_state(B, cap)
+    kshape = (cfg["layers"], B, cfg["kv_heads"], cap, cfg["head_dim"])
+    st["k_cache"].copy_(torch.from_numpy(qg_synth.gaussian_bf16_bits(kshape, 1.0, 70).view(np.int16))
+                        .view(torch.bfloat16))
+    st["v_cache"].copy_(torch.from_numpy(qg_synth.gaussian_bf16_bits(kshape, 1.0, 71).view(np.int16))
+                        .view(torch.bfloat16))
+    toks_np = qg_synth.tokens(B, cfg["vocab"], 72 + rank)
+    pos_np = np.full(B, KV_LEN - 1, dtype=np.int32)
+    toks = torch.from_numpy(toks_np).cuda()
+    pos = torch.from_numpy(pos_np).cuda()
+    stream = torch.cuda.Stream()
+
+    # ---- capture one step into a CUDA graph
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            model.qg_decode_step(st, toks, pos)
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    n0 = qg.lib.qg_kernel_launch_count()
+    with torch.cuda.graph(graph, stream=stream):
+        model.qg_decode_step(st, toks, pos)
+    launches_per_step = qg.lib.qg_kernel_launch_count() - n0
+
+    # ---- warm-up, then K timed replays
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            graph.replay()
+    stream.synchronize()
+    barrier()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        torch.cuda.synchronize()
+        barrier()
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            for _ in range(args.steps):
+                graph.replay()
+            ev1.record(stream)
+        stream.synchronize()
+        torch.cuda.synchronize()
+        barrier()
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+    value = world * args.steps / (ms / 1000.0)
+
+    # ---- dominant kernel: the LM-head GEMV (151936 x 1024), timed per launch
+    hbm_peak, peak_kind = measured_peaks()
+    V, h = cfg["vocab"], cfg["hidden"]
+    ew, es, eb = [torch.from_numpy(a.view({2: np.int16, 4: np.int32}[a.dtype.itemsize])).cuda()
+                  for a in weights["embed"]]
+    xb = torch.from_numpy(qg_synth.gaussian_bf16_bits((B, h), 1.0, 5).view(np.int16)).cuda() \
+        .view(torch.bfloat16)
+    yl = torch.empty((B, V), dtype=torch.float32, device="cuda")
+    nlaunch = max(20, min(200, args.steps))
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(nlaunch)]
+    with torch.cuda.stream(stream):
+        for _ in range(5):
+            qg.qg_gemv_affine8_g64(ew, es, eb, xb, yl, stream=stream)
+        for a, b in evs:
+            a.record(stream)
+            qg.qg_gemv_affine8_g64(ew, es, eb, xb, yl, stream=stream)
+            b.record(stream)
+    stream.synchronize()
+    lm_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    lm_bytes = affine8_bytes(V, h, B)
+    lm_gbs = lm_bytes / (lm_ms / 1000.0) / 1e9
+    traffic = traffic_from_profile(os.path.join(ROOT, "weight_only_quantized_03_b200", "csrc",
+                                                "gemv_affine8.cu")) if B == 1 else None
+
+    # ---- e2e through the public API with host buffers
+    h_tok = torch.from_numpy(toks_np).pin_memory()
+    h_pos = torch.from_numpy(pos_np).pin_memory()
+    h_logits = torch.empty((B, V), dtype=torch.float32).pin_memory()
+    e2e_steps = max(10, min(args.steps, 200))
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            toks.copy_(h_tok, non_blocking=True)
+            pos.copy_(h_pos, non_blocking=True)
+            model.qg_decode_step(st, toks, pos, stream=stream)
+            h_logits.copy_(st["logits"], non_blocking=True)
+    stream.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            toks.copy_(h_tok, non_blocking=True)
+            pos.copy_(h_pos, non_blocking=True)
+            model.qg_decode_step(st, toks, pos, stream=stream)
+            h_logits.copy_(st["logits"], non_blocking=True)
+        e1.record(stream)
+    stream.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * e2e_steps / (e2e_ms / 1000.0)
+
+    sb = step_bytes(cfg, B, KV_LEN)
+    line = {
+        "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded random packed weights, N(0,1) bf16 KV cache)",
+        "config": {
+            "workload": f"Qwen3-0.6B-shaped affine-INT8 g64 decode step, batch {B}, KV {KV_LEN}",
+            "batch": B, "kv_len": KV_LEN, "layers": cfg["layers"], "hidden": cfg["hidden"],
+            "vocab": cfg["vocab"], "parallelism": f"replicas x{world}",
+            "l2": f"inputs larger than L2 ({sb / 1e6:.0f} MB per step)", "graph": "CUDA graph + PDL",
+        },
+        "roofline": {"bound": "hbm", "kernel": "gemv_affine8 (LM head 151936x1024)",
+                     "achieved": lm_gbs, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": lm_gbs / hbm_peak, "traffic": traffic,
+                     "algorithmic_bytes": lm_bytes, "launch_us": lm_ms * 1000.0,
+                     "peak_kind": peak_kind},
+        "step_roofline": {"algorithmic_bytes": sb, "achieved": sb / (ms_per_step / 1000.0) / 1e9,
+                          "peak": hbm_peak, "unit": "GB/s",
+                          "frac": sb / (ms_per_step / 1000.0) / 1e9 / hbm_peak},
+        "e2e": {"value": e2e_value, "unit": "steps/s", "h2d_bytes_per_step": 2 * 4 * B,
+                "d2h_bytes_per_step": 4 * B * V},
+        "gpu_launches": int(launches_per_step * args.steps),
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, desc = oracle_sample(cfg, weights, budget_steps=1)
+        line["cpu_baseline"] = {"value": v, "unit": "steps/s", "cores": cpu_cores(),
+                                "kind": "oracle", "sample": desc}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del graph
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--batch", type=int, default=1)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

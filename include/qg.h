@@ -1,0 +1,295 @@
+/*
+ * qg.h -- C ABI of libqg, weight-only-quantized decode kernels for NVIDIA
+ * B200 (sm_100a).
+ *
+ * Sources the operations follow (cited per entry point):
+ *   [TS] turbospark-runtime 0.3.0, src/qwen3_asr_metal.rs: resident packed
+ *        affine-INT8 (group 64) Qwen3 text decoder (`PackedLinear`,
+ *        `load_packed_linear`, `embed_row_bytes`, `step`, `argmax`).
+ *   [FT] fuel-transformers 0.19.1, src/models/lazy_quantized_whisper.rs:
+ *        GGUF Q4_0 Whisper (`quantize_in_out_to_q4_0`, `q_linear`,
+ *        `encoder_layer`).
+ *   [MK] makima commit eabd130, src/tts/qwen3/model.rs: candle Qwen3
+ *        decoder (`RotaryEmbedding`, `Qwen3Attention::forward`, `repeat_kv`,
+ *        `Qwen3Mlp::forward`).
+ *
+ * Conventions (every entry point):
+ *   - Returns a qg_status. On failure qg_last_error() gives a message that
+ *     names the offending argument. A call that fails validation launches
+ *     nothing and writes nothing.
+ *   - Pointers documented as "device" must point to device memory of the
+ *     current CUDA device. The library borrows them for the call; it never
+ *     allocates, frees or retains them. The caller owns all memory,
+ *     workspace included.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is
+ *     the legacy default stream). Results are valid once the stream has
+ *     been synchronised. No entry point synchronises, allocates, or
+ *     branches on device data on the host, so every compute entry point may
+ *     be captured into a CUDA graph.
+ *   - Dimensions are int and must be >= 0; an element count that overflows
+ *     int64 or a shape rule below is refused with QG_ERR_UNSUPPORTED_SHAPE.
+ *     A zero batch or zero row count is a valid no-op.
+ *   - bf16 values travel as uint16_t bit patterns.
+ *   - Every device pointer must be 16-byte aligned unless stated otherwise
+ *     (QG_ERR_MISALIGNED).
+ *   - A CUDA launch error returns QG_ERR_CUDA with the CUDA error string.
+ */
+#ifndef QG_H
+#define QG_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum qg_status {
+  QG_OK = 0,
+  QG_ERR_INVALID_ARGUMENT = 1,
+  QG_ERR_UNSUPPORTED_SHAPE = 2,
+  QG_ERR_MISALIGNED = 3,
+  QG_ERR_WORKSPACE_TOO_SMALL = 4,
+  QG_ERR_CUDA = 5,
+  QG_ERR_TIMEOUT = 6
+} qg_status;
+
+typedef enum qg_dtype { QG_F32 = 0, QG_BF16 = 1 } qg_dtype;
+
+/* Thread-local message for the last failing call on this host thread
+ * ("" after a successful call). Never NULL. */
+const char* qg_last_error(void);
+
+/* Version of this ABI (incremented on any incompatible change). */
+int qg_abi_version(void);
+
+/* Number of CUDA kernels this library has enqueued in this process (all
+ * entry points, all host threads). Capturing a call into a CUDA graph and
+ * reading the count before and after gives the kernels per graph replay. */
+unsigned long long qg_kernel_launch_count(void);
+
+/* ------------------------------------------------------------------------
+ * Affine-INT8 group-64 dequant GEMV  [TS: PackedLinear / load_packed_linear,
+ * the per-linear GEMV of `step`]
+ *
+ *   y[b][r] = sum_c (q[r][c] * s[r][c/64] + beta[r][c/64]) * x[b][c]
+ *             (+ residual[b][r] when residual != NULL)
+ *
+ * w       device, uint32 [N][K/4]: row r holds the K code bytes of row r,
+ *         column 4j+i in byte i (bits 8i..8i+7) of word j (little endian).
+ * scales  device, bf16 [N][K/64] (2-byte alignment suffices).
+ * biases  device, bf16 [N][K/64] (2-byte alignment suffices).
+ * x       device, [B][K] of x_dtype (QG_BF16 or QG_F32).
+ * y       device, [B][N] of y_dtype; fp32 accumulation, one rounding at the
+ *         store when y_dtype is QG_BF16. May alias `residual` (in-place
+ *         y += W x); must not overlap w, scales, biases or x.
+ * residual device fp32 [B][N] or NULL (4-byte alignment suffices).
+ * Shape rules: K % 64 == 0, 1 <= B <= 32 (B == 0 is a no-op), N >= 0.
+ * ---------------------------------------------------------------------- */
+qg_status qg_gemv_affine8_g64(const uint32_t* w, const uint16_t* scales,
+                              const uint16_t* biases, const void* x,
+                              qg_dtype x_dtype, void* y, qg_dtype y_dtype,
+                              const float* residual, int N, int K, int B,
+                              void* stream);
+
+/* ------------------------------------------------------------------------
+ * Q4_0 dequant GEMV  [FT: quantize_in_out_to_q4_0 (block layout), q_linear]
+ *
+ *   y[b][r] = sum_blk d[r][blk] * sum_{j<32} (n[r][blk][j] - 8) * x[b][32 blk + j]
+ *             (+ bias[r] when bias != NULL)
+ *
+ * blocks  device, uint8 [N][(K/32) * 18]: per block an fp16 d (little
+ *         endian) then 16 bytes; byte j holds code j (low nibble) and code
+ *         j+16 (high nibble). Rows are contiguous; no padding. 2-byte
+ *         alignment suffices.
+ * x       device fp32 [B][K].   bias device fp32 [N] or NULL (4-byte align).
+ * y       device fp32 [B][N].
+ * Shape rules: K % 32 == 0, 1 <= B <= 32 (B == 0 is a no-op).
+ * ---------------------------------------------------------------------- */
+qg_status qg_gemv_q4_0(const uint8_t* blocks, const float* x, const float* bias,
+                       float* y, int N, int K, int B, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Q4_0 matmul on the tensor cores  [FT: encoder_layer -> q_linear with
+ * M = frames]
+ *
+ *   C[m][r] = sum_k bf16(A[m][k]) * bf16(d * (n - 8))[r][k] (+ bias[r])
+ *
+ * Operands are rounded to bf16 (nearest even) and multiplied on the
+ * tcgen05 tensor cores with fp32 accumulation in tensor memory.
+ * blocks  device, Q4_0 [N][(K/32)*18] as in qg_gemv_q4_0.
+ * A       device fp32 [M][K].  bias device fp32 [N] or NULL.  C device fp32 [M][N].
+ * ws      device workspace of at least qg_gemm_q4_0_workspace_size(M,N,K)
+ *         bytes (contents need not be initialised).
+ * Shape rules: K % 64 == 0, N % 128 == 0, M >= 0.
+ * ---------------------------------------------------------------------- */
+size_t qg_gemm_q4_0_workspace_size(int M, int N, int K);
+qg_status qg_gemm_q4_0(const uint8_t* blocks, const float* A, const float* bias,
+                       float* C, int M, int N, int K, void* ws, size_t ws_bytes,
+                       void* stream);
+
+/* ------------------------------------------------------------------------
+ * RMSNorm  [TS: encode_rms_norm_bf16w in `step`; MK: rms_norm layers]
+ *   y[r][i] = x[r][i] / sqrt(mean_i(x[r][i]^2) + eps) * w[i]
+ * x device fp32 [rows][dim]; w device bf16 [dim] (2-byte alignment);
+ * y device [rows][dim] of y_dtype (may alias x when y_dtype is QG_F32).
+ * Shape rules: 1 <= dim <= 65536, dim % 4 == 0.
+ * ---------------------------------------------------------------------- */
+qg_status qg_rmsnorm(const float* x, const uint16_t* w, float eps, void* y,
+                     qg_dtype y_dtype, int rows, int dim, void* stream);
+
+/* Per-head RMSNorm (Qwen3 q_norm / k_norm)  [TS: encode_rms_norm_bf16w_perhead;
+ * MK: apply_head_norm]: the RMSNorm above on every D-wide slice of
+ * x [rows][heads*D] with one shared weight w [D]. x and y fp32 or bf16
+ * (x_dtype, y_dtype); y may alias x when the dtypes match.
+ * Shape rules: D % 32 == 0, D <= 1024. */
+qg_status qg_rmsnorm_perhead(const void* x, qg_dtype x_dtype, const uint16_t* w,
+                             float eps, void* y, qg_dtype y_dtype, int rows,
+                             int heads, int D, void* stream);
+
+/* ------------------------------------------------------------------------
+ * NeoX rotate-half RoPE, in place  [MK: RotaryEmbedding::new / apply /
+ * rotate_half; TS: encode_rope_neox_subdim]
+ *   for i < rotary_dim/2, a = pos[r] * theta^(-2i/rotary_dim) (float64):
+ *   x'[i]      = x[i] cos a - x[i+half] sin a
+ *   x'[i+half] = x[i+half] cos a + x[i] sin a,   half = rotary_dim/2;
+ *   dims >= rotary_dim are untouched.
+ * x device [rows][heads*D] of dtype; pos device int32 [rows] (4-byte align).
+ * Shape rules: rotary_dim even, 2 <= rotary_dim <= D, D % 2 == 0.
+ * ---------------------------------------------------------------------- */
+qg_status qg_rope_neox(void* x, qg_dtype dtype, const int32_t* pos, double theta,
+                       int rows, int heads, int D, int rotary_dim, void* stream);
+
+/* SiLU-mul  [TS: encode_silu_mul; MK: Qwen3Mlp::forward]
+ *   out[i] = gate[i] / (1 + exp(-gate[i])) * up[i]
+ * gate, up device fp32 [n]; out device [n] of out_dtype (may alias gate
+ * when QG_F32). 4-byte alignment suffices. */
+qg_status qg_silu_mul(const float* gate, const float* up, void* out,
+                      qg_dtype out_dtype, int n, void* stream);
+
+/* Residual add  [TS: encode_residual_add]: x[i] += delta[i], fp32, device,
+ * 4-byte alignment suffices. */
+qg_status qg_residual_add(float* x, const float* delta, int n, void* stream);
+
+/* Tied-embedding row dequantization  [TS: embed_row_bytes]
+ *   x[b][c] = q_E[t_b][c] * s_E[t_b][c/64] + beta_E[t_b][c/64]   (fp32)
+ * table as in qg_gemv_affine8_g64 with N = vocab, K = hidden; tokens
+ * device int32 [B]. A token outside [0, vocab) yields a row of NaN.
+ * Shape rules: hidden % 64 == 0. */
+qg_status qg_embed_affine8_g64(const uint32_t* w, const uint16_t* scales,
+                               const uint16_t* biases, const int32_t* tokens,
+                               float* x, int vocab, int hidden, int B,
+                               void* stream);
+
+/* ------------------------------------------------------------------------
+ * Split-softmax GQA decode attention  [TS: encode_attention_decode with
+ * kv_start = 0 and its AttentionScratch; MK: Qwen3Attention::forward,
+ * repeat_kv]
+ *   For sequence b and query head h (KV head h / (H/Hkv)), L = kv_len[b]:
+ *   out[b][h] = sum_{t<L} softmax_t(q[b][h] . k[b][kv][t] * scale) v[b][kv][t]
+ * The L rows are cut into chunks scored by separate CTAs; per-chunk
+ * (max, sum, weighted V) partials are merged in a fixed order (results do
+ * not depend on scheduling).
+ * q        device fp32 [B][H][D].
+ * k_cache, v_cache device bf16 [B][Hkv][cap][D] (row t of head kv at
+ *          ((b*Hkv + kv)*cap + t)*D).
+ * kv_len   device int32 [B]; read on the device. A value outside [1, cap]
+ *          gives a zero output row for that sequence (nothing is read out
+ *          of bounds).
+ * out      device [B][H][D] of out_dtype.
+ * ws       device workspace, >= qg_decode_attention_workspace_size(...)
+ *          bytes, 256-byte aligned; its contents need not be initialised.
+ * Shape rules: H % Hkv == 0, H/Hkv <= 8, D % 32 == 0, D <= 256, cap >= 1.
+ * ---------------------------------------------------------------------- */
+size_t qg_decode_attention_workspace_size(int B, int H, int Hkv, int D, int cap);
+qg_status qg_decode_attention(const float* q, const uint16_t* k_cache,
+                              const uint16_t* v_cache, const int32_t* kv_len,
+                              void* out, qg_dtype out_dtype, int B, int H,
+                              int Hkv, int D, int cap, float scale, void* ws,
+                              size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Whole Qwen3 decode step  [TS: step; MK: Qwen3DecoderLayer::forward]
+ * ---------------------------------------------------------------------- */
+typedef struct qg_affine8_matrix {
+  const uint32_t* w;       /* device uint32 [rows][cols/4] */
+  const uint16_t* scales;  /* device bf16 [rows][cols/64] */
+  const uint16_t* biases;  /* device bf16 [rows][cols/64] */
+} qg_affine8_matrix;
+
+typedef struct qg_qwen3_layer {
+  const uint16_t* input_norm; /* device bf16 [hidden] */
+  const uint16_t* post_norm;  /* device bf16 [hidden] */
+  const uint16_t* q_norm;     /* device bf16 [head_dim] */
+  const uint16_t* k_norm;     /* device bf16 [head_dim] */
+  qg_affine8_matrix q;        /* [heads*head_dim][hidden] */
+  qg_affine8_matrix k;        /* [kv_heads*head_dim][hidden] */
+  qg_affine8_matrix v;        /* [kv_heads*head_dim][hidden] */
+  qg_affine8_matrix o;        /* [hidden][heads*head_dim] */
+  qg_affine8_matrix gate;     /* [ffn][hidden] */
+  qg_affine8_matrix up;       /* [ffn][hidden] */
+  qg_affine8_matrix down;     /* [hidden][ffn] */
+} qg_qwen3_layer;
+
+typedef struct qg_qwen3_config {
+  int hidden, layers, heads, kv_heads, head_dim, ffn, vocab;
+  float eps;     /* RMSNorm epsilon */
+  double theta;  /* RoPE base */
+} qg_qwen3_config;
+
+typedef struct qg_qwen3_weights {
+  qg_affine8_matrix embed;       /* tied embedding and LM head [vocab][hidden] */
+  const uint16_t* final_norm;    /* device bf16 [hidden] */
+  const qg_qwen3_layer* layers;  /* HOST array of cfg->layers entries */
+} qg_qwen3_weights;
+
+/* Workspace bytes for qg_decode_step at batch B and cache capacity cap. */
+size_t qg_decode_step_workspace_size(const qg_qwen3_config* cfg, int B, int cap);
+
+/* One decode step for B independent sequences sharing the weights.
+ * For each sequence b: embed tokens[b]; run every layer at position
+ * positions[b] (RMSNorm -> q,k,v -> per-head q/k RMSNorm -> RoPE -> K and V
+ * written at cache row positions[b] -> attention over rows
+ * [0, positions[b]] -> o_proj + residual -> RMSNorm -> gate, up -> SiLU-mul
+ * -> down + residual); then the final RMSNorm and the tied LM head.
+ *
+ * cfg, w      HOST structs (read during the call only).
+ * k_cache, v_cache device bf16 [layers][B][kv_heads][cap][head_dim].
+ * tokens, positions device int32 [B], read on the device. A sequence whose
+ *             token is outside [0, vocab) or position outside [0, cap)
+ *             gets NaN logits and its cache is not written.
+ * logits      device fp32 [B][vocab].
+ * ws          device workspace >= qg_decode_step_workspace_size(cfg,B,cap)
+ *             bytes, 256-byte aligned; contents need not be initialised.
+ *             On return its first B*hidden*4 bytes hold the residual stream
+ *             after the last layer (fp32 [B][hidden], before the final norm).
+ * Precision: residual stream, q/k/v and gate/up outputs and logits fp32;
+ * norm outputs feeding a GEMV, cached K/V, attention output and SiLU-mul
+ * output bf16.
+ * Shape rules: hidden, heads*head_dim and ffn multiples of 64;
+ * heads % kv_heads == 0, heads/kv_heads <= 8; head_dim % 32 == 0,
+ * head_dim <= 256; 1 <= B <= 32; cap >= 1. */
+qg_status qg_decode_step(const qg_qwen3_config* cfg, const qg_qwen3_weights* w,
+                         uint16_t* k_cache, uint16_t* v_cache, int cap,
+                         const int32_t* tokens, const int32_t* positions,
+                         float* logits, int B, void* ws, size_t ws_bytes,
+                         void* stream);
+
+/* ------------------------------------------------------------------------
+ * Test exports: the unpack and dequant the kernels use, written out.
+ * ---------------------------------------------------------------------- */
+/* q[r][c] as fp32 (0..255) from packed words; out device fp32 [N][K]. */
+qg_status qg_unpack_affine8(const uint32_t* w, float* out, int N, int K, void* stream);
+/* q*s+beta as fp32 (one rounding); out device fp32 [N][K]. */
+qg_status qg_dequant_affine8_g64(const uint32_t* w, const uint16_t* scales,
+                                 const uint16_t* biases, float* out, int N,
+                                 int K, void* stream);
+/* d*(n-8) as fp32 (exact); out device fp32 [N][K]. */
+qg_status qg_dequant_q4_0(const uint8_t* blocks, float* out, int N, int K,
+                          void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QG_H */

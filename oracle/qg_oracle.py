@@ -356,46 +356,57 @@ def argmax_first(logits):
 # The decode step  [TS: step]
 # ---------------------------------------------------------------------------
 
-def decode_step(cfg, weights, k_cache, v_cache, token, pos):
-    """One token of one sequence through every layer, in the op order of
-    [TS] ``step``: input norm -> q, k, v GEMVs -> per-head q/k norm -> NeoX
-    RoPE on q and on k -> K/V written at cache row ``pos`` -> attention over
-    rows ``[0, pos]`` -> o_proj -> residual add -> post-attention norm ->
-    gate, up -> SiLU-mul -> down -> residual add; then the final norm and
-    the tied LM head. The embedding row is the dequantized packed row of
-    [TS] ``embed_row_bytes``.
+def decode_layer(cfg, lw, x, k_cache_l, v_cache_l, pos):
+    """One decoder layer of [TS] ``step`` on the residual stream ``x``
+    (``[hidden]``, float64): input norm -> q, k, v GEMVs -> per-head q/k norm
+    -> NeoX RoPE on q and on k -> K/V written at cache row ``pos`` ->
+    attention over rows ``[0, pos]`` -> o_proj -> residual add ->
+    post-attention norm -> gate, up -> SiLU-mul -> down -> residual add.
 
-    Precision points (where the GPU stores bf16, rounded here as well):
-    norm outputs feeding a GEMV, K and V written to the cache, the attention
-    output, and the SiLU-mul output. The residual stream, q/k/v GEMV
-    outputs and logits are float64 here (float32 on the GPU).
+    Precision points (where the GPU stores bf16, rounded here as well): norm
+    outputs feeding a GEMV, K and V written to the cache, the attention
+    output and the SiLU-mul output. The residual stream and q/k/v and
+    gate/up outputs stay float64 (float32 on the GPU).
 
-    ``k_cache``/``v_cache`` are float64 arrays ``[layers, Hkv, cap, D]``
-    holding bf16 values; row ``pos`` of every layer is overwritten.
-    Returns the logits ``[vocab]`` (float64).
-    """
+    ``k_cache_l``/``v_cache_l`` are ``[Hkv, cap, D]`` float64 arrays of bf16
+    values; row ``pos`` is overwritten. Returns the new residual stream."""
     H, Hkv, D = cfg["heads"], cfg["kv_heads"], cfg["head_dim"]
     eps, theta = cfg["eps"], cfg["theta"]
+    xn = round_bf16(rmsnorm(x, lw["input_norm"], eps))
+    q = gemv_affine8(*lw["q"], xn[None])[0]
+    k = gemv_affine8(*lw["k"], xn[None])[0]
+    v = gemv_affine8(*lw["v"], xn[None])[0]
+    q = rope_neox(rmsnorm_perhead(q, lw["q_norm"], eps, D), pos, theta, D)
+    k = rope_neox(rmsnorm_perhead(k, lw["k_norm"], eps, D), pos, theta, D)
+    k_cache_l[:, pos, :] = round_bf16(k).reshape(Hkv, D)
+    v_cache_l[:, pos, :] = round_bf16(v).reshape(Hkv, D)
+    att = round_bf16(decode_attention(q, k_cache_l, v_cache_l, pos + 1, H, Hkv, D))
+    x = x + gemv_affine8(*lw["o"], att[None])[0]
+    xn = round_bf16(rmsnorm(x, lw["post_norm"], eps))
+    gate = gemv_affine8(*lw["gate"], xn[None])[0]
+    up = gemv_affine8(*lw["up"], xn[None])[0]
+    hmid = round_bf16(silu_mul(gate, up))
+    return x + gemv_affine8(*lw["down"], hmid[None])[0]
+
+
+def lm_head(cfg, weights, x):
+    """Final RMSNorm (bf16 output) and the tied LM head of [TS] ``step``."""
+    ew, es, eb = weights["embed"]
+    xn = round_bf16(rmsnorm(x, weights["final_norm"], cfg["eps"]))
+    return gemv_affine8(ew, es, eb, xn[None])[0]
+
+
+def decode_step(cfg, weights, k_cache, v_cache, token, pos):
+    """One token of one sequence through every layer ([TS] ``step``): the
+    dequantized embedding row of [TS] ``embed_row_bytes``, ``decode_layer``
+    for each layer, then ``lm_head``. ``k_cache``/``v_cache`` are float64
+    ``[layers, Hkv, cap, D]``; row ``pos`` of every layer is overwritten.
+    Returns the logits ``[vocab]`` (float64)."""
     ew, es, eb = weights["embed"]
     x = embed_rows(ew, es, eb, [token])[0]
     for l, lw in enumerate(weights["layers"]):
-        xn = round_bf16(rmsnorm(x, lw["input_norm"], eps))
-        q = gemv_affine8(*lw["q"], xn[None])[0]
-        k = gemv_affine8(*lw["k"], xn[None])[0]
-        v = gemv_affine8(*lw["v"], xn[None])[0]
-        q = rope_neox(rmsnorm_perhead(q, lw["q_norm"], eps, D), pos, theta, D)
-        k = rope_neox(rmsnorm_perhead(k, lw["k_norm"], eps, D), pos, theta, D)
-        k_cache[l, :, pos, :] = round_bf16(k).reshape(Hkv, D)
-        v_cache[l, :, pos, :] = round_bf16(v).reshape(Hkv, D)
-        att = round_bf16(decode_attention(q, k_cache[l], v_cache[l], pos + 1, H, Hkv, D))
-        x = x + gemv_affine8(*lw["o"], att[None])[0]
-        xn = round_bf16(rmsnorm(x, lw["post_norm"], eps))
-        gate = gemv_affine8(*lw["gate"], xn[None])[0]
-        up = gemv_affine8(*lw["up"], xn[None])[0]
-        hmid = round_bf16(silu_mul(gate, up))
-        x = x + gemv_affine8(*lw["down"], hmid[None])[0]
-    xn = round_bf16(rmsnorm(x, weights["final_norm"], eps))
-    return gemv_affine8(ew, es, eb, xn[None])[0]
+        x = decode_layer(cfg, lw, x, k_cache[l], v_cache[l], pos)
+    return lm_head(cfg, weights, x)
 
 
 def new_kv_cache(cfg, cap):

@@ -1,0 +1,122 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry
+point include/qg.h declares, and refuses bad arguments before any launch with
+a message that names the argument (the refusal pattern of turbospark-runtime
+0.3.0, src/qwen3_asr_metal.rs, `open` / `load_packed_linear` and its
+`open_rejects_undersized_norm_tensors` test)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import weight_only_quantized_03_b200 as qg
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+FAKE = 0x7F0000000000  # a 256-byte aligned address that is never dereferenced
+
+
+def declared_functions():
+    with open(os.path.join(ROOT, "include", "qg.h")) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(qg_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for must in ["qg_gemv_affine8_g64", "qg_gemv_q4_0", "qg_gemm_q4_0", "qg_rmsnorm",
+                 "qg_rmsnorm_perhead", "qg_rope_neox", "qg_silu_mul", "qg_residual_add",
+                 "qg_decode_attention", "qg_decode_step", "qg_last_error"]:
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol():
+    for name in declared_functions():
+        assert hasattr(qg.lib, name), name
+    assert qg.lib.qg_abi_version() >= 1
+
+
+def _status(name, *args):
+    st = getattr(qg.lib, name)(*args)
+    return st, qg.last_error()
+
+
+def test_gemv_rejects_bad_k_batch_and_pointers():
+    st, msg = _status("qg_gemv_affine8_g64", FAKE, FAKE, FAKE, FAKE, qg.QG_BF16, FAKE, qg.QG_F32,
+                      None, 128, 100, 1, None)
+    assert st == qg.QG_ERR_UNSUPPORTED_SHAPE and "K=100" in msg
+    st, msg = _status("qg_gemv_affine8_g64", FAKE, FAKE, FAKE, FAKE, qg.QG_BF16, FAKE, qg.QG_F32,
+                      None, 128, 128, 33, None)
+    assert st == qg.QG_ERR_UNSUPPORTED_SHAPE and "B=33" in msg
+    st, msg = _status("qg_gemv_affine8_g64", None, FAKE, FAKE, FAKE, qg.QG_BF16, FAKE, qg.QG_F32,
+                      None, 128, 128, 1, None)
+    assert st == qg.QG_ERR_INVALID_ARGUMENT and "w=" in msg
+    st, msg = _status("qg_gemv_affine8_g64", FAKE + 4, FAKE, FAKE, FAKE, qg.QG_BF16, FAKE,
+                      qg.QG_F32, None, 128, 128, 1, None)
+    assert st == qg.QG_ERR_MISALIGNED and "w is not 16-byte aligned" in msg
+    st, msg = _status("qg_gemv_affine8_g64", FAKE, FAKE, FAKE, FAKE, 7, FAKE, qg.QG_F32, None,
+                      128, 128, 1, None)
+    assert st == qg.QG_ERR_INVALID_ARGUMENT and "x_dtype" in msg
+    # empty work is a valid no-op that launches nothing
+    st, msg = _status("qg_gemv_affine8_g64", None, None, None, None, qg.QG_BF16, None, qg.QG_F32,
+                      None, 0, 128, 1, None)
+    assert st == qg.QG_OK and msg == ""
+
+
+def test_q4_0_rejects_bad_k():
+    st, msg = _status("qg_gemv_q4_0", FAKE, FAKE, None, FAKE, 16, 48, 1, None)
+    assert st == qg.QG_ERR_UNSUPPORTED_SHAPE and "K=48" in msg
+
+
+def test_attention_rejects_bad_group_and_small_workspace():
+    st, msg = _status("qg_decode_attention", FAKE, FAKE, FAKE, FAKE, FAKE, qg.QG_BF16, 1, 12, 8,
+                      128, 64, 1.0, FAKE, 1 << 20, None)
+    assert st == qg.QG_ERR_UNSUPPORTED_SHAPE and "Hkv=8" in msg
+    need = qg.lib.qg_decode_attention_workspace_size(1, 16, 8, 128, 513)
+    assert need > 0
+    st, msg = _status("qg_decode_attention", FAKE, FAKE, FAKE, FAKE, FAKE, qg.QG_BF16, 1, 16, 8,
+                      128, 513, 1.0, FAKE, need - 1, None)
+    assert st == qg.QG_ERR_WORKSPACE_TOO_SMALL and str(need) in msg
+
+
+def test_elementwise_reject_bad_shapes():
+    assert _status("qg_rmsnorm", FAKE, FAKE, 1e-6, FAKE, qg.QG_BF16, 1, 6, None)[0] == \
+        qg.QG_ERR_UNSUPPORTED_SHAPE
+    st, msg = _status("qg_rope_neox", FAKE, qg.QG_F32, FAKE, 1e6, 1, 2, 128, 130, None)
+    assert st == qg.QG_ERR_UNSUPPORTED_SHAPE and "rotary_dim=130" in msg
+    assert _status("qg_rmsnorm_perhead", FAKE, qg.QG_F32, FAKE, 1e-6, FAKE, qg.QG_F32, 1, 2, 48,
+                   None)[0] == qg.QG_ERR_UNSUPPORTED_SHAPE
+
+
+def _tiny_model_structs(layers=2):
+    cfg = qg.qg_qwen3_config(64, layers, 2, 1, 64, 128, 261, 1e-5, 1e4)
+    mat = qg.qg_affine8_matrix(FAKE, FAKE, FAKE)
+    arr = (qg.qg_qwen3_layer * layers)()
+    for i in range(layers):
+        arr[i].input_norm = arr[i].post_norm = arr[i].q_norm = arr[i].k_norm = FAKE
+        for n in ("q", "k", "v", "o", "gate", "up", "down"):
+            setattr(arr[i], n, mat)
+    w = qg.qg_qwen3_weights(mat, FAKE, ctypes.cast(arr, ctypes.POINTER(qg.qg_qwen3_layer)))
+    return cfg, w, arr
+
+
+def test_decode_step_names_the_bad_tensor():
+    cfg, w, arr = _tiny_model_structs()
+    arr[1].down.w = None          # a missing matrix in layer 1
+    need = qg.lib.qg_decode_step_workspace_size(ctypes.byref(cfg), 1, 16)
+    st, msg = _status("qg_decode_step", ctypes.byref(cfg), ctypes.byref(w), FAKE, FAKE, 16, FAKE,
+                      FAKE, FAKE, 1, FAKE, need, None)
+    assert st == qg.QG_ERR_INVALID_ARGUMENT and "layer 1" in msg and "down" in msg
+    arr[1].down.w = FAKE
+    arr[0].k_norm = None          # a missing norm weight
+    st, msg = _status("qg_decode_step", ctypes.byref(cfg), ctypes.byref(w), FAKE, FAKE, 16, FAKE,
+                      FAKE, FAKE, 1, FAKE, need, None)
+    assert st == qg.QG_ERR_INVALID_ARGUMENT and "layer 0" in msg and "norm" in msg
+    arr[0].k_norm = FAKE
+    st, msg = _status("qg_decode_step", ctypes.byref(cfg), ctypes.byref(w), FAKE, FAKE, 16, FAKE,
+                      FAKE, FAKE, 1, FAKE, need - 256, None)
+    assert st == qg.QG_ERR_WORKSPACE_TOO_SMALL
+    bad = qg.qg_qwen3_config(64, 2, 3, 2, 64, 128, 261, 1e-5, 1e4)
+    st, msg = _status("qg_decode_step", ctypes.byref(bad), ctypes.byref(w), FAKE, FAKE, 16, FAKE,
+                      FAKE, FAKE, 1, FAKE, need, None)
+    assert st == qg.QG_ERR_UNSUPPORTED_SHAPE and "kv_heads=2" in msg

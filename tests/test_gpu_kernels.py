@@ -1,0 +1,255 @@
+"""GPU parity of the single-op kernels against the oracle (through the C ABI).
+
+Unpack and dequant are compared bit for bit; fp32-accumulated outputs within
+|gpu - ref| <= 2e-3 + 1e-3 |ref| (plus half a bf16 ulp for bf16 stores).
+Shapes span several tiles with ragged tails, the degenerate sizes (one row,
+one group, batch 1 and 32) and the full model shapes (sampled rows where the
+oracle would be too slow for all of them).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import qg_synth
+from oracle import qg_oracle as O
+from tests.gpu_util import assert_parity, bf16_dev, dev, host64
+
+pytestmark = pytest.mark.gpu
+
+qg = pytest.importorskip("weight_only_quantized_03_b200")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+
+
+def _affine8(N, K, seed, quantized):
+    if quantized:
+        return O.affine8_quantize(qg_synth.gaussian((N, K), 0.02, seed))
+    return qg_synth.affine8_packed(N, K, seed)
+
+
+# ----------------------------------------------------------- bit-exact -----
+
+@pytest.mark.parametrize("N,K,kind", [(3, 64, "fixture"), (33, 192, "quantized"),
+                                      (2048, 1024, "random")])
+def test_unpack_and_dequant_affine8_bit_exact(N, K, kind):
+    if kind == "fixture":
+        w, s, b = qg_synth.affine8_fixture(N, K, 0x5EED12340001)
+    else:
+        w, s, b = _affine8(N, K, 7, kind == "quantized")
+    out = torch.empty((N, K), dtype=torch.float32, device="cuda")
+    qg.qg_unpack_affine8(dev(w), out)
+    np.testing.assert_array_equal(out.cpu().numpy(), O.affine8_unpack(w).astype(np.float32))
+    qg.qg_dequant_affine8_g64(dev(w), dev(s), dev(b), out)
+    np.testing.assert_array_equal(out.cpu().numpy().view(np.uint32),
+                                  O.affine8_dequant_f32(w, s, b).view(np.uint32))
+
+
+@pytest.mark.parametrize("N,K,kind", [(17, 96, "quantized"), (1280, 1280, "random"),
+                                      (5, 5120, "random")])
+def test_dequant_q4_0_bit_exact(N, K, kind):
+    blocks = (O.q4_0_quantize(qg_synth.gaussian((N, K), 0.02, 8)) if kind == "quantized"
+              else qg_synth.q4_0_packed(N, K, 9))
+    out = torch.empty((N, K), dtype=torch.float32, device="cuda")
+    qg.qg_dequant_q4_0(dev(blocks), out)
+    got = out.cpu().numpy()
+    want = O.q4_0_dequant_exact(blocks, K).astype(np.float32)
+    np.testing.assert_array_equal(got, want)                       # -0.0 == +0.0 here
+    np.testing.assert_array_equal(np.signbit(got), np.signbit(want))
+
+
+# ------------------------------------------------------- affine8 GEMV ------
+
+GEMV_CASES = [
+    # N, K, B, x_dtype, y_dtype, residual, quantized weights
+    (1, 64, 1, "bf16", "f32", False, True),
+    (7, 128, 3, "bf16", "f32", True, True),
+    (1000, 1024, 1, "bf16", "f32", False, False),
+    (1024, 1024, 1, "bf16", "bf16", False, True),
+    (2048, 1024, 4, "bf16", "f32", False, False),
+    (3072, 1024, 16, "bf16", "f32", False, False),
+    (1024, 3072, 1, "bf16", "f32", True, False),
+    (1024, 2048, 2, "f32", "f32", True, False),
+    (33, 192, 32, "bf16", "bf16", False, True),
+    (4100, 64, 9, "f32", "f32", False, False),
+    (300, 6144, 5, "bf16", "f32", False, False),
+    (9473, 256, 1, "bf16", "f32", False, False),
+    (40000, 128, 2, "bf16", "f32", False, False),
+]
+
+
+@pytest.mark.parametrize("N,K,B,xd,yd,res,quant", GEMV_CASES)
+def test_gemv_affine8(N, K, B, xd, yd, res, quant):
+    w, s, b = _affine8(N, K, 100 + N + K + B, quant)
+    xbits = qg_synth.gaussian_bf16_bits((B, K), 1.0, 200 + B)
+    if xd == "bf16":
+        x_d = bf16_dev(xbits)
+        x64 = O.bf16_bits_to_f64(xbits)
+    else:
+        xf = qg_synth.gaussian((B, K), 1.0, 201 + B)
+        x_d = dev(xf)
+        x64 = xf.astype(np.float64)
+    r = qg_synth.gaussian((B, N), 1.0, 300) if res else None
+    y = torch.empty((B, N), dtype=torch.float32 if yd == "f32" else torch.bfloat16, device="cuda")
+    if res and yd == "f32":
+        y.copy_(dev(r))            # in place: y = W x + y
+        rr = y
+    else:
+        rr = dev(r) if res else None
+    qg.qg_gemv_affine8_g64(dev(w), dev(s), dev(b), x_d, y, residual=rr)
+    ref = O.gemv_affine8(w, s, b, x64, residual=r)
+    assert_parity(host64(y), ref, bf16_out=(yd == "bf16"), what=f"gemv {N}x{K} B={B}")
+
+
+def test_gemv_affine8_lm_head_full_size_sampled_rows():
+    # the tied LM head of the 0.6B shape: 151936 x 1024, batch 1 (and 4)
+    N, K = 151936, 1024
+    w, s, b = qg_synth.affine8_packed(N, K, 4242)
+    for B in (1, 4):
+        xbits = qg_synth.gaussian_bf16_bits((B, K), 1.0, 4243 + B)
+        y = torch.empty((B, N), dtype=torch.float32, device="cuda")
+        qg.qg_gemv_affine8_g64(dev(w), dev(s), dev(b), bf16_dev(xbits), y)
+        rows = np.sort(np.random.default_rng(B).choice(N, 3000, replace=False))
+        rows = np.concatenate([[0, N - 1], rows])
+        ref = O.gemv_affine8(w[rows], s[rows], b[rows], O.bf16_bits_to_f64(xbits))
+        assert_parity(host64(y)[:, rows], ref, what=f"lm head B={B}")
+
+
+# ---------------------------------------------------------- Q4_0 GEMV ------
+
+Q4_CASES = [
+    (1280, 1280, 1, True, False), (5120, 1280, 1, True, False), (1280, 5120, 1, True, False),
+    (1280, 1280, 1, False, True), (7, 32, 3, True, True), (100, 96, 32, False, False),
+    (64, 256, 8, True, False), (333, 2048, 5, False, False),
+]
+
+
+@pytest.mark.parametrize("N,K,B,bias,quant", Q4_CASES)
+def test_gemv_q4_0(N, K, B, bias, quant):
+    blocks = (O.q4_0_quantize(qg_synth.gaussian((N, K), 0.02, 11)) if quant
+              else qg_synth.q4_0_packed(N, K, 12))
+    x = qg_synth.gaussian((B, K), 1.0, 13)
+    bv = qg_synth.gaussian((N,), 1.0, 14) if bias else None
+    y = torch.empty((B, N), dtype=torch.float32, device="cuda")
+    qg.qg_gemv_q4_0(dev(blocks), dev(x), y, bias=dev(bv) if bias else None)
+    ref = O.gemv_q4_0(blocks, x.astype(np.float64), None if bv is None else bv.astype(np.float64))
+    assert_parity(host64(y), ref, what=f"q4_0 gemv {N}x{K} B={B}")
+
+
+# -------------------------------------------------------- elementwise ------
+
+@pytest.mark.parametrize("rows,dim,eps,yd", [(1, 1024, 1e-6, "bf16"), (10, 1024, 1e-6, "f32"),
+                                             (3, 64, 1e-5, "bf16"), (2, 2048, 1e-6, "bf16"),
+                                             (5, 4, 1e-6, "f32")])
+def test_rmsnorm(rows, dim, eps, yd):
+    x = qg_synth.gaussian((rows, dim), 3.0, 20)
+    w = qg_synth.f32_to_bf16_bits((1 + 0.2 * qg_synth.gaussian((dim,), 1.0, 21)).astype(np.float32))
+    y = torch.empty((rows, dim), dtype=torch.float32 if yd == "f32" else torch.bfloat16,
+                    device="cuda")
+    qg.qg_rmsnorm(dev(x), dev(w), eps, y)
+    assert_parity(host64(y), O.rmsnorm(x, w, eps), bf16_out=(yd == "bf16"), what="rmsnorm")
+
+
+@pytest.mark.parametrize("xd,yd,D", [("f32", "f32", 128), ("bf16", "bf16", 128),
+                                     ("f32", "bf16", 64), ("f32", "f32", 256)])
+def test_rmsnorm_perhead(xd, yd, D):
+    rows, heads = 3, 16
+    xf = qg_synth.gaussian((rows, heads * D), 2.0, 22)
+    w = qg_synth.f32_to_bf16_bits((1 + 0.2 * qg_synth.gaussian((D,), 1.0, 23)).astype(np.float32))
+    if xd == "bf16":
+        bits = qg_synth.f32_to_bf16_bits(xf)
+        x_d, x64 = bf16_dev(bits), O.bf16_bits_to_f64(bits)
+    else:
+        x_d, x64 = dev(xf), xf.astype(np.float64)
+    y = torch.empty((rows, heads * D), dtype=torch.float32 if yd == "f32" else torch.bfloat16,
+                    device="cuda")
+    qg.qg_rmsnorm_perhead(x_d, dev(w), 1e-6, y, heads)
+    assert_parity(host64(y), O.rmsnorm_perhead(x64, w, 1e-6, D), bf16_out=(yd == "bf16"),
+                  what="perhead")
+
+
+@pytest.mark.parametrize("dt,rd,theta", [("f32", 128, 1e6), ("bf16", 128, 1e6), ("f32", 64, 1e4)])
+def test_rope_neox(dt, rd, theta):
+    D, heads = 128, 8
+    pos = np.array([0, 1, 511, 2047, 32767], dtype=np.int32)
+    xf = qg_synth.gaussian((len(pos), heads * D), 1.0, 24)
+    if dt == "bf16":
+        bits = qg_synth.f32_to_bf16_bits(xf)
+        x_d, x64 = bf16_dev(bits), O.bf16_bits_to_f64(bits)
+    else:
+        x_d, x64 = dev(xf), xf.astype(np.float64)
+    qg.qg_rope_neox(x_d, dev(pos), theta, heads, rotary_dim=rd)
+    ref = np.stack([O.rope_neox(x64[i], int(p), theta, D, rd) for i, p in enumerate(pos)])
+    assert_parity(host64(x_d), ref, bf16_out=(dt == "bf16"), what="rope")
+
+
+@pytest.mark.parametrize("n,od", [(3072, "bf16"), (30720, "f32"), (1, "bf16")])
+def test_silu_mul(n, od):
+    g = qg_synth.gaussian((n,), 4.0, 25)
+    u = qg_synth.gaussian((n,), 1.0, 26)
+    out = torch.empty(n, dtype=torch.float32 if od == "f32" else torch.bfloat16, device="cuda")
+    qg.qg_silu_mul(dev(g), dev(u), out)
+    assert_parity(host64(out), O.silu_mul(g, u), bf16_out=(od == "bf16"), what="silu_mul")
+
+
+def test_residual_add():
+    x = qg_synth.gaussian((5000,), 1.0, 27)
+    d = qg_synth.gaussian((5000,), 1.0, 28)
+    xd = dev(x)
+    qg.qg_residual_add(xd, dev(d))
+    assert_parity(host64(xd), x.astype(np.float64) + d, what="residual")
+
+
+def test_embed_rows_bit_exact_and_bad_token():
+    V, Hd = 261, 64
+    w, s, b = qg_synth.affine8_fixture(V, Hd, 0x5EED12340001)
+    toks = np.array([0, 260, 17, -1, 261], dtype=np.int32)
+    x = torch.empty((len(toks), Hd), dtype=torch.float32, device="cuda")
+    qg.qg_embed_affine8_g64(dev(w), dev(s), dev(b), dev(toks), x)
+    got = x.cpu().numpy()
+    np.testing.assert_array_equal(got[:3], O.embed_rows(w, s, b, toks[:3]).astype(np.float32))
+    assert np.isnan(got[3:]).all()
+
+
+# ---------------------------------------------------------- attention ------
+
+ATTN_CASES = [
+    # B, H, Hkv, D, cap, kv_len per sequence
+    (1, 16, 8, 128, 513, [512]),
+    (1, 16, 8, 128, 513, [1]),
+    (2, 16, 8, 128, 600, [33, 600]),
+    (3, 2, 1, 64, 70, [31, 32, 64]),
+    (1, 4, 4, 256, 40, [40]),
+    (10, 16, 8, 128, 513, [512, 1, 100, 511, 256, 2, 3, 400, 512, 77]),
+    (1, 16, 8, 128, 2048, [2048]),
+    (2, 8, 1, 32, 5, [0, 6]),          # invalid lengths -> zero rows
+]
+
+
+@pytest.mark.parametrize("B,H,Hkv,D,cap,lens", ATTN_CASES)
+def test_decode_attention(B, H, Hkv, D, cap, lens):
+    kbits = qg_synth.gaussian_bf16_bits((B, Hkv, cap, D), 1.0, 30)
+    vbits = qg_synth.gaussian_bf16_bits((B, Hkv, cap, D), 1.0, 31)
+    q = qg_synth.gaussian((B, H * D), 1.0, 32)
+    kv_len = np.array(lens, dtype=np.int32)
+    ws = torch.empty(qg.qg_decode_attention_workspace_size(B, H, Hkv, D, cap), dtype=torch.uint8,
+                     device="cuda")
+    for od in ("f32", "bf16"):
+        out = torch.empty((B, H * D), dtype=torch.float32 if od == "f32" else torch.bfloat16,
+                          device="cuda")
+        qg.qg_decode_attention(dev(q), bf16_dev(kbits), bf16_dev(vbits), dev(kv_len), out, H, Hkv,
+                               1.0 / math.sqrt(D), ws)
+        got = host64(out)
+        k64, v64 = O.bf16_bits_to_f64(kbits), O.bf16_bits_to_f64(vbits)
+        for b in range(B):
+            L = int(kv_len[b])
+            if 1 <= L <= cap:
+                ref = O.decode_attention(q[b], k64[b], v64[b], L, H, Hkv, D)
+                assert_parity(got[b], ref, bf16_out=(od == "bf16"), what=f"attn b={b} L={L}")
+            else:
+                assert np.all(got[b] == 0.0)

@@ -1,0 +1,283 @@
+"""Python binding of libqg, weight-only-quantized decode kernels for B200.
+
+Argument marshalling only: every function here forwards torch tensors' device
+pointers, shapes and the current CUDA stream to the C ABI of the same name
+(include/qg.h) and raises QGError when it returns a non-zero status. No
+computation happens in Python and there is no fallback: importing this module
+fails if libqg.so is missing.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqg.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m weight_only_quantized_03_b200.build`"
+    )
+lib = ctypes.CDLL(LIB_PATH)
+
+QG_OK = 0
+QG_ERR_INVALID_ARGUMENT = 1
+QG_ERR_UNSUPPORTED_SHAPE = 2
+QG_ERR_MISALIGNED = 3
+QG_ERR_WORKSPACE_TOO_SMALL = 4
+QG_ERR_CUDA = 5
+QG_ERR_TIMEOUT = 6
+QG_F32 = 0
+QG_BF16 = 1
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_f = ctypes.c_float
+_d = ctypes.c_double
+_sz = ctypes.c_size_t
+
+
+class QGError(RuntimeError):
+    def __init__(self, name, status, msg):
+        super().__init__(f"{name} returned {status}: {msg}")
+        self.status = status
+
+
+class qg_affine8_matrix(ctypes.Structure):
+    _fields_ = [("w", _vp), ("scales", _vp), ("biases", _vp)]
+
+
+class qg_qwen3_layer(ctypes.Structure):
+    _fields_ = [("input_norm", _vp), ("post_norm", _vp), ("q_norm", _vp), ("k_norm", _vp)] + [
+        (n, qg_affine8_matrix) for n in ("q", "k", "v", "o", "gate", "up", "down")]
+
+
+class qg_qwen3_config(ctypes.Structure):
+    _fields_ = [("hidden", _i), ("layers", _i), ("heads", _i), ("kv_heads", _i),
+                ("head_dim", _i), ("ffn", _i), ("vocab", _i), ("eps", _f), ("theta", _d)]
+
+
+class qg_qwen3_weights(ctypes.Structure):
+    _fields_ = [("embed", qg_affine8_matrix), ("final_norm", _vp),
+                ("layers", ctypes.POINTER(qg_qwen3_layer))]
+
+
+_SIGS = {
+    "qg_last_error": (ctypes.c_char_p, []),
+    "qg_abi_version": (_i, []),
+    "qg_kernel_launch_count": (ctypes.c_ulonglong, []),
+    "qg_gemv_affine8_g64": (_i, [_vp, _vp, _vp, _vp, _i, _vp, _i, _vp, _i, _i, _i, _vp]),
+    "qg_gemv_q4_0": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _vp]),
+    "qg_gemm_q4_0_workspace_size": (_sz, [_i, _i, _i]),
+    "qg_gemm_q4_0": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _vp, _sz, _vp]),
+    "qg_rmsnorm": (_i, [_vp, _vp, _f, _vp, _i, _i, _i, _vp]),
+    "qg_rmsnorm_perhead": (_i, [_vp, _i, _vp, _f, _vp, _i, _i, _i, _i, _vp]),
+    "qg_rope_neox": (_i, [_vp, _i, _vp, _d, _i, _i, _i, _i, _vp]),
+    "qg_silu_mul": (_i, [_vp, _vp, _vp, _i, _i, _vp]),
+    "qg_residual_add": (_i, [_vp, _vp, _i, _vp]),
+    "qg_embed_affine8_g64": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp]),
+    "qg_decode_attention_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
+    "qg_decode_attention": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _sz,
+                                 _vp]),
+    "qg_decode_step_workspace_size": (_sz, [ctypes.POINTER(qg_qwen3_config), _i, _i]),
+    "qg_decode_step": (_i, [ctypes.POINTER(qg_qwen3_config), ctypes.POINTER(qg_qwen3_weights),
+                            _vp, _vp, _i, _vp, _vp, _vp, _i, _vp, _sz, _vp]),
+    "qg_unpack_affine8": (_i, [_vp, _vp, _i, _i, _vp]),
+    "qg_dequant_affine8_g64": (_i, [_vp, _vp, _vp, _vp, _i, _i, _vp]),
+    "qg_dequant_q4_0": (_i, [_vp, _vp, _i, _i, _vp]),
+}
+
+for _name, (_res, _args) in _SIGS.items():
+    _fn = getattr(lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+
+def last_error() -> str:
+    return lib.qg_last_error().decode()
+
+
+def _call(name, *args):
+    st = getattr(lib, name)(*args)
+    if st != QG_OK:
+        raise QGError(name, st, last_error())
+
+
+def _p(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream=None):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
+
+
+def _dt(t):
+    if t.dtype == torch.float32:
+        return QG_F32
+    if t.dtype == torch.bfloat16:
+        return QG_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+# ------------------------------------------------------------------ ops ----
+
+def qg_gemv_affine8_g64(w, scales, biases, x, y, residual=None, stream=None):
+    """y[B,N] = dequant(w, scales, biases)[N,K] @ x[B,K] (+ residual). w is
+    int32/uint32-viewed [N, K/4]; scales/biases int16/bf16 bits [N, K/64]."""
+    N, K = w.shape[0], w.shape[1] * 4
+    B = x.shape[0] if x.dim() == 2 else 1
+    _call("qg_gemv_affine8_g64", _p(w), _p(scales), _p(biases), _p(x), _dt(x), _p(y), _dt(y),
+          _p(residual), N, K, B, _stream(stream))
+
+
+def qg_gemv_q4_0(blocks, x, y, bias=None, stream=None):
+    N = blocks.shape[0]
+    K = blocks.shape[1] // 18 * 32
+    B = x.shape[0] if x.dim() == 2 else 1
+    _call("qg_gemv_q4_0", _p(blocks), _p(x), _p(bias), _p(y), N, K, B, _stream(stream))
+
+
+def qg_gemm_q4_0_workspace_size(M, N, K):
+    return int(lib.qg_gemm_q4_0_workspace_size(M, N, K))
+
+
+def qg_gemm_q4_0(blocks, A, C, bias=None, ws=None, stream=None):
+    N = blocks.shape[0]
+    K = blocks.shape[1] // 18 * 32
+    M = A.shape[0]
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _call("qg_gemm_q4_0", _p(blocks), _p(A), _p(bias), _p(C), M, N, K, _p(ws), nbytes,
+          _stream(stream))
+
+
+def qg_rmsnorm(x, w, eps, y, stream=None):
+    rows, dim = x.shape
+    _call("qg_rmsnorm", _p(x), _p(w), float(eps), _p(y), _dt(y), rows, dim, _stream(stream))
+
+
+def qg_rmsnorm_perhead(x, w, eps, y, heads, stream=None):
+    rows = x.shape[0]
+    D = x.shape[1] // heads
+    _call("qg_rmsnorm_perhead", _p(x), _dt(x), _p(w), float(eps), _p(y), _dt(y), rows, heads, D,
+          _stream(stream))
+
+
+def qg_rope_neox(x, pos, theta, heads, rotary_dim=None, stream=None):
+    rows = x.shape[0]
+    D = x.shape[1] // heads
+    _call("qg_rope_neox", _p(x), _dt(x), _p(pos), float(theta), rows, heads, D,
+          D if rotary_dim is None else rotary_dim, _stream(stream))
+
+
+def qg_silu_mul(gate, up, out, stream=None):
+    _call("qg_silu_mul", _p(gate), _p(up), _p(out), _dt(out), gate.numel(), _stream(stream))
+
+
+def qg_residual_add(x, delta, stream=None):
+    _call("qg_residual_add", _p(x), _p(delta), x.numel(), _stream(stream))
+
+
+def qg_embed_affine8_g64(w, scales, biases, tokens, x, stream=None):
+    _call("qg_embed_affine8_g64", _p(w), _p(scales), _p(biases), _p(tokens), _p(x), w.shape[0],
+          w.shape[1] * 4, tokens.numel(), _stream(stream))
+
+
+def qg_decode_attention_workspace_size(B, H, Hkv, D, cap):
+    return int(lib.qg_decode_attention_workspace_size(B, H, Hkv, D, cap))
+
+
+def qg_decode_attention(q, k_cache, v_cache, kv_len, out, H, Hkv, scale, ws, stream=None):
+    """q [B, H*D] fp32; caches [B, Hkv, cap, D] bf16; kv_len int32 [B]."""
+    B, _, cap, D = k_cache.shape
+    _call("qg_decode_attention", _p(q), _p(k_cache), _p(v_cache), _p(kv_len), _p(out), _dt(out),
+          B, H, Hkv, D, cap, float(scale), _p(ws), ws.numel() * ws.element_size(),
+          _stream(stream))
+
+
+def qg_unpack_affine8(w, out, stream=None):
+    _call("qg_unpack_affine8", _p(w), _p(out), w.shape[0], w.shape[1] * 4, _stream(stream))
+
+
+def qg_dequant_affine8_g64(w, scales, biases, out, stream=None):
+    _call("qg_dequant_affine8_g64", _p(w), _p(scales), _p(biases), _p(out), w.shape[0],
+          w.shape[1] * 4, _stream(stream))
+
+
+def qg_dequant_q4_0(blocks, out, stream=None):
+    _call("qg_dequant_q4_0", _p(blocks), _p(out), blocks.shape[0], blocks.shape[1] // 18 * 32,
+          _stream(stream))
+
+
+# ---------------------------------------------------------- decode step ----
+
+class Qwen3Model:
+    """Device-resident packed Qwen3 weights plus the C structs that point at
+    them. ``weights`` is the host dict layout of ``qg_synth.qwen3_weights``
+    (numpy arrays); everything is uploaded once to ``device``."""
+
+    def __init__(self, cfg: dict, weights: dict, device="cuda"):
+        self.cfg = dict(cfg)
+        self._keep = []
+
+        def up(a):
+            t = torch.from_numpy(a.view({2: "int16", 4: "int32"}[a.dtype.itemsize])).to(device)
+            self._keep.append(t)
+            return t.data_ptr()
+
+        def mat(triple):
+            w, s, b = triple
+            return qg_affine8_matrix(up(w), up(s), up(b))
+
+        self.c_cfg = qg_qwen3_config(cfg["hidden"], cfg["layers"], cfg["heads"], cfg["kv_heads"],
+                                     cfg["head_dim"], cfg["ffn"], cfg["vocab"], cfg["eps"],
+                                     cfg["theta"])
+        L = cfg["layers"]
+        self.c_layers = (qg_qwen3_layer * max(L, 1))()
+        for i, lw in enumerate(weights["layers"]):
+            cl = self.c_layers[i]
+            cl.input_norm = up(lw["input_norm"])
+            cl.post_norm = up(lw["post_norm"])
+            cl.q_norm = up(lw["q_norm"])
+            cl.k_norm = up(lw["k_norm"])
+            for n in ("q", "k", "v", "o", "gate", "up", "down"):
+                setattr(cl, n, mat(lw[n]))
+        self.c_weights = qg_qwen3_weights(mat(weights["embed"]), up(weights["final_norm"]),
+                                          ctypes.cast(self.c_layers, ctypes.POINTER(qg_qwen3_layer)))
+        self.device = device
+
+    def workspace_size(self, B, cap):
+        return int(lib.qg_decode_step_workspace_size(ctypes.byref(self.c_cfg), B, cap))
+
+    def new_state(self, B, cap):
+        """Zeroed KV caches [layers, B, kv_heads, cap, head_dim] bf16, a
+        workspace and a logits buffer for batch B."""
+        c = self.cfg
+        shape = (c["layers"], B, c["kv_heads"], cap, c["head_dim"])
+        return dict(
+            k_cache=torch.zeros(shape, dtype=torch.bfloat16, device=self.device),
+            v_cache=torch.zeros(shape, dtype=torch.bfloat16, device=self.device),
+            ws=torch.empty(self.workspace_size(B, cap), dtype=torch.uint8, device=self.device),
+            logits=torch.empty((B, c["vocab"]), dtype=torch.float32, device=self.device),
+            B=B, cap=cap)
+
+    def residual(self, state):
+        """The fp32 residual stream [B, hidden] after the last layer of the
+        latest step (the head of the step workspace, per include/qg.h)."""
+        n = state["B"] * self.cfg["hidden"]
+        return state["ws"][: 4 * n].view(torch.float32).view(state["B"], self.cfg["hidden"])
+
+    def qg_decode_step(self, state, tokens, positions, stream=None, layers=None):
+        """tokens, positions: device int32 [B]. Writes state['logits'].
+        ``layers`` runs only the first that many layers (then the head)."""
+        cfg = self.c_cfg
+        if layers is not None:
+            cfg = qg_qwen3_config.from_buffer_copy(self.c_cfg)
+            cfg.layers = layers
+        _call("qg_decode_step", ctypes.byref(cfg), ctypes.byref(self.c_weights),
+              _p(state["k_cache"]), _p(state["v_cache"]), state["cap"], _p(tokens),
+              _p(positions), _p(state["logits"]), state["B"], _p(state["ws"]),
+              state["ws"].numel(), _stream(stream))

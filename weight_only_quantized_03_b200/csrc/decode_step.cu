@@ -1,0 +1,286 @@
+// One Qwen3 decode step for B independent sequences.
+//
+// Op order: turbospark-runtime 0.3.0, src/qwen3_asr_metal.rs, `step`:
+// input norm -> q, k, v -> per-head q/k norm -> NeoX RoPE on q and on k ->
+// K/V stored at cache row `position` -> attention over rows [0, position]
+// -> o_proj -> residual -> post-attention norm -> gate, up -> SiLU-mul ->
+// down -> residual; then the final norm and the tied LM head. The embedding
+// row is dequantized from the packed table (embed_row_bytes).
+//
+// Every launch after the first uses Programmatic Dependent Launch: a GEMV
+// issues its first weight loads before waiting for the previous kernel, so
+// weight streaming overlaps the previous kernel's tail. Nothing here
+// synchronises or allocates, so a step can be captured into a CUDA graph.
+#include "qg_internal.cuh"
+
+namespace qg {
+
+size_t attention_ws_counter_offset(int B, int H, int Hkv, int D, int cap);
+
+struct StepLayout {
+  size_t x, xn, q, k, v, attn, gate, up, h, attn_ws, total;
+};
+
+static size_t a256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+static StepLayout step_layout(const qg_qwen3_config& c, int B, int cap) {
+  StepLayout L;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off += a256(bytes); return o; };
+  const size_t qd = (size_t)c.heads * c.head_dim, kd = (size_t)c.kv_heads * c.head_dim;
+  L.x = take((size_t)B * c.hidden * 4);
+  L.xn = take((size_t)B * c.hidden * 2);
+  L.q = take((size_t)B * qd * 4);
+  L.k = take((size_t)B * kd * 4);
+  L.v = take((size_t)B * kd * 4);
+  L.attn = take((size_t)B * qd * 2);
+  L.gate = take((size_t)B * c.ffn * 4);
+  L.up = take((size_t)B * c.ffn * 4);
+  L.h = take((size_t)B * c.ffn * 2);
+  L.attn_ws = take(attention_ws_bytes(B, c.heads, c.kv_heads, c.head_dim, cap));
+  L.total = off;
+  return L;
+}
+
+// Embedding rows; a sequence with a bad token or position gets NaN.
+__global__ void step_embed_kernel(const uint32_t* __restrict__ w, const uint16_t* __restrict__ s,
+                                  const uint16_t* __restrict__ bi, const int32_t* __restrict__ tok,
+                                  const int32_t* __restrict__ pos, float* __restrict__ x, int vocab,
+                                  int hidden, int cap) {
+  pdl_wait();
+  const int b = blockIdx.x;
+  const int t = tok[b], p = pos[b];
+  const bool ok = t >= 0 && t < vocab && p >= 0 && p < cap;
+  float* xr = x + (size_t)b * hidden;
+  for (int c = threadIdx.x; c < hidden; c += blockDim.x) {
+    if (!ok) {
+      xr[c] = __int_as_float(0x7fc00000);
+      continue;
+    }
+    const uint32_t word = w[(size_t)t * (hidden / 4) + c / 4];
+    const float q = (float)((word >> (8 * (c % 4))) & 0xFFu);
+    const size_t g = (size_t)t * (hidden / 64) + c / 64;
+    xr[c] = fmaf(q, bf16_bits_to_f32(s[g]), bf16_bits_to_f32(bi[g]));
+  }
+  pdl_trigger();
+}
+
+// Per-head q/k RMSNorm + NeoX RoPE (rotary_dim = head_dim) + K/V append.
+// Grid (H + 2*Hkv, B); one warp per head. q is rewritten in place (fp32);
+// K (normed, rotated) and V go to cache row pos as bf16.
+__global__ void step_qk_rope_append_kernel(float* __restrict__ q, const float* __restrict__ k,
+                                           const float* __restrict__ v,
+                                           const uint16_t* __restrict__ qn,
+                                           const uint16_t* __restrict__ kn,
+                                           const int32_t* __restrict__ pos,
+                                           const int32_t* __restrict__ tok,
+                                           uint16_t* __restrict__ kc, uint16_t* __restrict__ vc,
+                                           int H, int Hkv, int D, int cap, int vocab, float eps,
+                                           double theta) {
+  pdl_wait();
+  const int head = blockIdx.x, b = blockIdx.y, lane = threadIdx.x;
+  const int p = pos[b], t = tok[b];
+  // a bad token or position: nothing is written to the cache
+  const bool pos_ok = p >= 0 && p < cap && t >= 0 && t < vocab;
+  const int half = D >> 1, per = half >> 5;  // pairs per lane (D % 64 == 0) or 0
+  float* src;
+  const uint16_t* nw = nullptr;
+  uint16_t* dst = nullptr;
+  bool is_v = false;
+  if (head < H) {
+    src = q + ((size_t)b * H + head) * D;
+    nw = qn;
+  } else if (head < H + Hkv) {
+    const int kh = head - H;
+    src = const_cast<float*>(k) + ((size_t)b * Hkv + kh) * D;
+    nw = kn;
+    dst = kc + (((size_t)b * Hkv + kh) * cap + (pos_ok ? p : 0)) * D;
+  } else {
+    const int kh = head - H - Hkv;
+    src = const_cast<float*>(v) + ((size_t)b * Hkv + kh) * D;
+    dst = vc + (((size_t)b * Hkv + kh) * cap + (pos_ok ? p : 0)) * D;
+    is_v = true;
+  }
+  if (is_v) {
+    if (pos_ok)
+      for (int d = lane; d < D; d += 32) dst[d] = f32_to_bf16_bits(src[d]);
+    pdl_trigger();
+    return;
+  }
+  // D <= 256: each lane holds the pair (i, i+half) for i = lane + 32*j
+  float x1[4], x2[4];
+  float ss = 0.f;
+  for (int j = 0; j < 4; ++j) {
+    const int i = lane + 32 * j;
+    x1[j] = i < half ? src[i] : 0.f;
+    x2[j] = i < half ? src[i + half] : 0.f;
+    ss = fmaf(x1[j], x1[j], fmaf(x2[j], x2[j], ss));
+  }
+  ss = warp_sum(ss);
+  const float inv = 1.0f / sqrtf(ss / (float)D + eps);
+  for (int j = 0; j < 4; ++j) {
+    const int i = lane + 32 * j;
+    if (i >= half) break;
+    const float a = x1[j] * inv * bf16_bits_to_f32(nw[i]);
+    const float c2 = x2[j] * inv * bf16_bits_to_f32(nw[i + half]);
+    const double inv_freq = pow(theta, -2.0 * (double)i / (double)D);
+    double sd, cd;
+    sincos((double)(pos_ok ? p : 0) * inv_freq, &sd, &cd);
+    const float cs = (float)cd, sn = (float)sd;
+    const float r1 = a * cs - c2 * sn, r2 = c2 * cs + a * sn;
+    if (dst) {
+      if (pos_ok) {
+        dst[i] = f32_to_bf16_bits(r1);
+        dst[i + half] = f32_to_bf16_bits(r2);
+      }
+    } else {
+      src[i] = r1;
+      src[i + half] = r2;
+    }
+  }
+  (void)per;
+  pdl_trigger();
+}
+
+__global__ void step_silu_mul_kernel(const float* __restrict__ g, const float* __restrict__ u,
+                                     uint16_t* __restrict__ out, int n) {
+  pdl_wait();
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    const float z = g[i];
+    out[i] = f32_to_bf16_bits(z / (1.0f + expf(-z)) * u[i]);
+  }
+  pdl_trigger();
+}
+
+}  // namespace qg
+
+using namespace qg;
+
+static qg_status validate_matrix(const qg_affine8_matrix& m, const char* name, int layer) {
+  QG_REQUIRE(m.w && m.scales && m.biases, QG_ERR_INVALID_ARGUMENT,
+             "qg_decode_step: layer %d matrix %s has a null pointer", layer, name);
+  QG_REQUIRE(aligned(m.w, 16), QG_ERR_MISALIGNED,
+             "qg_decode_step: layer %d matrix %s weights not 16-byte aligned", layer, name);
+  QG_REQUIRE(aligned(m.scales, 2) && aligned(m.biases, 2), QG_ERR_MISALIGNED,
+             "qg_decode_step: layer %d matrix %s scales/biases misaligned", layer, name);
+  return QG_OK;
+}
+
+static qg_status validate_cfg(const qg_qwen3_config* c, int B, int cap) {
+  QG_REQUIRE(c, QG_ERR_INVALID_ARGUMENT, "qg_decode_step: cfg is NULL");
+  QG_REQUIRE(c->hidden > 0 && c->hidden % 64 == 0, QG_ERR_UNSUPPORTED_SHAPE,
+             "qg_decode_step: hidden=%d must be a positive multiple of 64", c->hidden);
+  QG_REQUIRE(c->layers >= 0, QG_ERR_UNSUPPORTED_SHAPE, "qg_decode_step: layers=%d", c->layers);
+  QG_REQUIRE(c->heads >= 1 && c->kv_heads >= 1 && c->heads % c->kv_heads == 0 &&
+                 c->heads / c->kv_heads <= 8,
+             QG_ERR_UNSUPPORTED_SHAPE,
+             "qg_decode_step: heads=%d kv_heads=%d (heads must be a multiple of kv_heads, ratio <= 8)",
+             c->heads, c->kv_heads);
+  QG_REQUIRE(c->head_dim >= 64 && c->head_dim <= 256 && c->head_dim % 64 == 0,
+             QG_ERR_UNSUPPORTED_SHAPE,
+             "qg_decode_step: head_dim=%d must be a multiple of 64 in [64, 256]", c->head_dim);
+  QG_REQUIRE(((long long)c->heads * c->head_dim) % 64 == 0, QG_ERR_UNSUPPORTED_SHAPE,
+             "qg_decode_step: heads*head_dim must be a multiple of 64");
+  QG_REQUIRE(c->ffn > 0 && c->ffn % 64 == 0, QG_ERR_UNSUPPORTED_SHAPE,
+             "qg_decode_step: ffn=%d must be a positive multiple of 64", c->ffn);
+  QG_REQUIRE(c->vocab >= 1, QG_ERR_UNSUPPORTED_SHAPE, "qg_decode_step: vocab=%d", c->vocab);
+  QG_REQUIRE(c->eps >= 0.f && c->theta > 0.0, QG_ERR_INVALID_ARGUMENT,
+             "qg_decode_step: eps must be >= 0 and theta > 0");
+  QG_REQUIRE(B >= 1 && B <= 32, QG_ERR_UNSUPPORTED_SHAPE, "qg_decode_step: B=%d must be in [1, 32]",
+             B);
+  QG_REQUIRE(cap >= 1, QG_ERR_UNSUPPORTED_SHAPE, "qg_decode_step: cap=%d must be >= 1", cap);
+  return QG_OK;
+}
+
+extern "C" size_t qg_decode_step_workspace_size(const qg_qwen3_config* cfg, int B, int cap) {
+  if (!cfg || B < 1 || cap < 1 || cfg->heads < 1 || cfg->kv_heads < 1) return 0;
+  return step_layout(*cfg, B, cap).total;
+}
+
+extern "C" qg_status qg_decode_step(const qg_qwen3_config* cfg, const qg_qwen3_weights* w,
+                                    uint16_t* k_cache, uint16_t* v_cache, int cap,
+                                    const int32_t* tokens, const int32_t* positions, float* logits,
+                                    int B, void* ws, size_t ws_bytes, void* stream) {
+  clear_error();
+  qg_status st = validate_cfg(cfg, B, cap);
+  if (st != QG_OK) return st;
+  const qg_qwen3_config& c = *cfg;
+  QG_REQUIRE(w, QG_ERR_INVALID_ARGUMENT, "qg_decode_step: weights is NULL");
+  QG_REQUIRE(c.layers == 0 || w->layers, QG_ERR_INVALID_ARGUMENT,
+             "qg_decode_step: weights->layers is NULL");
+  if ((st = validate_matrix(w->embed, "embed", -1)) != QG_OK) return st;
+  QG_REQUIRE(w->final_norm && aligned(w->final_norm, 2), QG_ERR_INVALID_ARGUMENT,
+             "qg_decode_step: final_norm is NULL or misaligned");
+  for (int l = 0; l < c.layers; ++l) {
+    const qg_qwen3_layer& L = w->layers[l];
+    const qg_affine8_matrix* ms[7] = {&L.q, &L.k, &L.v, &L.o, &L.gate, &L.up, &L.down};
+    const char* names[7] = {"q", "k", "v", "o", "gate", "up", "down"};
+    for (int i = 0; i < 7; ++i)
+      if ((st = validate_matrix(*ms[i], names[i], l)) != QG_OK) return st;
+    QG_REQUIRE(L.input_norm && L.post_norm && L.q_norm && L.k_norm, QG_ERR_INVALID_ARGUMENT,
+               "qg_decode_step: layer %d has a null norm weight", l);
+  }
+  QG_REQUIRE(c.layers == 0 || (k_cache && v_cache), QG_ERR_INVALID_ARGUMENT,
+             "qg_decode_step: null k_cache or v_cache");
+  QG_REQUIRE(aligned(k_cache, 16) && aligned(v_cache, 16), QG_ERR_MISALIGNED,
+             "qg_decode_step: k_cache/v_cache not 16-byte aligned");
+  QG_REQUIRE(tokens && positions && logits, QG_ERR_INVALID_ARGUMENT,
+             "qg_decode_step: null tokens, positions or logits");
+  QG_REQUIRE(aligned(tokens, 4) && aligned(positions, 4) && aligned(logits, 4), QG_ERR_MISALIGNED,
+             "qg_decode_step: tokens/positions/logits misaligned");
+  const StepLayout Ly = step_layout(c, B, cap);
+  QG_REQUIRE(ws && ws_bytes >= Ly.total, QG_ERR_WORKSPACE_TOO_SMALL,
+             "qg_decode_step: workspace of %zu bytes given, %zu needed", ws_bytes, Ly.total);
+  QG_REQUIRE(aligned(ws, 256), QG_ERR_MISALIGNED, "qg_decode_step: ws not 256-byte aligned");
+
+  cudaStream_t s = (cudaStream_t)stream;
+  uint8_t* base = reinterpret_cast<uint8_t*>(ws);
+  float* x = reinterpret_cast<float*>(base + Ly.x);
+  uint16_t* xn = reinterpret_cast<uint16_t*>(base + Ly.xn);
+  float* q = reinterpret_cast<float*>(base + Ly.q);
+  float* k = reinterpret_cast<float*>(base + Ly.k);
+  float* v = reinterpret_cast<float*>(base + Ly.v);
+  uint16_t* attn = reinterpret_cast<uint16_t*>(base + Ly.attn);
+  float* gate = reinterpret_cast<float*>(base + Ly.gate);
+  float* up = reinterpret_cast<float*>(base + Ly.up);
+  uint16_t* hm = reinterpret_cast<uint16_t*>(base + Ly.h);
+  void* aws = base + Ly.attn_ws;
+  const int H = c.heads, Hkv = c.kv_heads, D = c.head_dim;
+  const size_t cnt_off = attention_ws_counter_offset(B, H, Hkv, D, cap);
+  const size_t layer_cache = (size_t)B * Hkv * cap * D;
+  const float scale = 1.0f / sqrtf((float)D);
+
+  cudaMemsetAsync(reinterpret_cast<uint8_t*>(aws) + cnt_off, 0, (size_t)B * Hkv * 4, s);
+  launch_pdl(step_embed_kernel, dim3(B), dim3(256), 0, s, true, w->embed.w, w->embed.scales,
+             w->embed.biases, tokens, positions, x, c.vocab, c.hidden, cap);
+  for (int l = 0; l < c.layers; ++l) {
+    const qg_qwen3_layer& L = w->layers[l];
+    uint16_t* kc = k_cache + l * layer_cache;
+    uint16_t* vc = v_cache + l * layer_cache;
+    rmsnorm_launch(x, L.input_norm, c.eps, xn, true, B, c.hidden, s, true);
+    GemvSeg qkv[3] = {{L.q.w, L.q.scales, L.q.biases, q, nullptr, H * D, 0},
+                      {L.k.w, L.k.scales, L.k.biases, k, nullptr, Hkv * D, 0},
+                      {L.v.w, L.v.scales, L.v.biases, v, nullptr, Hkv * D, 0}};
+    gemv_affine8_launch(qkv, 3, xn, false, c.hidden, B, s, true);
+    launch_pdl(step_qk_rope_append_kernel, dim3(H + 2 * Hkv, B), dim3(32), 0, s, true, q,
+               (const float*)k, (const float*)v, L.q_norm, L.k_norm, positions, tokens, kc, vc, H,
+               Hkv, D, cap, c.vocab, c.eps, c.theta);
+    attention_launch(q, kc, vc, nullptr, positions, attn, true, B, H, Hkv, D, cap, scale, aws, s,
+                     true);
+    GemvSeg o = {L.o.w, L.o.scales, L.o.biases, x, x, c.hidden, 0};
+    gemv_affine8_launch(&o, 1, attn, false, H * D, B, s, true);
+    rmsnorm_launch(x, L.post_norm, c.eps, xn, true, B, c.hidden, s, true);
+    GemvSeg gu[2] = {{L.gate.w, L.gate.scales, L.gate.biases, gate, nullptr, c.ffn, 0},
+                     {L.up.w, L.up.scales, L.up.biases, up, nullptr, c.ffn, 0}};
+    gemv_affine8_launch(gu, 2, xn, false, c.hidden, B, s, true);
+    const int n = B * c.ffn;
+    launch_pdl(step_silu_mul_kernel, dim3((n + 255) / 256), dim3(256), 0, s, true,
+               (const float*)gate, (const float*)up, hm, n);
+    GemvSeg dn = {L.down.w, L.down.scales, L.down.biases, x, x, c.hidden, 0};
+    gemv_affine8_launch(&dn, 1, hm, false, c.ffn, B, s, true);
+  }
+  rmsnorm_launch(x, w->final_norm, c.eps, xn, true, B, c.hidden, s, true);
+  GemvSeg head = {w->embed.w, w->embed.scales, w->embed.biases, logits, nullptr, c.vocab, 0};
+  gemv_affine8_launch(&head, 1, xn, false, c.hidden, B, s, true);
+  return check_launch("qg_decode_step");
+}

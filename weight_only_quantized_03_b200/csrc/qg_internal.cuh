@@ -1,0 +1,160 @@
+// Internal helpers shared by the libqg translation units (GPU side only).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+#include <stdio.h>
+#include <string>
+
+#include "qg.h"
+
+namespace qg {
+
+// ---------------------------------------------------------------- errors --
+
+void set_error(const char* fmt, ...);
+void clear_error();
+
+#define QG_REQUIRE(cond, code, ...)  \
+  do {                               \
+    if (!(cond)) {                   \
+      ::qg::set_error(__VA_ARGS__);  \
+      return (code);                 \
+    }                                \
+  } while (0)
+
+inline bool aligned(const void* p, size_t a) {
+  return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
+}
+
+qg_status check_launch(const char* what);
+
+// ---------------------------------------------------------------- launch --
+
+// Launch with Programmatic Dependent Launch allowed: the kernel may start
+// while its predecessor on the stream drains, and must call
+// pdl_wait() before touching anything the predecessor writes.
+void count_launch();
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block,
+                              size_t smem, cudaStream_t stream, bool pdl,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  count_launch();
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// griddepcontrol: wait for the predecessor grid's memory to be visible /
+// allow the successor grid to begin launching.
+__device__ __forceinline__ void pdl_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ----------------------------------------------------------------- loads --
+
+// L2 policy for data read exactly once (packed weights): evict first.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// 16-byte streaming load: not kept in L1, evict-first in L2.
+__device__ __forceinline__ uint4 ld_stream_u4(const void* ptr, uint64_t pol) {
+  uint4 v;
+  asm volatile(
+      "ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+      : "l"(ptr), "l"(pol));
+  return v;
+}
+
+__device__ __forceinline__ uint4 ld_nc_u4(const void* p) {
+  return __ldg(reinterpret_cast<const uint4*>(p));
+}
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t bits16) {
+  return __uint_as_float(bits16 << 16);
+}
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+}
+
+// Byte i of a 32-bit word as an exact float: the byte is placed in the low
+// mantissa bits of 2^23 and 2^23 is subtracted.
+template <int I>
+__device__ __forceinline__ float byte_to_f32(uint32_t w) {
+  const uint32_t magic = __byte_perm(w, 0x4B000000u, 0x7440u | I);
+  return __uint_as_float(magic) - 8388608.0f;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+inline int num_sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+}  // namespace qg
+
+// Internal launchers shared between translation units (the decode step
+// composes the single-op kernels). All arguments have been validated.
+namespace qg {
+
+struct GemvSeg {           // one affine8 matrix of a multi-matrix GEMV launch
+  const uint32_t* w;
+  const uint16_t* s;
+  const uint16_t* b;
+  void* y;                 // [B][N] of y_bf16 ? bf16 : fp32
+  const float* res;        // nullable fp32 [B][N]
+  int N;
+  int y_bf16;
+};
+
+cudaError_t gemv_affine8_launch(const GemvSeg* segs, int nseg, const void* x,
+                                bool x_f32, int K, int B, cudaStream_t st,
+                                bool pdl);
+
+cudaError_t rmsnorm_launch(const float* x, const uint16_t* w, float eps, void* y,
+                           bool y_bf16, int rows, int dim, cudaStream_t st, bool pdl);
+
+cudaError_t attention_launch(const float* q, const uint16_t* kc, const uint16_t* vc,
+                             const int32_t* kv_len, const int32_t* pos_for_len,
+                             void* out, bool out_bf16, int B, int H, int Hkv, int D,
+                             int cap, float scale, void* ws, cudaStream_t st, bool pdl);
+
+size_t attention_ws_bytes(int B, int H, int Hkv, int D, int cap);
+
+}  // namespace qg
