@@ -260,9 +260,13 @@ size_t qg_decode_step_workspace_size(const qg_qwen3_config* cfg, int B, int cap)
  *             gets NaN logits and its cache is not written.
  * logits      device fp32 [B][vocab].
  * ws          device workspace >= qg_decode_step_workspace_size(cfg,B,cap)
- *             bytes, 256-byte aligned; contents need not be initialised.
- *             On return its first B*hidden*4 bytes hold the residual stream
- *             after the last layer (fp32 [B][hidden], before the final norm).
+ *             bytes, 256-byte aligned, ZERO-FILLED before its first use (and
+ *             again if it was used for anything else in between): it carries
+ *             a step counter from one call to the next, which tags the data
+ *             the persistent kernel's CTAs exchange. Use one workspace per
+ *             stream at a time. On return its first B*hidden*4 bytes hold the
+ *             residual stream after the last layer (fp32 [B][hidden], before
+ *             the final norm).
  * Precision: residual stream, q/k/v and gate/up outputs and logits fp32;
  * norm outputs feeding a GEMV, cached K/V, attention output and SiLU-mul
  * output bf16.
@@ -274,6 +278,39 @@ qg_status qg_decode_step(const qg_qwen3_config* cfg, const qg_qwen3_weights* w,
                          const int32_t* tokens, const int32_t* positions,
                          float* logits, int B, void* ws, size_t ws_bytes,
                          void* stream);
+
+/* qg_decode_step with option flags. QG_STEP_MULTI_KERNEL forces the
+ * kernel-per-op path (one launch per norm / GEMV / attention / elementwise
+ * stage, chained with Programmatic Dependent Launch) instead of the
+ * persistent one-launch kernel. Without the flag the persistent kernel runs
+ * whenever the shapes allow it (B <= 4; hidden, heads*head_dim and ffn
+ * multiples of 512 and <= 16384; head_dim 64 or 128; layers <= 64; 16-byte
+ * aligned scales and biases) and the kernel-per-op path otherwise. Both
+ * paths compute the same operations with the same precision points. */
+#define QG_STEP_MULTI_KERNEL 1u
+/* Test hook for the persistent kernel: one device-side wait targets a
+ * counter that nothing sets, so it gives up after its 1 s bound and the
+ * step records an error word (read it with qg_decode_step_error). The
+ * step's outputs are then undefined; the context stays usable. */
+#define QG_STEP_TEST_STALL 0x80000000u
+/* Profiling aid for the persistent kernel: thread 0 of every CTA writes
+ * %globaltimer stamps (ns, uint64) at each phase boundary into the
+ * workspace region that qg_decode_step_trace_offset() locates, laid out
+ * [CTA][layer (last slot: LM head)][16 events]. */
+#define QG_STEP_TRACE 0x40000000u
+size_t qg_decode_step_trace_offset(const qg_qwen3_config* cfg, int B, int cap);
+qg_status qg_decode_step_ex(const qg_qwen3_config* cfg, const qg_qwen3_weights* w,
+                            uint16_t* k_cache, uint16_t* v_cache, int cap,
+                            const int32_t* tokens, const int32_t* positions,
+                            float* logits, int B, void* ws, size_t ws_bytes,
+                            unsigned flags, void* stream);
+
+/* Reads the device error word of the last step that used `ws` (this call
+ * synchronises `stream`). The persistent kernel bounds every device-side
+ * wait; a wait that gives up records a nonzero code, the kernel leaves, and
+ * this call then returns QG_ERR_TIMEOUT with the code in *code. */
+qg_status qg_decode_step_error(const qg_qwen3_config* cfg, int B, int cap,
+                               const void* ws, unsigned* code, void* stream);
 
 /* ------------------------------------------------------------------------
  * Test exports: the unpack and dequant the kernels use, written out.

@@ -3,7 +3,9 @@ device results with the oracle under the library's tolerance.
 
 Tolerance (fp32-accumulated outputs): |gpu - ref| <= 2e-3 + 1e-3 |ref|.
 For outputs stored as bf16 the bf16 store adds at most half a bf16 ulp of the
-value, bounded here by 2^-8 |ref|.
+value, bounded here by 2^-8 |ref| (``bf16_out=True``). When both sides store
+bf16 (the oracle rounds too, e.g. K/V cache rows), values a hair apart can
+round to neighbouring bf16 numbers: one full ulp, 2^-7 |ref| (``ulps=1``).
 """
 import numpy as np
 import torch
@@ -31,13 +33,13 @@ def host64(t):
     return t.detach().float().cpu().numpy().astype(np.float64)
 
 
-def assert_parity(gpu, ref, bf16_out=False, what=""):
+def assert_parity(gpu, ref, bf16_out=False, what="", ulps=0.5):
     gpu = np.asarray(gpu, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     assert gpu.shape == ref.shape, (what, gpu.shape, ref.shape)
     tol = ATOL + RTOL * np.abs(ref)
     if bf16_out:
-        tol = tol + BF16_HALF_ULP_REL * np.abs(ref)
+        tol = tol + 2 * ulps * BF16_HALF_ULP_REL * np.abs(ref)
     err = np.abs(gpu - ref)
     bad = ~(err <= tol)
     if bad.any():

@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(_HERE, "libqg.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m weight_only_quantized_03_b200.build`"
+        f"{LIB_PATH} is missing: build it with `python weight_only_quantized_03_b200/build.py`"
     )
 lib = ctypes.CDLL(LIB_PATH)
 
@@ -31,6 +31,9 @@ QG_ERR_CUDA = 5
 QG_ERR_TIMEOUT = 6
 QG_F32 = 0
 QG_BF16 = 1
+QG_STEP_MULTI_KERNEL = 1
+QG_STEP_TEST_STALL = 0x80000000
+QG_STEP_TRACE = 0x40000000
 
 _vp = ctypes.c_void_p
 _i = ctypes.c_int
@@ -84,6 +87,11 @@ _SIGS = {
     "qg_decode_step_workspace_size": (_sz, [ctypes.POINTER(qg_qwen3_config), _i, _i]),
     "qg_decode_step": (_i, [ctypes.POINTER(qg_qwen3_config), ctypes.POINTER(qg_qwen3_weights),
                             _vp, _vp, _i, _vp, _vp, _vp, _i, _vp, _sz, _vp]),
+    "qg_decode_step_ex": (_i, [ctypes.POINTER(qg_qwen3_config), ctypes.POINTER(qg_qwen3_weights),
+                               _vp, _vp, _i, _vp, _vp, _vp, _i, _vp, _sz, ctypes.c_uint, _vp]),
+    "qg_decode_step_error": (_i, [ctypes.POINTER(qg_qwen3_config), _i, _i, _vp,
+                                  ctypes.POINTER(ctypes.c_uint), _vp]),
+    "qg_decode_step_trace_offset": (_sz, [ctypes.POINTER(qg_qwen3_config), _i, _i]),
     "qg_unpack_affine8": (_i, [_vp, _vp, _i, _i, _vp]),
     "qg_dequant_affine8_g64": (_i, [_vp, _vp, _vp, _vp, _i, _i, _vp]),
     "qg_dequant_q4_0": (_i, [_vp, _vp, _i, _i, _vp]),
@@ -254,13 +262,14 @@ class Qwen3Model:
 
     def new_state(self, B, cap):
         """Zeroed KV caches [layers, B, kv_heads, cap, head_dim] bf16, a
-        workspace and a logits buffer for batch B."""
+        zero-filled workspace (required before its first use) and a logits
+        buffer for batch B."""
         c = self.cfg
         shape = (c["layers"], B, c["kv_heads"], cap, c["head_dim"])
         return dict(
             k_cache=torch.zeros(shape, dtype=torch.bfloat16, device=self.device),
             v_cache=torch.zeros(shape, dtype=torch.bfloat16, device=self.device),
-            ws=torch.empty(self.workspace_size(B, cap), dtype=torch.uint8, device=self.device),
+            ws=torch.zeros(self.workspace_size(B, cap), dtype=torch.uint8, device=self.device),
             logits=torch.empty((B, c["vocab"]), dtype=torch.float32, device=self.device),
             B=B, cap=cap)
 
@@ -270,14 +279,21 @@ class Qwen3Model:
         n = state["B"] * self.cfg["hidden"]
         return state["ws"][: 4 * n].view(torch.float32).view(state["B"], self.cfg["hidden"])
 
-    def qg_decode_step(self, state, tokens, positions, stream=None, layers=None):
+    def qg_decode_step_error(self, state, stream=None):
+        """Device error word of the latest step (synchronises the stream)."""
+        code = ctypes.c_uint(0)
+        st = lib.qg_decode_step_error(ctypes.byref(self.c_cfg), state["B"], state["cap"],
+                                      _p(state["ws"]), ctypes.byref(code), _stream(stream))
+        return st, code.value
+
+    def qg_decode_step(self, state, tokens, positions, stream=None, layers=None, flags=0):
         """tokens, positions: device int32 [B]. Writes state['logits'].
         ``layers`` runs only the first that many layers (then the head)."""
         cfg = self.c_cfg
         if layers is not None:
             cfg = qg_qwen3_config.from_buffer_copy(self.c_cfg)
             cfg.layers = layers
-        _call("qg_decode_step", ctypes.byref(cfg), ctypes.byref(self.c_weights),
+        _call("qg_decode_step_ex", ctypes.byref(cfg), ctypes.byref(self.c_weights),
               _p(state["k_cache"]), _p(state["v_cache"]), state["cap"], _p(tokens),
               _p(positions), _p(state["logits"]), state["B"], _p(state["ws"]),
-              state["ws"].numel(), _stream(stream))
+              state["ws"].numel(), flags, _stream(stream))

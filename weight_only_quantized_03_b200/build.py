@@ -1,6 +1,6 @@
 """Build libqg.so (sm_100a) in-tree with nvcc.
 
-Usage: python -m weight_only_quantized_03_b200.build [--force] [-v]
+Usage: python weight_only_quantized_03_b200/build.py [--force] [-v] [--ptxas-v]
 Objects go to _build/ at the repository root; the shared library lands next
 to this file so that it travels with the source tree.
 """

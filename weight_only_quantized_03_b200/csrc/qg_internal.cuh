@@ -157,4 +157,12 @@ cudaError_t attention_launch(const float* q, const uint16_t* kc, const uint16_t*
 
 size_t attention_ws_bytes(int B, int H, int Hkv, int D, int cap);
 
+// persistent decode-step kernel (decode_mega.cu)
+bool mega_eligible(const qg_qwen3_config& c, int B, int cap);
+size_t mega_ws_bytes(const qg_qwen3_config& c, int B, int cap);
+cudaError_t mega_launch(const qg_qwen3_config& c, const qg_qwen3_weights& w, uint16_t* kc,
+                        uint16_t* vc, int cap, const int32_t* tokens, const int32_t* positions,
+                        float* logits, int B, float* x, void* xws, unsigned* cnt, unsigned* step,
+                        bool test_stall, unsigned long long* trace, cudaStream_t st);
+
 }  // namespace qg
