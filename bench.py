@@ -312,7 +312,7 @@ def run_ours(args):
     lm_bytes = affine8_bytes(V, h, B)
     lm_gbs = lm_bytes / (lm_ms / 1000.0) / 1e9
     traffic = traffic_from_profile(os.path.join(ROOT, "weight_only_quantized_03_b200", "csrc",
-                                                "gemv_affine8.cu")) if B == 1 else None
+                                                "gemv_affine8_tc.cu")) if B == 1 else None
 
     # ---- e2e through the public API with host buffers
     h_tok = torch.from_numpy(toks_np).pin_memory()

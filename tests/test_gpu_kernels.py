@@ -80,6 +80,18 @@ GEMV_CASES = [
     (300, 6144, 5, "bf16", "f32", False, False),
     (9473, 256, 1, "bf16", "f32", False, False),
     (40000, 128, 2, "bf16", "f32", False, False),
+    # the tensor-core streaming path (bf16 x, K % 512 == 0, B <= 8): ragged
+    # rows, one or two batch tiles, column splits over 2, 4 and 8 warps
+    # (uneven when K / 512 is not a multiple), residual, bf16 output
+    (1001, 512, 8, "bf16", "bf16", True, True),
+    (1001, 512, 32, "bf16", "bf16", True, True),
+    (2050, 2048, 8, "bf16", "f32", True, False),
+    (17, 1024, 3, "bf16", "f32", False, True),
+    (5000, 3072, 5, "bf16", "f32", False, False),
+    (64, 3072, 1, "bf16", "f32", True, False),
+    (3, 1536, 6, "bf16", "bf16", False, False),
+    (16, 4096, 1, "bf16", "bf16", False, False),
+    (200, 8192, 2, "bf16", "f32", False, False),
 ]
 
 
@@ -104,6 +116,19 @@ def test_gemv_affine8(N, K, B, xd, yd, res, quant):
     qg.qg_gemv_affine8_g64(dev(w), dev(s), dev(b), x_d, y, residual=rr)
     ref = O.gemv_affine8(w, s, b, x64, residual=r)
     assert_parity(host64(y), ref, bf16_out=(yd == "bf16"), what=f"gemv {N}x{K} B={B}")
+
+
+def test_gemv_affine8_large_activations_prescaled():
+    # |x| far beyond fp16's range: the tensor-core path prescales x by a
+    # power of two, so the products stay exact and nothing overflows
+    N, K = 300, 1024
+    w, s, b = qg_synth.affine8_packed(N, K, 77)
+    xf = (qg_synth.gaussian((2, K), 1.0, 78) * 2.0 ** 20).astype(np.float32)
+    xbits = qg_synth.f32_to_bf16_bits(xf)
+    y = torch.empty((2, N), dtype=torch.float32, device="cuda")
+    qg.qg_gemv_affine8_g64(dev(w), dev(s), dev(b), bf16_dev(xbits), y)
+    ref = O.gemv_affine8(w, s, b, O.bf16_bits_to_f64(xbits))
+    assert_parity(host64(y), ref, what="prescaled x")
 
 
 def test_gemv_affine8_lm_head_full_size_sampled_rows():

@@ -296,11 +296,17 @@ extern "C" qg_status qg_decode_step_ex(const qg_qwen3_config* cfg, const qg_qwen
     const qg_qwen3_layer& L = w->layers[l];
     uint16_t* kc = k_cache + l * layer_cache;
     uint16_t* vc = v_cache + l * layer_cache;
-    rmsnorm_launch(x, L.input_norm, c.eps, xn, true, B, c.hidden, s, true);
     GemvSeg qkv[3] = {{L.q.w, L.q.scales, L.q.biases, q, nullptr, H * D, 0},
                       {L.k.w, L.k.scales, L.k.biases, k, nullptr, Hkv * D, 0},
                       {L.v.w, L.v.scales, L.v.biases, v, nullptr, Hkv * D, 0}};
-    gemv_affine8_launch(qkv, 3, xn, false, c.hidden, B, s, true);
+    // RMSNorm and SiLU-mul run in the next GEMV's prologue where the
+    // tensor-core GEMV takes the shape, as separate kernels otherwise
+    if (gemv_tc_eligible(qkv, 3, c.hidden, B, false)) {
+      gemv_tc_launch_rmsnorm(qkv, 3, x, L.input_norm, c.eps, c.hidden, B, s, true);
+    } else {
+      rmsnorm_launch(x, L.input_norm, c.eps, xn, true, B, c.hidden, s, true);
+      gemv_affine8_launch(qkv, 3, xn, false, c.hidden, B, s, true);
+    }
     launch_pdl(step_qk_rope_append_kernel, dim3(H + 2 * Hkv, B), dim3(32), 0, s, true, q,
                (const float*)k, (const float*)v, L.q_norm, L.k_norm, positions, tokens, kc, vc, H,
                Hkv, D, cap, c.vocab, c.eps, c.theta);
@@ -308,19 +314,31 @@ extern "C" qg_status qg_decode_step_ex(const qg_qwen3_config* cfg, const qg_qwen
                      true);
     GemvSeg o = {L.o.w, L.o.scales, L.o.biases, x, x, c.hidden, 0};
     gemv_affine8_launch(&o, 1, attn, false, H * D, B, s, true);
-    rmsnorm_launch(x, L.post_norm, c.eps, xn, true, B, c.hidden, s, true);
     GemvSeg gu[2] = {{L.gate.w, L.gate.scales, L.gate.biases, gate, nullptr, c.ffn, 0},
                      {L.up.w, L.up.scales, L.up.biases, up, nullptr, c.ffn, 0}};
-    gemv_affine8_launch(gu, 2, xn, false, c.hidden, B, s, true);
-    const int n = B * c.ffn;
-    launch_pdl(step_silu_mul_kernel, dim3((n + 255) / 256), dim3(256), 0, s, true,
-               (const float*)gate, (const float*)up, hm, n);
+    if (gemv_tc_eligible(gu, 2, c.hidden, B, false)) {
+      gemv_tc_launch_rmsnorm(gu, 2, x, L.post_norm, c.eps, c.hidden, B, s, true);
+    } else {
+      rmsnorm_launch(x, L.post_norm, c.eps, xn, true, B, c.hidden, s, true);
+      gemv_affine8_launch(gu, 2, xn, false, c.hidden, B, s, true);
+    }
     GemvSeg dn = {L.down.w, L.down.scales, L.down.biases, x, x, c.hidden, 0};
-    gemv_affine8_launch(&dn, 1, hm, false, c.ffn, B, s, true);
+    if (gemv_tc_eligible(&dn, 1, c.ffn, B, false)) {
+      gemv_tc_launch_silu_mul(&dn, 1, gate, up, c.ffn, B, s, true);
+    } else {
+      const int n = B * c.ffn;
+      launch_pdl(step_silu_mul_kernel, dim3((n + 255) / 256), dim3(256), 0, s, true,
+                 (const float*)gate, (const float*)up, hm, n);
+      gemv_affine8_launch(&dn, 1, hm, false, c.ffn, B, s, true);
+    }
   }
-  rmsnorm_launch(x, w->final_norm, c.eps, xn, true, B, c.hidden, s, true);
   GemvSeg head = {w->embed.w, w->embed.scales, w->embed.biases, logits, nullptr, c.vocab, 0};
-  gemv_affine8_launch(&head, 1, xn, false, c.hidden, B, s, true);
+  if (gemv_tc_eligible(&head, 1, c.hidden, B, false)) {
+    gemv_tc_launch_rmsnorm(&head, 1, x, w->final_norm, c.eps, c.hidden, B, s, true);
+  } else {
+    rmsnorm_launch(x, w->final_norm, c.eps, xn, true, B, c.hidden, s, true);
+    gemv_affine8_launch(&head, 1, xn, false, c.hidden, B, s, true);
+  }
   return check_launch("qg_decode_step");
 }
 

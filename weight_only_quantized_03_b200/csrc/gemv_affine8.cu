@@ -214,6 +214,7 @@ static cudaError_t launch_nb(GemvParams& P, bool xf32, cudaStream_t st, bool pdl
 
 cudaError_t gemv_affine8_launch(const GemvSeg* segs, int nseg, const void* x, bool x_f32,
                                 int K, int B, cudaStream_t st, bool pdl) {
+  if (gemv_tc_eligible(segs, nseg, K, B, x_f32)) return gemv_tc_launch(segs, nseg, x, K, B, st, pdl);
   const size_t esz = x_f32 ? 4 : 2;
   for (int b0 = 0; b0 < B; b0 += 8) {
     const int nb = B - b0 < 8 ? B - b0 : 8;

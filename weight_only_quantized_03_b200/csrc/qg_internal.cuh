@@ -147,6 +147,19 @@ cudaError_t gemv_affine8_launch(const GemvSeg* segs, int nseg, const void* x,
                                 bool x_f32, int K, int B, cudaStream_t st,
                                 bool pdl);
 
+// tensor-core streaming path of the affine8 GEMV (gemv_affine8_tc.cu)
+bool gemv_tc_eligible(const GemvSeg* segs, int nseg, int K, int B, bool x_f32);
+cudaError_t gemv_tc_launch(const GemvSeg* segs, int nseg, const void* x, int K, int B,
+                           cudaStream_t st, bool pdl);
+// The same GEMV with its input formed in the prologue: bf16(RMSNorm(x) * w)
+// of fp32 x [B][K], or bf16(silu(gate) * up) of fp32 [B][K] (eligibility as
+// gemv_tc_eligible with x_f32 = false).
+cudaError_t gemv_tc_launch_rmsnorm(const GemvSeg* segs, int nseg, const float* x,
+                                   const uint16_t* norm_w, float eps, int K, int B,
+                                   cudaStream_t st, bool pdl);
+cudaError_t gemv_tc_launch_silu_mul(const GemvSeg* segs, int nseg, const float* gate,
+                                    const float* up, int K, int B, cudaStream_t st, bool pdl);
+
 cudaError_t rmsnorm_launch(const float* x, const uint16_t* w, float eps, void* y,
                            bool y_bf16, int rows, int dim, cudaStream_t st, bool pdl);
 
