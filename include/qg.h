@@ -120,13 +120,20 @@ qg_status qg_gemv_q4_0(const uint8_t* blocks, const float* x, const float* bias,
  * blocks  device, Q4_0 [N][(K/32)*18] as in qg_gemv_q4_0.
  * A       device fp32 [M][K].  bias device fp32 [N] or NULL.  C device fp32 [M][N].
  * ws      device workspace of at least qg_gemm_q4_0_workspace_size(M,N,K)
- *         bytes (contents need not be initialised).
+ *         bytes, 256-byte aligned (contents need not be initialised): A as
+ *         bf16, then the error word.
+ * A and C must be 16-byte aligned, blocks 2-byte aligned.
  * Shape rules: K % 64 == 0, N % 128 == 0, M >= 0.
  * ---------------------------------------------------------------------- */
 size_t qg_gemm_q4_0_workspace_size(int M, int N, int K);
 qg_status qg_gemm_q4_0(const uint8_t* blocks, const float* A, const float* bias,
                        float* C, int M, int N, int K, void* ws, size_t ws_bytes,
                        void* stream);
+/* Reads the device error word of the last qg_gemm_q4_0 call that used `ws`
+ * (synchronises `stream`). Every device-side wait in the GEMM is bounded
+ * (1 s); one that gives up leaves C undefined, records a nonzero code, and
+ * this call then returns QG_ERR_TIMEOUT with the code in *code. */
+qg_status qg_gemm_q4_0_error(int M, int K, const void* ws, unsigned* code, void* stream);
 
 /* ------------------------------------------------------------------------
  * RMSNorm  [TS: encode_rms_norm_bf16w in `step`; MK: rms_norm layers]

@@ -166,6 +166,35 @@ def test_gemv_q4_0(N, K, B, bias, quant):
     assert_parity(host64(y), ref, what=f"q4_0 gemv {N}x{K} B={B}")
 
 
+# ---------------------------------------------------- Q4_0 GEMM (tcgen05) -
+
+GEMM_CASES = [
+    # M, N, K, bias, quantized weights
+    (1, 128, 64, False, True),
+    (130, 256, 128, True, True),       # ragged M, one 256-column tile
+    (200, 384, 192, True, False),      # 128-column tiles, three K stages
+    (257, 512, 1280, False, False),    # K ring wraps (20 stages over 4)
+    # the Whisper-large-v3 encoder projections at M = 1500 frames
+    (1500, 1280, 1280, True, False),
+    (1500, 5120, 1280, True, False),
+    (1500, 1280, 5120, True, False),
+]
+
+
+@pytest.mark.parametrize("M,N,K,bias,quant", GEMM_CASES)
+def test_gemm_q4_0(M, N, K, bias, quant):
+    blocks = (O.q4_0_quantize(qg_synth.gaussian((N, K), 0.02, 21)) if quant
+              else qg_synth.q4_0_packed(N, K, 22))
+    A = qg_synth.gaussian((M, K), 1.0, 23)
+    bv = qg_synth.gaussian((N,), 1.0, 24) if bias else None
+    C = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    ws = torch.empty(qg.qg_gemm_q4_0_workspace_size(M, N, K), dtype=torch.uint8, device="cuda")
+    qg.qg_gemm_q4_0(dev(blocks), dev(A), C, bias=dev(bv) if bias else None, ws=ws)
+    assert qg.qg_gemm_q4_0_error(M, K, ws) == (0, 0)
+    ref = O.gemm_q4_0_bf16(blocks, A, None if bv is None else bv.astype(np.float64))
+    assert_parity(host64(C), ref, what=f"q4_0 gemm {M}x{N}x{K}")
+
+
 # -------------------------------------------------------- elementwise ------
 
 @pytest.mark.parametrize("rows,dim,eps,yd", [(1, 1024, 1e-6, "bf16"), (10, 1024, 1e-6, "f32"),

@@ -75,6 +75,7 @@ _SIGS = {
     "qg_gemv_q4_0": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _vp]),
     "qg_gemm_q4_0_workspace_size": (_sz, [_i, _i, _i]),
     "qg_gemm_q4_0": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _vp, _sz, _vp]),
+    "qg_gemm_q4_0_error": (_i, [_i, _i, _vp, ctypes.POINTER(ctypes.c_uint), _vp]),
     "qg_rmsnorm": (_i, [_vp, _vp, _f, _vp, _i, _i, _i, _vp]),
     "qg_rmsnorm_perhead": (_i, [_vp, _i, _vp, _f, _vp, _i, _i, _i, _i, _vp]),
     "qg_rope_neox": (_i, [_vp, _i, _vp, _d, _i, _i, _i, _i, _vp]),
@@ -160,6 +161,13 @@ def qg_gemm_q4_0(blocks, A, C, bias=None, ws=None, stream=None):
     nbytes = 0 if ws is None else ws.numel() * ws.element_size()
     _call("qg_gemm_q4_0", _p(blocks), _p(A), _p(bias), _p(C), M, N, K, _p(ws), nbytes,
           _stream(stream))
+
+
+def qg_gemm_q4_0_error(M, K, ws, stream=None):
+    """(status, code) of the device error word of the last GEMM on ``ws``."""
+    code = ctypes.c_uint(0)
+    st = lib.qg_gemm_q4_0_error(M, K, _p(ws), ctypes.byref(code), _stream(stream))
+    return st, code.value
 
 
 def qg_rmsnorm(x, w, eps, y, stream=None):

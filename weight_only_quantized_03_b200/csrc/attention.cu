@@ -50,6 +50,75 @@ size_t attention_ws_bytes(int B, int H, int Hkv, int D, int cap) {
   return align256(o) + align256(ml) + align256(cnt);
 }
 
+// Decode-step fusion: the per-head RMSNorm and NeoX RoPE of q and k and the
+// K/V append at the current position (turbospark-runtime 0.3.0,
+// src/qwen3_asr_metal.rs, `step`: encode_rms_norm_bf16w_perhead,
+// encode_rope_neox_subdim, the cache writes; makima src/tts/qwen3/model.rs,
+// apply_head_norm and RotaryEmbedding) run inside the attention kernel.
+struct AttnFuse {
+  int on;
+  const float* k;        // raw k [B][Hkv][D] fp32
+  const float* v;        // raw v [B][Hkv][D] fp32
+  const uint16_t* qn;    // q_norm weight bf16 [D]
+  const uint16_t* kn;    // k_norm weight bf16 [D]
+  const int32_t* tok;    // [B]: a bad token writes nothing to the cache
+  int vocab;
+  float eps;
+  double theta;
+};
+
+// RMSNorm of one head row src[0..D) with weight w, then NeoX rotation at
+// position p; lane owns the pairs (i, i + D/2) for i = lane + 32 j.
+// Writes the rotated fp32 values through `put(i, value)`.
+template <typename Put>
+__device__ __forceinline__ void norm_rope_head(const float* src, const uint16_t* w, int D, float eps,
+                                               double theta, int p, int lane, Put put) {
+  const int half = D >> 1;
+  float x1[4], x2[4];
+  float ss = 0.f;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int i = lane + 32 * j;
+    x1[j] = i < half ? src[i] : 0.f;
+    x2[j] = i < half ? src[i + half] : 0.f;
+    ss = fmaf(x1[j], x1[j], fmaf(x2[j], x2[j], ss));
+  }
+  ss = warp_sum(ss);
+  const float inv = 1.0f / sqrtf(ss / (float)D + eps);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int i = lane + 32 * j;
+    if (i >= half) break;
+    const float a = x1[j] * inv * bf16_bits_to_f32(w[i]);
+    const float c2 = x2[j] * inv * bf16_bits_to_f32(w[i + half]);
+    const double inv_freq = pow(theta, -2.0 * (double)i / (double)D);
+    double sd, cd;
+    sincos((double)p * inv_freq, &sd, &cd);
+    const float cs = (float)cd, sn = (float)sd;
+    put(i, a * cs - c2 * sn);
+    put(i + half, c2 * cs + a * sn);
+  }
+}
+
+// VPL consecutive bf16 values (one lane's share of a head row) as fp32, in
+// 32-bit words when VPL is even (the row offset lane * VPL is then 4-byte
+// aligned). Plain (coherent) loads: in the decode step the kernel itself
+// writes the row at the current position before reading it.
+template <int VPL>
+__device__ __forceinline__ void load_bf16_row(const uint16_t* p, float (&out)[VPL]) {
+  if constexpr (VPL % 2 == 0) {
+#pragma unroll
+    for (int i = 0; i < VPL / 2; ++i) {
+      const uint32_t w = reinterpret_cast<const unsigned int*>(p)[i];
+      out[2 * i] = bf16_lo(w);
+      out[2 * i + 1] = bf16_hi(w);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) out[i] = bf16_bits_to_f32(p[i]);
+  }
+}
+
 template <int VPL>  // values of a head row per lane: D = 32 * VPL
 __global__ void __launch_bounds__(kAttnWarps * 32)
 attention_split_kernel(const float* __restrict__ q, const uint16_t* __restrict__ kc,
@@ -57,7 +126,7 @@ attention_split_kernel(const float* __restrict__ q, const uint16_t* __restrict__
                        const int32_t* __restrict__ pos_for_len, void* __restrict__ out,
                        int out_bf16, int H, int Hkv, int cap, float scale, int ch, int nsplit,
                        float* __restrict__ ws_o, float* __restrict__ ws_ml,
-                       unsigned int* __restrict__ ws_cnt) {
+                       unsigned int* __restrict__ ws_cnt, const AttnFuse fz) {
   constexpr int D = 32 * VPL;
   const int s = blockIdx.x, kv = blockIdx.y, b = blockIdx.z;
   const int g = H / Hkv;
@@ -74,8 +143,35 @@ attention_split_kernel(const float* __restrict__ q, const uint16_t* __restrict__
   const int t0 = s * ch;
   const int t1 = valid ? min(L, t0 + ch) : 0;
 
-  for (int i = threadIdx.x; i < g * D; i += blockDim.x)
-    sq[i / D][i % D] = q[((size_t)b * H + kv * g + i / D) * D + i % D] * scale;
+  if (!fz.on) {
+    for (int i = threadIdx.x; i < g * D; i += blockDim.x)
+      sq[i / D][i % D] = q[((size_t)b * H + kv * g + i / D) * D + i % D] * scale;
+  } else {
+    // q heads: norm + rope into shared memory (every split recomputes its
+    // own); the split holding row p also norms + ropes k and appends k, v
+    const int p = pos_for_len[b], tk = fz.tok[b];
+    const bool pos_ok = p >= 0 && p < cap && tk >= 0 && tk < fz.vocab;
+    const int pr = pos_ok ? p : 0;
+    const bool owner = pos_ok && p >= t0 && p < t0 + ch;
+    const size_t row = (((size_t)b * Hkv + kv) * cap + pr) * D;
+    for (int hh = warp; hh < g + 2; hh += kAttnWarps) {
+      if (hh < g) {
+        float* dst = sq[hh];
+        norm_rope_head(q + ((size_t)b * H + kv * g + hh) * D, fz.qn, D, fz.eps, fz.theta, pr, lane,
+                       [&](int i, float r) { dst[i] = r * scale; });
+      } else if (hh == g) {
+        if (owner) {
+          uint16_t* kdst = const_cast<uint16_t*>(kc) + row;
+          norm_rope_head(fz.k + ((size_t)b * Hkv + kv) * D, fz.kn, D, fz.eps, fz.theta, pr, lane,
+                         [&](int i, float r) { kdst[i] = f32_to_bf16_bits(r); });
+        }
+      } else if (owner) {
+        uint16_t* vdst = const_cast<uint16_t*>(vc) + row;
+        const float* vs = fz.v + ((size_t)b * Hkv + kv) * D;
+        for (int d = lane; d < D; d += 32) vdst[d] = f32_to_bf16_bits(vs[d]);
+      }
+    }
+  }
   __syncthreads();
 
   float m[kMaxGroup], l[kMaxGroup], o[kMaxGroup][VPL], qr[kMaxGroup][VPL];
@@ -91,29 +187,37 @@ attention_split_kernel(const float* __restrict__ q, const uint16_t* __restrict__
   }
 
   const size_t head_base = ((size_t)b * Hkv + kv) * cap;
-  for (int t = t0 + warp; t < t1; t += kAttnWarps) {
-    const uint16_t* kr = kc + (head_base + t) * D + lane * VPL;
-    const uint16_t* vr = vc + (head_base + t) * D + lane * VPL;
-    float kf[VPL], vf[VPL];
+  // RB rows per warp in flight: all their K/V loads are issued before the
+  // first score, so the rows' memory latencies overlap
+  constexpr int RB = VPL <= 4 ? 8 : 4;
+  for (int tb = t0 + warp; tb < t1; tb += kAttnWarps * RB) {
+    float kf[RB][VPL], vf[RB][VPL];
 #pragma unroll
-    for (int i = 0; i < VPL; ++i) {
-      kf[i] = bf16_bits_to_f32(kr[i]);
-      vf[i] = bf16_bits_to_f32(vr[i]);
+    for (int r = 0; r < RB; ++r) {
+      const int t = tb + r * kAttnWarps;
+      if (t < t1) {
+        load_bf16_row<VPL>(kc + (head_base + t) * D + lane * VPL, kf[r]);
+        load_bf16_row<VPL>(vc + (head_base + t) * D + lane * VPL, vf[r]);
+      }
     }
 #pragma unroll
-    for (int h = 0; h < kMaxGroup; ++h) {
-      if (h < g) {
-        float d = 0.f;
+    for (int r = 0; r < RB; ++r) {
+      if (tb + r * kAttnWarps >= t1) break;
 #pragma unroll
-        for (int i = 0; i < VPL; ++i) d = fmaf(qr[h][i], kf[i], d);
-        d = warp_sum(d);
-        const float mn = fmaxf(m[h], d);
-        const float a = expf(m[h] - mn);
-        const float p = expf(d - mn);
-        l[h] = l[h] * a + p;
+      for (int h = 0; h < kMaxGroup; ++h) {
+        if (h < g) {
+          float d = 0.f;
 #pragma unroll
-        for (int i = 0; i < VPL; ++i) o[h][i] = fmaf(o[h][i], a, p * vf[i]);
-        m[h] = mn;
+          for (int i = 0; i < VPL; ++i) d = fmaf(qr[h][i], kf[r][i], d);
+          d = warp_sum(d);
+          const float mn = fmaxf(m[h], d);
+          const float a = expf(m[h] - mn);
+          const float p = expf(d - mn);
+          l[h] = l[h] * a + p;
+#pragma unroll
+          for (int i = 0; i < VPL; ++i) o[h][i] = fmaf(o[h][i], a, p * vf[r][i]);
+          m[h] = mn;
+        }
       }
     }
   }
@@ -180,10 +284,11 @@ attention_split_kernel(const float* __restrict__ q, const uint16_t* __restrict__
   if (threadIdx.x == 0) ws_cnt[b * Hkv + kv] = 0u;  // ready for the next launch
 }
 
-cudaError_t attention_launch(const float* q, const uint16_t* kc, const uint16_t* vc,
-                             const int32_t* kv_len, const int32_t* pos_for_len, void* out,
-                             bool out_bf16, int B, int H, int Hkv, int D, int cap, float scale,
-                             void* ws, cudaStream_t st, bool pdl) {
+static cudaError_t attention_launch_any(const float* q, const uint16_t* kc, const uint16_t* vc,
+                                        const int32_t* kv_len, const int32_t* pos_for_len,
+                                        void* out, bool out_bf16, int B, int H, int Hkv, int D,
+                                        int cap, float scale, void* ws, cudaStream_t st, bool pdl,
+                                        const AttnFuse& fz) {
   const AttnPlan p = attn_plan(B, Hkv, cap);
   uint8_t* w = reinterpret_cast<uint8_t*>(ws);
   float* ws_o = reinterpret_cast<float*>(w);
@@ -196,7 +301,7 @@ cudaError_t attention_launch(const float* q, const uint16_t* kc, const uint16_t*
   case V:                                                                                      \
     return launch_pdl(attention_split_kernel<V>, grid, block, 0, st, pdl, q, kc, vc, kv_len,   \
                       pos_for_len, out, (int)out_bf16, H, Hkv, cap, scale, p.ch, p.nsplit,     \
-                      ws_o, ws_ml, ws_cnt);
+                      ws_o, ws_ml, ws_cnt, fz);
   switch (D / 32) {
     QG_ATTN_CASE(1)
     QG_ATTN_CASE(2)
@@ -210,6 +315,26 @@ cudaError_t attention_launch(const float* q, const uint16_t* kc, const uint16_t*
       return cudaErrorInvalidValue;
   }
 #undef QG_ATTN_CASE
+}
+
+cudaError_t attention_launch(const float* q, const uint16_t* kc, const uint16_t* vc,
+                             const int32_t* kv_len, const int32_t* pos_for_len, void* out,
+                             bool out_bf16, int B, int H, int Hkv, int D, int cap, float scale,
+                             void* ws, cudaStream_t st, bool pdl) {
+  AttnFuse fz = {};
+  return attention_launch_any(q, kc, vc, kv_len, pos_for_len, out, out_bf16, B, H, Hkv, D, cap,
+                              scale, ws, st, pdl, fz);
+}
+
+cudaError_t attention_launch_step(const float* q, const float* k, const float* v,
+                                  const uint16_t* q_norm, const uint16_t* k_norm,
+                                  const int32_t* tokens, int vocab, float eps, double theta,
+                                  uint16_t* kc, uint16_t* vc, const int32_t* positions, void* out,
+                                  int B, int H, int Hkv, int D, int cap, float scale, void* ws,
+                                  cudaStream_t st, bool pdl) {
+  AttnFuse fz = {1, k, v, q_norm, k_norm, tokens, vocab, eps, theta};
+  return attention_launch_any(q, kc, vc, nullptr, positions, out, true, B, H, Hkv, D, cap, scale,
+                              ws, st, pdl, fz);
 }
 
 // Offset of the ticket counters inside an attention workspace.

@@ -71,83 +71,6 @@ __global__ void step_embed_kernel(const uint32_t* __restrict__ w, const uint16_t
   pdl_trigger();
 }
 
-// Per-head q/k RMSNorm + NeoX RoPE (rotary_dim = head_dim) + K/V append.
-// Grid (H + 2*Hkv, B); one warp per head. q is rewritten in place (fp32);
-// K (normed, rotated) and V go to cache row pos as bf16.
-__global__ void step_qk_rope_append_kernel(float* __restrict__ q, const float* __restrict__ k,
-                                           const float* __restrict__ v,
-                                           const uint16_t* __restrict__ qn,
-                                           const uint16_t* __restrict__ kn,
-                                           const int32_t* __restrict__ pos,
-                                           const int32_t* __restrict__ tok,
-                                           uint16_t* __restrict__ kc, uint16_t* __restrict__ vc,
-                                           int H, int Hkv, int D, int cap, int vocab, float eps,
-                                           double theta) {
-  pdl_wait();
-  const int head = blockIdx.x, b = blockIdx.y, lane = threadIdx.x;
-  const int p = pos[b], t = tok[b];
-  // a bad token or position: nothing is written to the cache
-  const bool pos_ok = p >= 0 && p < cap && t >= 0 && t < vocab;
-  const int half = D >> 1, per = half >> 5;  // pairs per lane (D % 64 == 0) or 0
-  float* src;
-  const uint16_t* nw = nullptr;
-  uint16_t* dst = nullptr;
-  bool is_v = false;
-  if (head < H) {
-    src = q + ((size_t)b * H + head) * D;
-    nw = qn;
-  } else if (head < H + Hkv) {
-    const int kh = head - H;
-    src = const_cast<float*>(k) + ((size_t)b * Hkv + kh) * D;
-    nw = kn;
-    dst = kc + (((size_t)b * Hkv + kh) * cap + (pos_ok ? p : 0)) * D;
-  } else {
-    const int kh = head - H - Hkv;
-    src = const_cast<float*>(v) + ((size_t)b * Hkv + kh) * D;
-    dst = vc + (((size_t)b * Hkv + kh) * cap + (pos_ok ? p : 0)) * D;
-    is_v = true;
-  }
-  if (is_v) {
-    if (pos_ok)
-      for (int d = lane; d < D; d += 32) dst[d] = f32_to_bf16_bits(src[d]);
-    pdl_trigger();
-    return;
-  }
-  // D <= 256: each lane holds the pair (i, i+half) for i = lane + 32*j
-  float x1[4], x2[4];
-  float ss = 0.f;
-  for (int j = 0; j < 4; ++j) {
-    const int i = lane + 32 * j;
-    x1[j] = i < half ? src[i] : 0.f;
-    x2[j] = i < half ? src[i + half] : 0.f;
-    ss = fmaf(x1[j], x1[j], fmaf(x2[j], x2[j], ss));
-  }
-  ss = warp_sum(ss);
-  const float inv = 1.0f / sqrtf(ss / (float)D + eps);
-  for (int j = 0; j < 4; ++j) {
-    const int i = lane + 32 * j;
-    if (i >= half) break;
-    const float a = x1[j] * inv * bf16_bits_to_f32(nw[i]);
-    const float c2 = x2[j] * inv * bf16_bits_to_f32(nw[i + half]);
-    const double inv_freq = pow(theta, -2.0 * (double)i / (double)D);
-    double sd, cd;
-    sincos((double)(pos_ok ? p : 0) * inv_freq, &sd, &cd);
-    const float cs = (float)cd, sn = (float)sd;
-    const float r1 = a * cs - c2 * sn, r2 = c2 * cs + a * sn;
-    if (dst) {
-      if (pos_ok) {
-        dst[i] = f32_to_bf16_bits(r1);
-        dst[i + half] = f32_to_bf16_bits(r2);
-      }
-    } else {
-      src[i] = r1;
-      src[i + half] = r2;
-    }
-  }
-  (void)per;
-  pdl_trigger();
-}
-
 __global__ void step_silu_mul_kernel(const float* __restrict__ g, const float* __restrict__ u,
                                      uint16_t* __restrict__ out, int n) {
   pdl_wait();
@@ -307,11 +230,8 @@ extern "C" qg_status qg_decode_step_ex(const qg_qwen3_config* cfg, const qg_qwen
       rmsnorm_launch(x, L.input_norm, c.eps, xn, true, B, c.hidden, s, true);
       gemv_affine8_launch(qkv, 3, xn, false, c.hidden, B, s, true);
     }
-    launch_pdl(step_qk_rope_append_kernel, dim3(H + 2 * Hkv, B), dim3(32), 0, s, true, q,
-               (const float*)k, (const float*)v, L.q_norm, L.k_norm, positions, tokens, kc, vc, H,
-               Hkv, D, cap, c.vocab, c.eps, c.theta);
-    attention_launch(q, kc, vc, nullptr, positions, attn, true, B, H, Hkv, D, cap, scale, aws, s,
-                     true);
+    attention_launch_step(q, k, v, L.q_norm, L.k_norm, tokens, c.vocab, c.eps, c.theta, kc, vc,
+                          positions, attn, B, H, Hkv, D, cap, scale, aws, s, true);
     GemvSeg o = {L.o.w, L.o.scales, L.o.biases, x, x, c.hidden, 0};
     gemv_affine8_launch(&o, 1, attn, false, H * D, B, s, true);
     GemvSeg gu[2] = {{L.gate.w, L.gate.scales, L.gate.biases, gate, nullptr, c.ffn, 0},

@@ -231,27 +231,25 @@ __global__ void __launch_bounds__(Cfg<NT>::kThreads, 1)
     }
     __syncthreads();
   }
-  // 2) the input values, rounded to bf16, into xh (as bf16 bits for now)
+  // 2) the input values, rounded to bf16, into xh (as bf16 bits for now);
+  // batch rows past B are never read by a live B-operand lane
   float mx = 0.f;
-  for (int i = tid; i < 4 * NT * K; i += kThreads) {
-    const int b = i / K, c = i % K;
-    uint16_t h = 0;
-    if (b < P.B) {
-      const size_t o = (size_t)b * K + c;
-      if (P.xmode == kXBf16) {
-        h = P.x[o];
-      } else if (P.xmode == kXRmsNorm) {
-        float ib = inv[0];
+  for (int i = tid; i < P.B * K; i += kThreads) {
+    const int b = i / K, c = i - b * K;
+    uint16_t h;
+    if (P.xmode == kXBf16) {
+      h = P.x[i];
+    } else if (P.xmode == kXRmsNorm) {
+      float ib = inv[0];
 #pragma unroll
-        for (int j = 1; j < 4 * NT; ++j)
-          if (b == j) ib = inv[j];
-        h = f32_to_bf16_bits(P.xa[o] * ib * bf16_bits_to_f32(P.nw[c]));
-      } else {
-        const float z = P.xa[o];
-        h = f32_to_bf16_bits(z / (1.0f + expf(-z)) * P.xb[o]);
-      }
-      mx = fmaxf(mx, fabsf(bf16_bits_to_f32(h)));
+      for (int j = 1; j < 4 * NT; ++j)
+        if (b == j) ib = inv[j];
+      h = f32_to_bf16_bits(P.xa[i] * ib * bf16_bits_to_f32(P.nw[c]));
+    } else {
+      const float z = P.xa[i];
+      h = f32_to_bf16_bits(z / (1.0f + expf(-z)) * P.xb[i]);
     }
+    mx = fmaxf(mx, fabsf(bf16_bits_to_f32(h)));
     xh[b * xs + c] = h;
   }
   // 3) prescale 2^-e so that max|x| * 2^-e < 2^15 (fp16 max is 65504)
@@ -265,16 +263,21 @@ __global__ void __launch_bounds__(Cfg<NT>::kThreads, 1)
   if (mx >= 32768.f && mx <= 3.0e38f) e = (int)ceilf(log2f(mx / 16384.f));
   const float down = exp2f((float)-e), up = exp2f((float)e);
   // 4) bf16 -> fp16 in place (each thread converts the entries it wrote)
-  for (int i = tid; i < 4 * NT * K; i += kThreads) {
-    const int b = i / K, c = i % K;
+  for (int i = tid; i < P.B * K; i += kThreads) {
+    const int b = i / K, c = i - b * K;
     xh[b * xs + c] = __half_as_ushort(__float2half_rn(bf16_bits_to_f32(xh[b * xs + c]) * down));
   }
   __syncthreads();
-  for (int i = tid; i < 4 * NT * Kg; i += kThreads) {
-    const int b = i / Kg, gg = i % Kg;
-    float s = 0.f;
-    for (int j = 0; j < 64; ++j) s += __half2float(__ushort_as_half(xh[b * xs + 64 * gg + j]));
-    gsum[i] = s;
+  // 5) per 64-column group sums of the fp16 values, one warp per group
+  // (lanes read consecutive words: no bank conflicts); zero past B
+  for (int i = warp; i < 4 * NT * Kg; i += kWarps) {
+    const int b = i / Kg, gg = i - b * Kg;
+    float sum = 0.f;
+    if (b < P.B) {
+      const __half2 v = *reinterpret_cast<const __half2*>(xh + b * xs + 64 * gg + 2 * lane);
+      sum = warp_sum(__low2float(v) + __high2float(v));
+    }
+    if (lane == 0) gsum[i] = sum;
   }
   __syncthreads();
 

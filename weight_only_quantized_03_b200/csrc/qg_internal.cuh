@@ -168,6 +168,15 @@ cudaError_t attention_launch(const float* q, const uint16_t* kc, const uint16_t*
                              void* out, bool out_bf16, int B, int H, int Hkv, int D,
                              int cap, float scale, void* ws, cudaStream_t st, bool pdl);
 
+// The decode step's attention: q/k per-head RMSNorm, NeoX RoPE at
+// positions[b] and the K/V append at row positions[b] done inside the
+// attention kernel (raw fp32 q, k, v in), output bf16 [B][H][D]. D <= 256.
+cudaError_t attention_launch_step(const float* q, const float* k, const float* v,
+                                  const uint16_t* q_norm, const uint16_t* k_norm,
+                                  const int32_t* tokens, int vocab, float eps, double theta,
+                                  uint16_t* kc, uint16_t* vc, const int32_t* positions, void* out,
+                                  int B, int H, int Hkv, int D, int cap, float scale, void* ws,
+                                  cudaStream_t st, bool pdl);
 size_t attention_ws_bytes(int B, int H, int Hkv, int D, int cap);
 
 // persistent decode-step kernel (decode_mega.cu)
