@@ -215,6 +215,40 @@ qg_status qg_decode_attention(const float* q, const uint16_t* k_cache,
                               int Hkv, int D, int cap, float scale, void* ws,
                               size_t ws_bytes, void* stream);
 
+/* qg_decode_attention without a caller workspace. The pages have no
+ * counterpart: this is a library convenience, not a step of the method.
+ *
+ * Who needs it: callers that cannot hand the library device memory at the
+ * point of the call -- a plain C host that holds only the cache and
+ * activation buffers and has no device allocator, or a decode loop that
+ * must not call cudaMalloc / cudaFree between steps (cudaFree synchronises
+ * the whole device, and cudaMalloc may). This call allocates nothing. Its
+ * scratch (split partials and ticket counters) is a fixed device array
+ * inside libqg of qg_decode_attention_static_scratch_capacity() bytes
+ * (4 MiB) per device.
+ *
+ * Arguments, layouts and results as qg_decode_attention (same kernel, same
+ * numerics); there is no ws / ws_bytes.
+ * Limit: a shape whose scratch (qg_decode_attention_workspace_size) exceeds
+ * the fixed capacity is refused with QG_ERR_WORKSPACE_TOO_SMALL before any
+ * launch; use qg_decode_attention with a workspace for it.
+ * Setup: the first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current) and caches it; a failed
+ * lookup returns QG_ERR_CUDA. Make the first call on a device before any
+ * stream capture begins. Each call clears the ticket counters (an async
+ * memset on `stream`) before the launch.
+ * Concurrency: every call on one device shares the one scratch array, so
+ * calls must not overlap in time: issue them on one stream, or order them
+ * with events. Overlapping calls race on the scratch and give undefined
+ * results. */
+size_t qg_decode_attention_static_scratch_capacity(void);
+qg_status qg_decode_attention_static_scratch(const float* q, const uint16_t* k_cache,
+                                             const uint16_t* v_cache,
+                                             const int32_t* kv_len, void* out,
+                                             qg_dtype out_dtype, int B, int H,
+                                             int Hkv, int D, int cap, float scale,
+                                             void* stream);
+
 /* ------------------------------------------------------------------------
  * Whole Qwen3 decode step  [TS: step; MK: Qwen3DecoderLayer::forward]
  * ---------------------------------------------------------------------- */

@@ -79,6 +79,16 @@ def test_attention_rejects_bad_group_and_small_workspace():
     assert st == qg.QG_ERR_WORKSPACE_TOO_SMALL and str(need) in msg
 
 
+def test_attention_static_scratch_refuses_shapes_beyond_its_capacity():
+    cap_bytes = qg.lib.qg_decode_attention_static_scratch_capacity()
+    assert cap_bytes == 4 << 20
+    need = qg.lib.qg_decode_attention_workspace_size(32, 16, 8, 128, 32768)
+    assert need > cap_bytes
+    st, msg = _status("qg_decode_attention_static_scratch", FAKE, FAKE, FAKE, FAKE, FAKE,
+                      qg.QG_BF16, 32, 16, 8, 128, 32768, 1.0, None)
+    assert st == qg.QG_ERR_WORKSPACE_TOO_SMALL and str(need) in msg and str(cap_bytes) in msg
+
+
 def test_elementwise_reject_bad_shapes():
     assert _status("qg_rmsnorm", FAKE, FAKE, 1e-6, FAKE, qg.QG_BF16, 1, 6, None)[0] == \
         qg.QG_ERR_UNSUPPORTED_SHAPE

@@ -85,6 +85,9 @@ _SIGS = {
     "qg_decode_attention_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
     "qg_decode_attention": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _sz,
                                  _vp]),
+    "qg_decode_attention_static_scratch_capacity": (_sz, []),
+    "qg_decode_attention_static_scratch": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
+                                                _f, _vp]),
     "qg_decode_step_workspace_size": (_sz, [ctypes.POINTER(qg_qwen3_config), _i, _i]),
     "qg_decode_step": (_i, [ctypes.POINTER(qg_qwen3_config), ctypes.POINTER(qg_qwen3_weights),
                             _vp, _vp, _i, _vp, _vp, _vp, _i, _vp, _sz, _vp]),
@@ -212,6 +215,18 @@ def qg_decode_attention(q, k_cache, v_cache, kv_len, out, H, Hkv, scale, ws, str
     _call("qg_decode_attention", _p(q), _p(k_cache), _p(v_cache), _p(kv_len), _p(out), _dt(out),
           B, H, Hkv, D, cap, float(scale), _p(ws), ws.numel() * ws.element_size(),
           _stream(stream))
+
+
+def qg_decode_attention_static_scratch_capacity():
+    return int(lib.qg_decode_attention_static_scratch_capacity())
+
+
+def qg_decode_attention_static_scratch(q, k_cache, v_cache, kv_len, out, H, Hkv, scale,
+                                       stream=None):
+    """qg_decode_attention with the library's fixed scratch (no workspace)."""
+    B, _, cap, D = k_cache.shape
+    _call("qg_decode_attention_static_scratch", _p(q), _p(k_cache), _p(v_cache), _p(kv_len),
+          _p(out), _dt(out), B, H, Hkv, D, cap, float(scale), _stream(stream))
 
 
 def qg_unpack_affine8(w, out, stream=None):

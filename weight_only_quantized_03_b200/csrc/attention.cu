@@ -15,6 +15,8 @@
 //
 // Cache layout [B][Hkv][cap][D]: the rows of one head are contiguous, so a
 // split reads one contiguous CH*D*2-byte run of K and one of V.
+#include <mutex>
+
 #include "qg_internal.cuh"
 
 namespace qg {
@@ -393,4 +395,85 @@ extern "C" qg_status qg_decode_attention(const float* q, const uint16_t* k_cache
   attention_launch(q, k_cache, v_cache, kv_len, nullptr, out, out_dtype == QG_BF16, B, H, Hkv, D,
                    cap, scale, ws, s, false);
   return check_launch("qg_decode_attention");
+}
+
+// --------------------------------------------------------------------------
+// qg_decode_attention_static_scratch: the same attention with its scratch in
+// a fixed device array of this library instead of a caller workspace.
+//
+// Some callers cannot hand the library device memory at the point of the
+// call: a plain C host that holds only the cache and activation buffers
+// and no device allocator, or a decode loop that must not call cudaMalloc /
+// cudaFree between steps (cudaFree synchronises the device, cudaMalloc may).
+// This entry point allocates nothing: its split partials and ticket
+// counters live in g_attn_scratch below, a file-scope device array of
+// kAttnStaticScratchBytes, whose address the host looks up once per device.
+// --------------------------------------------------------------------------
+
+namespace qg {
+
+constexpr size_t kAttnStaticScratchBytes = 4u << 20;  // 4 MiB per device
+static __device__ __align__(256) uint8_t g_attn_scratch[kAttnStaticScratchBytes];
+
+constexpr int kMaxDevices = 64;
+
+// Device address of g_attn_scratch on the current device, looked up once per
+// device (with that device current) and cached.
+static cudaError_t attn_scratch_address(void** out) {
+  static std::mutex mu;
+  static void* addr[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_attn_scratch);
+    if (e != cudaSuccess) return e;
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace qg
+
+extern "C" size_t qg_decode_attention_static_scratch_capacity(void) {
+  return kAttnStaticScratchBytes;
+}
+
+extern "C" qg_status qg_decode_attention_static_scratch(const float* q, const uint16_t* k_cache,
+                                                        const uint16_t* v_cache,
+                                                        const int32_t* kv_len, void* out,
+                                                        qg_dtype out_dtype, int B, int H, int Hkv,
+                                                        int D, int cap, float scale,
+                                                        void* stream) {
+  clear_error();
+  qg_status st = validate_attention(q, k_cache, v_cache, kv_len, out, out_dtype, B, H, Hkv, D, cap);
+  if (st != QG_OK || B == 0) return st;
+  const size_t need = attention_ws_bytes(B, H, Hkv, D, cap);
+  QG_REQUIRE(need <= kAttnStaticScratchBytes, QG_ERR_WORKSPACE_TOO_SMALL,
+             "qg_decode_attention_static_scratch: this shape needs %zu bytes of scratch, more "
+             "than the fixed %zu; use qg_decode_attention with a caller workspace",
+             need, kAttnStaticScratchBytes);
+  void* ws = nullptr;
+  cudaError_t e = attn_scratch_address(&ws);
+  if (e != cudaSuccess) {
+    set_error("qg_decode_attention_static_scratch: scratch address lookup failed: %s",
+              cudaGetErrorString(e));
+    return QG_ERR_CUDA;
+  }
+  cudaStream_t s = (cudaStream_t)stream;
+  // the ticket counters must start at zero (the kernel also leaves them at
+  // zero; a cleared start does not depend on how the last call ended)
+  const size_t off = attention_ws_counter_offset(B, H, Hkv, D, cap);
+  e = cudaMemsetAsync(reinterpret_cast<uint8_t*>(ws) + off, 0, (size_t)B * Hkv * sizeof(unsigned int), s);
+  if (e != cudaSuccess) {
+    set_error("qg_decode_attention_static_scratch: %s", cudaGetErrorString(e));
+    return QG_ERR_CUDA;
+  }
+  attention_launch(q, k_cache, v_cache, kv_len, nullptr, out, out_dtype == QG_BF16, B, H, Hkv, D,
+                   cap, scale, ws, s, false);
+  return check_launch("qg_decode_attention_static_scratch");
 }
