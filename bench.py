@@ -71,21 +71,32 @@ def step_bytes(cfg, B, L):
 
 # ------------------------------------------------------------- plumbing -----
 
-def event_time_ms(fn, stream, n, warm=3):
-    """Mean duration of fn() over n launches, each bracketed by CUDA events
-    on `stream` (the stream the kernels run on)."""
+def graph_time_ms(fns, stream, n, warm=3):
+    """Mean device time of one launch: n launches (fns[i % len(fns)], so
+    inputs rotate over several copies) captured back to back in one CUDA graph
+    and bracketed by CUDA events on `stream`, the stream they run on; host
+    launch overhead is not in the figure."""
     import torch
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(n)]
     with torch.cuda.stream(stream):
-        for _ in range(warm):
-            fn()
-        for a, b in evs:
-            a.record(stream)
-            fn()
-            b.record(stream)
+        for i in range(warm):
+            fns[i % len(fns)]()
     stream.synchronize()
-    return statistics.mean(a.elapsed_time(b) for a, b in evs)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(n):
+            fns[i % len(fns)]()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        g.replay()
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+    stream.synchronize()
+    del g
+    return e0.elapsed_time(e1) / n
+
+
+L2_BYTES = 126 << 20
 
 
 def other_kernels(qg, stream, hbm_peak, n):
@@ -95,27 +106,35 @@ def other_kernels(qg, stream, hbm_peak, n):
     import torch
     to = lambda a: torch.from_numpy(a).cuda()
     M, N, K = 1500, 5120, 1280
-    blocks = to(qg_synth.q4_0_packed(N, K, 22))
+    bnp = qg_synth.q4_0_packed(N, K, 22)
+    blocks = to(bnp)
     A = to(qg_synth.gaussian((M, K), 1.0, 23).astype(np.float32))
     C = torch.empty((M, N), dtype=torch.float32, device="cuda")
     ws = torch.empty(qg.qg_gemm_q4_0_workspace_size(M, N, K), dtype=torch.uint8, device="cuda")
-    ms = event_time_ms(lambda: qg.qg_gemm_q4_0(blocks, A, C, ws=ws, stream=stream), stream, n)
+    ms = graph_time_ms([lambda: qg.qg_gemm_q4_0(blocks, A, C, ws=ws, stream=stream)], stream, n)
     tf_peak, tf_kind = measured_tensor_peak()
     tflops = 2.0 * M * N * K / (ms / 1000.0) / 1e12
+    # the GEMV streams copies of the matrix that together exceed L2 three times
+    vbytes = N * (K // 32) * 18 + K * 4 + N * 4
+    copies = -(-3 * L2_BYTES // bnp.nbytes)
+    mats = [to(bnp) for _ in range(copies)]
     x = to(qg_synth.gaussian((1, K), 1.0, 13).astype(np.float32))
     y = torch.empty((1, N), dtype=torch.float32, device="cuda")
-    ms_v = event_time_ms(lambda: qg.qg_gemv_q4_0(blocks, x, y, stream=stream), stream, n)
-    vbytes = N * (K // 32) * 18 + K * 4 + N * 4
+    fns = [(lambda m=m: qg.qg_gemv_q4_0(m, x, y, stream=stream)) for m in mats]
+    ms_v = graph_time_ms(fns, stream, max(n, 2 * copies))
     return {
         "gemm_q4_0_whisper_fc1": {
             "shape": [M, N, K], "bound": "tensor", "achieved": tflops, "peak": tf_peak,
             "unit": "TFLOP/s", "frac": tflops / tf_peak, "launch_us": ms * 1000.0,
             "peak_kind": tf_kind,
-            "note": "includes the A fp32->bf16 pass; FLOPs 2*M*N*K (dequant work not counted)"},
+            "note": "includes the A fp32->bf16 pass; FLOPs 2*M*N*K (dequant work not counted); "
+                    "back-to-back launches in a CUDA graph"},
         "gemv_q4_0_5120x1280_b1": {
             "bound": "hbm", "achieved": vbytes / (ms_v / 1000.0) / 1e9, "peak": hbm_peak,
             "unit": "GB/s", "frac": vbytes / (ms_v / 1000.0) / 1e9 / hbm_peak,
-            "algorithmic_bytes": vbytes, "launch_us": ms_v * 1000.0},
+            "algorithmic_bytes": vbytes, "launch_us": ms_v * 1000.0,
+            "note": f"back-to-back launches in a CUDA graph over {copies} copies of the matrix "
+                    "(more than 3x L2)"},
     }
 
 
@@ -355,17 +374,9 @@ def run_ours(args):
         .view(torch.bfloat16)
     yl = torch.empty((B, V), dtype=torch.float32, device="cuda")
     nlaunch = max(20, min(200, args.steps))
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(nlaunch)]
-    with torch.cuda.stream(stream):
-        for _ in range(5):
-            qg.qg_gemv_affine8_g64(ew, es, eb, xb, yl, stream=stream)
-        for a, b in evs:
-            a.record(stream)
-            qg.qg_gemv_affine8_g64(ew, es, eb, xb, yl, stream=stream)
-            b.record(stream)
-    stream.synchronize()
-    lm_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    # back to back in a CUDA graph; the 166 MB table exceeds L2 on its own
+    lm_ms = graph_time_ms([lambda: qg.qg_gemv_affine8_g64(ew, es, eb, xb, yl, stream=stream)],
+                          stream, nlaunch)
     lm_bytes = affine8_bytes(V, h, B)
     lm_gbs = lm_bytes / (lm_ms / 1000.0) / 1e9
     traffic = traffic_from_profile(os.path.join(ROOT, "weight_only_quantized_03_b200", "csrc",
@@ -472,6 +483,83 @@ def run_ncu_case(args):
     return 0
 
 
+def run_sweep(args):
+    """The Qwen3-1.7B-shaped decode (28 layers, hidden 2048, FFN 6144, vocab
+    151936, affine-INT8 g64): a 256-row prefill run row at a time as decode
+    steps at positions 0..255 (batch 1), then decode steps at KV lengths 512,
+    1024 and 2048 for batch 1, 2, 4, 8, 16 and 32, each a CUDA-graph replay
+    timed with CUDA events. Prints one JSON line (not the bench contract's
+    line)."""
+    import torch
+    import weight_only_quantized_03_b200 as qg
+    cfg = dict(qg_synth.QWEN3_1_7B)
+    weights = qg_synth.qwen3_weights(cfg, 19)
+    model = qg.Qwen3Model(cfg, weights)
+    cap = 2049
+    stream = torch.cuda.Stream()
+    gen = torch.Generator(device="cuda").manual_seed(90)
+    out = {"metric": "decode steps/s and tokens/s (Qwen3-1.7B shape, affine-INT8 g64)",
+           "data": "synthetic (seeded random packed weights; K/V cache N(0,1) bf16 drawn on device)",
+           "points": []}
+
+    def graph_step(st, toks, pos):
+        with torch.cuda.stream(stream):
+            for _ in range(2):
+                model.qg_decode_step(st, toks, pos, stream=stream)
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            model.qg_decode_step(st, toks, pos, stream=stream)
+        return g
+
+    # prefill: 256 rows, one decode step per row, batch 1
+    st = model.new_state(1, cap)
+    toks = torch.from_numpy(qg_synth.tokens(256, cfg["vocab"], 91)).cuda()
+    pos = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tok1 = toks[:1].clone()
+    g = graph_step(st, tok1, pos)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for r in range(256):
+            pos.fill_(r)
+            tok1.copy_(toks[r:r + 1])
+            g.replay()
+        e1.record(stream)
+    stream.synchronize()
+    ms = e0.elapsed_time(e1)
+    out["prefill_256_rows"] = {"ms": ms, "rows_per_s": 256 / (ms / 1000.0), "batch": 1}
+    del g, st
+
+    for B in (1, 2, 4, 8, 16, 32):
+        st = model.new_state(B, cap)
+        st["k_cache"].normal_(generator=gen)
+        st["v_cache"].normal_(generator=gen)
+        toks = torch.from_numpy(qg_synth.tokens(B, cfg["vocab"], 92)).cuda()
+        pos = torch.zeros(B, dtype=torch.int32, device="cuda")
+        per = {}
+        for L in (512, 1024, 2048):
+            pos.fill_(L - 1)
+            g = graph_step(st, toks, pos)
+            n = max(5, args.steps)
+            with torch.cuda.stream(stream):
+                for _ in range(args.warmup):
+                    g.replay()
+                e0.record(stream)
+                for _ in range(n):
+                    g.replay()
+                e1.record(stream)
+            stream.synchronize()
+            us = e0.elapsed_time(e1) / n * 1000.0
+            per[str(L)] = {"us_per_step": us, "steps_per_s": 1e6 / us, "tokens_per_s": B * 1e6 / us}
+            del g
+        out["points"].append({"batch": B, "kv_len": per})
+        del st
+        torch.cuda.empty_cache()
+    print(json.dumps(out), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -482,9 +570,15 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ncu-case", choices=["lm_head", "gemm"], default=None,
                     help="launch one kernel only (for an ncu capture); prints no JSON line")
+    ap.add_argument("--sweep", action="store_true",
+                    help="the Qwen3-1.7B-shaped prefill and batch sweep (its own JSON line)")
     args = ap.parse_args()
     if args.ncu_case:
         return run_ncu_case(args)
+    if args.sweep:
+        if args.warmup < 3:
+            args.warmup = 3
+        return run_sweep(args)
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":

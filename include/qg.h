@@ -320,16 +320,20 @@ qg_status qg_decode_step(const qg_qwen3_config* cfg, const qg_qwen3_weights* w,
                          float* logits, int B, void* ws, size_t ws_bytes,
                          void* stream);
 
-/* qg_decode_step with option flags. QG_STEP_MULTI_KERNEL forces the
- * kernel-per-op path (one launch per norm / GEMV / attention / elementwise
- * stage, chained with Programmatic Dependent Launch) instead of the
- * persistent one-launch kernel. Without the flag the persistent kernel runs
- * whenever the shapes allow it (B <= 4; hidden, heads*head_dim and ffn
- * multiples of 512 and <= 16384; head_dim 64 or 128; layers <= 64; 16-byte
- * aligned scales and biases) and the kernel-per-op path otherwise. Both
- * paths compute the same operations with the same precision points. */
+/* qg_decode_step with option flags. By default the step runs kernel-per-op
+ * (one launch per fused GEMV / attention stage, chained with Programmatic
+ * Dependent Launch; 5 launches per layer plus the embedding and the LM
+ * head). QG_STEP_PERSISTENT asks for the persistent one-launch kernel
+ * instead, which runs whenever the shapes allow it (B <= 4; hidden,
+ * heads*head_dim and ffn multiples of 512 and <= 16384; head_dim 64 or 128;
+ * layers <= 64; 16-byte aligned scales and biases) and falls back to the
+ * kernel-per-op path otherwise. QG_STEP_MULTI_KERNEL forces the
+ * kernel-per-op path (it overrides QG_STEP_PERSISTENT). Both paths compute
+ * the same operations with the same precision points. */
 #define QG_STEP_MULTI_KERNEL 1u
-/* Test hook for the persistent kernel: one device-side wait targets a
+#define QG_STEP_PERSISTENT 2u
+/* Test hook for the persistent kernel (with QG_STEP_PERSISTENT): one
+ * device-side wait targets a
  * counter that nothing sets, so it gives up after its 1 s bound and the
  * step records an error word (read it with qg_decode_step_error). The
  * step's outputs are then undefined; the context stays usable. */
@@ -340,6 +344,13 @@ qg_status qg_decode_step(const qg_qwen3_config* cfg, const qg_qwen3_weights* w,
  * [CTA][layer (last slot: LM head)][16 events]. */
 #define QG_STEP_TRACE 0x40000000u
 size_t qg_decode_step_trace_offset(const qg_qwen3_config* cfg, int B, int cap);
+/* Inspection aid for the kernel-per-op path (tests): byte offsets in the
+ * workspace of four bf16 arrays that, after a step, hold the LAST decoder
+ * layer's values at its bf16 rounding points: offsets[0] the input-norm
+ * output [B][hidden], offsets[1] the attention output [B][heads*head_dim],
+ * offsets[2] the post-attention-norm output [B][hidden], offsets[3] the
+ * SiLU-mul output [B][ffn]. (The persistent kernel does not write them.) */
+qg_status qg_decode_step_inspect(const qg_qwen3_config* cfg, int B, int cap, size_t offsets[4]);
 qg_status qg_decode_step_ex(const qg_qwen3_config* cfg, const qg_qwen3_weights* w,
                             uint16_t* k_cache, uint16_t* v_cache, int cap,
                             const int32_t* tokens, const int32_t* positions,

@@ -389,11 +389,119 @@ def decode_layer(cfg, lw, x, k_cache_l, v_cache_l, pos):
     return x + gemv_affine8(*lw["down"], hmid[None])[0]
 
 
+def bf16_alternative(v, rel):
+    """The other bf16 rounding of each value that lies within ``rel * |v|`` of
+    a bf16 rounding midpoint, NaN elsewhere.
+
+    A value computed in lower precision (float32 on the GPU) can land on
+    either side of such a midpoint, so both bf16 neighbours are correct
+    results there; this is the one ``round_bf16`` does not pick."""
+    v = np.asarray(v, dtype=np.float64)
+    r = round_bf16(v)
+    lo, hi = round_bf16_down(v), round_bf16_up(v)
+    near = (lo != hi) & (np.abs(v - (lo + hi) / 2.0) <= rel * np.abs(v))
+    return np.where(near, np.where(r == lo, hi, lo), np.nan)
+
+
+def bf16_rounding_ok(v, r, rel=2.0 ** -16, abs_tol=0.0):
+    """Whether each ``r`` is the bf16 rounding (to nearest even) of some
+    value within ``eps = rel * |v| + abs_tol`` of the float64 value ``v``.
+
+    This is the set of results that an implementation computing ``v`` with an
+    error of at most ``eps`` (float32 arithmetic, another summation order)
+    can store. ``round_bf16`` is monotonic, so the set is every bf16 value
+    from ``round_bf16(v - eps)`` to ``round_bf16(v + eps)``. Away from a
+    rounding midpoint and for ``eps`` below half a bf16 step, that is
+    ``round_bf16(v)`` alone. NaN matches NaN."""
+    v = np.asarray(v, dtype=np.float64)
+    r = np.asarray(r, dtype=np.float64)
+    eps = rel * np.abs(v) + abs_tol
+    ok = (r >= round_bf16(v - eps)) & (r <= round_bf16(v + eps))
+    return ok | (np.isnan(v) & np.isnan(r))
+
+
+def decode_layer_forced(cfg, lw, x, k_cache_l, v_cache_l, pos, forced, rel=2.0 ** -16,
+                        abs_rel=2.0 ** -12, details=None):
+    """``decode_layer`` teacher-forced at its bf16 rounding points.
+
+    ``forced`` maps points to the values another implementation stored there:
+    ``xn`` (input norm, [hidden]), ``k`` and ``v`` (the cache rows written at
+    ``pos``, [Hkv*D]), ``att`` (attention output, [H*D]), ``xn2``
+    (post-attention norm, [hidden]), ``h`` (SiLU-mul output, [ffn]). At each
+    point the layer's own float64 value is computed from what came before,
+    each forced value is checked to be a correct bf16 rounding of it
+    (``bf16_rounding_ok``: the rounding of a value within
+    ``rel * |v| + abs_rel * rms`` of it, rms that of the point's vector --
+    float32 errors of an element scale with its vector, and where the
+    residual stream is small they are magnified by the norm after it), and the
+    layer continues from the forced values. Where two roundings are both
+    correct, the rest of the layer follows the other implementation's choice.
+    Returns ``(y, bad)``: the new residual stream and, per point, the indices
+    whose forced value is not a correct rounding (with ``details``, a dict,
+    filled per point with those indices' own values, the forced values, their
+    distance to the rounding midpoint and the point's RMS). Rows ``pos`` of the caches
+    receive the forced (else the rounded) K and V."""
+    H, Hkv, D = cfg["heads"], cfg["kv_heads"], cfg["head_dim"]
+    eps, theta = cfg["eps"], cfg["theta"]
+    bad = {}
+
+    def at(name, val):
+        if name not in forced:
+            return round_bf16(val)
+        f = np.asarray(forced[name], dtype=np.float64).reshape(val.shape)
+        # float32 errors of a vector's elements (cancellation in a dot
+        # product, in a rotation, in a residual add) scale with the vector,
+        # not the element: the error bound has a part relative to its RMS
+        scale = float(np.sqrt(np.mean(np.square(val[np.isfinite(val)])))) if val.size else 0.0
+        bad[name] = np.flatnonzero(~bf16_rounding_ok(val, f, rel, abs_rel * scale))
+        if details is not None and bad[name].size:
+            i = bad[name]
+            mid = (round_bf16_down(val[i]) + round_bf16_up(val[i])) / 2.0
+            details[name] = {"index": i, "value": val[i], "forced": f[i],
+                             "to_midpoint": np.abs(val[i] - mid), "rms": scale}
+        return f
+
+    xn = at("xn", rmsnorm(x, lw["input_norm"], eps))
+    q = gemv_affine8(*lw["q"], xn[None])[0]
+    k = gemv_affine8(*lw["k"], xn[None])[0]
+    v = gemv_affine8(*lw["v"], xn[None])[0]
+    q = rope_neox(rmsnorm_perhead(q, lw["q_norm"], eps, D), pos, theta, D)
+    k = rope_neox(rmsnorm_perhead(k, lw["k_norm"], eps, D), pos, theta, D)
+    k_cache_l[:, pos, :] = at("k", k).reshape(Hkv, D)
+    v_cache_l[:, pos, :] = at("v", v).reshape(Hkv, D)
+    att = at("att", decode_attention(q, k_cache_l, v_cache_l, pos + 1, H, Hkv, D))
+    x = x + gemv_affine8(*lw["o"], att[None])[0]
+    xn2 = at("xn2", rmsnorm(x, lw["post_norm"], eps))
+    gate = gemv_affine8(*lw["gate"], xn2[None])[0]
+    up = gemv_affine8(*lw["up"], xn2[None])[0]
+    hmid = at("h", silu_mul(gate, up))
+    return x + gemv_affine8(*lw["down"], hmid[None])[0], bad
+
+
 def lm_head(cfg, weights, x):
     """Final RMSNorm (bf16 output) and the tied LM head of [TS] ``step``."""
     ew, es, eb = weights["embed"]
     xn = round_bf16(rmsnorm(x, weights["final_norm"], cfg["eps"]))
     return gemv_affine8(ew, es, eb, xn[None])[0]
+
+
+def lm_head_tie_bound(cfg, weights, x, rel=2.0 ** -18):
+    """``lm_head`` plus the bound on the effect of bf16 rounding ties of the
+    final norm (see ``decode_layer_tie_bound``): the head is linear in the
+    normed vector, so a tie at element j moves logit r by
+    ``|w[r][j]| * |alt_j - round_j|`` exactly. Returns ``(logits, extra)``."""
+    ew, es, eb = weights["embed"]
+    v = rmsnorm(x, weights["final_norm"], cfg["eps"])
+    xn = round_bf16(v)
+    logits = gemv_affine8(ew, es, eb, xn[None])[0]
+    alt = bf16_alternative(v, rel)
+    extra = np.zeros_like(logits)
+    codes = affine8_unpack(ew)
+    sc, bi = bf16_bits_to_f64(es), bf16_bits_to_f64(eb)
+    for j in np.flatnonzero(~np.isnan(alt)):
+        col = codes[:, j] * sc[:, j // GROUP] + bi[:, j // GROUP]
+        extra += np.abs(col) * abs(alt[j] - xn[j])
+    return logits, extra
 
 
 def decode_step(cfg, weights, k_cache, v_cache, token, pos):

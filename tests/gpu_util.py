@@ -6,6 +6,8 @@ For outputs stored as bf16 the bf16 store adds at most half a bf16 ulp of the
 value, bounded here by 2^-8 |ref| (``bf16_out=True``). When both sides store
 bf16 (the oracle rounds too, e.g. K/V cache rows), values a hair apart can
 round to neighbouring bf16 numbers: one full ulp, 2^-7 |ref| (``ulps=1``).
+Downstream of such a rounding inside a decoder layer, the oracle's
+``decode_layer_tie_bound`` gives the added bound (``extra``).
 """
 import numpy as np
 import torch
@@ -33,11 +35,15 @@ def host64(t):
     return t.detach().float().cpu().numpy().astype(np.float64)
 
 
-def assert_parity(gpu, ref, bf16_out=False, what="", ulps=0.5):
+def assert_parity(gpu, ref, bf16_out=False, what="", ulps=0.5, extra=None):
+    """``extra``: an added per-element bound, for outputs downstream of bf16
+    roundings that sit on a tie (the oracle's ``decode_layer_tie_bound``)."""
     gpu = np.asarray(gpu, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     assert gpu.shape == ref.shape, (what, gpu.shape, ref.shape)
     tol = ATOL + RTOL * np.abs(ref)
+    if extra is not None:
+        tol = tol + np.asarray(extra, dtype=np.float64)
     if bf16_out:
         tol = tol + 2 * ulps * BF16_HALF_ULP_REL * np.abs(ref)
     err = np.abs(gpu - ref)

@@ -50,20 +50,41 @@ def _greedy_ok(gpu_logits, ref_logits):
     return abs(top[1] - top[0]) <= 2 * (ATOL + RTOL * abs(top[1]))
 
 
+def _forced_layer(cfg, lw, x, kc_l, vc_l, p, inter_b, k_row, v_row, what):
+    """The oracle layer teacher-forced with the GPU's bf16 values at its
+    rounding points (each checked to be a correct rounding of the oracle's
+    own value there: exact, or the other side of a near-tie)."""
+    forced = dict(inter_b, k=k_row.ravel(), v=v_row.ravel())
+    det = {}
+    ref, bad = O.decode_layer_forced(cfg, lw, x, kc_l, vc_l, p, forced, details=det)
+    for name, idx in bad.items():
+        assert idx.size == 0, f"{what}: {name} is not a correct bf16 rounding: {det.get(name)}"
+    return ref
+
+
+def _intermediates(model, st):
+    return {k: host64(t) for k, t in model.intermediates(st).items()}
+
+
 def _step_checked(model, st, cfg, w, caches, toks, p, flags=0):
     """One decode step at position p for every sequence, checked stage by
     stage from identical inputs: the GPU prefix runs (the same step cut to l
     layers) give the residual stream entering each layer; the oracle runs
-    that one layer from the GPU's input and the shared cache state; the
-    appended K/V rows are compared (one bf16 ulp, both sides round) and then
-    the oracle continues from the GPU's rows; the LM head is checked from the
-    GPU's final residual stream. Returns the GPU logits."""
+    that one layer from the GPU's input. On the kernel-per-op path the oracle
+    is teacher-forced at the layer's bf16 rounding points with the GPU's own
+    values (after checking each is a correct rounding); on the persistent
+    path the appended K/V rows are compared (one bf16 ulp) and the oracle
+    continues from the GPU's rows. The LM head is checked from the GPU's
+    final residual stream. Returns the GPU logits."""
     B = len(toks)
+    persistent = bool(flags & qg.QG_STEP_PERSISTENT)
     t, pos = dev(np.array(toks, np.int32)), dev(np.full(B, p, np.int32))
-    xs = []
+    xs, inter = [], []
     for l in range(cfg["layers"] + 1):
         model.qg_decode_step(st, t, pos, layers=l, flags=flags)
         xs.append(host64(model.residual(st)))
+        if l >= 1 and not persistent:
+            inter.append(_intermediates(model, st))
     logits = host64(st["logits"])
     kg, vg = host64(st["k_cache"]), host64(st["v_cache"])
     ew, es, eb = w["embed"]
@@ -71,15 +92,22 @@ def _step_checked(model, st, cfg, w, caches, toks, p, flags=0):
     for b in range(B):
         kc, vc = caches[b]
         for l in range(cfg["layers"]):
-            ref = O.decode_layer(cfg, w["layers"][l], xs[l][b], kc[l], vc[l], p)
-            assert_parity(xs[l + 1][b], ref, what=f"b={b} p={p} layer {l}")
-            assert_parity(kg[l, b, :, p, :], kc[l, :, p, :], bf16_out=True, ulps=1,
-                          what=f"b={b} p={p} layer {l} K row")
-            assert_parity(vg[l, b, :, p, :], vc[l, :, p, :], bf16_out=True, ulps=1,
-                          what=f"b={b} p={p} layer {l} V row")
-            kc[l, :, p, :] = kg[l, b, :, p, :]
-            vc[l, :, p, :] = vg[l, b, :, p, :]
-        assert_parity(logits[b], O.lm_head(cfg, w, xs[-1][b]), what=f"b={b} p={p} LM head")
+            what = f"b={b} p={p} layer {l}"
+            if persistent:
+                ref = O.decode_layer(cfg, w["layers"][l], xs[l][b], kc[l], vc[l], p)
+                assert_parity(kg[l, b, :, p, :], kc[l, :, p, :], bf16_out=True, ulps=1,
+                              what=f"{what} K row")
+                assert_parity(vg[l, b, :, p, :], vc[l, :, p, :], bf16_out=True, ulps=1,
+                              what=f"{what} V row")
+                kc[l, :, p, :] = kg[l, b, :, p, :]
+                vc[l, :, p, :] = vg[l, b, :, p, :]
+            else:
+                ref = _forced_layer(cfg, w["layers"][l], xs[l][b], kc[l], vc[l], p,
+                                    {k: a[b] for k, a in inter[l].items()},
+                                    kg[l, b, :, p, :], vg[l, b, :, p, :], what)
+            assert_parity(xs[l + 1][b], ref, what=what)
+        ref, tie = O.lm_head_tie_bound(cfg, w, xs[-1][b])
+        assert_parity(logits[b], ref, extra=tie, what=f"b={b} p={p} LM head")
     assert model.qg_decode_step_error(st) == (0, 0)
     return logits
 
@@ -106,11 +134,11 @@ SMALL = dict(hidden=512, layers=3, heads=4, kv_heads=2, head_dim=128, ffn=1024, 
              eps=1e-6, theta=1e6)
 
 
-@pytest.mark.parametrize("B,flags", [(1, 0), (3, 0), (3, 1), (4, 0)])
+@pytest.mark.parametrize("B,flags", [(1, 2), (3, 2), (3, 0), (4, 2), (1, 0)])
 def test_small_decoder_stagewise_greedy_both_paths(B, flags):
     """A decoder small enough for a 40-step oracle run yet shaped for the
-    persistent kernel (flags=0) -- and the same run on the kernel-per-op path
-    (flags=QG_STEP_MULTI_KERNEL). Positions 0..39 cross the 32-row attention
+    persistent kernel (flags=QG_STEP_PERSISTENT) -- and the same run on the
+    default kernel-per-op path (flags=0). Positions 0..39 cross the 32-row attention
     chunks; B sequences start from different tokens and follow the GPU's
     greedy tokens; every step is checked stage by stage (_step_checked)."""
     cfg = dict(SMALL)
@@ -125,7 +153,7 @@ def test_small_decoder_stagewise_greedy_both_paths(B, flags):
         toks = [int(np.argmax(logits[b])) for b in range(B)]
 
 
-@pytest.mark.parametrize("B,flags", [(1, 0), (2, 0), (1, 1)])
+@pytest.mark.parametrize("B,flags", [(1, 2), (2, 2), (1, 0), (2, 0)])
 def test_qwen3_0_6b_step_layer_by_layer_at_position_511(B, flags):
     """Teacher-forced per layer: layer l of the oracle starts from the GPU's
     residual stream after l-1 layers, so each comparison covers the bf16
@@ -144,10 +172,13 @@ def test_qwen3_0_6b_step_layer_by_layer_at_position_511(B, flags):
     toks = dev(qg_synth.tokens(B, cfg["vocab"], 72))
     pos_np = np.array([511, 300][:B], dtype=np.int32)
     pos = dev(pos_np)
-    xs = []
+    persistent = bool(flags & qg.QG_STEP_PERSISTENT)
+    xs, inter = [], []
     for l in range(Lr + 1):
         model.qg_decode_step(st, toks, pos, layers=l, flags=flags)
         xs.append(host64(model.residual(st)))
+        if l >= 1 and not persistent:
+            inter.append(_intermediates(model, st))
     logits = host64(st["logits"])
     kg, vg = host64(st["k_cache"]), host64(st["v_cache"])
     ew, es, eb = w["embed"]
@@ -157,14 +188,63 @@ def test_qwen3_0_6b_step_layer_by_layer_at_position_511(B, flags):
         kc = O.bf16_bits_to_f64(kbits[:, b])
         vc = O.bf16_bits_to_f64(vbits[:, b])
         for l in range(Lr):
-            ref = O.decode_layer(cfg, w["layers"][l], xs[l][b], kc[l], vc[l], p)
-            assert_parity(xs[l + 1][b], ref, what=f"b={b} layer {l} residual")
-            assert_parity(kg[l, b, :, p, :], kc[l, :, p, :], bf16_out=True, ulps=1,
-                          what=f"layer {l} K row")
-            assert_parity(vg[l, b, :, p, :], vc[l, :, p, :], bf16_out=True, ulps=1,
-                          what=f"layer {l} V row")
+            what = f"b={b} layer {l}"
+            if persistent:
+                ref = O.decode_layer(cfg, w["layers"][l], xs[l][b], kc[l], vc[l], p)
+                assert_parity(kg[l, b, :, p, :], kc[l, :, p, :], bf16_out=True, ulps=1,
+                              what=f"{what} K row")
+                assert_parity(vg[l, b, :, p, :], vc[l, :, p, :], bf16_out=True, ulps=1,
+                              what=f"{what} V row")
+            else:
+                ref = _forced_layer(cfg, w["layers"][l], xs[l][b], kc[l], vc[l], p,
+                                    {k: a[b] for k, a in inter[l].items()},
+                                    kg[l, b, :, p, :], vg[l, b, :, p, :], what)
+            assert_parity(xs[l + 1][b], ref, what=f"{what} residual")
             np.testing.assert_array_equal(kg[l, b, :, p + 1, :], kc[l, :, p + 1, :])
-        assert_parity(logits[b], O.lm_head(cfg, w, xs[Lr][b]), what=f"b={b} LM head")
+        ref, tie = O.lm_head_tie_bound(cfg, w, xs[Lr][b])
+        assert_parity(logits[b], ref, extra=tie, what=f"b={b} LM head")
+
+
+@pytest.mark.parametrize("B,layers", [(2, 3), (12, 2)])
+def test_qwen3_1_7b_shaped_layers_at_position_2047(B, layers):
+    """The 1.7B layer shapes (hidden 2048, FFN 6144, K/V cache of 2049 rows)
+    with a few layers, teacher-forced per layer at positions up to 2047 on the
+    default kernel-per-op path. B = 12 takes the CUDA-core GEMV (batch past
+    the tensor-core path's 8) with RMSNorm and SiLU-mul as separate kernels."""
+    cfg = dict(qg_synth.QWEN3_1_7B, layers=layers)
+    w = qg_synth.qwen3_weights(cfg, 17)
+    model = qg.Qwen3Model(cfg, w)
+    cap = 2049
+    st = model.new_state(B, cap)
+    Lr, Hkv, D = cfg["layers"], cfg["kv_heads"], cfg["head_dim"]
+    kbits = _prefill((Lr, B, Hkv, cap, D), 80)
+    vbits = _prefill((Lr, B, Hkv, cap, D), 81)
+    st["k_cache"].copy_(dev(kbits).view(torch.bfloat16))
+    st["v_cache"].copy_(dev(vbits).view(torch.bfloat16))
+    toks = dev(qg_synth.tokens(B, cfg["vocab"], 82))
+    pos_np = np.array([2047, 1000, 5, 2048, 0, 777, 1500, 31, 32, 33, 1999, 64][:B], dtype=np.int32)
+    pos = dev(pos_np)
+    xs, inter = [], []
+    for l in range(Lr + 1):
+        model.qg_decode_step(st, toks, pos, layers=l)
+        xs.append(host64(model.residual(st)))
+        if l >= 1:
+            inter.append(_intermediates(model, st))
+    logits = host64(st["logits"])
+    kg, vg = host64(st["k_cache"]), host64(st["v_cache"])
+    for b in range(B):
+        p = int(pos_np[b])
+        kc = O.bf16_bits_to_f64(kbits[:, b])
+        vc = O.bf16_bits_to_f64(vbits[:, b])
+        for l in range(Lr):
+            what = f"b={b} p={p} layer {l}"
+            ref = _forced_layer(cfg, w["layers"][l], xs[l][b], kc[l], vc[l], p,
+                                {k: a[b] for k, a in inter[l].items()},
+                                kg[l, b, :, p, :], vg[l, b, :, p, :], what)
+            assert_parity(xs[l + 1][b], ref, what=f"{what} residual")
+        if b < 2:  # the LM head oracle (151936 x 2048 in f64) for two rows
+            ref, tie = O.lm_head_tie_bound(cfg, w, xs[Lr][b])
+            assert_parity(logits[b], ref, extra=tie, what=f"b={b} LM head")
 
 
 def test_qwen3_0_6b_step_whole_depth_bf16_cascade_bound():
@@ -223,9 +303,9 @@ def test_device_wait_timeout_is_reported_and_context_survives():
     model = qg.Qwen3Model(cfg, w)
     st = model.new_state(1, 8)
     t, p = dev(np.array([3], np.int32)), dev(np.array([0], np.int32))
-    model.qg_decode_step(st, t, p, flags=qg.QG_STEP_TEST_STALL)
+    model.qg_decode_step(st, t, p, flags=qg.QG_STEP_PERSISTENT | qg.QG_STEP_TEST_STALL)
     status, code = model.qg_decode_step_error(st)
     assert status == qg.QG_ERR_TIMEOUT and code != 0
-    model.qg_decode_step(st, t, p)
+    model.qg_decode_step(st, t, p, flags=qg.QG_STEP_PERSISTENT)
     assert model.qg_decode_step_error(st) == (0, 0)
-    _step_checked(model, st, cfg, w, [O.new_kv_cache(cfg, 8)], [3], 0)
+    _step_checked(model, st, cfg, w, [O.new_kv_cache(cfg, 8)], [3], 0, flags=qg.QG_STEP_PERSISTENT)

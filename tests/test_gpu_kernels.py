@@ -178,6 +178,8 @@ GEMM_CASES = [
     (1500, 1280, 1280, True, False),
     (1500, 5120, 1280, True, False),
     (1500, 1280, 5120, True, False),
+    # two 128-row A sub-tiles per CTA, the last CTA's second one wholly past M
+    (1300, 5120, 128, True, False),
 ]
 
 
@@ -193,6 +195,21 @@ def test_gemm_q4_0(M, N, K, bias, quant):
     assert qg.qg_gemm_q4_0_error(M, K, ws) == (0, 0)
     ref = O.gemm_q4_0_bf16(blocks, A, None if bv is None else bv.astype(np.float64))
     assert_parity(host64(C), ref, what=f"q4_0 gemm {M}x{N}x{K}")
+
+
+def test_gemm_q4_0_two_byte_aligned_blocks():
+    # blocks only 2-byte aligned: W bytes are read 16 bits at a time
+    M, N, K = 300, 512, 256
+    blocks = qg_synth.q4_0_packed(N, K, 31)
+    buf = torch.zeros(blocks.size + 2, dtype=torch.uint8, device="cuda")
+    buf[2:].copy_(dev(blocks).view(-1))
+    bl = buf[2:].view(N, -1)
+    A = qg_synth.gaussian((M, K), 1.0, 32)
+    C = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    ws = torch.empty(qg.qg_gemm_q4_0_workspace_size(M, N, K), dtype=torch.uint8, device="cuda")
+    qg.qg_gemm_q4_0(bl, dev(A), C, ws=ws)
+    assert qg.qg_gemm_q4_0_error(M, K, ws) == (0, 0)
+    assert_parity(host64(C), O.gemm_q4_0_bf16(blocks, A), what="q4_0 gemm, 2-byte aligned blocks")
 
 
 # -------------------------------------------------------- elementwise ------

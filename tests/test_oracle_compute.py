@@ -278,3 +278,136 @@ def test_decode_step_zero_weights_closed_form():
     row = e[t].astype(np.float32).astype(np.float64)
     xn = torch.from_numpy(row / np.sqrt(np.mean(row ** 2) + cfg["eps"])).to(torch.bfloat16).double().numpy()
     np.testing.assert_allclose(logits, e @ xn, rtol=1e-12, atol=1e-12)
+
+
+def test_bf16_alternative_marks_only_near_midpoint_values():
+    # 1 and 1 + 2^-7 are neighbouring bf16 values; 1 + 2^-8 is their midpoint
+    mid = 1.0 + 2.0 ** -8
+    v = np.array([mid, mid * (1 + 2.0 ** -20), mid * (1 - 2.0 ** -20), 1.0 + 2.0 ** -10,
+                  -mid, 3.0, 0.0])
+    alt = O.bf16_alternative(v, 2.0 ** -18)
+    # the midpoint rounds to even (1.0); the other neighbour is 1 + 2^-7
+    assert alt[0] == 1.0 + 2.0 ** -7
+    assert alt[1] == 1.0 and alt[2] == 1.0 + 2.0 ** -7   # just above / below: the other side
+    assert np.isnan(alt[3]) and np.isnan(alt[5]) and np.isnan(alt[6])
+    assert alt[4] == -(1.0 + 2.0 ** -7)
+    # with rel = 0 only exact midpoints count
+    assert np.isnan(O.bf16_alternative(v[1:2], 0.0)[0])
+    # the alternative is always a bf16 value adjacent to round_bf16(v)
+    r = O.round_bf16(v[:3])
+    assert np.all(np.abs(alt[:3] - r) == 2.0 ** -7)
+
+
+def test_bf16_rounding_ok_is_the_set_of_roundings_within_the_error_bound():
+    mid = 1.0 + 2.0 ** -8                        # midpoint of 1 and 1 + 2^-7
+    up, down = 1.0 + 2.0 ** -7, 1.0
+    near = mid * (1 + 2.0 ** -20)
+    # within the bound of a midpoint both neighbours are roundings of a value
+    # in [v - eps, v + eps]
+    assert O.bf16_rounding_ok([near], [up])[0] and O.bf16_rounding_ok([near], [down])[0]
+    # far from it only the nearest one
+    far = 1.0 + 2.0 ** -10
+    assert O.bf16_rounding_ok([far], [down])[0] and not O.bf16_rounding_ok([far], [up])[0]
+    # a value on the grid rounds to itself; two steps away is never right
+    assert O.bf16_rounding_ok([1.0], [1.0])[0] and not O.bf16_rounding_ok([1.0], [up])[0]
+    assert not O.bf16_rounding_ok([near], [1.0 + 2.0 ** -6])[0]
+    assert O.bf16_rounding_ok([np.nan], [np.nan])[0]
+    # an absolute bound well above a tiny value's own bf16 step admits every
+    # rounding inside it, and nothing outside
+    t = 3.6e-6
+    step = 2.0 ** -26                            # bf16 step at 2^-19 .. 2^-18
+    cand = O.round_bf16(t) + step * np.arange(-4, 5)
+    ok = O.bf16_rounding_ok(np.full(cand.shape, t), cand, abs_tol=2.5 * step)
+    want = [bool(np.any(O.round_bf16(np.linspace(t - 2.5 * step, t + 2.5 * step, 4001)) == c))
+            for c in cand]
+    assert list(ok) == want and 5 <= sum(want) <= 6
+    # brute force: r is accepted exactly when some value within eps rounds to it
+    g = np.random.default_rng(7)
+    v = g.normal(size=400)
+    eps = 2.0 ** -9 * np.abs(v)
+    below = lambda a: float(O.round_bf16_down(np.nextafter(a, -np.inf)))   # next bf16 down
+    above = lambda a: float(O.round_bf16_up(np.nextafter(a, np.inf)))      # next bf16 up
+    for vi, ei in zip(v, eps):
+        grid = np.linspace(vi - ei, vi + ei, 2001)
+        reach = set(O.round_bf16(grid).tolist())
+        lo, hi = min(reach), max(reach)
+        for r in (lo, hi, below(lo), above(hi)):
+            assert bool(O.bf16_rounding_ok([vi], [r], rel=2.0 ** -9)[0]) == (r in reach), (vi, r)
+
+
+def _small_layer():
+    cfg = dict(hidden=512, layers=1, heads=4, kv_heads=2, head_dim=128, ffn=1024, vocab=300,
+               eps=1e-6, theta=1e6)
+    w = qg_synth.qwen3_weights(cfg, 9, norm_jitter=0.1)
+    x = O.embed_rows(*w["embed"], [17])[0]
+    kc, vc = O.new_kv_cache(cfg, 16)
+    kc[:] = O.bf16_bits_to_f64(qg_synth.gaussian_bf16_bits(kc.shape, 1.0, 3))
+    vc[:] = O.bf16_bits_to_f64(qg_synth.gaussian_bf16_bits(vc.shape, 1.0, 4))
+    return cfg, w["layers"][0], x, kc[0], vc[0]
+
+
+def test_decode_layer_forced_with_its_own_roundings_is_decode_layer():
+    cfg, lw, x, kc, vc = _small_layer()
+    k1, v1 = kc.copy(), vc.copy()
+    y = O.decode_layer(cfg, lw, x, k1, v1, 9)
+    # no forced values: the same layer
+    k2, v2 = kc.copy(), vc.copy()
+    y2, bad = O.decode_layer_forced(cfg, lw, x, k2, v2, 9, {})
+    np.testing.assert_array_equal(y2, y)
+    np.testing.assert_array_equal(k2, k1)
+    assert bad == {}
+    # forcing the rounded values the layer computes itself changes nothing
+    D, eps = cfg["head_dim"], cfg["eps"]
+    xn = O.round_bf16(O.rmsnorm(x, lw["input_norm"], eps))
+    k3, v3 = kc.copy(), vc.copy()
+    y3, bad3 = O.decode_layer_forced(cfg, lw, x, k3, v3, 9,
+                                     {"xn": xn, "k": k1[:, 9, :].ravel(), "v": v1[:, 9, :].ravel()})
+    np.testing.assert_array_equal(y3, y)
+    assert all(b.size == 0 for b in bad3.values())
+
+
+def test_decode_layer_forced_flags_wrong_values_and_follows_valid_ones():
+    cfg, lw, x, kc, vc = _small_layer()
+    eps = cfg["eps"]
+    v = O.rmsnorm(x, lw["input_norm"], eps)
+    xn = O.round_bf16(v)
+    # a value two bf16 steps off is flagged at its index
+    wrong = xn.copy()
+    wrong[5] = O.round_bf16_up(xn[5] * (1 + 2.0 ** -7) + 1e-30)
+    wrong[5] = O.round_bf16_up(wrong[5] * (1 + 2.0 ** -7) + 1e-30)
+    _, bad = O.decode_layer_forced(cfg, lw, x, kc.copy(), vc.copy(), 9, {"xn": wrong})
+    assert list(bad["xn"]) == [5]
+    # the other neighbour is accepted only where the value is near a tie: with
+    # a tie window of a full bf16 step every neighbour passes, and the layer
+    # then follows the forced value (its output differs from the plain layer)
+    lo, hi = O.round_bf16_down(v), O.round_bf16_up(v)
+    other = np.where(xn == lo, hi, lo)
+    y_plain = O.decode_layer(cfg, lw, x, kc.copy(), vc.copy(), 9)
+    y_f, bad_f = O.decode_layer_forced(cfg, lw, x, kc.copy(), vc.copy(), 9, {"xn": other},
+                                       rel=2.0 ** -7, abs_rel=0.0)
+    assert bad_f["xn"].size == 0 and np.abs(y_f - y_plain).max() > 0
+    _, bad_t = O.decode_layer_forced(cfg, lw, x, kc.copy(), vc.copy(), 9, {"xn": other})
+    assert bad_t["xn"].size > 300   # with the default bound most are wrong
+
+
+def test_lm_head_tie_bound_is_the_exact_linear_effect_of_each_tie():
+    cfg = dict(hidden=256, layers=0, heads=2, kv_heads=1, head_dim=128, ffn=256, vocab=500,
+               eps=1e-6, theta=1e6)
+    w = qg_synth.qwen3_weights(cfg, 4, norm_jitter=0.2)
+    x = qg_synth.gaussian((256,), 1.0, 5).astype(np.float64)
+    logits, ex0 = O.lm_head_tie_bound(cfg, w, x, rel=0.0)
+    np.testing.assert_array_equal(logits, O.lm_head(cfg, w, x))
+    assert np.all(ex0 == 0)
+    rel = 2.0 ** -9   # a quarter of the values count as ties
+    _, ex = O.lm_head_tie_bound(cfg, w, x, rel=rel)
+    v = O.rmsnorm(x, w["final_norm"], cfg["eps"])
+    xn = O.round_bf16(v)
+    alt = O.bf16_alternative(v, rel)
+    ties = np.flatnonzero(~np.isnan(alt))
+    assert ties.size > 0
+    brute = np.zeros_like(logits)
+    for j in ties:   # one tie at a time through the full head
+        xa = xn.copy()
+        xa[j] = alt[j]
+        brute += np.abs(O.gemv_affine8(*w["embed"], xa[None])[0] - logits)
+    np.testing.assert_allclose(ex, brute, rtol=1e-9, atol=1e-12)

@@ -32,6 +32,7 @@ QG_ERR_TIMEOUT = 6
 QG_F32 = 0
 QG_BF16 = 1
 QG_STEP_MULTI_KERNEL = 1
+QG_STEP_PERSISTENT = 2
 QG_STEP_TEST_STALL = 0x80000000
 QG_STEP_TRACE = 0x40000000
 
@@ -96,6 +97,8 @@ _SIGS = {
     "qg_decode_step_error": (_i, [ctypes.POINTER(qg_qwen3_config), _i, _i, _vp,
                                   ctypes.POINTER(ctypes.c_uint), _vp]),
     "qg_decode_step_trace_offset": (_sz, [ctypes.POINTER(qg_qwen3_config), _i, _i]),
+    "qg_decode_step_inspect": (_i, [ctypes.POINTER(qg_qwen3_config), _i, _i,
+                                    ctypes.POINTER(ctypes.c_size_t)]),
     "qg_unpack_affine8": (_i, [_vp, _vp, _i, _i, _vp]),
     "qg_dequant_affine8_g64": (_i, [_vp, _vp, _vp, _vp, _i, _i, _vp]),
     "qg_dequant_q4_0": (_i, [_vp, _vp, _i, _i, _vp]),
@@ -301,6 +304,20 @@ class Qwen3Model:
         latest step (the head of the step workspace, per include/qg.h)."""
         n = state["B"] * self.cfg["hidden"]
         return state["ws"][: 4 * n].view(torch.float32).view(state["B"], self.cfg["hidden"])
+
+    def intermediates(self, state):
+        """The last decoder layer's bf16 values at its rounding points after
+        a kernel-per-op step (``qg_decode_step_inspect``): dict of torch
+        bf16 views ``xn`` [B, hidden], ``attn`` [B, heads*head_dim], ``xn2``
+        [B, hidden], ``h`` [B, ffn] into the workspace."""
+        off = (ctypes.c_size_t * 4)()
+        _call("qg_decode_step_inspect", ctypes.byref(self.c_cfg), state["B"], state["cap"], off)
+        c, B = self.cfg, state["B"]
+        ws = state["ws"]
+        def view(o, n):
+            return ws[o:o + 2 * B * n].view(torch.bfloat16).view(B, n)
+        return {"xn": view(off[0], c["hidden"]), "attn": view(off[1], c["heads"] * c["head_dim"]),
+                "xn2": view(off[2], c["hidden"]), "h": view(off[3], c["ffn"])}
 
     def qg_decode_step_error(self, state, stream=None):
         """Device error word of the latest step (synchronises the stream)."""

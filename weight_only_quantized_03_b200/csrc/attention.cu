@@ -23,6 +23,7 @@ namespace qg {
 
 constexpr int kAttnWarps = 4;
 constexpr int kMaxGroup = 8;
+constexpr int kMergeMax = 1024;  // (head, split) pairs the last CTA merges from shared memory
 
 struct AttnPlan {
   int ch;      // rows per split
@@ -30,12 +31,14 @@ struct AttnPlan {
 };
 
 static AttnPlan attn_plan(int B, int Hkv, int cap) {
-  // Aim for about two CTAs per SM across B * Hkv * splits.
-  const long long want = 2LL * 148;
+  // About four CTAs per SM across B * Hkv * splits, splits of 32 to 256 rows
+  // (a warp then walks at most 64 rows, 8 of them in flight at a time); the
+  // last CTA of each (sequence, kv head) merges the splits.
+  const long long want = 4LL * 148;
   long long ch = ((long long)cap * B * Hkv + want - 1) / want;
   ch = ((ch + 31) / 32) * 32;
   if (ch < 32) ch = 32;
-  if (ch > 1024) ch = 1024;
+  if (ch > 256) ch = 256;
   AttnPlan p;
   p.ch = (int)ch;
   p.nsplit = (int)((cap + ch - 1) / ch);
@@ -66,15 +69,15 @@ struct AttnFuse {
   const int32_t* tok;    // [B]: a bad token writes nothing to the cache
   int vocab;
   float eps;
-  double theta;
+  const float2* rope;    // (cos, sin) [B][D/2] of the step's positions
 };
 
-// RMSNorm of one head row src[0..D) with weight w, then NeoX rotation at
-// position p; lane owns the pairs (i, i + D/2) for i = lane + 32 j.
-// Writes the rotated fp32 values through `put(i, value)`.
+// RMSNorm of one head row src[0..D) with weight w, then the NeoX rotation
+// with the (cos, sin) pairs cs[0..D/2); lane owns the pairs (i, i + D/2) for
+// i = lane + 32 j. Writes the rotated fp32 values through `put(i, value)`.
 template <typename Put>
 __device__ __forceinline__ void norm_rope_head(const float* src, const uint16_t* w, int D, float eps,
-                                               double theta, int p, int lane, Put put) {
+                                               const float2* cs, int lane, Put put) {
   const int half = D >> 1;
   float x1[4], x2[4];
   float ss = 0.f;
@@ -93,12 +96,9 @@ __device__ __forceinline__ void norm_rope_head(const float* src, const uint16_t*
     if (i >= half) break;
     const float a = x1[j] * inv * bf16_bits_to_f32(w[i]);
     const float c2 = x2[j] * inv * bf16_bits_to_f32(w[i + half]);
-    const double inv_freq = pow(theta, -2.0 * (double)i / (double)D);
-    double sd, cd;
-    sincos((double)p * inv_freq, &sd, &cd);
-    const float cs = (float)cd, sn = (float)sd;
-    put(i, a * cs - c2 * sn);
-    put(i + half, c2 * cs + a * sn);
+    const float2 r = cs[i];
+    put(i, a * r.x - c2 * r.y);
+    put(i + half, c2 * r.x + a * r.y);
   }
 }
 
@@ -138,11 +138,47 @@ attention_split_kernel(const float* __restrict__ q, const uint16_t* __restrict__
   __shared__ float sm[kAttnWarps][kMaxGroup], sl[kAttnWarps][kMaxGroup];
   __shared__ float so[kAttnWarps][kMaxGroup][D];
   __shared__ unsigned int s_ticket;
+  // after the warp merge, `so` is free: the split merge reuses it
+  constexpr int kMerge = kAttnWarps * kMaxGroup * D / 2 < kMergeMax ? kAttnWarps * kMaxGroup * D / 2
+                                                                     : kMergeMax;
+  float* s_m = &so[0][0][0];
+  float* s_l = s_m + kMerge;
 
+  const int t0 = s * ch;
+  const size_t head_base = ((size_t)b * Hkv + kv) * cap;
+  // RB rows per warp in flight: all their K/V loads are issued before the
+  // first score, so the rows' memory latencies overlap
+  constexpr int RB = VPL <= 4 ? 8 : 4;
+  float kf[RB][VPL], vf[RB][VPL];
+#pragma unroll
+  for (int r = 0; r < RB; ++r)
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) kf[r][i] = vf[r][i] = 0.f;
+  // Decode step: the positions are an input of the step (final before its
+  // first kernel ran), and the cached rows below the position were written
+  // by earlier steps, so the first batch of rows is fetched before waiting
+  // for the previous kernel; the row at the position is this step's own.
+  int pre_p = -1;
+  if (fz.on) {
+    const int p = pos_for_len[b];
+    if (p >= 0 && p < cap) {
+      pre_p = p;
+      const int t1p = min(p + 1, t0 + ch);
+#pragma unroll
+      for (int r = 0; r < RB; ++r) {
+        const int t = t0 + warp + r * kAttnWarps;
+        if (t < t1p && t != p) {
+          load_bf16_row<VPL>(kc + (head_base + t) * D + lane * VPL, kf[r]);
+          load_bf16_row<VPL>(vc + (head_base + t) * D + lane * VPL, vf[r]);
+        }
+      }
+    }
+  }
+  // the next kernel may be scheduled now: its own wait covers all of this one
+  pdl_trigger();
   pdl_wait();
   const int L = pos_for_len ? pos_for_len[b] + 1 : kv_len[b];
   const bool valid = L >= 1 && L <= cap;
-  const int t0 = s * ch;
   const int t1 = valid ? min(L, t0 + ch) : 0;
 
   if (!fz.on) {
@@ -154,17 +190,18 @@ attention_split_kernel(const float* __restrict__ q, const uint16_t* __restrict__
     const int p = pos_for_len[b], tk = fz.tok[b];
     const bool pos_ok = p >= 0 && p < cap && tk >= 0 && tk < fz.vocab;
     const int pr = pos_ok ? p : 0;
+    const float2* cs = fz.rope + (size_t)b * (D / 2);
     const bool owner = pos_ok && p >= t0 && p < t0 + ch;
     const size_t row = (((size_t)b * Hkv + kv) * cap + pr) * D;
     for (int hh = warp; hh < g + 2; hh += kAttnWarps) {
       if (hh < g) {
         float* dst = sq[hh];
-        norm_rope_head(q + ((size_t)b * H + kv * g + hh) * D, fz.qn, D, fz.eps, fz.theta, pr, lane,
+        norm_rope_head(q + ((size_t)b * H + kv * g + hh) * D, fz.qn, D, fz.eps, cs, lane,
                        [&](int i, float r) { dst[i] = r * scale; });
       } else if (hh == g) {
         if (owner) {
           uint16_t* kdst = const_cast<uint16_t*>(kc) + row;
-          norm_rope_head(fz.k + ((size_t)b * Hkv + kv) * D, fz.kn, D, fz.eps, fz.theta, pr, lane,
+          norm_rope_head(fz.k + ((size_t)b * Hkv + kv) * D, fz.kn, D, fz.eps, cs, lane,
                          [&](int i, float r) { kdst[i] = f32_to_bf16_bits(r); });
         }
       } else if (owner) {
@@ -188,42 +225,55 @@ attention_split_kernel(const float* __restrict__ q, const uint16_t* __restrict__
     }
   }
 
-  const size_t head_base = ((size_t)b * Hkv + kv) * cap;
-  // RB rows per warp in flight: all their K/V loads are issued before the
-  // first score, so the rows' memory latencies overlap
-  constexpr int RB = VPL <= 4 ? 8 : 4;
   for (int tb = t0 + warp; tb < t1; tb += kAttnWarps * RB) {
-    float kf[RB][VPL], vf[RB][VPL];
+    // the first batch was fetched before the wait except the current row
+    const bool prefetched = pre_p >= 0 && tb == t0 + warp;
 #pragma unroll
     for (int r = 0; r < RB; ++r) {
       const int t = tb + r * kAttnWarps;
-      if (t < t1) {
+      if (t < t1 && (!prefetched || t == pre_p)) {
         load_bf16_row<VPL>(kc + (head_base + t) * D + lane * VPL, kf[r]);
         load_bf16_row<VPL>(vc + (head_base + t) * D + lane * VPL, vf[r]);
       }
     }
+    // per head: the batch's scores (dot products and warp reductions are
+    // independent, so their latencies overlap), then one online-softmax
+    // update for the whole batch: running max over the batch, one rescale
+    // of (l, o), and the batch's exp-weighted V rows added
 #pragma unroll
-    for (int r = 0; r < RB; ++r) {
-      if (tb + r * kAttnWarps >= t1) break;
+    for (int h = 0; h < kMaxGroup; ++h) {
+      if (h < g) {
+        float dsc[RB];
 #pragma unroll
-      for (int h = 0; h < kMaxGroup; ++h) {
-        if (h < g) {
+        for (int r = 0; r < RB; ++r) {
           float d = 0.f;
 #pragma unroll
           for (int i = 0; i < VPL; ++i) d = fmaf(qr[h][i], kf[r][i], d);
-          d = warp_sum(d);
-          const float mn = fmaxf(m[h], d);
-          const float a = expf(m[h] - mn);
-          const float p = expf(d - mn);
-          l[h] = l[h] * a + p;
-#pragma unroll
-          for (int i = 0; i < VPL; ++i) o[h][i] = fmaf(o[h][i], a, p * vf[r][i]);
-          m[h] = mn;
+          dsc[r] = d;
         }
+#pragma unroll
+        for (int r = 0; r < RB; ++r) dsc[r] = warp_sum(dsc[r]);
+        float mx = m[h];
+#pragma unroll
+        for (int r = 0; r < RB; ++r)
+          if (tb + r * kAttnWarps < t1) mx = fmaxf(mx, dsc[r]);
+        const float a = expf(m[h] - mx);  // 0 while m is still -inf
+        l[h] *= a;
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) o[h][i] *= a;
+#pragma unroll
+        for (int r = 0; r < RB; ++r) {
+          if (tb + r * kAttnWarps < t1) {
+            const float p = expf(dsc[r] - mx);
+            l[h] += p;
+#pragma unroll
+            for (int i = 0; i < VPL; ++i) o[h][i] = fmaf(p, vf[r][i], o[h][i]);
+          }
+        }
+        m[h] = mx;
       }
     }
   }
-  pdl_trigger();
 
   // merge the warps of this CTA
 #pragma unroll
@@ -262,26 +312,75 @@ attention_split_kernel(const float* __restrict__ q, const uint16_t* __restrict__
   if (s_ticket != (unsigned)(nsplit - 1)) return;
   __threadfence();
 
-  for (int i = threadIdx.x; i < g * D; i += blockDim.x) {
-    const int h = i / D, d = i % D;
-    const size_t pb = part + (size_t)h * nsplit;
-    float M = -INFINITY;
-    for (int j = 0; j < nsplit; ++j) M = fmaxf(M, __ldcg(ws_ml + (pb + j) * 2));
-    float Lsum = 0.f, O = 0.f;
-    if (M != -INFINITY) {
-      for (int j = 0; j < nsplit; ++j) {
-        const float mj = __ldcg(ws_ml + (pb + j) * 2);
-        const float e = mj == -INFINITY ? 0.f : expf(mj - M);
-        Lsum = fmaf(__ldcg(ws_ml + (pb + j) * 2 + 1), e, Lsum);
-        O = fmaf(__ldcg(ws_o + (pb + j) * D + d), e, O);
-      }
-    }
-    const float r = (valid && Lsum > 0.f) ? O / Lsum : 0.f;
+  auto store_out = [&](int h, int d, float r) {
     const size_t oi = ((size_t)b * H + kv * g + h) * D + d;
     if (out_bf16)
       reinterpret_cast<uint16_t*>(out)[oi] = f32_to_bf16_bits(r);
     else
       reinterpret_cast<float*>(out)[oi] = r;
+  };
+  const int nw = g * nsplit;
+  if (nw <= kMerge) {
+    // 1) every split's (max, sum) of the kv head's query heads: one round of
+    // loads; 2) per head, the weight of split j, exp(m_j - M) / L (0 for an
+    // empty split or an invalid length); 3) the weighted sum of the split
+    // outputs, with the loads of several splits in flight together
+    for (int i = threadIdx.x; i < nw; i += blockDim.x) {
+      s_m[i] = __ldcg(ws_ml + (part + i) * 2);
+      s_l[i] = __ldcg(ws_ml + (part + i) * 2 + 1);
+    }
+    __syncthreads();
+    for (int h = warp; h < g; h += kAttnWarps) {
+      float M = -INFINITY;
+      for (int j = lane; j < nsplit; j += 32) M = fmaxf(M, s_m[h * nsplit + j]);
+      M = warp_max(M);
+      float Lsum = 0.f;
+      for (int j = lane; j < nsplit; j += 32) {
+        const float mj = s_m[h * nsplit + j];
+        Lsum += (mj == -INFINITY) ? 0.f : s_l[h * nsplit + j] * expf(mj - M);
+      }
+      Lsum = warp_sum(Lsum);
+      const float scale_out = (valid && Lsum > 0.f) ? 1.0f / Lsum : 0.f;
+      for (int j = lane; j < nsplit; j += 32) {
+        const float mj = s_m[h * nsplit + j];
+        s_m[h * nsplit + j] = (mj == -INFINITY) ? 0.f : expf(mj - M) * scale_out;
+      }
+    }
+    __syncthreads();
+    for (int i0 = threadIdx.x; i0 < g * D; i0 += 2 * blockDim.x) {
+      const int i1 = i0 + blockDim.x;
+      const bool has1 = i1 < g * D;
+      const int h0 = i0 / D, d0 = i0 % D, h1 = has1 ? i1 / D : h0, d1 = has1 ? i1 % D : d0;
+      const float* o0 = ws_o + (part + (size_t)h0 * nsplit) * D + d0;
+      const float* o1 = ws_o + (part + (size_t)h1 * nsplit) * D + d1;
+      float O0 = 0.f, O1 = 0.f;
+#pragma unroll 8
+      for (int j = 0; j < nsplit; ++j) {
+        O0 = fmaf(s_m[h0 * nsplit + j], __ldcg(o0 + (size_t)j * D), O0);
+        O1 = fmaf(s_m[h1 * nsplit + j], __ldcg(o1 + (size_t)j * D), O1);
+      }
+      store_out(h0, d0, O0);
+      if (has1) store_out(h1, d1, O1);
+    }
+  } else {
+    for (int i = threadIdx.x; i < g * D; i += blockDim.x) {
+      const int h = i / D, d = i % D;
+      const size_t pb = part + (size_t)h * nsplit;
+      float M = -INFINITY;
+#pragma unroll 8
+      for (int j = 0; j < nsplit; ++j) M = fmaxf(M, __ldcg(ws_ml + (pb + j) * 2));
+      float Lsum = 0.f, O = 0.f;
+      if (M != -INFINITY) {
+#pragma unroll 8
+        for (int j = 0; j < nsplit; ++j) {
+          const float mj = __ldcg(ws_ml + (pb + j) * 2);
+          const float e = mj == -INFINITY ? 0.f : expf(mj - M);
+          Lsum = fmaf(__ldcg(ws_ml + (pb + j) * 2 + 1), e, Lsum);
+          O = fmaf(__ldcg(ws_o + (pb + j) * D + d), e, O);
+        }
+      }
+      store_out(h, d, (valid && Lsum > 0.f) ? O / Lsum : 0.f);
+    }
   }
   if (threadIdx.x == 0) ws_cnt[b * Hkv + kv] = 0u;  // ready for the next launch
 }
@@ -330,11 +429,11 @@ cudaError_t attention_launch(const float* q, const uint16_t* kc, const uint16_t*
 
 cudaError_t attention_launch_step(const float* q, const float* k, const float* v,
                                   const uint16_t* q_norm, const uint16_t* k_norm,
-                                  const int32_t* tokens, int vocab, float eps, double theta,
+                                  const int32_t* tokens, int vocab, float eps, const float2* rope,
                                   uint16_t* kc, uint16_t* vc, const int32_t* positions, void* out,
                                   int B, int H, int Hkv, int D, int cap, float scale, void* ws,
                                   cudaStream_t st, bool pdl) {
-  AttnFuse fz = {1, k, v, q_norm, k_norm, tokens, vocab, eps, theta};
+  AttnFuse fz = {1, k, v, q_norm, k_norm, tokens, vocab, eps, rope};
   return attention_launch_any(q, kc, vc, nullptr, positions, out, true, B, H, Hkv, D, cap, scale,
                               ws, st, pdl, fz);
 }

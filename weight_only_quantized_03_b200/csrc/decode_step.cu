@@ -18,7 +18,7 @@ namespace qg {
 size_t attention_ws_counter_offset(int B, int H, int Hkv, int D, int cap);
 
 struct StepLayout {
-  size_t x, xn, q, k, v, attn, gate, up, h, attn_ws, mx, cnt, step, trace, total;
+  size_t x, xn, xn2, xnf, q, k, v, attn, gate, up, h, attn_ws, rope, mx, cnt, step, trace, total;
 };
 
 static size_t a256(size_t v) { return (v + 255) & ~(size_t)255; }
@@ -34,6 +34,8 @@ static StepLayout step_layout(const qg_qwen3_config& c, int B, int cap) {
   L.cnt = take(64);
   L.step = take(64);
   L.xn = take((size_t)B * c.hidden * 2);
+  L.xn2 = take((size_t)B * c.hidden * 2);
+  L.xnf = take((size_t)B * c.hidden * 2);
   L.q = take((size_t)B * qd * 4);
   L.k = take((size_t)B * kd * 4);
   L.v = take((size_t)B * kd * 4);
@@ -42,21 +44,32 @@ static StepLayout step_layout(const qg_qwen3_config& c, int B, int cap) {
   L.up = take((size_t)B * c.ffn * 4);
   L.h = take((size_t)B * c.ffn * 2);
   L.attn_ws = take(attention_ws_bytes(B, c.heads, c.kv_heads, c.head_dim, cap));
+  L.rope = take((size_t)B * (c.head_dim / 2) * 8);
   L.mx = take(mega_ws_bytes(c, B, cap));
   L.trace = take((size_t)num_sms() * ((c.layers + 1) * 16 + 1024) * 8);
   L.total = off;
   return L;
 }
 
-// Embedding rows; a sequence with a bad token or position gets NaN.
+// Embedding rows; a sequence with a bad token or position gets NaN. Also
+// the step's RoPE table: (cos, sin) of pos * theta^(-2i/D) for the D/2
+// pairs of every sequence, angles in double (position 0 for a bad
+// sequence, whose outputs are NaN anyway); every layer's attention reads it.
 __global__ void step_embed_kernel(const uint32_t* __restrict__ w, const uint16_t* __restrict__ s,
                                   const uint16_t* __restrict__ bi, const int32_t* __restrict__ tok,
                                   const int32_t* __restrict__ pos, float* __restrict__ x, int vocab,
-                                  int hidden, int cap) {
+                                  int hidden, int cap, float2* __restrict__ rope, int D,
+                                  double theta) {
   pdl_wait();
   const int b = blockIdx.x;
   const int t = tok[b], p = pos[b];
   const bool ok = t >= 0 && t < vocab && p >= 0 && p < cap;
+  for (int i = threadIdx.x; i < D / 2; i += blockDim.x) {
+    const double inv_freq = pow(theta, -2.0 * (double)i / (double)D);
+    double sd, cd;
+    sincos((double)(ok ? p : 0) * inv_freq, &sd, &cd);
+    rope[(size_t)b * (D / 2) + i] = make_float2((float)cd, (float)sd);
+  }
   float* xr = x + (size_t)b * hidden;
   for (int c = threadIdx.x; c < hidden; c += blockDim.x) {
     if (!ok) {
@@ -188,6 +201,8 @@ extern "C" qg_status qg_decode_step_ex(const qg_qwen3_config* cfg, const qg_qwen
   uint8_t* base = reinterpret_cast<uint8_t*>(ws);
   float* x = reinterpret_cast<float*>(base + Ly.x);
   uint16_t* xn = reinterpret_cast<uint16_t*>(base + Ly.xn);
+  uint16_t* xn2 = reinterpret_cast<uint16_t*>(base + Ly.xn2);
+  uint16_t* xnf = reinterpret_cast<uint16_t*>(base + Ly.xnf);
   float* q = reinterpret_cast<float*>(base + Ly.q);
   float* k = reinterpret_cast<float*>(base + Ly.k);
   float* v = reinterpret_cast<float*>(base + Ly.v);
@@ -201,7 +216,8 @@ extern "C" qg_status qg_decode_step_ex(const qg_qwen3_config* cfg, const qg_qwen
   const size_t layer_cache = (size_t)B * Hkv * cap * D;
   const float scale = 1.0f / sqrtf((float)D);
 
-  if (!(flags & QG_STEP_MULTI_KERNEL) && c.layers >= 1 && mega_eligible(c, B, cap) &&
+  if ((flags & QG_STEP_PERSISTENT) && !(flags & QG_STEP_MULTI_KERNEL) && c.layers >= 1 &&
+      mega_eligible(c, B, cap) &&
       mega_pointers_ok(c, w)) {
     mega_launch(c, *w, k_cache, v_cache, cap, tokens, positions, logits, B, x, base + Ly.mx,
                 reinterpret_cast<unsigned*>(base + Ly.cnt), reinterpret_cast<unsigned*>(base + Ly.step),
@@ -213,8 +229,9 @@ extern "C" qg_status qg_decode_step_ex(const qg_qwen3_config* cfg, const qg_qwen
   }
   cudaMemsetAsync(reinterpret_cast<uint8_t*>(base + Ly.cnt), 0, 64, s);
   cudaMemsetAsync(reinterpret_cast<uint8_t*>(aws) + cnt_off, 0, (size_t)B * Hkv * 4, s);
+  float2* rope = reinterpret_cast<float2*>(base + Ly.rope);
   launch_pdl(step_embed_kernel, dim3(B), dim3(256), 0, s, true, w->embed.w, w->embed.scales,
-             w->embed.biases, tokens, positions, x, c.vocab, c.hidden, cap);
+             w->embed.biases, tokens, positions, x, c.vocab, c.hidden, cap, rope, D, c.theta);
   for (int l = 0; l < c.layers; ++l) {
     const qg_qwen3_layer& L = w->layers[l];
     uint16_t* kc = k_cache + l * layer_cache;
@@ -225,26 +242,26 @@ extern "C" qg_status qg_decode_step_ex(const qg_qwen3_config* cfg, const qg_qwen
     // RMSNorm and SiLU-mul run in the next GEMV's prologue where the
     // tensor-core GEMV takes the shape, as separate kernels otherwise
     if (gemv_tc_eligible(qkv, 3, c.hidden, B, false)) {
-      gemv_tc_launch_rmsnorm(qkv, 3, x, L.input_norm, c.eps, c.hidden, B, s, true);
+      gemv_tc_launch_rmsnorm(qkv, 3, x, L.input_norm, c.eps, c.hidden, B, s, true, xn);
     } else {
       rmsnorm_launch(x, L.input_norm, c.eps, xn, true, B, c.hidden, s, true);
       gemv_affine8_launch(qkv, 3, xn, false, c.hidden, B, s, true);
     }
-    attention_launch_step(q, k, v, L.q_norm, L.k_norm, tokens, c.vocab, c.eps, c.theta, kc, vc,
+    attention_launch_step(q, k, v, L.q_norm, L.k_norm, tokens, c.vocab, c.eps, rope, kc, vc,
                           positions, attn, B, H, Hkv, D, cap, scale, aws, s, true);
     GemvSeg o = {L.o.w, L.o.scales, L.o.biases, x, x, c.hidden, 0};
     gemv_affine8_launch(&o, 1, attn, false, H * D, B, s, true);
     GemvSeg gu[2] = {{L.gate.w, L.gate.scales, L.gate.biases, gate, nullptr, c.ffn, 0},
                      {L.up.w, L.up.scales, L.up.biases, up, nullptr, c.ffn, 0}};
     if (gemv_tc_eligible(gu, 2, c.hidden, B, false)) {
-      gemv_tc_launch_rmsnorm(gu, 2, x, L.post_norm, c.eps, c.hidden, B, s, true);
+      gemv_tc_launch_rmsnorm(gu, 2, x, L.post_norm, c.eps, c.hidden, B, s, true, xn2);
     } else {
-      rmsnorm_launch(x, L.post_norm, c.eps, xn, true, B, c.hidden, s, true);
-      gemv_affine8_launch(gu, 2, xn, false, c.hidden, B, s, true);
+      rmsnorm_launch(x, L.post_norm, c.eps, xn2, true, B, c.hidden, s, true);
+      gemv_affine8_launch(gu, 2, xn2, false, c.hidden, B, s, true);
     }
     GemvSeg dn = {L.down.w, L.down.scales, L.down.biases, x, x, c.hidden, 0};
     if (gemv_tc_eligible(&dn, 1, c.ffn, B, false)) {
-      gemv_tc_launch_silu_mul(&dn, 1, gate, up, c.ffn, B, s, true);
+      gemv_tc_launch_silu_mul(&dn, 1, gate, up, c.ffn, B, s, true, hm);
     } else {
       const int n = B * c.ffn;
       launch_pdl(step_silu_mul_kernel, dim3((n + 255) / 256), dim3(256), 0, s, true,
@@ -256,8 +273,8 @@ extern "C" qg_status qg_decode_step_ex(const qg_qwen3_config* cfg, const qg_qwen
   if (gemv_tc_eligible(&head, 1, c.hidden, B, false)) {
     gemv_tc_launch_rmsnorm(&head, 1, x, w->final_norm, c.eps, c.hidden, B, s, true);
   } else {
-    rmsnorm_launch(x, w->final_norm, c.eps, xn, true, B, c.hidden, s, true);
-    gemv_affine8_launch(&head, 1, xn, false, c.hidden, B, s, true);
+    rmsnorm_launch(x, w->final_norm, c.eps, xnf, true, B, c.hidden, s, true);
+    gemv_affine8_launch(&head, 1, xnf, false, c.hidden, B, s, true);
   }
   return check_launch("qg_decode_step");
 }
@@ -281,6 +298,20 @@ extern "C" qg_status qg_decode_step_error(const qg_qwen3_config* cfg, int B, int
     set_error("qg_decode_step: a device-side wait gave up (code 0x%x)", *code);
     return QG_ERR_TIMEOUT;
   }
+  return QG_OK;
+}
+
+extern "C" qg_status qg_decode_step_inspect(const qg_qwen3_config* cfg, int B, int cap,
+                                           size_t offsets[4]) {
+  clear_error();
+  qg_status st = validate_cfg(cfg, B, cap);
+  if (st != QG_OK) return st;
+  QG_REQUIRE(offsets, QG_ERR_INVALID_ARGUMENT, "qg_decode_step_inspect: null offsets");
+  const StepLayout Ly = step_layout(*cfg, B, cap);
+  offsets[0] = Ly.xn;
+  offsets[1] = Ly.attn;
+  offsets[2] = Ly.xn2;
+  offsets[3] = Ly.h;
   return QG_OK;
 }
 

@@ -11,16 +11,16 @@
 //   * mma.sync m16n8k16, fp16 operands, fp32 accumulation. A is 16 rows of
 //     W: lane (g, t) loads 32 contiguous code bytes of row g and 32 of row
 //     g + 8 with one 256-bit load each. A code byte q becomes the fp16 value
-//     1024 + q with one byte permute per two codes (exact: fp16 has 11
-//     significant bits). The k order inside an mma is free (a dot product
+//     q - 128 with one byte permute and one packed subtract per two codes
+//     (exact: fp16 has 11 significant bits). The k order inside an mma is free (a dot product
 //     does not care), so k-slots {2t, 2t+1, 2t+8, 2t+9} of mma j are bytes
 //     4j .. 4j+3 of lane t's 32-byte piece.
 //   * B carries x with a group selector: column n = 2 b + h holds batch b's
 //     x on the k-slots of 64-column group h of the 128-column chunk and zero
 //     on the others. Lanes t = 0, 1 hold group 0 of a chunk and t = 2, 3
 //     group 1, so one mma leaves both groups' partial sums
-//     S_h = sum (1024 + q) x apart, for 16 rows and 4 batch rows, already
-//     reduced over the quad. Per group, y += s S + (beta - 1024 s) sum(x):
+//     S_h = sum (q - 128) x apart, for 16 rows and 4 batch rows, already
+//     reduced over the quad. Per group, y += s S + (beta + 128 s) sum(x):
 //     the affine factorisation; no cross-lane reduction at all.
 //   * x is converted once per CTA to fp16 in shared memory after a
 //     power-of-two prescale 2^-e chosen from max|x| (so nothing overflows
@@ -44,12 +44,9 @@
 namespace qg {
 namespace gtc {
 
-// warps per CTA: 16 with one batch tile (128 registers a thread), 8 with two
-template <int NT>
-struct Cfg {
-  static constexpr int kWarps = NT == 1 ? 16 : 8;
-  static constexpr int kThreads = kWarps * 32;
-};
+// Warps per CTA (template W): 16 with one batch tile (128 registers a
+// thread, the whole register file: the most loads in flight), 8 with two
+// batch tiles (about 255 registers a thread).
 constexpr int kRB = 16;        // rows per block (mma M)
 constexpr int kSC = 512;       // columns per super-chunk
 constexpr int kMaxSegs = 4;
@@ -80,6 +77,7 @@ struct Params {
   const float* xb;     // kXSiluMul
   const uint16_t* nw;  // kXRmsNorm weight, bf16 [K]
   float eps;
+  uint16_t* xout;      // optional: CTA 0 records the formed bf16 input [B][K]
 };
 
 __device__ __forceinline__ void ld_w8(const uint8_t* p, uint64_t pol, uint32_t* r) {
@@ -102,9 +100,22 @@ __device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1,
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
-// codes (0,1) and (2,3) of a word as fp16 pairs of 1024 + q
-__device__ __forceinline__ uint32_t codes01(uint32_t w) { return __byte_perm(w, 0x64646464u, 0x4140u); }
-__device__ __forceinline__ uint32_t codes23(uint32_t w) { return __byte_perm(w, 0x64646464u, 0x4342u); }
+// codes (0,1) and (2,3) of a word as fp16 pairs of q - 128: the byte
+// permute makes 1024 + q (fp16 0x6400 | q), one packed subtract of 1152
+// (0x6480) centres it; both steps are exact. Centred codes keep the fp32
+// partial sums of a group near sum (q - 128) x instead of carrying a
+// 1024 * sum(x) term, so their rounding error is that much smaller.
+__device__ __forceinline__ uint32_t centre(uint32_t h2) {
+  const __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&h2),
+                            __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480)));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+__device__ __forceinline__ uint32_t codes01(uint32_t w) {
+  return centre(__byte_perm(w, 0x64646464u, 0x4140u));
+}
+__device__ __forceinline__ uint32_t codes23(uint32_t w) {
+  return centre(__byte_perm(w, 0x64646464u, 0x4342u));
+}
 
 // which segment a global block index belongs to
 __device__ __forceinline__ int seg_of(const Params& P, int blk) {
@@ -166,10 +177,10 @@ __device__ __forceinline__ void chunk_mma(const uint32_t (&w)[16], const uint4& 
   mma_f16(d1, codes01(w[7]), codes01(w[15]), codes23(w[7]), codes23(w[15]), x3.z, x3.w);
 }
 
-template <int NT>
-__global__ void __launch_bounds__(Cfg<NT>::kThreads, 1)
+template <int NT, int W>
+__global__ void __launch_bounds__(W * 32, NT == 1 ? 512 / (W * 32) : 1)
     gemv_tc_kernel(const __grid_constant__ Params P) {
-  constexpr int kWarps = Cfg<NT>::kWarps, kThreads = Cfg<NT>::kThreads;
+  constexpr int kWarps = W, kThreads = W * 32;
   extern __shared__ __align__(16) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
@@ -204,6 +215,9 @@ __global__ void __launch_bounds__(Cfg<NT>::kThreads, 1)
     for (int p = 0; p < 4; ++p) load_chunk(lr, K, lsc, p, pol, wb[p]);
   }
 
+  // the next kernel may be scheduled now (its own wait still covers all of
+  // this one); only weights were read so far
+  pdl_trigger();
   pdl_wait();  // x (and residuals) are written by the previous kernel
   // 1) RMSNorm statistics per batch row (fixed summation order)
   float inv[4 * NT];
@@ -231,28 +245,49 @@ __global__ void __launch_bounds__(Cfg<NT>::kThreads, 1)
     }
     __syncthreads();
   }
-  // 2) the input values, rounded to bf16, into xh (as bf16 bits for now);
-  // batch rows past B are never read by a live B-operand lane
-  float mx = 0.f;
-  for (int i = tid; i < P.B * K; i += kThreads) {
-    const int b = i / K, c = i - b * K;
-    uint16_t h;
-    if (P.xmode == kXBf16) {
-      h = P.x[i];
-    } else if (P.xmode == kXRmsNorm) {
-      float ib = inv[0];
+  // 2) one warp per 64-column group: the input values, rounded to bf16, go
+  // to xh as fp16 and the group's fp16 sum to gsum. fp16 holds them exactly
+  // unless max|x| >= 2^15, checked after the pass; then (rarely) the pass is
+  // redone on x * 2^-e. Batch rows past B are never read by a live B lane.
+  auto form = [&](float down) -> float {
+    float mloc = 0.f;
+    for (int i = warp; i < P.B * Kg; i += kWarps) {
+      const int b = i / Kg, c = (i - b * Kg) * 64 + 2 * lane;
+      const size_t o = (size_t)b * K + c;
+      float v0, v1;
+      if (P.xmode == kXBf16) {
+        const uint32_t w2 = *reinterpret_cast<const uint32_t*>(P.x + o);
+        v0 = bf16_lo(w2);
+        v1 = bf16_hi(w2);
+      } else if (P.xmode == kXRmsNorm) {
+        float ib = inv[0];
 #pragma unroll
-      for (int j = 1; j < 4 * NT; ++j)
-        if (b == j) ib = inv[j];
-      h = f32_to_bf16_bits(P.xa[i] * ib * bf16_bits_to_f32(P.nw[c]));
-    } else {
-      const float z = P.xa[i];
-      h = f32_to_bf16_bits(z / (1.0f + expf(-z)) * P.xb[i]);
+        for (int j = 1; j < 4 * NT; ++j)
+          if (b == j) ib = inv[j];
+        const float2 xv = *reinterpret_cast<const float2*>(P.xa + o);
+        // (the norm weight may be only 2-byte aligned)
+        v0 = bf16_bits_to_f32(f32_to_bf16_bits(xv.x * ib * bf16_bits_to_f32(P.nw[c])));
+        v1 = bf16_bits_to_f32(f32_to_bf16_bits(xv.y * ib * bf16_bits_to_f32(P.nw[c + 1])));
+      } else {
+        const float2 z = *reinterpret_cast<const float2*>(P.xa + o);
+        const float2 u = *reinterpret_cast<const float2*>(P.xb + o);
+        v0 = bf16_bits_to_f32(f32_to_bf16_bits(z.x / (1.0f + expf(-z.x)) * u.x));
+        v1 = bf16_bits_to_f32(f32_to_bf16_bits(z.y / (1.0f + expf(-z.y)) * u.y));
+      }
+      mloc = fmaxf(mloc, fmaxf(fabsf(v0), fabsf(v1)));
+      if (P.xout && blockIdx.x == 0 && down == 1.0f)
+        *reinterpret_cast<uint32_t*>(P.xout + o) =
+            (uint32_t)f32_to_bf16_bits(v0) | ((uint32_t)f32_to_bf16_bits(v1) << 16);
+      const __half2 h2 = __floats2half2_rn(v0 * down, v1 * down);
+      *reinterpret_cast<__half2*>(xh + b * xs + c) = h2;
+      const float sum = warp_sum(__low2float(h2) + __high2float(h2));
+      if (lane == 0) gsum[i] = sum;
     }
-    mx = fmaxf(mx, fabsf(bf16_bits_to_f32(h)));
-    xh[b * xs + c] = h;
-  }
-  // 3) prescale 2^-e so that max|x| * 2^-e < 2^15 (fp16 max is 65504)
+    return mloc;
+  };
+  float mx = form(1.0f);
+  for (int i = P.B * Kg + tid; i < 4 * NT * Kg; i += kThreads) gsum[i] = 0.f;
+  // 3) max|x| over the CTA; prescale 2^-e so that max|x| * 2^-e < 2^15
   mx = warp_max(mx);
   if (lane == 0) red[warp] = mx;
   __syncthreads();
@@ -261,23 +296,9 @@ __global__ void __launch_bounds__(Cfg<NT>::kThreads, 1)
   for (int w = 0; w < kWarps; ++w) mx = fmaxf(mx, red[w]);
   int e = 0;  // NaN or inf in x propagate to y without a prescale
   if (mx >= 32768.f && mx <= 3.0e38f) e = (int)ceilf(log2f(mx / 16384.f));
-  const float down = exp2f((float)-e), up = exp2f((float)e);
-  // 4) bf16 -> fp16 in place (each thread converts the entries it wrote)
-  for (int i = tid; i < P.B * K; i += kThreads) {
-    const int b = i / K, c = i - b * K;
-    xh[b * xs + c] = __half_as_ushort(__float2half_rn(bf16_bits_to_f32(xh[b * xs + c]) * down));
-  }
-  __syncthreads();
-  // 5) per 64-column group sums of the fp16 values, one warp per group
-  // (lanes read consecutive words: no bank conflicts); zero past B
-  for (int i = warp; i < 4 * NT * Kg; i += kWarps) {
-    const int b = i / Kg, gg = i - b * Kg;
-    float sum = 0.f;
-    if (b < P.B) {
-      const __half2 v = *reinterpret_cast<const __half2*>(xh + b * xs + 64 * gg + 2 * lane);
-      sum = warp_sum(__low2float(v) + __high2float(v));
-    }
-    if (lane == 0) gsum[i] = sum;
+  const float up = exp2f((float)e);
+  if (e != 0) {  // uniform over the CTA
+    form(exp2f((float)-e));
   }
   __syncthreads();
 
@@ -313,10 +334,10 @@ __global__ void __launch_bounds__(Cfg<NT>::kThreads, 1)
       const uint32_t s1 = __shfl_sync(0xffffffffu, sv[1], src);
       const uint32_t b0 = __shfl_sync(0xffffffffu, sv[2], src);
       const uint32_t b1 = __shfl_sync(0xffffffffu, sv[3], src);
-      // (scale, bias - 1024 scale) of rows g, g+8 for groups A, B of the chunk
+      // (scale, bias + 128 scale) of rows g, g+8 for groups A, B of the chunk
       const float sA0 = bf16_lo(s0), sB0 = bf16_hi(s0), sA1 = bf16_lo(s1), sB1 = bf16_hi(s1);
-      const float cA0 = fmaf(-1024.f, sA0, bf16_lo(b0)), cB0 = fmaf(-1024.f, sB0, bf16_hi(b0));
-      const float cA1 = fmaf(-1024.f, sA1, bf16_lo(b1)), cB1 = fmaf(-1024.f, sB1, bf16_hi(b1));
+      const float cA0 = fmaf(128.f, sA0, bf16_lo(b0)), cB0 = fmaf(128.f, sB0, bf16_hi(b0));
+      const float cA1 = fmaf(128.f, sA1, bf16_lo(b1)), cB1 = fmaf(128.f, sB1, bf16_hi(b1));
       const int chunk = csc * 4 + p;
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
@@ -397,13 +418,11 @@ __global__ void __launch_bounds__(Cfg<NT>::kThreads, 1)
     cblk += T;
     ++nb;
   }
-  pdl_trigger();
 }
 
 }  // namespace gtc
 
-static size_t gtc_smem(int K, int NT) {
-  const int W = NT == 1 ? gtc::Cfg<1>::kWarps : gtc::Cfg<2>::kWarps;
+static size_t gtc_smem(int K, int NT, int W) {
   return (size_t)4 * NT * W * 4 + (size_t)2 * W * 32 * 2 * NT * 4 +
          (size_t)4 * NT * (K / 64) * 4 + (size_t)4 * NT * (K + 8) * 2;
 }
@@ -417,20 +436,19 @@ bool gemv_tc_eligible(const GemvSeg* segs, int nseg, int K, int B, bool x_f32) {
     return false;
   for (int i = 0; i < nseg; ++i)
     if (!aligned(segs[i].w, 32) || !aligned(segs[i].s, 4) || !aligned(segs[i].b, 4)) return false;
-  return gtc_smem(K, (B + 3) / 4) <= 200 * 1024;
+  return gtc_smem(K, (B + 3) / 4, 16) <= 200 * 1024;
 }
 
-template <int NT>
+template <int NT, int W>
 static cudaError_t gtc_launch_nt(const gtc::Params& P, int grid, cudaStream_t st, bool pdl) {
-  const size_t smem = gtc_smem(P.K, NT);
+  const size_t smem = gtc_smem(P.K, NT, W);
   static int attr = 0;
   if (smem > 48 * 1024 && attr < (int)smem) {
-    cudaFuncSetAttribute(gtc::gemv_tc_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(gtc::gemv_tc_kernel<NT, W>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          200 * 1024);
     attr = 200 * 1024;
   }
-  return launch_pdl(gtc::gemv_tc_kernel<NT>, dim3(grid), dim3(gtc::Cfg<NT>::kThreads), smem, st,
-                    pdl, P);
+  return launch_pdl(gtc::gemv_tc_kernel<NT, W>, dim3(grid), dim3(W * 32), smem, st, pdl, P);
 }
 
 static cudaError_t gtc_launch(const GemvSeg* segs, int nseg, gtc::Params& P, int K, int B,
@@ -446,16 +464,18 @@ static cudaError_t gtc_launch(const GemvSeg* segs, int nseg, gtc::Params& P, int
   }
   P.nblocks = blk;
   if (blk == 0) return cudaSuccess;
-  // split each block's columns over S warps while that leaves warp slots idle
+  // 16 warps with one batch tile, 8 with two (measured: 16 is faster also
+  // for the small matrices of a decode step); then split each block's
+  // columns over S warps while slots stay idle
   const int NT = (B + 3) / 4;
-  const int W = NT == 1 ? gtc::Cfg<1>::kWarps : gtc::Cfg<2>::kWarps;
   const int sms = num_sms(), nsc = K / gtc::kSC;
+  const int W = NT == 1 ? 16 : 8;
   int S = 1;
   while (S < W && 2 * S <= nsc && (long long)blk * S < (long long)sms * W) S *= 2;
   P.S = S;
   const int grid = std::min(sms, blk);
-  if (NT == 1) return gtc_launch_nt<1>(P, grid, st, pdl);
-  return gtc_launch_nt<2>(P, grid, st, pdl);
+  if (NT == 2) return gtc_launch_nt<2, 8>(P, grid, st, pdl);
+  return gtc_launch_nt<1, 16>(P, grid, st, pdl);
 }
 
 cudaError_t gemv_tc_launch(const GemvSeg* segs, int nseg, const void* x, int K, int B,
@@ -468,9 +488,10 @@ cudaError_t gemv_tc_launch(const GemvSeg* segs, int nseg, const void* x, int K, 
 
 cudaError_t gemv_tc_launch_rmsnorm(const GemvSeg* segs, int nseg, const float* x,
                                    const uint16_t* norm_w, float eps, int K, int B,
-                                   cudaStream_t st, bool pdl) {
+                                   cudaStream_t st, bool pdl, uint16_t* xout) {
   gtc::Params P = {};
   P.xmode = gtc::kXRmsNorm;
+  P.xout = xout;
   P.xa = x;
   P.nw = norm_w;
   P.eps = eps;
@@ -478,9 +499,11 @@ cudaError_t gemv_tc_launch_rmsnorm(const GemvSeg* segs, int nseg, const float* x
 }
 
 cudaError_t gemv_tc_launch_silu_mul(const GemvSeg* segs, int nseg, const float* gate,
-                                    const float* up, int K, int B, cudaStream_t st, bool pdl) {
+                                    const float* up, int K, int B, cudaStream_t st, bool pdl,
+                                    uint16_t* xout) {
   gtc::Params P = {};
   P.xmode = gtc::kXSiluMul;
+  P.xout = xout;
   P.xa = gate;
   P.xb = up;
   return gtc_launch(segs, nseg, P, K, B, st, pdl);

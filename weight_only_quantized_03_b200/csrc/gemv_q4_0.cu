@@ -105,9 +105,122 @@ gemv_q4_0_kernel(const uint8_t* __restrict__ blocks, const float* __restrict__ x
     }
 }
 
+// Staged variant (rows 16-byte aligned: K % 256 == 0 and an aligned base):
+// the CTA's 8*R rows are copied to shared memory first with coalesced
+// 16-byte streaming loads, all in flight at once and issued before waiting
+// for the previous kernel (weights never depend on it); then each warp forms
+// its R rows from shared memory exactly as above.
+template <int NB, int R>
+__global__ void __launch_bounds__(kQ4Warps * 32)
+gemv_q4_0_staged_kernel(const uint8_t* __restrict__ blocks, const float* __restrict__ x,
+                        const float* __restrict__ bias, float* __restrict__ y, int N, int K, int B) {
+  extern __shared__ __align__(16) uint8_t tile[];
+  constexpr int RT = kQ4Warps * R;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r0 = blockIdx.x * RT;
+  const int nrows = min(RT, N - r0);
+  const int nb = K >> 5;
+  const size_t rowbytes = (size_t)nb * 18;
+  const uint64_t pol = l2_evict_first_policy();
+  const uint4* src = reinterpret_cast<const uint4*>(blocks + (size_t)r0 * rowbytes);
+  uint4* dst = reinterpret_cast<uint4*>(tile);
+  const int n16 = (int)((size_t)nrows * rowbytes / 16);
+  for (int base = threadIdx.x; base < n16; base += blockDim.x * 8) {
+    uint4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = base + u * blockDim.x;
+      if (i < n16) v[u] = ld_stream_u4(src + i, pol);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = base + u * blockDim.x;
+      if (i < n16) dst[i] = v[u];
+    }
+  }
+  __syncthreads();
+  pdl_wait();  // x and bias may be written by the previous kernel
+  float acc[R][NB];
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int b = 0; b < NB; ++b) acc[r][b] = 0.f;
+  for (int j = lane; j < nb; j += 32) {
+    Q4Block blk[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int lr = min(warp * R + r, nrows - 1);
+      const uint16_t* h = reinterpret_cast<const uint16_t*>(tile + lr * rowbytes + (size_t)j * 18);
+      blk[r].d = __half2float(__ushort_as_half(h[0]));
+#pragma unroll
+      for (int i = 0; i < 4; ++i) blk[r].q[i] = (uint32_t)h[1 + 2 * i] | ((uint32_t)h[2 + 2 * i] << 16);
+    }
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      if (b < B) {
+        float xv[32];
+        const float4* xp = reinterpret_cast<const float4*>(x + (size_t)b * K + 32 * j);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float4 t = __ldg(xp + i);
+          xv[4 * i] = t.x; xv[4 * i + 1] = t.y; xv[4 * i + 2] = t.z; xv[4 * i + 3] = t.w;
+        }
+#pragma unroll
+        for (int r = 0; r < R; ++r) acc[r][b] = fmaf(blk[r].d, q4_dot(blk[r], xv), acc[r][b]);
+      }
+    }
+  }
+  pdl_trigger();
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int b = 0; b < NB; ++b) acc[r][b] = warp_sum(acc[r][b]);
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      const int row = r0 + warp * R + r;
+      if (lane == ((r * NB + b) & 31) && warp * R + r < nrows && b < B)
+        y[(size_t)b * N + row] = acc[r][b] + (bias ? bias[row] : 0.f);
+    }
+}
+
+constexpr size_t kQ4StagedSmem = 96 * 1024;
+
+template <int NB, int R>
+static cudaError_t q4_staged_launch_r(const uint8_t* blocks, const float* x, const float* bias,
+                                      float* y, int N, int K, int B, cudaStream_t st, bool pdl) {
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(gemv_q4_0_staged_kernel<NB, R>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kQ4StagedSmem);
+    attr = true;
+  }
+  constexpr int RT = kQ4Warps * R;
+  const size_t smem = (size_t)RT * (K / 32) * 18;
+  return launch_pdl(gemv_q4_0_staged_kernel<NB, R>, dim3((N + RT - 1) / RT),
+                    dim3(kQ4Warps * 32), smem, st, pdl, blocks, x, bias, y, N, K, B);
+}
+
+// rows per warp: as many as keep about one CTA per SM busy and the tile in
+// shared memory
+template <int NB>
+static cudaError_t q4_staged_launch(const uint8_t* blocks, const float* x, const float* bias,
+                                    float* y, int N, int K, int B, cudaStream_t st, bool pdl) {
+  const size_t rowbytes = (size_t)(K / 32) * 18;
+  const int sms = num_sms();
+  if ((long long)N >= 4LL * kQ4Warps * sms && 4 * kQ4Warps * rowbytes <= kQ4StagedSmem)
+    return q4_staged_launch_r<NB, 4>(blocks, x, bias, y, N, K, B, st, pdl);
+  if ((long long)N >= 2LL * kQ4Warps * sms && 2 * kQ4Warps * rowbytes <= kQ4StagedSmem)
+    return q4_staged_launch_r<NB, 2>(blocks, x, bias, y, N, K, B, st, pdl);
+  return q4_staged_launch_r<NB, 1>(blocks, x, bias, y, N, K, B, st, pdl);
+}
+
 template <int NB>
 static cudaError_t q4_launch(const uint8_t* blocks, const float* x, const float* bias, float* y,
                              int N, int K, int B, cudaStream_t st, bool pdl) {
+  if (K % 256 == 0 && aligned(blocks, 16) && (size_t)kQ4Warps * (K / 32) * 18 <= kQ4StagedSmem)
+    return q4_staged_launch<NB>(blocks, x, bias, y, N, K, B, st, pdl);
   const int R = 4;
   const int grid = (N + kQ4Warps * R - 1) / (kQ4Warps * R);
   return launch_pdl(gemv_q4_0_kernel<NB, R>, dim3(grid), dim3(kQ4Warps * 32), 0, st, pdl, blocks,

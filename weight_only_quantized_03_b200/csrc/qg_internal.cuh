@@ -153,12 +153,14 @@ cudaError_t gemv_tc_launch(const GemvSeg* segs, int nseg, const void* x, int K, 
                            cudaStream_t st, bool pdl);
 // The same GEMV with its input formed in the prologue: bf16(RMSNorm(x) * w)
 // of fp32 x [B][K], or bf16(silu(gate) * up) of fp32 [B][K] (eligibility as
-// gemv_tc_eligible with x_f32 = false).
+// gemv_tc_eligible with x_f32 = false). When xout is not null the formed
+// bf16 input is also written there ([B][K], by one CTA).
 cudaError_t gemv_tc_launch_rmsnorm(const GemvSeg* segs, int nseg, const float* x,
                                    const uint16_t* norm_w, float eps, int K, int B,
-                                   cudaStream_t st, bool pdl);
+                                   cudaStream_t st, bool pdl, uint16_t* xout = nullptr);
 cudaError_t gemv_tc_launch_silu_mul(const GemvSeg* segs, int nseg, const float* gate,
-                                    const float* up, int K, int B, cudaStream_t st, bool pdl);
+                                    const float* up, int K, int B, cudaStream_t st, bool pdl,
+                                    uint16_t* xout = nullptr);
 
 cudaError_t rmsnorm_launch(const float* x, const uint16_t* w, float eps, void* y,
                            bool y_bf16, int rows, int dim, cudaStream_t st, bool pdl);
@@ -169,11 +171,12 @@ cudaError_t attention_launch(const float* q, const uint16_t* kc, const uint16_t*
                              int cap, float scale, void* ws, cudaStream_t st, bool pdl);
 
 // The decode step's attention: q/k per-head RMSNorm, NeoX RoPE at
-// positions[b] and the K/V append at row positions[b] done inside the
-// attention kernel (raw fp32 q, k, v in), output bf16 [B][H][D]. D <= 256.
+// positions[b] (the (cos, sin) table [B][D/2] of the step) and the K/V
+// append at row positions[b] done inside the attention kernel (raw fp32 q,
+// k, v in), output bf16 [B][H][D]. D <= 256.
 cudaError_t attention_launch_step(const float* q, const float* k, const float* v,
                                   const uint16_t* q_norm, const uint16_t* k_norm,
-                                  const int32_t* tokens, int vocab, float eps, double theta,
+                                  const int32_t* tokens, int vocab, float eps, const float2* rope,
                                   uint16_t* kc, uint16_t* vc, const int32_t* positions, void* out,
                                   int B, int H, int Hkv, int D, int cap, float scale, void* ws,
                                   cudaStream_t st, bool pdl);
