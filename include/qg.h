@@ -293,6 +293,14 @@ size_t qg_decode_step_workspace_size(const qg_qwen3_config* cfg, int B, int cap)
  * written at cache row positions[b] -> attention over rows
  * [0, positions[b]] -> o_proj + residual -> RMSNorm -> gate, up -> SiLU-mul
  * -> down + residual); then the final RMSNorm and the tied LM head.
+ * Execution: one launch per fused stage, chained with Programmatic Dependent
+ * Launch (each GEMV streams its first weights while the previous kernel
+ * finishes): the embedding, then per layer the q/k/v GEMV (input RMSNorm in
+ * its prologue), attention (q/k norm, RoPE and the K/V append fused), o_proj
+ * + residual, the gate/up GEMV (post-attention RMSNorm in its prologue), the
+ * down GEMV (SiLU-mul in its prologue) + residual, then the LM head (final
+ * RMSNorm in its prologue): 5 launches per layer plus 2. Nothing
+ * synchronises or allocates, so a step can be captured in a CUDA graph.
  *
  * cfg, w      HOST structs (read during the call only).
  * k_cache, v_cache device bf16 [layers][B][kv_heads][cap][head_dim].
@@ -301,13 +309,12 @@ size_t qg_decode_step_workspace_size(const qg_qwen3_config* cfg, int B, int cap)
  *             gets NaN logits and its cache is not written.
  * logits      device fp32 [B][vocab].
  * ws          device workspace >= qg_decode_step_workspace_size(cfg,B,cap)
- *             bytes, 256-byte aligned, ZERO-FILLED before its first use (and
- *             again if it was used for anything else in between): it carries
- *             a step counter from one call to the next, which tags the data
- *             the persistent kernel's CTAs exchange. Use one workspace per
- *             stream at a time. On return its first B*hidden*4 bytes hold the
- *             residual stream after the last layer (fp32 [B][hidden], before
- *             the final norm).
+ *             bytes, 256-byte aligned; no initialisation needed (each step
+ *             clears the attention counters with one small memset on
+ *             `stream`).
+ *             Use one workspace per stream at a time. On return its first
+ *             B*hidden*4 bytes hold the residual stream after the last layer
+ *             (fp32 [B][hidden], before the final norm).
  * Precision: residual stream, q/k/v and gate/up outputs and logits fp32;
  * norm outputs feeding a GEMV, cached K/V, attention output and SiLU-mul
  * output bf16.
@@ -320,49 +327,13 @@ qg_status qg_decode_step(const qg_qwen3_config* cfg, const qg_qwen3_weights* w,
                          float* logits, int B, void* ws, size_t ws_bytes,
                          void* stream);
 
-/* qg_decode_step with option flags. By default the step runs kernel-per-op
- * (one launch per fused GEMV / attention stage, chained with Programmatic
- * Dependent Launch; 5 launches per layer plus the embedding and the LM
- * head). QG_STEP_PERSISTENT asks for the persistent one-launch kernel
- * instead, which runs whenever the shapes allow it (B <= 4; hidden,
- * heads*head_dim and ffn multiples of 512 and <= 16384; head_dim 64 or 128;
- * layers <= 64; 16-byte aligned scales and biases) and falls back to the
- * kernel-per-op path otherwise. QG_STEP_MULTI_KERNEL forces the
- * kernel-per-op path (it overrides QG_STEP_PERSISTENT). Both paths compute
- * the same operations with the same precision points. */
-#define QG_STEP_MULTI_KERNEL 1u
-#define QG_STEP_PERSISTENT 2u
-/* Test hook for the persistent kernel (with QG_STEP_PERSISTENT): one
- * device-side wait targets a
- * counter that nothing sets, so it gives up after its 1 s bound and the
- * step records an error word (read it with qg_decode_step_error). The
- * step's outputs are then undefined; the context stays usable. */
-#define QG_STEP_TEST_STALL 0x80000000u
-/* Profiling aid for the persistent kernel: thread 0 of every CTA writes
- * %globaltimer stamps (ns, uint64) at each phase boundary into the
- * workspace region that qg_decode_step_trace_offset() locates, laid out
- * [CTA][layer (last slot: LM head)][16 events]. */
-#define QG_STEP_TRACE 0x40000000u
-size_t qg_decode_step_trace_offset(const qg_qwen3_config* cfg, int B, int cap);
-/* Inspection aid for the kernel-per-op path (tests): byte offsets in the
- * workspace of four bf16 arrays that, after a step, hold the LAST decoder
- * layer's values at its bf16 rounding points: offsets[0] the input-norm
- * output [B][hidden], offsets[1] the attention output [B][heads*head_dim],
- * offsets[2] the post-attention-norm output [B][hidden], offsets[3] the
- * SiLU-mul output [B][ffn]. (The persistent kernel does not write them.) */
+/* Inspection aid (tests): byte offsets in the workspace of four bf16 arrays
+ * that, after a step, hold the LAST decoder layer's values at its bf16
+ * rounding points: offsets[0] the input-norm output [B][hidden], offsets[1]
+ * the attention output [B][heads*head_dim], offsets[2] the
+ * post-attention-norm output [B][hidden], offsets[3] the SiLU-mul output
+ * [B][ffn]. */
 qg_status qg_decode_step_inspect(const qg_qwen3_config* cfg, int B, int cap, size_t offsets[4]);
-qg_status qg_decode_step_ex(const qg_qwen3_config* cfg, const qg_qwen3_weights* w,
-                            uint16_t* k_cache, uint16_t* v_cache, int cap,
-                            const int32_t* tokens, const int32_t* positions,
-                            float* logits, int B, void* ws, size_t ws_bytes,
-                            unsigned flags, void* stream);
-
-/* Reads the device error word of the last step that used `ws` (this call
- * synchronises `stream`). The persistent kernel bounds every device-side
- * wait; a wait that gives up records a nonzero code, the kernel leaves, and
- * this call then returns QG_ERR_TIMEOUT with the code in *code. */
-qg_status qg_decode_step_error(const qg_qwen3_config* cfg, int B, int cap,
-                               const void* ws, unsigned* code, void* stream);
 
 /* ------------------------------------------------------------------------
  * Test exports: the unpack and dequant the kernels use, written out.

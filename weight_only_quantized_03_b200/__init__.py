@@ -31,10 +31,6 @@ QG_ERR_CUDA = 5
 QG_ERR_TIMEOUT = 6
 QG_F32 = 0
 QG_BF16 = 1
-QG_STEP_MULTI_KERNEL = 1
-QG_STEP_PERSISTENT = 2
-QG_STEP_TEST_STALL = 0x80000000
-QG_STEP_TRACE = 0x40000000
 
 _vp = ctypes.c_void_p
 _i = ctypes.c_int
@@ -92,11 +88,6 @@ _SIGS = {
     "qg_decode_step_workspace_size": (_sz, [ctypes.POINTER(qg_qwen3_config), _i, _i]),
     "qg_decode_step": (_i, [ctypes.POINTER(qg_qwen3_config), ctypes.POINTER(qg_qwen3_weights),
                             _vp, _vp, _i, _vp, _vp, _vp, _i, _vp, _sz, _vp]),
-    "qg_decode_step_ex": (_i, [ctypes.POINTER(qg_qwen3_config), ctypes.POINTER(qg_qwen3_weights),
-                               _vp, _vp, _i, _vp, _vp, _vp, _i, _vp, _sz, ctypes.c_uint, _vp]),
-    "qg_decode_step_error": (_i, [ctypes.POINTER(qg_qwen3_config), _i, _i, _vp,
-                                  ctypes.POINTER(ctypes.c_uint), _vp]),
-    "qg_decode_step_trace_offset": (_sz, [ctypes.POINTER(qg_qwen3_config), _i, _i]),
     "qg_decode_step_inspect": (_i, [ctypes.POINTER(qg_qwen3_config), _i, _i,
                                     ctypes.POINTER(ctypes.c_size_t)]),
     "qg_unpack_affine8": (_i, [_vp, _vp, _i, _i, _vp]),
@@ -288,7 +279,7 @@ class Qwen3Model:
 
     def new_state(self, B, cap):
         """Zeroed KV caches [layers, B, kv_heads, cap, head_dim] bf16, a
-        zero-filled workspace (required before its first use) and a logits
+        workspace and a logits
         buffer for batch B."""
         c = self.cfg
         shape = (c["layers"], B, c["kv_heads"], cap, c["head_dim"])
@@ -319,21 +310,14 @@ class Qwen3Model:
         return {"xn": view(off[0], c["hidden"]), "attn": view(off[1], c["heads"] * c["head_dim"]),
                 "xn2": view(off[2], c["hidden"]), "h": view(off[3], c["ffn"])}
 
-    def qg_decode_step_error(self, state, stream=None):
-        """Device error word of the latest step (synchronises the stream)."""
-        code = ctypes.c_uint(0)
-        st = lib.qg_decode_step_error(ctypes.byref(self.c_cfg), state["B"], state["cap"],
-                                      _p(state["ws"]), ctypes.byref(code), _stream(stream))
-        return st, code.value
-
-    def qg_decode_step(self, state, tokens, positions, stream=None, layers=None, flags=0):
+    def qg_decode_step(self, state, tokens, positions, stream=None, layers=None):
         """tokens, positions: device int32 [B]. Writes state['logits'].
         ``layers`` runs only the first that many layers (then the head)."""
         cfg = self.c_cfg
         if layers is not None:
             cfg = qg_qwen3_config.from_buffer_copy(self.c_cfg)
             cfg.layers = layers
-        _call("qg_decode_step_ex", ctypes.byref(cfg), ctypes.byref(self.c_weights),
+        _call("qg_decode_step", ctypes.byref(cfg), ctypes.byref(self.c_weights),
               _p(state["k_cache"]), _p(state["v_cache"]), state["cap"], _p(tokens),
               _p(positions), _p(state["logits"]), state["B"], _p(state["ws"]),
-              state["ws"].numel(), flags, _stream(stream))
+              state["ws"].numel(), _stream(stream))

@@ -18,7 +18,7 @@ namespace qg {
 size_t attention_ws_counter_offset(int B, int H, int Hkv, int D, int cap);
 
 struct StepLayout {
-  size_t x, xn, xn2, xnf, q, k, v, attn, gate, up, h, attn_ws, rope, mx, cnt, step, trace, total;
+  size_t x, xn, xn2, xnf, q, k, v, attn, gate, up, h, attn_ws, rope, total;
 };
 
 static size_t a256(size_t v) { return (v + 255) & ~(size_t)255; }
@@ -28,11 +28,8 @@ static StepLayout step_layout(const qg_qwen3_config& c, int B, int cap) {
   size_t off = 0;
   auto take = [&](size_t bytes) { size_t o = off; off += a256(bytes); return o; };
   const size_t qd = (size_t)c.heads * c.head_dim, kd = (size_t)c.kv_heads * c.head_dim;
-  // fixed head of the workspace (offsets independent of the layer count):
-  // the residual stream, the counters and the persistent step counter
+  // the residual stream heads the workspace
   L.x = take((size_t)B * c.hidden * 4);
-  L.cnt = take(64);
-  L.step = take(64);
   L.xn = take((size_t)B * c.hidden * 2);
   L.xn2 = take((size_t)B * c.hidden * 2);
   L.xnf = take((size_t)B * c.hidden * 2);
@@ -45,8 +42,6 @@ static StepLayout step_layout(const qg_qwen3_config& c, int B, int cap) {
   L.h = take((size_t)B * c.ffn * 2);
   L.attn_ws = take(attention_ws_bytes(B, c.heads, c.kv_heads, c.head_dim, cap));
   L.rope = take((size_t)B * (c.head_dim / 2) * 8);
-  L.mx = take(mega_ws_bytes(c, B, cap));
-  L.trace = take((size_t)num_sms() * ((c.layers + 1) * 16 + 1024) * 8);
   L.total = off;
   return L;
 }
@@ -139,32 +134,10 @@ extern "C" size_t qg_decode_step_workspace_size(const qg_qwen3_config* cfg, int 
   return step_layout(*cfg, B, cap).total;
 }
 
-static bool mega_pointers_ok(const qg_qwen3_config& c, const qg_qwen3_weights* w) {
-  auto ok = [](const qg_affine8_matrix& m) {
-    return aligned(m.w, 16) && aligned(m.scales, 16) && aligned(m.biases, 16);
-  };
-  if (!ok(w->embed)) return false;
-  for (int l = 0; l < c.layers; ++l) {
-    const qg_qwen3_layer& L = w->layers[l];
-    if (!ok(L.q) || !ok(L.k) || !ok(L.v) || !ok(L.o) || !ok(L.gate) || !ok(L.up) || !ok(L.down))
-      return false;
-  }
-  return true;
-}
-
 extern "C" qg_status qg_decode_step(const qg_qwen3_config* cfg, const qg_qwen3_weights* w,
                                     uint16_t* k_cache, uint16_t* v_cache, int cap,
                                     const int32_t* tokens, const int32_t* positions, float* logits,
                                     int B, void* ws, size_t ws_bytes, void* stream) {
-  return qg_decode_step_ex(cfg, w, k_cache, v_cache, cap, tokens, positions, logits, B, ws,
-                           ws_bytes, 0u, stream);
-}
-
-extern "C" qg_status qg_decode_step_ex(const qg_qwen3_config* cfg, const qg_qwen3_weights* w,
-                                       uint16_t* k_cache, uint16_t* v_cache, int cap,
-                                       const int32_t* tokens, const int32_t* positions,
-                                       float* logits, int B, void* ws, size_t ws_bytes,
-                                       unsigned flags, void* stream) {
   clear_error();
   qg_status st = validate_cfg(cfg, B, cap);
   if (st != QG_OK) return st;
@@ -216,18 +189,6 @@ extern "C" qg_status qg_decode_step_ex(const qg_qwen3_config* cfg, const qg_qwen
   const size_t layer_cache = (size_t)B * Hkv * cap * D;
   const float scale = 1.0f / sqrtf((float)D);
 
-  if ((flags & QG_STEP_PERSISTENT) && !(flags & QG_STEP_MULTI_KERNEL) && c.layers >= 1 &&
-      mega_eligible(c, B, cap) &&
-      mega_pointers_ok(c, w)) {
-    mega_launch(c, *w, k_cache, v_cache, cap, tokens, positions, logits, B, x, base + Ly.mx,
-                reinterpret_cast<unsigned*>(base + Ly.cnt), reinterpret_cast<unsigned*>(base + Ly.step),
-                (flags & QG_STEP_TEST_STALL) != 0,
-                (flags & QG_STEP_TRACE) ? reinterpret_cast<unsigned long long*>(base + Ly.trace)
-                                        : nullptr,
-                s);
-    return check_launch("qg_decode_step");
-  }
-  cudaMemsetAsync(reinterpret_cast<uint8_t*>(base + Ly.cnt), 0, 64, s);
   cudaMemsetAsync(reinterpret_cast<uint8_t*>(aws) + cnt_off, 0, (size_t)B * Hkv * 4, s);
   float2* rope = reinterpret_cast<float2*>(base + Ly.rope);
   launch_pdl(step_embed_kernel, dim3(B), dim3(256), 0, s, true, w->embed.w, w->embed.scales,
@@ -279,28 +240,6 @@ extern "C" qg_status qg_decode_step_ex(const qg_qwen3_config* cfg, const qg_qwen
   return check_launch("qg_decode_step");
 }
 
-extern "C" qg_status qg_decode_step_error(const qg_qwen3_config* cfg, int B, int cap,
-                                          const void* ws, unsigned* code, void* stream) {
-  clear_error();
-  qg_status st = validate_cfg(cfg, B, cap);
-  if (st != QG_OK) return st;
-  QG_REQUIRE(ws && code, QG_ERR_INVALID_ARGUMENT, "qg_decode_step_error: null ws or code");
-  const StepLayout Ly = step_layout(*cfg, B, cap);
-  cudaStream_t s = (cudaStream_t)stream;
-  cudaError_t e = cudaMemcpyAsync(code, reinterpret_cast<const uint8_t*>(ws) + Ly.cnt,
-                                  sizeof(unsigned), cudaMemcpyDeviceToHost, s);
-  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
-  if (e != cudaSuccess) {
-    set_error("qg_decode_step_error: %s", cudaGetErrorString(e));
-    return QG_ERR_CUDA;
-  }
-  if (*code != 0) {
-    set_error("qg_decode_step: a device-side wait gave up (code 0x%x)", *code);
-    return QG_ERR_TIMEOUT;
-  }
-  return QG_OK;
-}
-
 extern "C" qg_status qg_decode_step_inspect(const qg_qwen3_config* cfg, int B, int cap,
                                            size_t offsets[4]) {
   clear_error();
@@ -313,9 +252,4 @@ extern "C" qg_status qg_decode_step_inspect(const qg_qwen3_config* cfg, int B, i
   offsets[2] = Ly.xn2;
   offsets[3] = Ly.h;
   return QG_OK;
-}
-
-extern "C" size_t qg_decode_step_trace_offset(const qg_qwen3_config* cfg, int B, int cap) {
-  if (!cfg || B < 1 || cap < 1 || cfg->heads < 1 || cfg->kv_heads < 1) return 0;
-  return step_layout(*cfg, B, cap).trace;
 }

@@ -39,393 +39,25 @@
 //     (g, p) by shuffle.
 #include <algorithm>
 
-#include "qg_internal.cuh"
+#include "gemv_tc.cuh"
 
 namespace qg {
 namespace gtc {
 
-// Warps per CTA (template W): 16 with one batch tile (128 registers a
-// thread, the whole register file: the most loads in flight), 8 with two
-// batch tiles (about 255 registers a thread).
-constexpr int kRB = 16;        // rows per block (mma M)
-constexpr int kSC = 512;       // columns per super-chunk
-constexpr int kMaxSegs = 4;
-constexpr int kMaxB = 8;       // two n-tiles of four batch rows
-
-struct Seg {
-  const uint8_t* w;
-  const uint16_t* s;
-  const uint16_t* b;
-  void* y;
-  const float* res;
-  int N;
-  int y_bf16;
-  int blk0;  // first global block index of this segment
-};
-
-// How the GEMV input is formed in the prologue (every CTA forms all of it):
-//   kXBf16     x bf16 [B][K] as given;
-//   kXRmsNorm  bf16(xa / sqrt(mean(xa^2) + eps) * nw) per batch row, xa fp32;
-//   kXSiluMul  bf16(silu(xa) * xb), xa = gate and xb = up, both fp32.
-enum XMode { kXBf16 = 0, kXRmsNorm = 1, kXSiluMul = 2 };
-
-struct Params {
-  Seg seg[kMaxSegs];
-  int nseg, K, B, nblocks, S, xmode;
-  const uint16_t* x;   // kXBf16
-  const float* xa;     // kXRmsNorm, kXSiluMul
-  const float* xb;     // kXSiluMul
-  const uint16_t* nw;  // kXRmsNorm weight, bf16 [K]
-  float eps;
-  uint16_t* xout;      // optional: CTA 0 records the formed bf16 input [B][K]
-};
-
-__device__ __forceinline__ void ld_w8(const uint8_t* p, uint64_t pol, uint32_t* r) {
-  asm volatile(
-      "ld.global.nc.L1::no_allocate.L2::cache_hint.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8], %9;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7])
-      : "l"(p), "l"(pol));
-}
-__device__ __forceinline__ uint32_t ld_u32_nc(const uint16_t* p) {
-  uint32_t v;
-  asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
-  return v;
-}
-__device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                        uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-// codes (0,1) and (2,3) of a word as fp16 pairs of q - 128: the byte
-// permute makes 1024 + q (fp16 0x6400 | q), one packed subtract of 1152
-// (0x6480) centres it; both steps are exact. Centred codes keep the fp32
-// partial sums of a group near sum (q - 128) x instead of carrying a
-// 1024 * sum(x) term, so their rounding error is that much smaller.
-__device__ __forceinline__ uint32_t centre(uint32_t h2) {
-  const __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&h2),
-                            __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480)));
-  return *reinterpret_cast<const uint32_t*>(&r);
-}
-__device__ __forceinline__ uint32_t codes01(uint32_t w) {
-  return centre(__byte_perm(w, 0x64646464u, 0x4140u));
-}
-__device__ __forceinline__ uint32_t codes23(uint32_t w) {
-  return centre(__byte_perm(w, 0x64646464u, 0x4342u));
-}
-
-// which segment a global block index belongs to
-__device__ __forceinline__ int seg_of(const Params& P, int blk) {
-  int si = 0;
-#pragma unroll
-  for (int i = 1; i < kMaxSegs; ++i)
-    if (i < P.nseg && blk >= P.seg[i].blk0) si = i;
-  return si;
-}
-
-// Per-lane pointers into one 16-row block: rows g and g + 8 (clamped to the
-// matrix; rows past N are loaded but never stored). dr = row distance.
-struct Rows {
-  const uint8_t* w;
-  const uint16_t* s;
-  const uint16_t* b;
-  int dr;
-};
-
-__device__ __forceinline__ Rows rows_of(const Params& P, int blk, int g, int t) {
-  const Seg& S = P.seg[seg_of(P, blk)];
-  const int row0 = (blk - S.blk0) * kRB;
-  const int r0 = min(row0 + g, S.N - 1), r1 = min(row0 + g + 8, S.N - 1);
-  const int K = P.K, Kg = K / 64;
-  Rows R;
-  R.w = S.w + (size_t)r0 * K + 32 * t;
-  R.s = S.s + (size_t)r0 * Kg + 2 * t;
-  R.b = S.b + (size_t)r0 * Kg + 2 * t;
-  R.dr = r1 - r0;
-  return R;
-}
-
-__device__ __forceinline__ void load_scales(const Rows& R, int Kg, int sc, uint32_t (&v)[4]) {
-  const int o1 = R.dr * Kg + sc * 8;
-  v[0] = ld_u32_nc(R.s + sc * 8);
-  v[1] = ld_u32_nc(R.s + o1);
-  v[2] = ld_u32_nc(R.b + sc * 8);
-  v[3] = ld_u32_nc(R.b + o1);
-}
-__device__ __forceinline__ void load_chunk(const Rows& R, int K, int sc, int p, uint64_t pol,
-                                           uint32_t (&w)[16]) {
-  const uint8_t* a = R.w + sc * kSC + p * 128;
-  ld_w8(a, pol, w);
-  ld_w8(a + (size_t)R.dr * K, pol, w + 8);
-}
-
-// 8 mma of one 128-column chunk: two chains, A from the code words of rows
-// g (w[0..7]) and g + 8 (w[8..15]), B from x words xa (mma 0..3), xb (4..7)
-__device__ __forceinline__ void chunk_mma(const uint32_t (&w)[16], const uint4& x0, const uint4& x1,
-                                          const uint4& x2, const uint4& x3, float (&d0)[4],
-                                          float (&d1)[4]) {
-  mma_f16(d0, codes01(w[0]), codes01(w[8]), codes23(w[0]), codes23(w[8]), x0.x, x0.y);
-  mma_f16(d1, codes01(w[1]), codes01(w[9]), codes23(w[1]), codes23(w[9]), x0.z, x0.w);
-  mma_f16(d0, codes01(w[2]), codes01(w[10]), codes23(w[2]), codes23(w[10]), x1.x, x1.y);
-  mma_f16(d1, codes01(w[3]), codes01(w[11]), codes23(w[3]), codes23(w[11]), x1.z, x1.w);
-  mma_f16(d0, codes01(w[4]), codes01(w[12]), codes23(w[4]), codes23(w[12]), x2.x, x2.y);
-  mma_f16(d1, codes01(w[5]), codes01(w[13]), codes23(w[5]), codes23(w[13]), x2.z, x2.w);
-  mma_f16(d0, codes01(w[6]), codes01(w[14]), codes23(w[6]), codes23(w[14]), x3.x, x3.y);
-  mma_f16(d1, codes01(w[7]), codes01(w[15]), codes23(w[7]), codes23(w[15]), x3.z, x3.w);
-}
-
 template <int NT, int W>
 __global__ void __launch_bounds__(W * 32, NT == 1 ? 512 / (W * 32) : 1)
     gemv_tc_kernel(const __grid_constant__ Params P) {
-  constexpr int kWarps = W, kThreads = W * 32;
   extern __shared__ __align__(16) uint8_t smem[];
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g = lane >> 2, t = lane & 3;
-  const int K = P.K, Kg = K / 64, nsc = K / kSC, S = P.S;
-  const int xs = K + 8;  // fp16 row stride of x (pad: batch rows on other banks)
-  float* red = reinterpret_cast<float*>(smem);                      // [4 NT][kWarps]
-  float* part = red + 4 * NT * kWarps;                               // [2][kWarps][32][2 NT]
-  float* gsum = part + 2 * kWarps * 32 * 2 * NT;                    // [4 NT][Kg]
-  uint16_t* xh = reinterpret_cast<uint16_t*>(gsum + 4 * NT * Kg);   // [4 NT][xs]
-
-  // team = S warps sharing each block's columns; team slots are numbered
-  // across CTAs first so that few blocks spread over many SMs
-  const int tpc = kWarps / S, tl = warp / S, pw = warp % S;
-  const int T = gridDim.x * tpc, team = tl * gridDim.x + blockIdx.x;
-  const int sc_lo = pw * nsc / S, sc_hi = (pw + 1) * nsc / S, nscw = sc_hi - sc_lo;
-  const int nblk = team < P.nblocks ? (P.nblocks - 1 - team) / T + 1 : 0;
-  const int total = nblk * nscw;
-
-  uint64_t pol;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
-
-  // the first loads go out before waiting for the previous kernel: weights
-  // never depend on it
-  uint32_t wb[4][16];
-  uint32_t sv[4] = {0u, 0u, 0u, 0u};
-  int lblk = team, lsc = sc_lo;  // position of the next super-chunk to load
-  Rows lr = {};
-  if (total > 0) {
-    lr = rows_of(P, lblk, g, t);
-    load_scales(lr, Kg, lsc, sv);
-#pragma unroll
-    for (int p = 0; p < 4; ++p) load_chunk(lr, K, lsc, p, pol, wb[p]);
-  }
-
-  // the next kernel may be scheduled now (its own wait still covers all of
-  // this one); only weights were read so far
-  pdl_trigger();
-  pdl_wait();  // x (and residuals) are written by the previous kernel
-  // 1) RMSNorm statistics per batch row (fixed summation order)
-  float inv[4 * NT];
-#pragma unroll
-  for (int b = 0; b < 4 * NT; ++b) inv[b] = 0.f;
-  if (P.xmode == kXRmsNorm) {
-#pragma unroll
-    for (int b = 0; b < 4 * NT; ++b) {
-      if (b >= P.B) break;
-      float ss = 0.f;
-      for (int c = tid; c < K; c += kThreads) {
-        const float v = P.xa[(size_t)b * K + c];
-        ss = fmaf(v, v, ss);
-      }
-      ss = warp_sum(ss);
-      if (lane == 0) red[b * kWarps + warp] = ss;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int b = 0; b < 4 * NT; ++b) {
-      if (b >= P.B) break;
-      float ss = 0.f;
-      for (int w = 0; w < kWarps; ++w) ss += red[b * kWarps + w];
-      inv[b] = 1.0f / sqrtf(ss / (float)K + P.eps);
-    }
-    __syncthreads();
-  }
-  // 2) one warp per 64-column group: the input values, rounded to bf16, go
-  // to xh as fp16 and the group's fp16 sum to gsum. fp16 holds them exactly
-  // unless max|x| >= 2^15, checked after the pass; then (rarely) the pass is
-  // redone on x * 2^-e. Batch rows past B are never read by a live B lane.
-  auto form = [&](float down) -> float {
-    float mloc = 0.f;
-    for (int i = warp; i < P.B * Kg; i += kWarps) {
-      const int b = i / Kg, c = (i - b * Kg) * 64 + 2 * lane;
-      const size_t o = (size_t)b * K + c;
-      float v0, v1;
-      if (P.xmode == kXBf16) {
-        const uint32_t w2 = *reinterpret_cast<const uint32_t*>(P.x + o);
-        v0 = bf16_lo(w2);
-        v1 = bf16_hi(w2);
-      } else if (P.xmode == kXRmsNorm) {
-        float ib = inv[0];
-#pragma unroll
-        for (int j = 1; j < 4 * NT; ++j)
-          if (b == j) ib = inv[j];
-        const float2 xv = *reinterpret_cast<const float2*>(P.xa + o);
-        // (the norm weight may be only 2-byte aligned)
-        v0 = bf16_bits_to_f32(f32_to_bf16_bits(xv.x * ib * bf16_bits_to_f32(P.nw[c])));
-        v1 = bf16_bits_to_f32(f32_to_bf16_bits(xv.y * ib * bf16_bits_to_f32(P.nw[c + 1])));
-      } else {
-        const float2 z = *reinterpret_cast<const float2*>(P.xa + o);
-        const float2 u = *reinterpret_cast<const float2*>(P.xb + o);
-        v0 = bf16_bits_to_f32(f32_to_bf16_bits(z.x / (1.0f + expf(-z.x)) * u.x));
-        v1 = bf16_bits_to_f32(f32_to_bf16_bits(z.y / (1.0f + expf(-z.y)) * u.y));
-      }
-      mloc = fmaxf(mloc, fmaxf(fabsf(v0), fabsf(v1)));
-      if (P.xout && blockIdx.x == 0 && down == 1.0f)
-        *reinterpret_cast<uint32_t*>(P.xout + o) =
-            (uint32_t)f32_to_bf16_bits(v0) | ((uint32_t)f32_to_bf16_bits(v1) << 16);
-      const __half2 h2 = __floats2half2_rn(v0 * down, v1 * down);
-      *reinterpret_cast<__half2*>(xh + b * xs + c) = h2;
-      const float sum = warp_sum(__low2float(h2) + __high2float(h2));
-      if (lane == 0) gsum[i] = sum;
-    }
-    return mloc;
-  };
-  float mx = form(1.0f);
-  for (int i = P.B * Kg + tid; i < 4 * NT * Kg; i += kThreads) gsum[i] = 0.f;
-  // 3) max|x| over the CTA; prescale 2^-e so that max|x| * 2^-e < 2^15
-  mx = warp_max(mx);
-  if (lane == 0) red[warp] = mx;
-  __syncthreads();
-  mx = 0.f;
-#pragma unroll
-  for (int w = 0; w < kWarps; ++w) mx = fmaxf(mx, red[w]);
-  int e = 0;  // NaN or inf in x propagate to y without a prescale
-  if (mx >= 32768.f && mx <= 3.0e38f) e = (int)ceilf(log2f(mx / 16384.f));
-  const float up = exp2f((float)e);
-  if (e != 0) {  // uniform over the CTA
-    form(exp2f((float)-e));
-  }
-  __syncthreads();
-
-  // B-operand lanes: column n = g = 2 b + h, live on the k-slots of group h
-  bool xl[NT];
-  const uint16_t* xrow[NT];
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    const int b = 4 * nt + (g >> 1);
-    xl[nt] = b < P.B && (t >> 1) == (g & 1);
-    xrow[nt] = xh + b * xs + 32 * t;
-  }
-
-  float acc[NT][2];
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = 0.f;
-  int cblk = team, csc = sc_lo, nb = 0;
-  for (int it = 0; it < total; ++it) {
-    const bool more = it + 1 < total;
-    if (more) {
-      if (++lsc == sc_hi) {
-        lsc = sc_lo;
-        lblk += T;
-        lr = rows_of(P, lblk, g, t);
-      }
-    }
-    uint32_t svn[4] = {0u, 0u, 0u, 0u};
-    if (more) load_scales(lr, Kg, lsc, svn);
-#pragma unroll
-    for (int p = 0; p < 4; ++p) {
-      const int src = (lane & ~3) | p;
-      const uint32_t s0 = __shfl_sync(0xffffffffu, sv[0], src);
-      const uint32_t s1 = __shfl_sync(0xffffffffu, sv[1], src);
-      const uint32_t b0 = __shfl_sync(0xffffffffu, sv[2], src);
-      const uint32_t b1 = __shfl_sync(0xffffffffu, sv[3], src);
-      // (scale, bias + 128 scale) of rows g, g+8 for groups A, B of the chunk
-      const float sA0 = bf16_lo(s0), sB0 = bf16_hi(s0), sA1 = bf16_lo(s1), sB1 = bf16_hi(s1);
-      const float cA0 = fmaf(128.f, sA0, bf16_lo(b0)), cB0 = fmaf(128.f, sB0, bf16_hi(b0));
-      const float cA1 = fmaf(128.f, sA1, bf16_lo(b1)), cB1 = fmaf(128.f, sB1, bf16_hi(b1));
-      const int chunk = csc * 4 + p;
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        uint4 x0 = make_uint4(0u, 0u, 0u, 0u), x1 = x0, x2 = x0, x3 = x0;
-        if (xl[nt]) {
-          const uint4* xp = reinterpret_cast<const uint4*>(xrow[nt] + chunk * 128);
-          x0 = xp[0];
-          x1 = xp[1];
-          x2 = xp[2];
-          x3 = xp[3];
-        }
-        float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
-        chunk_mma(wb[p], x0, x1, x2, x3, d0, d1);
-        // lane (g, t): batch 4 nt + t; [0] row g group A, [1] row g group B,
-        // [2] row g+8 group A, [3] row g+8 group B
-        const float2 gs = *reinterpret_cast<const float2*>(gsum + (4 * nt + t) * Kg + 2 * chunk);
-        acc[nt][0] = fmaf(sA0, d0[0] + d1[0], fmaf(cA0, gs.x, fmaf(sB0, d0[1] + d1[1],
-                                                                   fmaf(cB0, gs.y, acc[nt][0]))));
-        acc[nt][1] = fmaf(sA1, d0[2] + d1[2], fmaf(cA1, gs.x, fmaf(sB1, d0[3] + d1[3],
-                                                                   fmaf(cB1, gs.y, acc[nt][1]))));
-      }
-      if (more) load_chunk(lr, K, lsc, p, pol, wb[p]);
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) sv[i] = svn[i];
-
-    if (++csc < sc_hi) continue;
-    // ------------------------------------------------ block done: store
-    bool store = true;
-    if (S > 1) {
-      // partial sums of the team meet in shared memory (double-buffered by
-      // block parity, one named barrier per block), summed in part order
-      float* pb = part + (((nb & 1) * kWarps + tl * S) * 32) * 2 * NT;
-      if (pw != 0) {
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          pb[((pw * 32) + lane) * 2 * NT + 2 * nt] = acc[nt][0];
-          pb[((pw * 32) + lane) * 2 * NT + 2 * nt + 1] = acc[nt][1];
-        }
-      }
-      asm volatile("bar.sync %0, %1;" ::"r"(1 + tl), "r"(S * 32) : "memory");
-      if (pw == 0) {
-        for (int q = 1; q < S; ++q) {
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            acc[nt][0] += pb[((q * 32) + lane) * 2 * NT + 2 * nt];
-            acc[nt][1] += pb[((q * 32) + lane) * 2 * NT + 2 * nt + 1];
-          }
-        }
-      } else {
-        store = false;
-      }
-    }
-    if (store) {
-      const Seg& Sg = P.seg[seg_of(P, cblk)];
-      const int row0 = (cblk - Sg.blk0) * kRB;
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const int b = 4 * nt + t;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int r = row0 + g + 8 * h;
-          if (b < P.B && r < Sg.N) {
-            const size_t o = (size_t)b * Sg.N + r;
-            float v = acc[nt][h] * up;
-            if (Sg.res) v += Sg.res[o];
-            if (Sg.y_bf16)
-              reinterpret_cast<uint16_t*>(Sg.y)[o] = f32_to_bf16_bits(v);
-            else
-              reinterpret_cast<float*>(Sg.y)[o] = v;
-          }
-        }
-      }
-    }
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = 0.f;
-    csc = sc_lo;
-    cblk += T;
-    ++nb;
-  }
+  // the next kernel may be scheduled as soon as the weight loads are out (its
+  // own wait still covers all of this one)
+  gemv_tc_body<NT, W>(P, smem, [] {
+    pdl_trigger();
+    pdl_wait();
+  });
 }
 
 }  // namespace gtc
 
-static size_t gtc_smem(int K, int NT, int W) {
-  return (size_t)4 * NT * W * 4 + (size_t)2 * W * 32 * 2 * NT * 4 +
-         (size_t)4 * NT * (K / 64) * 4 + (size_t)4 * NT * (K + 8) * 2;
-}
 
 // Whether the tensor-core path takes this GEMV: bf16 x, 1 <= B <= 8, K a
 // multiple of 512, codes 32-byte aligned (256-bit loads), scales and biases
@@ -468,11 +100,9 @@ static cudaError_t gtc_launch(const GemvSeg* segs, int nseg, gtc::Params& P, int
   // for the small matrices of a decode step); then split each block's
   // columns over S warps while slots stay idle
   const int NT = (B + 3) / 4;
-  const int sms = num_sms(), nsc = K / gtc::kSC;
+  const int sms = num_sms();
   const int W = NT == 1 ? 16 : 8;
-  int S = 1;
-  while (S < W && 2 * S <= nsc && (long long)blk * S < (long long)sms * W) S *= 2;
-  P.S = S;
+  P.S = gtc_split(blk, K, W, sms);
   const int grid = std::min(sms, blk);
   if (NT == 2) return gtc_launch_nt<2, 8>(P, grid, st, pdl);
   return gtc_launch_nt<1, 16>(P, grid, st, pdl);

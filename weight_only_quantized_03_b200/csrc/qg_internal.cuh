@@ -180,14 +180,12 @@ cudaError_t attention_launch_step(const float* q, const float* k, const float* v
                                   uint16_t* kc, uint16_t* vc, const int32_t* positions, void* out,
                                   int B, int H, int Hkv, int D, int cap, float scale, void* ws,
                                   cudaStream_t st, bool pdl);
+// The split plan of the attention kernels (rows per split, splits) and the
+// three parts of an attention workspace (split outputs, split (max, sum),
+// ticket counters).
+void attention_plan(int B, int Hkv, int cap, int* ch, int* nsplit);
+void attention_ws_split(void* ws, int B, int H, int Hkv, int D, int cap, float** ws_o,
+                        float** ws_ml, unsigned int** ws_cnt);
 size_t attention_ws_bytes(int B, int H, int Hkv, int D, int cap);
-
-// persistent decode-step kernel (decode_mega.cu)
-bool mega_eligible(const qg_qwen3_config& c, int B, int cap);
-size_t mega_ws_bytes(const qg_qwen3_config& c, int B, int cap);
-cudaError_t mega_launch(const qg_qwen3_config& c, const qg_qwen3_weights& w, uint16_t* kc,
-                        uint16_t* vc, int cap, const int32_t* tokens, const int32_t* positions,
-                        float* logits, int B, float* x, void* xws, unsigned* cnt, unsigned* step,
-                        bool test_stall, unsigned long long* trace, cudaStream_t st);
 
 }  // namespace qg
