@@ -157,10 +157,22 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def traffic_from_profile(kernel_file):
+def source_sha256(paths):
+    """sha256 over the given source files, concatenated in order."""
+    h = hashlib.sha256()
+    for p in paths:
+        h.update(open(p, "rb").read())
+    return h.hexdigest()
+
+
+LM_HEAD_SOURCES = [os.path.join(ROOT, "weight_only_quantized_03_b200", "csrc", f)
+                   for f in ("gemv_affine8_tc.cu", "gemv_tc.cuh")]
+
+
+def traffic_from_profile(kernel_files):
     """DRAM bytes per launch of the LM-head GEMV from the committed ncu
     summary, or None when that summary is missing or was taken on a different
-    version of the kernel source (its sha256 must match)."""
+    version of the kernel sources (their sha256 must match)."""
     path = os.path.join(ROOT, "profiles", "gemv_affine8_lm_head_151936x1024_b1.md")
     try:
         text = open(path).read()
@@ -170,8 +182,7 @@ def traffic_from_profile(kernel_file):
     h = re.search(r"kernel_source_sha256:\s*([0-9a-f]{64})", text)
     if not m or not h:
         return None
-    cur = hashlib.sha256(open(kernel_file, "rb").read()).hexdigest()
-    return int(m.group(1)) if cur == h.group(1) else None
+    return int(m.group(1)) if source_sha256(kernel_files) == h.group(1) else None
 
 
 class ClockSampler:
@@ -379,8 +390,7 @@ def run_ours(args):
                           stream, nlaunch)
     lm_bytes = affine8_bytes(V, h, B)
     lm_gbs = lm_bytes / (lm_ms / 1000.0) / 1e9
-    traffic = traffic_from_profile(os.path.join(ROOT, "weight_only_quantized_03_b200", "csrc",
-                                                "gemv_affine8_tc.cu")) if B == 1 else None
+    traffic = traffic_from_profile(LM_HEAD_SOURCES) if B == 1 else None
 
     # ---- the other rows of the path, each timed per launch on its stream
     kernels = other_kernels(qg, stream, hbm_peak, max(20, min(100, args.steps)))
@@ -458,7 +468,8 @@ def run_ncu_case(args):
     """One kernel alone, warm-up then ``--steps`` launches, for an ncu capture
     (no timing, no JSON line): ``lm_head`` is the tied LM-head GEMV of the
     0.6B shape at ``--batch``; ``gemm`` the Whisper FC1 Q4_0 GEMM
-    (1500 x 5120 x 1280)."""
+    (1500 x 5120 x 1280); ``attn`` the decode attention at the 1.7B shape,
+    batch 32, KV 2048."""
     import torch
     import weight_only_quantized_03_b200 as qg
     to = lambda a: torch.from_numpy(a.view({1: np.uint8, 2: np.int16, 4: np.int32}[a.dtype.itemsize])).cuda()
@@ -469,6 +480,17 @@ def run_ncu_case(args):
         x = to(qg_synth.gaussian_bf16_bits((args.batch, h), 1.0, 5)).view(torch.bfloat16)
         y = torch.empty((args.batch, V), dtype=torch.float32, device="cuda")
         run = lambda: qg.qg_gemv_affine8_g64(w, s, b, x, y)
+    elif args.ncu_case == "attn":
+        # the 1.7B attention shape at batch 32 and KV 2048: 268 MB of K/V
+        B, H, Hkv, D, L = 32, 16, 8, 128, 2048
+        q = to(qg_synth.gaussian((B, H * D), 1.0, 30).astype(np.float32)).view(torch.float32)
+        kc = to(qg_synth.gaussian_bf16_bits((B, Hkv, L, D), 1.0, 31)).view(torch.bfloat16)
+        vc = to(qg_synth.gaussian_bf16_bits((B, Hkv, L, D), 1.0, 32)).view(torch.bfloat16)
+        kv_len = torch.full((B,), L, dtype=torch.int32, device="cuda")
+        out = torch.empty((B, H * D), dtype=torch.bfloat16, device="cuda")
+        ws = torch.empty(qg.qg_decode_attention_workspace_size(B, H, Hkv, D, L),
+                         dtype=torch.uint8, device="cuda")
+        run = lambda: qg.qg_decode_attention(q, kc, vc, kv_len, out, H, Hkv, D ** -0.5, ws)
     else:
         M, N, K = 1500, 5120, 1280
         blocks = to(qg_synth.q4_0_packed(N, K, 22))
@@ -568,7 +590,7 @@ def main():
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--ncu-case", choices=["lm_head", "gemm"], default=None,
+    ap.add_argument("--ncu-case", choices=["lm_head", "gemm", "attn"], default=None,
                     help="launch one kernel only (for an ncu capture); prints no JSON line")
     ap.add_argument("--sweep", action="store_true",
                     help="the Qwen3-1.7B-shaped prefill and batch sweep (its own JSON line)")
