@@ -443,6 +443,9 @@ def decode_layer_forced(cfg, lw, x, k_cache_l, v_cache_l, pos, forced, rel=2.0 *
     receive the forced (else the rounded) K and V."""
     H, Hkv, D = cfg["heads"], cfg["kv_heads"], cfg["head_dim"]
     eps, theta = cfg["eps"], cfg["theta"]
+    unknown = set(forced) - {"xn", "k", "v", "att", "xn2", "h"}
+    if unknown:  # a misnamed point would silently go unforced
+        raise KeyError(f"decode_layer_forced: unknown rounding points {sorted(unknown)}")
     bad = {}
 
     def at(name, val):

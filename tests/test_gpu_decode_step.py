@@ -56,6 +56,7 @@ def _forced_layer(cfg, lw, x, kc_l, vc_l, p, inter_b, k_row, v_row, what):
     rounding points (each checked to be a correct rounding of the oracle's
     own value there: exact, or the other side of a near-tie)."""
     forced = dict(inter_b, k=k_row.ravel(), v=v_row.ravel())
+    forced["att"] = forced.pop("attn")  # the oracle's name for the attention output
     det = {}
     ref, bad = O.decode_layer_forced(cfg, lw, x, kc_l, vc_l, p, forced, details=det)
     for name, idx in bad.items():

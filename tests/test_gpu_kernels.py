@@ -299,6 +299,11 @@ ATTN_CASES = [
     (10, 16, 8, 128, 513, [512, 1, 100, 511, 256, 2, 3, 400, 512, 77]),
     (1, 16, 8, 128, 2048, [2048]),
     (2, 8, 1, 32, 5, [0, 6]),          # invalid lengths -> zero rows
+    (4, 16, 4, 128, 300, [300, 1, 150, 299]),   # 4 query heads per kv head
+    (2, 6, 2, 64, 100, [100, 37]),              # 3 query heads per kv head
+    (1, 4, 2, 96, 50, [50]),                    # head_dim 96: the split kernel
+    (32, 16, 8, 128, 16, [16, 1, 2, 15] * 8),   # many sequences, one-CTA clusters
+    (1, 2, 2, 32, 1000, [999]),                 # head_dim 32, long chunks
 ]
 
 

@@ -390,6 +390,33 @@ def test_decode_layer_forced_flags_wrong_values_and_follows_valid_ones():
     assert bad_t["xn"].size > 300   # with the default bound most are wrong
 
 
+def test_decode_layer_forced_follows_a_forced_attention_and_rejects_unknown_points():
+    cfg, lw, x, kc, vc = _small_layer()
+    # forcing the attention output to its other rounding neighbour at one
+    # element changes the layer's output by exactly that element's effect
+    # through o_proj onward; a misnamed point is an error, not a silent no-op
+    y_plain = O.decode_layer(cfg, lw, x, kc.copy(), vc.copy(), 9)
+    H, D = cfg["heads"], cfg["head_dim"]
+    xn = O.round_bf16(O.rmsnorm(x, lw["input_norm"], cfg["eps"]))
+    k1, v1 = kc.copy(), vc.copy()
+    O.decode_layer(cfg, lw, x, k1, v1, 9)
+    q = O.gemv_affine8(*lw["q"], xn[None])[0]
+    q = O.rope_neox(O.rmsnorm_perhead(q, lw["q_norm"], cfg["eps"], D), 9, cfg["theta"], D)
+    att_v = O.decode_attention(q, k1, v1, 10, H, cfg["kv_heads"], D)
+    att = O.round_bf16(att_v)
+    flipped = att.copy()
+    j = int(np.argmax(np.abs(att)))
+    flipped[j] = O.round_bf16_up(att_v[j]) if att[j] == O.round_bf16_down(att_v[j]) \
+        else O.round_bf16_down(att_v[j])
+    y_same, _ = O.decode_layer_forced(cfg, lw, x, kc.copy(), vc.copy(), 9, {"att": att})
+    np.testing.assert_array_equal(y_same, y_plain)
+    y_flip, bad = O.decode_layer_forced(cfg, lw, x, kc.copy(), vc.copy(), 9, {"att": flipped},
+                                        rel=2.0 ** -7, abs_rel=0.0)
+    assert bad["att"].size == 0 and np.abs(y_flip - y_plain).max() > 0
+    with pytest.raises(KeyError):
+        O.decode_layer_forced(cfg, lw, x, kc.copy(), vc.copy(), 9, {"attn": att})
+
+
 def test_lm_head_tie_bound_is_the_exact_linear_effect_of_each_tie():
     cfg = dict(hidden=256, layers=0, heads=2, kv_heads=1, head_dim=128, ffn=256, vocab=500,
                eps=1e-6, theta=1e6)

@@ -15,6 +15,7 @@
 //
 // Cache layout [B][Hkv][cap][D]: the rows of one head are contiguous, so a
 // split reads one contiguous CH*D*2-byte run of K and one of V.
+#include <algorithm>
 #include <mutex>
 
 #include "attention_body.cuh"
@@ -70,11 +71,423 @@ attention_split_kernel(const float* __restrict__ q, const uint16_t* __restrict__
       });
 }
 
+// ---------------------------------------------------------------------------
+// Cluster kernel (head_dim 32/64/128/256, at most 4 query heads per KV head).
+//
+// Grid (cs, Hkv, B) launched as clusters of cs CTAs along x: the cs CTAs of
+// one (sequence, kv head) pair split its rows [0, L) into cs contiguous
+// chunks of ch rows. Each row of K or V is D bf16 = D/8 lanes x 16 bytes, so
+// one warp load instruction covers 32/(D/8) consecutive rows (a "slot");
+// each lane keeps the 8 columns of its 16 bytes. A warp holds U slots of K
+// and V in registers per batch, and two batches are in flight: the next one
+// loads while the current one is scored (in the decode step the first two
+// are issued before the programmatic-dependent-launch wait, since cached
+// rows below the position are final). Per lane group (the lanes of one row):
+// a running (max, sum, weighted V) per query head, updated once per batch.
+// The warps' states merge in shared memory; the cluster's CTAs then merge in
+// rank order through distributed shared memory (rank 0 reads every rank's
+// partial), so the result is deterministic and needs no workspace, atomics
+// or global round trip.
+//
+// Decode step (AttnFuse): every CTA norms and ropes its own query heads; the
+// CTA whose chunk holds row p = position computes the new K and V rows, stores
+// them in the cache for later steps and uses them from shared memory as row
+// p, so no CTA reads a cache row this kernel writes.
+// ---------------------------------------------------------------------------
+
+namespace ac {
+
+constexpr int kNW = 8;                 // warps per CTA
+constexpr int kThreads = kNW * 32;
+constexpr int kMaxCluster = 8;         // portable cluster size
+
+template <int D>
+struct Geo {
+  static constexpr int LPR = D / 8;             // lanes per row (16 bytes each)
+  static constexpr int RPI = 32 / LPR;          // rows per warp load instruction
+  static constexpr int U = D >= 256 ? 2 : (D == 128 ? 3 : (RPI >= 8 ? 1 : 8 / RPI));  // slots per batch
+  static constexpr int ROWS = kNW * U * RPI;    // rows per CTA batch
+};
+
+__device__ __forceinline__ uint4 ld_row16(const uint16_t* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ unsigned cluster_rank() {
+  unsigned r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+               "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// fp32 at `p` (this CTA's shared memory) in the shared memory of CTA `rank`
+// of the cluster.
+__device__ __forceinline__ float ld_cluster(const float* p, unsigned rank) {
+  const uint32_t local = (uint32_t)__cvta_generic_to_shared(p);
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(rank));
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+  return v;
+}
+
+// Merge (m2, l2, o2) into (m, l, o): the larger max wins, the other side is
+// scaled by exp(its max - new max). An empty side has max -inf, sum 0.
+__device__ __forceinline__ void merge_state(float& m, float& l, float* o, float m2, float l2,
+                                            const float* o2, int n) {
+  const float M = fmaxf(m, m2);
+  if (M == -INFINITY) return;
+  const float a = expf(m - M), a2 = expf(m2 - M);
+  l = l * a + l2 * a2;
+  for (int i = 0; i < n; ++i) o[i] = o[i] * a + o2[i] * a2;
+  m = M;
+}
+
+template <int D, int GM>
+__global__ void __launch_bounds__(kThreads, GM <= 2 ? 2 : 1)
+attention_cluster_kernel(const float* q, const uint16_t* kc, const uint16_t* vc,
+                         const int32_t* __restrict__ kv_len, const int32_t* __restrict__ pos_for_len,
+                         void* out, int out_bf16, int H, int Hkv, int cap, float scale, int ch,
+                         const AttnFuse fz) {
+  using G = Geo<D>;
+  constexpr int LPR = G::LPR, RPI = G::RPI, U = G::U;
+  __shared__ float sq[GM][D];          // query heads (normed, roped) * scale
+  __shared__ float kp[D], vp[D];       // the new row p (bf16 values), owner CTA only
+  __shared__ float sp[GM];             // scores of row p
+  __shared__ float wm[kNW][GM], wl[kNW][GM];
+  __shared__ float wo[kNW][GM][D];
+  __shared__ float cm[GM], cl[GM];     // this CTA's partial, read by rank 0
+  __shared__ float co[GM][D];
+
+  const unsigned s = cluster_rank();
+  const unsigned cs = gridDim.x;
+  const int kv = blockIdx.y, b = blockIdx.z;
+  const int g = H / Hkv;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c = lane % LPR, r = lane / LPR;  // 16-byte chunk of the row; row in the slot
+  const size_t head_base = ((size_t)b * Hkv + kv) * cap;
+  const int t0 = (int)s * ch;
+
+  // cached rows this CTA scores: [t0, tend)
+  int tend = t0;
+  bool valid = false;
+  int p = -1;
+  if (fz.on) {
+    p = pos_for_len[b];
+    valid = p >= 0 && p < cap;
+    if (valid) tend = max(t0, min(t0 + ch, p));  // row p itself comes from shared memory
+  }
+
+  uint4 ka[U], va[U], kb[U], vb[U];
+  auto load = [&](int batch, uint4(&kr)[U], uint4(&vr)[U]) {
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int t = t0 + ((batch * U + u) * kNW + warp) * RPI + r;
+      if (t < tend) {
+        const size_t off = (head_base + t) * D + c * 8;
+        kr[u] = ld_row16(kc + off);
+        vr[u] = ld_row16(vc + off);
+      } else {
+        kr[u] = vr[u] = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+  };
+  int nb = (tend - t0 + G::ROWS - 1) / G::ROWS;
+  if (fz.on) {
+    if (nb > 0) load(0, ka, va);
+    if (nb > 1) load(1, kb, vb);
+  }
+  // the next kernel may be scheduled now: its own wait covers all of this one
+  pdl_trigger();
+  pdl_wait();
+  if (!fz.on) {
+    const int L = kv_len[b];
+    valid = L >= 1 && L <= cap;
+    tend = valid ? max(t0, min(t0 + ch, L)) : t0;
+    nb = (tend - t0 + G::ROWS - 1) / G::ROWS;
+    if (nb > 0) load(0, ka, va);
+    if (nb > 1) load(1, kb, vb);
+  }
+
+  // ---- query heads (and, in the decode step, the new K/V row)
+  const bool owner = fz.on && valid && p >= t0 && p < t0 + ch;
+  if (!fz.on) {
+    for (int i = threadIdx.x; i < g * D; i += kThreads)
+      sq[i / D][i % D] = __ldcg(q + ((size_t)b * H + kv * g + i / D) * D + i % D) * scale;
+  } else {
+    const int tk = fz.tok[b];
+    const bool write = owner && tk >= 0 && tk < fz.vocab;  // a bad token leaves the cache
+    const float2* rcs = fz.rope + (size_t)b * (D / 2);
+    const size_t row = (head_base + (valid ? p : 0)) * D;
+    if (warp < g) {
+      float* dst = sq[warp];
+      norm_rope_head(q + ((size_t)b * H + kv * g + warp) * D, fz.qn, D, fz.eps, rcs, lane,
+                     [&](int i, float v) { dst[i] = v * scale; });
+    } else if (warp == g && owner) {
+      norm_rope_head(fz.k + ((size_t)b * Hkv + kv) * D, fz.kn, D, fz.eps, rcs, lane,
+                     [&](int i, float v) {
+                       const uint16_t bits = f32_to_bf16_bits(v);
+                       kp[i] = bf16_bits_to_f32(bits);
+                       if (write) const_cast<uint16_t*>(kc)[row + i] = bits;
+                     });
+    } else if (warp == g + 1 && owner) {
+      const float* vs = fz.v + ((size_t)b * Hkv + kv) * D;
+      for (int d = lane; d < D; d += 32) {
+        const uint16_t bits = f32_to_bf16_bits(__ldcg(vs + d));
+        vp[d] = bf16_bits_to_f32(bits);
+        if (write) const_cast<uint16_t*>(vc)[row + d] = bits;
+      }
+    }
+  }
+  __syncthreads();
+  if (owner && warp < g) {  // score of row p for query head `warp`
+    float d = 0.f;
+    for (int i = lane; i < D; i += 32) d = fmaf(sq[warp][i], kp[i], d);
+    d = warp_sum(d);
+    if (lane == 0) sp[warp] = d;
+  }
+
+  // ---- this warp's rows: online softmax per lane group
+  float qv[GM][8], o[GM][8], m[GM], l[GM];
+#pragma unroll
+  for (int h = 0; h < GM; ++h) {
+    m[h] = -INFINITY;
+    l[h] = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      qv[h][i] = h < g ? sq[h][c * 8 + i] : 0.f;
+      o[h][i] = 0.f;
+    }
+  }
+  auto process = [&](int batch, const uint4(&kr)[U], const uint4(&vr)[U]) {
+    bool ok[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) ok[u] = t0 + ((batch * U + u) * kNW + warp) * RPI + r < tend;
+#pragma unroll
+    for (int h = 0; h < GM; ++h) {
+      if (h >= g) break;
+      float sc[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const uint4 k = kr[u];
+        float d = qv[h][0] * bf16_lo(k.x);
+        d = fmaf(qv[h][1], bf16_hi(k.x), d);
+        d = fmaf(qv[h][2], bf16_lo(k.y), d);
+        d = fmaf(qv[h][3], bf16_hi(k.y), d);
+        d = fmaf(qv[h][4], bf16_lo(k.z), d);
+        d = fmaf(qv[h][5], bf16_hi(k.z), d);
+        d = fmaf(qv[h][6], bf16_lo(k.w), d);
+        d = fmaf(qv[h][7], bf16_hi(k.w), d);
+        sc[u] = d;
+      }
+#pragma unroll
+      for (int off = LPR / 2; off >= 1; off >>= 1)
+#pragma unroll
+        for (int u = 0; u < U; ++u) sc[u] += __shfl_xor_sync(0xffffffffu, sc[u], off);
+      float mx = m[h];
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        if (ok[u]) mx = fmaxf(mx, sc[u]);
+      if (mx == -INFINITY) continue;
+      const float a = expf(m[h] - mx);  // 0 while m is still -inf
+      l[h] *= a;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o[h][i] *= a;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        if (!ok[u]) continue;
+        const float pr = expf(sc[u] - mx);
+        l[h] += pr;
+        const uint4 v = vr[u];
+        o[h][0] = fmaf(pr, bf16_lo(v.x), o[h][0]);
+        o[h][1] = fmaf(pr, bf16_hi(v.x), o[h][1]);
+        o[h][2] = fmaf(pr, bf16_lo(v.y), o[h][2]);
+        o[h][3] = fmaf(pr, bf16_hi(v.y), o[h][3]);
+        o[h][4] = fmaf(pr, bf16_lo(v.z), o[h][4]);
+        o[h][5] = fmaf(pr, bf16_hi(v.z), o[h][5]);
+        o[h][6] = fmaf(pr, bf16_lo(v.w), o[h][6]);
+        o[h][7] = fmaf(pr, bf16_hi(v.w), o[h][7]);
+      }
+      m[h] = mx;
+    }
+  };
+  for (int i = 0; i < nb; i += 2) {
+    process(i, ka, va);
+    if (i + 2 < nb) load(i + 2, ka, va);
+    if (i + 1 < nb) {
+      process(i + 1, kb, vb);
+      if (i + 3 < nb) load(i + 3, kb, vb);
+    }
+  }
+
+  // ---- merge the lane groups of the warp (lanes with the same chunk c)
+#pragma unroll
+  for (int off = LPR; off < 32; off <<= 1) {
+#pragma unroll
+    for (int h = 0; h < GM; ++h) {
+      const float m2 = __shfl_xor_sync(0xffffffffu, m[h], off);
+      const float l2 = __shfl_xor_sync(0xffffffffu, l[h], off);
+      float o2[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o2[i] = __shfl_xor_sync(0xffffffffu, o[h][i], off);
+      merge_state(m[h], l[h], o[h], m2, l2, o2, 8);
+    }
+  }
+  if (r == 0) {
+#pragma unroll
+    for (int h = 0; h < GM; ++h) {
+      if (h >= g) break;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) wo[warp][h][c * 8 + i] = o[h][i];
+      if (c == 0) {
+        wm[warp][h] = m[h];
+        wl[warp][h] = l[h];
+      }
+    }
+  }
+  __syncthreads();
+
+  // ---- this CTA's partial: its warps in order, then row p
+  for (int i = threadIdx.x; i < g * D; i += kThreads) {
+    const int h = i / D, d = i % D;
+    float M = owner ? sp[h] : -INFINITY;
+    for (int w = 0; w < kNW; ++w) M = fmaxf(M, wm[w][h]);
+    float Ls = 0.f, O = 0.f;
+    if (M != -INFINITY) {
+      for (int w = 0; w < kNW; ++w) {
+        const float e = wm[w][h] == -INFINITY ? 0.f : expf(wm[w][h] - M);
+        Ls = fmaf(wl[w][h], e, Ls);
+        O = fmaf(wo[w][h][d], e, O);
+      }
+      if (owner) {
+        const float e = expf(sp[h] - M);
+        Ls += e;
+        O = fmaf(vp[d], e, O);
+      }
+    }
+    co[h][d] = O;
+    if (d == 0) {
+      cm[h] = M;
+      cl[h] = Ls;
+    }
+  }
+  cluster_sync();  // every CTA's partial is in its shared memory
+
+  // ---- rank 0 merges the cluster's partials in rank order
+  if (s == 0) {
+    for (int i = threadIdx.x; i < g * D; i += kThreads) {
+      const int h = i / D, d = i % D;
+      float M = -INFINITY;
+      for (unsigned j = 0; j < cs; ++j) M = fmaxf(M, ld_cluster(&cm[h], j));
+      float Ls = 0.f, O = 0.f;
+      if (M != -INFINITY) {
+        for (unsigned j = 0; j < cs; ++j) {
+          const float mj = ld_cluster(&cm[h], j);
+          if (mj == -INFINITY) continue;
+          const float e = expf(mj - M);
+          Ls = fmaf(ld_cluster(&cl[h], j), e, Ls);
+          O = fmaf(ld_cluster(&co[h][d], j), e, O);
+        }
+      }
+      const float res = (valid && Ls > 0.f) ? O / Ls : 0.f;
+      const size_t oi = ((size_t)b * H + kv * g + h) * D + d;
+      if (out_bf16)
+        reinterpret_cast<uint16_t*>(out)[oi] = f32_to_bf16_bits(res);
+      else
+        reinterpret_cast<float*>(out)[oi] = res;
+    }
+  }
+  cluster_sync();  // no CTA leaves while rank 0 still reads its shared memory
+}
+
+// Whether the cluster kernel takes the shape.
+inline bool cluster_ok(int H, int Hkv, int D) {
+  const int g = H / Hkv;
+  return (D == 32 || D == 64 || D == 128 || D == 256) && g >= 1 && g <= 4 && H % Hkv == 0;
+}
+
+// CTAs per (sequence, kv head): enough CTAs for about four waves of two
+// CTAs per SM, at most 8 (a portable cluster), and chunks of at least 16 rows.
+inline int cluster_size(int B, int Hkv, int cap) {
+  const long long pairs = (long long)B * Hkv;
+  long long cs = (8LL * num_sms() + pairs - 1) / pairs;
+  cs = std::min<long long>(cs, (cap + 15) / 16);
+  cs = std::max<long long>(1, std::min<long long>(cs, kMaxCluster));
+  return (int)cs;
+}
+
+template <int D, int GM>
+cudaError_t launch(const float* q, const uint16_t* kc, const uint16_t* vc, const int32_t* kv_len,
+                   const int32_t* pos_for_len, void* out, bool out_bf16, int B, int H, int Hkv,
+                   int cap, float scale, cudaStream_t st, bool pdl, const AttnFuse& fz) {
+  const int cs = cluster_size(B, Hkv, cap);
+  const int ch = (cap + cs - 1) / cs;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(cs, Hkv, B);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute a[2];
+  a[0].id = cudaLaunchAttributeClusterDimension;
+  a[0].val.clusterDim.x = cs;
+  a[0].val.clusterDim.y = 1;
+  a[0].val.clusterDim.z = 1;
+  a[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  a[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = a;
+  cfg.numAttrs = pdl ? 2 : 1;
+  count_launch();
+  return cudaLaunchKernelEx(&cfg, attention_cluster_kernel<D, GM>, q, kc, vc, kv_len, pos_for_len,
+                            out, (int)out_bf16, H, Hkv, cap, scale, ch, fz);
+}
+
+template <int D>
+cudaError_t launch_d(const float* q, const uint16_t* kc, const uint16_t* vc, const int32_t* kv_len,
+                     const int32_t* pos_for_len, void* out, bool out_bf16, int B, int H, int Hkv,
+                     int cap, float scale, cudaStream_t st, bool pdl, const AttnFuse& fz) {
+  const int g = H / Hkv;
+  if (g <= 1)
+    return launch<D, 1>(q, kc, vc, kv_len, pos_for_len, out, out_bf16, B, H, Hkv, cap, scale, st,
+                        pdl, fz);
+  if (g <= 2)
+    return launch<D, 2>(q, kc, vc, kv_len, pos_for_len, out, out_bf16, B, H, Hkv, cap, scale, st,
+                        pdl, fz);
+  return launch<D, 4>(q, kc, vc, kv_len, pos_for_len, out, out_bf16, B, H, Hkv, cap, scale, st,
+                      pdl, fz);
+}
+
+}  // namespace ac
+
 static cudaError_t attention_launch_any(const float* q, const uint16_t* kc, const uint16_t* vc,
                                         const int32_t* kv_len, const int32_t* pos_for_len,
                                         void* out, bool out_bf16, int B, int H, int Hkv, int D,
                                         int cap, float scale, void* ws, cudaStream_t st, bool pdl,
                                         const AttnFuse& fz) {
+  if (ac::cluster_ok(H, Hkv, D)) {
+    switch (D) {
+      case 32:
+        return ac::launch_d<32>(q, kc, vc, kv_len, pos_for_len, out, out_bf16, B, H, Hkv, cap,
+                                scale, st, pdl, fz);
+      case 64:
+        return ac::launch_d<64>(q, kc, vc, kv_len, pos_for_len, out, out_bf16, B, H, Hkv, cap,
+                                scale, st, pdl, fz);
+      case 128:
+        return ac::launch_d<128>(q, kc, vc, kv_len, pos_for_len, out, out_bf16, B, H, Hkv, cap,
+                                 scale, st, pdl, fz);
+      default:
+        return ac::launch_d<256>(q, kc, vc, kv_len, pos_for_len, out, out_bf16, B, H, Hkv, cap,
+                                 scale, st, pdl, fz);
+    }
+  }
+  // other head sizes and groups: the split kernel with a workspace merge
   const AttnPlan p = attn_plan(B, Hkv, cap);
   uint8_t* w = reinterpret_cast<uint8_t*>(ws);
   float* ws_o = reinterpret_cast<float*>(w);
