@@ -80,8 +80,8 @@ GEMV_CASES = [
     (300, 6144, 5, "bf16", "f32", False, False),
     (9473, 256, 1, "bf16", "f32", False, False),
     (40000, 128, 2, "bf16", "f32", False, False),
-    # the tensor-core streaming path (bf16 x, K % 512 == 0, B <= 8): ragged
-    # rows, one or two batch tiles, column splits over 2, 4 and 8 warps
+    # the tensor-core streaming path (bf16 x, K % 512 == 0, B <= 32): ragged
+    # rows, one or two n-tiles, batch tiles of 8 past B = 8, column splits over 2, 4 and 8 warps
     # (uneven when K / 512 is not a multiple), residual, bf16 output
     (1001, 512, 8, "bf16", "bf16", True, True),
     (1001, 512, 32, "bf16", "bf16", True, True),
@@ -92,6 +92,8 @@ GEMV_CASES = [
     (3, 1536, 6, "bf16", "bf16", False, False),
     (16, 4096, 1, "bf16", "bf16", False, False),
     (200, 8192, 2, "bf16", "f32", False, False),
+    (2050, 2048, 9, "bf16", "f32", True, False),    # two batch tiles, the second of 1 row
+    (1024, 3072, 24, "bf16", "bf16", True, False),  # three batch tiles
 ]
 
 

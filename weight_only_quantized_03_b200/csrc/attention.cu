@@ -536,23 +536,6 @@ cudaError_t attention_launch_step(const float* q, const float* k, const float* v
                               ws, st, pdl, fz);
 }
 
-void attention_plan(int B, int Hkv, int cap, int* ch, int* nsplit) {
-  const AttnPlan p = attn_plan(B, Hkv, cap);
-  *ch = p.ch;
-  *nsplit = p.nsplit;
-}
-
-void attention_ws_split(void* ws, int B, int H, int Hkv, int D, int cap, float** ws_o,
-                        float** ws_ml, unsigned int** ws_cnt) {
-  const AttnPlan p = attn_plan(B, Hkv, cap);
-  uint8_t* w = reinterpret_cast<uint8_t*>(ws);
-  *ws_o = reinterpret_cast<float*>(w);
-  w += align256((size_t)B * H * p.nsplit * D * sizeof(float));
-  *ws_ml = reinterpret_cast<float*>(w);
-  w += align256((size_t)B * H * p.nsplit * 2 * sizeof(float));
-  *ws_cnt = reinterpret_cast<unsigned int*>(w);
-}
-
 // Offset of the ticket counters inside an attention workspace.
 size_t attention_ws_counter_offset(int B, int H, int Hkv, int D, int cap) {
   const AttnPlan p = attn_plan(B, Hkv, cap);

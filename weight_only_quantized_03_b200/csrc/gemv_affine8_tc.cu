@@ -1,5 +1,5 @@
 // Affine-INT8 group-64 dequant GEMV on the tensor cores (the streaming
-// path of qg_gemv_affine8_g64 for bf16 activations and B <= 8).
+// path of qg_gemv_affine8_g64 for bf16 activations and B <= 32).
 //
 // Format and arithmetic as in gemv_affine8.cu (turbospark-runtime 0.3.0,
 // src/qwen3_asr_metal.rs, PackedLinear / load_packed_linear; y = W x with
@@ -37,6 +37,10 @@
 //   * Scales and biases of a super-chunk: lane (g, t) loads the bf16 pairs of
 //     groups 2t, 2t + 1 for rows g and g + 8; chunk p takes them from lane
 //     (g, p) by shuffle.
+//   * A CTA holds up to 8 batch rows (two n-tiles). Past 8, the batch splits
+//     into tiles of 8 along gridDim.y; the tiles stream the same weights at
+//     about the same time, so HBM sees them about once and L2 serves the
+//     rest (the CUDA-core path would be ALU-bound there).
 #include <algorithm>
 
 #include "gemv_tc.cuh"
@@ -59,20 +63,20 @@ __global__ void __launch_bounds__(W * 32, NT == 1 ? 512 / (W * 32) : 1)
 }  // namespace gtc
 
 
-// Whether the tensor-core path takes this GEMV: bf16 x, 1 <= B <= 8, K a
+// Whether the tensor-core path takes this GEMV: bf16 x, 1 <= B <= 32, K a
 // multiple of 512, codes 32-byte aligned (256-bit loads), scales and biases
 // 4-byte aligned, and x fits in shared memory as fp16.
 bool gemv_tc_eligible(const GemvSeg* segs, int nseg, int K, int B, bool x_f32) {
-  if (x_f32 || K < gtc::kSC || K % gtc::kSC != 0 || B < 1 || B > gtc::kMaxB || nseg < 1 ||
+  if (x_f32 || K < gtc::kSC || K % gtc::kSC != 0 || B < 1 || B > gtc::kMaxBatch || nseg < 1 ||
       nseg > gtc::kMaxSegs)
     return false;
   for (int i = 0; i < nseg; ++i)
     if (!aligned(segs[i].w, 32) || !aligned(segs[i].s, 4) || !aligned(segs[i].b, 4)) return false;
-  return gtc_smem(K, (B + 3) / 4, 16) <= 200 * 1024;
+  return gtc_smem(K, B > 4 ? 2 : 1, 16) <= 200 * 1024;
 }
 
 template <int NT, int W>
-static cudaError_t gtc_launch_nt(const gtc::Params& P, int grid, cudaStream_t st, bool pdl) {
+static cudaError_t gtc_launch_nt(const gtc::Params& P, dim3 grid, cudaStream_t st, bool pdl) {
   const size_t smem = gtc_smem(P.K, NT, W);
   static int attr = 0;
   if (smem > 48 * 1024 && attr < (int)smem) {
@@ -80,7 +84,7 @@ static cudaError_t gtc_launch_nt(const gtc::Params& P, int grid, cudaStream_t st
                          200 * 1024);
     attr = 200 * 1024;
   }
-  return launch_pdl(gtc::gemv_tc_kernel<NT, W>, dim3(grid), dim3(W * 32), smem, st, pdl, P);
+  return launch_pdl(gtc::gemv_tc_kernel<NT, W>, grid, dim3(W * 32), smem, st, pdl, P);
 }
 
 static cudaError_t gtc_launch(const GemvSeg* segs, int nseg, gtc::Params& P, int K, int B,
@@ -99,11 +103,13 @@ static cudaError_t gtc_launch(const GemvSeg* segs, int nseg, gtc::Params& P, int
   // 16 warps with one batch tile, 8 with two (measured: 16 is faster also
   // for the small matrices of a decode step); then split each block's
   // columns over S warps while slots stay idle
-  const int NT = (B + 3) / 4;
+  // batch tiles of 8 rows along gridDim.y past B = 8: the tiles stream the
+  // same weights at about the same time, so all but the first mostly hit L2
+  const int NT = B > 4 ? 2 : 1;
   const int sms = num_sms();
   const int W = NT == 1 ? 16 : 8;
   P.S = gtc_split(blk, K, W, sms);
-  const int grid = std::min(sms, blk);
+  const dim3 grid(std::min(sms, blk), (B + 4 * NT - 1) / (4 * NT));
   if (NT == 2) return gtc_launch_nt<2, 8>(P, grid, st, pdl);
   return gtc_launch_nt<1, 16>(P, grid, st, pdl);
 }

@@ -13,7 +13,8 @@ namespace gtc {
 constexpr int kRB = 16;        // rows per block (mma M)
 constexpr int kSC = 512;       // columns per super-chunk
 constexpr int kMaxSegs = 4;
-constexpr int kMaxB = 8;       // two n-tiles of four batch rows
+constexpr int kMaxB = 8;       // batch rows per CTA: two n-tiles of four
+constexpr int kMaxBatch = 32;  // batch rows per launch: tiles of kMaxB along gridDim.y
 
 struct Seg {
   const uint8_t* w;
@@ -141,7 +142,7 @@ __device__ __forceinline__ void chunk_mma(const uint32_t (&w)[16], const uint4& 
 }
 
 // The GEMV of one launch, for a CTA of W warps (of a grid of gridDim.x CTAs,
-// this one blockIdx.x). `wait()` runs once the first weight loads are in
+// this one blockIdx.x) and the batch tile blockIdx.y (4 NT rows each). `wait()` runs once the first weight loads are in
 // flight and before anything written upstream is read (the
 // programmatic-dependent-launch trigger and wait). smem: gtc_smem(K, NT, W)
 // bytes.
@@ -151,6 +152,8 @@ __device__ __forceinline__ void gemv_tc_body(const Params& P, uint8_t* smem, Wai
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
   const int K = P.K, Kg = K / 64, nsc = K / kSC, S = P.S;
+  // batch tile of this CTA: rows [b0, b0 + Bt) of the launch's P.B
+  const int b0 = blockIdx.y * 4 * NT, Bt = min(4 * NT, P.B - b0);
   const int xs = K + 8;  // fp16 row stride of x (pad: batch rows on other banks)
   float* red = reinterpret_cast<float*>(smem);                      // [4 NT][kWarps]
   float* part = red + 4 * NT * kWarps;                               // [2][kWarps][32][2 NT]
@@ -191,10 +194,10 @@ __device__ __forceinline__ void gemv_tc_body(const Params& P, uint8_t* smem, Wai
   if (P.xmode == kXRmsNorm) {
 #pragma unroll
     for (int b = 0; b < 4 * NT; ++b) {
-      if (b >= P.B) break;
+      if (b >= Bt) break;
       float ss = 0.f;
       for (int c = tid; c < K; c += kThreads) {
-        const float v = __ldcg(P.xa + (size_t)b * K + c);
+        const float v = __ldcg(P.xa + (size_t)(b0 + b) * K + c);
         ss = fmaf(v, v, ss);
       }
       ss = warp_sum(ss);
@@ -203,7 +206,7 @@ __device__ __forceinline__ void gemv_tc_body(const Params& P, uint8_t* smem, Wai
     __syncthreads();
 #pragma unroll
     for (int b = 0; b < 4 * NT; ++b) {
-      if (b >= P.B) break;
+      if (b >= Bt) break;
       float ss = 0.f;
       for (int w = 0; w < kWarps; ++w) ss += red[b * kWarps + w];
       inv[b] = 1.0f / sqrtf(ss / (float)K + P.eps);
@@ -216,9 +219,9 @@ __device__ __forceinline__ void gemv_tc_body(const Params& P, uint8_t* smem, Wai
   // redone on x * 2^-e. Batch rows past B are never read by a live B lane.
   auto form = [&](float down) -> float {
     float mloc = 0.f;
-    for (int i = warp; i < P.B * Kg; i += kWarps) {
+    for (int i = warp; i < Bt * Kg; i += kWarps) {
       const int b = i / Kg, c = (i - b * Kg) * 64 + 2 * lane;
-      const size_t o = (size_t)b * K + c;
+      const size_t o = (size_t)(b0 + b) * K + c;
       float v0, v1;
       if (P.xmode == kXBf16) {
         const uint32_t w2 = __ldcg(reinterpret_cast<const unsigned int*>(P.x + o));
@@ -251,7 +254,7 @@ __device__ __forceinline__ void gemv_tc_body(const Params& P, uint8_t* smem, Wai
     return mloc;
   };
   float mx = form(1.0f);
-  for (int i = P.B * Kg + tid; i < 4 * NT * Kg; i += kThreads) gsum[i] = 0.f;
+  for (int i = Bt * Kg + tid; i < 4 * NT * Kg; i += kThreads) gsum[i] = 0.f;
   // 3) max|x| over the CTA; prescale 2^-e so that max|x| * 2^-e < 2^15
   mx = warp_max(mx);
   if (lane == 0) red[warp] = mx;
@@ -273,7 +276,7 @@ __device__ __forceinline__ void gemv_tc_body(const Params& P, uint8_t* smem, Wai
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     const int b = 4 * nt + (g >> 1);
-    xl[nt] = b < P.B && (t >> 1) == (g & 1);
+    xl[nt] = b < Bt && (t >> 1) == (g & 1);
     xrow[nt] = xh + b * xs + 32 * t;
   }
 
@@ -365,8 +368,8 @@ __device__ __forceinline__ void gemv_tc_body(const Params& P, uint8_t* smem, Wai
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const int r = row0 + g + 8 * h;
-          if (b < P.B && r < Sg.N) {
-            const size_t o = (size_t)b * Sg.N + r;
+          if (b < Bt && r < Sg.N) {
+            const size_t o = (size_t)(b0 + b) * Sg.N + r;
             float v = acc[nt][h] * up;
             if (Sg.res) v += __ldcg(Sg.res + o);
             if (Sg.y_bf16)

@@ -180,12 +180,6 @@ cudaError_t attention_launch_step(const float* q, const float* k, const float* v
                                   uint16_t* kc, uint16_t* vc, const int32_t* positions, void* out,
                                   int B, int H, int Hkv, int D, int cap, float scale, void* ws,
                                   cudaStream_t st, bool pdl);
-// The split plan of the attention kernels (rows per split, splits) and the
-// three parts of an attention workspace (split outputs, split (max, sum),
-// ticket counters).
-void attention_plan(int B, int Hkv, int cap, int* ch, int* nsplit);
-void attention_ws_split(void* ws, int B, int H, int Hkv, int D, int cap, float** ws_o,
-                        float** ws_ml, unsigned int** ws_cnt);
 size_t attention_ws_bytes(int B, int H, int Hkv, int D, int cap);
 
 }  // namespace qg
