@@ -395,35 +395,50 @@ def run_ours(args):
     # ---- the other rows of the path, each timed per launch on its stream
     kernels = other_kernels(qg, stream, hbm_peak, max(20, min(100, args.steps)))
 
-    # ---- e2e through the public API with host buffers
+    # ---- e2e through the public API with host buffers: token and position
+    # in from pinned host memory, then either the greedy token (argmax on the
+    # device, 4 bytes a sequence) or the whole logits back to the host
     h_tok = torch.from_numpy(toks_np).pin_memory()
     h_pos = torch.from_numpy(pos_np).pin_memory()
     h_logits = torch.empty((B, V), dtype=torch.float32).pin_memory()
+    h_next = torch.empty(B, dtype=torch.int32).pin_memory()
+    next_tok = torch.empty(B, dtype=torch.int32, device="cuda")
+    am_ws = torch.empty(qg.qg_argmax_workspace_size(B, V), dtype=torch.uint8, device="cuda")
     e2e_steps = max(10, min(args.steps, 200))
-    with torch.cuda.stream(stream):
-        for _ in range(3):
+
+    def e2e_run(on_device_argmax):
+        def one():
             toks.copy_(h_tok, non_blocking=True)
             pos.copy_(h_pos, non_blocking=True)
             model.qg_decode_step(st, toks, pos, stream=stream)
-            h_logits.copy_(st["logits"], non_blocking=True)
-    stream.synchronize()
-    barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for _ in range(e2e_steps):
-            toks.copy_(h_tok, non_blocking=True)
-            pos.copy_(h_pos, non_blocking=True)
-            model.qg_decode_step(st, toks, pos, stream=stream)
-            h_logits.copy_(st["logits"], non_blocking=True)
-        e1.record(stream)
-    stream.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * e2e_steps / (e2e_ms / 1000.0)
+            if on_device_argmax:
+                qg.qg_argmax_f32(st["logits"], next_tok, am_ws, stream=stream)
+                h_next.copy_(next_tok, non_blocking=True)
+            else:
+                h_logits.copy_(st["logits"], non_blocking=True)
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                one()
+        stream.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(e2e_steps):
+                one()
+            e1.record(stream)
+        stream.synchronize()
+        ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([ms], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+        return world * e2e_steps / (ms / 1000.0)
+
+    e2e_value = e2e_run(True)
+    e2e_logits_value = e2e_run(False)
+    # the same step both times: the device's greedy token is the host's
+    e2e_token_ok = all(int(h_next[b]) == int(torch.argmax(h_logits[b])) for b in range(B))
 
     sb = step_bytes(cfg, B, KV_LEN)
     line = {
@@ -446,7 +461,10 @@ def run_ours(args):
                           "peak": hbm_peak, "unit": "GB/s",
                           "frac": sb / (ms_per_step / 1000.0) / 1e9 / hbm_peak},
         "e2e": {"value": e2e_value, "unit": "steps/s", "h2d_bytes_per_step": 2 * 4 * B,
-                "d2h_bytes_per_step": 4 * B * V},
+                "d2h_bytes_per_step": 4 * B, "result": "greedy token (argmax on the device)",
+                "token_matches_host_argmax": e2e_token_ok},
+        "e2e_logits": {"value": e2e_logits_value, "unit": "steps/s",
+                       "h2d_bytes_per_step": 2 * 4 * B, "d2h_bytes_per_step": 4 * B * V},
         "kernels": kernels,
         "gpu_launches": int(launches_per_step * args.steps),
         "clocks": clk.summary(),

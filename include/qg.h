@@ -65,7 +65,8 @@ int qg_abi_version(void);
 
 /* Number of CUDA kernels this library has enqueued in this process (all
  * entry points, all host threads). Capturing a call into a CUDA graph and
- * reading the count before and after gives the kernels per graph replay. */
+ * reading the count before and after gives the kernels per graph replay;
+ * a replay of a recorded step graph (qg_decode_step) adds nothing. */
 unsigned long long qg_kernel_launch_count(void);
 
 /* ------------------------------------------------------------------------
@@ -301,6 +302,15 @@ size_t qg_decode_step_workspace_size(const qg_qwen3_config* cfg, int B, int cap)
  * down GEMV (SiLU-mul in its prologue) + residual, then the LM head (final
  * RMSNorm in its prologue): 5 launches per layer plus 2. Nothing
  * synchronises or allocates, so a step can be captured in a CUDA graph.
+ * Step graphs: on a stream other than the legacy or per-thread default
+ * stream, and not while that stream is being captured, the call records
+ * its launches into a CUDA graph the first time it sees this exact set of
+ * arguments (every pointer and size, and the contents of *w and of its
+ * layer table) and replays that graph on later calls with the same set: one
+ * graph launch instead of ~140 kernel launches of host time. Up to 8 graphs
+ * are kept, the least recently used dropped first; qg_step_graphs_enable(0)
+ * turns this off and qg_step_graphs_clear() frees them. Results are the
+ * same either way (the same kernels run).
  *
  * cfg, w      HOST structs (read during the call only).
  * k_cache, v_cache device bf16 [layers][B][kv_heads][cap][head_dim].
@@ -327,6 +337,9 @@ qg_status qg_decode_step(const qg_qwen3_config* cfg, const qg_qwen3_weights* w,
                          float* logits, int B, void* ws, size_t ws_bytes,
                          void* stream);
 
+void qg_step_graphs_enable(int on);
+void qg_step_graphs_clear(void);
+
 /* Inspection aid (tests): byte offsets in the workspace of four bf16 arrays
  * that, after a step, hold the LAST decoder layer's values at its bf16
  * rounding points: offsets[0] the input-norm output [B][hidden], offsets[1]
@@ -334,6 +347,22 @@ qg_status qg_decode_step(const qg_qwen3_config* cfg, const qg_qwen3_weights* w,
  * post-attention-norm output [B][hidden], offsets[3] the SiLU-mul output
  * [B][ffn]. */
 qg_status qg_decode_step_inspect(const qg_qwen3_config* cfg, int B, int cap, size_t offsets[4]);
+
+/* ------------------------------------------------------------------------
+ * Greedy token  [TS: turbospark-runtime 0.3.0, src/qwen3_asr_metal.rs, `argmax`]
+ *   out[b] = index of the first strict maximum of logits[b][0..V), NaNs
+ *   skipped; 0 when no value beats -inf (all -inf or NaN). -0 and +0 are
+ *   equal (the first wins). The result is exact and deterministic.
+ *
+ * logits  device fp32 [B][V], 4-byte aligned.
+ * out     device int32 [B].
+ * ws      device workspace >= qg_argmax_workspace_size(B, V) bytes, 8-byte
+ *         aligned; no initialisation needed.
+ * Two launches on `stream`; 1 <= V, 0 <= B (B = 0 does nothing).
+ * ---------------------------------------------------------------------- */
+size_t qg_argmax_workspace_size(int B, int V);
+qg_status qg_argmax_f32(const float* logits, int B, int V, int32_t* out, void* ws,
+                        size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
  * Test exports: the unpack and dequant the kernels use, written out.

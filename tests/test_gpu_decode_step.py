@@ -288,3 +288,41 @@ def test_step_launch_count(shape, B):
     n0 = qg.lib.qg_kernel_launch_count()
     model.qg_decode_step(st, t, p)
     assert qg.lib.qg_kernel_launch_count() - n0 == 5 * cfg["layers"] + 2
+
+
+def test_step_graph_replay_equals_eager_launches():
+    """On a non-default stream qg_decode_step records its launches into a
+    CUDA graph once and replays it: the replay reads tokens and positions at
+    run time (a new token gives new logits), enqueues no kernel launches of
+    its own, and gives bit-identical logits and cache rows to the eager
+    launches of the same steps."""
+    cfg = dict(SMALL)
+    w = qg_synth.qwen3_weights(cfg, 24)
+    model = qg.Qwen3Model(cfg, w)
+    s = torch.cuda.Stream()
+    outs = {}
+    for mode in ("graph", "eager"):
+        qg.lib.qg_step_graphs_enable(1 if mode == "graph" else 0)
+        qg.lib.qg_step_graphs_clear()
+        st = model.new_state(2, 16)
+        t = dev(np.array([5, 900], np.int32))
+        pos = dev(np.array([0, 0], np.int32))
+        res, launches = [], []
+        for p, toks in enumerate(([5, 900], [17, 3], [17, 3], [999, 0])):
+            with torch.cuda.stream(s):
+                t.copy_(torch.tensor(toks, dtype=torch.int32))
+                pos.fill_(p)
+                n0 = qg.lib.qg_kernel_launch_count()
+                model.qg_decode_step(st, t, pos, stream=s)
+                launches.append(qg.lib.qg_kernel_launch_count() - n0)
+            s.synchronize()
+            res.append((st["logits"].clone(), st["k_cache"].clone()))
+        outs[mode] = (res, launches)
+    qg.lib.qg_step_graphs_enable(1)
+    qg.lib.qg_step_graphs_clear()
+    per_step = 5 * cfg["layers"] + 2
+    assert outs["eager"][1] == [per_step] * 4
+    assert outs["graph"][1] == [per_step, 0, 0, 0]  # recorded once, then replayed
+    for (lg, kg), (le, ke) in zip(outs["graph"][0], outs["eager"][0]):
+        assert torch.equal(lg, le) and torch.equal(kg, ke)
+    assert not torch.equal(outs["graph"][0][0][0], outs["graph"][0][1][0])

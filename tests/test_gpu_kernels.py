@@ -331,3 +331,36 @@ def test_decode_attention(B, H, Hkv, D, cap, lens):
                 assert_parity(got[b], ref, bf16_out=(od == "bf16"), what=f"attn b={b} L={L}")
             else:
                 assert np.all(got[b] == 0.0)
+
+
+# ---------------------------------------------------------- argmax -------
+
+@pytest.mark.parametrize("B,V", [(1, 1), (3, 7), (1, 151936), (4, 2048), (32, 151936), (2, 5000)])
+def test_argmax_first_strict_max_bit_exact(B, V):
+    """Index of the first strict maximum per row, NaNs skipped, 0 when no
+    value beats -inf: equal to the oracle's fold on every row, including
+    rows with repeated maxima (ties across chunks), NaNs, -0/+0 ties, +inf,
+    and rows of only -inf or only NaN."""
+    rng = np.random.default_rng(7 * B + V)
+    x = rng.standard_normal((B, V)).astype(np.float32)
+    for b in range(B):
+        kind = b % 6
+        if kind == 1 and V > 3:      # the maximum repeated, last copy in another chunk
+            m = x[b].max() + 1.0
+            x[b, [V // 3, V - 1, 2 * V // 3]] = m
+        elif kind == 2:              # NaNs everywhere but a few values
+            x[b, ::2] = np.nan
+        elif kind == 3:              # -0 and +0 as the maximum
+            x[b] = -1.0
+            x[b, V // 2:] = 0.0
+            x[b, V // 4] = -0.0
+        elif kind == 4:              # nothing beats -inf
+            x[b] = -np.inf if b % 12 == 4 else np.nan
+        elif kind == 5 and V > 1:    # +inf after a larger finite run
+            x[b, V - 1] = np.inf
+    out = torch.empty(B, dtype=torch.int32, device="cuda")
+    ws = torch.empty(qg.qg_argmax_workspace_size(B, V), dtype=torch.uint8, device="cuda")
+    qg.qg_argmax_f32(dev(x), out, ws)
+    got = out.cpu().numpy()
+    want = np.array([O.argmax_first(x[b]) for b in range(B)], dtype=np.int32)
+    np.testing.assert_array_equal(got, want)

@@ -90,6 +90,10 @@ _SIGS = {
                             _vp, _vp, _i, _vp, _vp, _vp, _i, _vp, _sz, _vp]),
     "qg_decode_step_inspect": (_i, [ctypes.POINTER(qg_qwen3_config), _i, _i,
                                     ctypes.POINTER(ctypes.c_size_t)]),
+    "qg_step_graphs_enable": (None, [_i]),
+    "qg_step_graphs_clear": (None, []),
+    "qg_argmax_workspace_size": (_sz, [_i, _i]),
+    "qg_argmax_f32": (_i, [_vp, _i, _i, _vp, _vp, _sz, _vp]),
     "qg_unpack_affine8": (_i, [_vp, _vp, _i, _i, _vp]),
     "qg_dequant_affine8_g64": (_i, [_vp, _vp, _vp, _vp, _i, _i, _vp]),
     "qg_dequant_q4_0": (_i, [_vp, _vp, _i, _i, _vp]),
@@ -208,6 +212,18 @@ def qg_decode_attention(q, k_cache, v_cache, kv_len, out, H, Hkv, scale, ws, str
     B, _, cap, D = k_cache.shape
     _call("qg_decode_attention", _p(q), _p(k_cache), _p(v_cache), _p(kv_len), _p(out), _dt(out),
           B, H, Hkv, D, cap, float(scale), _p(ws), ws.numel() * ws.element_size(),
+          _stream(stream))
+
+
+def qg_argmax_workspace_size(B, V):
+    return int(lib.qg_argmax_workspace_size(B, V))
+
+
+def qg_argmax_f32(logits, out, ws, stream=None):
+    """out[b] (int32, device) = first strict maximum of logits[b] (fp32
+    [B, V]), NaNs skipped, 0 when nothing beats -inf."""
+    B, V = logits.shape
+    _call("qg_argmax_f32", _p(logits), B, V, _p(out), _p(ws), ws.numel() * ws.element_size(),
           _stream(stream))
 
 

@@ -11,6 +11,10 @@
 // issues its first weight loads before waiting for the previous kernel, so
 // weight streaming overlaps the previous kernel's tail. Nothing here
 // synchronises or allocates, so a step can be captured into a CUDA graph.
+#include <cstring>
+#include <mutex>
+#include <vector>
+
 #include "qg_internal.cuh"
 
 namespace qg {
@@ -134,43 +138,12 @@ extern "C" size_t qg_decode_step_workspace_size(const qg_qwen3_config* cfg, int 
   return step_layout(*cfg, B, cap).total;
 }
 
-extern "C" qg_status qg_decode_step(const qg_qwen3_config* cfg, const qg_qwen3_weights* w,
-                                    uint16_t* k_cache, uint16_t* v_cache, int cap,
-                                    const int32_t* tokens, const int32_t* positions, float* logits,
-                                    int B, void* ws, size_t ws_bytes, void* stream) {
-  clear_error();
-  qg_status st = validate_cfg(cfg, B, cap);
-  if (st != QG_OK) return st;
-  const qg_qwen3_config& c = *cfg;
-  QG_REQUIRE(w, QG_ERR_INVALID_ARGUMENT, "qg_decode_step: weights is NULL");
-  QG_REQUIRE(c.layers == 0 || w->layers, QG_ERR_INVALID_ARGUMENT,
-             "qg_decode_step: weights->layers is NULL");
-  if ((st = validate_matrix(w->embed, "embed", -1)) != QG_OK) return st;
-  QG_REQUIRE(w->final_norm && aligned(w->final_norm, 2), QG_ERR_INVALID_ARGUMENT,
-             "qg_decode_step: final_norm is NULL or misaligned");
-  for (int l = 0; l < c.layers; ++l) {
-    const qg_qwen3_layer& L = w->layers[l];
-    const qg_affine8_matrix* ms[7] = {&L.q, &L.k, &L.v, &L.o, &L.gate, &L.up, &L.down};
-    const char* names[7] = {"q", "k", "v", "o", "gate", "up", "down"};
-    for (int i = 0; i < 7; ++i)
-      if ((st = validate_matrix(*ms[i], names[i], l)) != QG_OK) return st;
-    QG_REQUIRE(L.input_norm && L.post_norm && L.q_norm && L.k_norm, QG_ERR_INVALID_ARGUMENT,
-               "qg_decode_step: layer %d has a null norm weight", l);
-  }
-  QG_REQUIRE(c.layers == 0 || (k_cache && v_cache), QG_ERR_INVALID_ARGUMENT,
-             "qg_decode_step: null k_cache or v_cache");
-  QG_REQUIRE(aligned(k_cache, 16) && aligned(v_cache, 16), QG_ERR_MISALIGNED,
-             "qg_decode_step: k_cache/v_cache not 16-byte aligned");
-  QG_REQUIRE(tokens && positions && logits, QG_ERR_INVALID_ARGUMENT,
-             "qg_decode_step: null tokens, positions or logits");
-  QG_REQUIRE(aligned(tokens, 4) && aligned(positions, 4) && aligned(logits, 4), QG_ERR_MISALIGNED,
-             "qg_decode_step: tokens/positions/logits misaligned");
-  const StepLayout Ly = step_layout(c, B, cap);
-  QG_REQUIRE(ws && ws_bytes >= Ly.total, QG_ERR_WORKSPACE_TOO_SMALL,
-             "qg_decode_step: workspace of %zu bytes given, %zu needed", ws_bytes, Ly.total);
-  QG_REQUIRE(aligned(ws, 256), QG_ERR_MISALIGNED, "qg_decode_step: ws not 256-byte aligned");
-
-  cudaStream_t s = (cudaStream_t)stream;
+// Every launch of one step, in stream order on s (the eager path, and what
+// a graph capture of a step records).
+static void enqueue_step(const qg_qwen3_config& c, const qg_qwen3_weights* w, uint16_t* k_cache,
+                         uint16_t* v_cache, int cap, const int32_t* tokens,
+                         const int32_t* positions, float* logits, int B, void* ws,
+                         const StepLayout& Ly, cudaStream_t s) {
   uint8_t* base = reinterpret_cast<uint8_t*>(ws);
   float* x = reinterpret_cast<float*>(base + Ly.x);
   uint16_t* xn = reinterpret_cast<uint16_t*>(base + Ly.xn);
@@ -237,7 +210,183 @@ extern "C" qg_status qg_decode_step(const qg_qwen3_config* cfg, const qg_qwen3_w
     rmsnorm_launch(x, w->final_norm, c.eps, xnf, true, B, c.hidden, s, true);
     gemv_affine8_launch(&head, 1, xnf, false, c.hidden, B, s, true);
   }
-  return check_launch("qg_decode_step");
+}
+
+// ---------------------------------------------------------------------------
+// Step graphs. Launching a step's 5 launches per layer one by one costs host
+// time comparable to the step itself, so a call on a non-default stream that
+// is not being captured records its launches into a CUDA graph once and
+// replays that graph afterwards. The graph holds every pointer and size of
+// the call, so it is keyed on all of them, the weight tables' contents
+// included (a caller may rewrite its host weight struct in place); any
+// difference records a new graph. Up to kMaxGraphs graphs are kept, the
+// least recently used is dropped first.
+// ---------------------------------------------------------------------------
+
+namespace {
+
+constexpr size_t kMaxGraphs = 8;
+
+struct StepGraph {
+  std::vector<uint64_t> key;
+  cudaGraphExec_t exec;
+  uint64_t used;
+};
+
+std::mutex g_graph_mu;
+std::vector<StepGraph> g_graphs;
+uint64_t g_graph_tick = 0;
+bool g_graphs_on = true;
+
+void key_push(std::vector<uint64_t>& k, const void* p) { k.push_back((uint64_t)(uintptr_t)p); }
+
+std::vector<uint64_t> step_key(const qg_qwen3_config& c, const qg_qwen3_weights* w,
+                               const void* kc, const void* vc, int cap, const void* tokens,
+                               const void* positions, const void* logits, int B, const void* ws,
+                               int device) {
+  std::vector<uint64_t> k;
+  k.reserve(32 + (size_t)c.layers * 25);
+  const int ints[] = {c.hidden, c.layers, c.heads, c.kv_heads, c.head_dim, c.ffn, c.vocab, B, cap,
+                      device};
+  for (int v : ints) k.push_back((uint64_t)(uint32_t)v);
+  uint32_t eps_bits;
+  memcpy(&eps_bits, &c.eps, 4);
+  uint64_t theta_bits;
+  memcpy(&theta_bits, &c.theta, 8);
+  k.push_back(eps_bits);
+  k.push_back(theta_bits);
+  for (const void* p : {kc, vc, tokens, positions, logits, ws}) key_push(k, p);
+  key_push(k, w->embed.w);
+  key_push(k, w->embed.scales);
+  key_push(k, w->embed.biases);
+  key_push(k, w->final_norm);
+  for (int l = 0; l < c.layers; ++l) {
+    const qg_qwen3_layer& L = w->layers[l];
+    for (const qg_affine8_matrix* m : {&L.q, &L.k, &L.v, &L.o, &L.gate, &L.up, &L.down}) {
+      key_push(k, m->w);
+      key_push(k, m->scales);
+      key_push(k, m->biases);
+    }
+    for (const void* p : {(const void*)L.input_norm, (const void*)L.post_norm,
+                          (const void*)L.q_norm, (const void*)L.k_norm})
+      key_push(k, p);
+  }
+  return k;
+}
+
+}  // namespace
+
+extern "C" void qg_step_graphs_enable(int on) {
+  std::lock_guard<std::mutex> lock(g_graph_mu);
+  g_graphs_on = on != 0;
+}
+
+extern "C" void qg_step_graphs_clear(void) {
+  std::lock_guard<std::mutex> lock(g_graph_mu);
+  for (StepGraph& g : g_graphs) cudaGraphExecDestroy(g.exec);
+  g_graphs.clear();
+}
+
+extern "C" qg_status qg_decode_step(const qg_qwen3_config* cfg, const qg_qwen3_weights* w,
+                                    uint16_t* k_cache, uint16_t* v_cache, int cap,
+                                    const int32_t* tokens, const int32_t* positions, float* logits,
+                                    int B, void* ws, size_t ws_bytes, void* stream) {
+  clear_error();
+  qg_status st = validate_cfg(cfg, B, cap);
+  if (st != QG_OK) return st;
+  const qg_qwen3_config& c = *cfg;
+  QG_REQUIRE(w, QG_ERR_INVALID_ARGUMENT, "qg_decode_step: weights is NULL");
+  QG_REQUIRE(c.layers == 0 || w->layers, QG_ERR_INVALID_ARGUMENT,
+             "qg_decode_step: weights->layers is NULL");
+  if ((st = validate_matrix(w->embed, "embed", -1)) != QG_OK) return st;
+  QG_REQUIRE(w->final_norm && aligned(w->final_norm, 2), QG_ERR_INVALID_ARGUMENT,
+             "qg_decode_step: final_norm is NULL or misaligned");
+  for (int l = 0; l < c.layers; ++l) {
+    const qg_qwen3_layer& L = w->layers[l];
+    const qg_affine8_matrix* ms[7] = {&L.q, &L.k, &L.v, &L.o, &L.gate, &L.up, &L.down};
+    const char* names[7] = {"q", "k", "v", "o", "gate", "up", "down"};
+    for (int i = 0; i < 7; ++i)
+      if ((st = validate_matrix(*ms[i], names[i], l)) != QG_OK) return st;
+    QG_REQUIRE(L.input_norm && L.post_norm && L.q_norm && L.k_norm, QG_ERR_INVALID_ARGUMENT,
+               "qg_decode_step: layer %d has a null norm weight", l);
+  }
+  QG_REQUIRE(c.layers == 0 || (k_cache && v_cache), QG_ERR_INVALID_ARGUMENT,
+             "qg_decode_step: null k_cache or v_cache");
+  QG_REQUIRE(aligned(k_cache, 16) && aligned(v_cache, 16), QG_ERR_MISALIGNED,
+             "qg_decode_step: k_cache/v_cache not 16-byte aligned");
+  QG_REQUIRE(tokens && positions && logits, QG_ERR_INVALID_ARGUMENT,
+             "qg_decode_step: null tokens, positions or logits");
+  QG_REQUIRE(aligned(tokens, 4) && aligned(positions, 4) && aligned(logits, 4), QG_ERR_MISALIGNED,
+             "qg_decode_step: tokens/positions/logits misaligned");
+  const StepLayout Ly = step_layout(c, B, cap);
+  QG_REQUIRE(ws && ws_bytes >= Ly.total, QG_ERR_WORKSPACE_TOO_SMALL,
+             "qg_decode_step: workspace of %zu bytes given, %zu needed", ws_bytes, Ly.total);
+  QG_REQUIRE(aligned(ws, 256), QG_ERR_MISALIGNED, "qg_decode_step: ws not 256-byte aligned");
+
+  cudaStream_t s = (cudaStream_t)stream;
+  bool graphs_on;
+  {
+    std::lock_guard<std::mutex> lock(g_graph_mu);
+    graphs_on = g_graphs_on;
+  }
+  cudaStreamCaptureStatus cap_status = cudaStreamCaptureStatusActive;
+  int device = 0;
+  if (!graphs_on || s == nullptr || s == cudaStreamLegacy || s == cudaStreamPerThread ||
+      cudaStreamIsCapturing(s, &cap_status) != cudaSuccess ||
+      cap_status != cudaStreamCaptureStatusNone || cudaGetDevice(&device) != cudaSuccess) {
+    cudaGetLastError();
+    enqueue_step(c, w, k_cache, v_cache, cap, tokens, positions, logits, B, ws, Ly, s);
+    return check_launch("qg_decode_step");
+  }
+  std::vector<uint64_t> key =
+      step_key(c, w, k_cache, v_cache, cap, tokens, positions, logits, B, ws, device);
+  {
+    std::lock_guard<std::mutex> lock(g_graph_mu);
+    for (StepGraph& g : g_graphs) {
+      if (g.key == key) {
+        g.used = ++g_graph_tick;
+        const cudaError_t e = cudaGraphLaunch(g.exec, s);
+        if (e != cudaSuccess) {
+          set_error("qg_decode_step: %s", cudaGetErrorString(e));
+          return QG_ERR_CUDA;
+        }
+        return QG_OK;
+      }
+    }
+  }
+  // record this call's launches, then replay the recording
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+  cudaError_t e = cudaStreamBeginCapture(s, cudaStreamCaptureModeThreadLocal);
+  if (e == cudaSuccess) {
+    enqueue_step(c, w, k_cache, v_cache, cap, tokens, positions, logits, B, ws, Ly, s);
+    e = cudaStreamEndCapture(s, &graph);
+  }
+  if (e == cudaSuccess) e = cudaGraphInstantiate(&exec, graph, 0);
+  if (graph) cudaGraphDestroy(graph);
+  if (e != cudaSuccess) {  // no graph: launch eagerly
+    cudaGetLastError();
+    if (exec) cudaGraphExecDestroy(exec);
+    enqueue_step(c, w, k_cache, v_cache, cap, tokens, positions, logits, B, ws, Ly, s);
+    return check_launch("qg_decode_step");
+  }
+  e = cudaGraphLaunch(exec, s);
+  {
+    std::lock_guard<std::mutex> lock(g_graph_mu);
+    if (g_graphs.size() >= kMaxGraphs) {
+      size_t lru = 0;
+      for (size_t i = 1; i < g_graphs.size(); ++i)
+        if (g_graphs[i].used < g_graphs[lru].used) lru = i;
+      cudaGraphExecDestroy(g_graphs[lru].exec);
+      g_graphs.erase(g_graphs.begin() + lru);
+    }
+    g_graphs.push_back(StepGraph{std::move(key), exec, ++g_graph_tick});
+  }
+  if (e != cudaSuccess) {
+    set_error("qg_decode_step: %s", cudaGetErrorString(e));
+    return QG_ERR_CUDA;
+  }
+  return QG_OK;
 }
 
 extern "C" qg_status qg_decode_step_inspect(const qg_qwen3_config* cfg, int B, int cap,
