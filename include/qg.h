@@ -349,6 +349,52 @@ void qg_step_graphs_clear(void);
 qg_status qg_decode_step_inspect(const qg_qwen3_config* cfg, int B, int cap, size_t offsets[4]);
 
 /* ------------------------------------------------------------------------
+ * Code predictor  [MK: makima src/tts/qwen3/code_predictor.rs,
+ * CodePredictor::predict and CodePredictorLayer::forward]
+ *
+ * After the main model's LM head has chosen the group-0 code, the code
+ * predictor chooses codes 1..groups-1 one after another. For each group g:
+ *   x = input_proj @ bf16(concat(lm_hidden, embed_{g-1}(code[g-1])));
+ *   the cfg->layers decoder layers on x, each with a fresh KV cache (so
+ *   attention runs at position 0 over that one row);
+ *   logits_g = heads[g] @ bf16(RMSNorm(x) * final_norm);
+ *   code[g] = the first strict maximum of logits_g (as qg_argmax_f32).
+ * Everything runs on the device with no host round trip between groups.
+ *
+ * cfg        HOST: hidden, layers, heads, kv_heads (= heads on the pages),
+ *            head_dim, ffn, vocab = the codebook vocabulary, eps, theta;
+ *            shape rules as qg_decode_step.
+ * w          HOST struct: input_proj [hidden][2*hidden]; code_embed and
+ *            heads point to HOST arrays of `groups` affine8 matrices
+ *            [vocab][hidden] each (code_embed[g-1] embeds code g-1;
+ *            heads[g] scores group g; code_embed[groups-1] and heads[0] are
+ *            not used); layers a HOST array of cfg->layers layers;
+ *            final_norm bf16 [hidden]; 2 <= groups <= 64.
+ * lm_hidden  device fp32 [B][hidden]: the main model's last hidden state.
+ * code0      device int32 [B]: the group-0 codes. A code outside [0, vocab)
+ *            gives NaN logits downstream.
+ * codes      device int32 [groups][B] out; codes[0] = code0.
+ * logits     device fp32 [groups][B][vocab] out, or NULL: logits of group
+ *            g >= 1 in row g (row 0 not written).
+ * ws         >= qg_code_predict_workspace_size(cfg, B) bytes, 256-byte
+ *            aligned; no initialisation needed.
+ * Like qg_decode_step, on a non-default stream the call is recorded into a
+ * CUDA graph once and replayed (qg_step_graphs_enable / _clear apply). */
+typedef struct qg_code_predictor_weights {
+  qg_affine8_matrix input_proj;
+  const qg_affine8_matrix* code_embed;
+  const qg_affine8_matrix* heads;
+  const qg_qwen3_layer* layers;
+  const uint16_t* final_norm;
+  int groups;
+} qg_code_predictor_weights;
+
+size_t qg_code_predict_workspace_size(const qg_qwen3_config* cfg, int B);
+qg_status qg_code_predict(const qg_qwen3_config* cfg, const qg_code_predictor_weights* w,
+                          const float* lm_hidden, const int32_t* code0, int32_t* codes,
+                          float* logits, int B, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * Greedy token  [TS: turbospark-runtime 0.3.0, src/qwen3_asr_metal.rs, `argmax`]
  *   out[b] = index of the first strict maximum of logits[b][0..V), NaNs
  *   skipped; 0 when no value beats -inf (all -inf or NaN). -0 and +0 are

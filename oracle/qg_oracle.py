@@ -525,6 +525,43 @@ def new_kv_cache(cfg, cap):
             np.zeros((cfg["layers"], cfg["kv_heads"], cap, cfg["head_dim"])))
 
 
+# ---------------------------------------------------------------------------
+# The code predictor  [MK: src/tts/qwen3/code_predictor.rs]
+# ---------------------------------------------------------------------------
+
+def code_predict_group(cfg, w, lm_hidden, prev_code, g):
+    """Logits of code group ``g`` (>= 1) of [MK] ``CodePredictor::predict``
+    given the previous group's code: embed ``prev_code`` with table g-1,
+    concatenate it after ``lm_hidden``, project with ``input_proj``, run every
+    layer with a fresh KV cache (so each attends to its own row at position
+    0), final RMSNorm, head g. The concatenation feeds a GEMV and is rounded
+    to bf16 like every GEMV input here (reading: the page runs the whole
+    predictor in one dtype; this library's activations into a GEMV are
+    bf16)."""
+    emb = embed_rows(*w["code_embed"][g - 1], [prev_code])[0]
+    comb = round_bf16(np.concatenate([np.asarray(lm_hidden, dtype=np.float64), emb]))
+    x = gemv_affine8(*w["input_proj"], comb[None])[0]
+    Hkv, D = cfg["kv_heads"], cfg["head_dim"]
+    for lw in w["layers"]:
+        kc, vc = np.zeros((Hkv, 1, D)), np.zeros((Hkv, 1, D))
+        x = decode_layer(cfg, lw, x, kc, vc, 0)
+    xn = round_bf16(rmsnorm(x, w["final_norm"], cfg["eps"]))
+    return gemv_affine8(*w["heads"][g], xn[None])[0]
+
+
+def code_predict(cfg, w, lm_hidden, code0):
+    """[MK] ``CodePredictor::predict`` for one sequence: codes of groups
+    1..groups-1 chosen greedily one after another (``argmax_first``), each
+    from the previous one. Returns ``(codes, logits)``: the ``groups`` codes
+    starting with ``code0`` and the logits of groups 1.. (a list)."""
+    codes, logits = [int(code0)], []
+    for g in range(1, len(w["heads"])):
+        lg = code_predict_group(cfg, w, lm_hidden, codes[-1], g)
+        logits.append(lg)
+        codes.append(argmax_first(lg))
+    return codes, logits
+
+
 def prefix_forward(cfg, weights, token_ids):
     """Whole-prefix forward with a causal mask ([MK] ``Qwen3Model::forward``
     with the mask of ``causal_mask`` and ``Qwen3Attention::forward``): all

@@ -130,6 +130,12 @@ QWEN3_0_6B = dict(hidden=1024, layers=28, heads=16, kv_heads=8, head_dim=128,
                   ffn=3072, vocab=151936, eps=1e-6, theta=1e6)
 QWEN3_1_7B = dict(hidden=2048, layers=28, heads=16, kv_heads=8, head_dim=128,
                   ffn=6144, vocab=151936, eps=1e-6, theta=1e6)
+# The code predictor of makima's Qwen3-TTS (CodePredictorConfig defaults:
+# hidden 1024, 5 layers, 16 heads without GQA, head_dim 64, FFN 3 x hidden,
+# 16 code groups of 2048 codes, eps 1e-6; RoPE base of the main model).
+CODE_PREDICTOR = dict(hidden=1024, layers=5, heads=16, kv_heads=16, head_dim=64,
+                      ffn=3072, vocab=2048, eps=1e-6, theta=1e6)
+CODE_GROUPS = 16
 # The synthetic text decoder of the turbospark parity gate.
 QWEN3_TINY = dict(hidden=64, layers=2, heads=2, kv_heads=1, head_dim=64,
                   ffn=128, vocab=261, eps=1e-5, theta=1e4)
@@ -172,3 +178,18 @@ def qwen3_weights(cfg: dict, seed: int, fixture: bool = False, norm_jitter: floa
         lw["k_norm"] = norm(D, base + 13)
         out["layers"].append(lw)
     return out
+
+
+def code_predictor_weights(cfg: dict, groups: int, seed: int, norm_jitter: float = 0.0):
+    """Random-init packed weights for a code predictor: the decoder layers
+    and final norm of ``qwen3_weights`` (its embedding table unused), plus
+    ``input_proj`` [hidden][2 hidden] and ``groups`` code-embedding tables
+    and output heads [vocab][hidden] (affine8 triples)."""
+    base = qwen3_weights(cfg, seed, norm_jitter=norm_jitter)
+    h, V = cfg["hidden"], cfg["vocab"]
+    sd = seed * 1000 + 900
+    return {"input_proj": affine8_packed(h, 2 * h, sd),
+            "code_embed": [affine8_packed(V, h, sd + 1 + g) for g in range(groups)],
+            "heads": [affine8_packed(V, h, sd + 101 + g) for g in range(groups)],
+            "layers": base["layers"], "final_norm": base["final_norm"]}
+

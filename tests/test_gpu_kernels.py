@@ -306,6 +306,8 @@ ATTN_CASES = [
     (1, 4, 2, 96, 50, [50]),                    # head_dim 96: the split kernel
     (32, 16, 8, 128, 16, [16, 1, 2, 15] * 8),   # many sequences, one-CTA clusters
     (1, 2, 2, 32, 1000, [999]),                 # head_dim 32, long chunks
+    (2, 16, 16, 64, 1, [1, 1]),                 # MHA, head_dim 64, one row (code predictor)
+    (1, 16, 16, 64, 300, [300]),                # MHA, head_dim 64
 ]
 
 

@@ -438,3 +438,32 @@ def test_lm_head_tie_bound_is_the_exact_linear_effect_of_each_tie():
         xa[j] = alt[j]
         brute += np.abs(O.gemv_affine8(*w["embed"], xa[None])[0] - logits)
     np.testing.assert_allclose(ex, brute, rtol=1e-9, atol=1e-12)
+
+
+def test_code_predict_chain_indices_and_concat_order():
+    """A code predictor built by hand (no layers, hidden = vocab = 64, 4 code
+    groups): input_proj = [0 | I] passes the code embedding through and drops
+    the LM hidden state; table j maps code t to a one-hot at (t + j) mod 64;
+    head g maps a one-hot at c to the logit row (c + 10 g) mod 64. So group
+    g's code is (previous + (g - 1) + 10 g) mod 64: from 5 the chain is 15,
+    36, 4. Using table g or head g - 1, or the concatenation in the other
+    order, gives another chain."""
+    h = V = 64
+    G = 4
+    cfg = dict(hidden=h, layers=0, heads=1, kv_heads=1, head_dim=64, ffn=64, vocab=V,
+               eps=1e-6, theta=1e6)
+    eye = np.eye(h)
+    ip = np.concatenate([np.zeros((h, h)), eye], axis=1)
+    tables = [np.roll(eye, j, axis=1) for j in range(G)]       # row t: one-hot at t + j
+    heads = [np.roll(eye, 10 * g, axis=0) for g in range(G)]   # column c -> row c + 10 g
+    w = {"input_proj": O.affine8_quantize(ip),
+         "code_embed": [O.affine8_quantize(t) for t in tables],
+         "heads": [O.affine8_quantize(m) for m in heads],
+         "layers": [], "final_norm": np.full(h, 0x3F80, dtype=np.uint16)}
+    lm_hidden = qg_synth.gaussian((h,), 1.0, 3)
+    codes, logits = O.code_predict(cfg, w, lm_hidden, 5)
+    assert codes == [5, 15, 36, 4]
+    assert len(logits) == G - 1 and all(lg.shape == (V,) for lg in logits)
+    # group 1's logits directly: one nonzero logit, at 15
+    lg = O.code_predict_group(cfg, w, lm_hidden, 5, 1)
+    assert np.count_nonzero(lg > 1.0) == 1 and int(np.argmax(lg)) == 15

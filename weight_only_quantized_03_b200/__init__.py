@@ -64,6 +64,13 @@ class qg_qwen3_weights(ctypes.Structure):
                 ("layers", ctypes.POINTER(qg_qwen3_layer))]
 
 
+class qg_code_predictor_weights(ctypes.Structure):
+    _fields_ = [("input_proj", qg_affine8_matrix),
+                ("code_embed", ctypes.POINTER(qg_affine8_matrix)),
+                ("heads", ctypes.POINTER(qg_affine8_matrix)),
+                ("layers", ctypes.POINTER(qg_qwen3_layer)), ("final_norm", _vp), ("groups", _i)]
+
+
 _SIGS = {
     "qg_last_error": (ctypes.c_char_p, []),
     "qg_abi_version": (_i, []),
@@ -90,6 +97,10 @@ _SIGS = {
                             _vp, _vp, _i, _vp, _vp, _vp, _i, _vp, _sz, _vp]),
     "qg_decode_step_inspect": (_i, [ctypes.POINTER(qg_qwen3_config), _i, _i,
                                     ctypes.POINTER(ctypes.c_size_t)]),
+    "qg_code_predict_workspace_size": (_sz, [ctypes.POINTER(qg_qwen3_config), _i]),
+    "qg_code_predict": (_i, [ctypes.POINTER(qg_qwen3_config),
+                             ctypes.POINTER(qg_code_predictor_weights), _vp, _vp, _vp, _vp, _i,
+                             _vp, _sz, _vp]),
     "qg_step_graphs_enable": (None, [_i]),
     "qg_step_graphs_clear": (None, []),
     "qg_argmax_workspace_size": (_sz, [_i, _i]),
@@ -337,3 +348,57 @@ class Qwen3Model:
               _p(state["k_cache"]), _p(state["v_cache"]), state["cap"], _p(tokens),
               _p(positions), _p(state["logits"]), state["B"], _p(state["ws"]),
               state["ws"].numel(), _stream(stream))
+
+
+class CodePredictor:
+    """Device-resident packed code-predictor weights (the host dict layout of
+    ``qg_synth.code_predictor_weights``) and ``qg_code_predict``."""
+
+    def __init__(self, cfg: dict, weights: dict, device="cuda"):
+        self.cfg = dict(cfg)
+        self._keep = []
+
+        def up(a):
+            t = torch.from_numpy(a.view({2: "int16", 4: "int32"}[a.dtype.itemsize])).to(device)
+            self._keep.append(t)
+            return t.data_ptr()
+
+        def mat(triple):
+            w, s, b = triple
+            return qg_affine8_matrix(up(w), up(s), up(b))
+
+        self.c_cfg = qg_qwen3_config(cfg["hidden"], cfg["layers"], cfg["heads"], cfg["kv_heads"],
+                                     cfg["head_dim"], cfg["ffn"], cfg["vocab"], cfg["eps"],
+                                     cfg["theta"])
+        G = len(weights["heads"])
+        self.groups = G
+        self.c_embed = (qg_affine8_matrix * G)(*[mat(t) for t in weights["code_embed"]])
+        self.c_heads = (qg_affine8_matrix * G)(*[mat(t) for t in weights["heads"]])
+        L = cfg["layers"]
+        self.c_layers = (qg_qwen3_layer * max(L, 1))()
+        for i, lw in enumerate(weights["layers"]):
+            cl = self.c_layers[i]
+            cl.input_norm = up(lw["input_norm"])
+            cl.post_norm = up(lw["post_norm"])
+            cl.q_norm = up(lw["q_norm"])
+            cl.k_norm = up(lw["k_norm"])
+            for n in ("q", "k", "v", "o", "gate", "up", "down"):
+                setattr(cl, n, mat(lw[n]))
+        self.c_weights = qg_code_predictor_weights(
+            mat(weights["input_proj"]), ctypes.cast(self.c_embed, ctypes.POINTER(qg_affine8_matrix)),
+            ctypes.cast(self.c_heads, ctypes.POINTER(qg_affine8_matrix)),
+            ctypes.cast(self.c_layers, ctypes.POINTER(qg_qwen3_layer)), up(weights["final_norm"]), G)
+        self.device = device
+
+    def workspace(self, B):
+        n = int(lib.qg_code_predict_workspace_size(ctypes.byref(self.c_cfg), B))
+        return torch.empty(n, dtype=torch.uint8, device=self.device)
+
+    def qg_code_predict(self, lm_hidden, code0, codes, ws, logits=None, stream=None):
+        """lm_hidden fp32 [B, hidden], code0 int32 [B] (device) -> codes int32
+        [groups, B]; logits fp32 [groups, B, vocab] when given."""
+        B = lm_hidden.shape[0]
+        _call("qg_code_predict", ctypes.byref(self.c_cfg), ctypes.byref(self.c_weights),
+              _p(lm_hidden), _p(code0), _p(codes), _p(logits), B, _p(ws),
+              ws.numel(), _stream(stream))
+

@@ -138,78 +138,112 @@ extern "C" size_t qg_decode_step_workspace_size(const qg_qwen3_config* cfg, int 
   return step_layout(*cfg, B, cap).total;
 }
 
+// The step's buffers inside its workspace.
+struct StepBufs {
+  float* x;
+  uint16_t *xn, *xn2, *xnf;
+  float *q, *k, *v;
+  uint16_t* attn;
+  float *gate, *up;
+  uint16_t* hm;
+  void* aws;
+  float2* rope;
+};
+
+static StepBufs step_bufs(void* ws, const StepLayout& Ly) {
+  uint8_t* base = reinterpret_cast<uint8_t*>(ws);
+  StepBufs b;
+  b.x = reinterpret_cast<float*>(base + Ly.x);
+  b.xn = reinterpret_cast<uint16_t*>(base + Ly.xn);
+  b.xn2 = reinterpret_cast<uint16_t*>(base + Ly.xn2);
+  b.xnf = reinterpret_cast<uint16_t*>(base + Ly.xnf);
+  b.q = reinterpret_cast<float*>(base + Ly.q);
+  b.k = reinterpret_cast<float*>(base + Ly.k);
+  b.v = reinterpret_cast<float*>(base + Ly.v);
+  b.attn = reinterpret_cast<uint16_t*>(base + Ly.attn);
+  b.gate = reinterpret_cast<float*>(base + Ly.gate);
+  b.up = reinterpret_cast<float*>(base + Ly.up);
+  b.hm = reinterpret_cast<uint16_t*>(base + Ly.h);
+  b.aws = base + Ly.attn_ws;
+  b.rope = reinterpret_cast<float2*>(base + Ly.rope);
+  return b;
+}
+
+// The decoder layers on the residual stream sb.x (5 launches a layer where
+// the tensor-core GEMV takes the shapes), in stream order on s.
+static void enqueue_layers(const qg_qwen3_config& c, const qg_qwen3_layer* layers,
+                           uint16_t* k_cache, uint16_t* v_cache, int cap, const int32_t* tokens,
+                           const int32_t* positions, int B, const StepBufs& sb, cudaStream_t s) {
+  const int H = c.heads, Hkv = c.kv_heads, D = c.head_dim;
+  const size_t layer_cache = (size_t)B * Hkv * cap * D;
+  const float scale = 1.0f / sqrtf((float)D);
+  float* x = sb.x;
+  for (int l = 0; l < c.layers; ++l) {
+    const qg_qwen3_layer& L = layers[l];
+    uint16_t* kc = k_cache + l * layer_cache;
+    uint16_t* vc = v_cache + l * layer_cache;
+    GemvSeg qkv[3] = {{L.q.w, L.q.scales, L.q.biases, sb.q, nullptr, H * D, 0},
+                      {L.k.w, L.k.scales, L.k.biases, sb.k, nullptr, Hkv * D, 0},
+                      {L.v.w, L.v.scales, L.v.biases, sb.v, nullptr, Hkv * D, 0}};
+    // RMSNorm and SiLU-mul run in the next GEMV's prologue where the
+    // tensor-core GEMV takes the shape, as separate kernels otherwise
+    if (gemv_tc_eligible(qkv, 3, c.hidden, B, false)) {
+      gemv_tc_launch_rmsnorm(qkv, 3, x, L.input_norm, c.eps, c.hidden, B, s, true, sb.xn);
+    } else {
+      rmsnorm_launch(x, L.input_norm, c.eps, sb.xn, true, B, c.hidden, s, true);
+      gemv_affine8_launch(qkv, 3, sb.xn, false, c.hidden, B, s, true);
+    }
+    attention_launch_step(sb.q, sb.k, sb.v, L.q_norm, L.k_norm, tokens, c.vocab, c.eps, sb.rope,
+                          kc, vc, positions, sb.attn, B, H, Hkv, D, cap, scale, sb.aws, s, true);
+    GemvSeg o = {L.o.w, L.o.scales, L.o.biases, x, x, c.hidden, 0};
+    gemv_affine8_launch(&o, 1, sb.attn, false, H * D, B, s, true);
+    GemvSeg gu[2] = {{L.gate.w, L.gate.scales, L.gate.biases, sb.gate, nullptr, c.ffn, 0},
+                     {L.up.w, L.up.scales, L.up.biases, sb.up, nullptr, c.ffn, 0}};
+    if (gemv_tc_eligible(gu, 2, c.hidden, B, false)) {
+      gemv_tc_launch_rmsnorm(gu, 2, x, L.post_norm, c.eps, c.hidden, B, s, true, sb.xn2);
+    } else {
+      rmsnorm_launch(x, L.post_norm, c.eps, sb.xn2, true, B, c.hidden, s, true);
+      gemv_affine8_launch(gu, 2, sb.xn2, false, c.hidden, B, s, true);
+    }
+    GemvSeg dn = {L.down.w, L.down.scales, L.down.biases, x, x, c.hidden, 0};
+    if (gemv_tc_eligible(&dn, 1, c.ffn, B, false)) {
+      gemv_tc_launch_silu_mul(&dn, 1, sb.gate, sb.up, c.ffn, B, s, true, sb.hm);
+    } else {
+      const int n = B * c.ffn;
+      launch_pdl(step_silu_mul_kernel, dim3((n + 255) / 256), dim3(256), 0, s, true,
+                 (const float*)sb.gate, (const float*)sb.up, sb.hm, n);
+      gemv_affine8_launch(&dn, 1, sb.hm, false, c.ffn, B, s, true);
+    }
+  }
+}
+
+// Final RMSNorm and an output head [N][hidden] on sb.x: logits [B][N].
+static void enqueue_head(const qg_qwen3_config& c, const qg_affine8_matrix& head, int N,
+                         const uint16_t* final_norm, float* logits, int B, const StepBufs& sb,
+                         cudaStream_t s) {
+  GemvSeg h = {head.w, head.scales, head.biases, logits, nullptr, N, 0};
+  if (gemv_tc_eligible(&h, 1, c.hidden, B, false)) {
+    gemv_tc_launch_rmsnorm(&h, 1, sb.x, final_norm, c.eps, c.hidden, B, s, true);
+  } else {
+    rmsnorm_launch(sb.x, final_norm, c.eps, sb.xnf, true, B, c.hidden, s, true);
+    gemv_affine8_launch(&h, 1, sb.xnf, false, c.hidden, B, s, true);
+  }
+}
+
 // Every launch of one step, in stream order on s (the eager path, and what
-// a graph capture of a step records).
+// a graph recording of a step holds).
 static void enqueue_step(const qg_qwen3_config& c, const qg_qwen3_weights* w, uint16_t* k_cache,
                          uint16_t* v_cache, int cap, const int32_t* tokens,
                          const int32_t* positions, float* logits, int B, void* ws,
                          const StepLayout& Ly, cudaStream_t s) {
-  uint8_t* base = reinterpret_cast<uint8_t*>(ws);
-  float* x = reinterpret_cast<float*>(base + Ly.x);
-  uint16_t* xn = reinterpret_cast<uint16_t*>(base + Ly.xn);
-  uint16_t* xn2 = reinterpret_cast<uint16_t*>(base + Ly.xn2);
-  uint16_t* xnf = reinterpret_cast<uint16_t*>(base + Ly.xnf);
-  float* q = reinterpret_cast<float*>(base + Ly.q);
-  float* k = reinterpret_cast<float*>(base + Ly.k);
-  float* v = reinterpret_cast<float*>(base + Ly.v);
-  uint16_t* attn = reinterpret_cast<uint16_t*>(base + Ly.attn);
-  float* gate = reinterpret_cast<float*>(base + Ly.gate);
-  float* up = reinterpret_cast<float*>(base + Ly.up);
-  uint16_t* hm = reinterpret_cast<uint16_t*>(base + Ly.h);
-  void* aws = base + Ly.attn_ws;
-  const int H = c.heads, Hkv = c.kv_heads, D = c.head_dim;
-  const size_t cnt_off = attention_ws_counter_offset(B, H, Hkv, D, cap);
-  const size_t layer_cache = (size_t)B * Hkv * cap * D;
-  const float scale = 1.0f / sqrtf((float)D);
-
-  cudaMemsetAsync(reinterpret_cast<uint8_t*>(aws) + cnt_off, 0, (size_t)B * Hkv * 4, s);
-  float2* rope = reinterpret_cast<float2*>(base + Ly.rope);
+  const StepBufs sb = step_bufs(ws, Ly);
+  const size_t cnt_off = attention_ws_counter_offset(B, c.heads, c.kv_heads, c.head_dim, cap);
+  cudaMemsetAsync(reinterpret_cast<uint8_t*>(sb.aws) + cnt_off, 0, (size_t)B * c.kv_heads * 4, s);
   launch_pdl(step_embed_kernel, dim3(B), dim3(256), 0, s, true, w->embed.w, w->embed.scales,
-             w->embed.biases, tokens, positions, x, c.vocab, c.hidden, cap, rope, D, c.theta);
-  for (int l = 0; l < c.layers; ++l) {
-    const qg_qwen3_layer& L = w->layers[l];
-    uint16_t* kc = k_cache + l * layer_cache;
-    uint16_t* vc = v_cache + l * layer_cache;
-    GemvSeg qkv[3] = {{L.q.w, L.q.scales, L.q.biases, q, nullptr, H * D, 0},
-                      {L.k.w, L.k.scales, L.k.biases, k, nullptr, Hkv * D, 0},
-                      {L.v.w, L.v.scales, L.v.biases, v, nullptr, Hkv * D, 0}};
-    // RMSNorm and SiLU-mul run in the next GEMV's prologue where the
-    // tensor-core GEMV takes the shape, as separate kernels otherwise
-    if (gemv_tc_eligible(qkv, 3, c.hidden, B, false)) {
-      gemv_tc_launch_rmsnorm(qkv, 3, x, L.input_norm, c.eps, c.hidden, B, s, true, xn);
-    } else {
-      rmsnorm_launch(x, L.input_norm, c.eps, xn, true, B, c.hidden, s, true);
-      gemv_affine8_launch(qkv, 3, xn, false, c.hidden, B, s, true);
-    }
-    attention_launch_step(q, k, v, L.q_norm, L.k_norm, tokens, c.vocab, c.eps, rope, kc, vc,
-                          positions, attn, B, H, Hkv, D, cap, scale, aws, s, true);
-    GemvSeg o = {L.o.w, L.o.scales, L.o.biases, x, x, c.hidden, 0};
-    gemv_affine8_launch(&o, 1, attn, false, H * D, B, s, true);
-    GemvSeg gu[2] = {{L.gate.w, L.gate.scales, L.gate.biases, gate, nullptr, c.ffn, 0},
-                     {L.up.w, L.up.scales, L.up.biases, up, nullptr, c.ffn, 0}};
-    if (gemv_tc_eligible(gu, 2, c.hidden, B, false)) {
-      gemv_tc_launch_rmsnorm(gu, 2, x, L.post_norm, c.eps, c.hidden, B, s, true, xn2);
-    } else {
-      rmsnorm_launch(x, L.post_norm, c.eps, xn2, true, B, c.hidden, s, true);
-      gemv_affine8_launch(gu, 2, xn2, false, c.hidden, B, s, true);
-    }
-    GemvSeg dn = {L.down.w, L.down.scales, L.down.biases, x, x, c.hidden, 0};
-    if (gemv_tc_eligible(&dn, 1, c.ffn, B, false)) {
-      gemv_tc_launch_silu_mul(&dn, 1, gate, up, c.ffn, B, s, true, hm);
-    } else {
-      const int n = B * c.ffn;
-      launch_pdl(step_silu_mul_kernel, dim3((n + 255) / 256), dim3(256), 0, s, true,
-                 (const float*)gate, (const float*)up, hm, n);
-      gemv_affine8_launch(&dn, 1, hm, false, c.ffn, B, s, true);
-    }
-  }
-  GemvSeg head = {w->embed.w, w->embed.scales, w->embed.biases, logits, nullptr, c.vocab, 0};
-  if (gemv_tc_eligible(&head, 1, c.hidden, B, false)) {
-    gemv_tc_launch_rmsnorm(&head, 1, x, w->final_norm, c.eps, c.hidden, B, s, true);
-  } else {
-    rmsnorm_launch(x, w->final_norm, c.eps, xnf, true, B, c.hidden, s, true);
-    gemv_affine8_launch(&head, 1, xnf, false, c.hidden, B, s, true);
-  }
+             w->embed.biases, tokens, positions, sb.x, c.vocab, c.hidden, cap, sb.rope, c.head_dim,
+             c.theta);
+  enqueue_layers(c, w->layers, k_cache, v_cache, cap, tokens, positions, B, sb, s);
+  enqueue_head(c, w->embed, c.vocab, w->final_norm, logits, B, sb, s);
 }
 
 // ---------------------------------------------------------------------------
@@ -240,14 +274,8 @@ bool g_graphs_on = true;
 
 void key_push(std::vector<uint64_t>& k, const void* p) { k.push_back((uint64_t)(uintptr_t)p); }
 
-std::vector<uint64_t> step_key(const qg_qwen3_config& c, const qg_qwen3_weights* w,
-                               const void* kc, const void* vc, int cap, const void* tokens,
-                               const void* positions, const void* logits, int B, const void* ws,
-                               int device) {
-  std::vector<uint64_t> k;
-  k.reserve(32 + (size_t)c.layers * 25);
-  const int ints[] = {c.hidden, c.layers, c.heads, c.kv_heads, c.head_dim, c.ffn, c.vocab, B, cap,
-                      device};
+void key_cfg(std::vector<uint64_t>& k, const qg_qwen3_config& c, int B, int cap) {
+  const int ints[] = {c.hidden, c.layers, c.heads, c.kv_heads, c.head_dim, c.ffn, c.vocab, B, cap};
   for (int v : ints) k.push_back((uint64_t)(uint32_t)v);
   uint32_t eps_bits;
   memcpy(&eps_bits, &c.eps, 4);
@@ -255,22 +283,36 @@ std::vector<uint64_t> step_key(const qg_qwen3_config& c, const qg_qwen3_weights*
   memcpy(&theta_bits, &c.theta, 8);
   k.push_back(eps_bits);
   k.push_back(theta_bits);
-  for (const void* p : {kc, vc, tokens, positions, logits, ws}) key_push(k, p);
-  key_push(k, w->embed.w);
-  key_push(k, w->embed.scales);
-  key_push(k, w->embed.biases);
-  key_push(k, w->final_norm);
-  for (int l = 0; l < c.layers; ++l) {
-    const qg_qwen3_layer& L = w->layers[l];
-    for (const qg_affine8_matrix* m : {&L.q, &L.k, &L.v, &L.o, &L.gate, &L.up, &L.down}) {
-      key_push(k, m->w);
-      key_push(k, m->scales);
-      key_push(k, m->biases);
-    }
+}
+
+void key_matrix(std::vector<uint64_t>& k, const qg_affine8_matrix& m) {
+  key_push(k, m.w);
+  key_push(k, m.scales);
+  key_push(k, m.biases);
+}
+
+void key_layers(std::vector<uint64_t>& k, const qg_qwen3_layer* layers, int n) {
+  for (int l = 0; l < n; ++l) {
+    const qg_qwen3_layer& L = layers[l];
+    for (const qg_affine8_matrix* m : {&L.q, &L.k, &L.v, &L.o, &L.gate, &L.up, &L.down})
+      key_matrix(k, *m);
     for (const void* p : {(const void*)L.input_norm, (const void*)L.post_norm,
                           (const void*)L.q_norm, (const void*)L.k_norm})
       key_push(k, p);
   }
+}
+
+std::vector<uint64_t> step_key(const qg_qwen3_config& c, const qg_qwen3_weights* w,
+                               const void* kc, const void* vc, int cap, const void* tokens,
+                               const void* positions, const void* logits, int B, const void* ws) {
+  std::vector<uint64_t> k;
+  k.reserve(32 + (size_t)c.layers * 25);
+  k.push_back(1);  // what: a decode step
+  key_cfg(k, c, B, cap);
+  for (const void* p : {kc, vc, tokens, positions, logits, ws}) key_push(k, p);
+  key_matrix(k, w->embed);
+  key_push(k, w->final_norm);
+  key_layers(k, w->layers, c.layers);
   return k;
 }
 
@@ -285,6 +327,76 @@ extern "C" void qg_step_graphs_clear(void) {
   std::lock_guard<std::mutex> lock(g_graph_mu);
   for (StepGraph& g : g_graphs) cudaGraphExecDestroy(g.exec);
   g_graphs.clear();
+}
+
+// Runs `enqueue` on stream s: replayed from a recorded graph keyed on `key`
+// when the stream allows it (recorded on first use), launched eagerly
+// otherwise or when recording fails.
+template <class Enqueue>
+static qg_status run_recorded(std::vector<uint64_t> key, cudaStream_t s, Enqueue&& enqueue,
+                              const char* what) {
+  bool graphs_on;
+  {
+    std::lock_guard<std::mutex> lock(g_graph_mu);
+    graphs_on = g_graphs_on;
+  }
+  cudaStreamCaptureStatus cap_status = cudaStreamCaptureStatusActive;
+  int device = 0;
+  if (!graphs_on || s == nullptr || s == cudaStreamLegacy || s == cudaStreamPerThread ||
+      cudaStreamIsCapturing(s, &cap_status) != cudaSuccess ||
+      cap_status != cudaStreamCaptureStatusNone || cudaGetDevice(&device) != cudaSuccess) {
+    cudaGetLastError();
+    enqueue();
+    return check_launch(what);
+  }
+  key.push_back((uint64_t)(uint32_t)device);
+  {
+    std::lock_guard<std::mutex> lock(g_graph_mu);
+    for (StepGraph& g : g_graphs) {
+      if (g.key == key) {
+        g.used = ++g_graph_tick;
+        const cudaError_t e = cudaGraphLaunch(g.exec, s);
+        if (e != cudaSuccess) {
+          set_error("%s: %s", what, cudaGetErrorString(e));
+          return QG_ERR_CUDA;
+        }
+        return QG_OK;
+      }
+    }
+  }
+  // record this call's launches, then replay the recording
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+  cudaError_t e = cudaStreamBeginCapture(s, cudaStreamCaptureModeThreadLocal);
+  if (e == cudaSuccess) {
+    enqueue();
+    e = cudaStreamEndCapture(s, &graph);
+  }
+  if (e == cudaSuccess) e = cudaGraphInstantiate(&exec, graph, 0);
+  if (graph) cudaGraphDestroy(graph);
+  if (e != cudaSuccess) {  // no graph: launch eagerly
+    cudaGetLastError();
+    if (exec) cudaGraphExecDestroy(exec);
+    enqueue();
+    return check_launch(what);
+  }
+  e = cudaGraphLaunch(exec, s);
+  {
+    std::lock_guard<std::mutex> lock(g_graph_mu);
+    if (g_graphs.size() >= kMaxGraphs) {
+      size_t lru = 0;
+      for (size_t i = 1; i < g_graphs.size(); ++i)
+        if (g_graphs[i].used < g_graphs[lru].used) lru = i;
+      cudaGraphExecDestroy(g_graphs[lru].exec);
+      g_graphs.erase(g_graphs.begin() + lru);
+    }
+    g_graphs.push_back(StepGraph{std::move(key), exec, ++g_graph_tick});
+  }
+  if (e != cudaSuccess) {
+    set_error("%s: %s", what, cudaGetErrorString(e));
+    return QG_ERR_CUDA;
+  }
+  return QG_OK;
 }
 
 extern "C" qg_status qg_decode_step(const qg_qwen3_config* cfg, const qg_qwen3_weights* w,
@@ -324,69 +436,12 @@ extern "C" qg_status qg_decode_step(const qg_qwen3_config* cfg, const qg_qwen3_w
   QG_REQUIRE(aligned(ws, 256), QG_ERR_MISALIGNED, "qg_decode_step: ws not 256-byte aligned");
 
   cudaStream_t s = (cudaStream_t)stream;
-  bool graphs_on;
-  {
-    std::lock_guard<std::mutex> lock(g_graph_mu);
-    graphs_on = g_graphs_on;
-  }
-  cudaStreamCaptureStatus cap_status = cudaStreamCaptureStatusActive;
-  int device = 0;
-  if (!graphs_on || s == nullptr || s == cudaStreamLegacy || s == cudaStreamPerThread ||
-      cudaStreamIsCapturing(s, &cap_status) != cudaSuccess ||
-      cap_status != cudaStreamCaptureStatusNone || cudaGetDevice(&device) != cudaSuccess) {
-    cudaGetLastError();
-    enqueue_step(c, w, k_cache, v_cache, cap, tokens, positions, logits, B, ws, Ly, s);
-    return check_launch("qg_decode_step");
-  }
-  std::vector<uint64_t> key =
-      step_key(c, w, k_cache, v_cache, cap, tokens, positions, logits, B, ws, device);
-  {
-    std::lock_guard<std::mutex> lock(g_graph_mu);
-    for (StepGraph& g : g_graphs) {
-      if (g.key == key) {
-        g.used = ++g_graph_tick;
-        const cudaError_t e = cudaGraphLaunch(g.exec, s);
-        if (e != cudaSuccess) {
-          set_error("qg_decode_step: %s", cudaGetErrorString(e));
-          return QG_ERR_CUDA;
-        }
-        return QG_OK;
-      }
-    }
-  }
-  // record this call's launches, then replay the recording
-  cudaGraph_t graph = nullptr;
-  cudaGraphExec_t exec = nullptr;
-  cudaError_t e = cudaStreamBeginCapture(s, cudaStreamCaptureModeThreadLocal);
-  if (e == cudaSuccess) {
-    enqueue_step(c, w, k_cache, v_cache, cap, tokens, positions, logits, B, ws, Ly, s);
-    e = cudaStreamEndCapture(s, &graph);
-  }
-  if (e == cudaSuccess) e = cudaGraphInstantiate(&exec, graph, 0);
-  if (graph) cudaGraphDestroy(graph);
-  if (e != cudaSuccess) {  // no graph: launch eagerly
-    cudaGetLastError();
-    if (exec) cudaGraphExecDestroy(exec);
-    enqueue_step(c, w, k_cache, v_cache, cap, tokens, positions, logits, B, ws, Ly, s);
-    return check_launch("qg_decode_step");
-  }
-  e = cudaGraphLaunch(exec, s);
-  {
-    std::lock_guard<std::mutex> lock(g_graph_mu);
-    if (g_graphs.size() >= kMaxGraphs) {
-      size_t lru = 0;
-      for (size_t i = 1; i < g_graphs.size(); ++i)
-        if (g_graphs[i].used < g_graphs[lru].used) lru = i;
-      cudaGraphExecDestroy(g_graphs[lru].exec);
-      g_graphs.erase(g_graphs.begin() + lru);
-    }
-    g_graphs.push_back(StepGraph{std::move(key), exec, ++g_graph_tick});
-  }
-  if (e != cudaSuccess) {
-    set_error("qg_decode_step: %s", cudaGetErrorString(e));
-    return QG_ERR_CUDA;
-  }
-  return QG_OK;
+  return run_recorded(step_key(c, w, k_cache, v_cache, cap, tokens, positions, logits, B, ws), s,
+                      [&] {
+                        enqueue_step(c, w, k_cache, v_cache, cap, tokens, positions, logits, B,
+                                     ws, Ly, s);
+                      },
+                      "qg_decode_step");
 }
 
 extern "C" qg_status qg_decode_step_inspect(const qg_qwen3_config* cfg, int B, int cap,
@@ -401,4 +456,166 @@ extern "C" qg_status qg_decode_step_inspect(const qg_qwen3_config* cfg, int B, i
   offsets[2] = Ly.xn2;
   offsets[3] = Ly.h;
   return QG_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Code predictor: makima src/tts/qwen3/code_predictor.rs, CodePredictor::
+// predict. Per group g = 1 .. groups-1: embed code g-1 with table g-1,
+// concatenate it after the main model's hidden state, project with
+// input_proj, run the layers (each with a fresh KV cache: one row at
+// position 0), final norm, head g, greedy code. The concatenated input is a
+// GEMV input and is stored as bf16, like every activation that feeds a GEMV
+// in this library.
+// ---------------------------------------------------------------------------
+
+namespace qg {
+
+// codes[0] = code0 and every sequence's position 0; the RoPE table of
+// position 0 (all angles 0).
+__global__ void cp_start_kernel(const int32_t* __restrict__ code0, int32_t* __restrict__ codes0,
+                                int32_t* __restrict__ pos, float2* __restrict__ rope, int D) {
+  pdl_wait();
+  const int b = blockIdx.x;
+  if (threadIdx.x == 0) {
+    codes0[b] = code0[b];
+    pos[b] = 0;
+  }
+  for (int i = threadIdx.x; i < D / 2; i += blockDim.x)
+    rope[(size_t)b * (D / 2) + i] = make_float2(1.0f, 0.0f);
+}
+
+// bf16(concat(lm_hidden[b], embed(prev[b]))) [B][2 hidden]; an out-of-range
+// code gives NaN in its half.
+__global__ void cp_input_kernel(const float* __restrict__ lm_hidden, const uint32_t* __restrict__ ew,
+                                const uint16_t* __restrict__ es, const uint16_t* __restrict__ eb,
+                                const int32_t* __restrict__ prev, uint16_t* __restrict__ out,
+                                int hidden, int vocab) {
+  pdl_wait();
+  const int b = blockIdx.x;
+  const int t = __ldcg(prev + b);
+  const bool ok = t >= 0 && t < vocab;
+  uint16_t* o = out + (size_t)b * 2 * hidden;
+  for (int c = threadIdx.x; c < hidden; c += blockDim.x) {
+    o[c] = f32_to_bf16_bits(__ldcg(lm_hidden + (size_t)b * hidden + c));
+    float e = __int_as_float(0x7fc00000);
+    if (ok) {
+      const uint32_t word = ew[(size_t)t * (hidden / 4) + c / 4];
+      const float q = (float)((word >> (8 * (c % 4))) & 0xFFu);
+      const size_t g = (size_t)t * (hidden / 64) + c / 64;
+      e = fmaf(q, bf16_bits_to_f32(es[g]), bf16_bits_to_f32(eb[g]));
+    }
+    o[hidden + c] = f32_to_bf16_bits(e);
+  }
+}
+
+}  // namespace qg
+
+namespace {
+
+struct CpLayout {
+  StepLayout step;  // the step's buffers for cap = 1 (from offset 0)
+  size_t comb, kc, vc, pos, am, logits, total;
+};
+
+CpLayout cp_layout(const qg_qwen3_config& c, int B) {
+  CpLayout L;
+  L.step = step_layout(c, B, 1);
+  size_t off = L.step.total;
+  auto take = [&](size_t bytes) { size_t o = off; off += (bytes + 255) & ~(size_t)255; return o; };
+  const size_t cache = (size_t)c.layers * B * c.kv_heads * 1 * c.head_dim * 2;
+  L.comb = take((size_t)B * 2 * c.hidden * 2);
+  L.kc = take(cache);
+  L.vc = take(cache);
+  L.pos = take((size_t)B * 4);
+  L.am = take(argmax_ws_bytes(B, c.vocab));
+  L.logits = take((size_t)B * c.vocab * 4);
+  L.total = off;
+  return L;
+}
+
+}  // namespace
+
+extern "C" size_t qg_code_predict_workspace_size(const qg_qwen3_config* cfg, int B) {
+  if (!cfg || B < 1 || cfg->heads < 1 || cfg->kv_heads < 1 || cfg->vocab < 1) return 0;
+  return cp_layout(*cfg, B).total;
+}
+
+extern "C" qg_status qg_code_predict(const qg_qwen3_config* cfg, const qg_code_predictor_weights* w,
+                                     const float* lm_hidden, const int32_t* code0, int32_t* codes,
+                                     float* logits, int B, void* ws, size_t ws_bytes,
+                                     void* stream) {
+  clear_error();
+  qg_status st = validate_cfg(cfg, B, 1);
+  if (st != QG_OK) return st;
+  const qg_qwen3_config& c = *cfg;
+  QG_REQUIRE(w, QG_ERR_INVALID_ARGUMENT, "qg_code_predict: weights is NULL");
+  QG_REQUIRE(w->groups >= 2 && w->groups <= 64, QG_ERR_UNSUPPORTED_SHAPE,
+             "qg_code_predict: groups=%d must be in [2, 64]", w->groups);
+  QG_REQUIRE(w->code_embed && w->heads && w->final_norm && (c.layers == 0 || w->layers),
+             QG_ERR_INVALID_ARGUMENT, "qg_code_predict: null table, head, norm or layer array");
+  if ((st = validate_matrix(w->input_proj, "input_proj", -1)) != QG_OK) return st;
+  for (int g = 1; g < w->groups; ++g) {
+    if ((st = validate_matrix(w->code_embed[g - 1], "code_embed", g - 1)) != QG_OK) return st;
+    if ((st = validate_matrix(w->heads[g], "heads", g)) != QG_OK) return st;
+  }
+  for (int l = 0; l < c.layers; ++l) {
+    const qg_qwen3_layer& L = w->layers[l];
+    for (const qg_affine8_matrix* m : {&L.q, &L.k, &L.v, &L.o, &L.gate, &L.up, &L.down})
+      if ((st = validate_matrix(*m, "layer", l)) != QG_OK) return st;
+    QG_REQUIRE(L.input_norm && L.post_norm && L.q_norm && L.k_norm, QG_ERR_INVALID_ARGUMENT,
+               "qg_code_predict: layer %d has a null norm weight", l);
+  }
+  QG_REQUIRE(lm_hidden && code0 && codes, QG_ERR_INVALID_ARGUMENT,
+             "qg_code_predict: null lm_hidden, code0 or codes");
+  QG_REQUIRE(aligned(lm_hidden, 4) && aligned(code0, 4) && aligned(codes, 4) &&
+                 aligned(logits, 4),
+             QG_ERR_MISALIGNED, "qg_code_predict: lm_hidden/code0/codes/logits misaligned");
+  const CpLayout Ly = cp_layout(c, B);
+  QG_REQUIRE(ws && ws_bytes >= Ly.total, QG_ERR_WORKSPACE_TOO_SMALL,
+             "qg_code_predict: workspace of %zu bytes given, %zu needed", ws_bytes, Ly.total);
+  QG_REQUIRE(aligned(ws, 256), QG_ERR_MISALIGNED, "qg_code_predict: ws not 256-byte aligned");
+
+  cudaStream_t s = (cudaStream_t)stream;
+  uint8_t* base = reinterpret_cast<uint8_t*>(ws);
+  auto enqueue = [&] {
+    const StepBufs sb = step_bufs(ws, Ly.step);
+    uint16_t* comb = reinterpret_cast<uint16_t*>(base + Ly.comb);
+    uint16_t* kc = reinterpret_cast<uint16_t*>(base + Ly.kc);
+    uint16_t* vc = reinterpret_cast<uint16_t*>(base + Ly.vc);
+    int32_t* pos = reinterpret_cast<int32_t*>(base + Ly.pos);
+    void* am = base + Ly.am;
+    const size_t cnt_off = attention_ws_counter_offset(B, c.heads, c.kv_heads, c.head_dim, 1);
+    cudaMemsetAsync(reinterpret_cast<uint8_t*>(sb.aws) + cnt_off, 0, (size_t)B * c.kv_heads * 4,
+                    s);
+    launch_pdl(cp_start_kernel, dim3(B), dim3(64), 0, s, true, code0, codes, pos, sb.rope,
+               c.head_dim);
+    for (int g = 1; g < w->groups; ++g) {
+      const int32_t* prev = codes + (size_t)(g - 1) * B;
+      const qg_affine8_matrix& E = w->code_embed[g - 1];
+      launch_pdl(cp_input_kernel, dim3(B), dim3(256), 0, s, true, lm_hidden, E.w, E.scales,
+                 E.biases, prev, comb, c.hidden, c.vocab);
+      GemvSeg ip = {w->input_proj.w, w->input_proj.scales, w->input_proj.biases, sb.x, nullptr,
+                    c.hidden, 0};
+      gemv_affine8_launch(&ip, 1, comb, false, 2 * c.hidden, B, s, true);
+      enqueue_layers(c, w->layers, kc, vc, 1, prev, pos, B, sb, s);
+      float* lg = logits ? logits + (size_t)g * B * c.vocab
+                         : reinterpret_cast<float*>(base + Ly.logits);
+      enqueue_head(c, w->heads[g], c.vocab, w->final_norm, lg, B, sb, s);
+      argmax_launch(lg, B, c.vocab, codes + (size_t)g * B, am, s, true);
+    }
+  };
+  std::vector<uint64_t> key;
+  key.push_back(2);  // what: a code prediction
+  key_cfg(key, c, B, 1);
+  for (const void* p : {(const void*)lm_hidden, (const void*)code0, (const void*)codes,
+                        (const void*)logits, (const void*)ws, (const void*)w->final_norm})
+    key_push(key, p);
+  key.push_back((uint64_t)w->groups);
+  key_matrix(key, w->input_proj);
+  for (int g = 0; g < w->groups; ++g) {
+    if (g >= 1) key_matrix(key, w->code_embed[g - 1]);
+    if (g >= 1) key_matrix(key, w->heads[g]);
+  }
+  key_layers(key, w->layers, c.layers);
+  return run_recorded(std::move(key), s, enqueue, "qg_code_predict");
 }

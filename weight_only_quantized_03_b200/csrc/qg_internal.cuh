@@ -182,4 +182,9 @@ cudaError_t attention_launch_step(const float* q, const float* k, const float* v
                                   cudaStream_t st, bool pdl);
 size_t attention_ws_bytes(int B, int H, int Hkv, int D, int cap);
 
+// greedy token per row (argmax.cu); ws of argmax_ws_bytes(B, V) bytes
+size_t argmax_ws_bytes(int B, int V);
+cudaError_t argmax_launch(const float* logits, int B, int V, int32_t* out, void* ws,
+                          cudaStream_t st, bool pdl);
+
 }  // namespace qg
