@@ -130,3 +130,52 @@ def test_decode_step_names_the_bad_tensor():
     st, msg = _status("qg_decode_step", ctypes.byref(bad), ctypes.byref(w), FAKE, FAKE, 16, FAKE,
                       FAKE, FAKE, 1, FAKE, need, None)
     assert st == qg.QG_ERR_UNSUPPORTED_SHAPE and "kv_heads=2" in msg
+
+
+def test_argmax_rejects_bad_arguments():
+    need = qg.lib.qg_argmax_workspace_size(2, 1000)
+    assert need >= 2 * 8
+    st, msg = _status("qg_argmax_f32", FAKE, 2, 0, FAKE, FAKE, need, None)
+    assert st == qg.QG_ERR_UNSUPPORTED_SHAPE and "V=0" in msg
+    st, msg = _status("qg_argmax_f32", None, 2, 1000, FAKE, FAKE, need, None)
+    assert st == qg.QG_ERR_INVALID_ARGUMENT and "logits" in msg
+    st, msg = _status("qg_argmax_f32", FAKE + 2, 2, 1000, FAKE, FAKE, need, None)
+    assert st == qg.QG_ERR_MISALIGNED
+    st, msg = _status("qg_argmax_f32", FAKE, 2, 1000, FAKE, FAKE, need - 8, None)
+    assert st == qg.QG_ERR_WORKSPACE_TOO_SMALL and str(need) in msg
+    assert _status("qg_argmax_f32", None, 0, 1000, None, None, 0, None)[0] == qg.QG_OK
+
+
+def test_code_predict_names_the_bad_table():
+    cfg, _, arr = _tiny_model_structs()
+    G = 3
+    mats = lambda: (qg.qg_affine8_matrix * G)(*[qg.qg_affine8_matrix(FAKE, FAKE, FAKE)
+                                                for _ in range(G)])
+    emb, heads = mats(), mats()
+    w = qg.qg_code_predictor_weights(
+        qg.qg_affine8_matrix(FAKE, FAKE, FAKE),
+        ctypes.cast(emb, ctypes.POINTER(qg.qg_affine8_matrix)),
+        ctypes.cast(heads, ctypes.POINTER(qg.qg_affine8_matrix)),
+        ctypes.cast(arr, ctypes.POINTER(qg.qg_qwen3_layer)), FAKE, G)
+    need = qg.lib.qg_code_predict_workspace_size(ctypes.byref(cfg), 1)
+    assert need > qg.lib.qg_decode_step_workspace_size(ctypes.byref(cfg), 1, 1)
+
+    def call(ws_bytes=need, codes=FAKE):
+        return _status("qg_code_predict", ctypes.byref(cfg), ctypes.byref(w), FAKE, FAKE, codes,
+                       None, 1, FAKE, ws_bytes, None)
+
+    heads[2].w = None
+    st, msg = call()
+    assert st == qg.QG_ERR_INVALID_ARGUMENT and "heads" in msg
+    heads[2].w = FAKE
+    emb[0].scales = None
+    st, msg = call()
+    assert st == qg.QG_ERR_INVALID_ARGUMENT and "code_embed" in msg
+    emb[0].scales = FAKE
+    st, msg = call(codes=None)
+    assert st == qg.QG_ERR_INVALID_ARGUMENT and "codes" in msg
+    st, msg = call(ws_bytes=need - 256)
+    assert st == qg.QG_ERR_WORKSPACE_TOO_SMALL and str(need) in msg
+    w.groups = 1
+    st, msg = call()
+    assert st == qg.QG_ERR_UNSUPPORTED_SHAPE and "groups=1" in msg
