@@ -122,7 +122,25 @@ def other_kernels(qg, stream, hbm_peak, n):
     y = torch.empty((1, N), dtype=torch.float32, device="cuda")
     fns = [(lambda m=m: qg.qg_gemv_q4_0(m, x, y, stream=stream)) for m in mats]
     ms_v = graph_time_ms(fns, stream, max(n, 2 * copies))
+    # C1: the single 1024 x 1024 affine8 GEMV at B = 1, as a chain of 512
+    # launches over rotated copies (together more than 3x L2)
+    wnp, snp, bnp8 = qg_synth.affine8_packed(1024, 1024, 31)
+    tob = lambda a: torch.from_numpy(a.view({2: np.int16, 4: np.int32}[a.dtype.itemsize])).cuda()
+    c1_bytes = affine8_bytes(1024, 1024, 1)
+    c1_copies = -(-3 * L2_BYTES // (wnp.nbytes + snp.nbytes + bnp8.nbytes))
+    c1_mats = [(tob(wnp), tob(snp), tob(bnp8)) for _ in range(c1_copies)]
+    x1 = torch.from_numpy(qg_synth.gaussian_bf16_bits((1, 1024), 1.0, 32)).view(torch.bfloat16).cuda()
+    y1 = torch.empty((1, 1024), dtype=torch.float32, device="cuda")
+    c1_fns = [(lambda m=m: qg.qg_gemv_affine8_g64(*m, x1, y1, stream=stream)) for m in c1_mats]
+    ms_c1 = graph_time_ms(c1_fns, stream, 512)
+    del c1_mats
     return {
+        "gemv_affine8_1024x1024_b1_chain": {
+            "bound": "hbm", "achieved": c1_bytes / (ms_c1 / 1000.0) / 1e9, "peak": hbm_peak,
+            "unit": "GB/s", "frac": c1_bytes / (ms_c1 / 1000.0) / 1e9 / hbm_peak,
+            "algorithmic_bytes": c1_bytes, "launch_us": ms_c1 * 1000.0,
+            "note": f"512 launches back to back in a CUDA graph (PDL) over {c1_copies} "
+                    "copies of the matrix (more than 3x L2)"},
         "gemm_q4_0_whisper_fc1": {
             "shape": [M, N, K], "bound": "tensor", "achieved": tflops, "peak": tf_peak,
             "unit": "TFLOP/s", "frac": tflops / tf_peak, "launch_us": ms * 1000.0,

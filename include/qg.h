@@ -86,6 +86,9 @@ unsigned long long qg_kernel_launch_count(void);
  *         y += W x); must not overlap w, scales, biases or x.
  * residual device fp32 [B][N] or NULL (4-byte alignment suffices).
  * Shape rules: K % 64 == 0, 1 <= B <= 32 (B == 0 is a no-op), N >= 0.
+ * Launch: with Programmatic Dependent Launch, so a chain of calls overlaps
+ * each GEMV's first weight loads with the previous kernel's tail; the kernel
+ * waits for the stream's previous kernel before it reads x or residual.
  * ---------------------------------------------------------------------- */
 qg_status qg_gemv_affine8_g64(const uint32_t* w, const uint16_t* scales,
                               const uint16_t* biases, const void* x,
@@ -106,6 +109,8 @@ qg_status qg_gemv_affine8_g64(const uint32_t* w, const uint16_t* scales,
  * x       device fp32 [B][K].   bias device fp32 [N] or NULL (4-byte align).
  * y       device fp32 [B][N].
  * Shape rules: K % 32 == 0, 1 <= B <= 32 (B == 0 is a no-op).
+ * Launch: with Programmatic Dependent Launch (as qg_gemv_affine8_g64); the
+ * kernel waits for the stream's previous kernel before it reads x or bias.
  * ---------------------------------------------------------------------- */
 qg_status qg_gemv_q4_0(const uint8_t* blocks, const float* x, const float* bias,
                        float* y, int N, int K, int B, void* stream);

@@ -301,7 +301,9 @@ extern "C" qg_status qg_gemv_affine8_g64(const uint32_t* w, const uint16_t* scal
   qg_status st = validate_gemv(w, scales, biases, x, x_dtype, y, y_dtype, residual, N, K, B);
   if (st != QG_OK || N == 0 || B == 0) return st;
   GemvSeg seg = {w, scales, biases, y, residual, N, y_dtype == QG_BF16 ? 1 : 0};
-  gemv_affine8_launch(&seg, 1, x, x_dtype == QG_F32, K, B, (cudaStream_t)stream, false);
+  // PDL: the kernel may start while the stream's previous kernel drains; it
+  // waits for that kernel before reading x or the residual
+  gemv_affine8_launch(&seg, 1, x, x_dtype == QG_F32, K, B, (cudaStream_t)stream, true);
   return check_launch("qg_gemv_affine8_g64");
 }
 

@@ -276,7 +276,9 @@ extern "C" qg_status qg_gemv_q4_0(const uint8_t* blocks, const float* x, const f
   QG_REQUIRE(aligned(y, 4) && (!bias || aligned(bias, 4)), QG_ERR_MISALIGNED,
              "qg_gemv_q4_0: y or bias misaligned");
   QG_REQUIRE((long long)N * K < (1LL << 40), QG_ERR_UNSUPPORTED_SHAPE, "qg_gemv_q4_0: N*K too large");
-  gemv_q4_0_launch(blocks, x, bias, y, N, K, B, (cudaStream_t)stream, false);
+  // PDL: the kernel may start (and stage its weights) while the stream's
+  // previous kernel drains; it waits for that kernel before reading x or bias
+  gemv_q4_0_launch(blocks, x, bias, y, N, K, B, (cudaStream_t)stream, true);
   return check_launch("qg_gemv_q4_0");
 }
 
