@@ -363,6 +363,26 @@ def run_reference(args):
     return 0
 
 
+# ------------------------------------------------------------ ranks ---------
+
+def max_over_ranks(ms, world, dist=None, device="cpu"):
+    """The slowest rank's time: every rank contributes its own device time
+    and all get the maximum (an all-reduce, the same collective on every
+    rank); with one rank, the time itself."""
+    if world <= 1:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_value(world, units_per_rank, max_ms):
+    """Whole-job throughput of independent replicas: the units all ranks
+    processed over the slowest rank's time."""
+    return world * units_per_rank / (max_ms / 1000.0)
+
+
 # ------------------------------------------------------------ GPU arm -------
 
 def run_ours(args):
@@ -428,13 +448,9 @@ def run_ours(args):
         stream.synchronize()
         torch.cuda.synchronize()
         barrier()
-    ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world, dist, "cuda")
     ms_per_step = ms / args.steps
-    value = world * args.steps / (ms / 1000.0)
+    value = aggregate_value(world, args.steps, ms)
 
     # ---- dominant kernel: the LM-head GEMV (151936 x 1024), timed per launch
     hbm_peak, peak_kind = measured_peaks()
@@ -490,12 +506,8 @@ def run_ours(args):
                 one()
             e1.record(stream)
         stream.synchronize()
-        ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([ms], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = float(t.item())
-        return world * e2e_steps / (ms / 1000.0)
+        ms = max_over_ranks(e0.elapsed_time(e1), world, dist, "cuda")
+        return aggregate_value(world, e2e_steps, ms)
 
     e2e_value = e2e_run(True)
     e2e_logits_value = e2e_run(False)
