@@ -354,6 +354,33 @@ void qg_step_graphs_clear(void);
 qg_status qg_decode_step_inspect(const qg_qwen3_config* cfg, int B, int cap, size_t offsets[4]);
 
 /* ------------------------------------------------------------------------
+ * Token sampling  [MK: makima src/tts/qwen3, `sample_token` and
+ * `apply_repetition_penalty`], in fp32 in the page's order:
+ *   s = logits[b]; for each past[b][j] in [0, V), in order (every
+ *   occurrence counts): s_t = s_t < 0 ? s_t * penalty : s_t / penalty;
+ *   top_k == 0 or temperature == 0: out[b] = the first strict maximum of s
+ *   (as qg_argmax_f32);
+ *   otherwise: t = s / temperature; the k = min(top_k, V) largest t in
+ *   descending order, equal values by index; e_j = exp(t_j - t_0);
+ *   out[b] = the index of the first j whose running sum of e_j / sum(e)
+ *   reaches r[b] (the first of the k if none does). NaN scores are never
+ *   chosen.
+ * logits  device fp32 [B][V] (not modified).
+ * past    device int32 [B][P] or NULL with P = 0; entries outside [0, V)
+ *         are skipped (use -1 for empty slots).
+ * r       device fp32 [B], the uniform draws in [0, 1) (caller's random
+ *         numbers); may be NULL for the greedy case.
+ * out     device int32 [B].
+ * Shape rules: 1 <= V; 0 <= top_k <= 64; ceil(V / 2048) * top_k <= 8192;
+ * penalty > 0; temperature >= 0.
+ * ws      >= qg_sample_workspace_size(B, V, top_k) bytes, 256-byte aligned.
+ * ---------------------------------------------------------------------- */
+size_t qg_sample_workspace_size(int B, int V, int top_k);
+qg_status qg_sample(const float* logits, int B, int V, const int32_t* past, int P,
+                    float penalty, float temperature, int top_k, const float* r,
+                    int32_t* out, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * Code predictor  [MK: makima src/tts/qwen3/code_predictor.rs,
  * CodePredictor::predict and CodePredictorLayer::forward]
  *

@@ -352,6 +352,50 @@ def argmax_first(logits):
     return best_i
 
 
+def apply_repetition_penalty(logits, past, penalty):
+    """[MK] ``apply_repetition_penalty``: for every past token in order (each
+    occurrence counts; tokens outside the vocabulary are skipped), a negative
+    score is multiplied by the penalty and any other divided by it, in
+    float32 as on the page. Returns a new float32 array."""
+    s = np.array(logits, dtype=np.float32)
+    p = np.float32(penalty)
+    for t in past:
+        t = int(t)
+        if 0 <= t < s.shape[0]:
+            s[t] = s[t] * p if s[t] < 0 else s[t] / p
+    return s
+
+
+def sample_token(logits, past, penalty, temperature, top_k, r):
+    """[MK] ``sample_token`` in float32, step by step as on the page:
+    repetition penalty; greedy when top_k == 0 or temperature == 0 (the
+    first strict maximum, ``argmax_first``: this library's greedy rule);
+    otherwise divide by the temperature, sort descending (stable: equal
+    values by index), keep the first k = min(top_k, V), exp(t - t_0) summed
+    in order, and return the first index whose running sum of probabilities
+    reaches ``r`` (the first of the k if none does). NaN scores are left out
+    of the sort (the page's comparison leaves their place unspecified)."""
+    s = apply_repetition_penalty(logits, past, penalty) if penalty != 1.0 else \
+        np.array(logits, dtype=np.float32)
+    if top_k == 0 or temperature == 0.0:
+        return argmax_first(s)
+    t = s / np.float32(temperature)
+    order = [i for i in np.argsort(-t, kind="stable") if not np.isnan(t[i])]
+    top = order[:min(top_k, len(t))]
+    if not top:
+        return 0
+    t0 = t[top[0]]
+    total = np.float32(0.0)
+    for i in top:
+        total = np.float32(total + np.exp(np.float32(t[i] - t0)))
+    cum = np.float32(0.0)
+    for i in top:
+        cum = np.float32(cum + np.float32(np.exp(np.float32(t[i] - t0)) / total))
+        if cum >= np.float32(r):
+            return int(i)
+    return int(top[0])
+
+
 # ---------------------------------------------------------------------------
 # The decode step  [TS: step]
 # ---------------------------------------------------------------------------

@@ -179,3 +179,20 @@ def test_code_predict_names_the_bad_table():
     w.groups = 1
     st, msg = call()
     assert st == qg.QG_ERR_UNSUPPORTED_SHAPE and "groups=1" in msg
+
+
+def test_sample_rejects_bad_arguments():
+    need = qg.lib.qg_sample_workspace_size(2, 151936, 50)
+    args = lambda **kw: [kw.get("logits", FAKE), 2, kw.get("V", 151936), FAKE, 4,
+                         ctypes.c_float(kw.get("penalty", 1.2)), ctypes.c_float(1.0),
+                         kw.get("top_k", 50), kw.get("r", FAKE), FAKE, FAKE, kw.get("ws", need), None]
+    st, msg = _status("qg_sample", *args(top_k=65))
+    assert st == qg.QG_ERR_UNSUPPORTED_SHAPE and "top_k=65" in msg
+    st, msg = _status("qg_sample", *args(penalty=0.0))
+    assert st == qg.QG_ERR_INVALID_ARGUMENT and "penalty" in msg
+    st, msg = _status("qg_sample", *args(r=None))
+    assert st == qg.QG_ERR_INVALID_ARGUMENT
+    st, msg = _status("qg_sample", *args(V=8192 * 2048 // 50 + 4096))
+    assert st == qg.QG_ERR_UNSUPPORTED_SHAPE and "candidates" in msg
+    st, msg = _status("qg_sample", *args(ws=need - 256))
+    assert st == qg.QG_ERR_WORKSPACE_TOO_SMALL and str(need) in msg

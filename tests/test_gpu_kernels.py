@@ -366,3 +366,50 @@ def test_argmax_first_strict_max_bit_exact(B, V):
     got = out.cpu().numpy()
     want = np.array([O.argmax_first(x[b]) for b in range(B)], dtype=np.int32)
     np.testing.assert_array_equal(got, want)
+
+
+# ---------------------------------------------------------- sampling -----
+
+def _allowed_draws(logits, past, penalty, temperature, top_k, r, slack=1e-6):
+    """The indices the oracle's draw can give when its running sums move by
+    `slack` (the fp32 exp of two libraries may differ in the last bit)."""
+    s = O.apply_repetition_penalty(logits, past, penalty)
+    t = s / np.float32(temperature)
+    order = [i for i in np.argsort(-t, kind="stable") if not np.isnan(t[i])][:min(top_k, len(t))]
+    e = np.exp((t[order] - t[order[0]]).astype(np.float32))
+    cum = np.cumsum(e / e.sum(dtype=np.float32), dtype=np.float32)
+    ok = {order[j] for j in range(len(order))
+          if cum[j] >= r - slack and (j == 0 or cum[j - 1] < r + slack)}
+    if cum[-1] < r + slack:
+        ok.add(order[0])
+    return ok
+
+
+@pytest.mark.parametrize("B,V,top_k,temperature", [(3, 2048, 50, 0.8), (2, 151936, 64, 1.0),
+                                                   (4, 2048, 1, 0.7), (2, 5000, 8, 1.3),
+                                                   (3, 2048, 0, 1.0), (2, 151936, 20, 0.0)])
+def test_sample_matches_the_oracle(B, V, top_k, temperature):
+    """Repetition penalty over past tokens (duplicates, -1 and out-of-range
+    entries), then greedy (top_k 0 or temperature 0: bit-exact against the
+    oracle) or a top-k draw with given uniform numbers (the oracle's index,
+    up to the last-bit freedom of fp32 exp at a running-sum boundary)."""
+    rng = np.random.default_rng(100 * B + top_k)
+    logits = (3.0 * rng.standard_normal((B, V))).astype(np.float32)
+    P = 40
+    past = rng.integers(0, min(V, 300), size=(B, P)).astype(np.int32)
+    past[:, 5] = past[:, 4]          # a repeated token
+    past[:, -3:] = [-1, V, V + 7]    # empty slot and out-of-range entries
+    logits[:, past[0, 0]] = -2.5     # a negative score that is penalized
+    r = rng.random(B).astype(np.float32)
+    out = torch.empty(B, dtype=torch.int32, device="cuda")
+    ws = torch.empty(qg.qg_sample_workspace_size(B, V, top_k), dtype=torch.uint8, device="cuda")
+    qg.qg_sample(dev(logits), out, ws, past=dev(past), penalty=1.2, temperature=temperature,
+                 top_k=top_k, r=dev(r))
+    got = out.cpu().numpy()
+    for b in range(B):
+        want = O.sample_token(logits[b], past[b], 1.2, temperature, top_k, r[b])
+        if top_k == 0 or temperature == 0.0:
+            assert got[b] == want
+        else:
+            assert got[b] == want or got[b] in _allowed_draws(
+                logits[b], past[b], 1.2, temperature, top_k, r[b]), (b, got[b], want)

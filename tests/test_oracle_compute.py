@@ -8,6 +8,7 @@ whole-prefix causal forward and a zero-weight closed form.
 """
 import cmath
 import math
+import os
 
 import numpy as np
 import pytest
@@ -467,3 +468,57 @@ def test_code_predict_chain_indices_and_concat_order():
     # group 1's logits directly: one nonzero logit, at 15
     lg = O.code_predict_group(cfg, w, lm_hidden, 5, 1)
     assert np.count_nonzero(lg > 1.0) == 1 and int(np.argmax(lg)) == 15
+
+
+def _golden_penalty():
+    path = os.path.join(os.path.dirname(__file__), "golden", "repetition_penalty_example.txt")
+    d = {}
+    for line in open(path):
+        if line.strip() and not line.startswith("#"):
+            k, *v = line.split()
+            d[k] = v
+    return d
+
+
+def test_repetition_penalty_worked_example_and_order():
+    d = _golden_penalty()
+    got = O.apply_repetition_penalty([float(v) for v in d["logits"]], [int(v) for v in d["past"]],
+                                     float(d["penalty"][0]))
+    np.testing.assert_allclose(got, [float(v) for v in d["expected"]], rtol=1e-6)
+    # negative scores are multiplied; every occurrence counts, in float32;
+    # tokens outside the vocabulary are skipped
+    got = O.apply_repetition_penalty([-1.0, 2.0, 0.5], [0, 0, 1, -1, 3], 1.2)
+    p = np.float32(1.2)
+    assert got[0] == np.float32(np.float32(-1.0) * p) * p
+    assert got[1] == np.float32(2.0) / p and got[2] == np.float32(0.5)
+
+
+def test_sample_token_distribution_ties_nan_and_greedy():
+    lg = np.log(np.array([1.0, 2.0, 3.0], dtype=np.float32))   # probabilities 1/6, 2/6, 3/6
+    # descending order 2, 1, 0 with running sums 1/2, 5/6, 1
+    assert O.sample_token(lg, [], 1.0, 1.0, 3, 0.4) == 2
+    assert O.sample_token(lg, [], 1.0, 1.0, 3, 0.6) == 1
+    assert O.sample_token(lg, [], 1.0, 1.0, 3, 0.95) == 0
+    rs = (np.arange(1000) + 0.5) / 1000
+    counts = np.bincount([O.sample_token(lg, [], 1.0, 1.0, 3, r) for r in rs], minlength=3)
+    np.testing.assert_allclose(counts / 1000, [1 / 6, 2 / 6, 3 / 6], atol=2e-3)
+    # top_k = 1 and r = 0 give the maximum; top_k = 2 drops index 0
+    assert O.sample_token(lg, [], 1.0, 1.0, 1, 0.99) == 2
+    assert O.sample_token(lg, [], 1.0, 1.0, 3, 0.0) == 2
+    assert all(O.sample_token(lg, [], 1.0, 1.0, 2, r) in (1, 2) for r in rs)
+    # equal values keep index order (a stable sort)
+    eq = np.array([5.0, 5.0, 1.0], dtype=np.float32)
+    assert O.sample_token(eq, [], 1.0, 1.0, 2, 0.3) == 0
+    assert O.sample_token(eq, [], 1.0, 1.0, 2, 0.7) == 1
+    # a NaN score is never drawn; temperature 0 or top_k 0 is greedy after
+    # the penalty (which here moves the maximum from 2 to 1)
+    nanl = np.array([np.nan, 1.0, 2.0], dtype=np.float32)
+    assert all(O.sample_token(nanl, [], 1.0, 1.0, 3, r) in (1, 2) for r in rs)
+    pen = np.array([0.0, 1.9, 2.0], dtype=np.float32)
+    assert O.sample_token(pen, [2], 1.2, 0.0, 5, 0.5) == 1
+    assert O.sample_token(pen, [2], 1.2, 1.0, 0, 0.5) == 1
+    # a lower temperature sharpens: at T = 0.1 the probabilities are in the
+    # ratio 1 : 2^10 : 3^10
+    counts = np.bincount([O.sample_token(lg, [], 1.0, 0.1, 3, r) for r in rs], minlength=3)
+    tot = 1 + 2 ** 10 + 3 ** 10
+    np.testing.assert_allclose(counts / 1000, [1 / tot, 2 ** 10 / tot, 3 ** 10 / tot], atol=2e-3)

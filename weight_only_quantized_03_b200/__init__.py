@@ -101,6 +101,8 @@ _SIGS = {
     "qg_code_predict": (_i, [ctypes.POINTER(qg_qwen3_config),
                              ctypes.POINTER(qg_code_predictor_weights), _vp, _vp, _vp, _vp, _i,
                              _vp, _sz, _vp]),
+    "qg_sample_workspace_size": (_sz, [_i, _i, _i]),
+    "qg_sample": (_i, [_vp, _i, _i, _vp, _i, _f, _f, _i, _vp, _vp, _vp, _sz, _vp]),
     "qg_step_graphs_enable": (None, [_i]),
     "qg_step_graphs_clear": (None, []),
     "qg_argmax_workspace_size": (_sz, [_i, _i]),
@@ -236,6 +238,21 @@ def qg_argmax_f32(logits, out, ws, stream=None):
     B, V = logits.shape
     _call("qg_argmax_f32", _p(logits), B, V, _p(out), _p(ws), ws.numel() * ws.element_size(),
           _stream(stream))
+
+
+def qg_sample_workspace_size(B, V, top_k):
+    return int(lib.qg_sample_workspace_size(B, V, top_k))
+
+
+def qg_sample(logits, out, ws, past=None, penalty=1.0, temperature=1.0, top_k=0, r=None,
+              stream=None):
+    """out[b] (int32, device): repetition penalty over past[b] (int32 [B, P],
+    -1 = empty), then greedy (top_k 0 or temperature 0) or a top-k draw with
+    the uniform numbers r (fp32 [B]) from the temperature softmax."""
+    B, V = logits.shape
+    P = 0 if past is None else past.shape[1]
+    _call("qg_sample", _p(logits), B, V, _p(past), P, float(penalty), float(temperature),
+          int(top_k), _p(r), _p(out), _p(ws), ws.numel() * ws.element_size(), _stream(stream))
 
 
 def qg_decode_attention_static_scratch_capacity():
