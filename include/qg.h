@@ -354,6 +354,19 @@ void qg_step_graphs_clear(void);
 qg_status qg_decode_step_inspect(const qg_qwen3_config* cfg, int B, int cap, size_t offsets[4]);
 
 /* ------------------------------------------------------------------------
+ * Selected-token log-probability  [TS: compute_selected_logprob of the
+ * greedy token; not printed on the page, read as the log-softmax]
+ *   out[b] = logits[b][tokens[b]] - log(sum_i exp(logits[b][i])), in fp32
+ *   with the row maximum subtracted first. A NaN logit or a token outside
+ *   [0, V) gives NaN.
+ * logits device fp32 [B][V]; tokens device int32 [B]; out device fp32 [B].
+ * ws     >= qg_token_logprob_workspace_size(B, V) bytes, 8-byte aligned.
+ * ---------------------------------------------------------------------- */
+size_t qg_token_logprob_workspace_size(int B, int V);
+qg_status qg_token_logprob(const float* logits, int B, int V, const int32_t* tokens,
+                           float* out, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * Token sampling  [MK: makima src/tts/qwen3, `sample_token` and
  * `apply_repetition_penalty`], in fp32 in the page's order:
  *   s = logits[b]; for each past[b][j] in [0, V), in order (every

@@ -352,6 +352,19 @@ def argmax_first(logits):
     return best_i
 
 
+def token_logprob(logits, token):
+    """The log-probability of ``token`` under the softmax of ``logits``
+    ([TS] ``compute_selected_logprob`` of the greedy token, whose body the
+    page does not print: read as the log-softmax), float64 with the maximum
+    subtracted: x[t] - (m + log sum exp(x - m)). NaN for a NaN logit or a
+    token outside the row."""
+    x = np.asarray(logits, dtype=np.float64)
+    if not 0 <= int(token) < x.shape[0] or np.isnan(x).any():
+        return math.nan
+    m = x.max()
+    return float(x[int(token)] - (m + math.log(np.exp(x - m).sum())))
+
+
 def apply_repetition_penalty(logits, past, penalty):
     """[MK] ``apply_repetition_penalty``: for every past token in order (each
     occurrence counts; tokens outside the vocabulary are skipped), a negative

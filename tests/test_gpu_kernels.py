@@ -413,3 +413,26 @@ def test_sample_matches_the_oracle(B, V, top_k, temperature):
         else:
             assert got[b] == want or got[b] in _allowed_draws(
                 logits[b], past[b], 1.2, temperature, top_k, r[b]), (b, got[b], want)
+
+
+@pytest.mark.parametrize("B,V", [(3, 2048), (2, 151936), (1, 7)])
+def test_token_logprob_matches_the_oracle(B, V):
+    """Log-softmax at the selected token (the greedy one, another, an
+    out-of-range one -> NaN) against the float64 oracle."""
+    rng = np.random.default_rng(V + B)
+    x = (4.0 * rng.standard_normal((B, V))).astype(np.float32)
+    toks = np.array([int(np.argmax(x[b])) if b % 3 == 0 else (b * 37) % V for b in range(B)],
+                    dtype=np.int32)
+    if B > 2:
+        toks[2] = V
+    out = torch.empty(B, dtype=torch.float32, device="cuda")
+    ws = torch.empty(qg.lib.qg_token_logprob_workspace_size(B, V), dtype=torch.uint8,
+                     device="cuda")
+    qg.qg_token_logprob(dev(x), dev(toks), out, ws)
+    got = out.cpu().numpy().astype(np.float64)
+    for b in range(B):
+        ref = O.token_logprob(x[b].astype(np.float64), int(toks[b]))
+        if math.isnan(ref):
+            assert math.isnan(got[b])
+        else:
+            assert abs(got[b] - ref) <= 2e-3 + 1e-3 * abs(ref), (b, got[b], ref)

@@ -522,3 +522,19 @@ def test_sample_token_distribution_ties_nan_and_greedy():
     counts = np.bincount([O.sample_token(lg, [], 1.0, 0.1, 3, r) for r in rs], minlength=3)
     tot = 1 + 2 ** 10 + 3 ** 10
     np.testing.assert_allclose(counts / 1000, [1 / tot, 2 ** 10 / tot, 3 ** 10 / tot], atol=2e-3)
+
+
+def test_token_logprob_closed_forms_and_library_logsumexp():
+    from scipy.special import logsumexp
+    V = 1000
+    assert O.token_logprob(np.zeros(V), 17) == pytest.approx(-math.log(V), abs=1e-12)
+    x = qg_synth.gaussian((V,), 3.0, 8).astype(np.float64)
+    for t in (0, 17, int(np.argmax(x))):
+        assert O.token_logprob(x, t) == pytest.approx(x[t] - logsumexp(x), abs=1e-12)
+        assert O.token_logprob(x + 1e4, t) == pytest.approx(O.token_logprob(x, t), abs=1e-9)
+    one_hot = np.full(V, -1e4)
+    one_hot[3] = 0.0
+    assert O.token_logprob(one_hot, 3) == pytest.approx(0.0, abs=1e-12)
+    assert math.isnan(O.token_logprob(x, V)) and math.isnan(O.token_logprob(x, -1))
+    x[5] = np.nan
+    assert math.isnan(O.token_logprob(x, 0))

@@ -101,6 +101,8 @@ _SIGS = {
     "qg_code_predict": (_i, [ctypes.POINTER(qg_qwen3_config),
                              ctypes.POINTER(qg_code_predictor_weights), _vp, _vp, _vp, _vp, _i,
                              _vp, _sz, _vp]),
+    "qg_token_logprob_workspace_size": (_sz, [_i, _i]),
+    "qg_token_logprob": (_i, [_vp, _i, _i, _vp, _vp, _vp, _sz, _vp]),
     "qg_sample_workspace_size": (_sz, [_i, _i, _i]),
     "qg_sample": (_i, [_vp, _i, _i, _vp, _i, _f, _f, _i, _vp, _vp, _vp, _sz, _vp]),
     "qg_step_graphs_enable": (None, [_i]),
@@ -238,6 +240,14 @@ def qg_argmax_f32(logits, out, ws, stream=None):
     B, V = logits.shape
     _call("qg_argmax_f32", _p(logits), B, V, _p(out), _p(ws), ws.numel() * ws.element_size(),
           _stream(stream))
+
+
+def qg_token_logprob(logits, tokens, out, ws, stream=None):
+    """out[b] (fp32, device) = log-softmax of logits[b] (fp32 [B, V]) at
+    tokens[b] (int32, device)."""
+    B, V = logits.shape
+    _call("qg_token_logprob", _p(logits), B, V, _p(tokens), _p(out), _p(ws),
+          ws.numel() * ws.element_size(), _stream(stream))
 
 
 def qg_sample_workspace_size(B, V, top_k):
