@@ -463,12 +463,7 @@ template <int BN, int MT, bool W32>
 static cudaError_t gq4_launch(const CUtensorMap& tmA, const uint8_t* blocks, const float* bias,
                               float* C, int M, int N, int K, unsigned* err, cudaStream_t st) {
   using G = gq4::Cfg<BN, MT>;
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(gq4::gemm_q4_0_tc_kernel<BN, MT, W32>,
-                         cudaFuncAttributeMaxDynamicSharedMemorySize, G::kSmem);
-    attr = true;
-  }
+  ensure_smem((const void*)gq4::gemm_q4_0_tc_kernel<BN, MT, W32>, G::kSmem);
   dim3 grid(N / BN, (M + MT * gq4::kBM - 1) / (MT * gq4::kBM));
   return launch_pdl(gq4::gemm_q4_0_tc_kernel<BN, MT, W32>, grid, dim3(gq4::kThreads),
                     (size_t)G::kSmem, st, false, tmA, blocks, bias, C, M, N, K, err);

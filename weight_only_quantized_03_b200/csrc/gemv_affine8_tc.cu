@@ -78,12 +78,7 @@ bool gemv_tc_eligible(const GemvSeg* segs, int nseg, int K, int B, bool x_f32) {
 template <int NT, int W>
 static cudaError_t gtc_launch_nt(const gtc::Params& P, dim3 grid, cudaStream_t st, bool pdl) {
   const size_t smem = gtc_smem(P.K, NT, W);
-  static int attr = 0;
-  if (smem > 48 * 1024 && attr < (int)smem) {
-    cudaFuncSetAttribute(gtc::gemv_tc_kernel<NT, W>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         200 * 1024);
-    attr = 200 * 1024;
-  }
+  if (smem > 48 * 1024) ensure_smem((const void*)gtc::gemv_tc_kernel<NT, W>, 200 * 1024);
   return launch_pdl(gtc::gemv_tc_kernel<NT, W>, grid, dim3(W * 32), smem, st, pdl, P);
 }
 

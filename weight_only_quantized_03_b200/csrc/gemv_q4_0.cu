@@ -190,12 +190,7 @@ constexpr size_t kQ4StagedSmem = 96 * 1024;
 template <int NB, int R>
 static cudaError_t q4_staged_launch_r(const uint8_t* blocks, const float* x, const float* bias,
                                       float* y, int N, int K, int B, cudaStream_t st, bool pdl) {
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(gemv_q4_0_staged_kernel<NB, R>,
-                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kQ4StagedSmem);
-    attr = true;
-  }
+  ensure_smem((const void*)gemv_q4_0_staged_kernel<NB, R>, (int)kQ4StagedSmem);
   constexpr int RT = kQ4Warps * R;
   const size_t smem = (size_t)RT * (K / 32) * 18;
   return launch_pdl(gemv_q4_0_staged_kernel<NB, R>, dim3((N + RT - 1) / RT),

@@ -36,6 +36,9 @@ qg_status check_launch(const char* what);
 // while its predecessor on the stream drains, and must call
 // pdl_wait() before touching anything the predecessor writes.
 void count_launch();
+// Raises `func`'s dynamic shared memory limit to `bytes` on the current
+// device, once per (kernel, device).
+void ensure_smem(const void* func, int bytes);
 
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block,

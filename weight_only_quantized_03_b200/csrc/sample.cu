@@ -198,12 +198,7 @@ extern "C" qg_status qg_sample(const float* logits, int B, int V, const int32_t*
   int n = 1;
   while (n < nc * k) n <<= 1;
   const size_t smem = (size_t)n * 8;
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(sp::draw_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         sp::kMaxCand * 8);
-    attr = true;
-  }
+  ensure_smem((const void*)sp::draw_kernel, sp::kMaxCand * 8);
   launch_pdl(sp::draw_kernel, dim3(B), dim3(sp::kThreads), smem, st, true,
              (const unsigned long long*)cand, nc * k, k, r, out);
   return check_launch("qg_sample");
