@@ -202,7 +202,11 @@ qg_status qg_embed_affine8_g64(const uint32_t* w, const uint16_t* scales,
  *   out[b][h] = sum_{t<L} softmax_t(q[b][h] . k[b][kv][t] * scale) v[b][kv][t]
  * The L rows are cut into chunks scored by separate CTAs; per-chunk
  * (max, sum, weighted V) partials are merged in a fixed order (results do
- * not depend on scheduling).
+ * not depend on scheduling). For head_dim 32, 64, 128 or 256 with at most 4
+ * query heads per KV head, the chunks of one (sequence, KV head) form a
+ * thread-block cluster and merge through distributed shared memory (the
+ * workspace is then not touched); other shapes merge through the
+ * workspace.
  * q        device fp32 [B][H][D].
  * k_cache, v_cache device bf16 [B][Hkv][cap][D] (row t of head kv at
  *          ((b*Hkv + kv)*cap + t)*D).
