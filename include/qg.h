@@ -239,14 +239,17 @@ qg_status qg_decode_attention(const float* q, const uint16_t* k_cache,
  *
  * Arguments, layouts and results as qg_decode_attention (same kernel, same
  * numerics); there is no ws / ws_bytes.
- * Limit: a shape whose scratch (qg_decode_attention_workspace_size) exceeds
- * the fixed capacity is refused with QG_ERR_WORKSPACE_TOO_SMALL before any
- * launch; use qg_decode_attention with a workspace for it.
+ * Limit: only shapes that merge through scratch (head_dim other than 32, 64,
+ * 128 or 256, or more than 4 query heads per KV head) use the array; such a
+ * shape whose scratch (qg_decode_attention_workspace_size) exceeds the fixed
+ * capacity is refused with QG_ERR_WORKSPACE_TOO_SMALL before any launch (use
+ * qg_decode_attention with a workspace for it). Cluster shapes use none and
+ * are not limited.
  * Setup: the first call on each device looks up the array's device address
  * (cudaGetSymbolAddress, with that device current) and caches it; a failed
  * lookup returns QG_ERR_CUDA. Make the first call on a device before any
- * stream capture begins. Each call clears the ticket counters (an async
- * memset on `stream`) before the launch.
+ * stream capture begins. A call that uses the array clears its ticket
+ * counters (an async memset on `stream`) before the launch.
  * Concurrency: every call on one device shares the one scratch array, so
  * calls must not overlap in time: issue them on one stream, or order them
  * with events. Overlapping calls race on the scratch and give undefined

@@ -26,12 +26,27 @@ def _cuda():
         pytest.skip("no CUDA device")
 
 
-# two calls in a row with different shapes: the second call's split plan and
-# counters differ from the first's
+# Calls in a row with different shapes. The first two take the cluster
+# kernel (head_dim 128, 2 query heads per KV head), which merges through
+# distributed shared memory and leaves the scratch untouched. The others take
+# the split kernel, whose partials and ticket counters live in the static
+# scratch: 8 query heads per KV head, then head_dim 96, then the first split
+# shape again with other lengths, so each call starts from the scratch the
+# previous call left (other split plans, counters left at zero or not).
 CALLS = [
     (1, 16, 8, 128, 513, [512], 60, "f32"),
     (3, 16, 8, 128, 600, [33, 600, 1], 70, "bf16"),
+    (2, 16, 2, 128, 700, [700, 350], 80, "f32"),
+    (3, 12, 4, 96, 300, [257, 1, 300], 90, "bf16"),
+    (2, 16, 2, 128, 700, [513, 64], 100, "f32"),
 ]
+
+
+def _takes_split_kernel(H, Hkv, D):
+    """The library's rule: the cluster kernel serves head_dim 32/64/128/256
+    with at most 4 query heads per KV head; every other shape merges its
+    splits through the scratch."""
+    return not (D in (32, 64, 128, 256) and H // Hkv <= 4)
 
 
 def _inputs(B, H, Hkv, D, cap, lens, seed):
@@ -43,6 +58,7 @@ def _inputs(B, H, Hkv, D, cap, lens, seed):
 
 def test_static_scratch_matches_workspace_entry_point_on_consecutive_calls():
     assert qg.qg_decode_attention_static_scratch_capacity() == 4 << 20
+    assert sum(_takes_split_kernel(c[1], c[2], c[3]) for c in CALLS) == 3
     for B, H, Hkv, D, cap, lens, seed, od in CALLS:
         kbits, vbits, q, kv_len = _inputs(B, H, Hkv, D, cap, lens, seed)
         qd, kd, vd, ld = dev(q), bf16_dev(kbits), bf16_dev(vbits), dev(kv_len)

@@ -649,11 +649,16 @@ extern "C" qg_status qg_decode_attention_static_scratch(const float* q, const ui
   clear_error();
   qg_status st = validate_attention(q, k_cache, v_cache, kv_len, out, out_dtype, B, H, Hkv, D, cap);
   if (st != QG_OK || B == 0) return st;
-  const size_t need = attention_ws_bytes(B, H, Hkv, D, cap);
-  QG_REQUIRE(need <= kAttnStaticScratchBytes, QG_ERR_WORKSPACE_TOO_SMALL,
-             "qg_decode_attention_static_scratch: this shape needs %zu bytes of scratch, more "
-             "than the fixed %zu; use qg_decode_attention with a caller workspace",
-             need, kAttnStaticScratchBytes);
+  // Only the split kernel touches scratch; the cluster kernel merges through
+  // distributed shared memory, so its shapes are not limited by the array.
+  const bool split = !ac::cluster_ok(H, Hkv, D);
+  if (split) {
+    const size_t need = attention_ws_bytes(B, H, Hkv, D, cap);
+    QG_REQUIRE(need <= kAttnStaticScratchBytes, QG_ERR_WORKSPACE_TOO_SMALL,
+               "qg_decode_attention_static_scratch: this shape needs %zu bytes of scratch, more "
+               "than the fixed %zu; use qg_decode_attention with a caller workspace",
+               need, kAttnStaticScratchBytes);
+  }
   void* ws = nullptr;
   cudaError_t e = attn_scratch_address(&ws);
   if (e != cudaSuccess) {
@@ -662,13 +667,16 @@ extern "C" qg_status qg_decode_attention_static_scratch(const float* q, const ui
     return QG_ERR_CUDA;
   }
   cudaStream_t s = (cudaStream_t)stream;
-  // the ticket counters must start at zero (the kernel also leaves them at
-  // zero; a cleared start does not depend on how the last call ended)
-  const size_t off = attention_ws_counter_offset(B, H, Hkv, D, cap);
-  e = cudaMemsetAsync(reinterpret_cast<uint8_t*>(ws) + off, 0, (size_t)B * Hkv * sizeof(unsigned int), s);
-  if (e != cudaSuccess) {
-    set_error("qg_decode_attention_static_scratch: %s", cudaGetErrorString(e));
-    return QG_ERR_CUDA;
+  if (split) {
+    // the ticket counters must start at zero (the kernel also leaves them at
+    // zero; a cleared start does not depend on how the last call ended)
+    const size_t off = attention_ws_counter_offset(B, H, Hkv, D, cap);
+    e = cudaMemsetAsync(reinterpret_cast<uint8_t*>(ws) + off, 0,
+                        (size_t)B * Hkv * sizeof(unsigned int), s);
+    if (e != cudaSuccess) {
+      set_error("qg_decode_attention_static_scratch: %s", cudaGetErrorString(e));
+      return QG_ERR_CUDA;
+    }
   }
   attention_launch(q, k_cache, v_cache, kv_len, nullptr, out, out_dtype == QG_BF16, B, H, Hkv, D,
                    cap, scale, ws, s, false);
