@@ -462,7 +462,8 @@ def bf16_alternative(v, rel):
 
 def bf16_rounding_ok(v, r, rel=2.0 ** -16, abs_tol=0.0):
     """Whether each ``r`` is the bf16 rounding (to nearest even) of some
-    value within ``eps = rel * |v| + abs_tol`` of the float64 value ``v``.
+    value within ``eps = rel * |v| + abs_tol`` of the float64 value ``v``
+    (``abs_tol`` a scalar or an array shaped like ``v``).
 
     This is the set of results that an implementation computing ``v`` with an
     error of at most ``eps`` (float32 arithmetic, another summation order)
@@ -477,65 +478,194 @@ def bf16_rounding_ok(v, r, rel=2.0 ** -16, abs_tol=0.0):
     return ok | (np.isnan(v) & np.isnan(r))
 
 
-def decode_layer_forced(cfg, lw, x, k_cache_l, v_cache_l, pos, forced, rel=2.0 ** -16,
-                        abs_rel=2.0 ** -12, details=None):
-    """``decode_layer`` teacher-forced at its bf16 rounding points.
+# ---------------------------------------------------------------------------
+# float32 error bounds of the short op chains between a GEMV output and the
+# next bf16 rounding point. They decide which bf16 values the teacher-forced
+# check accepts at a rounding point: every value that rounds from within the
+# bound of the exact result. Standard forward error analysis with the unit
+# roundoff u = 2^-24 of float32 (round to nearest): a chain of n roundings
+# has relative error at most gamma_n = n u / (1 - n u); a sum of n terms
+# evaluated along a tree of depth n is within gamma_n * sum|terms| of exact.
+# The depths below bound those of any summation order this library's kernels
+# use (the kernel sources state theirs); expf is taken to be within 2 ulp
+# (4u relative), sqrtf and division correctly rounded.
+# ---------------------------------------------------------------------------
 
-    ``forced`` maps points to the values another implementation stored there:
-    ``xn`` (input norm, [hidden]), ``k`` and ``v`` (the cache rows written at
-    ``pos``, [Hkv*D]), ``att`` (attention output, [H*D]), ``xn2``
-    (post-attention norm, [hidden]), ``h`` (SiLU-mul output, [ffn]). At each
-    point the layer's own float64 value is computed from what came before,
-    each forced value is checked to be a correct bf16 rounding of it
-    (``bf16_rounding_ok``: the rounding of a value within
-    ``rel * |v| + abs_rel * rms`` of it, rms that of the point's vector --
-    float32 errors of an element scale with its vector, and where the
-    residual stream is small they are magnified by the norm after it), and the
-    layer continues from the forced values. Where two roundings are both
-    correct, the rest of the layer follows the other implementation's choice.
-    Returns ``(y, bad)``: the new residual stream and, per point, the indices
+U32 = 2.0 ** -24
+EXPF_REL = 4.0 * U32
+
+
+def gamma(n):
+    """Relative error bound of a chain of n float32 roundings."""
+    return n * U32 / (1.0 - n * U32)
+
+
+def sumsq_depth(n):
+    """Longest chain of roundings in the float32 sum of squares of an
+    n-vector (a norm's statistic): n/32 + 32 covers per-thread partial sums
+    over a strided slice, a warp reduction and a sum over warps."""
+    return n // 32 + 32
+
+
+def rmsnorm_rel_bound(n):
+    """Relative error bound of each output of an RMSNorm of an exact float32
+    n-vector computed in float32: the sum of squares (all terms positive, so
+    relative ``gamma(sumsq_depth(n))``), the division by n and the add of
+    eps (2), the square root (halves the relative error, +1), the reciprocal
+    (+1), then x * inv * w (+2)."""
+    return 1.01 * (0.5 * gamma(sumsq_depth(n) + 3) + gamma(4))
+
+
+def norm_rope_bound(x, w_bits, eps, pos, theta, D):
+    """(value, bound) of NeoX RoPE applied to the per-head RMSNorm of an
+    exact float32 vector ``x [heads*D]``: the value in float64 and, per
+    element, the float32 error bound. Each rotated element is a*c - b*s (or
+    b*c + a*s) of two normed elements a, b (relative error
+    ``rmsnorm_rel_bound(D)`` each) and the float32 cos/sin of the angle
+    (computed in double and rounded once: relative u); the two products and
+    the difference add 3 roundings: bound (rho + 3u) (|a c| + |b s|)."""
+    n = rmsnorm_perhead(x, w_bits, eps, D)
+    v = rope_neox(n, pos, theta, D)
+    hn = np.abs(n).reshape(-1, D)
+    half = D // 2
+    a = pos * rope_inv_freq(theta, D)
+    c, sn = np.abs(np.cos(a)), np.abs(np.sin(a))
+    mag = np.empty_like(hn)
+    mag[:, :half] = hn[:, :half] * c + hn[:, half:] * sn
+    mag[:, half:] = hn[:, half:] * c + hn[:, :half] * sn
+    rho = rmsnorm_rel_bound(D) + gamma(4)
+    return v, 1.01 * rho * mag.reshape(v.shape)
+
+
+def attention_depths(L, D):
+    """(dot, rescale, accumulate) depths of the decode attention kernels: a
+    score is a float32 dot of D products (per-lane partial sums over D/32 to
+    D/8 columns and a shuffle tree: D/8 + 8); along any cached row's path the
+    running softmax state is rescaled by a computed exp at most L/32 + 16
+    times (once per batch of rows, then the merges of warps, CTAs and
+    splits); the weighted sums of V and of the weights take at most
+    L/4 + 96 roundings."""
+    return D // 8 + 8, L // 32 + 16, L // 4 + 96
+
+
+def attention_bound(qp, dqp, k_cache, v_cache, kv_len, H, Hkv, D):
+    """(value, bound) of ``decode_attention`` computed in float32 from a
+    query ``qp [H*D]`` known within ``dqp`` (per element) and exact bf16
+    cache rows.
+
+    Score t: s_t = scale * sum_d q_d k_td with scale = 1/sqrt(D) as a float32
+    (2 roundings) times q (1): its error is within
+    scale * (sum_d dq_d |k_td| + (3u + gamma(dot)) sum_d |q_d k_td|).
+    Softmax: a perturbation e_t of the log-weight of row t moves the output
+    by sum_t p_t (e^{e_t} - 1) (v_t - o) / sum_t p_t e^{e_t}, at most
+    e^{2 max e} sum_t p_t |e_t| |v_t - o|. The log-weight of row t is off by
+    its score's error, the rounding of s_t - m (u |s_t - m|), its exp (4u)
+    and each computed rescale on its path (4u, plus u |m_old - m_new|,
+    which summed along the path is at most the score range). The weighted
+    sums add gamma(accumulate) (sum_t p_t |v_t| + |o|) and the final division
+    u |o|."""
+    q = np.asarray(qp, dtype=np.float64).reshape(H, D)
+    dq = np.asarray(dqp, dtype=np.float64).reshape(H, D)
+    g = H // Hkv
+    scale = 1.0 / math.sqrt(D)
+    n_dot, n_res, n_acc = attention_depths(kv_len, D)
+    out = np.zeros((H, D))
+    err = np.zeros((H, D))
+    for h in range(H):
+        K_ = k_cache[h // g, :kv_len, :]
+        V_ = v_cache[h // g, :kv_len, :]
+        s = (K_ @ q[h]) * scale
+        ds = scale * (np.abs(K_) @ dq[h] + (3 * U32 + gamma(n_dot)) * (np.abs(K_) @ np.abs(q[h])))
+        m = s.max()
+        p = np.exp(s - m)
+        p = p / p.sum()
+        o = p @ V_
+        rng = m - s.min()
+        e = ds + U32 * (m - s) + EXPF_REL * (n_res + 2) + U32 * rng
+        out[h] = o
+        err[h] = (np.exp(2 * e.max()) * (p * e) @ np.abs(V_ - o[None, :])
+                  + gamma(n_acc) * (p @ np.abs(V_) + np.abs(o)) + U32 * np.abs(o))
+    return out.reshape(H * D), 1.01 * err.reshape(H * D)
+
+
+def silu_mul_rel_bound():
+    """Relative error bound of silu(z) * up from exact float32 z and up:
+    expf (4u) on 1 + e^{-z} gives at most 4u relative there, the add, the
+    division and the product one rounding each."""
+    return 1.01 * (EXPF_REL + gamma(3))
+
+
+LAYER_FP32_POINTS = ("q_proj", "k_proj", "v_proj", "x_attn", "gate", "up")
+LAYER_BF16_POINTS = ("xn", "k", "v", "att", "xn2", "h")
+
+
+def decode_layer_forced(cfg, lw, x, k_cache_l, v_cache_l, pos, forced, details=None):
+    """``decode_layer`` checked op by op against another implementation's
+    values of one layer (teacher-forced).
+
+    ``forced`` holds that implementation's values: its float32 GEMV outputs
+    ``q_proj`` [H*D], ``k_proj``, ``v_proj`` [Hkv*D] (before the per-head
+    norm), ``x_attn`` (the residual stream after o_proj and its residual
+    add) [hidden], ``gate``, ``up`` [ffn]; and its bf16 values at the
+    layer's rounding points ``xn`` (input norm) [hidden], ``k`` and ``v``
+    (the cache rows written at ``pos``) [Hkv*D], ``att`` (attention output)
+    [H*D], ``xn2`` (post-attention norm) [hidden], ``h`` (SiLU-mul) [ffn].
+
+    Every step is computed in float64 from the forced values before it, so
+    each comparison covers one op chain:
+      * the GEMV outputs are returned as references (``refs``), to be held
+        to the float32-accumulation tolerance by the caller: q/k/v_proj =
+        W xn, x_attn = x + W_o att, gate/up = W xn2, and ``y`` = x_attn +
+        W_down h (the layer's output);
+      * each rounding point is checked to be a correct bf16 rounding of the
+        float64 value of its op chain within that chain's float32 error
+        bound (``bf16_rounding_ok`` with the bounds above): xn from x, k from
+        k_proj (norm and RoPE), v from v_proj (exact), att from q_proj and
+        the cache (norm, RoPE, attention), xn2 from x_attn, h from gate and
+        up.
+    Returns ``(refs, bad)``: ``bad`` maps each rounding point to the indices
     whose forced value is not a correct rounding (with ``details``, a dict,
-    filled per point with those indices' own values, the forced values, their
-    distance to the rounding midpoint and the point's RMS). Rows ``pos`` of the caches
-    receive the forced (else the rounded) K and V."""
-    H, Hkv, D = cfg["heads"], cfg["kv_heads"], cfg["head_dim"]
+    filled per point with their values, the forced values and the bounds).
+    Rows ``pos`` of the caches receive the forced K and V rows."""
+    H, Hkv, D, hid = cfg["heads"], cfg["kv_heads"], cfg["head_dim"], cfg["hidden"]
     eps, theta = cfg["eps"], cfg["theta"]
-    unknown = set(forced) - {"xn", "k", "v", "att", "xn2", "h"}
-    if unknown:  # a misnamed point would silently go unforced
-        raise KeyError(f"decode_layer_forced: unknown rounding points {sorted(unknown)}")
+    names = set(LAYER_FP32_POINTS) | set(LAYER_BF16_POINTS)
+    if set(forced) != names:  # a misnamed or missing point would go unchecked
+        raise KeyError("decode_layer_forced: points must be exactly "
+                       f"{sorted(names)}, got {sorted(forced)}")
+    f = {k: np.asarray(v, dtype=np.float64).ravel() for k, v in forced.items()}
     bad = {}
 
-    def at(name, val):
-        if name not in forced:
-            return round_bf16(val)
-        f = np.asarray(forced[name], dtype=np.float64).reshape(val.shape)
-        # float32 errors of a vector's elements (cancellation in a dot
-        # product, in a rotation, in a residual add) scale with the vector,
-        # not the element: the error bound has a part relative to its RMS
-        scale = float(np.sqrt(np.mean(np.square(val[np.isfinite(val)])))) if val.size else 0.0
-        bad[name] = np.flatnonzero(~bf16_rounding_ok(val, f, rel, abs_rel * scale))
+    def check(name, val, bound):
+        bad[name] = np.flatnonzero(~bf16_rounding_ok(val, f[name], 0.0, bound))
         if details is not None and bad[name].size:
             i = bad[name]
-            mid = (round_bf16_down(val[i]) + round_bf16_up(val[i])) / 2.0
-            details[name] = {"index": i, "value": val[i], "forced": f[i],
-                             "to_midpoint": np.abs(val[i] - mid), "rms": scale}
-        return f
+            b = np.broadcast_to(bound, val.shape)[i]
+            details[name] = {"index": i, "value": val[i], "forced": f[name][i], "bound": b}
 
-    xn = at("xn", rmsnorm(x, lw["input_norm"], eps))
-    q = gemv_affine8(*lw["q"], xn[None])[0]
-    k = gemv_affine8(*lw["k"], xn[None])[0]
-    v = gemv_affine8(*lw["v"], xn[None])[0]
-    q = rope_neox(rmsnorm_perhead(q, lw["q_norm"], eps, D), pos, theta, D)
-    k = rope_neox(rmsnorm_perhead(k, lw["k_norm"], eps, D), pos, theta, D)
-    k_cache_l[:, pos, :] = at("k", k).reshape(Hkv, D)
-    v_cache_l[:, pos, :] = at("v", v).reshape(Hkv, D)
-    att = at("att", decode_attention(q, k_cache_l, v_cache_l, pos + 1, H, Hkv, D))
-    x = x + gemv_affine8(*lw["o"], att[None])[0]
-    xn2 = at("xn2", rmsnorm(x, lw["post_norm"], eps))
-    gate = gemv_affine8(*lw["gate"], xn2[None])[0]
-    up = gemv_affine8(*lw["up"], xn2[None])[0]
-    hmid = at("h", silu_mul(gate, up))
-    return x + gemv_affine8(*lw["down"], hmid[None])[0], bad
+    x = np.asarray(x, dtype=np.float64)
+    v = rmsnorm(x, lw["input_norm"], eps)
+    check("xn", v, rmsnorm_rel_bound(hid) * np.abs(v))
+    refs = {"q_proj": gemv_affine8(*lw["q"], f["xn"][None])[0],
+            "k_proj": gemv_affine8(*lw["k"], f["xn"][None])[0],
+            "v_proj": gemv_affine8(*lw["v"], f["xn"][None])[0]}
+    kr, kb = norm_rope_bound(f["k_proj"], lw["k_norm"], eps, pos, theta, D)
+    check("k", kr, kb)
+    check("v", f["v_proj"], 0.0)
+    k_cache_l[:, pos, :] = f["k"].reshape(Hkv, D)
+    v_cache_l[:, pos, :] = f["v"].reshape(Hkv, D)
+    qr, qb = norm_rope_bound(f["q_proj"], lw["q_norm"], eps, pos, theta, D)
+    att, ab = attention_bound(qr, qb, k_cache_l, v_cache_l, pos + 1, H, Hkv, D)
+    check("att", att, ab)
+    refs["x_attn"] = x + gemv_affine8(*lw["o"], f["att"][None])[0]
+    v2 = rmsnorm(f["x_attn"], lw["post_norm"], eps)
+    check("xn2", v2, rmsnorm_rel_bound(hid) * np.abs(v2))
+    refs["gate"] = gemv_affine8(*lw["gate"], f["xn2"][None])[0]
+    refs["up"] = gemv_affine8(*lw["up"], f["xn2"][None])[0]
+    hm = silu_mul(f["gate"], f["up"])
+    check("h", hm, silu_mul_rel_bound() * np.abs(hm))
+    refs["y"] = f["x_attn"] + gemv_affine8(*lw["down"], f["h"][None])[0]
+    return refs, bad
 
 
 def lm_head(cfg, weights, x):
@@ -545,11 +675,15 @@ def lm_head(cfg, weights, x):
     return gemv_affine8(ew, es, eb, xn[None])[0]
 
 
-def lm_head_tie_bound(cfg, weights, x, rel=2.0 ** -18):
-    """``lm_head`` plus the bound on the effect of bf16 rounding ties of the
-    final norm (see ``decode_layer_tie_bound``): the head is linear in the
-    normed vector, so a tie at element j moves logit r by
+def lm_head_tie_bound(cfg, weights, x, rel=None):
+    """``lm_head`` of an exact float32 residual ``x`` plus the bound on the
+    effect of bf16 rounding ties of the final norm: an element within the
+    norm's float32 error bound (``rmsnorm_rel_bound``) of a rounding
+    midpoint may round either way, and the head is linear in the normed
+    vector, so such a tie at element j moves logit r by
     ``|w[r][j]| * |alt_j - round_j|`` exactly. Returns ``(logits, extra)``."""
+    if rel is None:
+        rel = rmsnorm_rel_bound(cfg["hidden"])
     ew, es, eb = weights["embed"]
     v = rmsnorm(x, weights["final_norm"], cfg["eps"])
     xn = round_bf16(v)

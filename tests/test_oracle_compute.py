@@ -347,75 +347,174 @@ def _small_layer():
     return cfg, w["layers"][0], x, kc[0], vc[0]
 
 
-def test_decode_layer_forced_with_its_own_roundings_is_decode_layer():
-    cfg, lw, x, kc, vc = _small_layer()
+# ---- float32 emulation of one decoder layer (test code): the same ops as the
+# oracle's layer in numpy float32, in orders of its own (sequential sums,
+# an online softmax over row batches), for the bound pins below.
+
+F32 = np.float32
+
+
+def _f32_rmsnorm(x, w_bits, eps):
+    x = np.asarray(x, F32)
+    ss = F32(0)
+    for v in x:                        # sequential: the longest chain
+        ss = F32(ss + F32(v * v))
+    inv = F32(1) / F32(np.sqrt(F32(F32(ss / F32(x.size)) + F32(eps))))
+    return F32(x * inv) * F32(O.bf16_bits_to_f64(w_bits))
+
+
+def _f32_norm_rope(x, w_bits, eps, pos, theta, D):
+    h = np.asarray(x, F32).reshape(-1, D)
+    out = np.empty_like(h)
+    a = pos * O.rope_inv_freq(theta, D)
+    c, s = F32(np.cos(a)), F32(np.sin(a))
+    for i in range(h.shape[0]):
+        n = _f32_rmsnorm(h[i], w_bits, eps)
+        x1, x2 = n[:D // 2], n[D // 2:]
+        out[i, :D // 2] = F32(x1 * c) - F32(x2 * s)
+        out[i, D // 2:] = F32(x2 * c) + F32(x1 * s)
+    return out.ravel()
+
+
+def _f32_attention(q, kc, vc, L, H, Hkv, D, batch=24):
+    """Online softmax over batches of rows, float32, like the kernels."""
+    q = np.asarray(q, F32).reshape(H, D) * F32(F32(1) / F32(np.sqrt(F32(D))))
+    out = np.zeros((H, D), F32)
+    g = H // Hkv
+    for h in range(H):
+        K_, V_ = kc[h // g, :L].astype(F32), vc[h // g, :L].astype(F32)
+        m, l, o = F32(-np.inf), F32(0), np.zeros(D, F32)
+        for t0 in range(0, L, batch):
+            sc = (K_[t0:t0 + batch] @ q[h]).astype(F32)
+            mx = F32(max(m, sc.max()))
+            a = F32(np.exp(F32(m - mx)))
+            l, o = F32(l * a), (o * a).astype(F32)
+            for t in range(sc.size):
+                p = F32(np.exp(F32(sc[t] - mx)))
+                l = F32(l + p)
+                o = (o + p * V_[t0 + t]).astype(F32)
+            m = mx
+        out[h] = o / l
+    return out.ravel()
+
+
+def _f32_gemv(lw_m, x):
+    w = O.affine8_dequant_f32(*lw_m)
+    return (w @ np.asarray(x, F32)).astype(F32)
+
+
+def _f32_silu_mul(gate, up):
+    z = np.asarray(gate, F32)
+    return (F32(z / F32(F32(1) + np.exp(-z).astype(F32))) * np.asarray(up, F32)).astype(F32)
+
+
+def _f32_layer(cfg, lw, x, kc, vc, pos):
+    """One layer in float32 with bf16 stores at the rounding points: the
+    values another implementation would hand to decode_layer_forced."""
+    H, Hkv, D, eps, th = cfg["heads"], cfg["kv_heads"], cfg["head_dim"], cfg["eps"], cfg["theta"]
+    r = {}
+    r["xn"] = O.round_bf16(_f32_rmsnorm(x, lw["input_norm"], eps))
+    r["q_proj"] = _f32_gemv(lw["q"], r["xn"])
+    r["k_proj"] = _f32_gemv(lw["k"], r["xn"])
+    r["v_proj"] = _f32_gemv(lw["v"], r["xn"])
+    r["k"] = O.round_bf16(_f32_norm_rope(r["k_proj"], lw["k_norm"], eps, pos, th, D))
+    r["v"] = O.round_bf16(r["v_proj"])
     k1, v1 = kc.copy(), vc.copy()
-    y = O.decode_layer(cfg, lw, x, k1, v1, 9)
-    # no forced values: the same layer
+    k1[:, pos, :] = r["k"].reshape(Hkv, D)
+    v1[:, pos, :] = r["v"].reshape(Hkv, D)
+    qp = _f32_norm_rope(r["q_proj"], lw["q_norm"], eps, pos, th, D)
+    r["att"] = O.round_bf16(_f32_attention(qp, k1, v1, pos + 1, H, Hkv, D))
+    r["x_attn"] = (np.asarray(x, F32) + _f32_gemv(lw["o"], r["att"])).astype(F32)
+    r["xn2"] = O.round_bf16(_f32_rmsnorm(r["x_attn"], lw["post_norm"], eps))
+    r["gate"] = _f32_gemv(lw["gate"], r["xn2"])
+    r["up"] = _f32_gemv(lw["up"], r["xn2"])
+    r["h"] = O.round_bf16(_f32_silu_mul(r["gate"], r["up"]))
+    y = (r["x_attn"] + _f32_gemv(lw["down"], r["h"])).astype(F32)
+    return {k: np.asarray(v, np.float64) for k, v in r.items()}, y.astype(np.float64)
+
+
+def test_float32_op_chains_stay_within_their_derived_bounds():
+    """Each bound holds for a float32 evaluation of its chain (sequential
+    sums, batched online softmax), and is not vacuous: far below half a bf16
+    step relative to the values it bounds."""
+    rng = np.random.default_rng(5)
+    cfg, lw, x, kc, vc = _small_layer()
+    eps, th, D = cfg["eps"], cfg["theta"], cfg["head_dim"]
+    xf = rng.standard_normal(512).astype(F32) * F32(3)
+    v = O.rmsnorm(xf, lw["input_norm"], eps)
+    err = np.abs(_f32_rmsnorm(xf, lw["input_norm"], eps) - v)
+    rel = O.rmsnorm_rel_bound(512)
+    assert np.all(err <= rel * np.abs(v)) and rel < 2.0 ** -17
+    kp = rng.standard_normal(2 * D).astype(F32)
+    kr, kb = O.norm_rope_bound(kp, lw["k_norm"], eps, 9, th, D)
+    assert np.all(np.abs(_f32_norm_rope(kp, lw["k_norm"], eps, 9, th, D) - kr) <= kb)
+    assert np.max(kb) < 2.0 ** -16 * np.sqrt(np.mean(kr ** 2)) * 8
+    H, Hkv = cfg["heads"], cfg["kv_heads"]
+    qp = rng.standard_normal(H * D).astype(F32)
+    att, ab = O.attention_bound(qp, np.zeros(H * D), kc, vc, 10, H, Hkv, D)
+    np.testing.assert_allclose(att, O.decode_attention(qp, kc, vc, 10, H, Hkv, D), atol=1e-12)
+    assert np.all(np.abs(_f32_attention(qp, kc, vc, 10, H, Hkv, D) - att) <= ab)
+    assert np.max(ab) < 2.0 ** -14 * np.max(np.abs(vc))
+    # a query known only within dq widens the bound by about the score error
+    _, ab2 = O.attention_bound(qp, np.full(H * D, 1e-3), kc, vc, 10, H, Hkv, D)
+    assert np.all(ab2 > ab)
+    g, u = rng.standard_normal(1000).astype(F32) * F32(4), rng.standard_normal(1000).astype(F32)
+    hm = O.silu_mul(g, u)
+    assert np.all(np.abs(_f32_silu_mul(g, u) - hm) <= O.silu_mul_rel_bound() * np.abs(hm))
+
+
+def test_decode_layer_forced_accepts_a_float32_layer_and_follows_it():
+    """A float32 layer with bf16 stores passes every rounding check; its GEMV
+    outputs meet the float32-accumulation tolerance against the references;
+    and the returned output follows the forced values."""
+    cfg, lw, x, kc, vc = _small_layer()
+    forced, y32 = _f32_layer(cfg, lw, x, kc, vc, 9)
     k2, v2 = kc.copy(), vc.copy()
-    y2, bad = O.decode_layer_forced(cfg, lw, x, k2, v2, 9, {})
-    np.testing.assert_array_equal(y2, y)
-    np.testing.assert_array_equal(k2, k1)
-    assert bad == {}
-    # forcing the rounded values the layer computes itself changes nothing
-    D, eps = cfg["head_dim"], cfg["eps"]
-    xn = O.round_bf16(O.rmsnorm(x, lw["input_norm"], eps))
-    k3, v3 = kc.copy(), vc.copy()
-    y3, bad3 = O.decode_layer_forced(cfg, lw, x, k3, v3, 9,
-                                     {"xn": xn, "k": k1[:, 9, :].ravel(), "v": v1[:, 9, :].ravel()})
-    np.testing.assert_array_equal(y3, y)
-    assert all(b.size == 0 for b in bad3.values())
+    refs, bad = O.decode_layer_forced(cfg, lw, x, k2, v2, 9, forced)
+    assert set(bad) == set(O.LAYER_BF16_POINTS)
+    assert all(b.size == 0 for b in bad.values()), {k: b[:5] for k, b in bad.items()}
+    for name in O.LAYER_FP32_POINTS:
+        np.testing.assert_allclose(forced[name], refs[name], rtol=1e-3, atol=2e-3)
+    np.testing.assert_allclose(y32, refs["y"], rtol=1e-3, atol=2e-3)
+    np.testing.assert_array_equal(k2[:, 9, :].ravel(), forced["k"])
+    # with its own rounded values forced, the float64 layer is reproduced
+    # up to the float32 GEMV outputs it is then fed
+    y64 = O.decode_layer(cfg, lw, x, kc.copy(), vc.copy(), 9)
+    np.testing.assert_allclose(refs["y"], y64, rtol=1e-3, atol=2e-3)
 
 
-def test_decode_layer_forced_flags_wrong_values_and_follows_valid_ones():
+def test_decode_layer_forced_flags_planted_mistakes():
+    """Mistakes a kernel could make are flagged at their rounding point: a
+    value two bf16 steps off, gate and up swapped in the SiLU-mul, the RoPE
+    sign flipped, a K/V head taken from the wrong head, an attention output
+    row of another head; a missing or misnamed point is an error."""
     cfg, lw, x, kc, vc = _small_layer()
-    eps = cfg["eps"]
-    v = O.rmsnorm(x, lw["input_norm"], eps)
-    xn = O.round_bf16(v)
-    # a value two bf16 steps off is flagged at its index
-    wrong = xn.copy()
-    wrong[5] = O.round_bf16_up(xn[5] * (1 + 2.0 ** -7) + 1e-30)
-    wrong[5] = O.round_bf16_up(wrong[5] * (1 + 2.0 ** -7) + 1e-30)
-    _, bad = O.decode_layer_forced(cfg, lw, x, kc.copy(), vc.copy(), 9, {"xn": wrong})
-    assert list(bad["xn"]) == [5]
-    # the other neighbour is accepted only where the value is near a tie: with
-    # a tie window of a full bf16 step every neighbour passes, and the layer
-    # then follows the forced value (its output differs from the plain layer)
-    lo, hi = O.round_bf16_down(v), O.round_bf16_up(v)
-    other = np.where(xn == lo, hi, lo)
-    y_plain = O.decode_layer(cfg, lw, x, kc.copy(), vc.copy(), 9)
-    y_f, bad_f = O.decode_layer_forced(cfg, lw, x, kc.copy(), vc.copy(), 9, {"xn": other},
-                                       rel=2.0 ** -7, abs_rel=0.0)
-    assert bad_f["xn"].size == 0 and np.abs(y_f - y_plain).max() > 0
-    _, bad_t = O.decode_layer_forced(cfg, lw, x, kc.copy(), vc.copy(), 9, {"xn": other})
-    assert bad_t["xn"].size > 300   # with the default bound most are wrong
+    H, Hkv, D = cfg["heads"], cfg["kv_heads"], cfg["head_dim"]
+    forced, _ = _f32_layer(cfg, lw, x, kc, vc, 9)
 
+    def bad_of(**change):
+        f = dict(forced, **change)
+        return O.decode_layer_forced(cfg, lw, x, kc.copy(), vc.copy(), 9, f)[1]
 
-def test_decode_layer_forced_follows_a_forced_attention_and_rejects_unknown_points():
-    cfg, lw, x, kc, vc = _small_layer()
-    # forcing the attention output to its other rounding neighbour at one
-    # element changes the layer's output by exactly that element's effect
-    # through o_proj onward; a misnamed point is an error, not a silent no-op
-    y_plain = O.decode_layer(cfg, lw, x, kc.copy(), vc.copy(), 9)
-    H, D = cfg["heads"], cfg["head_dim"]
-    xn = O.round_bf16(O.rmsnorm(x, lw["input_norm"], cfg["eps"]))
-    k1, v1 = kc.copy(), vc.copy()
-    O.decode_layer(cfg, lw, x, k1, v1, 9)
-    q = O.gemv_affine8(*lw["q"], xn[None])[0]
-    q = O.rope_neox(O.rmsnorm_perhead(q, lw["q_norm"], cfg["eps"], D), 9, cfg["theta"], D)
-    att_v = O.decode_attention(q, k1, v1, 10, H, cfg["kv_heads"], D)
-    att = O.round_bf16(att_v)
-    flipped = att.copy()
-    j = int(np.argmax(np.abs(att)))
-    flipped[j] = O.round_bf16_up(att_v[j]) if att[j] == O.round_bf16_down(att_v[j]) \
-        else O.round_bf16_down(att_v[j])
-    y_same, _ = O.decode_layer_forced(cfg, lw, x, kc.copy(), vc.copy(), 9, {"att": att})
-    np.testing.assert_array_equal(y_same, y_plain)
-    y_flip, bad = O.decode_layer_forced(cfg, lw, x, kc.copy(), vc.copy(), 9, {"att": flipped},
-                                        rel=2.0 ** -7, abs_rel=0.0)
-    assert bad["att"].size == 0 and np.abs(y_flip - y_plain).max() > 0
+    two = forced["xn"].copy()
+    two[5] = O.round_bf16_up(O.round_bf16_up(two[5] * (1 + 2.0 ** -7)) * (1 + 2.0 ** -7))
+    assert list(bad_of(xn=two)["xn"]) == [5]
+    swapped = O.round_bf16(O.silu_mul(forced["up"], forced["gate"]))
+    assert bad_of(h=swapped)["h"].size > 0.5 * swapped.size
+    kp = O.rmsnorm_perhead(forced["k_proj"], lw["k_norm"], cfg["eps"], D)
+    wrong_sign = O.round_bf16(O.rope_neox(kp, -9, cfg["theta"], D))
+    assert bad_of(k=wrong_sign)["k"].size > 0.5 * wrong_sign.size
+    v_heads = forced["v"].reshape(Hkv, D)[::-1].ravel()
+    assert bad_of(v=v_heads)["v"].size > 0.5 * v_heads.size
+    att_rows = forced["att"].reshape(H, D)[[1, 0] + list(range(2, H))].ravel()
+    assert bad_of(att=att_rows)["att"].size > 0.5 * D
     with pytest.raises(KeyError):
-        O.decode_layer_forced(cfg, lw, x, kc.copy(), vc.copy(), 9, {"attn": att})
+        O.decode_layer_forced(cfg, lw, x, kc.copy(), vc.copy(), 9,
+                              {k: v for k, v in forced.items() if k != "h"})
+    f = dict(forced)
+    f["attn"] = f.pop("att")
+    with pytest.raises(KeyError):
+        O.decode_layer_forced(cfg, lw, x, kc.copy(), vc.copy(), 9, f)
 
 
 def test_lm_head_tie_bound_is_the_exact_linear_effect_of_each_tie():
