@@ -717,6 +717,86 @@ def new_kv_cache(cfg, cap):
 
 
 # ---------------------------------------------------------------------------
+# The Whisper encoder layer  [FT: encoder_layer, multi_head_attn,
+# layer_norm_affine, q_linear]
+# ---------------------------------------------------------------------------
+
+def layer_norm(x, gamma, beta, eps):
+    """LayerNorm over the last axis with an affine f32 gamma and beta ([FT]
+    ``layer_norm_affine``: ``layer_norm_last_dim`` then ``* g + b``): the
+    mean and the biased variance of the row, ``(x - mean) / sqrt(var + eps)
+    * gamma + beta``."""
+    x = np.asarray(x, dtype=np.float64)
+    mu = x.mean(axis=-1, keepdims=True)
+    var = np.mean((x - mu) ** 2, axis=-1, keepdims=True)
+    return (x - mu) / np.sqrt(var + eps) * np.asarray(gamma, np.float64) + np.asarray(beta, np.float64)
+
+
+def gelu_tanh(x):
+    """The tanh form of GELU named by [FT] (``gelu_tanh``):
+    ``0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3)))``."""
+    x = np.asarray(x, dtype=np.float64)
+    return 0.5 * x * (1.0 + np.tanh(math.sqrt(2.0 / math.pi) * (x + 0.044715 * x ** 3)))
+
+
+def mha_rows(q, k, v, n_heads, causal=False, kv_heads=None):
+    """Multi-head softmax attention of [FT] ``multi_head_attn`` for all rows
+    at once: q ``[T, H*D]``, k and v ``[S, Hkv*D]``, per head
+    ``softmax(q_h k_h^T / sqrt(D)) v_h`` over all S rows, or with
+    ``causal`` over rows ``j <= i`` (the mask of [FT] and of [MK]
+    ``causal_mask``). With ``kv_heads`` < heads, query head h reads KV head
+    ``h // (H / Hkv)`` ([MK] ``repeat_kv``). float64; returns ``[T, H*D]``."""
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    T = q.shape[0]
+    S = k.shape[0]
+    Hkv = n_heads if kv_heads is None else kv_heads
+    D = q.shape[1] // n_heads
+    g = n_heads // Hkv
+    out = np.zeros((T, n_heads * D))
+    for h in range(n_heads):
+        kh = h // g
+        s = q[:, h * D:(h + 1) * D] @ k[:, kh * D:(kh + 1) * D].T / math.sqrt(D)
+        if causal:
+            s = s + np.triu(np.full((T, S), -np.inf), k=1 + S - T)
+        p = np.exp(s - s.max(axis=1, keepdims=True))
+        p = p / p.sum(axis=1, keepdims=True)
+        out[:, h * D:(h + 1) * D] = p @ v[:, kh * D:(kh + 1) * D]
+    return out
+
+
+def whisper_encoder_layer(x, lw, n_heads, eps=1e-5, details=None):
+    """One Whisper encoder layer ([FT] ``encoder_layer``), pre-LayerNorm:
+    ``x + out(attn(LN1(x)))`` then ``+ fc2(gelu_tanh(fc1(LN2(.))))``, with
+    ``q_linear`` as the Q4_0 matmul under this library's tensor-core operand
+    contract (``gemm_q4_0_bf16``: operands rounded to bf16). k_proj has no
+    bias; q, v, out, fc1 and fc2 have f32 biases.
+
+    Precision points (where the GPU stores bf16; rounded here as well): the
+    LayerNorm outputs, q, k and v (the attention operands), the attention
+    output (the out projection's input) and the GELU output (fc2's input).
+    The residual stream stays float64 (float32 on the GPU).
+
+    ``x`` ``[T, d]``; ``lw`` holds ``ln1_g, ln1_b, q, q_b, k, v, v_b, o, o_b,
+    ln2_g, ln2_b, fc1, fc1_b, fc2, fc2_b`` (Q4_0 blocks and f32 vectors).
+    With ``details`` (a dict) the intermediate values are stored in it."""
+    x = np.asarray(x, np.float64)
+    xl = round_bf16(layer_norm(x, lw["ln1_g"], lw["ln1_b"], eps))
+    q = round_bf16(gemm_q4_0_bf16(lw["q"], xl, lw["q_b"]))
+    k = round_bf16(gemm_q4_0_bf16(lw["k"], xl))
+    v = round_bf16(gemm_q4_0_bf16(lw["v"], xl, lw["v_b"]))
+    ctx = round_bf16(mha_rows(q, k, v, n_heads))
+    xa = x + gemm_q4_0_bf16(lw["o"], ctx, lw["o_b"])
+    xl2 = round_bf16(layer_norm(xa, lw["ln2_g"], lw["ln2_b"], eps))
+    mid = round_bf16(gelu_tanh(gemm_q4_0_bf16(lw["fc1"], xl2, lw["fc1_b"])))
+    y = xa + gemm_q4_0_bf16(lw["fc2"], mid, lw["fc2_b"])
+    if details is not None:
+        details.update(xl=xl, q=q, k=k, v=v, ctx=ctx, xa=xa, xl2=xl2, mid=mid, y=y)
+    return y
+
+
+# ---------------------------------------------------------------------------
 # The code predictor  [MK: src/tts/qwen3/code_predictor.rs]
 # ---------------------------------------------------------------------------
 
