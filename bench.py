@@ -99,61 +99,206 @@ def graph_time_ms(fns, stream, n, warm=3):
 L2_BYTES = 126 << 20
 
 
-def other_kernels(qg, stream, hbm_peak, n):
-    """The Whisper-shaped Q4_0 rows: the FC1 GEMM (M=1500, N=5120, K=1280) on
-    the tensor cores against the measured bf16 peak, and the same matrix as a
-    batch-1 Q4_0 GEMV against the HBM peak."""
+def _tob(a):
+    """numpy -> torch on the device (uint16/uint32 travel as int16/int32)."""
     import torch
-    to = lambda a: torch.from_numpy(a).cuda()
-    M, N, K = 1500, 5120, 1280
-    bnp = qg_synth.q4_0_packed(N, K, 22)
-    blocks = to(bnp)
-    A = to(qg_synth.gaussian((M, K), 1.0, 23).astype(np.float32))
-    C = torch.empty((M, N), dtype=torch.float32, device="cuda")
-    ws = torch.empty(qg.qg_gemm_q4_0_workspace_size(M, N, K), dtype=torch.uint8, device="cuda")
-    ms = graph_time_ms([lambda: qg.qg_gemm_q4_0(blocks, A, C, ws=ws, stream=stream)], stream, n)
+    return torch.from_numpy(a.view({1: np.uint8, 2: np.int16, 4: np.int32}[a.dtype.itemsize])).cuda()
+
+
+def _hbm_entry(nbytes, ms, peak, **extra):
+    gbs = nbytes / (ms / 1000.0) / 1e9
+    d = {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+         "algorithmic_bytes": nbytes, "launch_us": ms * 1000.0}
+    d.update(extra)
+    return d
+
+
+def affine8_chain(qg, stream, N, K, B, seed, n_min, hbm_peak):
+    """One affine8 GEMV N x K at batch B, timed per launch as a chain of
+    launches back to back in a CUDA graph over rotated copies of the matrix
+    that together exceed L2 three times (so every launch streams from HBM)."""
+    import torch
+    wnp, snp, bnp = qg_synth.affine8_packed(N, K, seed)
+    per = wnp.nbytes + snp.nbytes + bnp.nbytes
+    copies = max(1, -(-3 * L2_BYTES // per))
+    mats = [(_tob(wnp), _tob(snp), _tob(bnp)) for _ in range(copies)]
+    x = torch.from_numpy(qg_synth.gaussian_bf16_bits((B, K), 1.0, seed + 1).view(np.int16)) \
+        .cuda().view(torch.bfloat16)
+    y = torch.empty((B, N), dtype=torch.float32, device="cuda")
+    fns = [(lambda m=m: qg.qg_gemv_affine8_g64(*m, x, y, stream=stream)) for m in mats]
+    ms = graph_time_ms(fns, stream, max(n_min, 2 * copies))
+    del mats
+    return _hbm_entry(affine8_bytes(N, K, B), ms, hbm_peak,
+                      note=f"chain in a CUDA graph over {copies} copies (> 3x L2)")
+
+
+def c1_c2_gemvs(qg, stream, hbm_peak):
+    """C1: the 1024 x 1024 GEMV at B = 1 as a chain of 512 launches. C2: the
+    Qwen3-0.6B layer set (q, k, v, o, gate, up, down) and the tied LM head
+    151936 x 1024 at B = 1, 4 and 16."""
+    out = {"gemv_affine8_1024x1024_b1_chain": affine8_chain(qg, stream, 1024, 1024, 1, 31, 512,
+                                                           hbm_peak)}
+    cfg = qg_synth.QWEN3_0_6B
+    sh = dict(qg_synth.linear_shapes(cfg))
+    sh["lm_head"] = (cfg["vocab"], cfg["hidden"])
+    c2 = {}
+    for B in (1, 4, 16):
+        for i, (name, (N, K)) in enumerate(sh.items()):
+            c2[f"{name}_b{B}"] = affine8_chain(qg, stream, N, K, B, 40 + i, 64, hbm_peak)
+    tot = {B: sum(c2[f"{n}_b{B}"]["algorithmic_bytes"] for n in sh) for B in (1, 4, 16)}
+    us = {B: sum(c2[f"{n}_b{B}"]["launch_us"] for n in sh) for B in (1, 4, 16)}
+    out["c2_qwen3_0.6b_layer_set"] = {
+        "workload": "Qwen3-0.6B layer GEMVs q 2048x1024, k/v 1024x1024, o 1024x2048, gate/up "
+                    "3072x1024, down 1024x3072 and the tied LM head 151936x1024, affine8 g64",
+        "per_matrix": c2,
+        "set_gbs": {f"b{B}": tot[B] / (us[B] / 1e6) / 1e9 for B in (1, 4, 16)},
+        "set_frac": {f"b{B}": tot[B] / (us[B] / 1e6) / 1e9 / hbm_peak for B in (1, 4, 16)},
+        "note": "each matrix timed alone per launch (chained launches in a CUDA graph, "
+                "inputs rotated over > 3x L2); set figures = total bytes / summed launch times"}
+    return out
+
+
+def c4_whisper(qg, stream, hbm_peak):
+    """C4: the Whisper-large-v3 encoder's Q4_0 matmuls at M = 1500 on the
+    tensor cores (Q/K/V/O 1280x1280, FC1 5120x1280, FC2 1280x5120) and the
+    same matrices as batch-1 Q4_0 GEMVs."""
+    import torch
+    M = 1500
     tf_peak, tf_kind = measured_tensor_peak()
-    tflops = 2.0 * M * N * K / (ms / 1000.0) / 1e12
-    # the GEMV streams copies of the matrix that together exceed L2 three times
-    vbytes = N * (K // 32) * 18 + K * 4 + N * 4
-    copies = -(-3 * L2_BYTES // bnp.nbytes)
-    mats = [to(bnp) for _ in range(copies)]
-    x = to(qg_synth.gaussian((1, K), 1.0, 13).astype(np.float32))
-    y = torch.empty((1, N), dtype=torch.float32, device="cuda")
-    fns = [(lambda m=m: qg.qg_gemv_q4_0(m, x, y, stream=stream)) for m in mats]
-    ms_v = graph_time_ms(fns, stream, max(n, 2 * copies))
-    # C1: the single 1024 x 1024 affine8 GEMV at B = 1, as a chain of 512
-    # launches over rotated copies (together more than 3x L2)
-    wnp, snp, bnp8 = qg_synth.affine8_packed(1024, 1024, 31)
-    tob = lambda a: torch.from_numpy(a.view({2: np.int16, 4: np.int32}[a.dtype.itemsize])).cuda()
-    c1_bytes = affine8_bytes(1024, 1024, 1)
-    c1_copies = -(-3 * L2_BYTES // (wnp.nbytes + snp.nbytes + bnp8.nbytes))
-    c1_mats = [(tob(wnp), tob(snp), tob(bnp8)) for _ in range(c1_copies)]
-    x1 = torch.from_numpy(qg_synth.gaussian_bf16_bits((1, 1024), 1.0, 32)).view(torch.bfloat16).cuda()
-    y1 = torch.empty((1, 1024), dtype=torch.float32, device="cuda")
-    c1_fns = [(lambda m=m: qg.qg_gemv_affine8_g64(*m, x1, y1, stream=stream)) for m in c1_mats]
-    ms_c1 = graph_time_ms(c1_fns, stream, 512)
-    del c1_mats
-    return {
-        "gemv_affine8_1024x1024_b1_chain": {
-            "bound": "hbm", "achieved": c1_bytes / (ms_c1 / 1000.0) / 1e9, "peak": hbm_peak,
-            "unit": "GB/s", "frac": c1_bytes / (ms_c1 / 1000.0) / 1e9 / hbm_peak,
-            "algorithmic_bytes": c1_bytes, "launch_us": ms_c1 * 1000.0,
-            "note": f"512 launches back to back in a CUDA graph (PDL) over {c1_copies} "
-                    "copies of the matrix (more than 3x L2)"},
-        "gemm_q4_0_whisper_fc1": {
-            "shape": [M, N, K], "bound": "tensor", "achieved": tflops, "peak": tf_peak,
-            "unit": "TFLOP/s", "frac": tflops / tf_peak, "launch_us": ms * 1000.0,
-            "peak_kind": tf_kind,
-            "note": "includes the A fp32->bf16 pass; FLOPs 2*M*N*K (dequant work not counted); "
-                    "back-to-back launches in a CUDA graph"},
-        "gemv_q4_0_5120x1280_b1": {
-            "bound": "hbm", "achieved": vbytes / (ms_v / 1000.0) / 1e9, "peak": hbm_peak,
-            "unit": "GB/s", "frac": vbytes / (ms_v / 1000.0) / 1e9 / hbm_peak,
-            "algorithmic_bytes": vbytes, "launch_us": ms_v * 1000.0,
-            "note": f"back-to-back launches in a CUDA graph over {copies} copies of the matrix "
-                    "(more than 3x L2)"},
-    }
+    gemm = {}
+    for name, (N, K) in (("qkvo_1280x1280", (1280, 1280)), ("fc1_5120x1280", (5120, 1280)),
+                         ("fc2_1280x5120", (1280, 5120))):
+        blocks = _tob(qg_synth.q4_0_packed(N, K, 22))
+        A = torch.from_numpy(qg_synth.gaussian((M, K), 1.0, 23).astype(np.float32)).cuda()
+        bias = torch.from_numpy(qg_synth.gaussian((N,), 0.1, 24).astype(np.float32)).cuda()
+        C = torch.empty((M, N), dtype=torch.float32, device="cuda")
+        ws = torch.empty(qg.qg_gemm_q4_0_workspace_size(M, N, K), dtype=torch.uint8, device="cuda")
+        ms = graph_time_ms([lambda: qg.qg_gemm_q4_0(blocks, A, C, bias=bias, ws=ws, stream=stream)],
+                           stream, 50)
+        tf = 2.0 * M * N * K / (ms / 1000.0) / 1e12
+        gemm[name] = {"shape": [M, N, K], "bound": "tensor", "achieved": tf, "peak": tf_peak,
+                      "unit": "TFLOP/s", "frac": tf / tf_peak, "launch_us": ms * 1000.0,
+                      "peak_kind": tf_kind}
+    gemv = {}
+    for name, (N, K) in (("1280x1280", (1280, 1280)), ("5120x1280", (5120, 1280)),
+                         ("1280x5120", (1280, 5120))):
+        bnp = qg_synth.q4_0_packed(N, K, 25)
+        copies = -(-3 * L2_BYTES // bnp.nbytes)
+        mats = [_tob(bnp) for _ in range(copies)]
+        x = torch.from_numpy(qg_synth.gaussian((1, K), 1.0, 13).astype(np.float32)).cuda()
+        bias = torch.from_numpy(qg_synth.gaussian((N,), 0.1, 26).astype(np.float32)).cuda()
+        y = torch.empty((1, N), dtype=torch.float32, device="cuda")
+        fns = [(lambda m=m: qg.qg_gemv_q4_0(m, x, y, bias=bias, stream=stream)) for m in mats]
+        ms = graph_time_ms(fns, stream, max(100, 2 * copies))
+        vbytes = N * (K // 32) * 18 + K * 4 + N * 4 + N * 4
+        gemv[name] = _hbm_entry(vbytes, ms, hbm_peak,
+                                note=f"chain in a CUDA graph over {copies} copies (> 3x L2)")
+        del mats
+    return {"c4_whisper_q4_0": {
+        "workload": "Whisper-large-v3 encoder projections as Q4_0 blk32, M = 1500 frames "
+                    "(GEMM, f32 activations rounded to bf16) and batch 1 (GEMV)",
+        "gemm": gemm, "gemv_b1": gemv,
+        "note": "GEMM FLOPs 2*M*N*K (dequant work not counted), includes the A fp32->bf16 pass"}}
+
+
+def step_graph(model, st, toks, pos, stream):
+    """One decode step captured into a CUDA graph (after two eager steps)."""
+    import torch
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            model.qg_decode_step(st, toks, pos, stream=stream)
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        model.qg_decode_step(st, toks, pos, stream=stream)
+    return g
+
+
+def time_replays(g, stream, n, warm=3):
+    import torch
+    with torch.cuda.stream(stream):
+        for _ in range(warm):
+            g.replay()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(n):
+            g.replay()
+        e1.record(stream)
+    stream.synchronize()
+    return e0.elapsed_time(e1) / n
+
+
+def c3_batch10(qg, stream, hbm_peak, model, cfg):
+    """C3 at batch 10: the 0.6B step at KV 512 for 10 sequences."""
+    import torch
+    B = 10
+    st = model.new_state(B, KV_LEN + 1)
+    st["k_cache"].normal_()
+    st["v_cache"].normal_()
+    toks = torch.from_numpy(qg_synth.tokens(B, cfg["vocab"], 73)).cuda()
+    pos = torch.full((B,), KV_LEN - 1, dtype=torch.int32, device="cuda")
+    g = step_graph(model, st, toks, pos, stream)
+    ms = time_replays(g, stream, 100)
+    del g, st
+    sb = step_bytes(cfg, B, KV_LEN)
+    return {"c3_qwen3_0.6b_step_b10_kv512": {
+        "steps_per_s": 1000.0 / ms, "tokens_per_s": B * 1000.0 / ms, "us_per_step": ms * 1000.0,
+        "algorithmic_bytes": sb, "achieved": sb / (ms / 1000.0) / 1e9, "peak": hbm_peak,
+        "unit": "GB/s", "frac": sb / (ms / 1000.0) / 1e9 / hbm_peak}}
+
+
+def c5_1_7b(qg, stream, hbm_peak):
+    """C5: the Qwen3-1.7B-shaped decode (hidden 2048, FFN 6144, 28 layers,
+    vocab 151936) at KV 2048 (position 2047) for batch 1, 8 and 32, and the
+    256-row prefill (as decode steps at positions 0..255, batch 1)."""
+    import torch
+    import weight_only_quantized_03_b200 as qgm
+    cfg = dict(qg_synth.QWEN3_1_7B)
+    model = qgm.Qwen3Model(cfg, qg_synth.qwen3_weights(cfg, 19))
+    cap = 2049
+    out = {"workload": "Qwen3-1.7B-shaped affine-INT8 g64 decode, KV 2048", "points": {}}
+    for B in (1, 8, 32):
+        st = model.new_state(B, cap)
+        st["k_cache"].normal_()
+        st["v_cache"].normal_()
+        toks = torch.from_numpy(qg_synth.tokens(B, cfg["vocab"], 92)).cuda()
+        pos = torch.full((B,), 2047, dtype=torch.int32, device="cuda")
+        g = step_graph(model, st, toks, pos, stream)
+        ms = time_replays(g, stream, 30)
+        sb = step_bytes(cfg, B, 2048)
+        out["points"][f"b{B}"] = {"us_per_step": ms * 1000.0, "tokens_per_s": B * 1000.0 / ms,
+                                  "algorithmic_bytes": sb, "achieved": sb / (ms / 1000.0) / 1e9,
+                                  "frac": sb / (ms / 1000.0) / 1e9 / hbm_peak}
+        del g, st
+        torch.cuda.empty_cache()
+    out["prefill_256_rows"] = prefill_rows(qg, model, cfg, stream)
+    out["peak"] = hbm_peak
+    out["unit"] = "GB/s"
+    return {"c5_qwen3_1.7b": out}
+
+
+def prefill_rows(qg, model, cfg, stream):
+    """256 prompt rows of one sequence, each run as a decode step (graph
+    replay) at positions 0..255."""
+    import torch
+    st = model.new_state(1, 2049)
+    toks = torch.from_numpy(qg_synth.tokens(256, cfg["vocab"], 91)).cuda()
+    pos = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tok1 = toks[:1].clone()
+    g = step_graph(model, st, tok1, pos, stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for r in range(256):
+            pos.fill_(r)
+            tok1.copy_(toks[r:r + 1])
+            g.replay()
+        e1.record(stream)
+    stream.synchronize()
+    ms = e0.elapsed_time(e1)
+    del g, st
+    return {"ms": ms, "rows_per_s": 256 / (ms / 1000.0), "method": "row at a time (decode steps)"}
 
 
 def code_predictor_frame(qg, stream, hbm_peak, n):
@@ -225,24 +370,33 @@ def source_sha256(paths):
     return h.hexdigest()
 
 
-LM_HEAD_SOURCES = [os.path.join(ROOT, "weight_only_quantized_03_b200", "csrc", f)
-                   for f in ("gemv_affine8_tc.cu", "gemv_tc.cuh")]
+GEMV_SOURCES = [os.path.join(ROOT, "weight_only_quantized_03_b200", "csrc", f)
+                for f in ("gemv_affine8_tc.cu", "gemv_tc.cuh", "qg_internal.cuh")]
+LM_HEAD_SOURCES = GEMV_SOURCES
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 
 
-def traffic_from_profile(kernel_files):
-    """DRAM bytes per launch of the LM-head GEMV from the committed ncu
-    summary, or None when that summary is missing or was taken on a different
-    version of the kernel sources (their sha256 must match)."""
-    path = os.path.join(ROOT, "profiles", "gemv_affine8_lm_head_151936x1024_b1.md")
+def traffic_from_profile(kernel_files, key="gemv_affine8_lm_head_151936x1024_b1",
+                         field="dram_bytes_per_launch"):
+    """DRAM bytes (read + written) of a kernel from one ncu capture, kept in
+    profiles/traffic.json, or None when the entry is missing or was taken on
+    a different version of the kernel sources (their sha256 must match)."""
     try:
-        text = open(path).read()
-    except OSError:
+        with open(TRAFFIC_FILE) as f:
+            d = json.load(f)[key]
+    except (OSError, KeyError, ValueError):
         return None
-    m = re.search(r"traffic_bytes_per_launch:\s*(\d+)", text)
-    h = re.search(r"kernel_source_sha256:\s*([0-9a-f]{64})", text)
-    if not m or not h:
+    if d.get("kernel_source_sha256") != source_sha256(kernel_files):
         return None
-    return int(m.group(1)) if source_sha256(kernel_files) == h.group(1) else None
+    return d.get(field)
+
+
+def step_gemv_traffic(B):
+    """DRAM bytes per step of the step's layer GEMV launches (batch 1 only)."""
+    if B != 1:
+        return None
+    return traffic_from_profile(GEMV_SOURCES, "step_layer_gemvs_qwen3_0.6b_b1_kv512",
+                                "dram_bytes_per_step")
 
 
 class ClockSampler:
@@ -340,21 +494,49 @@ def oracle_sample(cfg, weights, budget_steps=None, layers_only=None):
 
 
 def run_reference(args):
+    """The oracle on the host cores, as it stands. Each of the W + K steps is
+    a bounded sample of the workload: one decoder layer of the 0.6B step at
+    position 511 (a full step is 28 layers and the LM head). The LM head is
+    timed once after the timed samples. ``ms_per_step`` is the measured time
+    of one sample; ``value`` is the full-step rate those times give
+    (1 / (28 x mean layer time + LM head time)), marked as extrapolated."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
+    from oracle import qg_oracle as O
     cfg = dict(qg_synth.QWEN3_0_6B)
     weights = qg_synth.qwen3_weights(cfg, 11)
-    # warm-up: W single layers; timed: K single layers (each a bounded sample)
-    oracle_sample(cfg, weights, layers_only=max(1, args.warmup))
-    v, desc = oracle_sample(cfg, weights, layers_only=max(1, args.steps))
+    Hk, D = cfg["kv_heads"], cfg["head_dim"]
+    cap = KV_LEN + 1
+    kc = O.bf16_bits_to_f64(qg_synth.gaussian_bf16_bits((cfg["layers"], Hk, cap, D), 1.0, 70))
+    vc = O.bf16_bits_to_f64(qg_synth.gaussian_bf16_bits((cfg["layers"], Hk, cap, D), 1.0, 71))
+    tok = int(qg_synth.tokens(1, cfg["vocab"], 72)[0])
+    x = O.embed_rows(*weights["embed"], [tok])[0]
+    for i in range(args.warmup):
+        O.decode_layer(cfg, weights["layers"][i % cfg["layers"]], x, kc[0], vc[0], KV_LEN - 1)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        l = i % cfg["layers"]
+        x = O.decode_layer(cfg, weights["layers"][l], x, kc[l], vc[l], KV_LEN - 1)
+    t_layers = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    O.lm_head(cfg, weights, x)
+    t_head = time.perf_counter() - t0
+    t_layer = t_layers / args.steps
+    v = 1.0 / (cfg["layers"] * t_layer + t_head)
     cores = cpu_cores()
+    desc = (f"each timed step: one decoder layer of the 28 at position {KV_LEN - 1}, batch 1 "
+            f"({args.steps} timed, layers in order); the LM head timed once ({t_head:.3f} s)")
     line = {
         "impl": "reference", "metric": METRIC, "value": v, "unit": "steps/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": 1000.0 / v, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": 1000.0 * t_layer, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": f"Qwen3-0.6B-shaped affine-INT8 g64 decode step, batch 1, KV {KV_LEN}"},
+        "sample": {"timed_step": "one decoder layer (1/28 of the layers of a decode step)",
+                   "ms_per_step_is": "measured time of one sample (one layer)",
+                   "value_is": "extrapolated full-step rate: 1 / (28 x mean layer time + LM head time)",
+                   "full_step_s": 1.0 / v, "lm_head_s": t_head},
         "cpu_baseline": {"value": v, "unit": "steps/s", "cores": cores, "kind": "oracle",
                          "sample": desc},
         "e2e": {"value": v, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -384,6 +566,106 @@ def aggregate_value(world, units_per_rank, max_ms):
 
 
 # ------------------------------------------------------------ GPU arm -------
+
+TIMELINE_NAMES = {1: "embed", 2: "qkv", 3: "attn", 4: "o", 5: "gate_up", 6: "down", 7: "head",
+                  8: "other"}
+GEMV_KINDS = ("qkv", "o", "gate_up", "down")
+
+
+def run_timeline(args):
+    """The timeline leg (run by the main arm as a subprocess on the
+    diagnostic build, QG_LIBRARY=libqg_timeline.so): one step of the bench
+    workload captured into a CUDA graph with per-launch %globaltimer records,
+    replayed 5 times with L2 flushed before each; per launch kind, the median
+    over replays of the summed step share (each launch's exit minus the
+    previous launch's exit, i.e. its part of the critical path). Prints one
+    JSON line."""
+    import ctypes
+    import torch
+    import weight_only_quantized_03_b200 as qg
+    if not qg.lib.qg_timeline_available():
+        print(json.dumps({"unavailable": "library built without QG_TIMELINE"}))
+        return 0
+    cfg = dict(qg_synth.QWEN3_0_6B)
+    B = args.batch
+    model = qg.Qwen3Model(cfg, qg_synth.qwen3_weights(cfg, 11))
+    st = model.new_state(B, KV_LEN + 1)
+    st["k_cache"].normal_()
+    st["v_cache"].normal_()
+    toks = torch.from_numpy(qg_synth.tokens(B, cfg["vocab"], 72)).cuda()
+    pos = torch.full((B,), KV_LEN - 1, dtype=torch.int32, device="cuda")
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            model.qg_decode_step(st, toks, pos, stream=stream)
+    stream.synchronize()
+    nrec = 1024
+    rec = torch.zeros(nrec * 4, dtype=torch.int64, device="cuda")
+    flush = torch.empty(L2_BYTES * 2, dtype=torch.uint8, device="cuda")
+    assert qg.lib.qg_timeline_begin(ctypes.c_void_p(rec.data_ptr()), nrec) == 0
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        model.qg_decode_step(st, toks, pos, stream=stream)
+    kinds = (ctypes.c_int * nrec)()
+    n = qg.lib.qg_timeline_end(kinds, nrec)
+    shares, spans = [], []
+    for rep in range(6):
+        with torch.cuda.stream(stream):
+            flush.fill_(rep & 0xFF)
+            rec.zero_()
+            g.replay()
+        stream.synchronize()
+        if rep == 0:
+            continue
+        r = rec.view(nrec, 4).cpu().numpy().astype(np.uint64)[:n]
+        entry = (~r[:, 0]).astype(np.int64)
+        ex = r[:, 2].astype(np.int64)
+        prev = np.concatenate([[entry[0]], ex[:-1]])
+        d = {}
+        for i in range(n):
+            k = TIMELINE_NAMES.get(kinds[i], "other")
+            d[k] = d.get(k, 0.0) + (ex[i] - prev[i]) / 1e3
+        shares.append(d)
+        spans.append((ex[-1] - entry[0]) / 1e3)
+    del g
+    med = {k: statistics.median(d[k] for d in shares) for k in shares[0]}
+    counts = {}
+    for i in range(n):
+        k = TIMELINE_NAMES.get(kinds[i], "other")
+        counts[k] = counts.get(k, 0) + 1
+    print(json.dumps({"launches": n, "span_us": statistics.median(spans), "share_us": med,
+                      "count": counts}), flush=True)
+    return 0
+
+
+def timeline_leg(batch):
+    """Runs the timeline leg in a subprocess (the diagnostic build is a
+    separate library); None when it is missing or fails."""
+    lib = os.path.join(ROOT, "weight_only_quantized_03_b200", "libqg_timeline.so")
+    if not os.path.exists(lib):
+        return None
+    env = dict(os.environ, QG_LIBRARY="libqg_timeline.so")
+    try:
+        r = subprocess.run([sys.executable, os.path.abspath(__file__), "--timeline-leg",
+                            "--batch", str(batch)], env=env, capture_output=True, text=True,
+                           timeout=600)
+        line = [l for l in r.stdout.splitlines() if l.startswith("{")][-1]
+        d = json.loads(line)
+        return None if "unavailable" in d else d
+    except Exception:
+        return None
+
+
+def gemv_class_bytes(cfg, B):
+    """Algorithmic bytes per step of the layer GEMV launches (q/k/v, o,
+    gate/up, down of every layer): codes, scales, biases, the bf16 inputs
+    and the fp32 outputs (and residual reads of o and down)."""
+    h, F = cfg["hidden"], cfg["ffn"]
+    HD, KD = cfg["heads"] * cfg["head_dim"], cfg["kv_heads"] * cfg["head_dim"]
+    per_layer = (affine8_bytes(HD + 2 * KD, h, B) + affine8_bytes(h, HD, B) + B * h * 4
+                 + affine8_bytes(2 * F, h, B) + affine8_bytes(h, F, B) + B * h * 4)
+    return cfg["layers"] * per_layer
+
 
 def run_ours(args):
     import torch
@@ -418,7 +700,10 @@ def run_ours(args):
     toks = torch.from_numpy(toks_np).cuda()
     pos = torch.from_numpy(pos_np).cuda()
     stream = torch.cuda.Stream()
+    hbm_peak, peak_kind = measured_peaks()
 
+    # the clock sampler runs from the warm-up to the end of the measurements
+    clk = ClockSampler(local).__enter__()
     # ---- capture one step into a CUDA graph
     with torch.cuda.stream(stream):
         for _ in range(3):
@@ -437,23 +722,21 @@ def run_ours(args):
     stream.synchronize()
     barrier()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clk:
-        torch.cuda.synchronize()
-        barrier()
-        with torch.cuda.stream(stream):
-            ev0.record(stream)
-            for _ in range(args.steps):
-                graph.replay()
-            ev1.record(stream)
-        stream.synchronize()
-        torch.cuda.synchronize()
-        barrier()
+    torch.cuda.synchronize()
+    barrier()
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        ev1.record(stream)
+    stream.synchronize()
+    torch.cuda.synchronize()
+    barrier()
     ms = max_over_ranks(ev0.elapsed_time(ev1), world, dist, "cuda")
     ms_per_step = ms / args.steps
     value = aggregate_value(world, args.steps, ms)
 
-    # ---- dominant kernel: the LM-head GEMV (151936 x 1024), timed per launch
-    hbm_peak, peak_kind = measured_peaks()
+    # ---- the tied LM-head GEMV (151936 x 1024) alone, timed per launch
     V, h = cfg["vocab"], cfg["hidden"]
     ew, es, eb = [torch.from_numpy(a.view({2: np.int16, 4: np.int32}[a.dtype.itemsize])).cuda()
                   for a in weights["embed"]]
@@ -465,13 +748,9 @@ def run_ours(args):
     lm_ms = graph_time_ms([lambda: qg.qg_gemv_affine8_g64(ew, es, eb, xb, yl, stream=stream)],
                           stream, nlaunch)
     lm_bytes = affine8_bytes(V, h, B)
-    lm_gbs = lm_bytes / (lm_ms / 1000.0) / 1e9
-    traffic = traffic_from_profile(LM_HEAD_SOURCES) if B == 1 else None
-
-    # ---- the other rows of the path, each timed per launch on its stream
-    kernels = other_kernels(qg, stream, hbm_peak, max(20, min(100, args.steps)))
-    kernels["code_predictor_frame"] = code_predictor_frame(qg, stream, hbm_peak,
-                                                           max(10, min(50, args.steps)))
+    kernels = {"gemv_affine8_lm_head_151936x1024": _hbm_entry(
+        lm_bytes, lm_ms, hbm_peak, batch=B, traffic=traffic_from_profile(LM_HEAD_SOURCES)
+        if B == 1 else None, note="back-to-back launches in a CUDA graph")}
 
     # ---- e2e through the public API with host buffers: token and position
     # in from pinned host memory, then either the greedy token (argmax on the
@@ -513,8 +792,39 @@ def run_ours(args):
     e2e_logits_value = e2e_run(False)
     # the same step both times: the device's greedy token is the host's
     e2e_token_ok = all(int(h_next[b]) == int(torch.argmax(h_logits[b])) for b in range(B))
+    del graph
 
+    # ---- the other configurations, each timed per launch on its stream
+    if not args.quick:
+        kernels.update(c1_c2_gemvs(qg, stream, hbm_peak))
+        kernels.update(c3_batch10(qg, stream, hbm_peak, model, cfg))
+        kernels.update(c4_whisper(qg, stream, hbm_peak))
+        kernels.update(c5_1_7b(qg, stream, hbm_peak))
+        kernels["code_predictor_frame"] = code_predictor_frame(qg, stream, hbm_peak,
+                                                               max(10, min(50, args.steps)))
+    clk.__exit__(None, None, None)
+
+    # ---- the step's dominant kernel class: its layer GEMV launches, from the
+    # in-graph timeline of the same step (diagnostic build, subprocess)
+    tl = timeline_leg(B) if rank == 0 and world == 1 else None
     sb = step_bytes(cfg, B, KV_LEN)
+    gb = gemv_class_bytes(cfg, B)
+    if tl:
+        gemv_us = sum(tl["share_us"].get(k, 0.0) for k in GEMV_KINDS)
+        roof = {"bound": "hbm", "kernel": "gemv_tc_kernel: the step's layer GEMV launches "
+                f"(q/k/v, o, gate/up, down; {sum(tl['count'].get(k, 0) for k in GEMV_KINDS)} "
+                "per step)",
+                "achieved": gb / (gemv_us / 1e6) / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                "frac": gb / (gemv_us / 1e6) / 1e9 / hbm_peak,
+                "traffic": step_gemv_traffic(B), "algorithmic_bytes": gb,
+                "in_graph_us_per_step": gemv_us, "peak_kind": peak_kind,
+                "timing": "in-graph %globaltimer timeline of the bench step (diagnostic build): "
+                          "each launch's exit minus the previous launch's exit, summed",
+                "timeline": tl}
+    else:
+        lm = kernels["gemv_affine8_lm_head_151936x1024"]
+        roof = dict(lm, kernel="gemv_affine8 (LM head 151936x1024)", peak_kind=peak_kind,
+                    note="timeline build unavailable: the LM-head launch alone")
     line = {
         "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
@@ -526,11 +836,7 @@ def run_ours(args):
             "vocab": cfg["vocab"], "parallelism": f"replicas x{world}",
             "l2": f"inputs larger than L2 ({sb / 1e6:.0f} MB per step)", "graph": "CUDA graph + PDL",
         },
-        "roofline": {"bound": "hbm", "kernel": "gemv_affine8 (LM head 151936x1024)",
-                     "achieved": lm_gbs, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": lm_gbs / hbm_peak, "traffic": traffic,
-                     "algorithmic_bytes": lm_bytes, "launch_us": lm_ms * 1000.0,
-                     "peak_kind": peak_kind},
+        "roofline": roof,
         "step_roofline": {"algorithmic_bytes": sb, "achieved": sb / (ms_per_step / 1000.0) / 1e9,
                           "peak": hbm_peak, "unit": "GB/s",
                           "frac": sb / (ms_per_step / 1000.0) / 1e9 / hbm_peak},
@@ -549,7 +855,6 @@ def run_ours(args):
                                 "kind": "oracle", "sample": desc}
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del graph
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -686,7 +991,12 @@ def main():
                     help="launch one kernel only (for an ncu capture); prints no JSON line")
     ap.add_argument("--sweep", action="store_true",
                     help="the Qwen3-1.7B-shaped prefill and batch sweep (its own JSON line)")
+    ap.add_argument("--quick", action="store_true",
+                    help="the decode step, e2e and LM head only (skip the other configurations)")
+    ap.add_argument("--timeline-leg", action="store_true", help=argparse.SUPPRESS)
     args = ap.parse_args()
+    if args.timeline_leg:
+        return run_timeline(args)
     if args.ncu_case:
         return run_ncu_case(args)
     if args.sweep:

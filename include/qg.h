@@ -138,8 +138,30 @@ qg_status qg_gemm_q4_0(const uint8_t* blocks, const float* A, const float* bias,
 /* Reads the device error word of the last qg_gemm_q4_0 call that used `ws`
  * (synchronises `stream`). Every device-side wait in the GEMM is bounded
  * (1 s); one that gives up leaves C undefined, records a nonzero code, and
- * this call then returns QG_ERR_TIMEOUT with the code in *code. */
+ * this call then returns QG_ERR_TIMEOUT with the code in *code. After a
+ * qg_gemm_q4_0_ex call with a bf16 A, pass M = K = 0 (the word then heads
+ * the workspace). */
 qg_status qg_gemm_q4_0_error(int M, int K, const void* ws, unsigned* code, void* stream);
+
+/* The same matmul with the operand and epilogue options the Whisper encoder
+ * layer needs  [FT: encoder_layer -> q_linear, gelu_tanh, residual adds]:
+ *
+ *   v = sum_k bf16(A[m][k]) * bf16(d * (n - 8))[r][k] + bias[r]
+ *       (+ residual[m][r]);   v = gelu_tanh(v) when gelu != 0;
+ *   C[m][r] = v as fp32, or rounded to bf16 (nearest even).
+ *
+ * gelu_tanh(v) = 0.5 v (1 + tanh(sqrt(2/pi) (v + 0.044715 v^3))), in fp32.
+ * A        device [M][K] of a_dtype: QG_BF16 is read as is (no conversion
+ *          pass), QG_F32 is rounded into the workspace first.
+ * bias     device fp32 [N] or NULL.  residual device fp32 [M][N] or NULL
+ *          (only with c_dtype QG_F32; C may alias it).
+ * C        device [M][N] of c_dtype.
+ * ws       >= 256 bytes with a bf16 A (the error word), else
+ *          qg_gemm_q4_0_workspace_size(M, N, K); 256-byte aligned.
+ * A, C and residual 16-byte aligned; shape rules as qg_gemm_q4_0. */
+qg_status qg_gemm_q4_0_ex(const uint8_t* blocks, const void* A, qg_dtype a_dtype,
+                          const float* bias, const float* residual, void* C, qg_dtype c_dtype,
+                          int gelu, int M, int N, int K, void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
  * RMSNorm  [TS: encode_rms_norm_bf16w in `step`; MK: rms_norm layers]
@@ -360,6 +382,15 @@ void qg_step_graphs_clear(void);
  * [B][ffn]. */
 qg_status qg_decode_step_inspect(const qg_qwen3_config* cfg, int B, int cap, size_t offsets[4]);
 
+/* Inspection aid (tests): byte offsets in the workspace of six fp32 arrays
+ * that, after a step, hold the LAST decoder layer's GEMV outputs:
+ * offsets[0] q [B][heads*head_dim], offsets[1] k and offsets[2] v
+ * [B][kv_heads*head_dim] (before the per-head norm and RoPE), offsets[3]
+ * the residual stream after o_proj and its residual add [B][hidden],
+ * offsets[4] gate and offsets[5] up [B][ffn]. */
+qg_status qg_decode_step_inspect_f32(const qg_qwen3_config* cfg, int B, int cap,
+                                     size_t offsets[6]);
+
 /* ------------------------------------------------------------------------
  * Selected-token log-probability  [TS: compute_selected_logprob of the
  * greedy token; not printed on the page, read as the log-softmax]
@@ -446,6 +477,27 @@ qg_status qg_code_predict(const qg_qwen3_config* cfg, const qg_code_predictor_we
                           const float* lm_hidden, const int32_t* code0, int32_t* codes,
                           float* logits, int B, void* ws, size_t ws_bytes, void* stream);
 
+/* Inspection aid (tests): qg_code_predict that also writes a trace of every
+ * group's layers to `trace` (device, 256-byte aligned, at least out[0] bytes
+ * of qg_code_predict_trace_layout). Layout, with out[] from that call:
+ * group g (1 .. groups-1) starts at (g-1) * out[1] and holds the bf16
+ * concatenated input [B][2 hidden] at offset 0, then slots s = 0 ..
+ * cfg->layers at out[2] + s * out[3]. Slot 0 is taken after input_proj,
+ * slot s >= 1 after layer s-1. A slot is a copy of the workspace head: the
+ * residual stream fp32 [B][hidden] at offset 0 and the other step buffers
+ * at the offsets qg_decode_step_inspect and qg_decode_step_inspect_f32
+ * give for (cfg, B, cap = 1), so that slot s >= 1 holds layer s-1's values;
+ * then the K row and the V row that layer wrote (bf16 [B][kv_heads]
+ * [head_dim] each, the second starting where the first is rounded up to 256
+ * bytes). The copies are ordinary stream copies between the launches: the
+ * results are those of qg_code_predict. */
+qg_status qg_code_predict_trace_layout(const qg_qwen3_config* cfg, int B, int groups,
+                                       size_t out[4]);
+qg_status qg_code_predict_traced(const qg_qwen3_config* cfg, const qg_code_predictor_weights* w,
+                                 const float* lm_hidden, const int32_t* code0, int32_t* codes,
+                                 float* logits, int B, void* ws, size_t ws_bytes, void* trace,
+                                 size_t trace_bytes, void* stream);
+
 /* ------------------------------------------------------------------------
  * Greedy token  [TS: turbospark-runtime 0.3.0, src/qwen3_asr_metal.rs, `argmax`]
  *   out[b] = index of the first strict maximum of logits[b][0..V), NaNs
@@ -461,6 +513,165 @@ qg_status qg_code_predict(const qg_qwen3_config* cfg, const qg_code_predictor_we
 size_t qg_argmax_workspace_size(int B, int V);
 qg_status qg_argmax_f32(const float* logits, int B, int V, int32_t* out, void* ws,
                         size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Affine-INT8 group-64 matmul on the tcgen05 tensor cores: the linears of
+ * many activation rows at once (a batched prefill, a batched decode step)
+ * [TS: PackedLinear / load_packed_linear; the prompt rows of
+ * transcribe_with_details]
+ *
+ *   y[t][r] = sum_c (q[r][c] * s[r][c/64] + beta[r][c/64]) * x[t][c]
+ *             (+ residual[t][r])
+ *
+ * w, scales, biases as qg_gemv_affine8_g64 ([N][K]); x device bf16 [T][K]
+ * (16-byte aligned); y device [T][N] of y_dtype (may alias residual);
+ * residual device fp32 [T][N] or NULL (only with a fp32 y).
+ * The weights are dequantized in fp32 and split into two bf16 halves
+ * (hi + lo carries w to about 2^-18 relative); both are multiplied with the
+ * bf16 x, fp32 accumulation in tensor memory.
+ * ws       device, >= 4 bytes, 4-byte aligned: the error word (cleared by
+ *          the call; nonzero after a device-side wait gave up (1 s bound);
+ *          read it with qg_gemm_q4_0_error(0, 0, ws, ...)).
+ * Shape rules: K % 64 == 0, T >= 0, N >= 0.
+ * ---------------------------------------------------------------------- */
+qg_status qg_gemm_affine8_g64(const uint32_t* w, const uint16_t* scales, const uint16_t* biases,
+                              const uint16_t* x, void* y, qg_dtype y_dtype,
+                              const float* residual, int N, int K, int T, void* ws,
+                              size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Batched prefill of one sequence  [TS: transcribe_with_details, the prompt
+ * rows through `step`; MK: Qwen3Model::forward with causal_mask]
+ *
+ * The T prompt rows tokens[0..T) at positions p0 .. p0+T-1 go through every
+ * layer together, in qg_decode_step's op order and precision points, with
+ * the linears on qg_gemm_affine8_g64's tensor-core matmul: embedding rows;
+ * per layer RMSNorm, q/k/v (one launch), per-head q/k RMSNorm + NeoX RoPE
+ * with K and V rows written to the cache at p0 + t, causal attention of
+ * every row over the cached rows [0, p0) and the prompt rows up to itself
+ * (qg_attention_rows' kernel reading the cache), o_proj + residual,
+ * RMSNorm, gate/up (one launch), SiLU-mul, down + residual; then the final
+ * RMSNorm and the tied LM head for the last row.
+ * cfg, w      HOST structs as qg_decode_step (head_dim 64 or 128).
+ * k_cache, v_cache device bf16 [layers][1][kv_heads][cap][head_dim]: rows
+ *             [0, p0) must hold the earlier rows; rows p0 .. p0+T-1 are
+ *             written (not for a token outside [0, vocab), whose row is NaN).
+ * tokens      device int32 [T].  Requires 0 <= p0, p0 + T <= cap.
+ * logits      device fp32 [vocab] (the last row's), or NULL.
+ * ws          >= qg_prefill_workspace_size(cfg, T) bytes, 256-byte aligned.
+ *             qg_prefill_inspect gives the byte offsets of the LAST layer's
+ *             values after a call: [0] the residual stream fp32 [T][hidden]
+ *             (after that layer), [1] input-norm output bf16 [T][hidden],
+ *             [2] q fp32 [T][heads*head_dim], [3] k and [4] v fp32
+ *             [T][kv_heads*head_dim], [5] normed and roped q bf16
+ *             [T][heads*head_dim], [6] attention output bf16, [7] residual
+ *             after o_proj fp32 [T][hidden], [8] post-norm output bf16,
+ *             [9] gate and [10] up fp32 [T][ffn], [11] SiLU-mul output bf16.
+ * ---------------------------------------------------------------------- */
+size_t qg_prefill_workspace_size(const qg_qwen3_config* cfg, int T);
+qg_status qg_prefill(const qg_qwen3_config* cfg, const qg_qwen3_weights* w, uint16_t* k_cache,
+                     uint16_t* v_cache, int cap, const int32_t* tokens, int T, int p0,
+                     float* logits, void* ws, size_t ws_bytes, void* stream);
+qg_status qg_prefill_inspect(const qg_qwen3_config* cfg, int T, size_t offsets[12]);
+
+/* ------------------------------------------------------------------------
+ * LayerNorm  [FT: layer_norm_affine (layer_norm_last_dim, then * g + b)]
+ *   y[r][i] = (x[r][i] - mean_r) / sqrt(var_r + eps) * gamma[i] + beta[i],
+ *   mean and biased variance over the row, in fp32.
+ * x device fp32 [rows][dim]; gamma, beta device fp32 [dim]; y device
+ * [rows][dim] of y_dtype (rounded to nearest even for QG_BF16). All 16-byte
+ * aligned. Shape rules: dim % 4 == 0, 4 <= dim <= 2048.
+ * ---------------------------------------------------------------------- */
+qg_status qg_layernorm(const float* x, const float* gamma, const float* beta, float eps,
+                       void* y, qg_dtype y_dtype, int rows, int dim, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Softmax attention of many query rows  [FT: multi_head_attn; MK:
+ * Qwen3Attention::forward with causal_mask and repeat_kv]
+ *   out[b][t][h] = sum_s softmax_s(q[b][t][h] . k[b][s][kv] / sqrt(D)) v[b][s][kv],
+ *   kv = h / (H / Hkv); s over all S keys, or with `causal` over
+ *   s <= S - T + t (row t at position S - T + t, after S - T earlier keys).
+ * q, out   device bf16 [B][T][H][D];  k, v device bf16 [B][S][Hkv][D].
+ * Tensor cores (bf16 operands, fp32 accumulation); the softmax weights are
+ * rounded to bf16 for the weighted sum of V (and summed as rounded), out is
+ * rounded to bf16. All pointers 16-byte aligned.
+ * Shape rules: D = 64 or 128, H % Hkv == 0, causal needs T <= S; S = 0
+ * gives zero rows.
+ * ---------------------------------------------------------------------- */
+qg_status qg_attention_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                            uint16_t* out, int B, int T, int S, int H, int Hkv, int D,
+                            int causal, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Whisper encoder layer  [FT: encoder_layer, pre-LayerNorm]
+ *   a = LN1(x); q = a Wq^T + bq; k = a Wk^T; v = a Wv^T + bv;
+ *   x1 = x + attention(q, k, v) Wo^T + bo        (every frame to every frame)
+ *   x  = x1 + gelu_tanh(LN2(x1) W1^T + b1) W2^T + b2
+ * The six matrices are Q4_0 blocks (qg_gemm_q4_0 layout) multiplied on the
+ * tensor cores with bf16 operands; the LN outputs, q, k, v, the attention
+ * output and the GELU output are stored as bf16; the residual stream is
+ * fp32. Nine launches: qg_layernorm, three qg_gemm_q4_0_ex (bf16 out),
+ * qg_attention_rows, qg_gemm_q4_0_ex with the residual (into x1),
+ * qg_layernorm, fc1 with GELU (bf16 out), fc2 with the residual (into x).
+ * cfg, w     HOST structs. LN vectors and biases device fp32 (LN vectors
+ *            16-byte aligned); matrices device Q4_0 [out][(in/32)*18].
+ * x          device fp32 [M][d_model], 16-byte aligned: input, then output.
+ * ws         >= qg_whisper_encoder_layer_workspace_size(cfg, M) bytes,
+ *            256-byte aligned; qg_whisper_encoder_layer_inspect gives the
+ *            byte offsets of a (bf16 [M][d]), q, k, v, the attention output
+ *            (bf16), x1 (fp32 [M][d]), LN2's output (bf16), the GELU output
+ *            (bf16 [M][ffn]) and, 9th, the six matmuls' error words (256
+ *            bytes apart; read with qg_gemm_q4_0_error(0, 0, ws + off + 256 i)).
+ * Shape rules: d_model and ffn multiples of 128, d_model <= 2048, head size
+ * d_model / heads of 64 or 128.
+ * ---------------------------------------------------------------------- */
+typedef struct qg_whisper_config {
+  int d_model, heads, ffn;
+  float eps;  /* LayerNorm epsilon (1e-5 on the page) */
+} qg_whisper_config;
+
+typedef struct qg_whisper_layer {
+  const float* ln1_g;
+  const float* ln1_b;
+  const uint8_t* q;
+  const float* q_b;
+  const uint8_t* k;   /* k_proj has no bias */
+  const uint8_t* v;
+  const float* v_b;
+  const uint8_t* o;
+  const float* o_b;
+  const float* ln2_g;
+  const float* ln2_b;
+  const uint8_t* fc1;
+  const float* fc1_b;
+  const uint8_t* fc2;
+  const float* fc2_b;
+} qg_whisper_layer;
+
+size_t qg_whisper_encoder_layer_workspace_size(const qg_whisper_config* cfg, int M);
+qg_status qg_whisper_encoder_layer(const qg_whisper_config* cfg, const qg_whisper_layer* w,
+                                   float* x, int M, void* ws, size_t ws_bytes, void* stream);
+qg_status qg_whisper_encoder_layer_inspect(const qg_whisper_config* cfg, int M,
+                                           size_t offsets[9]);
+
+/* ------------------------------------------------------------------------
+ * Timeline (diagnostics). The pages have no counterpart. In a library built
+ * with QG_TIMELINE (libqg_timeline.so; the default build records nothing
+ * and qg_timeline_available() returns 0), the decode step's kernels launched
+ * between qg_timeline_begin and qg_timeline_end each fill one record of
+ * `records` (device, 16-byte aligned, cap records of 32 bytes, zero-filled
+ * by the caller) when they run, also from a CUDA graph captured meanwhile:
+ * four uint64 per launch -- the bitwise complement of the earliest CTA
+ * entry, the latest return from the wait for the previous kernel, the
+ * latest CTA exit (all %globaltimer nanoseconds, maxima over the launch's
+ * CTAs), and a reserved zero. qg_timeline_end stops recording, copies the
+ * launch kinds (1 embedding, 2 q/k/v GEMV, 3 attention, 4 o_proj, 5 gate/up,
+ * 6 down, 7 output head, 8 other) of the first max_kinds launches to kinds
+ * (host, may be NULL) and returns the number of launches recorded.
+ * ---------------------------------------------------------------------- */
+int qg_timeline_available(void);
+qg_status qg_timeline_begin(void* records, int cap);
+int qg_timeline_end(int* kinds, int max_kinds);
 
 /* ------------------------------------------------------------------------
  * Test exports: the unpack and dequant the kernels use, written out.

@@ -548,7 +548,7 @@ def attention_depths(L, D):
     return D // 8 + 8, L // 32 + 16, L // 4 + 96
 
 
-def attention_bound(qp, dqp, k_cache, v_cache, kv_len, H, Hkv, D):
+def attention_bound(qp, dqp, k_cache, v_cache, kv_len, H, Hkv, D, q_round=0.0, p_round=0.0):
     """(value, bound) of ``decode_attention`` computed in float32 from a
     query ``qp [H*D]`` known within ``dqp`` (per element) and exact bf16
     cache rows.
@@ -563,9 +563,13 @@ def attention_bound(qp, dqp, k_cache, v_cache, kv_len, H, Hkv, D):
     and each computed rescale on its path (4u, plus u |m_old - m_new|,
     which summed along the path is at most the score range). The weighted
     sums add gamma(accumulate) (sum_t p_t |v_t| + |o|) and the final division
-    u |o|."""
+    u |o|. A kernel that rounds the query to bf16 before the scores
+    (``q_round`` = 2^-8, the bf16 unit roundoff) widens ``dqp`` by
+    q_round |q|; one that rounds the weights p_t to bf16 for the weighted
+    sum and its denominator (``p_round`` = 2^-8) reweights each row by at
+    most that much: log(1 + p_round) more on every log-weight."""
     q = np.asarray(qp, dtype=np.float64).reshape(H, D)
-    dq = np.asarray(dqp, dtype=np.float64).reshape(H, D)
+    dq = np.asarray(dqp, dtype=np.float64).reshape(H, D) + q_round * np.abs(q)
     g = H // Hkv
     scale = 1.0 / math.sqrt(D)
     n_dot, n_res, n_acc = attention_depths(kv_len, D)
@@ -581,7 +585,7 @@ def attention_bound(qp, dqp, k_cache, v_cache, kv_len, H, Hkv, D):
         p = p / p.sum()
         o = p @ V_
         rng = m - s.min()
-        e = ds + U32 * (m - s) + EXPF_REL * (n_res + 2) + U32 * rng
+        e = ds + U32 * (m - s) + EXPF_REL * (n_res + 2) + U32 * rng + math.log1p(p_round)
         out[h] = o
         err[h] = (np.exp(2 * e.max()) * (p * e) @ np.abs(V_ - o[None, :])
                   + gamma(n_acc) * (p @ np.abs(V_) + np.abs(o)) + U32 * np.abs(o))
@@ -599,7 +603,8 @@ LAYER_FP32_POINTS = ("q_proj", "k_proj", "v_proj", "x_attn", "gate", "up")
 LAYER_BF16_POINTS = ("xn", "k", "v", "att", "xn2", "h")
 
 
-def decode_layer_forced(cfg, lw, x, k_cache_l, v_cache_l, pos, forced, details=None):
+def decode_layer_forced(cfg, lw, x, k_cache_l, v_cache_l, pos, forced, details=None,
+                        q_round=0.0, p_round=0.0):
     """``decode_layer`` checked op by op against another implementation's
     values of one layer (teacher-forced).
 
@@ -623,6 +628,9 @@ def decode_layer_forced(cfg, lw, x, k_cache_l, v_cache_l, pos, forced, details=N
         k_proj (norm and RoPE), v from v_proj (exact), att from q_proj and
         the cache (norm, RoPE, attention), xn2 from x_attn, h from gate and
         up.
+    ``q_round`` and ``p_round`` pass to ``attention_bound`` for a kernel
+    that rounds the query or the softmax weights to bf16 (the multi-row
+    attention of a batched prefill does both).
     Returns ``(refs, bad)``: ``bad`` maps each rounding point to the indices
     whose forced value is not a correct rounding (with ``details``, a dict,
     filled per point with their values, the forced values and the bounds).
@@ -655,7 +663,7 @@ def decode_layer_forced(cfg, lw, x, k_cache_l, v_cache_l, pos, forced, details=N
     k_cache_l[:, pos, :] = f["k"].reshape(Hkv, D)
     v_cache_l[:, pos, :] = f["v"].reshape(Hkv, D)
     qr, qb = norm_rope_bound(f["q_proj"], lw["q_norm"], eps, pos, theta, D)
-    att, ab = attention_bound(qr, qb, k_cache_l, v_cache_l, pos + 1, H, Hkv, D)
+    att, ab = attention_bound(qr, qb, k_cache_l, v_cache_l, pos + 1, H, Hkv, D, q_round, p_round)
     check("att", att, ab)
     refs["x_attn"] = x + gemv_affine8(*lw["o"], f["att"][None])[0]
     v2 = rmsnorm(f["x_attn"], lw["post_norm"], eps)
@@ -739,13 +747,15 @@ def gelu_tanh(x):
     return 0.5 * x * (1.0 + np.tanh(math.sqrt(2.0 / math.pi) * (x + 0.044715 * x ** 3)))
 
 
-def mha_rows(q, k, v, n_heads, causal=False, kv_heads=None):
+def mha_rows(q, k, v, n_heads, causal=False, kv_heads=None, abs_weighted=False):
     """Multi-head softmax attention of [FT] ``multi_head_attn`` for all rows
     at once: q ``[T, H*D]``, k and v ``[S, Hkv*D]``, per head
     ``softmax(q_h k_h^T / sqrt(D)) v_h`` over all S rows, or with
     ``causal`` over rows ``j <= i`` (the mask of [FT] and of [MK]
     ``causal_mask``). With ``kv_heads`` < heads, query head h reads KV head
-    ``h // (H / Hkv)`` ([MK] ``repeat_kv``). float64; returns ``[T, H*D]``."""
+    ``h // (H / Hkv)`` ([MK] ``repeat_kv``). float64; returns ``[T, H*D]``,
+    and with ``abs_weighted`` also ``sum_s p_s |v_s|`` per output (what a
+    relative change of each weight moves the output by, at most)."""
     q = np.asarray(q, np.float64)
     k = np.asarray(k, np.float64)
     v = np.asarray(v, np.float64)
@@ -755,6 +765,7 @@ def mha_rows(q, k, v, n_heads, causal=False, kv_heads=None):
     D = q.shape[1] // n_heads
     g = n_heads // Hkv
     out = np.zeros((T, n_heads * D))
+    aw = np.zeros((T, n_heads * D))
     for h in range(n_heads):
         kh = h // g
         s = q[:, h * D:(h + 1) * D] @ k[:, kh * D:(kh + 1) * D].T / math.sqrt(D)
@@ -763,7 +774,9 @@ def mha_rows(q, k, v, n_heads, causal=False, kv_heads=None):
         p = np.exp(s - s.max(axis=1, keepdims=True))
         p = p / p.sum(axis=1, keepdims=True)
         out[:, h * D:(h + 1) * D] = p @ v[:, kh * D:(kh + 1) * D]
-    return out
+        if abs_weighted:
+            aw[:, h * D:(h + 1) * D] = p @ np.abs(v[:, kh * D:(kh + 1) * D])
+    return (out, aw) if abs_weighted else out
 
 
 def whisper_encoder_layer(x, lw, n_heads, eps=1e-5, details=None):

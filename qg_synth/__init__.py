@@ -193,3 +193,22 @@ def code_predictor_weights(cfg: dict, groups: int, seed: int, norm_jitter: float
             "heads": [affine8_packed(V, h, sd + 101 + g) for g in range(groups)],
             "layers": base["layers"], "final_norm": base["final_norm"]}
 
+
+# Whisper-large-v3 encoder layer shape (d_model 1280, 20 heads of 64, FFN
+# 5120, LayerNorm eps 1e-5; fuel-transformers lazy_quantized_whisper.rs).
+WHISPER_LARGE_V3 = dict(d_model=1280, heads=20, ffn=5120, eps=1e-5)
+
+
+def whisper_layer_weights(cfg: dict, seed: int) -> dict:
+    """Random-init weights of one Whisper encoder layer: the six projections
+    as Q4_0 blocks (``q4_0_packed``; k_proj has no bias) and float32
+    LayerNorm vectors (gamma near 1, beta near 0) and biases N(0, 0.1^2)."""
+    d, F = cfg["d_model"], cfg["ffn"]
+    shapes = {"q": (d, d), "k": (d, d), "v": (d, d), "o": (d, d), "fc1": (F, d), "fc2": (d, F)}
+    w = {n: q4_0_packed(N, K, seed + i) for i, (n, (N, K)) in enumerate(shapes.items())}
+    vecs = {"ln1_g": d, "ln1_b": d, "q_b": d, "v_b": d, "o_b": d, "ln2_g": d, "ln2_b": d,
+            "fc1_b": F, "fc2_b": d}
+    for i, (n, size) in enumerate(vecs.items()):
+        v = gaussian((size,), 0.1, seed + 100 + i)
+        w[n] = (v + 1.0).astype(np.float32) if n.endswith("_g") else v
+    return w

@@ -6,8 +6,9 @@ For outputs stored as bf16 the bf16 store adds at most half a bf16 ulp of the
 value, bounded here by 2^-8 |ref| (``bf16_out=True``). When both sides store
 bf16 (the oracle rounds too, e.g. K/V cache rows), values a hair apart can
 round to neighbouring bf16 numbers: one full ulp, 2^-7 |ref| (``ulps=1``).
-Downstream of such a rounding inside a decoder layer, the oracle's
-``decode_layer_tie_bound`` gives the added bound (``extra``).
+Downstream of a bf16 rounding tie (a value within float32 error of a
+rounding midpoint), an output may move by the tie's exact linear effect,
+which the oracle computes (``lm_head_tie_bound``); it is passed as ``extra``.
 """
 import numpy as np
 import torch
@@ -37,7 +38,7 @@ def host64(t):
 
 def assert_parity(gpu, ref, bf16_out=False, what="", ulps=0.5, extra=None):
     """``extra``: an added per-element bound, for outputs downstream of bf16
-    roundings that sit on a tie (the oracle's ``decode_layer_tie_bound``)."""
+    roundings that sit on a tie (the oracle's ``lm_head_tie_bound``)."""
     gpu = np.asarray(gpu, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     assert gpu.shape == ref.shape, (what, gpu.shape, ref.shape)

@@ -142,3 +142,91 @@ def test_code_predictor_layers_teacher_forced():
         logits = _step_checked(model, st, cfg, w, caches, toks, p)
         toks = [int(np.argmax(logits[b])) for b in range(2)]
 
+
+
+def _slot(trace, B, cfg, offs, base, kv_bytes):
+    """The values of one trace slot as float64 numpy arrays: the residual
+    ``x``, the layer's values under the oracle's point names, and the K/V
+    rows it wrote."""
+    (o_xn, o_att, o_xn2, o_h), (o_q, o_k, o_v, o_xa, o_g, o_u) = offs
+    HD, KD = cfg["heads"] * cfg["head_dim"], cfg["kv_heads"] * cfg["head_dim"]
+    hid, F = cfg["hidden"], cfg["ffn"]
+
+    def get(o, n, dt):
+        size = 2 if dt == torch.bfloat16 else 4
+        t = trace[base + o: base + o + size * B * n].view(dt).view(B, n)
+        return host64(t)
+    bf, f32 = torch.bfloat16, torch.float32
+    v = {"x": get(0, hid, f32), "xn": get(o_xn, hid, bf), "att": get(o_att, HD, bf),
+         "xn2": get(o_xn2, hid, bf), "h": get(o_h, F, bf), "q_proj": get(o_q, HD, f32),
+         "k_proj": get(o_k, KD, f32), "v_proj": get(o_v, KD, f32), "x_attn": get(o_xa, hid, f32),
+         "gate": get(o_g, F, f32), "up": get(o_u, F, f32)}
+    snap = kv_bytes[0]
+    v["k"] = get(snap, KD, bf)
+    v["v"] = get(snap + kv_bytes[1], KD, bf)
+    return v
+
+
+@pytest.mark.parametrize("B,G", [(1, 16), (2, 3)])
+def test_code_predict_layers_checked_op_by_op_per_group(B, G):
+    """qg_code_predict's own layer chain at the makima code predictor shape
+    (hidden 1024, 5 layers, MHA 16/16, head_dim 64, FFN 3072, 2048 codes),
+    traced group by group (qg_code_predict_traced): every group's bf16
+    input is the concatenation of the LM hidden state and the previous
+    code's embedding (bit-exact), input_proj meets the fp32 bound, every
+    layer is checked op by op against the oracle (each fp32 GEMV output
+    from the GPU's inputs, each bf16 rounding point a correct rounding
+    within its derived float32 bound, with a fresh one-row cache at
+    position 0), the head's logits meet the bound from the GPU's final
+    residual (plus the exact effect of final-norm ties), and each code is
+    the first maximum of the GPU's own logits. The traced results equal
+    the untraced call's bit for bit."""
+    from tests.test_gpu_decode_step import _forced_layer
+    cfg = dict(qg_synth.CODE_PREDICTOR)
+    w = qg_synth.code_predictor_weights(cfg, G, 47, norm_jitter=0.1)
+    model = qg.CodePredictor(cfg, w)
+    lm_hidden = qg_synth.gaussian((B, cfg["hidden"]), 1.0, 48).astype(np.float32)
+    code0 = qg_synth.tokens(B, cfg["vocab"], 49).astype(np.int32)
+    total, per_group, slot0, per_slot = model.trace_layout(B)
+    trace = torch.zeros(total, dtype=torch.uint8, device="cuda")
+    codes = torch.empty((G, B), dtype=torch.int32, device="cuda")
+    logits = torch.zeros((G, B, cfg["vocab"]), dtype=torch.float32, device="cuda")
+    ws = model.workspace(B)
+    model.qg_code_predict_traced(dev(lm_hidden), dev(code0), codes, ws, trace, logits=logits)
+    codes2 = torch.empty_like(codes)
+    logits2 = torch.zeros_like(logits)
+    model.qg_code_predict(dev(lm_hidden), dev(code0), codes2, ws, logits=logits2)
+    torch.cuda.synchronize()
+    assert torch.equal(codes, codes2) and torch.equal(logits[1:], logits2[1:])
+    got_codes = codes.cpu().numpy()
+    lg = host64(logits)
+    offs = model.step_offsets(B)
+    Hkv, D = cfg["kv_heads"], cfg["head_dim"]
+    kv_row = B * Hkv * D * 2
+    kv_bytes = ((per_slot - 2 * ((kv_row + 255) // 256 * 256)), (kv_row + 255) // 256 * 256)
+    np.testing.assert_array_equal(got_codes[0], code0)
+    for g in range(1, G):
+        gb = (g - 1) * per_group
+        comb = host64(trace[gb: gb + B * 2 * cfg["hidden"] * 2].view(torch.bfloat16)
+                      .view(B, 2 * cfg["hidden"]))
+        slots = [_slot(trace, B, cfg, offs, gb + slot0 + s * per_slot, kv_bytes)
+                 for s in range(cfg["layers"] + 1)]
+        for b in range(B):
+            what = f"b={b} group {g}"
+            emb = O.embed_rows(*w["code_embed"][g - 1], [int(got_codes[g - 1][b])])[0]
+            ref_comb = O.round_bf16(np.concatenate([lm_hidden[b].astype(np.float64), emb]))
+            np.testing.assert_array_equal(comb[b], ref_comb, err_msg=f"{what} input")
+            x0 = O.gemv_affine8(*w["input_proj"], comb[b][None])[0]
+            assert_parity(slots[0]["x"][b], x0, what=f"{what} input_proj")
+            for l in range(cfg["layers"]):
+                s_in, s_out = slots[l], slots[l + 1]
+                inter = {k: s_out[k][b] for k in ("xn", "xn2", "h", "q_proj", "k_proj", "v_proj",
+                                                 "x_attn", "gate", "up")}
+                inter["attn"] = s_out["att"][b]
+                kc, vc = np.zeros((Hkv, 1, D)), np.zeros((Hkv, 1, D))
+                _forced_layer(cfg, w["layers"][l], s_in["x"][b], kc, vc, 0, inter,
+                              s_out["k"][b], s_out["v"][b], s_out["x"][b], f"{what} layer {l}")
+            head = {"embed": w["heads"][g], "final_norm": w["final_norm"]}
+            ref, tie = O.lm_head_tie_bound(cfg, head, slots[-1]["x"][b])
+            assert_parity(lg[g][b], ref, extra=tie, what=f"{what} head")
+            assert int(got_codes[g][b]) == O.argmax_first(lg[g][b]), what

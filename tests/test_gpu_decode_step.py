@@ -51,17 +51,23 @@ def _greedy_ok(gpu_logits, ref_logits):
     return abs(top[1] - top[0]) <= 2 * (ATOL + RTOL * abs(top[1]))
 
 
-def _forced_layer(cfg, lw, x, kc_l, vc_l, p, inter_b, k_row, v_row, what):
-    """The oracle layer teacher-forced with the GPU's bf16 values at its
-    rounding points (each checked to be a correct rounding of the oracle's
-    own value there: exact, or the other side of a near-tie)."""
+def _forced_layer(cfg, lw, x, kc_l, vc_l, p, inter_b, k_row, v_row, x_out, what):
+    """One layer of the oracle checked op by op against the GPU's values of
+    that layer (``decode_layer_forced``): each fp32 GEMV output of the GPU
+    (q/k/v, the residual after o_proj, gate, up, and ``x_out``, the residual
+    after the layer) against the oracle's from the GPU's own inputs, under
+    the fp32-accumulation bound; each bf16 value at a rounding point as a
+    correct rounding of the oracle's value of its op chain within that
+    chain's derived float32 error bound."""
     forced = dict(inter_b, k=k_row.ravel(), v=v_row.ravel())
     forced["att"] = forced.pop("attn")  # the oracle's name for the attention output
     det = {}
-    ref, bad = O.decode_layer_forced(cfg, lw, x, kc_l, vc_l, p, forced, details=det)
+    refs, bad = O.decode_layer_forced(cfg, lw, x, kc_l, vc_l, p, forced, details=det)
     for name, idx in bad.items():
         assert idx.size == 0, f"{what}: {name} is not a correct bf16 rounding: {det.get(name)}"
-    return ref
+    for name in O.LAYER_FP32_POINTS:
+        assert_parity(forced[name], refs[name], what=f"{what} {name}")
+    assert_parity(x_out, refs["y"], what=f"{what} residual")
 
 
 def _intermediates(model, st):
@@ -92,12 +98,11 @@ def _step_checked(model, st, cfg, w, caches, toks, p):
         kc, vc = caches[b]
         for l in range(cfg["layers"]):
             what = f"b={b} p={p} layer {l}"
-            ref = _forced_layer(cfg, w["layers"][l], xs[l][b], kc[l], vc[l], p,
-                                {k: a[b] for k, a in inter[l].items()},
-                                kg[l, b, :, p, :], vg[l, b, :, p, :], what)
+            _forced_layer(cfg, w["layers"][l], xs[l][b], kc[l], vc[l], p,
+                          {k: a[b] for k, a in inter[l].items()},
+                          kg[l, b, :, p, :], vg[l, b, :, p, :], xs[l + 1][b], what)
             kc[l, :, p, :] = kg[l, b, :, p, :]
             vc[l, :, p, :] = vg[l, b, :, p, :]
-            assert_parity(xs[l + 1][b], ref, what=what)
         ref, tie = O.lm_head_tie_bound(cfg, w, xs[-1][b])
         assert_parity(logits[b], ref, extra=tie, what=f"b={b} p={p} LM head")
     return logits
@@ -178,10 +183,9 @@ def test_qwen3_0_6b_step_layer_by_layer_at_position_511(B):
         vc = O.bf16_bits_to_f64(vbits[:, b])
         for l in range(Lr):
             what = f"b={b} layer {l}"
-            ref = _forced_layer(cfg, w["layers"][l], xs[l][b], kc[l], vc[l], p,
-                                {k: a[b] for k, a in inter[l].items()},
-                                kg[l, b, :, p, :], vg[l, b, :, p, :], what)
-            assert_parity(xs[l + 1][b], ref, what=f"{what} residual")
+            _forced_layer(cfg, w["layers"][l], xs[l][b], kc[l], vc[l], p,
+                          {k: a[b] for k, a in inter[l].items()},
+                          kg[l, b, :, p, :], vg[l, b, :, p, :], xs[l + 1][b], what)
             np.testing.assert_array_equal(kg[l, b, :, p + 1, :], kc[l, :, p + 1, :])
         ref, tie = O.lm_head_tie_bound(cfg, w, xs[Lr][b])
         assert_parity(logits[b], ref, extra=tie, what=f"b={b} LM head")
@@ -220,10 +224,9 @@ def test_qwen3_1_7b_shaped_layers_at_position_2047(B, layers):
         vc = O.bf16_bits_to_f64(vbits[:, b])
         for l in range(Lr):
             what = f"b={b} p={p} layer {l}"
-            ref = _forced_layer(cfg, w["layers"][l], xs[l][b], kc[l], vc[l], p,
-                                {k: a[b] for k, a in inter[l].items()},
-                                kg[l, b, :, p, :], vg[l, b, :, p, :], what)
-            assert_parity(xs[l + 1][b], ref, what=f"{what} residual")
+            _forced_layer(cfg, w["layers"][l], xs[l][b], kc[l], vc[l], p,
+                          {k: a[b] for k, a in inter[l].items()},
+                          kg[l, b, :, p, :], vg[l, b, :, p, :], xs[l + 1][b], what)
         if b < 2:  # the LM head oracle (151936 x 2048 in f64) for two rows
             ref, tie = O.lm_head_tie_bound(cfg, w, xs[Lr][b])
             assert_parity(logits[b], ref, extra=tie, what=f"b={b} LM head")

@@ -376,8 +376,12 @@ def _f32_norm_rope(x, w_bits, eps, pos, theta, D):
     return out.ravel()
 
 
-def _f32_attention(q, kc, vc, L, H, Hkv, D, batch=24):
-    """Online softmax over batches of rows, float32, like the kernels."""
+def _f32_attention(q, kc, vc, L, H, Hkv, D, batch=24, round_q=False, round_p=False):
+    """Online softmax over batches of rows, float32, like the kernels; with
+    round_q / round_p the query / the weights are rounded to bf16 first (the
+    multi-row kernel's tensor-core operands)."""
+    if round_q:
+        q = O.round_bf16(np.asarray(q, F32))
     q = np.asarray(q, F32).reshape(H, D) * F32(F32(1) / F32(np.sqrt(F32(D))))
     out = np.zeros((H, D), F32)
     g = H // Hkv
@@ -391,6 +395,8 @@ def _f32_attention(q, kc, vc, L, H, Hkv, D, batch=24):
             l, o = F32(l * a), (o * a).astype(F32)
             for t in range(sc.size):
                 p = F32(np.exp(F32(sc[t] - mx)))
+                if round_p:
+                    p = F32(O.round_bf16(p))
                 l = F32(l + p)
                 o = (o + p * V_[t0 + t]).astype(F32)
             m = mx
@@ -455,6 +461,10 @@ def test_float32_op_chains_stay_within_their_derived_bounds():
     np.testing.assert_allclose(att, O.decode_attention(qp, kc, vc, 10, H, Hkv, D), atol=1e-12)
     assert np.all(np.abs(_f32_attention(qp, kc, vc, 10, H, Hkv, D) - att) <= ab)
     assert np.max(ab) < 2.0 ** -14 * np.max(np.abs(vc))
+    # bf16 query and weights (the multi-row kernel): within the widened bound
+    _, abr = O.attention_bound(qp, np.zeros(H * D), kc, vc, 10, H, Hkv, D, 2.0 ** -8, 2.0 ** -8)
+    f32r = _f32_attention(qp, kc, vc, 10, H, Hkv, D, round_q=True, round_p=True)
+    assert np.all(np.abs(f32r - att) <= abr) and np.any(np.abs(f32r - att) > ab)
     # a query known only within dq widens the bound by about the score error
     _, ab2 = O.attention_bound(qp, np.full(H * D, 1e-3), kc, vc, 10, H, Hkv, D)
     assert np.all(ab2 > ab)

@@ -14,7 +14,11 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libqg.so")
+# QG_LIBRARY may name the diagnostic build next to it (libqg_timeline.so)
+_NAME = os.environ.get("QG_LIBRARY", "libqg.so")
+if _NAME not in ("libqg.so", "libqg_timeline.so"):
+    raise ImportError(f"QG_LIBRARY={_NAME!r}: expected libqg.so or libqg_timeline.so")
+LIB_PATH = os.path.join(_HERE, _NAME)
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
@@ -64,6 +68,17 @@ class qg_qwen3_weights(ctypes.Structure):
                 ("layers", ctypes.POINTER(qg_qwen3_layer))]
 
 
+class qg_whisper_config(ctypes.Structure):
+    _fields_ = [("d_model", ctypes.c_int), ("heads", ctypes.c_int), ("ffn", ctypes.c_int),
+                ("eps", ctypes.c_float)]
+
+
+class qg_whisper_layer(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("ln1_g", "ln1_b", "q", "q_b", "k", "v", "v_b", "o", "o_b", "ln2_g", "ln2_b",
+                 "fc1", "fc1_b", "fc2", "fc2_b")]
+
+
 class qg_code_predictor_weights(ctypes.Structure):
     _fields_ = [("input_proj", qg_affine8_matrix),
                 ("code_embed", ctypes.POINTER(qg_affine8_matrix)),
@@ -97,7 +112,31 @@ _SIGS = {
                             _vp, _vp, _i, _vp, _vp, _vp, _i, _vp, _sz, _vp]),
     "qg_decode_step_inspect": (_i, [ctypes.POINTER(qg_qwen3_config), _i, _i,
                                     ctypes.POINTER(ctypes.c_size_t)]),
+    "qg_decode_step_inspect_f32": (_i, [ctypes.POINTER(qg_qwen3_config), _i, _i,
+                                        ctypes.POINTER(ctypes.c_size_t)]),
     "qg_code_predict_workspace_size": (_sz, [ctypes.POINTER(qg_qwen3_config), _i]),
+    "qg_gemm_q4_0_ex": (_i, [_vp, _vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "qg_gemm_affine8_g64": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _vp, _sz, _vp]),
+    "qg_prefill_workspace_size": (_sz, [ctypes.POINTER(qg_qwen3_config), _i]),
+    "qg_prefill": (_i, [ctypes.POINTER(qg_qwen3_config), ctypes.POINTER(qg_qwen3_weights), _vp,
+                        _vp, _i, _vp, _i, _i, _vp, _vp, _sz, _vp]),
+    "qg_prefill_inspect": (_i, [ctypes.POINTER(qg_qwen3_config), _i,
+                                ctypes.POINTER(ctypes.c_size_t)]),
+    "qg_layernorm": (_i, [_vp, _vp, _vp, _f, _vp, _i, _i, _i, _vp]),
+    "qg_attention_rows": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]),
+    "qg_whisper_encoder_layer_workspace_size": (_sz, [ctypes.POINTER(qg_whisper_config), _i]),
+    "qg_whisper_encoder_layer": (_i, [ctypes.POINTER(qg_whisper_config),
+                                      ctypes.POINTER(qg_whisper_layer), _vp, _i, _vp, _sz, _vp]),
+    "qg_whisper_encoder_layer_inspect": (_i, [ctypes.POINTER(qg_whisper_config), _i,
+                                              ctypes.POINTER(ctypes.c_size_t)]),
+    "qg_timeline_available": (_i, []),
+    "qg_timeline_begin": (_i, [_vp, _i]),
+    "qg_timeline_end": (_i, [ctypes.POINTER(ctypes.c_int), _i]),
+    "qg_code_predict_trace_layout": (_i, [ctypes.POINTER(qg_qwen3_config), _i, _i,
+                                          ctypes.POINTER(ctypes.c_size_t)]),
+    "qg_code_predict_traced": (_i, [ctypes.POINTER(qg_qwen3_config),
+                                    ctypes.POINTER(qg_code_predictor_weights), _vp, _vp, _vp,
+                                    _vp, _i, _vp, _sz, _vp, _sz, _vp]),
     "qg_code_predict": (_i, [ctypes.POINTER(qg_qwen3_config),
                              ctypes.POINTER(qg_code_predictor_weights), _vp, _vp, _vp, _vp, _i,
                              _vp, _sz, _vp]),
@@ -177,6 +216,44 @@ def qg_gemm_q4_0(blocks, A, C, bias=None, ws=None, stream=None):
     nbytes = 0 if ws is None else ws.numel() * ws.element_size()
     _call("qg_gemm_q4_0", _p(blocks), _p(A), _p(bias), _p(C), M, N, K, _p(ws), nbytes,
           _stream(stream))
+
+
+def qg_gemm_q4_0_ex(blocks, A, C, bias=None, residual=None, gelu=False, ws=None, stream=None):
+    """C = epilogue(bf16(A) @ bf16(W)^T + bias (+ residual)), A fp32 or bf16
+    [M, K], C fp32 or bf16 [M, N]; gelu applies gelu_tanh."""
+    N = blocks.shape[0]
+    K = blocks.shape[1] // 18 * 32
+    M = A.shape[0]
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _call("qg_gemm_q4_0_ex", _p(blocks), _p(A), _dt(A), _p(bias), _p(residual), _p(C), _dt(C),
+          1 if gelu else 0, M, N, K, _p(ws), nbytes, _stream(stream))
+
+
+def qg_gemm_affine8_g64(w, scales, biases, x, y, residual=None, ws=None, stream=None):
+    """y[T, N] = x[T, K] (bf16) @ dequant(w)[N, K]^T (+ residual) on the
+    tensor cores; ws holds the 4-byte error word."""
+    N, K = w.shape[0], w.shape[1] * 4
+    T = x.shape[0]
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _call("qg_gemm_affine8_g64", _p(w), _p(scales), _p(biases), _p(x), _p(y), _dt(y),
+          _p(residual), N, K, T, _p(ws), nbytes, _stream(stream))
+
+
+def qg_layernorm(x, gamma, beta, eps, y, stream=None):
+    _call("qg_layernorm", _p(x), _p(gamma), _p(beta), eps, _p(y), _dt(y), x.shape[0],
+          x.shape[1], _stream(stream))
+
+
+def qg_attention_rows(q, k, v, out, H, Hkv, causal=False, stream=None):
+    """q, out bf16 [B, T, H*D]; k, v bf16 [B, S, Hkv*D] (a leading batch
+    dimension may be omitted)."""
+    if q.dim() == 2:
+        q, k, v, out = q[None], k[None], v[None], out[None]
+    B, T = q.shape[0], q.shape[1]
+    S = k.shape[1]
+    D = q.shape[2] // H
+    _call("qg_attention_rows", _p(q), _p(k), _p(v), _p(out), B, T, S, H, Hkv, D,
+          1 if causal else 0, _stream(stream))
 
 
 def qg_gemm_q4_0_error(M, K, ws, stream=None):
@@ -351,18 +428,63 @@ class Qwen3Model:
         return state["ws"][: 4 * n].view(torch.float32).view(state["B"], self.cfg["hidden"])
 
     def intermediates(self, state):
-        """The last decoder layer's bf16 values at its rounding points after
-        a kernel-per-op step (``qg_decode_step_inspect``): dict of torch
-        bf16 views ``xn`` [B, hidden], ``attn`` [B, heads*head_dim], ``xn2``
-        [B, hidden], ``h`` [B, ffn] into the workspace."""
-        off = (ctypes.c_size_t * 4)()
-        _call("qg_decode_step_inspect", ctypes.byref(self.c_cfg), state["B"], state["cap"], off)
+        """The last decoder layer's values after a step
+        (``qg_decode_step_inspect`` and ``_inspect_f32``): dict of torch views
+        into the workspace -- bf16 ``xn`` [B, hidden], ``attn``
+        [B, heads*head_dim], ``xn2`` [B, hidden], ``h`` [B, ffn]; fp32
+        ``q_proj`` [B, heads*head_dim], ``k_proj``, ``v_proj``
+        [B, kv_heads*head_dim], ``x_attn`` [B, hidden], ``gate``, ``up``
+        [B, ffn]."""
         c, B = self.cfg, state["B"]
         ws = state["ws"]
-        def view(o, n):
-            return ws[o:o + 2 * B * n].view(torch.bfloat16).view(B, n)
-        return {"xn": view(off[0], c["hidden"]), "attn": view(off[1], c["heads"] * c["head_dim"]),
-                "xn2": view(off[2], c["hidden"]), "h": view(off[3], c["ffn"])}
+        off = (ctypes.c_size_t * 4)()
+        _call("qg_decode_step_inspect", ctypes.byref(self.c_cfg), B, state["cap"], off)
+        off32 = (ctypes.c_size_t * 6)()
+        _call("qg_decode_step_inspect_f32", ctypes.byref(self.c_cfg), B, state["cap"], off32)
+
+        def view(o, n, dt=torch.bfloat16):
+            size = 2 if dt == torch.bfloat16 else 4
+            return ws[o:o + size * B * n].view(dt).view(B, n)
+        HD, KD, h, F = c["heads"] * c["head_dim"], c["kv_heads"] * c["head_dim"], c["hidden"], c["ffn"]
+        f32 = torch.float32
+        return {"xn": view(off[0], h), "attn": view(off[1], HD), "xn2": view(off[2], h),
+                "h": view(off[3], F), "q_proj": view(off32[0], HD, f32),
+                "k_proj": view(off32[1], KD, f32), "v_proj": view(off32[2], KD, f32),
+                "x_attn": view(off32[3], h, f32), "gate": view(off32[4], F, f32),
+                "up": view(off32[5], F, f32)}
+
+    def prefill_workspace(self, T):
+        n = int(lib.qg_prefill_workspace_size(ctypes.byref(self.c_cfg), T))
+        return torch.empty(n, dtype=torch.uint8, device=self.device)
+
+    def qg_prefill(self, state, tokens, p0, ws, logits=None, stream=None, layers=None):
+        """The prompt rows ``tokens`` (device int32 [T]) of sequence 0 of
+        ``state`` at positions p0 .. p0+T-1; the last row's logits into
+        ``logits`` ([vocab]) when given. ``layers`` runs only the first that
+        many layers."""
+        cfg = self.c_cfg
+        if layers is not None:
+            cfg = qg_qwen3_config.from_buffer_copy(self.c_cfg)
+            cfg.layers = layers
+        _call("qg_prefill", ctypes.byref(cfg), ctypes.byref(self.c_weights),
+              _p(state["k_cache"]), _p(state["v_cache"]), state["cap"], _p(tokens),
+              tokens.shape[0], p0, _p(logits), _p(ws), ws.numel(), _stream(stream))
+
+    def prefill_intermediates(self, ws, T):
+        """The last layer's values after qg_prefill (qg_prefill_inspect)."""
+        off = (ctypes.c_size_t * 12)()
+        _call("qg_prefill_inspect", ctypes.byref(self.c_cfg), T, off)
+        c = self.cfg
+        HD, KD, h, F = c["heads"] * c["head_dim"], c["kv_heads"] * c["head_dim"], c["hidden"], c["ffn"]
+        bf, f32 = torch.bfloat16, torch.float32
+        spec = [("x", h, f32), ("xn", h, bf), ("q_proj", HD, f32), ("k_proj", KD, f32),
+                ("v_proj", KD, f32), ("q_rope", HD, bf), ("att", HD, bf), ("x_attn", h, f32),
+                ("xn2", h, bf), ("gate", F, f32), ("up", F, f32), ("h", F, bf)]
+        out = {}
+        for i, (name, n, dt) in enumerate(spec):
+            size = 2 if dt == bf else 4
+            out[name] = ws[off[i]:off[i] + size * T * n].view(dt).view(T, n)
+        return out
 
     def qg_decode_step(self, state, tokens, positions, stream=None, layers=None):
         """tokens, positions: device int32 [B]. Writes state['logits'].
@@ -429,3 +551,76 @@ class CodePredictor:
               _p(lm_hidden), _p(code0), _p(codes), _p(logits), B, _p(ws),
               ws.numel(), _stream(stream))
 
+    def trace_layout(self, B):
+        """(total bytes, bytes per group, offset of slot 0 in a group, bytes
+        per slot) of the trace of ``qg_code_predict_traced``."""
+        out = (ctypes.c_size_t * 4)()
+        _call("qg_code_predict_trace_layout", ctypes.byref(self.c_cfg), B, self.groups, out)
+        return tuple(int(v) for v in out)
+
+    def step_offsets(self, B):
+        """Offsets of the step buffers inside a trace slot (the workspace
+        head, cap 1): ``qg_decode_step_inspect`` and ``_inspect_f32``."""
+        off = (ctypes.c_size_t * 4)()
+        _call("qg_decode_step_inspect", ctypes.byref(self.c_cfg), B, 1, off)
+        off32 = (ctypes.c_size_t * 6)()
+        _call("qg_decode_step_inspect_f32", ctypes.byref(self.c_cfg), B, 1, off32)
+        return list(off), list(off32)
+
+    def qg_code_predict_traced(self, lm_hidden, code0, codes, ws, trace, logits=None,
+                               stream=None):
+        """qg_code_predict that also fills ``trace`` (uint8, trace_layout()[0]
+        bytes) with every group's layer values."""
+        B = lm_hidden.shape[0]
+        _call("qg_code_predict_traced", ctypes.byref(self.c_cfg), ctypes.byref(self.c_weights),
+              _p(lm_hidden), _p(code0), _p(codes), _p(logits), B, _p(ws), ws.numel(),
+              _p(trace), trace.numel(), _stream(stream))
+
+
+class WhisperEncoderLayer:
+    """Device-resident weights of one Whisper encoder layer (the host dict of
+    ``qg_synth.whisper_layer_weights``) and ``qg_whisper_encoder_layer``."""
+
+    NAMES = ("ln1_g", "ln1_b", "q", "q_b", "k", "v", "v_b", "o", "o_b", "ln2_g", "ln2_b", "fc1",
+             "fc1_b", "fc2", "fc2_b")
+
+    def __init__(self, cfg: dict, weights: dict, device="cuda"):
+        self.cfg = dict(cfg)
+        self._keep = {}
+        for n in self.NAMES:
+            a = weights[n]
+            t = torch.from_numpy(a if a.dtype == "uint8" else a.astype("float32")).to(device)
+            self._keep[n] = t
+        self.c_cfg = qg_whisper_config(cfg["d_model"], cfg["heads"], cfg["ffn"], cfg["eps"])
+        self.c_w = qg_whisper_layer(*[self._keep[n].data_ptr() for n in self.NAMES])
+        self.device = device
+
+    def tensor(self, name):
+        return self._keep[name]
+
+    def workspace(self, M):
+        n = int(lib.qg_whisper_encoder_layer_workspace_size(ctypes.byref(self.c_cfg), M))
+        return torch.empty(n, dtype=torch.uint8, device=self.device)
+
+    def qg_whisper_encoder_layer(self, x, ws, stream=None):
+        """x fp32 [M, d_model] in place."""
+        _call("qg_whisper_encoder_layer", ctypes.byref(self.c_cfg), ctypes.byref(self.c_w), _p(x),
+              x.shape[0], _p(ws), ws.numel(), _stream(stream))
+
+    def intermediates(self, ws, M):
+        """Views into the workspace after a call: bf16 ``xl``, ``q``, ``k``,
+        ``v``, ``ctx``, ``xl2`` [M, d], ``mid`` [M, ffn]; fp32 ``xa`` [M, d];
+        and the six matmuls' error words (``err``, int32)."""
+        off = (ctypes.c_size_t * 9)()
+        _call("qg_whisper_encoder_layer_inspect", ctypes.byref(self.c_cfg), M, off)
+        d, F = self.cfg["d_model"], self.cfg["ffn"]
+
+        def view(o, n, dt=torch.bfloat16):
+            size = 2 if dt == torch.bfloat16 else 4
+            return ws[o:o + size * M * n].view(dt).view(M, n)
+        out = {name: view(off[i], d) for i, name in enumerate(("xl", "q", "k", "v", "ctx"))}
+        out["xa"] = view(off[5], d, torch.float32)
+        out["xl2"] = view(off[6], d)
+        out["mid"] = view(off[7], F)
+        out["err"] = ws[off[8]:off[8] + 6 * 256].view(torch.int32).view(6, 64)[:, 0]
+        return out

@@ -1,6 +1,6 @@
 """Build libqg.so (sm_100a) in-tree with nvcc.
 
-Usage: python weight_only_quantized_03_b200/build.py [--force] [-v] [--ptxas-v]
+Usage: python weight_only_quantized_03_b200/build.py [--force] [-v] [--ptxas-v] [--timeline]
 Objects go to _build/ at the repository root; the shared library lands next
 to this file so that it travels with the source tree.
 """
@@ -19,6 +19,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libqg.so")
+TIMELINE_LIB = os.path.join(PKG, "libqg_timeline.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O3",
@@ -42,8 +43,8 @@ def _headers_mtime():
     return max(os.path.getmtime(h) for h in hs) if hs else 0.0
 
 
-def _compile(src, force, verbose, extra):
-    obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+def _compile(src, force, verbose, extra, objdir=BUILD):
+    obj = os.path.join(objdir, os.path.basename(src)[:-3] + ".o")
     if (not force and os.path.exists(obj)
             and os.path.getmtime(obj) >= max(os.path.getmtime(src), _headers_mtime())):
         return obj, ""
@@ -56,23 +57,29 @@ def _compile(src, force, verbose, extra):
     return obj, r.stderr
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, extra=(), timeline: bool = False) -> str:
+    """Build libqg.so, or with ``timeline`` the diagnostic variant
+    libqg_timeline.so (QG_TIMELINE: per-launch timestamps, see
+    qg_timeline_begin in include/qg.h) from objects of its own."""
+    objdir = os.path.join(BUILD, "timeline") if timeline else BUILD
+    lib = TIMELINE_LIB if timeline else LIB
+    extra = list(extra) + (["-DQG_TIMELINE"] if timeline else [])
+    os.makedirs(objdir, exist_ok=True)
     srcs = sources()
     with cf.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
-        results = list(ex.map(lambda s: _compile(s, force, verbose, list(extra)), srcs))
+        results = list(ex.map(lambda s: _compile(s, force, verbose, extra, objdir), srcs))
     objs = [o for o, _ in results]
     for _, log in results:
         if verbose and log:
             print(log)
-    if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < max(os.path.getmtime(o) for o in objs):
-        cmd = [nvcc(), *ARCH, "-shared", "-o", LIB, *objs]
+    if force or not os.path.exists(lib) or os.path.getmtime(lib) < max(os.path.getmtime(o) for o in objs):
+        cmd = [nvcc(), *ARCH, "-shared", "-o", lib, *objs]
         if verbose:
             print(" ".join(cmd), flush=True)
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    return LIB
+    return lib
 
 
 if __name__ == "__main__":
@@ -80,7 +87,10 @@ if __name__ == "__main__":
     ap.add_argument("--force", action="store_true")
     ap.add_argument("-v", "--verbose", action="store_true")
     ap.add_argument("--ptxas-v", action="store_true", help="print register/smem usage")
+    ap.add_argument("--timeline", action="store_true",
+                    help="build the diagnostic libqg_timeline.so (QG_TIMELINE)")
     a = ap.parse_args()
     extra = ["-Xptxas", "-v"] if a.ptxas_v else []
-    print(build(force=a.force or a.ptxas_v, verbose=a.verbose or a.ptxas_v, extra=extra))
+    print(build(force=a.force or a.ptxas_v, verbose=a.verbose or a.ptxas_v, extra=extra,
+                timeline=a.timeline))
     sys.exit(0)

@@ -64,10 +64,11 @@ attention_split_kernel(const float* __restrict__ q, const uint16_t* __restrict__
                        unsigned int* __restrict__ ws_cnt, const AttnFuse fz) {
   attention_body<VPL, kAttnWarps, kMaxGroup>(
       q, kc, vc, kv_len, pos_for_len, out, out_bf16, H, Hkv, cap, scale, ch, nsplit, ws_o, ws_ml,
-      ws_cnt, fz, blockIdx.x, blockIdx.y, blockIdx.z, [] {
+      ws_cnt, fz, blockIdx.x, blockIdx.y, blockIdx.z, [&] {
         // the next kernel may be scheduled now: its own wait covers all of this one
         pdl_trigger();
         pdl_wait();
+        tl_wait(fz.tl);
       });
 }
 
@@ -167,6 +168,8 @@ attention_cluster_kernel(const float* q, const uint16_t* kc, const uint16_t* vc,
   __shared__ float cm[GM], cl[GM];     // this CTA's partial, read by rank 0
   __shared__ float co[GM][D];
 
+  tl_entry(fz.tl);
+  attn_issue_prefetch(fz);
   const unsigned s = cluster_rank();
   const unsigned cs = gridDim.x;
   const int kv = blockIdx.y, b = blockIdx.z;
@@ -208,6 +211,7 @@ attention_cluster_kernel(const float* q, const uint16_t* kc, const uint16_t* vc,
   // the next kernel may be scheduled now: its own wait covers all of this one
   pdl_trigger();
   pdl_wait();
+  tl_wait(fz.tl);
   if (!fz.on) {
     const int L = kv_len[b];
     valid = L >= 1 && L <= cap;
@@ -406,6 +410,7 @@ attention_cluster_kernel(const float* q, const uint16_t* kc, const uint16_t* vc,
     }
   }
   cluster_sync();  // no CTA leaves while rank 0 still reads its shared memory
+  tl_exit(fz.tl);
 }
 
 // Whether the cluster kernel takes the shape.
@@ -530,8 +535,19 @@ cudaError_t attention_launch_step(const float* q, const float* k, const float* v
                                   const int32_t* tokens, int vocab, float eps, const float2* rope,
                                   uint16_t* kc, uint16_t* vc, const int32_t* positions, void* out,
                                   int B, int H, int Hkv, int D, int cap, float scale, void* ws,
-                                  cudaStream_t st, bool pdl) {
-  AttnFuse fz = {1, k, v, q_norm, k_norm, tokens, vocab, eps, rope};
+                                  cudaStream_t st, bool pdl, const Prefetch* pf) {
+  AttnFuse fz = {};
+  fz.on = 1;
+  fz.k = k;
+  fz.v = v;
+  fz.qn = q_norm;
+  fz.kn = k_norm;
+  fz.tok = tokens;
+  fz.vocab = vocab;
+  fz.eps = eps;
+  fz.rope = rope;
+  if (pf) fz.pf = *pf;
+  fz.tl = tl_take(0);
   return attention_launch_any(q, kc, vc, nullptr, positions, out, true, B, H, Hkv, D, cap, scale,
                               ws, st, pdl, fz);
 }

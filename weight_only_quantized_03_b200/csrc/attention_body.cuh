@@ -24,7 +24,17 @@ struct AttnFuse {
   int vocab;
   float eps;
   const float2* rope;    // (cos, sin) [B][D/2] of the step's positions
+  Prefetch pf;           // L2 prefetch work for a later kernel of the step
+  TlRec* tl;             // timeline record of this launch, or null
 };
+
+// The fused step's L2 prefetch, issued by one thread of each CTA at entry.
+__device__ __forceinline__ void attn_issue_prefetch(const AttnFuse& fz) {
+  if (fz.on && threadIdx.x == 0 && (fz.pf.n > 0 || fz.pf.kv.kc)) {
+    const unsigned cta = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+    issue_prefetch(fz.pf, cta, gridDim.x * gridDim.y * gridDim.z);
+  }
+}
 
 // q, k, v and the RoPE table are produced by the previous kernels of the
 // step; they are read through L2 (ld.global.cg), not kept in L1.
@@ -96,6 +106,8 @@ __device__ __forceinline__ void attention_body(
   constexpr int kAttnWarps = NW, kMaxGroup = GM;
   const int g = H / Hkv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  tl_entry(fz.tl);
+  attn_issue_prefetch(fz);
 
   __shared__ float sq[kMaxGroup][D];
   __shared__ float sm[kAttnWarps][kMaxGroup], sl[kAttnWarps][kMaxGroup];
@@ -270,7 +282,10 @@ __device__ __forceinline__ void attention_body(
   __syncthreads();
   if (threadIdx.x == 0) s_ticket = atomicAdd(&ws_cnt[b * Hkv + kv], 1u);
   __syncthreads();
-  if (s_ticket != (unsigned)(nsplit - 1)) return;
+  if (s_ticket != (unsigned)(nsplit - 1)) {
+    tl_exit(fz.tl);
+    return;
+  }
   __threadfence();
 
   auto store_out = [&](int h, int d, float r) {
@@ -344,6 +359,7 @@ __device__ __forceinline__ void attention_body(
     }
   }
   if (threadIdx.x == 0) ws_cnt[b * Hkv + kv] = 0u;  // ready for the next launch
+  tl_exit(fz.tl);
 }
 
 }  // namespace qg

@@ -22,7 +22,7 @@ namespace qg {
 size_t attention_ws_counter_offset(int B, int H, int Hkv, int D, int cap);
 
 struct StepLayout {
-  size_t x, xn, xn2, xnf, q, k, v, attn, gate, up, h, attn_ws, rope, total;
+  size_t x, xn, xn2, xnf, q, k, v, xa, attn, gate, up, h, attn_ws, rope, err, total;
 };
 
 static size_t a256(size_t v) { return (v + 255) & ~(size_t)255; }
@@ -40,12 +40,14 @@ static StepLayout step_layout(const qg_qwen3_config& c, int B, int cap) {
   L.q = take((size_t)B * qd * 4);
   L.k = take((size_t)B * kd * 4);
   L.v = take((size_t)B * kd * 4);
+  L.xa = take((size_t)B * c.hidden * 4);  // residual stream after o_proj
   L.attn = take((size_t)B * qd * 2);
   L.gate = take((size_t)B * c.ffn * 4);
   L.up = take((size_t)B * c.ffn * 4);
   L.h = take((size_t)B * c.ffn * 2);
   L.attn_ws = take(attention_ws_bytes(B, c.heads, c.kv_heads, c.head_dim, cap));
   L.rope = take((size_t)B * (c.head_dim / 2) * 8);
+  L.err = take(256);  // error word of the tensor-core matmuls (batched steps)
   L.total = off;
   return L;
 }
@@ -58,7 +60,14 @@ __global__ void step_embed_kernel(const uint32_t* __restrict__ w, const uint16_t
                                   const uint16_t* __restrict__ bi, const int32_t* __restrict__ tok,
                                   const int32_t* __restrict__ pos, float* __restrict__ x, int vocab,
                                   int hidden, int cap, float2* __restrict__ rope, int D,
-                                  double theta) {
+                                  double theta, const __grid_constant__ Prefetch pf,
+                                  TlRec* tl) {
+  tl_entry(tl);
+  // the first layer's weights and cached rows go to L2 (lane 0 of each warp)
+  if ((threadIdx.x & 31) == 0 && (pf.n > 0 || pf.kv.kc)) {
+    const unsigned wpb = blockDim.x >> 5;
+    issue_prefetch(pf, blockIdx.x * wpb + (threadIdx.x >> 5), gridDim.x * wpb);
+  }
   pdl_wait();
   const int b = blockIdx.x;
   const int t = tok[b], p = pos[b];
@@ -81,6 +90,7 @@ __global__ void step_embed_kernel(const uint32_t* __restrict__ w, const uint16_t
     xr[c] = fmaf(q, bf16_bits_to_f32(s[g]), bf16_bits_to_f32(bi[g]));
   }
   pdl_trigger();
+  tl_exit(tl);
 }
 
 __global__ void step_silu_mul_kernel(const float* __restrict__ g, const float* __restrict__ u,
@@ -142,12 +152,13 @@ extern "C" size_t qg_decode_step_workspace_size(const qg_qwen3_config* cfg, int 
 struct StepBufs {
   float* x;
   uint16_t *xn, *xn2, *xnf;
-  float *q, *k, *v;
+  float *q, *k, *v, *xa;
   uint16_t* attn;
   float *gate, *up;
   uint16_t* hm;
   void* aws;
   float2* rope;
+  unsigned* err;
 };
 
 static StepBufs step_bufs(void* ws, const StepLayout& Ly) {
@@ -160,20 +171,65 @@ static StepBufs step_bufs(void* ws, const StepLayout& Ly) {
   b.q = reinterpret_cast<float*>(base + Ly.q);
   b.k = reinterpret_cast<float*>(base + Ly.k);
   b.v = reinterpret_cast<float*>(base + Ly.v);
+  b.xa = reinterpret_cast<float*>(base + Ly.xa);
   b.attn = reinterpret_cast<uint16_t*>(base + Ly.attn);
   b.gate = reinterpret_cast<float*>(base + Ly.gate);
   b.up = reinterpret_cast<float*>(base + Ly.up);
   b.hm = reinterpret_cast<uint16_t*>(base + Ly.h);
   b.aws = base + Ly.attn_ws;
   b.rope = reinterpret_cast<float2*>(base + Ly.rope);
+  b.err = reinterpret_cast<unsigned*>(base + Ly.err);
   return b;
 }
 
 // The decoder layers on the residual stream sb.x (5 launches a layer where
 // the tensor-core GEMV takes the shapes), in stream order on s.
+// L2 prefetch lists of the step: each kernel hands L2 the data of the
+// kernel two launches after it (q/k/v -> o_proj, attention -> gate/up,
+// o_proj -> down, gate/up -> the next layer's q/k/v, down -> the next
+// layer's cached K/V rows), so the weight stream runs ahead of the chain.
+static void pf_matrix(Prefetch& pf, const qg_affine8_matrix& m, int N, int K) {
+  if (pf.n + 3 > kMaxPf) return;
+  pf.r[pf.n++] = PfRange{m.w, (unsigned long long)N * K};
+  pf.r[pf.n++] = PfRange{m.scales, (unsigned long long)N * (K / 64) * 2};
+  pf.r[pf.n++] = PfRange{m.biases, (unsigned long long)N * (K / 64) * 2};
+}
+
+static Prefetch pf_qkv(const qg_qwen3_config& c, const qg_qwen3_layer& L) {
+  Prefetch pf = {};
+  const int HD = c.heads * c.head_dim, KD = c.kv_heads * c.head_dim;
+  pf_matrix(pf, L.q, HD, c.hidden);
+  pf_matrix(pf, L.k, KD, c.hidden);
+  pf_matrix(pf, L.v, KD, c.hidden);
+  return pf;
+}
+
+static Prefetch pf_kv(const qg_qwen3_config& c, const uint16_t* kc, const uint16_t* vc,
+                      const int32_t* positions, int B, int cap) {
+  Prefetch pf = {};
+  pf.kv = KvPf{kc, vc, positions, B, c.kv_heads, cap, c.head_dim};
+  return pf;
+}
+
+// From this batch size on, the step's linears run as tensor-core matmuls
+// (gemm_affine8_sm100.cu: the batch rows are the MMA's N, each weight tile is
+// dequantized once for all rows) with RMSNorm and SiLU-mul as separate
+// kernels; below it, the tensor-core GEMV streams the weights with the
+// norms fused into its prologue.
+constexpr int kStepGemmBatch = 5;
+
+static bool step_uses_gemm(const qg_qwen3_config& c, int B) {
+  return B >= kStepGemmBatch && c.hidden % 64 == 0 && c.ffn % 64 == 0 &&
+         (c.heads * c.head_dim) % 64 == 0;
+}
+
+// `after_layer`, when given, is called with the layer index after each
+// layer's launches are enqueued.
+template <class AfterLayer>
 static void enqueue_layers(const qg_qwen3_config& c, const qg_qwen3_layer* layers,
                            uint16_t* k_cache, uint16_t* v_cache, int cap, const int32_t* tokens,
-                           const int32_t* positions, int B, const StepBufs& sb, cudaStream_t s) {
+                           const int32_t* positions, int B, const StepBufs& sb, cudaStream_t s,
+                           AfterLayer&& after_layer) {
   const int H = c.heads, Hkv = c.kv_heads, D = c.head_dim;
   const size_t layer_cache = (size_t)B * Hkv * cap * D;
   const float scale = 1.0f / sqrtf((float)D);
@@ -185,36 +241,93 @@ static void enqueue_layers(const qg_qwen3_config& c, const qg_qwen3_layer* layer
     GemvSeg qkv[3] = {{L.q.w, L.q.scales, L.q.biases, sb.q, nullptr, H * D, 0},
                       {L.k.w, L.k.scales, L.k.biases, sb.k, nullptr, Hkv * D, 0},
                       {L.v.w, L.v.scales, L.v.biases, sb.v, nullptr, Hkv * D, 0}};
+    Prefetch pf_o = {}, pf_gu = {}, pf_dn = {};
+    pf_matrix(pf_o, L.o, c.hidden, H * D);
+    pf_matrix(pf_gu, L.gate, c.ffn, c.hidden);
+    pf_matrix(pf_gu, L.up, c.ffn, c.hidden);
+    pf_matrix(pf_dn, L.down, c.hidden, c.ffn);
+    const bool last = l + 1 == c.layers;
+    const Prefetch pf_next_qkv = last ? Prefetch{} : pf_qkv(c, layers[l + 1]);
+    const Prefetch pf_next_kv =
+        last ? Prefetch{} : pf_kv(c, kc + layer_cache, vc + layer_cache, positions, B, cap);
+    if (step_uses_gemm(c, B)) {
+      tl_set_kind(kTlQkv);
+      rmsnorm_launch(x, L.input_norm, c.eps, sb.xn, true, B, c.hidden, s, true);
+      const A8Seg m_qkv[3] = {{L.q.w, L.q.scales, L.q.biases, sb.q, nullptr, H * D, 0},
+                              {L.k.w, L.k.scales, L.k.biases, sb.k, nullptr, Hkv * D, 0},
+                              {L.v.w, L.v.scales, L.v.biases, sb.v, nullptr, Hkv * D, 0}};
+      gemm_affine8_launch(m_qkv, 3, sb.xn, B, c.hidden, sb.err, s, true, nullptr);
+      tl_set_kind(kTlAttn);
+      attention_launch_step(sb.q, sb.k, sb.v, L.q_norm, L.k_norm, tokens, c.vocab, c.eps,
+                            sb.rope, kc, vc, positions, sb.attn, B, H, Hkv, D, cap, scale,
+                            sb.aws, s, true, &pf_gu);
+      tl_set_kind(kTlO);
+      const A8Seg m_o = {L.o.w, L.o.scales, L.o.biases, sb.xa, x, c.hidden, 0};
+      gemm_affine8_launch(&m_o, 1, sb.attn, B, H * D, sb.err, s, true, nullptr);
+      tl_set_kind(kTlGateUp);
+      rmsnorm_launch(sb.xa, L.post_norm, c.eps, sb.xn2, true, B, c.hidden, s, true);
+      const A8Seg m_gu[2] = {{L.gate.w, L.gate.scales, L.gate.biases, sb.gate, nullptr, c.ffn, 0},
+                             {L.up.w, L.up.scales, L.up.biases, sb.up, nullptr, c.ffn, 0}};
+      gemm_affine8_launch(m_gu, 2, sb.xn2, B, c.hidden, sb.err, s, true, nullptr);
+      tl_set_kind(kTlDown);
+      const int n = B * c.ffn;
+      launch_pdl(step_silu_mul_kernel, dim3((n + 255) / 256), dim3(256), 0, s, true,
+                 (const float*)sb.gate, (const float*)sb.up, sb.hm, n);
+      const A8Seg m_dn = {L.down.w, L.down.scales, L.down.biases, x, sb.xa, c.hidden, 0};
+      gemm_affine8_launch(&m_dn, 1, sb.hm, B, c.ffn, sb.err, s, true, nullptr);
+      after_layer(l);
+      continue;
+    }
     // RMSNorm and SiLU-mul run in the next GEMV's prologue where the
     // tensor-core GEMV takes the shape, as separate kernels otherwise
+    tl_set_kind(kTlQkv);
     if (gemv_tc_eligible(qkv, 3, c.hidden, B, false)) {
-      gemv_tc_launch_rmsnorm(qkv, 3, x, L.input_norm, c.eps, c.hidden, B, s, true, sb.xn);
+      gemv_tc_launch_rmsnorm(qkv, 3, x, L.input_norm, c.eps, c.hidden, B, s, true, sb.xn, &pf_o);
     } else {
       rmsnorm_launch(x, L.input_norm, c.eps, sb.xn, true, B, c.hidden, s, true);
       gemv_affine8_launch(qkv, 3, sb.xn, false, c.hidden, B, s, true);
     }
+    tl_set_kind(kTlAttn);
     attention_launch_step(sb.q, sb.k, sb.v, L.q_norm, L.k_norm, tokens, c.vocab, c.eps, sb.rope,
-                          kc, vc, positions, sb.attn, B, H, Hkv, D, cap, scale, sb.aws, s, true);
-    GemvSeg o = {L.o.w, L.o.scales, L.o.biases, x, x, c.hidden, 0};
-    gemv_affine8_launch(&o, 1, sb.attn, false, H * D, B, s, true);
+                          kc, vc, positions, sb.attn, B, H, Hkv, D, cap, scale, sb.aws, s, true,
+                          &pf_gu);
+    // o_proj: xa = x + W_o attn; down: x = xa + W_down h (the residual
+    // stream after attention stays readable until the next layer)
+    GemvSeg o = {L.o.w, L.o.scales, L.o.biases, sb.xa, x, c.hidden, 0};
+    tl_set_kind(kTlO);
+    if (gemv_tc_eligible(&o, 1, H * D, B, false))
+      gemv_tc_launch_pf(&o, 1, sb.attn, H * D, B, s, true, &pf_dn);
+    else
+      gemv_affine8_launch(&o, 1, sb.attn, false, H * D, B, s, true);
     GemvSeg gu[2] = {{L.gate.w, L.gate.scales, L.gate.biases, sb.gate, nullptr, c.ffn, 0},
                      {L.up.w, L.up.scales, L.up.biases, sb.up, nullptr, c.ffn, 0}};
+    tl_set_kind(kTlGateUp);
     if (gemv_tc_eligible(gu, 2, c.hidden, B, false)) {
-      gemv_tc_launch_rmsnorm(gu, 2, x, L.post_norm, c.eps, c.hidden, B, s, true, sb.xn2);
+      gemv_tc_launch_rmsnorm(gu, 2, sb.xa, L.post_norm, c.eps, c.hidden, B, s, true, sb.xn2,
+                             &pf_next_qkv);
     } else {
-      rmsnorm_launch(x, L.post_norm, c.eps, sb.xn2, true, B, c.hidden, s, true);
+      rmsnorm_launch(sb.xa, L.post_norm, c.eps, sb.xn2, true, B, c.hidden, s, true);
       gemv_affine8_launch(gu, 2, sb.xn2, false, c.hidden, B, s, true);
     }
-    GemvSeg dn = {L.down.w, L.down.scales, L.down.biases, x, x, c.hidden, 0};
+    GemvSeg dn = {L.down.w, L.down.scales, L.down.biases, x, sb.xa, c.hidden, 0};
+    tl_set_kind(kTlDown);
     if (gemv_tc_eligible(&dn, 1, c.ffn, B, false)) {
-      gemv_tc_launch_silu_mul(&dn, 1, sb.gate, sb.up, c.ffn, B, s, true, sb.hm);
+      gemv_tc_launch_silu_mul(&dn, 1, sb.gate, sb.up, c.ffn, B, s, true, sb.hm, &pf_next_kv);
     } else {
       const int n = B * c.ffn;
       launch_pdl(step_silu_mul_kernel, dim3((n + 255) / 256), dim3(256), 0, s, true,
                  (const float*)sb.gate, (const float*)sb.up, sb.hm, n);
       gemv_affine8_launch(&dn, 1, sb.hm, false, c.ffn, B, s, true);
     }
+    after_layer(l);
   }
+  tl_set_kind(kTlOther);
+}
+
+static void enqueue_layers(const qg_qwen3_config& c, const qg_qwen3_layer* layers,
+                           uint16_t* k_cache, uint16_t* v_cache, int cap, const int32_t* tokens,
+                           const int32_t* positions, int B, const StepBufs& sb, cudaStream_t s) {
+  enqueue_layers(c, layers, k_cache, v_cache, cap, tokens, positions, B, sb, s, [](int) {});
 }
 
 // Final RMSNorm and an output head [N][hidden] on sb.x: logits [B][N].
@@ -222,12 +335,18 @@ static void enqueue_head(const qg_qwen3_config& c, const qg_affine8_matrix& head
                          const uint16_t* final_norm, float* logits, int B, const StepBufs& sb,
                          cudaStream_t s) {
   GemvSeg h = {head.w, head.scales, head.biases, logits, nullptr, N, 0};
-  if (gemv_tc_eligible(&h, 1, c.hidden, B, false)) {
+  tl_set_kind(kTlHead);
+  if (step_uses_gemm(c, B)) {
+    rmsnorm_launch(sb.x, final_norm, c.eps, sb.xnf, true, B, c.hidden, s, true);
+    const A8Seg m = {head.w, head.scales, head.biases, logits, nullptr, N, 0};
+    gemm_affine8_launch(&m, 1, sb.xnf, B, c.hidden, sb.err, s, true, nullptr);
+  } else if (gemv_tc_eligible(&h, 1, c.hidden, B, false)) {
     gemv_tc_launch_rmsnorm(&h, 1, sb.x, final_norm, c.eps, c.hidden, B, s, true);
   } else {
     rmsnorm_launch(sb.x, final_norm, c.eps, sb.xnf, true, B, c.hidden, s, true);
     gemv_affine8_launch(&h, 1, sb.xnf, false, c.hidden, B, s, true);
   }
+  tl_set_kind(kTlOther);
 }
 
 // Every launch of one step, in stream order on s (the eager path, and what
@@ -239,9 +358,15 @@ static void enqueue_step(const qg_qwen3_config& c, const qg_qwen3_weights* w, ui
   const StepBufs sb = step_bufs(ws, Ly);
   const size_t cnt_off = attention_ws_counter_offset(B, c.heads, c.kv_heads, c.head_dim, cap);
   cudaMemsetAsync(reinterpret_cast<uint8_t*>(sb.aws) + cnt_off, 0, (size_t)B * c.kv_heads * 4, s);
+  if (step_uses_gemm(c, B)) cudaMemsetAsync(sb.err, 0, 4, s);
+  Prefetch pf0 = {};
+  if (c.layers > 0) {
+    pf0 = pf_qkv(c, w->layers[0]);
+    pf0.kv = KvPf{k_cache, v_cache, positions, B, c.kv_heads, cap, c.head_dim};
+  }
   launch_pdl(step_embed_kernel, dim3(B), dim3(256), 0, s, true, w->embed.w, w->embed.scales,
              w->embed.biases, tokens, positions, sb.x, c.vocab, c.hidden, cap, sb.rope, c.head_dim,
-             c.theta);
+             c.theta, pf0, tl_take(kTlEmbed));
   enqueue_layers(c, w->layers, k_cache, v_cache, cap, tokens, positions, B, sb, s);
   enqueue_head(c, w->embed, c.vocab, w->final_norm, logits, B, sb, s);
 }
@@ -458,6 +583,22 @@ extern "C" qg_status qg_decode_step_inspect(const qg_qwen3_config* cfg, int B, i
   return QG_OK;
 }
 
+extern "C" qg_status qg_decode_step_inspect_f32(const qg_qwen3_config* cfg, int B, int cap,
+                                               size_t offsets[6]) {
+  clear_error();
+  qg_status st = validate_cfg(cfg, B, cap);
+  if (st != QG_OK) return st;
+  QG_REQUIRE(offsets, QG_ERR_INVALID_ARGUMENT, "qg_decode_step_inspect_f32: null offsets");
+  const StepLayout Ly = step_layout(*cfg, B, cap);
+  offsets[0] = Ly.q;
+  offsets[1] = Ly.k;
+  offsets[2] = Ly.v;
+  offsets[3] = Ly.xa;
+  offsets[4] = Ly.gate;
+  offsets[5] = Ly.up;
+  return QG_OK;
+}
+
 // ---------------------------------------------------------------------------
 // Code predictor: makima src/tts/qwen3/code_predictor.rs, CodePredictor::
 // predict. Per group g = 1 .. groups-1: embed code g-1 with table g-1,
@@ -540,19 +681,41 @@ extern "C" size_t qg_code_predict_workspace_size(const qg_qwen3_config* cfg, int
   return cp_layout(*cfg, B).total;
 }
 
-extern "C" qg_status qg_code_predict(const qg_qwen3_config* cfg, const qg_code_predictor_weights* w,
-                                     const float* lm_hidden, const int32_t* code0, int32_t* codes,
-                                     float* logits, int B, void* ws, size_t ws_bytes,
-                                     void* stream) {
+namespace {
+
+// Trace of a traced code prediction: per group g = 1 .. groups-1, the bf16
+// concatenated input, then one slot after input_proj and one after each
+// layer, each a copy of the workspace head (the step buffers up to the
+// attention scratch) followed by the K and V rows the slot's layer wrote.
+struct CpTrace {
+  size_t comb, snap, kv, slot, group, total;
+};
+
+CpTrace cp_trace_layout(const qg_qwen3_config& c, int B, int groups) {
+  const CpLayout Ly = cp_layout(c, B);
+  CpTrace T;
+  T.comb = a256((size_t)B * 2 * c.hidden * 2);
+  T.snap = Ly.step.attn_ws;  // x .. h: every step buffer before the attention scratch
+  T.kv = a256((size_t)B * c.kv_heads * c.head_dim * 2);
+  T.slot = T.snap + 2 * T.kv;
+  T.group = T.comb + (size_t)(c.layers + 1) * T.slot;
+  T.total = (size_t)(groups > 1 ? groups - 1 : 0) * T.group;
+  return T;
+}
+
+qg_status code_predict_impl(const qg_qwen3_config* cfg, const qg_code_predictor_weights* w,
+                            const float* lm_hidden, const int32_t* code0, int32_t* codes,
+                            float* logits, int B, void* ws, size_t ws_bytes, void* trace,
+                            size_t trace_bytes, void* stream, const char* what) {
   clear_error();
   qg_status st = validate_cfg(cfg, B, 1);
   if (st != QG_OK) return st;
   const qg_qwen3_config& c = *cfg;
-  QG_REQUIRE(w, QG_ERR_INVALID_ARGUMENT, "qg_code_predict: weights is NULL");
+  QG_REQUIRE(w, QG_ERR_INVALID_ARGUMENT, "%s: weights is NULL", what);
   QG_REQUIRE(w->groups >= 2 && w->groups <= 64, QG_ERR_UNSUPPORTED_SHAPE,
-             "qg_code_predict: groups=%d must be in [2, 64]", w->groups);
+             "%s: groups=%d must be in [2, 64]", what, w->groups);
   QG_REQUIRE(w->code_embed && w->heads && w->final_norm && (c.layers == 0 || w->layers),
-             QG_ERR_INVALID_ARGUMENT, "qg_code_predict: null table, head, norm or layer array");
+             QG_ERR_INVALID_ARGUMENT, "%s: null table, head, norm or layer array", what);
   if ((st = validate_matrix(w->input_proj, "input_proj", -1)) != QG_OK) return st;
   for (int g = 1; g < w->groups; ++g) {
     if ((st = validate_matrix(w->code_embed[g - 1], "code_embed", g - 1)) != QG_OK) return st;
@@ -563,20 +726,28 @@ extern "C" qg_status qg_code_predict(const qg_qwen3_config* cfg, const qg_code_p
     for (const qg_affine8_matrix* m : {&L.q, &L.k, &L.v, &L.o, &L.gate, &L.up, &L.down})
       if ((st = validate_matrix(*m, "layer", l)) != QG_OK) return st;
     QG_REQUIRE(L.input_norm && L.post_norm && L.q_norm && L.k_norm, QG_ERR_INVALID_ARGUMENT,
-               "qg_code_predict: layer %d has a null norm weight", l);
+               "%s: layer %d has a null norm weight", what, l);
   }
   QG_REQUIRE(lm_hidden && code0 && codes, QG_ERR_INVALID_ARGUMENT,
-             "qg_code_predict: null lm_hidden, code0 or codes");
+             "%s: null lm_hidden, code0 or codes", what);
   QG_REQUIRE(aligned(lm_hidden, 4) && aligned(code0, 4) && aligned(codes, 4) &&
                  aligned(logits, 4),
-             QG_ERR_MISALIGNED, "qg_code_predict: lm_hidden/code0/codes/logits misaligned");
+             QG_ERR_MISALIGNED, "%s: lm_hidden/code0/codes/logits misaligned", what);
   const CpLayout Ly = cp_layout(c, B);
   QG_REQUIRE(ws && ws_bytes >= Ly.total, QG_ERR_WORKSPACE_TOO_SMALL,
-             "qg_code_predict: workspace of %zu bytes given, %zu needed", ws_bytes, Ly.total);
-  QG_REQUIRE(aligned(ws, 256), QG_ERR_MISALIGNED, "qg_code_predict: ws not 256-byte aligned");
+             "%s: workspace of %zu bytes given, %zu needed", what, ws_bytes, Ly.total);
+  QG_REQUIRE(aligned(ws, 256), QG_ERR_MISALIGNED, "%s: ws not 256-byte aligned", what);
+  const CpTrace T = cp_trace_layout(c, B, w->groups);
+  if (trace) {
+    QG_REQUIRE(trace_bytes >= T.total, QG_ERR_WORKSPACE_TOO_SMALL,
+               "%s: trace of %zu bytes given, %zu needed", what, trace_bytes, T.total);
+    QG_REQUIRE(aligned(trace, 256), QG_ERR_MISALIGNED, "%s: trace not 256-byte aligned", what);
+  }
 
   cudaStream_t s = (cudaStream_t)stream;
   uint8_t* base = reinterpret_cast<uint8_t*>(ws);
+  uint8_t* tr = reinterpret_cast<uint8_t*>(trace);
+  const size_t kv_row = (size_t)B * c.kv_heads * c.head_dim * 2;  // one layer's cache (cap 1)
   auto enqueue = [&] {
     const StepBufs sb = step_bufs(ws, Ly.step);
     uint16_t* comb = reinterpret_cast<uint16_t*>(base + Ly.comb);
@@ -597,7 +768,25 @@ extern "C" qg_status qg_code_predict(const qg_qwen3_config* cfg, const qg_code_p
       GemvSeg ip = {w->input_proj.w, w->input_proj.scales, w->input_proj.biases, sb.x, nullptr,
                     c.hidden, 0};
       gemv_affine8_launch(&ip, 1, comb, false, 2 * c.hidden, B, s, true);
-      enqueue_layers(c, w->layers, kc, vc, 1, prev, pos, B, sb, s);
+      uint8_t* tg = tr ? tr + (size_t)(g - 1) * T.group : nullptr;
+      auto snapshot = [&](int slot) {
+        uint8_t* d = tg + T.comb + (size_t)slot * T.slot;
+        cudaMemcpyAsync(d, base, T.snap, cudaMemcpyDeviceToDevice, s);
+        if (slot > 0) {
+          const size_t lo = (size_t)(slot - 1) * kv_row;
+          cudaMemcpyAsync(d + T.snap, reinterpret_cast<uint8_t*>(kc) + lo, kv_row,
+                          cudaMemcpyDeviceToDevice, s);
+          cudaMemcpyAsync(d + T.snap + T.kv, reinterpret_cast<uint8_t*>(vc) + lo, kv_row,
+                          cudaMemcpyDeviceToDevice, s);
+        }
+      };
+      if (tg) {
+        cudaMemcpyAsync(tg, comb, (size_t)B * 2 * c.hidden * 2, cudaMemcpyDeviceToDevice, s);
+        snapshot(0);
+      }
+      enqueue_layers(c, w->layers, kc, vc, 1, prev, pos, B, sb, s, [&](int l) {
+        if (tg) snapshot(l + 1);
+      });
       float* lg = logits ? logits + (size_t)g * B * c.vocab
                          : reinterpret_cast<float*>(base + Ly.logits);
       enqueue_head(c, w->heads[g], c.vocab, w->final_norm, lg, B, sb, s);
@@ -608,7 +797,8 @@ extern "C" qg_status qg_code_predict(const qg_qwen3_config* cfg, const qg_code_p
   key.push_back(2);  // what: a code prediction
   key_cfg(key, c, B, 1);
   for (const void* p : {(const void*)lm_hidden, (const void*)code0, (const void*)codes,
-                        (const void*)logits, (const void*)ws, (const void*)w->final_norm})
+                        (const void*)logits, (const void*)ws, (const void*)w->final_norm,
+                        (const void*)trace})
     key_push(key, p);
   key.push_back((uint64_t)w->groups);
   key_matrix(key, w->input_proj);
@@ -617,5 +807,46 @@ extern "C" qg_status qg_code_predict(const qg_qwen3_config* cfg, const qg_code_p
     if (g >= 1) key_matrix(key, w->heads[g]);
   }
   key_layers(key, w->layers, c.layers);
-  return run_recorded(std::move(key), s, enqueue, "qg_code_predict");
+  return run_recorded(std::move(key), s, enqueue, what);
+}
+
+}  // namespace
+
+extern "C" qg_status qg_code_predict(const qg_qwen3_config* cfg, const qg_code_predictor_weights* w,
+                                     const float* lm_hidden, const int32_t* code0, int32_t* codes,
+                                     float* logits, int B, void* ws, size_t ws_bytes,
+                                     void* stream) {
+  return code_predict_impl(cfg, w, lm_hidden, code0, codes, logits, B, ws, ws_bytes, nullptr, 0,
+                           stream, "qg_code_predict");
+}
+
+extern "C" qg_status qg_code_predict_trace_layout(const qg_qwen3_config* cfg, int B, int groups,
+                                                  size_t out[4]) {
+  clear_error();
+  qg_status st = validate_cfg(cfg, B, 1);
+  if (st != QG_OK) return st;
+  QG_REQUIRE(out, QG_ERR_INVALID_ARGUMENT, "qg_code_predict_trace_layout: null out");
+  QG_REQUIRE(groups >= 2 && groups <= 64, QG_ERR_UNSUPPORTED_SHAPE,
+             "qg_code_predict_trace_layout: groups=%d must be in [2, 64]", groups);
+  const CpTrace T = cp_trace_layout(*cfg, B, groups);
+  out[0] = T.total;
+  out[1] = T.group;
+  out[2] = T.comb;
+  out[3] = T.slot;
+  return QG_OK;
+}
+
+extern "C" qg_status qg_code_predict_traced(const qg_qwen3_config* cfg,
+                                            const qg_code_predictor_weights* w,
+                                            const float* lm_hidden, const int32_t* code0,
+                                            int32_t* codes, float* logits, int B, void* ws,
+                                            size_t ws_bytes, void* trace, size_t trace_bytes,
+                                            void* stream) {
+  if (!trace) {
+    clear_error();
+    set_error("qg_code_predict_traced: trace is NULL");
+    return QG_ERR_INVALID_ARGUMENT;
+  }
+  return code_predict_impl(cfg, w, lm_hidden, code0, codes, logits, B, ws, ws_bytes, trace,
+                           trace_bytes, stream, "qg_code_predict_traced");
 }

@@ -37,16 +37,18 @@
 #include <mutex>
 
 #include "qg_internal.cuh"
+#include "tcgen05_util.cuh"
 
 namespace qg {
 namespace gq4 {
+
+using namespace tc;
 
 constexpr int kBM = 128;
 constexpr int kBK = 64;               // one 128-byte swizzle row of bf16
 constexpr int kProducers = 256;       // warps 0-7: W
 constexpr int kThreads = kProducers + 64;  // + warp 8 (MMA) + warp 9 (TMA for A)
 constexpr int kPrefetch = 3;          // W stages in flight in registers
-constexpr unsigned long long kWaitNs = 1000000000ull;
 
 // BN output columns and MT 128-row sub-tiles of A per CTA: the MT sub-tiles
 // share each dequantized W tile (MT MMAs per K step into MT * BN tensor-memory
@@ -60,63 +62,6 @@ struct Cfg {
   static constexpr int kSmem = 1024 + kStages * kStage + 1024;  // + align slack + barriers
   static constexpr int kTmemCols = MT * BN;
 };
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-      " selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ unsigned long long now_ns() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-// bounded wait; gives up early once another role has aborted
-__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = now_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (*abort) return false;
-    if (now_ns() - t0 > kWaitNs) return false;
-  }
-  return true;
-}
-
-// K-major, 128-byte swizzle shared-memory matrix descriptor: 8-row groups
-// 1024 bytes apart (SBO), leading offset 16 bytes, descriptor version 1.
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr) {
-  uint64_t d = 0;
-  d |= (uint64_t)((addr >> 4) & 0x3FFFu);
-  d |= (uint64_t)1u << 16;             // LBO = 16 B (encoded >> 4)
-  d |= (uint64_t)(1024u >> 4) << 32;   // SBO = 1024 B
-  d |= (uint64_t)1u << 46;             // version
-  d |= (uint64_t)2u << 61;             // SWIZZLE_128B
-  return d;
-}
-
-// instruction descriptor: bf16 x bf16 -> fp32, both K-major, M = 128
-template <int BN>
-__host__ __device__ constexpr uint32_t instr_desc() {
-  return (1u << 4)                 // D fp32
-         | (1u << 7)               // A bf16
-         | (1u << 10)              // B bf16
-         | ((uint32_t)(BN >> 3) << 17)
-         | ((uint32_t)(kBM >> 4) << 24);
-}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return (uint32_t)f32_to_bf16_bits(lo) | ((uint32_t)f32_to_bf16_bits(hi) << 16);
@@ -133,11 +78,7 @@ __global__ void a_to_bf16_kernel(const float* __restrict__ A, uint32_t* __restri
   }
 }
 
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
-               "r"(bytes)
-               : "memory");
-}
+
 
 // dequantize two Q4_0 blocks (raw: 36 bytes as 9 words; fp16 d then 16 code
 // bytes, twice) and store them as row r's 64 bf16 values of the stage. A
@@ -198,11 +139,27 @@ __device__ __forceinline__ void load_w_raw(const uint8_t* wrow, int kb, uint32_t
   }
 }
 
+// What the epilogue does with an accumulator value v of C[m][n]:
+// v + bias[n] (+ res[m][n]), then gelu_tanh when `gelu`, stored as fp32 or
+// bf16 (round to nearest even). C may alias res (each element is read and
+// written by the same thread).
+struct Epi {
+  const float* bias;  // [N] or null
+  const float* res;   // fp32 [M][N] or null
+  void* C;            // [M][N]
+  int c_bf16;
+  int gelu;
+};
+
+// GELU, tanh form (fuel-transformers `gelu_tanh`), in fp32 with CUDA's tanhf
+__device__ __forceinline__ float gelu_tanh_f(float x) {
+  return 0.5f * x * (1.0f + tanhf(0.7978845608028654f * (x + 0.044715f * x * x * x)));
+}
+
 template <int BN, int MT, bool W32>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_q4_0_tc_kernel(const __grid_constant__ CUtensorMap tmA, const uint8_t* __restrict__ blocks,
-                        const float* __restrict__ bias, float* __restrict__ C, int M, int N, int K,
-                        unsigned* __restrict__ err) {
+                        const Epi ep, int M, int N, int K, unsigned* __restrict__ err) {
   using G = Cfg<BN, MT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -392,18 +349,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int mt = c0 / BN, n = c0 % BN;
         const int m = m0 + mt * kBM + 32 * q + lane;
         if (m < M) {
-          float* crow = C + (size_t)m * N + n0 + n;
+          const size_t ci = (size_t)m * N + n0 + n;
 #pragma unroll
           for (int j = 0; j < 32; j += 4) {
-            float4 o = make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
-                                   __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
-            if (bias) {
-              o.x += bias[n0 + n + j];
-              o.y += bias[n0 + n + j + 1];
-              o.z += bias[n0 + n + j + 2];
-              o.w += bias[n0 + n + j + 3];
+            float o[4] = {__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
+                          __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3])};
+            if (ep.bias) {
+#pragma unroll
+              for (int e = 0; e < 4; ++e) o[e] += ep.bias[n0 + n + j + e];
             }
-            *reinterpret_cast<float4*>(crow + j) = o;
+            if (ep.res) {
+              const float4 r = *reinterpret_cast<const float4*>(ep.res + ci + j);
+              o[0] += r.x;
+              o[1] += r.y;
+              o[2] += r.z;
+              o[3] += r.w;
+            }
+            if (ep.gelu) {
+#pragma unroll
+              for (int e = 0; e < 4; ++e) o[e] = gelu_tanh_f(o[e]);
+            }
+            if (ep.c_bf16)
+              *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(ep.C) + ci + j) =
+                  make_uint2(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]));
+            else
+              *reinterpret_cast<float4*>(reinterpret_cast<float*>(ep.C) + ci + j) =
+                  make_float4(o[0], o[1], o[2], o[3]);
           }
         }
       }
@@ -445,40 +416,65 @@ static EncodeTiledFn encode_tiled() {
   return fn;
 }
 
-// A (bf16 [M][K], row stride K*2 bytes) in boxes of 64 columns x 128 rows,
-// 128-byte swizzle; rows past M read as zero
-static bool make_a_map(CUtensorMap* map, const uint16_t* Ab, int M, int K) {
+// A bf16 [rows][cols] row-major tensor (row stride cols * 2 bytes) in boxes
+// of 64 columns x box_rows rows, 128-byte swizzle; rows past the end read as
+// zero.
+bool make_bf16_map(CUtensorMap* map, const void* base, int rows, int cols, int box_rows) {
   EncodeTiledFn enc = encode_tiled();
   if (!enc) return false;
-  const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
-  const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-  const cuuint32_t box[2] = {(cuuint32_t)gq4::kBK, (cuuint32_t)gq4::kBM};
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(Ab), dims, strides,
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+static bool make_a_map(CUtensorMap* map, const uint16_t* Ab, int M, int K) {
+  return make_bf16_map(map, Ab, M, K, gq4::kBM);
+}
+
 template <int BN, int MT, bool W32>
-static cudaError_t gq4_launch(const CUtensorMap& tmA, const uint8_t* blocks, const float* bias,
-                              float* C, int M, int N, int K, unsigned* err, cudaStream_t st) {
+static cudaError_t gq4_launch(const CUtensorMap& tmA, const uint8_t* blocks, const gq4::Epi& ep,
+                              int M, int N, int K, unsigned* err, cudaStream_t st) {
   using G = gq4::Cfg<BN, MT>;
   ensure_smem((const void*)gq4::gemm_q4_0_tc_kernel<BN, MT, W32>, G::kSmem);
   dim3 grid(N / BN, (M + MT * gq4::kBM - 1) / (MT * gq4::kBM));
   return launch_pdl(gq4::gemm_q4_0_tc_kernel<BN, MT, W32>, grid, dim3(gq4::kThreads),
-                    (size_t)G::kSmem, st, false, tmA, blocks, bias, C, M, N, K, err);
+                    (size_t)G::kSmem, st, false, tmA, blocks, ep, M, N, K, err);
 }
 
 // tile choice: 256 columns when N allows; two A sub-tiles per CTA (W
 // dequantized once per 256 rows of A) while that still gives half the SMs a
 // tile
 template <int BN, bool W32>
-static cudaError_t gq4_launch_mt(const CUtensorMap& tmA, const uint8_t* blocks, const float* bias,
-                                 float* C, int M, int N, int K, unsigned* err, cudaStream_t st) {
+static cudaError_t gq4_launch_mt(const CUtensorMap& tmA, const uint8_t* blocks, const gq4::Epi& ep,
+                                 int M, int N, int K, unsigned* err, cudaStream_t st) {
   const long long tiles2 = (long long)(N / BN) * ((M + 255) / 256);
   if (2 * tiles2 >= num_sms())
-    return gq4_launch<BN, 2, W32>(tmA, blocks, bias, C, M, N, K, err, st);
-  return gq4_launch<BN, 1, W32>(tmA, blocks, bias, C, M, N, K, err, st);
+    return gq4_launch<BN, 2, W32>(tmA, blocks, ep, M, N, K, err, st);
+  return gq4_launch<BN, 1, W32>(tmA, blocks, ep, M, N, K, err, st);
+}
+
+// The GEMM on a bf16 A already in device memory (`Ab`, [M][K]); `err` is the
+// workspace error word.
+static qg_status gq4_run(const uint8_t* blocks, const uint16_t* Ab, const gq4::Epi& ep, int M,
+                         int N, int K, unsigned* err, cudaStream_t s, const char* what) {
+  CUtensorMap tmA;
+  if (!make_a_map(&tmA, Ab, M, K)) {
+    set_error("%s: could not encode the TMA descriptor of A", what);
+    return QG_ERR_CUDA;
+  }
+  const bool w32 = aligned(blocks, 4);
+  if (N % 256 == 0) {
+    if (w32) gq4_launch_mt<256, true>(tmA, blocks, ep, M, N, K, err, s);
+    else gq4_launch_mt<256, false>(tmA, blocks, ep, M, N, K, err, s);
+  } else {
+    if (w32) gq4_launch_mt<128, true>(tmA, blocks, ep, M, N, K, err, s);
+    else gq4_launch_mt<128, false>(tmA, blocks, ep, M, N, K, err, s);
+  }
+  return check_launch(what);
 }
 
 }  // namespace qg
@@ -491,61 +487,78 @@ extern "C" size_t qg_gemm_q4_0_workspace_size(int M, int N, int K) {
   return a_bytes(M, K) + 256;
 }
 
+static qg_status gemm_q4_0_checked(const uint8_t* blocks, const void* A, qg_dtype a_dtype,
+                                   const float* bias, const float* residual, void* C,
+                                   qg_dtype c_dtype, int gelu, int M, int N, int K, void* ws,
+                                   size_t ws_bytes, void* stream, const char* what) {
+  clear_error();
+  QG_REQUIRE(M >= 0 && N >= 0 && K >= 0, QG_ERR_UNSUPPORTED_SHAPE,
+             "%s: M=%d N=%d K=%d must be >= 0", what, M, N, K);
+  QG_REQUIRE(K % 64 == 0 && K > 0, QG_ERR_UNSUPPORTED_SHAPE,
+             "%s: K=%d must be a positive multiple of 64", what, K);
+  QG_REQUIRE(N % 128 == 0 && N > 0, QG_ERR_UNSUPPORTED_SHAPE,
+             "%s: N=%d must be a positive multiple of 128", what, N);
+  QG_REQUIRE((long long)M * K < (1LL << 40) && (long long)M * N < (1LL << 40),
+             QG_ERR_UNSUPPORTED_SHAPE, "%s: M=%d too large", what, M);
+  QG_REQUIRE(M < (1 << 24) / 128 * 128, QG_ERR_UNSUPPORTED_SHAPE, "%s: M=%d too large", what, M);
+  QG_REQUIRE(a_dtype == QG_F32 || a_dtype == QG_BF16, QG_ERR_INVALID_ARGUMENT,
+             "%s: a_dtype=%d", what, (int)a_dtype);
+  QG_REQUIRE(c_dtype == QG_F32 || c_dtype == QG_BF16, QG_ERR_INVALID_ARGUMENT,
+             "%s: c_dtype=%d", what, (int)c_dtype);
+  QG_REQUIRE(!residual || c_dtype == QG_F32, QG_ERR_INVALID_ARGUMENT,
+             "%s: a residual needs an fp32 C", what);
+  if (M == 0) return QG_OK;
+  QG_REQUIRE(blocks && A && C, QG_ERR_INVALID_ARGUMENT, "%s: null blocks, A or C", what);
+  QG_REQUIRE(aligned(A, 16) && aligned(C, 16) && aligned(residual, 16), QG_ERR_MISALIGNED,
+             "%s: A, C and residual must be 16-byte aligned", what);
+  QG_REQUIRE(aligned(blocks, 2), QG_ERR_MISALIGNED, "%s: blocks must be 2-byte aligned", what);
+  QG_REQUIRE(!bias || aligned(bias, 4), QG_ERR_MISALIGNED, "%s: bias misaligned", what);
+  const size_t need = a_dtype == QG_F32 ? qg_gemm_q4_0_workspace_size(M, N, K) : 256;
+  QG_REQUIRE(ws && ws_bytes >= need, QG_ERR_WORKSPACE_TOO_SMALL,
+             "%s: workspace of %zu bytes given, %zu needed", what, ws_bytes, need);
+  QG_REQUIRE(aligned(ws, 256), QG_ERR_MISALIGNED, "%s: ws not 256-byte aligned", what);
+  cudaStream_t s = (cudaStream_t)stream;
+  const uint16_t* Ab = reinterpret_cast<const uint16_t*>(A);
+  unsigned* err = reinterpret_cast<unsigned*>(ws);
+  if (a_dtype == QG_F32) {
+    uint16_t* Aw = reinterpret_cast<uint16_t*>(ws);
+    err = reinterpret_cast<unsigned*>(reinterpret_cast<uint8_t*>(ws) + a_bytes(M, K));
+    const size_t n4 = (size_t)M * K / 4;
+    const int grid = (int)std::min<size_t>((n4 + 255) / 256, (size_t)num_sms() * 8);
+    launch_pdl(gq4::a_to_bf16_kernel, dim3(grid), dim3(256), 0, s, false,
+               reinterpret_cast<const float*>(A), reinterpret_cast<uint32_t*>(Aw), n4);
+    Ab = Aw;
+  }
+  cudaMemsetAsync(err, 0, sizeof(unsigned), s);
+  gq4::Epi ep = {bias, residual, C, c_dtype == QG_BF16 ? 1 : 0, gelu ? 1 : 0};
+  return gq4_run(blocks, Ab, ep, M, N, K, err, s, what);
+}
+
 extern "C" qg_status qg_gemm_q4_0(const uint8_t* blocks, const float* A, const float* bias,
                                   float* C, int M, int N, int K, void* ws, size_t ws_bytes,
                                   void* stream) {
-  clear_error();
-  QG_REQUIRE(M >= 0 && N >= 0 && K >= 0, QG_ERR_UNSUPPORTED_SHAPE,
-             "qg_gemm_q4_0: M=%d N=%d K=%d must be >= 0", M, N, K);
-  QG_REQUIRE(K % 64 == 0 && K > 0, QG_ERR_UNSUPPORTED_SHAPE,
-             "qg_gemm_q4_0: K=%d must be a positive multiple of 64", K);
-  QG_REQUIRE(N % 128 == 0 && N > 0, QG_ERR_UNSUPPORTED_SHAPE,
-             "qg_gemm_q4_0: N=%d must be a positive multiple of 128", N);
-  QG_REQUIRE((long long)M * K < (1LL << 40) && (long long)M * N < (1LL << 40),
-             QG_ERR_UNSUPPORTED_SHAPE, "qg_gemm_q4_0: M=%d too large", M);
-  QG_REQUIRE(M < (1 << 24) / 128 * 128, QG_ERR_UNSUPPORTED_SHAPE, "qg_gemm_q4_0: M=%d too large",
-             M);
-  if (M == 0) return QG_OK;
-  QG_REQUIRE(blocks && A && C, QG_ERR_INVALID_ARGUMENT, "qg_gemm_q4_0: null blocks, A or C");
-  QG_REQUIRE(aligned(A, 16) && aligned(C, 16), QG_ERR_MISALIGNED,
-             "qg_gemm_q4_0: A and C must be 16-byte aligned");
-  QG_REQUIRE(aligned(blocks, 2), QG_ERR_MISALIGNED, "qg_gemm_q4_0: blocks must be 2-byte aligned");
-  QG_REQUIRE(!bias || aligned(bias, 4), QG_ERR_MISALIGNED, "qg_gemm_q4_0: bias misaligned");
-  const size_t need = qg_gemm_q4_0_workspace_size(M, N, K);
-  QG_REQUIRE(ws && ws_bytes >= need, QG_ERR_WORKSPACE_TOO_SMALL,
-             "qg_gemm_q4_0: workspace of %zu bytes given, %zu needed", ws_bytes, need);
-  QG_REQUIRE(aligned(ws, 256), QG_ERR_MISALIGNED, "qg_gemm_q4_0: ws not 256-byte aligned");
-  cudaStream_t s = (cudaStream_t)stream;
-  uint16_t* Ab = reinterpret_cast<uint16_t*>(ws);
-  unsigned* err = reinterpret_cast<unsigned*>(reinterpret_cast<uint8_t*>(ws) + a_bytes(M, K));
-  cudaMemsetAsync(err, 0, sizeof(unsigned), s);
-  const size_t n4 = (size_t)M * K / 4;
-  const int grid = (int)std::min<size_t>((n4 + 255) / 256, (size_t)num_sms() * 8);
-  launch_pdl(gq4::a_to_bf16_kernel, dim3(grid), dim3(256), 0, s, false, A,
-             reinterpret_cast<uint32_t*>(Ab), n4);
-  CUtensorMap tmA;
-  if (!make_a_map(&tmA, Ab, M, K)) {
-    set_error("qg_gemm_q4_0: could not encode the TMA descriptor of A");
-    return QG_ERR_CUDA;
-  }
-  const bool w32 = aligned(blocks, 4);
-  if (N % 256 == 0) {
-    if (w32) gq4_launch_mt<256, true>(tmA, blocks, bias, C, M, N, K, err, s);
-    else gq4_launch_mt<256, false>(tmA, blocks, bias, C, M, N, K, err, s);
-  } else {
-    if (w32) gq4_launch_mt<128, true>(tmA, blocks, bias, C, M, N, K, err, s);
-    else gq4_launch_mt<128, false>(tmA, blocks, bias, C, M, N, K, err, s);
-  }
-  return check_launch("qg_gemm_q4_0");
+  return gemm_q4_0_checked(blocks, A, QG_F32, bias, nullptr, C, QG_F32, 0, M, N, K, ws, ws_bytes,
+                           stream, "qg_gemm_q4_0");
+}
+
+extern "C" qg_status qg_gemm_q4_0_ex(const uint8_t* blocks, const void* A, qg_dtype a_dtype,
+                                     const float* bias, const float* residual, void* C,
+                                     qg_dtype c_dtype, int gelu, int M, int N, int K, void* ws,
+                                     size_t ws_bytes, void* stream) {
+  return gemm_q4_0_checked(blocks, A, a_dtype, bias, residual, C, c_dtype, gelu, M, N, K, ws,
+                           ws_bytes, stream, "qg_gemm_q4_0_ex");
 }
 
 extern "C" qg_status qg_gemm_q4_0_error(int M, int K, const void* ws, unsigned* code,
                                         void* stream) {
   clear_error();
-  QG_REQUIRE(ws && code && M > 0 && K > 0, QG_ERR_INVALID_ARGUMENT,
-             "qg_gemm_q4_0_error: null ws or code, or empty shape");
+  QG_REQUIRE(ws && code && M >= 0 && K >= 0, QG_ERR_INVALID_ARGUMENT,
+             "qg_gemm_q4_0_error: null ws or code, or negative shape");
   cudaStream_t s = (cudaStream_t)stream;
-  cudaError_t e = cudaMemcpyAsync(code, reinterpret_cast<const uint8_t*>(ws) + a_bytes(M, K),
+  // after an fp32-A call the word follows A's bf16 copy; after a bf16-A
+  // call (M = K = 0 here) it heads the workspace
+  const size_t off = (M > 0 && K > 0) ? a_bytes(M, K) : 0;
+  cudaError_t e = cudaMemcpyAsync(code, reinterpret_cast<const uint8_t*>(ws) + off,
                                   sizeof(unsigned), cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) {

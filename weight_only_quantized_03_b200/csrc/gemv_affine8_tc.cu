@@ -52,12 +52,15 @@ template <int NT, int W>
 __global__ void __launch_bounds__(W * 32, NT == 1 ? 512 / (W * 32) : 1)
     gemv_tc_kernel(const __grid_constant__ Params P) {
   extern __shared__ __align__(16) uint8_t smem[];
+  tl_entry(P.tl);
   // the next kernel may be scheduled as soon as the weight loads are out (its
   // own wait still covers all of this one)
-  gemv_tc_body<NT, W>(P, smem, [] {
+  gemv_tc_body<NT, W>(P, smem, [&] {
     pdl_trigger();
     pdl_wait();
+    tl_wait(P.tl);
   });
+  tl_exit(P.tl);
 }
 
 }  // namespace gtc
@@ -83,10 +86,12 @@ static cudaError_t gtc_launch_nt(const gtc::Params& P, dim3 grid, cudaStream_t s
 }
 
 static cudaError_t gtc_launch(const GemvSeg* segs, int nseg, gtc::Params& P, int K, int B,
-                              cudaStream_t st, bool pdl) {
+                              cudaStream_t st, bool pdl, const Prefetch* pf) {
   P.nseg = nseg;
   P.K = K;
   P.B = B;
+  if (pf) P.pf = *pf;
+  P.tl = tl_take(0);
   int blk = 0;
   for (int i = 0; i < nseg; ++i) {
     P.seg[i] = gtc::Seg{reinterpret_cast<const uint8_t*>(segs[i].w), segs[i].s, segs[i].b, segs[i].y,
@@ -95,49 +100,58 @@ static cudaError_t gtc_launch(const GemvSeg* segs, int nseg, gtc::Params& P, int
   }
   P.nblocks = blk;
   if (blk == 0) return cudaSuccess;
-  // 16 warps with one batch tile, 8 with two (measured: 16 is faster also
-  // for the small matrices of a decode step); then split each block's
-  // columns over S warps while slots stay idle
-  // batch tiles of 8 rows along gridDim.y past B = 8: the tiles stream the
-  // same weights at about the same time, so all but the first mostly hit L2
+  // One batch tile (B <= 4): 16 warps for matrices that stream (more
+  // 16-row blocks than warp slots at 8 warps a CTA), 8 warps for the
+  // matrices of a decode layer, whose weights then all go out before the
+  // wait and whose CTAs leave room on each SM for the next kernel's CTA.
+  // Two batch tiles: 8 warps (about 255 registers a thread). Batch tiles of
+  // 8 rows along gridDim.y past B = 8: the tiles stream the same weights at
+  // about the same time, so all but the first mostly hit L2.
   const int NT = B > 4 ? 2 : 1;
   const int sms = num_sms();
-  const int W = NT == 1 ? 16 : 8;
+  const bool stream16 = NT == 1 && (long long)blk > 8LL * sms;
+  const int W = stream16 ? 16 : 8;
   P.S = gtc_split(blk, K, W, sms);
   const dim3 grid(std::min(sms, blk), (B + 4 * NT - 1) / (4 * NT));
   if (NT == 2) return gtc_launch_nt<2, 8>(P, grid, st, pdl);
-  return gtc_launch_nt<1, 16>(P, grid, st, pdl);
+  if (W == 16) return gtc_launch_nt<1, 16>(P, grid, st, pdl);
+  return gtc_launch_nt<1, 8>(P, grid, st, pdl);
 }
 
 cudaError_t gemv_tc_launch(const GemvSeg* segs, int nseg, const void* x, int K, int B,
                            cudaStream_t st, bool pdl) {
+  return gemv_tc_launch_pf(segs, nseg, x, K, B, st, pdl, nullptr);
+}
+
+cudaError_t gemv_tc_launch_pf(const GemvSeg* segs, int nseg, const void* x, int K, int B,
+                              cudaStream_t st, bool pdl, const Prefetch* pf) {
   gtc::Params P = {};
   P.xmode = gtc::kXBf16;
   P.x = reinterpret_cast<const uint16_t*>(x);
-  return gtc_launch(segs, nseg, P, K, B, st, pdl);
+  return gtc_launch(segs, nseg, P, K, B, st, pdl, pf);
 }
 
 cudaError_t gemv_tc_launch_rmsnorm(const GemvSeg* segs, int nseg, const float* x,
                                    const uint16_t* norm_w, float eps, int K, int B,
-                                   cudaStream_t st, bool pdl, uint16_t* xout) {
+                                   cudaStream_t st, bool pdl, uint16_t* xout, const Prefetch* pf) {
   gtc::Params P = {};
   P.xmode = gtc::kXRmsNorm;
   P.xout = xout;
   P.xa = x;
   P.nw = norm_w;
   P.eps = eps;
-  return gtc_launch(segs, nseg, P, K, B, st, pdl);
+  return gtc_launch(segs, nseg, P, K, B, st, pdl, pf);
 }
 
 cudaError_t gemv_tc_launch_silu_mul(const GemvSeg* segs, int nseg, const float* gate,
                                     const float* up, int K, int B, cudaStream_t st, bool pdl,
-                                    uint16_t* xout) {
+                                    uint16_t* xout, const Prefetch* pf) {
   gtc::Params P = {};
   P.xmode = gtc::kXSiluMul;
   P.xout = xout;
   P.xa = gate;
   P.xb = up;
-  return gtc_launch(segs, nseg, P, K, B, st, pdl);
+  return gtc_launch(segs, nseg, P, K, B, st, pdl, pf);
 }
 
 }  // namespace qg

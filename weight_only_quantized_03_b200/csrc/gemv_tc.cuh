@@ -42,6 +42,8 @@ struct Params {
   const uint16_t* nw;  // kXRmsNorm weight, bf16 [K]
   float eps;
   uint16_t* xout;      // optional: CTA 0 records the formed bf16 input [B][K]
+  Prefetch pf;         // L2 prefetch work for a later kernel (pf.n == 0, pf.kv.kc null: none)
+  TlRec* tl;           // timeline record of this launch, or null
 };
 
 __device__ __forceinline__ void ld_w8(const uint8_t* p, uint64_t pol, uint32_t* r) {
@@ -155,10 +157,14 @@ __device__ __forceinline__ void gemv_tc_body(const Params& P, uint8_t* smem, Wai
   // batch tile of this CTA: rows [b0, b0 + Bt) of the launch's P.B
   const int b0 = blockIdx.y * 4 * NT, Bt = min(4 * NT, P.B - b0);
   const int xs = K + 8;  // fp16 row stride of x (pad: batch rows on other banks)
-  float* red = reinterpret_cast<float*>(smem);                      // [4 NT][kWarps]
-  float* part = red + 4 * NT * kWarps;                               // [2][kWarps][32][2 NT]
+  float* red = reinterpret_cast<float*>(smem);                      // [4 NT + 1][kWarps]
+  float* part = red + (4 * NT + 1) * kWarps;                         // [2][kWarps][32][2 NT]
   float* gsum = part + 2 * kWarps * 32 * 2 * NT;                    // [4 NT][Kg]
   uint16_t* xh = reinterpret_cast<uint16_t*>(gsum + 4 * NT * Kg);   // [4 NT][xs]
+
+  // L2 prefetch for a later kernel of the chain (one thread per CTA)
+  if (tid == 0 && blockIdx.y == 0 && (P.pf.n > 0 || P.pf.kv.kc))
+    issue_prefetch(P.pf, blockIdx.x, gridDim.x);
 
   // team = S warps sharing each block's columns; team slots are numbered
   // across CTAs first so that few blocks spread over many SMs
@@ -166,7 +172,7 @@ __device__ __forceinline__ void gemv_tc_body(const Params& P, uint8_t* smem, Wai
   const int T = gridDim.x * tpc, team = tl * gridDim.x + blockIdx.x;
   const int sc_lo = pw * nsc / S, sc_hi = (pw + 1) * nsc / S, nscw = sc_hi - sc_lo;
   const int nblk = team < P.nblocks ? (P.nblocks - 1 - team) / T + 1 : 0;
-  const int total = nblk * nscw;
+  const int total = nscw > 0 ? nblk * nscw : 0;
 
   uint64_t pol;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
@@ -184,23 +190,92 @@ __device__ __forceinline__ void gemv_tc_body(const Params& P, uint8_t* smem, Wai
     for (int p = 0; p < 4; ++p) load_chunk(lr, K, lsc, p, pol, wb[p]);
   }
 
+  // The input is formed in items of 128 columns of one batch row (lane l
+  // holds columns 4l .. 4l + 3; lanes 0-15 cover one 64-column group, lanes
+  // 16-31 the next); warp w forms items w, w + W, ... The first kItems of a
+  // warp stay in registers from one load round to the forming pass (later
+  // ones, for large B * K, are loaded again).
+  constexpr int kItems = 3;
+  const int Kp = K / 128, nitems = Bt * Kp;
+  const int my_items = warp < nitems ? (nitems - 1 - warp) / kWarps + 1 : 0;
+  auto nw_of = [&](int c) {  // (the norm weight may be only 2-byte aligned)
+    return make_uint2((uint32_t)P.nw[c] | ((uint32_t)P.nw[c + 1] << 16),
+                      (uint32_t)P.nw[c + 2] | ((uint32_t)P.nw[c + 3] << 16));
+  };
+  uint2 nwr[kItems];  // RMSNorm weights of the kept items (bf16 x 4)
+#pragma unroll
+  for (int j = 0; j < kItems; ++j) {
+    nwr[j] = make_uint2(0u, 0u);
+    if (P.xmode == kXRmsNorm && j < my_items) nwr[j] = nw_of(((warp + j * kWarps) % Kp) * 128 + 4 * lane);
+  }
+
   wait();  // x (and residuals) are written upstream
   // what the previous kernels wrote (x, the residual) is read through L2
-  // (ld.global.cg): each value is read once per CTA, so L1 would not help
-  // 1) RMSNorm statistics per batch row (fixed summation order)
+  // (ld.global.cg): each value is read once per CTA, so L1 would not help.
+  // One round of loads: the kept input items and this warp's first residual
+  // values, all in flight together. In SiLU mode an item holds silu(gate) *
+  // up, not yet rounded.
+  auto load_item = [&](int i) -> float4 {
+    const int b = i / Kp, c = (i - b * Kp) * 128 + 4 * lane;
+    const size_t o = (size_t)(b0 + b) * K + c;
+    if (P.xmode == kXBf16) {
+      const uint2 w2 = __ldcg(reinterpret_cast<const uint2*>(P.x + o));
+      return make_float4(bf16_lo(w2.x), bf16_hi(w2.x), bf16_lo(w2.y), bf16_hi(w2.y));
+    }
+    float4 va = __ldcg(reinterpret_cast<const float4*>(P.xa + o));
+    if (P.xmode == kXSiluMul) {
+      const float4 u = __ldcg(reinterpret_cast<const float4*>(P.xb + o));
+      va = make_float4(va.x / (1.0f + expf(-va.x)) * u.x, va.y / (1.0f + expf(-va.y)) * u.y,
+                       va.z / (1.0f + expf(-va.z)) * u.z, va.w / (1.0f + expf(-va.w)) * u.w);
+    }
+    return va;
+  };
+  float4 xv[kItems];
+#pragma unroll
+  for (int j = 0; j < kItems; ++j)
+    xv[j] = j < my_items ? load_item(warp + j * kWarps) : make_float4(0.f, 0.f, 0.f, 0.f);
+  // residual of the first block this warp stores (lane (g, t): rows g, g + 8
+  // of batch row 4 nt + t)
+  float resv[NT][2];
+  const bool stores = total > 0 && (S == 1 || pw == 0);
+  {
+    const Seg& Sg = P.seg[seg_of(P, min(team, P.nblocks - 1))];
+    const int row0 = (team - Sg.blk0) * kRB;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int b = 4 * nt + t, r = row0 + g + 8 * h;
+        resv[nt][h] = 0.f;
+        if (stores && Sg.res && b < Bt && r < Sg.N)
+          resv[nt][h] = __ldcg(Sg.res + (size_t)(b0 + b) * Sg.N + r);
+      }
+    }
+  }
+
+  // 1) RMSNorm statistics per batch row: per lane over its items, then the
+  // warp, then the warps in order (deterministic)
   float inv[4 * NT];
 #pragma unroll
   for (int b = 0; b < 4 * NT; ++b) inv[b] = 0.f;
   if (P.xmode == kXRmsNorm) {
+    float ssb[4 * NT];
+#pragma unroll
+    for (int b = 0; b < 4 * NT; ++b) ssb[b] = 0.f;
+    auto stat = [&](int i, const float4& v) {
+      const int b = i / Kp;
+      const float ss = fmaf(v.w, v.w, fmaf(v.z, v.z, fmaf(v.y, v.y, v.x * v.x)));
+#pragma unroll
+      for (int bb = 0; bb < 4 * NT; ++bb)
+        if (b == bb) ssb[bb] += ss;
+    };
+#pragma unroll
+    for (int j = 0; j < kItems; ++j)
+      if (j < my_items) stat(warp + j * kWarps, xv[j]);
+    for (int j = kItems; j < my_items; ++j) stat(warp + j * kWarps, load_item(warp + j * kWarps));
 #pragma unroll
     for (int b = 0; b < 4 * NT; ++b) {
-      if (b >= Bt) break;
-      float ss = 0.f;
-      for (int c = tid; c < K; c += kThreads) {
-        const float v = __ldcg(P.xa + (size_t)(b0 + b) * K + c);
-        ss = fmaf(v, v, ss);
-      }
-      ss = warp_sum(ss);
+      const float ss = warp_sum(ssb[b]);
       if (lane == 0) red[b * kWarps + warp] = ss;
     }
     __syncthreads();
@@ -211,45 +286,55 @@ __device__ __forceinline__ void gemv_tc_body(const Params& P, uint8_t* smem, Wai
       for (int w = 0; w < kWarps; ++w) ss += red[b * kWarps + w];
       inv[b] = 1.0f / sqrtf(ss / (float)K + P.eps);
     }
-    __syncthreads();
   }
-  // 2) one warp per 64-column group: the input values, rounded to bf16, go
-  // to xh as fp16 and the group's fp16 sum to gsum. fp16 holds them exactly
-  // unless max|x| >= 2^15, checked after the pass; then (rarely) the pass is
-  // redone on x * 2^-e. Batch rows past B are never read by a live B lane.
+  // 2) the input values rounded to bf16 where the separate kernels round
+  // them go to xh as fp16 and each 64-column group's fp16 sum to gsum. fp16
+  // holds them exactly unless max|x| >= 2^15, checked after the pass; then
+  // (rarely) the pass is redone on x * 2^-e. Batch rows past B are never
+  // read by a live B lane.
+  auto form_item = [&](int i, const float4& va, const uint2& nw2, float down) -> float {
+    const int b = i / Kp, c = (i - b * Kp) * 128 + 4 * lane;
+    float v[4] = {va.x, va.y, va.z, va.w};
+    if (P.xmode == kXRmsNorm) {
+      float ib = inv[0];
+#pragma unroll
+      for (int jb = 1; jb < 4 * NT; ++jb)
+        if (b == jb) ib = inv[jb];
+      const float wv[4] = {bf16_lo(nw2.x), bf16_hi(nw2.x), bf16_lo(nw2.y), bf16_hi(nw2.y)};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) v[e] = v[e] * ib * wv[e];
+    }
+    float m = 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      v[e] = bf16_bits_to_f32(f32_to_bf16_bits(v[e]));  // no-op for bf16 input
+      m = fmaxf(m, fabsf(v[e]));
+    }
+    const size_t o = (size_t)(b0 + b) * K + c;
+    if (P.xout && blockIdx.x == 0 && down == 1.0f)
+      *reinterpret_cast<uint2*>(P.xout + o) =
+          make_uint2((uint32_t)f32_to_bf16_bits(v[0]) | ((uint32_t)f32_to_bf16_bits(v[1]) << 16),
+                     (uint32_t)f32_to_bf16_bits(v[2]) | ((uint32_t)f32_to_bf16_bits(v[3]) << 16));
+    const __half2 h01 = __floats2half2_rn(v[0] * down, v[1] * down);
+    const __half2 h23 = __floats2half2_rn(v[2] * down, v[3] * down);
+    *reinterpret_cast<uint2*>(xh + b * xs + c) =
+        make_uint2(*reinterpret_cast<const uint32_t*>(&h01), *reinterpret_cast<const uint32_t*>(&h23));
+    // the 64-column group's sum over its 16 lanes (fixed order)
+    float sum = (__low2float(h01) + __high2float(h01)) + (__low2float(h23) + __high2float(h23));
+#pragma unroll
+    for (int off = 8; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    if ((lane & 15) == 0) gsum[b * Kg + c / 64] = sum;
+    return m;
+  };
   auto form = [&](float down) -> float {
     float mloc = 0.f;
-    for (int i = warp; i < Bt * Kg; i += kWarps) {
-      const int b = i / Kg, c = (i - b * Kg) * 64 + 2 * lane;
-      const size_t o = (size_t)(b0 + b) * K + c;
-      float v0, v1;
-      if (P.xmode == kXBf16) {
-        const uint32_t w2 = __ldcg(reinterpret_cast<const unsigned int*>(P.x + o));
-        v0 = bf16_lo(w2);
-        v1 = bf16_hi(w2);
-      } else if (P.xmode == kXRmsNorm) {
-        float ib = inv[0];
 #pragma unroll
-        for (int j = 1; j < 4 * NT; ++j)
-          if (b == j) ib = inv[j];
-        const float2 xv = __ldcg(reinterpret_cast<const float2*>(P.xa + o));
-        // (the norm weight may be only 2-byte aligned)
-        v0 = bf16_bits_to_f32(f32_to_bf16_bits(xv.x * ib * bf16_bits_to_f32(P.nw[c])));
-        v1 = bf16_bits_to_f32(f32_to_bf16_bits(xv.y * ib * bf16_bits_to_f32(P.nw[c + 1])));
-      } else {
-        const float2 z = __ldcg(reinterpret_cast<const float2*>(P.xa + o));
-        const float2 u = __ldcg(reinterpret_cast<const float2*>(P.xb + o));
-        v0 = bf16_bits_to_f32(f32_to_bf16_bits(z.x / (1.0f + expf(-z.x)) * u.x));
-        v1 = bf16_bits_to_f32(f32_to_bf16_bits(z.y / (1.0f + expf(-z.y)) * u.y));
-      }
-      mloc = fmaxf(mloc, fmaxf(fabsf(v0), fabsf(v1)));
-      if (P.xout && blockIdx.x == 0 && down == 1.0f)
-        *reinterpret_cast<uint32_t*>(P.xout + o) =
-            (uint32_t)f32_to_bf16_bits(v0) | ((uint32_t)f32_to_bf16_bits(v1) << 16);
-      const __half2 h2 = __floats2half2_rn(v0 * down, v1 * down);
-      *reinterpret_cast<__half2*>(xh + b * xs + c) = h2;
-      const float sum = warp_sum(__low2float(h2) + __high2float(h2));
-      if (lane == 0) gsum[i] = sum;
+    for (int j = 0; j < kItems; ++j)
+      if (j < my_items) mloc = fmaxf(mloc, form_item(warp + j * kWarps, xv[j], nwr[j], down));
+    for (int j = kItems; j < my_items; ++j) {
+      const int i = warp + j * kWarps;
+      const uint2 nw2 = P.xmode == kXRmsNorm ? nw_of((i % Kp) * 128 + 4 * lane) : make_uint2(0u, 0u);
+      mloc = fmaxf(mloc, form_item(i, load_item(i), nw2, down));
     }
     return mloc;
   };
@@ -257,18 +342,19 @@ __device__ __forceinline__ void gemv_tc_body(const Params& P, uint8_t* smem, Wai
   for (int i = Bt * Kg + tid; i < 4 * NT * Kg; i += kThreads) gsum[i] = 0.f;
   // 3) max|x| over the CTA; prescale 2^-e so that max|x| * 2^-e < 2^15
   mx = warp_max(mx);
-  if (lane == 0) red[warp] = mx;
+  float* redm = red + 4 * NT * kWarps;
+  if (lane == 0) redm[warp] = mx;
   __syncthreads();
   mx = 0.f;
 #pragma unroll
-  for (int w = 0; w < kWarps; ++w) mx = fmaxf(mx, red[w]);
+  for (int w = 0; w < kWarps; ++w) mx = fmaxf(mx, redm[w]);
   int e = 0;  // NaN or inf in x propagate to y without a prescale
   if (mx >= 32768.f && mx <= 3.0e38f) e = (int)ceilf(log2f(mx / 16384.f));
   const float up = exp2f((float)e);
   if (e != 0) {  // uniform over the CTA
     form(exp2f((float)-e));
+    __syncthreads();
   }
-  __syncthreads();
 
   // B-operand lanes: column n = g = 2 b + h, live on the k-slots of group h
   bool xl[NT];
@@ -371,7 +457,7 @@ __device__ __forceinline__ void gemv_tc_body(const Params& P, uint8_t* smem, Wai
           if (b < Bt && r < Sg.N) {
             const size_t o = (size_t)(b0 + b) * Sg.N + r;
             float v = acc[nt][h] * up;
-            if (Sg.res) v += __ldcg(Sg.res + o);
+            if (Sg.res) v += nb == 0 ? resv[nt][h] : __ldcg(Sg.res + o);
             if (Sg.y_bf16)
               reinterpret_cast<uint16_t*>(Sg.y)[o] = f32_to_bf16_bits(v);
             else
@@ -392,16 +478,19 @@ __device__ __forceinline__ void gemv_tc_body(const Params& P, uint8_t* smem, Wai
 
 // dynamic shared memory of gemv_tc_body
 inline size_t gtc_smem(int K, int NT, int W) {
-  return (size_t)4 * NT * W * 4 + (size_t)2 * W * 32 * 2 * NT * 4 +
+  return (size_t)(4 * NT + 1) * W * 4 + (size_t)2 * W * 32 * 2 * NT * 4 +
          (size_t)4 * NT * (K / 64) * 4 + (size_t)4 * NT * (K + 8) * 2;
 }
 
-// columns of each 16-row block are split over S warps (1, 2, 4, ... < W)
-// while warp slots stay idle
+// Columns of each 16-row block are split over S warps (1, 2, 4, ... <= W,
+// at most one 512-column super-chunk of work per warp beyond the first
+// split) while the launch still has idle warp slots: a matrix of a decode
+// layer then has all its weights in flight before the kernel waits for its
+// input.
 __host__ __device__ inline int gtc_split(int nblocks, int K, int W, int sms) {
   const int nsc = K / gtc::kSC;
   int S = 1;
-  while (S < W && 2 * S <= nsc && (long long)nblocks * S < (long long)sms * W) S *= 2;
+  while (S < W && S < nsc && (long long)nblocks * 2 * S <= (long long)sms * W) S *= 2;
   return S;
 }
 

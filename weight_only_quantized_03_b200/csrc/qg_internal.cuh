@@ -67,6 +67,105 @@ __device__ __forceinline__ void pdl_trigger() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// --------------------------------------------------------- L2 prefetch --
+
+// Work a kernel of the decode step hands to L2 at entry for a kernel that
+// runs later in the chain: byte ranges (packed weights, their scales and
+// biases) and, optionally, the cached K/V rows [0, position) of every
+// sequence of one layer. Prefetches are hints: they move no data the kernel
+// reads and complete on their own.
+constexpr int kMaxPf = 12;
+struct PfRange {
+  const void* p;
+  unsigned long long bytes;
+};
+struct KvPf {
+  const uint16_t* kc;  // one layer's caches [B][Hkv][cap][D], or null for none
+  const uint16_t* vc;
+  const int32_t* pos;  // [B]: rows [0, pos[b]) of sequence b are prefetched
+  int B, Hkv, cap, D;
+};
+struct Prefetch {
+  PfRange r[kMaxPf];
+  int n;
+  KvPf kv;
+};
+
+// Share `part` of `parts` of the 16-byte-aligned interior of [p, p + bytes)
+// (the unaligned ends, under 16 bytes each, are left out so that no byte
+// outside the range is touched), in pieces of at most 32 KB.
+__device__ __forceinline__ void l2_prefetch_range(const void* p, unsigned long long bytes,
+                                                  unsigned part, unsigned parts) {
+  const unsigned long long a0 = ((unsigned long long)(uintptr_t)p + 15ull) & ~15ull;
+  const unsigned long long a1 = ((unsigned long long)(uintptr_t)p + bytes) & ~15ull;
+  if (a1 <= a0) return;
+  const unsigned long long per = ((a1 - a0 + parts - 1) / parts + 15ull) & ~15ull;
+  unsigned long long lo = a0 + (unsigned long long)part * per;
+  const unsigned long long hi = lo + per < a1 ? lo + per : a1;
+  for (; lo < hi; lo += 32768ull) {
+    const unsigned sz = (unsigned)(hi - lo < 32768ull ? hi - lo : 32768ull);
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(lo), "r"(sz) : "memory");
+  }
+}
+
+// Issued by one thread of each CTA (part = its CTA index among `parts`).
+// The positions are inputs of the step, final before its first kernel runs.
+__device__ __forceinline__ void issue_prefetch(const Prefetch& pf, unsigned part, unsigned parts) {
+  for (int r = 0; r < pf.n; ++r) l2_prefetch_range(pf.r[r].p, pf.r[r].bytes, part, parts);
+  if (pf.kv.kc) {
+    const int ranges = 2 * pf.kv.B * pf.kv.Hkv;  // (sequence, kv head) x (K, V)
+    for (int j = (int)part; j < ranges; j += (int)parts) {
+      const int pair = j >> 1, b = pair / pf.kv.Hkv;
+      const int rows = pf.kv.pos[b];
+      if (rows <= 0 || rows > pf.kv.cap) continue;
+      const uint16_t* base = ((j & 1) ? pf.kv.vc : pf.kv.kc) + (size_t)pair * pf.kv.cap * pf.kv.D;
+      l2_prefetch_range(base, (unsigned long long)rows * pf.kv.D * 2, 0, 1);
+    }
+  }
+}
+
+// ------------------------------------------------------------ timeline --
+
+// Per-launch timestamps for diagnosing a chain of kernels inside a CUDA
+// graph (qg_timeline_begin / _end). Only a library built with QG_TIMELINE
+// records; otherwise the hooks compile to nothing. Each record is filled
+// with atomic maxima over the launch's CTAs (zero-initialised by the
+// caller): the earliest CTA entry (stored as its bitwise complement), the
+// latest return from the wait for the previous kernel, the latest exit.
+struct TlRec {
+  unsigned long long neg_entry, wait, exit, reserved;
+};
+
+// Host side: the record for the next launch (nullptr when not recording).
+// `kind` labels the launch for qg_timeline_end.
+TlRec* tl_take(int kind);
+// Labels the next launches of this host thread (until changed) for tl_take.
+void tl_set_kind(int kind);
+
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+#ifdef QG_TIMELINE
+__device__ __forceinline__ void tl_entry(TlRec* r) {
+  if (r && threadIdx.x == 0) atomicMax(&r->neg_entry, ~global_ns());
+}
+__device__ __forceinline__ void tl_wait(TlRec* r) {
+  if (r && threadIdx.x == 0) atomicMax(&r->wait, global_ns());
+}
+__device__ __forceinline__ void tl_exit(TlRec* r) {
+  if (r && threadIdx.x == 0) atomicMax(&r->exit, global_ns());
+}
+#else
+__device__ __forceinline__ void tl_entry(TlRec*) {}
+__device__ __forceinline__ void tl_wait(TlRec*) {}
+__device__ __forceinline__ void tl_exit(TlRec*) {}
+#endif
+
+// Launch kinds of the decode step (labels of the timeline records).
+enum TlKind { kTlEmbed = 1, kTlQkv, kTlAttn, kTlO, kTlGateUp, kTlDown, kTlHead, kTlOther };
+
 // ----------------------------------------------------------------- loads --
 
 // L2 policy for data read exactly once (packed weights): evict first.
@@ -158,12 +257,16 @@ cudaError_t gemv_tc_launch(const GemvSeg* segs, int nseg, const void* x, int K, 
 // of fp32 x [B][K], or bf16(silu(gate) * up) of fp32 [B][K] (eligibility as
 // gemv_tc_eligible with x_f32 = false). When xout is not null the formed
 // bf16 input is also written there ([B][K], by one CTA).
+// `pf`, when given, is L2 prefetch work issued at kernel entry.
 cudaError_t gemv_tc_launch_rmsnorm(const GemvSeg* segs, int nseg, const float* x,
                                    const uint16_t* norm_w, float eps, int K, int B,
-                                   cudaStream_t st, bool pdl, uint16_t* xout = nullptr);
+                                   cudaStream_t st, bool pdl, uint16_t* xout = nullptr,
+                                   const Prefetch* pf = nullptr);
 cudaError_t gemv_tc_launch_silu_mul(const GemvSeg* segs, int nseg, const float* gate,
                                     const float* up, int K, int B, cudaStream_t st, bool pdl,
-                                    uint16_t* xout = nullptr);
+                                    uint16_t* xout = nullptr, const Prefetch* pf = nullptr);
+cudaError_t gemv_tc_launch_pf(const GemvSeg* segs, int nseg, const void* x, int K, int B,
+                              cudaStream_t st, bool pdl, const Prefetch* pf);
 
 cudaError_t rmsnorm_launch(const float* x, const uint16_t* w, float eps, void* y,
                            bool y_bf16, int rows, int dim, cudaStream_t st, bool pdl);
@@ -182,8 +285,23 @@ cudaError_t attention_launch_step(const float* q, const float* k, const float* v
                                   const int32_t* tokens, int vocab, float eps, const float2* rope,
                                   uint16_t* kc, uint16_t* vc, const int32_t* positions, void* out,
                                   int B, int H, int Hkv, int D, int cap, float scale, void* ws,
-                                  cudaStream_t st, bool pdl);
+                                  cudaStream_t st, bool pdl, const Prefetch* pf = nullptr);
 size_t attention_ws_bytes(int B, int H, int Hkv, int D, int cap);
+
+// affine8 matmul on the tensor cores (gemm_affine8_sm100.cu): up to 3
+// matrices sharing X bf16 [T][K], each Y [T][N] (+ residual); err is a
+// device error word (nonzero after a device-side wait gave up).
+struct A8Seg {
+  const uint32_t* w;
+  const uint16_t* s;
+  const uint16_t* b;
+  void* y;
+  const float* res;
+  int N;
+  int y_bf16;
+};
+cudaError_t gemm_affine8_launch(const A8Seg* segs, int nseg, const uint16_t* X, int T, int K,
+                                unsigned* err, cudaStream_t st, bool pdl, int* nt_used);
 
 // greedy token per row (argmax.cu); ws of argmax_ws_bytes(B, V) bytes
 size_t argmax_ws_bytes(int B, int V);

@@ -1,0 +1,82 @@
+// tcgen05 / mbarrier helpers shared by the tensor-core GEMMs (sm_100a).
+#pragma once
+
+#include <cuda.h>  // CUtensorMap
+
+#include "qg_internal.cuh"
+
+namespace qg {
+
+// Host: a TMA descriptor of a bf16 [rows][cols] row-major tensor in boxes of
+// 64 columns x box_rows rows with 128-byte swizzle (rows past the end read as
+// zero); false when the driver's encoder is unavailable or refuses it.
+bool make_bf16_map(CUtensorMap* map, const void* base, int rows, int cols, int box_rows);
+
+namespace tc {
+
+constexpr unsigned long long kWaitNs = 1000000000ull;  // every device-side wait gives up after 1 s
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ unsigned long long now_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+// bounded wait; gives up early once another role has aborted
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = now_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort) return false;
+    if (now_ns() - t0 > kWaitNs) return false;
+  }
+  return true;
+}
+
+// K-major, 128-byte swizzle shared-memory matrix descriptor: 8-row groups
+// 1024 bytes apart (SBO), leading offset 16 bytes, descriptor version 1.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1u << 16;             // LBO = 16 B (encoded >> 4)
+  d |= (uint64_t)(1024u >> 4) << 32;   // SBO = 1024 B
+  d |= (uint64_t)1u << 46;             // version
+  d |= (uint64_t)2u << 61;             // SWIZZLE_128B
+  return d;
+}
+
+// instruction descriptor: bf16 x bf16 -> fp32, both K-major, M = 128
+template <int BN>
+__host__ __device__ constexpr uint32_t instr_desc() {
+  return (1u << 4)                 // D fp32
+         | (1u << 7)               // A bf16
+         | (1u << 10)              // B bf16
+         | ((uint32_t)(BN >> 3) << 17)
+         | ((uint32_t)(128 >> 4) << 24);
+}
+
+}  // namespace tc
+}  // namespace qg
