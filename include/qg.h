@@ -143,6 +143,16 @@ qg_status qg_gemm_q4_0(const uint8_t* blocks, const float* A, const float* bias,
  * the workspace). */
 qg_status qg_gemm_q4_0_error(int M, int K, const void* ws, unsigned* code, void* stream);
 
+/* Test aid for the timeout path (no counterpart on the pages): runs the
+ * matmul's kernel (bf16 A [M][K]) with every load withheld and no producer
+ * arriving, so its MMA issuer's first bounded wait runs out after about
+ * 1 ms while nothing is in flight; the kernel then frees its tensor memory
+ * and records a nonzero error word in ws (256 bytes, 256-byte aligned),
+ * which qg_gemm_q4_0_error(0, 0, ws, ...) reports as QG_ERR_TIMEOUT. C is
+ * not written. */
+qg_status qg_gemm_q4_0_stall_test(const uint8_t* blocks, const uint16_t* A, float* C, int M,
+                                  int N, int K, void* ws, size_t ws_bytes, void* stream);
+
 /* The same matmul with the operand and epilogue options the Whisper encoder
  * layer needs  [FT: encoder_layer -> q_linear, gelu_tanh, residual adds]:
  *

@@ -207,3 +207,29 @@ def test_sample_rejects_bad_arguments():
     assert st == qg.QG_ERR_UNSUPPORTED_SHAPE and "candidates" in msg
     st, msg = _status("qg_sample", *args(ws=need - 256))
     assert st == qg.QG_ERR_WORKSPACE_TOO_SMALL and str(need) in msg
+
+
+def test_new_row_entry_points_refuse_bad_shapes():
+    """The multi-row attention, the extended Q4_0 matmul, the affine8
+    matmul, LayerNorm, the Whisper layer and the prefill refuse bad shapes
+    before any launch, naming the argument."""
+    st, msg = _status("qg_attention_rows", FAKE, FAKE, FAKE, FAKE, 1, 4, 4, 2, 2, 96, 0, None)
+    assert st == qg.QG_ERR_UNSUPPORTED_SHAPE and "D=96" in msg
+    st, msg = _status("qg_attention_rows", FAKE, FAKE, FAKE, FAKE, 1, 8, 4, 2, 2, 64, 1, None)
+    assert st == qg.QG_ERR_UNSUPPORTED_SHAPE and "causal" in msg
+    st, msg = _status("qg_gemm_q4_0_ex", FAKE, FAKE, qg.QG_BF16, None, FAKE, FAKE, qg.QG_BF16, 0,
+                      128, 128, 128, FAKE, 256, None)
+    assert st == qg.QG_ERR_INVALID_ARGUMENT and "residual" in msg
+    st, msg = _status("qg_gemm_affine8_g64", FAKE, FAKE, FAKE, FAKE, FAKE, qg.QG_F32, None, 128,
+                      96, 4, FAKE, 4, None)
+    assert st == qg.QG_ERR_UNSUPPORTED_SHAPE and "K=96" in msg
+    st, msg = _status("qg_layernorm", FAKE, FAKE, FAKE, 1e-5, FAKE, qg.QG_BF16, 4, 4096, None)
+    assert st == qg.QG_ERR_UNSUPPORTED_SHAPE and "dim=4096" in msg
+    wc = qg.qg_whisper_config(1280, 16, 5120, 1e-5)   # head size 80
+    st, msg = _status("qg_whisper_encoder_layer", ctypes.byref(wc), None, FAKE, 10, FAKE, 1 << 30,
+                      None)
+    assert st == qg.QG_ERR_UNSUPPORTED_SHAPE and "heads=16" in msg
+    cfg = qg.qg_qwen3_config(512, 1, 4, 2, 128, 1024, 1000, 1e-6, 1e6)
+    st, msg = _status("qg_prefill", ctypes.byref(cfg), None, FAKE, FAKE, 16, FAKE, 10, 8, FAKE,
+                      FAKE, 1 << 30, None)
+    assert st == qg.QG_ERR_UNSUPPORTED_SHAPE and "cap=16" in msg

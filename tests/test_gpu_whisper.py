@@ -144,3 +144,27 @@ def test_whisper_encoder_layer_stagewise(shape, M):
     ref_y = O.whisper_encoder_layer(x, w, H, eps)
     rel = np.sqrt(np.mean((y - ref_y) ** 2) / np.mean(ref_y ** 2))
     assert rel < 1e-2, rel
+
+
+def test_gemm_timeout_path_reports_and_the_context_stays_usable():
+    """The matmul's bounded waits: with every load withheld
+    (qg_gemm_q4_0_stall_test), the MMA issuer's first wait runs out after
+    about 1 ms with nothing in flight; the call's error word reads nonzero
+    (QG_ERR_TIMEOUT), C is untouched, and a normal call right after is
+    correct."""
+    M, N, K = 256, 256, 128
+    blocks = qg_synth.q4_0_packed(N, K, 40)
+    A = O.round_bf16(qg_synth.gaussian((M, K), 1.0, 41))
+    Ad = _bf16(A)
+    C = torch.zeros((M, N), dtype=torch.float32, device="cuda")
+    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    st = qg.lib.qg_gemm_q4_0_stall_test(qg._p(dev(blocks)), qg._p(Ad), qg._p(C), M, N, K,
+                                        qg._p(ws), 256, qg._stream(None))
+    assert st == qg.QG_OK
+    status, code = qg.qg_gemm_q4_0_error(0, 0, ws)
+    assert status == qg.QG_ERR_TIMEOUT and code != 0
+    assert torch.count_nonzero(C) == 0
+    qg.qg_gemm_q4_0_ex(dev(blocks), Ad, C, ws=ws)
+    torch.cuda.synchronize()
+    assert qg.qg_gemm_q4_0_error(0, 0, ws)[1] == 0
+    assert_parity(host64(C), O.gemm_q4_0_bf16(blocks, A), what="after the timeout")

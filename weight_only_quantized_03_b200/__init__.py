@@ -116,6 +116,7 @@ _SIGS = {
                                         ctypes.POINTER(ctypes.c_size_t)]),
     "qg_code_predict_workspace_size": (_sz, [ctypes.POINTER(qg_qwen3_config), _i]),
     "qg_gemm_q4_0_ex": (_i, [_vp, _vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "qg_gemm_q4_0_stall_test": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp, _sz, _vp]),
     "qg_gemm_affine8_g64": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _vp, _sz, _vp]),
     "qg_prefill_workspace_size": (_sz, [ctypes.POINTER(qg_qwen3_config), _i]),
     "qg_prefill": (_i, [ctypes.POINTER(qg_qwen3_config), ctypes.POINTER(qg_qwen3_weights), _vp,

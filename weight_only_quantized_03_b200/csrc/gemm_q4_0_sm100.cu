@@ -149,6 +149,10 @@ struct Epi {
   void* C;            // [M][N]
   int c_bf16;
   int gelu;
+  // test of the timeout path (gemm_q4_0_tc_kernel only): no load is issued
+  // and no producer arrives, so the MMA issuer's first wait runs out (after
+  // 1 ms) with nothing in flight
+  int stall;
 };
 
 // GELU, tanh form (fuel-transformers `gelu_tanh`), in fp32 with CUDA's tanhf
@@ -156,156 +160,13 @@ __device__ __forceinline__ float gelu_tanh_f(float x) {
   return 0.5f * x * (1.0f + tanhf(0.7978845608028654f * (x + 0.044715f * x * x * x)));
 }
 
-template <int BN, int MT, bool W32>
-__global__ void __launch_bounds__(kThreads, 1)
-    gemm_q4_0_tc_kernel(const __grid_constant__ CUtensorMap tmA, const uint8_t* __restrict__ blocks,
-                        const Epi ep, int M, int N, int K, unsigned* __restrict__ err) {
-  using G = Cfg<BN, MT>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t* stages = smem;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + G::kStages * G::kStage);
-  uint64_t* tfull = full + G::kStages;
-  uint64_t* empty = tfull + G::kStages;
-  uint64_t* done = empty + G::kStages;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
-  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * (MT * kBM);
-  const int nk = K / kBK;
-  const size_t rowbytes = (size_t)(K / 32) * 18;
-
-  if (tid == 0) {
-    for (int s = 0; s < G::kStages; ++s) {
-      mbar_init(&full[s], kProducers);
-      mbar_init(&tfull[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    mbar_init(done, 1);
-    *abort = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  if (warp == 8) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(tmem_slot)),
-                 "r"(G::kTmemCols));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
-  }
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-  __syncthreads();
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-  const uint32_t tmem = *tmem_slot;
-
-  bool ok = true;
-  if (warp < 8) {
-    // ------------------------------------------------------ W producers
-    const bool has_row = tid < BN;
-    const uint8_t* wrow = blocks + (size_t)(n0 + (has_row ? tid : 0)) * rowbytes;
-    uint32_t raw[kPrefetch][9];
-#pragma unroll
-    for (int u = 0; u < kPrefetch; ++u)
-      if (has_row && u < nk) load_w_raw<W32>(wrow, u, raw[u]);
-    for (int kb0 = 0; kb0 < nk && ok; kb0 += kPrefetch) {
-#pragma unroll
-      for (int u = 0; u < kPrefetch; ++u) {
-        const int kb = kb0 + u;
-        if (kb >= nk) break;
-        const int s = kb % G::kStages;
-        if (kb >= G::kStages &&
-            !wait_bar(&empty[s], (uint32_t)((kb / G::kStages) + 1) & 1u, abort)) {
-          ok = false;
-          break;
-        }
-        if (has_row) {
-          store_w_row(stages + (size_t)s * G::kStage + G::kStageA, tid, raw[u]);
-          if (kb + kPrefetch < nk) load_w_raw<W32>(wrow, kb + kPrefetch, raw[u]);
-        }
-        // make the generic-proxy stores visible to the tensor core
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        mbar_arrive(&full[s]);
-      }
-    }
-    if (!ok) *abort = 1;
-  } else if (warp == 9) {
-    // ------------------------------------------------- A by TMA (lane 0)
-    if (lane == 0) {
-      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
-      int issued = 0;
-      for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % G::kStages;
-        if (kb >= G::kStages &&
-            !wait_bar(&empty[s], (uint32_t)((kb / G::kStages) + 1) & 1u, abort)) {
-          ok = false;
-          *abort = 1;
-          break;
-        }
-        mbar_expect_tx(&tfull[s], (uint32_t)G::kStageA);
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt)
-          asm volatile(
-              "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-              " [%0], [%1, {%2, %3}], [%4];" ::"r"(
-                  smem_u32(stages + (size_t)s * G::kStage + mt * kBM * kBK * 2)),
-              "l"(reinterpret_cast<uint64_t>(&tmA)), "r"(kb * kBK), "r"(m0 + mt * kBM),
-              "r"(smem_u32(&tfull[s]))
-              : "memory");
-        ++issued;
-      }
-      // no copy may land after the CTA is gone: wait (bounded) for the last
-      // fill of every stage used
-      for (int j = issued - G::kStages > 0 ? issued - G::kStages : 0; j < issued; ++j) {
-        const int s = j % G::kStages;
-        const uint32_t par = (uint32_t)(j / G::kStages) & 1u;
-        if (!mbar_try_wait(&tfull[s], par)) {
-          const unsigned long long t0 = now_ns();
-          while (!mbar_try_wait(&tfull[s], par))
-            if (now_ns() - t0 > kWaitNs) break;
-        }
-      }
-    }
-  } else if (lane == 0) {
-    // ------------------------------------------------------- MMA issuer
-    const uint32_t idesc = instr_desc<BN>();
-    for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % G::kStages;
-      const uint32_t par = (uint32_t)(kb / G::kStages) & 1u;
-      if (!wait_bar(&tfull[s], par, abort) || !wait_bar(&full[s], par, abort)) {
-        ok = false;
-        *abort = 1;
-        break;
-      }
-      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      const uint32_t sa = smem_u32(stages + (size_t)s * G::kStage);
-      const uint32_t sb = sa + G::kStageA;
-#pragma unroll
-      for (int k = 0; k < kBK / 16; ++k) {
-        const uint64_t db = smem_desc(sb + k * 32);
-        const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-          const uint64_t da = smem_desc(sa + mt * kBM * kBK * 2 + k * 32);
-          asm volatile(
-              "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-              " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
-                  tmem + (uint32_t)(mt * BN)),
-              "l"(da), "l"(db), "r"(idesc), "r"(acc)
-              : "memory");
-        }
-      }
-      asm volatile(
-          "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-              smem_u32(&empty[s]))
-          : "memory");
-    }
-    // completes once every MMA issued above has finished
-    asm volatile(
-        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-            smem_u32(done))
-        : "memory");
-  }
-
-  // ---------------------------------------------------------- epilogue
+// The epilogue shared by both kernels: warps 0-7 wait (bounded) for the last
+// commit, read the accumulator and store C through the Epi rules; then
+// tensor memory is freed. `ok` is this thread's own status so far.
+template <int BN, int MT>
+__device__ __forceinline__ void epilogue(uint32_t tmem, uint64_t* done, volatile int* abort,
+                                         const Epi& ep, int M, int N, int m0, int n0, int warp,
+                                         int lane, bool ok, unsigned* err) {
   bool landed = true;
   if (warp < 8) {
     // wait for the last commit even after an abort: tensor memory may only
@@ -388,10 +249,376 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
-                 "r"(G::kTmemCols));
+                 "r"(MT * BN));
   }
 }
 
+template <int BN, int MT, bool W32>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_q4_0_tc_kernel(const __grid_constant__ CUtensorMap tmA, const uint8_t* __restrict__ blocks,
+                        const Epi ep, int M, int N, int K, unsigned* __restrict__ err) {
+  using G = Cfg<BN, MT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* stages = smem;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + G::kStages * G::kStage);
+  uint64_t* tfull = full + G::kStages;
+  uint64_t* empty = tfull + G::kStages;
+  uint64_t* done = empty + G::kStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * (MT * kBM);
+  const int nk = K / kBK;
+  const size_t rowbytes = (size_t)(K / 32) * 18;
+
+  if (tid == 0) {
+    for (int s = 0; s < G::kStages; ++s) {
+      mbar_init(&full[s], kProducers);
+      mbar_init(&tfull[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(done, 1);
+    *abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 8) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(G::kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tmem = *tmem_slot;
+
+  bool ok = true;
+  if (warp < 8) {
+    // ------------------------------------------------------ W producers
+    // (none of this runs when stalling: the timeout test)
+    const bool has_row = tid < BN && !ep.stall;
+    const int nkp = ep.stall ? 0 : nk;
+    const uint8_t* wrow = blocks + (size_t)(n0 + (has_row ? tid : 0)) * rowbytes;
+    uint32_t raw[kPrefetch][9];
+#pragma unroll
+    for (int u = 0; u < kPrefetch; ++u)
+      if (has_row && u < nkp) load_w_raw<W32>(wrow, u, raw[u]);
+    for (int kb0 = 0; kb0 < nkp && ok; kb0 += kPrefetch) {
+#pragma unroll
+      for (int u = 0; u < kPrefetch; ++u) {
+        const int kb = kb0 + u;
+        if (kb >= nkp) break;
+        const int s = kb % G::kStages;
+        if (kb >= G::kStages &&
+            !wait_bar(&empty[s], (uint32_t)((kb / G::kStages) + 1) & 1u, abort)) {
+          ok = false;
+          break;
+        }
+        if (has_row) {
+          store_w_row(stages + (size_t)s * G::kStage + G::kStageA, tid, raw[u]);
+          if (kb + kPrefetch < nkp) load_w_raw<W32>(wrow, kb + kPrefetch, raw[u]);
+        }
+        // make the generic-proxy stores visible to the tensor core
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_arrive(&full[s]);
+      }
+    }
+    if (!ok) *abort = 1;
+  } else if (warp == 9) {
+    // ------------------------------------------------- A by TMA (lane 0)
+    if (lane == 0 && !ep.stall) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
+      int issued = 0;
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % G::kStages;
+        if (kb >= G::kStages &&
+            !wait_bar(&empty[s], (uint32_t)((kb / G::kStages) + 1) & 1u, abort)) {
+          ok = false;
+          *abort = 1;
+          break;
+        }
+        mbar_expect_tx(&tfull[s], (uint32_t)G::kStageA);
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+          asm volatile(
+              "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+              " [%0], [%1, {%2, %3}], [%4];" ::"r"(
+                  smem_u32(stages + (size_t)s * G::kStage + mt * kBM * kBK * 2)),
+              "l"(reinterpret_cast<uint64_t>(&tmA)), "r"(kb * kBK), "r"(m0 + mt * kBM),
+              "r"(smem_u32(&tfull[s]))
+              : "memory");
+        ++issued;
+      }
+      // no copy may land after the CTA is gone: wait (bounded) for the last
+      // fill of every stage used
+      for (int j = issued - G::kStages > 0 ? issued - G::kStages : 0; j < issued; ++j) {
+        const int s = j % G::kStages;
+        const uint32_t par = (uint32_t)(j / G::kStages) & 1u;
+        if (!mbar_try_wait(&tfull[s], par)) {
+          const unsigned long long t0 = now_ns();
+          while (!mbar_try_wait(&tfull[s], par))
+            if (now_ns() - t0 > kWaitNs) break;
+        }
+      }
+    }
+  } else if (lane == 0) {
+    // ------------------------------------------------------- MMA issuer
+    const uint32_t idesc = instr_desc<BN>();
+    for (int kb = 0; kb < nk; ++kb) {
+      const int s = kb % G::kStages;
+      const uint32_t par = (uint32_t)(kb / G::kStages) & 1u;
+      const unsigned long long lim = ep.stall ? 1000000ull : kWaitNs;
+      if (!wait_bar_ns(&tfull[s], par, abort, lim) || !wait_bar_ns(&full[s], par, abort, lim)) {
+        ok = false;
+        *abort = 1;
+        break;
+      }
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      const uint32_t sa = smem_u32(stages + (size_t)s * G::kStage);
+      const uint32_t sb = sa + G::kStageA;
+#pragma unroll
+      for (int k = 0; k < kBK / 16; ++k) {
+        const uint64_t db = smem_desc(sb + k * 32);
+        const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          const uint64_t da = smem_desc(sa + mt * kBM * kBK * 2 + k * 32);
+          asm volatile(
+              "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+              " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
+                  tmem + (uint32_t)(mt * BN)),
+              "l"(da), "l"(db), "r"(idesc), "r"(acc)
+              : "memory");
+        }
+      }
+      asm volatile(
+          "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+              smem_u32(&empty[s]))
+          : "memory");
+    }
+    // completes once every MMA issued above has finished
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+            smem_u32(done))
+        : "memory");
+  }
+
+  epilogue<BN, MT>(tmem, done, abort, ep, M, N, m0, n0, warp, lane, ok, err);
+}
+
+
+// ---------------------------------------------------------------------------
+// The same matmul with W's raw bytes staged by TMA (K % 256 == 0, so every
+// row's byte length is a multiple of 16): warp 9 also copies, per four MMA
+// stages, a BN x 144-byte box of raw Q4_0 rows (two blocks a stage) into a
+// two-slot ring; the W producers then read their 36 bytes from shared memory
+// instead of issuing nine scattered global loads per stage. Everything else
+// (the stage ring, the MMA issue, the epilogue, the bounded waits) is as in
+// gemm_q4_0_tc_kernel.
+// ---------------------------------------------------------------------------
+constexpr int kRawStages = 4;                 // MMA stages per raw chunk
+constexpr int kRawRow = kRawStages * 36;      // 144 bytes of a row per chunk
+constexpr int kRawSlots = 2;
+
+template <int BN, int MT>
+struct Cfg2 {
+  static constexpr int kStageA = MT * kBM * kBK * 2;
+  static constexpr int kStageB = BN * kBK * 2;
+  static constexpr int kStage = kStageA + kStageB;
+  static constexpr int kRawSlot = ((BN * kRawRow) + 1023) / 1024 * 1024;
+  static constexpr int kBudget = 220 * 1024 - kRawSlots * kRawSlot;
+  static constexpr int kStages = kBudget / kStage < 4 ? kBudget / kStage : 4;
+  static constexpr int kSmem = 1024 + kStages * kStage + kRawSlots * kRawSlot + 1024;
+  static constexpr int kTmemCols = MT * BN;
+};
+
+template <int BN, int MT>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_q4_0_tc2_kernel(const __grid_constant__ CUtensorMap tmA,
+                         const __grid_constant__ CUtensorMap tmW, const Epi ep, int M, int N,
+                         int K, unsigned* __restrict__ err) {
+  using G = Cfg2<BN, MT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* stages = smem;
+  uint8_t* raws = smem + G::kStages * G::kStage;
+  uint64_t* full = reinterpret_cast<uint64_t*>(raws + kRawSlots * G::kRawSlot);
+  uint64_t* tfull = full + G::kStages;
+  uint64_t* empty = tfull + G::kStages;
+  uint64_t* rfull = empty + G::kStages;
+  uint64_t* rempty = rfull + kRawSlots;
+  uint64_t* done = rempty + kRawSlots;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * (MT * kBM);
+  const int nk = K / kBK, nchunk = (nk + kRawStages - 1) / kRawStages;
+
+  if (tid == 0) {
+    for (int s = 0; s < G::kStages; ++s) {
+      mbar_init(&full[s], kProducers);
+      mbar_init(&tfull[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int r = 0; r < kRawSlots; ++r) {
+      mbar_init(&rfull[r], 1);
+      mbar_init(&rempty[r], kProducers);
+    }
+    mbar_init(done, 1);
+    *abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 8) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(G::kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tmem = *tmem_slot;
+
+  bool ok = true;
+  if (warp < 8) {
+    // ------------------------------------------------------ W producers
+    const bool has_row = tid < BN;
+    for (int kb = 0; kb < nk && ok; ++kb) {
+      const int c = kb / kRawStages, sub = kb % kRawStages, slot = c % kRawSlots;
+      if (sub == 0 && !wait_bar(&rfull[slot], (uint32_t)(c / kRawSlots) & 1u, abort)) {
+        ok = false;
+        break;
+      }
+      const int s = kb % G::kStages;
+      if (kb >= G::kStages &&
+          !wait_bar(&empty[s], (uint32_t)((kb / G::kStages) + 1) & 1u, abort)) {
+        ok = false;
+        break;
+      }
+      if (has_row) {
+        const uint32_t* rw =
+            reinterpret_cast<const uint32_t*>(raws + slot * G::kRawSlot + tid * kRawRow + sub * 36);
+        uint32_t raw[9];
+#pragma unroll
+        for (int i = 0; i < 9; ++i) raw[i] = rw[i];
+        store_w_row(stages + (size_t)s * G::kStage + G::kStageA, tid, raw);
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive(&full[s]);
+      if (sub == kRawStages - 1 || kb == nk - 1) mbar_arrive(&rempty[slot]);
+    }
+    if (!ok) *abort = 1;
+  } else if (warp == 9) {
+    // ------------------------------ A and W's raw chunks by TMA (lane 0)
+    if (lane == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmW)) : "memory");
+      int issued = 0, rissued = 0;
+      auto issue_raw = [&](int c) -> bool {
+        const int slot = c % kRawSlots;
+        if (c >= kRawSlots &&
+            !wait_bar(&rempty[slot], (uint32_t)((c / kRawSlots) + 1) & 1u, abort))
+          return false;
+        mbar_expect_tx(&rfull[slot], (uint32_t)(BN * kRawRow));
+        asm volatile(
+            "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+            " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(raws + slot * G::kRawSlot)),
+            "l"(reinterpret_cast<uint64_t>(&tmW)), "r"(c * kRawRow), "r"(n0),
+            "r"(smem_u32(&rfull[slot]))
+            : "memory");
+        ++rissued;
+        return true;
+      };
+      if (!issue_raw(0)) {
+        ok = false;
+        *abort = 1;
+      }
+      for (int kb = 0; kb < nk && ok; ++kb) {
+        if (kb % kRawStages == 0 && kb / kRawStages + 1 < nchunk &&
+            !issue_raw(kb / kRawStages + 1)) {
+          ok = false;
+          *abort = 1;
+          break;
+        }
+        const int s = kb % G::kStages;
+        if (kb >= G::kStages &&
+            !wait_bar(&empty[s], (uint32_t)((kb / G::kStages) + 1) & 1u, abort)) {
+          ok = false;
+          *abort = 1;
+          break;
+        }
+        mbar_expect_tx(&tfull[s], (uint32_t)G::kStageA);
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+          asm volatile(
+              "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+              " [%0], [%1, {%2, %3}], [%4];" ::"r"(
+                  smem_u32(stages + (size_t)s * G::kStage + mt * kBM * kBK * 2)),
+              "l"(reinterpret_cast<uint64_t>(&tmA)), "r"(kb * kBK), "r"(m0 + mt * kBM),
+              "r"(smem_u32(&tfull[s]))
+              : "memory");
+        ++issued;
+      }
+      // no copy may land after the CTA is gone: wait (bounded) for the last
+      // fill of every stage and raw slot used
+      auto drain = [&](uint64_t* bars, int nslots, int count) {
+        for (int j = count - nslots > 0 ? count - nslots : 0; j < count; ++j) {
+          const int s = j % nslots;
+          const uint32_t par = (uint32_t)(j / nslots) & 1u;
+          if (!mbar_try_wait(&bars[s], par)) {
+            const unsigned long long t0 = now_ns();
+            while (!mbar_try_wait(&bars[s], par))
+              if (now_ns() - t0 > kWaitNs) break;
+          }
+        }
+      };
+      drain(tfull, G::kStages, issued);
+      drain(rfull, kRawSlots, rissued);
+    }
+  } else if (lane == 0) {
+    // ------------------------------------------------------- MMA issuer
+    const uint32_t idesc = instr_desc<BN>();
+    for (int kb = 0; kb < nk; ++kb) {
+      const int s = kb % G::kStages;
+      const uint32_t par = (uint32_t)(kb / G::kStages) & 1u;
+      if (!wait_bar(&tfull[s], par, abort) || !wait_bar(&full[s], par, abort)) {
+        ok = false;
+        *abort = 1;
+        break;
+      }
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      const uint32_t sa = smem_u32(stages + (size_t)s * G::kStage);
+      const uint32_t sb = sa + G::kStageA;
+#pragma unroll
+      for (int k = 0; k < kBK / 16; ++k) {
+        const uint64_t db = smem_desc(sb + k * 32);
+        const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          const uint64_t da = smem_desc(sa + mt * kBM * kBK * 2 + k * 32);
+          asm volatile(
+              "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+              " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
+                  tmem + (uint32_t)(mt * BN)),
+              "l"(da), "l"(db), "r"(idesc), "r"(acc)
+              : "memory");
+        }
+      }
+      asm volatile(
+          "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+              smem_u32(&empty[s]))
+          : "memory");
+    }
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+            smem_u32(done))
+        : "memory");
+  }
+  epilogue<BN, MT>(tmem, done, abort, ep, M, N, m0, n0, warp, lane, ok, err);
+}
 }  // namespace gq4
 
 static size_t a_bytes(int M, int K) { return (((size_t)M * K * 2) + 255) & ~(size_t)255; }
@@ -457,6 +684,41 @@ static cudaError_t gq4_launch_mt(const CUtensorMap& tmA, const uint8_t* blocks, 
   return gq4_launch<BN, 1, W32>(tmA, blocks, ep, M, N, K, err, st);
 }
 
+// W's raw Q4_0 rows ([N][K/32 * 18] bytes; K % 256 == 0 makes the row
+// stride a multiple of 16) in boxes of 144 bytes (four MMA stages) x BN rows;
+// bytes past a row's end read as zero.
+static bool make_w_raw_map(CUtensorMap* map, const uint8_t* blocks, int N, int K, int BN) {
+  EncodeTiledFn enc = encode_tiled();
+  if (!enc) return false;
+  const cuuint64_t rowbytes = (cuuint64_t)(K / 32) * 18;
+  const cuuint64_t dims[2] = {rowbytes, (cuuint64_t)N};
+  const cuuint64_t strides[1] = {rowbytes};
+  const cuuint32_t box[2] = {(cuuint32_t)gq4::kRawRow, (cuuint32_t)BN};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(blocks), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN, int MT>
+static cudaError_t gq4_launch2(const CUtensorMap& tmA, const CUtensorMap& tmW, const gq4::Epi& ep,
+                               int M, int N, int K, unsigned* err, cudaStream_t st) {
+  using G = gq4::Cfg2<BN, MT>;
+  ensure_smem((const void*)gq4::gemm_q4_0_tc2_kernel<BN, MT>, G::kSmem);
+  dim3 grid(N / BN, (M + MT * gq4::kBM - 1) / (MT * gq4::kBM));
+  return launch_pdl(gq4::gemm_q4_0_tc2_kernel<BN, MT>, grid, dim3(gq4::kThreads),
+                    (size_t)G::kSmem, st, false, tmA, tmW, ep, M, N, K, err);
+}
+
+template <int BN>
+static cudaError_t gq4_launch2_mt(const CUtensorMap& tmA, const CUtensorMap& tmW,
+                                  const gq4::Epi& ep, int M, int N, int K, unsigned* err,
+                                  cudaStream_t st) {
+  const long long tiles2 = (long long)(N / BN) * ((M + 255) / 256);
+  if (2 * tiles2 >= num_sms()) return gq4_launch2<BN, 2>(tmA, tmW, ep, M, N, K, err, st);
+  return gq4_launch2<BN, 1>(tmA, tmW, ep, M, N, K, err, st);
+}
+
 // The GEMM on a bf16 A already in device memory (`Ab`, [M][K]); `err` is the
 // workspace error word.
 static qg_status gq4_run(const uint8_t* blocks, const uint16_t* Ab, const gq4::Epi& ep, int M,
@@ -465,6 +727,18 @@ static qg_status gq4_run(const uint8_t* blocks, const uint16_t* Ab, const gq4::E
   if (!make_a_map(&tmA, Ab, M, K)) {
     set_error("%s: could not encode the TMA descriptor of A", what);
     return QG_ERR_CUDA;
+  }
+  if (K % 256 == 0 && aligned(blocks, 16)) {
+    // W's raw bytes staged by TMA
+    const int BN = N % 256 == 0 ? 256 : 128;
+    CUtensorMap tmW;
+    if (!make_w_raw_map(&tmW, blocks, N, K, BN)) {
+      set_error("%s: could not encode the TMA descriptor of W", what);
+      return QG_ERR_CUDA;
+    }
+    if (BN == 256) gq4_launch2_mt<256>(tmA, tmW, ep, M, N, K, err, s);
+    else gq4_launch2_mt<128>(tmA, tmW, ep, M, N, K, err, s);
+    return check_launch(what);
   }
   const bool w32 = aligned(blocks, 4);
   if (N % 256 == 0) {
@@ -530,7 +804,7 @@ static qg_status gemm_q4_0_checked(const uint8_t* blocks, const void* A, qg_dtyp
     Ab = Aw;
   }
   cudaMemsetAsync(err, 0, sizeof(unsigned), s);
-  gq4::Epi ep = {bias, residual, C, c_dtype == QG_BF16 ? 1 : 0, gelu ? 1 : 0};
+  gq4::Epi ep = {bias, residual, C, c_dtype == QG_BF16 ? 1 : 0, gelu ? 1 : 0, 0};
   return gq4_run(blocks, Ab, ep, M, N, K, err, s, what);
 }
 
@@ -570,4 +844,28 @@ extern "C" qg_status qg_gemm_q4_0_error(int M, int K, const void* ws, unsigned* 
     return QG_ERR_TIMEOUT;
   }
   return QG_OK;
+}
+
+extern "C" qg_status qg_gemm_q4_0_stall_test(const uint8_t* blocks, const uint16_t* A, float* C,
+                                             int M, int N, int K, void* ws, size_t ws_bytes,
+                                             void* stream) {
+  clear_error();
+  QG_REQUIRE(M > 0 && N > 0 && N % 128 == 0 && K > 0 && K % 64 == 0, QG_ERR_UNSUPPORTED_SHAPE,
+             "qg_gemm_q4_0_stall_test: M=%d N=%d K=%d", M, N, K);
+  QG_REQUIRE(blocks && A && C && aligned(A, 16) && aligned(C, 16) && aligned(blocks, 4),
+             QG_ERR_INVALID_ARGUMENT, "qg_gemm_q4_0_stall_test: bad pointer");
+  QG_REQUIRE(ws && ws_bytes >= 256 && aligned(ws, 256), QG_ERR_WORKSPACE_TOO_SMALL,
+             "qg_gemm_q4_0_stall_test: ws must be 256 bytes, 256-byte aligned");
+  cudaStream_t s = (cudaStream_t)stream;
+  unsigned* err = reinterpret_cast<unsigned*>(ws);
+  cudaMemsetAsync(err, 0, sizeof(unsigned), s);
+  CUtensorMap tmA;
+  if (!make_a_map(&tmA, A, M, K)) {
+    set_error("qg_gemm_q4_0_stall_test: could not encode the TMA descriptor of A");
+    return QG_ERR_CUDA;
+  }
+  gq4::Epi ep = {nullptr, nullptr, C, 0, 0, 1};
+  if (N % 256 == 0) gq4_launch<256, 1, true>(tmA, blocks, ep, M, N, K, err, s);
+  else gq4_launch<128, 1, true>(tmA, blocks, ep, M, N, K, err, s);
+  return check_launch("qg_gemm_q4_0_stall_test");
 }

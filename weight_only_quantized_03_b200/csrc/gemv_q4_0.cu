@@ -138,6 +138,9 @@ gemv_q4_0_staged_kernel(const uint8_t* __restrict__ blocks, const float* __restr
       if (i < n16) dst[i] = v[u];
     }
   }
+  // the next kernel may launch now and start its own weight loads (its wait
+  // still covers all of this one)
+  pdl_trigger();
   __syncthreads();
   pdl_wait();  // x and bias may be written by the previous kernel
   float acc[R][NB];
@@ -170,7 +173,6 @@ gemv_q4_0_staged_kernel(const uint8_t* __restrict__ blocks, const float* __restr
       }
     }
   }
-  pdl_trigger();
 #pragma unroll
   for (int r = 0; r < R; ++r)
 #pragma unroll

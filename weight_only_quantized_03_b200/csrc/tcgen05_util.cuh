@@ -45,15 +45,19 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
                "r"(bytes)
                : "memory");
 }
-// bounded wait; gives up early once another role has aborted
-__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort) {
+// bounded wait (limit_ns); gives up early once another role has aborted
+__device__ __forceinline__ bool wait_bar_ns(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                            unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = now_ns();
   while (!mbar_try_wait(bar, parity)) {
     if (*abort) return false;
-    if (now_ns() - t0 > kWaitNs) return false;
+    if (now_ns() - t0 > limit_ns) return false;
   }
   return true;
+}
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  return wait_bar_ns(bar, parity, abort, kWaitNs);
 }
 
 // K-major, 128-byte swizzle shared-memory matrix descriptor: 8-row groups
