@@ -342,6 +342,272 @@ def prefill_rows(qg, model, cfg, stream):
             "speedup": ms_r / ms_b}
 
 
+def code_predictor_frame(qg, stream, hbm_peak, n):
+    """One frame of the makima Qwen3-TTS code predictor (hidden 1024, 5
+    layers, 16 heads, head_dim 64, FFN 3072, 16 groups of 2048 codes; random
+    packed weights), batch 1: the 15 sequential groups of one
+    qg_code_predict call, timed with CUDA events over n back-to-back calls
+    (each call replays the recorded graph of the whole frame)."""
+    import torch
+    import weight_only_quantized_03_b200 as qgm
+    cfg, G = dict(qg_synth.CODE_PREDICTOR), qg_synth.CODE_GROUPS
+    model = qgm.CodePredictor(cfg, qg_synth.code_predictor_weights(cfg, G, 51))
+    lm = torch.from_numpy(qg_synth.gaussian((1, cfg["hidden"]), 1.0, 52).astype(np.float32)).cuda()
+    code0 = torch.tensor([7], dtype=torch.int32, device="cuda")
+    codes = torch.empty((G, 1), dtype=torch.int32, device="cuda")
+    ws = model.workspace(1)
+    n0 = qg.lib.qg_kernel_launch_count()  # the first call records the frame's launches
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            model.qg_code_predict(lm, code0, codes, ws, stream=stream)
+    stream.synchronize()
+    launches = qg.lib.qg_kernel_launch_count() - n0
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(n):
+            model.qg_code_predict(lm, code0, codes, ws, stream=stream)
+        e1.record(stream)
+    stream.synchronize()
+    ms = e0.elapsed_time(e1) / n
+    h, F, V = cfg["hidden"], cfg["ffn"], cfg["vocab"]
+    HD = cfg["heads"] * cfg["head_dim"]
+    layer = sum(affine8_bytes(N, K, 1) for N, K in
+                ((HD, h), (HD, h), (HD, h), (h, HD), (F, h), (F, h), (h, F)))
+    group = cfg["layers"] * layer + affine8_bytes(h, 2 * h, 1) + affine8_bytes(V, h, 1)
+    fbytes = (G - 1) * group
+    return {"workload": "Qwen3-TTS code predictor frame (makima CodePredictorConfig), batch 1",
+            "frames_per_s": 1000.0 / ms, "ms_per_frame": ms, "groups": G - 1,
+            "launches_per_frame": launches, "algorithmic_bytes": fbytes,
+            "achieved": fbytes / (ms / 1000.0) / 1e9, "peak": hbm_peak, "unit": "GB/s",
+            "note": "weights are read once per group (15 per frame); the 5 layers' 72 MB "
+                    "can stay in L2 between groups, so achieved may pass the HBM peak"}
+
+
+def measured_tensor_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured (bf16 burst)"
+    except Exception:
+        return 1590.0, "fallback"
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_sha256(paths):
+    """sha256 over the given source files, concatenated in order."""
+    h = hashlib.sha256()
+    for p in paths:
+        h.update(open(p, "rb").read())
+    return h.hexdigest()
+
+
+GEMV_SOURCES = [os.path.join(ROOT, "weight_only_quantized_03_b200", "csrc", f)
+                for f in ("gemv_affine8_tc.cu", "gemv_tc.cuh", "qg_internal.cuh")]
+LM_HEAD_SOURCES = GEMV_SOURCES
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def traffic_from_profile(kernel_files, key="gemv_affine8_lm_head_151936x1024_b1",
+                         field="dram_bytes_per_launch"):
+    """DRAM bytes (read + written) of a kernel from one ncu capture, kept in
+    profiles/traffic.json, or None when the entry is missing or was taken on
+    a different version of the kernel sources (their sha256 must match)."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            d = json.load(f)[key]
+    except (OSError, KeyError, ValueError):
+        return None
+    if d.get("kernel_source_sha256") != source_sha256(kernel_files):
+        return None
+    return d.get(field)
+
+
+def step_gemv_traffic(B):
+    """DRAM bytes per step of the step's layer GEMV launches (batch 1 only)."""
+    if B != 1:
+        return None
+    return traffic_from_profile(GEMV_SOURCES, "step_layer_gemvs_qwen3_0.6b_b1_kv512",
+                                "dram_bytes_per_step")
+
+
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons while running."""
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.rows = []
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) == 6:
+                self.rows.append(parts)
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[0]) for r in self.rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4) if r[2 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(self.rows)}
+
+
+def cpu_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n and n[0]:
+            return int(n[0])
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+# ------------------------------------------------------ oracle (CPU) legs ---
+
+def oracle_sample(cfg, weights, budget_steps=None, layers_only=None):
+    """Time the CPU oracle on a bounded sample of the decode step: whole
+    steps (28 layers + LM head) or, with ``layers_only``, that many single
+    layers plus one LM head, scaled to a whole step. Returns (steps/s,
+    description)."""
+    from oracle import qg_oracle as O
+    Hk, D = cfg["kv_heads"], cfg["head_dim"]
+    cap = KV_LEN + 1
+    kc = O.bf16_bits_to_f64(qg_synth.gaussian_bf16_bits((cfg["layers"], Hk, cap, D), 1.0, 70))
+    vc = O.bf16_bits_to_f64(qg_synth.gaussian_bf16_bits((cfg["layers"], Hk, cap, D), 1.0, 71))
+    tok = int(qg_synth.tokens(1, cfg["vocab"], 72)[0])
+    if layers_only is None:
+        t0 = time.perf_counter()
+        for _ in range(budget_steps):
+            O.decode_step(cfg, weights, kc, vc, tok, KV_LEN - 1)
+        dt = (time.perf_counter() - t0) / budget_steps
+        return 1.0 / dt, f"{budget_steps} full decode step(s) at position {KV_LEN - 1}, batch 1"
+    ew, es, eb = weights["embed"]
+    x = O.embed_rows(ew, es, eb, [tok])[0]
+    t0 = time.perf_counter()
+    for i in range(layers_only):
+        l = i % cfg["layers"]
+        x = O.decode_layer(cfg, weights["layers"][l], x, kc[l], vc[l], KV_LEN - 1)
+    t_layer = (time.perf_counter() - t0) / layers_only
+    t0 = time.perf_counter()
+    O.lm_head(cfg, weights, x)
+    t_head = time.perf_counter() - t0
+    return 1.0 / (cfg["layers"] * t_layer + t_head), (
+        f"{layers_only} single decoder layers at position {KV_LEN - 1} plus one LM head, "
+        f"scaled to 28 layers + head, batch 1")
+
+
+def run_reference(args):
+    """The oracle on the host cores, as it stands. Each of the W + K steps is
+    a bounded sample of the workload: one decoder layer of the 0.6B step at
+    position 511 (a full step is 28 layers and the LM head). The LM head is
+    timed once after the timed samples. ``ms_per_step`` is the measured time
+    of one sample; ``value`` is the full-step rate those times give
+    (1 / (28 x mean layer time + LM head time)), marked as extrapolated."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from oracle import qg_oracle as O
+    cfg = dict(qg_synth.QWEN3_0_6B)
+    weights = qg_synth.qwen3_weights(cfg, 11)
+    Hk, D = cfg["kv_heads"], cfg["head_dim"]
+    cap = KV_LEN + 1
+    kc = O.bf16_bits_to_f64(qg_synth.gaussian_bf16_bits((cfg["layers"], Hk, cap, D), 1.0, 70))
+    vc = O.bf16_bits_to_f64(qg_synth.gaussian_bf16_bits((cfg["layers"], Hk, cap, D), 1.0, 71))
+    tok = int(qg_synth.tokens(1, cfg["vocab"], 72)[0])
+    x = O.embed_rows(*weights["embed"], [tok])[0]
+    for i in range(args.warmup):
+        O.decode_layer(cfg, weights["layers"][i % cfg["layers"]], x, kc[0], vc[0], KV_LEN - 1)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        l = i % cfg["layers"]
+        x = O.decode_layer(cfg, weights["layers"][l], x, kc[l], vc[l], KV_LEN - 1)
+    t_layers = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    O.lm_head(cfg, weights, x)
+    t_head = time.perf_counter() - t0
+    t_layer = t_layers / args.steps
+    v = 1.0 / (cfg["layers"] * t_layer + t_head)
+    cores = cpu_cores()
+    desc = (f"each timed step: one decoder layer of the 28 at position {KV_LEN - 1}, batch 1 "
+            f"({args.steps} timed, layers in order); the LM head timed once ({t_head:.3f} s)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "steps/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * t_layer, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"Qwen3-0.6B-shaped affine-INT8 g64 decode step, batch 1, KV {KV_LEN}"},
+        "sample": {"timed_step": "one decoder layer (1/28 of the layers of a decode step)",
+                   "ms_per_step_is": "measured time of one sample (one layer)",
+                   "value_is": "extrapolated full-step rate: 1 / (28 x mean layer time + LM head time)",
+                   "full_step_s": 1.0 / v, "lm_head_s": t_head},
+        "cpu_baseline": {"value": v, "unit": "steps/s", "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": v, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------ ranks ---------
+
+def max_over_ranks(ms, world, dist=None, device="cpu"):
+    """The slowest rank's time: every rank contributes its own device time
+    and all get the maximum (an all-reduce, the same collective on every
+    rank); with one rank, the time itself."""
+    if world <= 1:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_value(world, units_per_rank, max_ms):
+    """Whole-job throughput of independent replicas: the units all ranks
+    processed over the slowest rank's time."""
+    return world * units_per_rank / (max_ms / 1000.0)
+
+
+# ------------------------------------------------------------ GPU arm -------
+
 TIMELINE_NAMES = {1: "embed", 2: "qkv", 3: "attn", 4: "o", 5: "gate_up", 6: "down", 7: "head",
                   8: "other"}
 GEMV_KINDS = ("qkv", "o", "gate_up", "down")
