@@ -904,14 +904,28 @@ def run_ours(args):
 
 def run_ncu_case(args):
     """One kernel alone, warm-up then ``--steps`` launches, for an ncu capture
-    (no timing, no JSON line): ``lm_head`` is the tied LM-head GEMV of the
+    (no timing, no JSON line): ``step`` is the bench's whole decode step
+    (launched eagerly, no step graph); ``lm_head`` is the tied LM-head GEMV of the
     0.6B shape at ``--batch``; ``gemm`` the Whisper FC1 Q4_0 GEMM
     (1500 x 5120 x 1280); ``attn`` the decode attention at the 1.7B shape,
     batch 32, KV 2048."""
     import torch
     import weight_only_quantized_03_b200 as qg
     to = lambda a: torch.from_numpy(a.view({1: np.uint8, 2: np.int16, 4: np.int32}[a.dtype.itemsize])).cuda()
-    if args.ncu_case == "lm_head":
+    if args.ncu_case == "step":
+        # the bench's decode step (0.6B shape, KV 512) launched eagerly: 5
+        # launches per layer plus the embedding and the LM head per step
+        cfg = dict(qg_synth.QWEN3_0_6B)
+        model = qg.Qwen3Model(cfg, qg_synth.qwen3_weights(cfg, 11))
+        B = args.batch
+        st = model.new_state(B, KV_LEN + 1)
+        st["k_cache"].normal_()
+        st["v_cache"].normal_()
+        toks = torch.from_numpy(qg_synth.tokens(B, cfg["vocab"], 72)).cuda()
+        pos = torch.full((B,), KV_LEN - 1, dtype=torch.int32, device="cuda")
+        qg.lib.qg_step_graphs_enable(0)
+        run = lambda: model.qg_decode_step(st, toks, pos)
+    elif args.ncu_case == "lm_head":
         cfg = qg_synth.QWEN3_0_6B
         V, h = cfg["vocab"], cfg["hidden"]
         w, s, b = (to(a) for a in qg_synth.affine8_packed(V, h, 4242))
@@ -1013,7 +1027,7 @@ def main():
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--ncu-case", choices=["lm_head", "gemm", "attn"], default=None,
+    ap.add_argument("--ncu-case", choices=["step", "lm_head", "gemm", "attn"], default=None,
                     help="launch one kernel only (for an ncu capture); prints no JSON line")
     ap.add_argument("--sweep", action="store_true",
                     help="the Qwen3-1.7B-shaped prefill and batch sweep (its own JSON line)")

@@ -152,7 +152,21 @@ __device__ __forceinline__ void merge_state(float& m, float& l, float* o, float 
   m = M;
 }
 
-template <int D, int GM>
+// 4-byte cp.async granule helpers for the fused o_proj slice
+__device__ __forceinline__ void cp_async_16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                   (uint32_t)__cvta_generic_to_shared(dst)),
+               "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_8(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(
+                   (uint32_t)__cvta_generic_to_shared(dst)),
+               "l"(src)
+               : "memory");
+}
+
+template <int D, int GM, bool OPROJ>
 __global__ void __launch_bounds__(kThreads, GM <= 2 ? 2 : 1)
 attention_cluster_kernel(const float* q, const uint16_t* kc, const uint16_t* vc,
                          const int32_t* __restrict__ kv_len, const int32_t* __restrict__ pos_for_len,
@@ -160,6 +174,7 @@ attention_cluster_kernel(const float* q, const uint16_t* kc, const uint16_t* vc,
                          const AttnFuse fz) {
   using G = Geo<D>;
   constexpr int LPR = G::LPR, RPI = G::RPI, U = G::U;
+  extern __shared__ __align__(16) uint8_t wslice[];  // fused o_proj: W_o rows of this CTA
   __shared__ float sq[GM][D];          // query heads (normed, roped) * scale
   __shared__ float kp[D], vp[D];       // the new row p (bf16 values), owner CTA only
   __shared__ float sp[GM];             // scores of row p
@@ -207,6 +222,36 @@ attention_cluster_kernel(const float* q, const uint16_t* kc, const uint16_t* vc,
   if (fz.on) {
     if (nb > 0) load(0, ka, va);
     if (nb > 1) load(1, kb, vb);
+  }
+  // fused o_proj: this CTA's W_o rows [s R, s R + R), the g*D columns of this
+  // KV head's query heads, to shared memory (weights: no wait needed)
+  const int gD = g * D;
+  const int R = OPROJ ? fz.hidden / (int)cs : 0;
+  // dynamic shared memory: W_o codes [R][gD], scales and biases [R][gD/64],
+  // then ofin (rank 0: the head group's output, bf16 values) and xo (every
+  // CTA's copy of it), gD floats each
+  uint8_t* wcodes = wslice;
+  uint16_t* wsc = reinterpret_cast<uint16_t*>(wslice + R * gD);
+  uint16_t* wbi = wsc + R * (gD / 64);
+  float* ofin = reinterpret_cast<float*>(wbi + R * (gD / 64));
+  float* xo = ofin + gD;
+  if constexpr (OPROJ) {
+    const int HD = H * D, r0 = (int)s * R, c0 = kv * gD;
+    const int chunks = R * gD / 16;
+    for (int i = threadIdx.x; i < chunks; i += kThreads) {
+      const int r = i / (gD / 16), c = (i % (gD / 16)) * 16;
+      cp_async_16(wcodes + r * gD + c, fz.ow + (size_t)(r0 + r) * HD + c0 + c);
+    }
+    // gD / 64 bf16 scales and biases a row: gD / 64 * 2 bytes = 8 bytes for
+    // gD = 256 (one granule), more granules for wider groups
+    const int sbytes = gD / 64 * 2;
+    for (int i = threadIdx.x; i < R * (sbytes / 8); i += kThreads) {
+      const int r = i / (sbytes / 8), c = (i % (sbytes / 8)) * 4;
+      const size_t gi = (size_t)(r0 + r) * (HD / 64) + c0 / 64 + c;
+      cp_async_8(wsc + r * (gD / 64) + c, fz.os + gi);
+      cp_async_8(wbi + r * (gD / 64) + c, fz.ob + gi);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
   }
   // the next kernel may be scheduled now: its own wait covers all of this one
   pdl_trigger();
@@ -407,9 +452,43 @@ attention_cluster_kernel(const float* q, const uint16_t* kc, const uint16_t* vc,
         reinterpret_cast<uint16_t*>(out)[oi] = f32_to_bf16_bits(res);
       else
         reinterpret_cast<float*>(out)[oi] = res;
+      if constexpr (OPROJ) ofin[i] = bf16_bits_to_f32(f32_to_bf16_bits(res));
     }
   }
   cluster_sync();  // no CTA leaves while rank 0 still reads its shared memory
+  if constexpr (OPROJ) {
+    // the head group's bf16 output from rank 0, then the o_proj partial rows
+    for (int i = threadIdx.x; i < gD; i += kThreads) xo[i] = ld_cluster(&ofin[i], 0);
+    cluster_sync();  // rank 0 stays until every CTA has read its output
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    __syncthreads();
+    // thread t: row t / tpr of the slice, columns [p * cpt, (p + 1) * cpt)
+    // (whole 64-column groups) with p = t % tpr; per group s * sum(q x) +
+    // beta * sum(x), products exact in fp32; the tpr parts then meet by
+    // shuffles in a fixed order
+    const int tpr = kThreads / R, cpt = gD / tpr;
+    const int r = threadIdx.x / tpr, p = threadIdx.x % tpr;
+    float acc = 0.f;
+    for (int c0 = p * cpt; c0 < (p + 1) * cpt; c0 += 64) {
+      const uint32_t* qw = reinterpret_cast<const uint32_t*>(wcodes + r * gD + c0);
+      float sq = 0.f, sx = 0.f;
+#pragma unroll 4
+      for (int j = 0; j < 16; ++j) {
+        const uint32_t w = qw[j];
+        const float* xv = xo + c0 + 4 * j;
+        sq = fmaf(byte_to_f32<0>(w), xv[0], sq);
+        sq = fmaf(byte_to_f32<1>(w), xv[1], sq);
+        sq = fmaf(byte_to_f32<2>(w), xv[2], sq);
+        sq = fmaf(byte_to_f32<3>(w), xv[3], sq);
+        sx += (xv[0] + xv[1]) + (xv[2] + xv[3]);
+      }
+      const int gi = r * (gD / 64) + c0 / 64;
+      acc = fmaf(bf16_bits_to_f32(wsc[gi]), sq, fmaf(bf16_bits_to_f32(wbi[gi]), sx, acc));
+    }
+    for (int off = 1; off < tpr; off <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (p == 0)
+      fz.opart[((size_t)b * Hkv + kv) * fz.hidden + (size_t)s * R + r] = valid ? acc : __int_as_float(0x7fc00000);
+  }
   tl_exit(fz.tl);
 }
 
@@ -429,7 +508,25 @@ inline int cluster_size(int B, int Hkv, int cap) {
   return (int)cs;
 }
 
-template <int D, int GM>
+// Whether the fused o_proj takes the launch: rows hidden / cs per CTA, each
+// thread whole 64-column groups of the head group's g*D columns, and the
+// slice within a dynamic shared-memory budget.
+inline int oproj_smem(int hidden, int cs, int gD) {
+  const int R = hidden / cs;
+  return R * gD + 2 * R * (gD / 64) * 2 + 2 * gD * 4;
+}
+inline bool oproj_ok(int hidden, int cs, int gD) {
+  if (cs < 1 || hidden % cs != 0) return false;
+  const int R = hidden / cs;
+  if (R < 1 || R > kThreads || kThreads % R != 0) return false;
+  const int tpr = kThreads / R;
+  if (gD % 64 != 0 || gD % tpr != 0 || (gD / tpr) % 64 != 0 || (gD / 64 * 2) % 8 != 0)
+    return false;
+  if (tpr > 32) return false;
+  return oproj_smem(hidden, cs, gD) <= 96 * 1024;
+}
+
+template <int D, int GM, bool OPROJ>
 cudaError_t launch(const float* q, const uint16_t* kc, const uint16_t* vc, const int32_t* kv_len,
                    const int32_t* pos_for_len, void* out, bool out_bf16, int B, int H, int Hkv,
                    int cap, float scale, cudaStream_t st, bool pdl, const AttnFuse& fz) {
@@ -438,7 +535,9 @@ cudaError_t launch(const float* q, const uint16_t* kc, const uint16_t* vc, const
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(cs, Hkv, B);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = OPROJ ? oproj_smem(fz.hidden, cs, (H / Hkv) * D) : 0;
+  if (OPROJ)
+    ensure_smem((const void*)attention_cluster_kernel<D, GM, true>, (int)cfg.dynamicSmemBytes);
   cfg.stream = st;
   cudaLaunchAttribute a[2];
   a[0].id = cudaLaunchAttributeClusterDimension;
@@ -450,8 +549,8 @@ cudaError_t launch(const float* q, const uint16_t* kc, const uint16_t* vc, const
   cfg.attrs = a;
   cfg.numAttrs = pdl ? 2 : 1;
   count_launch();
-  return cudaLaunchKernelEx(&cfg, attention_cluster_kernel<D, GM>, q, kc, vc, kv_len, pos_for_len,
-                            out, (int)out_bf16, H, Hkv, cap, scale, ch, fz);
+  return cudaLaunchKernelEx(&cfg, attention_cluster_kernel<D, GM, OPROJ>, q, kc, vc, kv_len,
+                            pos_for_len, out, (int)out_bf16, H, Hkv, cap, scale, ch, fz);
 }
 
 template <int D>
@@ -459,14 +558,24 @@ cudaError_t launch_d(const float* q, const uint16_t* kc, const uint16_t* vc, con
                      const int32_t* pos_for_len, void* out, bool out_bf16, int B, int H, int Hkv,
                      int cap, float scale, cudaStream_t st, bool pdl, const AttnFuse& fz) {
   const int g = H / Hkv;
+  if (fz.ow) {  // the caller checked oproj_ok
+    if (g <= 1)
+      return launch<D, 1, true>(q, kc, vc, kv_len, pos_for_len, out, out_bf16, B, H, Hkv, cap,
+                                scale, st, pdl, fz);
+    if (g <= 2)
+      return launch<D, 2, true>(q, kc, vc, kv_len, pos_for_len, out, out_bf16, B, H, Hkv, cap,
+                                scale, st, pdl, fz);
+    return launch<D, 4, true>(q, kc, vc, kv_len, pos_for_len, out, out_bf16, B, H, Hkv, cap,
+                              scale, st, pdl, fz);
+  }
   if (g <= 1)
-    return launch<D, 1>(q, kc, vc, kv_len, pos_for_len, out, out_bf16, B, H, Hkv, cap, scale, st,
-                        pdl, fz);
+    return launch<D, 1, false>(q, kc, vc, kv_len, pos_for_len, out, out_bf16, B, H, Hkv, cap,
+                               scale, st, pdl, fz);
   if (g <= 2)
-    return launch<D, 2>(q, kc, vc, kv_len, pos_for_len, out, out_bf16, B, H, Hkv, cap, scale, st,
-                        pdl, fz);
-  return launch<D, 4>(q, kc, vc, kv_len, pos_for_len, out, out_bf16, B, H, Hkv, cap, scale, st,
-                      pdl, fz);
+    return launch<D, 2, false>(q, kc, vc, kv_len, pos_for_len, out, out_bf16, B, H, Hkv, cap,
+                               scale, st, pdl, fz);
+  return launch<D, 4, false>(q, kc, vc, kv_len, pos_for_len, out, out_bf16, B, H, Hkv, cap, scale,
+                             st, pdl, fz);
 }
 
 }  // namespace ac
@@ -535,8 +644,16 @@ cudaError_t attention_launch_step(const float* q, const float* k, const float* v
                                   const int32_t* tokens, int vocab, float eps, const float2* rope,
                                   uint16_t* kc, uint16_t* vc, const int32_t* positions, void* out,
                                   int B, int H, int Hkv, int D, int cap, float scale, void* ws,
-                                  cudaStream_t st, bool pdl, const Prefetch* pf) {
+                                  cudaStream_t st, bool pdl, const Prefetch* pf,
+                                  const OProjFuse* op) {
   AttnFuse fz = {};
+  if (op) {
+    fz.ow = reinterpret_cast<const uint8_t*>(op->w);
+    fz.os = op->s;
+    fz.ob = op->b;
+    fz.opart = op->part;
+    fz.hidden = op->hidden;
+  }
   fz.on = 1;
   fz.k = k;
   fz.v = v;
@@ -550,6 +667,11 @@ cudaError_t attention_launch_step(const float* q, const float* k, const float* v
   fz.tl = tl_take(0);
   return attention_launch_any(q, kc, vc, nullptr, positions, out, true, B, H, Hkv, D, cap, scale,
                               ws, st, pdl, fz);
+}
+
+bool attention_oproj_fusable(int B, int H, int Hkv, int D, int cap, int hidden) {
+  if (!ac::cluster_ok(H, Hkv, D)) return false;
+  return ac::oproj_ok(hidden, ac::cluster_size(B, Hkv, cap), (H / Hkv) * D);
 }
 
 // Offset of the ticket counters inside an attention workspace.

@@ -26,6 +26,15 @@ struct AttnFuse {
   const float2* rope;    // (cos, sin) [B][D/2] of the step's positions
   Prefetch pf;           // L2 prefetch work for a later kernel of the step
   TlRec* tl;             // timeline record of this launch, or null
+  // o_proj fused into the cluster kernel (ow non-null): each CTA of the
+  // cluster of (b, kv) multiplies rows [rank * R, rank * R + R) of W_o's
+  // columns of this KV head's query heads by their (bf16) attention output
+  // and writes the partial rows to opart[b][kv][hidden]; R = hidden / cs.
+  const uint8_t* ow;     // codes [hidden][H*D]
+  const uint16_t* os;    // bf16 [hidden][H*D/64]
+  const uint16_t* ob;
+  float* opart;
+  int hidden;
 };
 
 // The fused step's L2 prefetch, issued by one thread of each CTA at entry.

@@ -22,7 +22,7 @@ namespace qg {
 size_t attention_ws_counter_offset(int B, int H, int Hkv, int D, int cap);
 
 struct StepLayout {
-  size_t x, xn, xn2, xnf, q, k, v, xa, attn, gate, up, h, attn_ws, rope, err, total;
+  size_t x, xn, xn2, xnf, q, k, v, xa, attn, gate, up, h, oparts, attn_ws, rope, err, total;
 };
 
 static size_t a256(size_t v) { return (v + 255) & ~(size_t)255; }
@@ -45,6 +45,7 @@ static StepLayout step_layout(const qg_qwen3_config& c, int B, int cap) {
   L.gate = take((size_t)B * c.ffn * 4);
   L.up = take((size_t)B * c.ffn * 4);
   L.h = take((size_t)B * c.ffn * 2);
+  L.oparts = take((size_t)B * c.kv_heads * c.hidden * 4);  // fused o_proj partial rows
   L.attn_ws = take(attention_ws_bytes(B, c.heads, c.kv_heads, c.head_dim, cap));
   L.rope = take((size_t)B * (c.head_dim / 2) * 8);
   L.err = take(256);  // error word of the tensor-core matmuls (batched steps)
@@ -159,6 +160,7 @@ struct StepBufs {
   void* aws;
   float2* rope;
   unsigned* err;
+  float* oparts;
 };
 
 static StepBufs step_bufs(void* ws, const StepLayout& Ly) {
@@ -179,6 +181,7 @@ static StepBufs step_bufs(void* ws, const StepLayout& Ly) {
   b.aws = base + Ly.attn_ws;
   b.rope = reinterpret_cast<float2*>(base + Ly.rope);
   b.err = reinterpret_cast<unsigned*>(base + Ly.err);
+  b.oparts = reinterpret_cast<float*>(base + Ly.oparts);
   return b;
 }
 
@@ -217,6 +220,14 @@ static Prefetch pf_kv(const qg_qwen3_config& c, const uint16_t* kc, const uint16
 // kernels; below it, the tensor-core GEMV streams the weights with the
 // norms fused into its prologue.
 constexpr int kStepGemmBatch = 5;
+
+// o_proj folded into the attention kernel (one launch fewer per layer) where
+// the shapes allow it; QG_NO_FUSE_OPROJ keeps it a GEMV launch of its own.
+#ifdef QG_NO_FUSE_OPROJ
+constexpr bool kStepFuseOProj = false;
+#else
+constexpr bool kStepFuseOProj = true;
+#endif
 
 static bool step_uses_gemm(const qg_qwen3_config& c, int B) {
   return B >= kStepGemmBatch && c.hidden % 64 == 0 && c.ffn % 64 == 0 &&
@@ -275,6 +286,35 @@ static void enqueue_layers(const qg_qwen3_config& c, const qg_qwen3_layer* layer
                  (const float*)sb.gate, (const float*)sb.up, sb.hm, n);
       const A8Seg m_dn = {L.down.w, L.down.scales, L.down.biases, x, sb.xa, c.hidden, 0};
       gemm_affine8_launch(&m_dn, 1, sb.hm, B, c.ffn, sb.err, s, true, nullptr);
+      after_layer(l);
+      continue;
+    }
+    GemvSeg gu_f[2] = {{L.gate.w, L.gate.scales, L.gate.biases, sb.gate, nullptr, c.ffn, 0},
+                       {L.up.w, L.up.scales, L.up.biases, sb.up, nullptr, c.ffn, 0}};
+    if (kStepFuseOProj && gemv_tc_eligible(qkv, 3, c.hidden, B, false) &&
+        gemv_tc_eligible(gu_f, 2, c.hidden, B, false) && aligned(L.o.scales, 8) &&
+        aligned(L.o.biases, 8) && attention_oproj_fusable(B, H, Hkv, D, cap, c.hidden)) {
+      // 4 launches: q/k/v (input norm in the prologue); attention with o_proj
+      // (partial rows per KV head); gate/up with the residual + partials and
+      // the post-attention norm in the prologue; down with SiLU-mul
+      Prefetch pf_att = {};
+      pf_matrix(pf_att, L.gate, c.ffn, c.hidden);
+      pf_matrix(pf_att, L.up, c.ffn, c.hidden);
+      pf_matrix(pf_att, L.down, c.hidden, c.ffn);
+      Prefetch pf_gu2 = pf_next_qkv;
+      tl_set_kind(kTlQkv);
+      gemv_tc_launch_rmsnorm(qkv, 3, x, L.input_norm, c.eps, c.hidden, B, s, true, sb.xn, &pf_o);
+      tl_set_kind(kTlAttn);
+      const OProjFuse op = {L.o.w, L.o.scales, L.o.biases, sb.oparts, c.hidden};
+      attention_launch_step(sb.q, sb.k, sb.v, L.q_norm, L.k_norm, tokens, c.vocab, c.eps, sb.rope,
+                            kc, vc, positions, sb.attn, B, H, Hkv, D, cap, scale, sb.aws, s, true,
+                            &pf_att, &op);
+      tl_set_kind(kTlGateUp);
+      gemv_tc_launch_rmsnorm_parts(gu_f, 2, x, sb.oparts, Hkv, sb.xa, L.post_norm, c.eps,
+                                   c.hidden, B, s, true, sb.xn2, &pf_gu2);
+      tl_set_kind(kTlDown);
+      GemvSeg dn = {L.down.w, L.down.scales, L.down.biases, x, sb.xa, c.hidden, 0};
+      gemv_tc_launch_silu_mul(&dn, 1, sb.gate, sb.up, c.ffn, B, s, true, sb.hm, &pf_next_kv);
       after_layer(l);
       continue;
     }

@@ -143,6 +143,23 @@ cudaError_t gemv_tc_launch_rmsnorm(const GemvSeg* segs, int nseg, const float* x
   return gtc_launch(segs, nseg, P, K, B, st, pdl, pf);
 }
 
+cudaError_t gemv_tc_launch_rmsnorm_parts(const GemvSeg* segs, int nseg, const float* x,
+                                         const float* parts, int nparts, float* xsum,
+                                         const uint16_t* norm_w, float eps, int K, int B,
+                                         cudaStream_t st, bool pdl, uint16_t* xout,
+                                         const Prefetch* pf) {
+  gtc::Params P = {};
+  P.xmode = gtc::kXRmsNormParts;
+  P.xout = xout;
+  P.xa = x;
+  P.parts = parts;
+  P.nparts = nparts;
+  P.xsum = xsum;
+  P.nw = norm_w;
+  P.eps = eps;
+  return gtc_launch(segs, nseg, P, K, B, st, pdl, pf);
+}
+
 cudaError_t gemv_tc_launch_silu_mul(const GemvSeg* segs, int nseg, const float* gate,
                                     const float* up, int K, int B, cudaStream_t st, bool pdl,
                                     uint16_t* xout, const Prefetch* pf) {

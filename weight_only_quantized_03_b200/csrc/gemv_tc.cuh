@@ -31,7 +31,11 @@ struct Seg {
 //   kXBf16     x bf16 [B][K] as given;
 //   kXRmsNorm  bf16(xa / sqrt(mean(xa^2) + eps) * nw) per batch row, xa fp32;
 //   kXSiluMul  bf16(silu(xa) * xb), xa = gate and xb = up, both fp32.
-enum XMode { kXBf16 = 0, kXRmsNorm = 1, kXSiluMul = 2 };
+//   kXRmsNormParts  as kXRmsNorm of xa + sum_{j < nparts} parts[j] (the
+//                   o_proj partial rows of the fused attention, summed in
+//                   order j = 0, 1, ...); CTA 0 also stores that sum (the
+//                   residual stream after o_proj) to xsum.
+enum XMode { kXBf16 = 0, kXRmsNorm = 1, kXSiluMul = 2, kXRmsNormParts = 3 };
 
 struct Params {
   Seg seg[kMaxSegs];
@@ -42,6 +46,9 @@ struct Params {
   const uint16_t* nw;  // kXRmsNorm weight, bf16 [K]
   float eps;
   uint16_t* xout;      // optional: CTA 0 records the formed bf16 input [B][K]
+  const float* parts;  // kXRmsNormParts: [B][nparts][K]
+  int nparts;
+  float* xsum;         // kXRmsNormParts: CTA 0 stores xa + sum(parts) [B][K]
   Prefetch pf;         // L2 prefetch work for a later kernel (pf.n == 0, pf.kv.kc null: none)
   TlRec* tl;           // timeline record of this launch, or null
 };
@@ -206,7 +213,8 @@ __device__ __forceinline__ void gemv_tc_body(const Params& P, uint8_t* smem, Wai
 #pragma unroll
   for (int j = 0; j < kItems; ++j) {
     nwr[j] = make_uint2(0u, 0u);
-    if (P.xmode == kXRmsNorm && j < my_items) nwr[j] = nw_of(((warp + j * kWarps) % Kp) * 128 + 4 * lane);
+    if ((P.xmode == kXRmsNorm || P.xmode == kXRmsNormParts) && j < my_items)
+      nwr[j] = nw_of(((warp + j * kWarps) % Kp) * 128 + 4 * lane);
   }
 
   wait();  // x (and residuals) are written upstream
@@ -223,6 +231,17 @@ __device__ __forceinline__ void gemv_tc_body(const Params& P, uint8_t* smem, Wai
       return make_float4(bf16_lo(w2.x), bf16_hi(w2.x), bf16_lo(w2.y), bf16_hi(w2.y));
     }
     float4 va = __ldcg(reinterpret_cast<const float4*>(P.xa + o));
+    if (P.xmode == kXRmsNormParts) {
+      const float* pb = P.parts + ((size_t)(b0 + b) * P.nparts) * K + c;
+      for (int j = 0; j < P.nparts; ++j) {
+        const float4 pj = __ldcg(reinterpret_cast<const float4*>(pb + (size_t)j * K));
+        va.x += pj.x;
+        va.y += pj.y;
+        va.z += pj.z;
+        va.w += pj.w;
+      }
+      if (blockIdx.x == 0) *reinterpret_cast<float4*>(P.xsum + o) = va;
+    }
     if (P.xmode == kXSiluMul) {
       const float4 u = __ldcg(reinterpret_cast<const float4*>(P.xb + o));
       va = make_float4(va.x / (1.0f + expf(-va.x)) * u.x, va.y / (1.0f + expf(-va.y)) * u.y,
@@ -258,7 +277,8 @@ __device__ __forceinline__ void gemv_tc_body(const Params& P, uint8_t* smem, Wai
   float inv[4 * NT];
 #pragma unroll
   for (int b = 0; b < 4 * NT; ++b) inv[b] = 0.f;
-  if (P.xmode == kXRmsNorm) {
+  const bool norm = P.xmode == kXRmsNorm || P.xmode == kXRmsNormParts;
+  if (norm) {
     float ssb[4 * NT];
 #pragma unroll
     for (int b = 0; b < 4 * NT; ++b) ssb[b] = 0.f;
@@ -295,7 +315,7 @@ __device__ __forceinline__ void gemv_tc_body(const Params& P, uint8_t* smem, Wai
   auto form_item = [&](int i, const float4& va, const uint2& nw2, float down) -> float {
     const int b = i / Kp, c = (i - b * Kp) * 128 + 4 * lane;
     float v[4] = {va.x, va.y, va.z, va.w};
-    if (P.xmode == kXRmsNorm) {
+    if (norm) {
       float ib = inv[0];
 #pragma unroll
       for (int jb = 1; jb < 4 * NT; ++jb)
@@ -333,7 +353,7 @@ __device__ __forceinline__ void gemv_tc_body(const Params& P, uint8_t* smem, Wai
       if (j < my_items) mloc = fmaxf(mloc, form_item(warp + j * kWarps, xv[j], nwr[j], down));
     for (int j = kItems; j < my_items; ++j) {
       const int i = warp + j * kWarps;
-      const uint2 nw2 = P.xmode == kXRmsNorm ? nw_of((i % Kp) * 128 + 4 * lane) : make_uint2(0u, 0u);
+      const uint2 nw2 = norm ? nw_of((i % Kp) * 128 + 4 * lane) : make_uint2(0u, 0u);
       mloc = fmaxf(mloc, form_item(i, load_item(i), nw2, down));
     }
     return mloc;

@@ -267,6 +267,13 @@ cudaError_t gemv_tc_launch_silu_mul(const GemvSeg* segs, int nseg, const float* 
                                     uint16_t* xout = nullptr, const Prefetch* pf = nullptr);
 cudaError_t gemv_tc_launch_pf(const GemvSeg* segs, int nseg, const void* x, int K, int B,
                               cudaStream_t st, bool pdl, const Prefetch* pf);
+// The RMSNorm prologue on x + sum_{j < nparts} parts[b][j] (fixed order),
+// parts [B][nparts][K] fp32; CTA 0 stores that sum to xsum [B][K].
+cudaError_t gemv_tc_launch_rmsnorm_parts(const GemvSeg* segs, int nseg, const float* x,
+                                         const float* parts, int nparts, float* xsum,
+                                         const uint16_t* norm_w, float eps, int K, int B,
+                                         cudaStream_t st, bool pdl, uint16_t* xout,
+                                         const Prefetch* pf);
 
 cudaError_t rmsnorm_launch(const float* x, const uint16_t* w, float eps, void* y,
                            bool y_bf16, int rows, int dim, cudaStream_t st, bool pdl);
@@ -275,6 +282,17 @@ cudaError_t attention_launch(const float* q, const uint16_t* kc, const uint16_t*
                              const int32_t* kv_len, const int32_t* pos_for_len,
                              void* out, bool out_bf16, int B, int H, int Hkv, int D,
                              int cap, float scale, void* ws, cudaStream_t st, bool pdl);
+
+// o_proj fused into the decode step's attention: W_o (codes [hidden][H*D],
+// scales/biases 8-byte aligned) and the partial rows out, fp32
+// [B][Hkv][hidden] (one row of partial sums per KV head's query heads).
+struct OProjFuse {
+  const uint32_t* w;
+  const uint16_t* s;
+  const uint16_t* b;
+  float* part;
+  int hidden;
+};
 
 // The decode step's attention: q/k per-head RMSNorm, NeoX RoPE at
 // positions[b] (the (cos, sin) table [B][D/2] of the step) and the K/V
@@ -285,7 +303,11 @@ cudaError_t attention_launch_step(const float* q, const float* k, const float* v
                                   const int32_t* tokens, int vocab, float eps, const float2* rope,
                                   uint16_t* kc, uint16_t* vc, const int32_t* positions, void* out,
                                   int B, int H, int Hkv, int D, int cap, float scale, void* ws,
-                                  cudaStream_t st, bool pdl, const Prefetch* pf = nullptr);
+                                  cudaStream_t st, bool pdl, const Prefetch* pf = nullptr,
+                                  const OProjFuse* op = nullptr);
+// Whether the step's attention can take o_proj into its cluster kernel
+// (attention_launch_step with an OProjFuse) for this shape.
+bool attention_oproj_fusable(int B, int H, int Hkv, int D, int cap, int hidden);
 size_t attention_ws_bytes(int B, int H, int Hkv, int D, int cap);
 
 // affine8 matmul on the tensor cores (gemm_affine8_sm100.cu): up to 3
