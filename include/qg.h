@@ -89,6 +89,12 @@ unsigned long long qg_kernel_launch_count(void);
  * Launch: with Programmatic Dependent Launch, so a chain of calls overlaps
  * each GEMV's first weight loads with the previous kernel's tail; the kernel
  * waits for the stream's previous kernel before it reads x or residual.
+ * w, scales and biases must not be written by the kernel just before the
+ * call on the stream (the first weight loads are issued before that wait).
+ * With bf16 x, B >= 5 and a matrix of at least one 128-row tile per SM (the
+ * LM head), the call runs qg_gemm_affine8_g64's tensor-core matmul kernel
+ * instead (same results within the tolerance; its bounded device-side
+ * waits report nothing through this entry point).
  * ---------------------------------------------------------------------- */
 qg_status qg_gemv_affine8_g64(const uint32_t* w, const uint16_t* scales,
                               const uint16_t* biases, const void* x,

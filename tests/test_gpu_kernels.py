@@ -134,10 +134,12 @@ def test_gemv_affine8_large_activations_prescaled():
 
 
 def test_gemv_affine8_lm_head_full_size_sampled_rows():
-    # the tied LM head of the 0.6B shape: 151936 x 1024, batch 1 (and 4)
+    # the tied LM head of the 0.6B shape: 151936 x 1024, batch 1 and 4 (the
+    # tensor-core GEMV) and 5, 16, 32 (the tensor-core matmul, which takes
+    # batches past 4 for matrices of a wave of 128-row tiles or more)
     N, K = 151936, 1024
     w, s, b = qg_synth.affine8_packed(N, K, 4242)
-    for B in (1, 4):
+    for B in (1, 4, 5, 16, 32):
         xbits = qg_synth.gaussian_bf16_bits((B, K), 1.0, 4243 + B)
         y = torch.empty((B, N), dtype=torch.float32, device="cuda")
         qg.qg_gemv_affine8_g64(dev(w), dev(s), dev(b), bf16_dev(xbits), y)

@@ -214,11 +214,11 @@ static Prefetch pf_kv(const qg_qwen3_config& c, const uint16_t* kc, const uint16
   return pf;
 }
 
-// From this batch size on, the step's linears run as tensor-core matmuls
-// (gemm_affine8_sm100.cu: the batch rows are the MMA's N, each weight tile is
-// dequantized once for all rows) with RMSNorm and SiLU-mul as separate
-// kernels; below it, the tensor-core GEMV streams the weights with the
-// norms fused into its prologue.
+// From this batch size on, the tied LM head (a wave of 128-row tiles or
+// more) runs as a tensor-core matmul (gemm_affine8_sm100.cu: the batch rows
+// are the MMA's N, each weight tile is dequantized once for all rows) after
+// a separate final RMSNorm; the layers' matrices, a few dozen tiles each,
+// stay on the tensor-core GEMV with its fused prologues.
 constexpr int kStepGemmBatch = 5;
 
 // o_proj folded into the attention kernel (one launch fewer per layer) where
@@ -229,9 +229,8 @@ constexpr bool kStepFuseOProj = false;
 constexpr bool kStepFuseOProj = true;
 #endif
 
-static bool step_uses_gemm(const qg_qwen3_config& c, int B) {
-  return B >= kStepGemmBatch && c.hidden % 64 == 0 && c.ffn % 64 == 0 &&
-         (c.heads * c.head_dim) % 64 == 0;
+static bool head_uses_gemm(const qg_qwen3_config& c, int N, int B) {
+  return B >= kStepGemmBatch && c.hidden % 64 == 0 && (N + 127) / 128 >= num_sms();
 }
 
 // `after_layer`, when given, is called with the layer index after each
@@ -261,34 +260,6 @@ static void enqueue_layers(const qg_qwen3_config& c, const qg_qwen3_layer* layer
     const Prefetch pf_next_qkv = last ? Prefetch{} : pf_qkv(c, layers[l + 1]);
     const Prefetch pf_next_kv =
         last ? Prefetch{} : pf_kv(c, kc + layer_cache, vc + layer_cache, positions, B, cap);
-    if (step_uses_gemm(c, B)) {
-      tl_set_kind(kTlQkv);
-      rmsnorm_launch(x, L.input_norm, c.eps, sb.xn, true, B, c.hidden, s, true);
-      const A8Seg m_qkv[3] = {{L.q.w, L.q.scales, L.q.biases, sb.q, nullptr, H * D, 0},
-                              {L.k.w, L.k.scales, L.k.biases, sb.k, nullptr, Hkv * D, 0},
-                              {L.v.w, L.v.scales, L.v.biases, sb.v, nullptr, Hkv * D, 0}};
-      gemm_affine8_launch(m_qkv, 3, sb.xn, B, c.hidden, sb.err, s, true, nullptr);
-      tl_set_kind(kTlAttn);
-      attention_launch_step(sb.q, sb.k, sb.v, L.q_norm, L.k_norm, tokens, c.vocab, c.eps,
-                            sb.rope, kc, vc, positions, sb.attn, B, H, Hkv, D, cap, scale,
-                            sb.aws, s, true, &pf_gu);
-      tl_set_kind(kTlO);
-      const A8Seg m_o = {L.o.w, L.o.scales, L.o.biases, sb.xa, x, c.hidden, 0};
-      gemm_affine8_launch(&m_o, 1, sb.attn, B, H * D, sb.err, s, true, nullptr);
-      tl_set_kind(kTlGateUp);
-      rmsnorm_launch(sb.xa, L.post_norm, c.eps, sb.xn2, true, B, c.hidden, s, true);
-      const A8Seg m_gu[2] = {{L.gate.w, L.gate.scales, L.gate.biases, sb.gate, nullptr, c.ffn, 0},
-                             {L.up.w, L.up.scales, L.up.biases, sb.up, nullptr, c.ffn, 0}};
-      gemm_affine8_launch(m_gu, 2, sb.xn2, B, c.hidden, sb.err, s, true, nullptr);
-      tl_set_kind(kTlDown);
-      const int n = B * c.ffn;
-      launch_pdl(step_silu_mul_kernel, dim3((n + 255) / 256), dim3(256), 0, s, true,
-                 (const float*)sb.gate, (const float*)sb.up, sb.hm, n);
-      const A8Seg m_dn = {L.down.w, L.down.scales, L.down.biases, x, sb.xa, c.hidden, 0};
-      gemm_affine8_launch(&m_dn, 1, sb.hm, B, c.ffn, sb.err, s, true, nullptr);
-      after_layer(l);
-      continue;
-    }
     GemvSeg gu_f[2] = {{L.gate.w, L.gate.scales, L.gate.biases, sb.gate, nullptr, c.ffn, 0},
                        {L.up.w, L.up.scales, L.up.biases, sb.up, nullptr, c.ffn, 0}};
     if (kStepFuseOProj && gemv_tc_eligible(qkv, 3, c.hidden, B, false) &&
@@ -376,7 +347,7 @@ static void enqueue_head(const qg_qwen3_config& c, const qg_affine8_matrix& head
                          cudaStream_t s) {
   GemvSeg h = {head.w, head.scales, head.biases, logits, nullptr, N, 0};
   tl_set_kind(kTlHead);
-  if (step_uses_gemm(c, B)) {
+  if (head_uses_gemm(c, N, B)) {
     rmsnorm_launch(sb.x, final_norm, c.eps, sb.xnf, true, B, c.hidden, s, true);
     const A8Seg m = {head.w, head.scales, head.biases, logits, nullptr, N, 0};
     gemm_affine8_launch(&m, 1, sb.xnf, B, c.hidden, sb.err, s, true, nullptr);
@@ -398,7 +369,7 @@ static void enqueue_step(const qg_qwen3_config& c, const qg_qwen3_weights* w, ui
   const StepBufs sb = step_bufs(ws, Ly);
   const size_t cnt_off = attention_ws_counter_offset(B, c.heads, c.kv_heads, c.head_dim, cap);
   cudaMemsetAsync(reinterpret_cast<uint8_t*>(sb.aws) + cnt_off, 0, (size_t)B * c.kv_heads * 4, s);
-  if (step_uses_gemm(c, B)) cudaMemsetAsync(sb.err, 0, 4, s);
+  if (head_uses_gemm(c, c.vocab, B)) cudaMemsetAsync(sb.err, 0, 4, s);
   Prefetch pf0 = {};
   if (c.layers > 0) {
     pf0 = pf_qkv(c, w->layers[0]);

@@ -212,8 +212,30 @@ static cudaError_t launch_nb(GemvParams& P, bool xf32, cudaStream_t st, bool pdl
   return launch_nb_r<NB, 1>(P, xf32, st, pdl);
 }
 
+// Past 4 batch rows, a matrix with at least a wave of 128-row tiles (the LM
+// head) takes the tensor-core matmul: each weight tile is dequantized once
+// for all batch rows (the GEMV would stream it once per 8 rows).
+static bool gemm_takes(const GemvSeg* segs, int nseg, const void* x, int K, int B, bool x_f32) {
+  if (x_f32 || B < 5 || K % 64 != 0 || nseg > 3 || !aligned(x, 16)) return false;
+  long long tiles = 0;
+  for (int i = 0; i < nseg; ++i) {
+    if (!aligned(segs[i].w, 16)) return false;
+    if (i + 1 < nseg && segs[i].N % 128 != 0) return false;  // tiles may not straddle matrices
+    tiles += (segs[i].N + 127) / 128;
+  }
+  return tiles >= num_sms();
+}
+
 cudaError_t gemv_affine8_launch(const GemvSeg* segs, int nseg, const void* x, bool x_f32,
                                 int K, int B, cudaStream_t st, bool pdl) {
+  if (gemm_takes(segs, nseg, x, K, B, x_f32)) {
+    A8Seg m[3];
+    for (int i = 0; i < nseg; ++i)
+      m[i] = A8Seg{segs[i].w, segs[i].s, segs[i].b, segs[i].y, segs[i].res, segs[i].N,
+                   segs[i].y_bf16};
+    return gemm_affine8_launch(m, nseg, reinterpret_cast<const uint16_t*>(x), B, K, nullptr, st,
+                               pdl, nullptr);
+  }
   if (gemv_tc_eligible(segs, nseg, K, B, x_f32)) return gemv_tc_launch(segs, nseg, x, K, B, st, pdl);
   const size_t esz = x_f32 ? 4 : 2;
   for (int b0 = 0; b0 < B; b0 += 8) {
