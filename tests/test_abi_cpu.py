@@ -81,23 +81,25 @@ def test_attention_rejects_bad_group_and_small_workspace():
 
 def test_attention_static_scratch_refuses_shapes_beyond_its_capacity():
     """The fixed scratch limits only the shapes that take the split kernel
-    (here 8 query heads per KV head); cluster shapes use no scratch."""
+    (here head_dim 96); cluster and tensor-core shapes use no scratch."""
     cap_bytes = qg.lib.qg_decode_attention_static_scratch_capacity()
     assert cap_bytes == 4 << 20
-    need = qg.lib.qg_decode_attention_workspace_size(32, 16, 2, 128, 32768)
+    need = qg.lib.qg_decode_attention_workspace_size(32, 16, 2, 96, 32768)
     assert need > cap_bytes
     st, msg = _status("qg_decode_attention_static_scratch", FAKE, FAKE, FAKE, FAKE, FAKE,
-                      qg.QG_BF16, 32, 16, 2, 128, 32768, 1.0, None)
+                      qg.QG_BF16, 32, 16, 2, 96, 32768, 1.0, None)
     assert st == qg.QG_ERR_WORKSPACE_TOO_SMALL and str(need) in msg and str(cap_bytes) in msg
     import torch
     if not torch.cuda.is_available():
-        # a cluster shape whose nominal split workspace exceeds the array is not
-        # refused for capacity (with no device it stops at the address lookup,
-        # before any launch)
-        assert qg.lib.qg_decode_attention_workspace_size(32, 16, 8, 128, 32768) > cap_bytes
-        st, msg = _status("qg_decode_attention_static_scratch", FAKE, FAKE, FAKE, FAKE, FAKE,
-                          qg.QG_BF16, 32, 16, 8, 128, 32768, 1.0, None)
-        assert st == qg.QG_ERR_CUDA and "address lookup" in msg
+        # shapes whose nominal split workspace exceeds the array but that take
+        # the cluster kernel (2 query heads per KV head) or the tensor-core
+        # kernel (8 per KV head, long cache) are not refused for capacity
+        # (with no device they stop at the address lookup, before any launch)
+        for Hkv in (8, 2):
+            assert qg.lib.qg_decode_attention_workspace_size(32, 16, Hkv, 128, 32768) > cap_bytes
+            st, msg = _status("qg_decode_attention_static_scratch", FAKE, FAKE, FAKE, FAKE, FAKE,
+                              qg.QG_BF16, 32, 16, Hkv, 128, 32768, 1.0, None)
+            assert st == qg.QG_ERR_CUDA and "address lookup" in msg
 
 
 def test_elementwise_reject_bad_shapes():

@@ -194,9 +194,10 @@ def test_qwen3_0_6b_step_layer_by_layer_at_position_511(B):
 @pytest.mark.parametrize("B,layers", [(2, 3), (12, 2)])
 def test_qwen3_1_7b_shaped_layers_at_position_2047(B, layers):
     """The 1.7B layer shapes (hidden 2048, FFN 6144, K/V cache of 2049 rows)
-    with a few layers, teacher-forced per layer at positions up to 2047 on the
-    default kernel-per-op path. B = 12 takes the CUDA-core GEMV (batch past
-    the tensor-core path's 8) with RMSNorm and SiLU-mul as separate kernels."""
+    with a few layers, teacher-forced per layer at positions up to 2047.
+    B = 2 takes the cluster attention kernel; B = 12 (12 x 8 x 2049 cached
+    rows) the tensor-core attention kernel with the step's fused q/k norm,
+    RoPE and K/V append, and the tensor-core GEMV in batch tiles of 8."""
     cfg = dict(qg_synth.QWEN3_1_7B, layers=layers)
     w = qg_synth.qwen3_weights(cfg, 17)
     model = qg.Qwen3Model(cfg, w)

@@ -310,6 +310,12 @@ ATTN_CASES = [
     (1, 2, 2, 32, 1000, [999]),                 # head_dim 32, long chunks
     (2, 16, 16, 64, 1, [1, 1]),                 # MHA, head_dim 64, one row (code predictor)
     (1, 16, 16, 64, 300, [300]),                # MHA, head_dim 64
+    # the tensor-core kernel (B * Hkv * cap >= 2^16): one CTA per pair,
+    # clusters of 4 and of 8, 8 query heads per KV head, ragged last blocks
+    (32, 16, 8, 128, 2048, [2048, 1, 2047, 64, 65, 1000, 0, 2048] * 4),
+    (8, 16, 8, 128, 2048, [2048, 1, 2047, 63, 513, 1000, 2049, 1536]),
+    (4, 16, 2, 64, 8192, [8192, 1, 5000, 129]),
+    (1, 8, 1, 128, 65536, [65536]),
 ]
 
 
@@ -327,11 +333,12 @@ def test_decode_attention(B, H, Hkv, D, cap, lens):
         qg.qg_decode_attention(dev(q), bf16_dev(kbits), bf16_dev(vbits), dev(kv_len), out, H, Hkv,
                                1.0 / math.sqrt(D), ws)
         got = host64(out)
-        k64, v64 = O.bf16_bits_to_f64(kbits), O.bf16_bits_to_f64(vbits)
         for b in range(B):
             L = int(kv_len[b])
             if 1 <= L <= cap:
-                ref = O.decode_attention(q[b], k64[b], v64[b], L, H, Hkv, D)
+                k64 = O.bf16_bits_to_f64(kbits[b, :, :L])
+                v64 = O.bf16_bits_to_f64(vbits[b, :, :L])
+                ref = O.decode_attention(q[b], k64, v64, L, H, Hkv, D)
                 assert_parity(got[b], ref, bf16_out=(od == "bf16"), what=f"attn b={b} L={L}")
             else:
                 assert np.all(got[b] == 0.0)

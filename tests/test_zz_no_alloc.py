@@ -42,11 +42,14 @@ CALLS = [
 ]
 
 
-def _takes_split_kernel(H, Hkv, D):
-    """The library's rule: the cluster kernel serves head_dim 32/64/128/256
-    with at most 4 query heads per KV head; every other shape merges its
-    splits through the scratch."""
-    return not (D in (32, 64, 128, 256) and H // Hkv <= 4)
+def _takes_split_kernel(B, H, Hkv, D, cap):
+    """The library's rule: the tensor-core kernel serves head_dim 64/128 with
+    at most 8 query heads per KV head when B * Hkv * cap >= 2^16, the cluster
+    kernel head_dim 32/64/128/256 with at most 4; every other shape merges
+    its splits through the scratch."""
+    g = H // Hkv
+    mma = D in (64, 128) and g <= 8 and B * Hkv * cap >= 1 << 16
+    return not mma and not (D in (32, 64, 128, 256) and g <= 4)
 
 
 def _inputs(B, H, Hkv, D, cap, lens, seed):
@@ -58,7 +61,7 @@ def _inputs(B, H, Hkv, D, cap, lens, seed):
 
 def test_static_scratch_matches_workspace_entry_point_on_consecutive_calls():
     assert qg.qg_decode_attention_static_scratch_capacity() == 4 << 20
-    assert sum(_takes_split_kernel(c[1], c[2], c[3]) for c in CALLS) == 3
+    assert sum(_takes_split_kernel(c[0], c[1], c[2], c[3], c[4]) for c in CALLS) == 3
     for B, H, Hkv, D, cap, lens, seed, od in CALLS:
         kbits, vbits, q, kv_len = _inputs(B, H, Hkv, D, cap, lens, seed)
         qd, kd, vd, ld = dev(q), bf16_dev(kbits), bf16_dev(vbits), dev(kv_len)

@@ -19,6 +19,7 @@
 #include <mutex>
 
 #include "attention_body.cuh"
+#include "mma_sync.cuh"
 
 namespace qg {
 
@@ -492,6 +493,377 @@ attention_cluster_kernel(const float* q, const uint16_t* kc, const uint16_t* vc,
   tl_exit(fz.tl);
 }
 
+// ---------------------------------------------------------------------------
+// Tensor-core kernel for long caches and many sequences (head_dim 64 or 128,
+// at most 8 query heads per KV head).
+//
+// Same grid, clusters, row chunks, decode-step fusion and rank-order cluster
+// merge as the cluster kernel above; what changes is how a CTA scores its
+// rows. Blocks of 64 cached rows of K and V are staged in shared memory by
+// cp.async, three blocks in flight, 16-byte chunks XOR-swizzled by row so
+// that ldmatrix reads are conflict-free. Each of the 4 warps takes 16 rows
+// of a block: S = Q K^T and O += P V run on the tensor cores (mma.sync
+// m16n8k16, bf16 operands, fp32 accumulation) with the g query heads as the
+// A operand's first g rows. The fp32 query (normed, roped, times the scale)
+// and the fp32 softmax weights enter as bf16 pairs hi + lo with
+// hi = bf16(x), lo = bf16(x - hi), so |x - hi - lo| <= 2^-16 |x| and the
+// products keep fp32-grade accuracy; the online softmax (max, sum) is in fp32
+// per query head over the quad of lanes that holds its row.
+// ---------------------------------------------------------------------------
+
+constexpr int kMW = 4;                 // warps per CTA
+constexpr int kMThreads = kMW * 32;
+constexpr int kMB = 64;                // cached rows per staged block
+constexpr int kMStages = 3;            // blocks in flight
+constexpr int kMG = 8;                 // query heads per KV head, at most
+
+template <int D>
+constexpr int mma_smem_bytes() {
+  return kMStages * 2 * kMB * D * 2;   // [stage][K, V][kMB][D] bf16
+}
+
+template <int D>
+__global__ void __launch_bounds__(kMThreads, 2)
+attention_mma_kernel(const float* q, const uint16_t* kc, const uint16_t* vc,
+                     const int32_t* __restrict__ kv_len, const int32_t* __restrict__ pos_for_len,
+                     void* out, int out_bf16, int H, int Hkv, int cap, float scale, int ch,
+                     const AttnFuse fz) {
+  using namespace mm;
+  constexpr int KS = D / 16;           // k-steps of Q K^T
+  constexpr int CPR = D / 8;           // 16-byte chunks per row
+  constexpr int TILE = kMB * D * 2;    // bytes of one K or V block
+  extern __shared__ __align__(128) uint8_t stage[];
+  __shared__ float sq[kMG][D];         // query heads (normed, roped) * scale
+  __shared__ float kp[D], vp[D];       // the new row p (bf16 values), owner CTA only
+  __shared__ float sp[kMG];            // scores of row p
+  __shared__ float wm[kMW][kMG], wl[kMW][kMG];
+  __shared__ float cm[kMG], cl[kMG];   // this CTA's partial, read by rank 0
+  __shared__ float co[kMG][D];
+
+  tl_entry(fz.tl);
+  attn_issue_prefetch(fz);
+  const unsigned s = cluster_rank();
+  const unsigned cs = gridDim.x;
+  const int kv = blockIdx.y, b = blockIdx.z;
+  const int g = H / Hkv;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const size_t head_base = ((size_t)b * Hkv + kv) * cap;
+  const int t0 = (int)s * ch;
+
+  // cached rows this CTA scores: [t0, tend)
+  int tend = t0;
+  bool valid = false;
+  int p = -1;
+  if (fz.on) {
+    p = pos_for_len[b];
+    valid = p >= 0 && p < cap;
+    if (valid) tend = max(t0, min(t0 + ch, p));  // row p itself comes from shared memory
+  }
+  const uint32_t sbase = smem_u32(stage);
+  // block j of the chunk into stage buffer j % kMStages; rows at or past
+  // tend are zero-filled (their scores are masked to -inf)
+  auto load_block = [&](int j) {
+    const int tb = t0 + j * kMB;
+    const uint32_t kd = sbase + (uint32_t)((j % kMStages) * 2 * TILE);
+    const uint32_t vd = kd + TILE;
+#pragma unroll
+    for (int i = 0; i < kMB * CPR / kMThreads; ++i) {
+      const int idx = tid + i * kMThreads;
+      const int row = idx / CPR, c = idx % CPR;
+      const int t = tb + row;
+      const bool ok = t < tend;
+      const size_t off = (head_base + (ok ? t : 0)) * D + c * 8;
+      const uint32_t so = swz<D>(row, c * 8);
+      cp_async16(kd + so, kc + off, ok);
+      cp_async16(vd + so, vc + off, ok);
+    }
+  };
+  int nb = (tend - t0 + kMB - 1) / kMB;
+  auto prologue = [&] {
+#pragma unroll
+    for (int j = 0; j < kMStages - 1; ++j) {
+      if (j < nb) load_block(j);
+      cp_async_commit();
+    }
+  };
+  // decode step: the cached rows below the position are final, so the first
+  // blocks are in flight before the programmatic-dependent-launch wait
+  if (fz.on) prologue();
+  pdl_trigger();
+  pdl_wait();
+  tl_wait(fz.tl);
+  if (!fz.on) {
+    const int L = kv_len[b];
+    valid = L >= 1 && L <= cap;
+    tend = valid ? max(t0, min(t0 + ch, L)) : t0;
+    nb = (tend - t0 + kMB - 1) / kMB;
+    prologue();
+  }
+
+  // ---- query heads (and, in the decode step, the new K/V row)
+  const bool owner = fz.on && valid && p >= t0 && p < t0 + ch;
+  if (!fz.on) {
+    for (int i = tid; i < g * D; i += kMThreads)
+      sq[i / D][i % D] = __ldcg(q + ((size_t)b * H + kv * g + i / D) * D + i % D) * scale;
+  } else {
+    const int tk = fz.tok[b];
+    const bool write = owner && tk >= 0 && tk < fz.vocab;  // a bad token leaves the cache
+    const float2* rcs = fz.rope + (size_t)b * (D / 2);
+    const size_t row = (head_base + (valid ? p : 0)) * D;
+    // items 0..g-1: query heads; g: the new K row; g + 1: the new V row
+    for (int it = warp; it < g + 2; it += kMW) {
+      if (it < g) {
+        float* dst = sq[it];
+        norm_rope_head(q + ((size_t)b * H + kv * g + it) * D, fz.qn, D, fz.eps, rcs, lane,
+                       [&](int i, float v) { dst[i] = v * scale; });
+      } else if (it == g && owner) {
+        norm_rope_head(fz.k + ((size_t)b * Hkv + kv) * D, fz.kn, D, fz.eps, rcs, lane,
+                       [&](int i, float v) {
+                         const uint16_t bits = f32_to_bf16_bits(v);
+                         kp[i] = bf16_bits_to_f32(bits);
+                         if (write) const_cast<uint16_t*>(kc)[row + i] = bits;
+                       });
+      } else if (it == g + 1 && owner) {
+        const float* vs = fz.v + ((size_t)b * Hkv + kv) * D;
+        for (int d = lane; d < D; d += 32) {
+          const uint16_t bits = f32_to_bf16_bits(__ldcg(vs + d));
+          vp[d] = bf16_bits_to_f32(bits);
+          if (write) const_cast<uint16_t*>(vc)[row + d] = bits;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (owner) {  // score of row p for each query head
+    for (int h = warp; h < g; h += kMW) {
+      float d = 0.f;
+      for (int i = lane; i < D; i += 32) d = fmaf(sq[h][i], kp[i], d);
+      d = warp_sum(d);
+      if (lane == 0) sp[h] = d;
+    }
+  }
+
+  // ---- A fragments of Q: row qr = lane / 4 (a query head when qr < g; rows
+  // 8..15 of the m16 tile are zero), columns 16 ks + 2 (lane % 4) + {0, 1}
+  // and + 8, as hi and lo bf16 pairs
+  const int qr = lane >> 2, qc = (lane & 3) * 2;
+  uint32_t qhi[KS][2], qlo[KS][2];
+#pragma unroll
+  for (int ks = 0; ks < KS; ++ks) {
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      const int d = ks * 16 + hf * 8 + qc;
+      const float x0 = qr < g ? sq[qr][d] : 0.f, x1 = qr < g ? sq[qr][d + 1] : 0.f;
+      const float h0 = bf16r(x0), h1 = bf16r(x1);
+      qhi[ks][hf] = pack_bf16(h0, h1);
+      qlo[ks][hf] = pack_bf16(x0 - h0, x1 - h1);
+    }
+  }
+
+  // ---- this warp's 16 rows of each block: online softmax of query head qr
+  float o[D / 8][4];
+#pragma unroll
+  for (int j = 0; j < D / 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+  float m_run = -INFINITY, l_run = 0.f;  // l_run: this lane's share of the sum
+  for (int j = 0; j < nb; ++j) {
+    cp_async_wait<kMStages - 2>();
+    __syncthreads();  // block j landed for every thread; buffer (j - 1) % kMStages is free
+    if (j + kMStages - 1 < nb) load_block(j + kMStages - 1);
+    cp_async_commit();
+    const uint32_t kb = sbase + (uint32_t)((j % kMStages) * 2 * TILE);
+    const uint32_t vb = kb + TILE;
+
+    // S = Q K^T over rows warp*16 + [0, 16): n-tiles of 8 rows; ldmatrix
+    // (no transpose) of K rows gives the col-major B fragment directly
+    float sacc[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < KS; ks += 2) {
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        const int row = warp * 16 + nt * 8 + (lane & 7);
+        uint32_t r0, r1, r2, r3;
+        ldsm_x4(kb + swz<D>(row, (ks * 2 + (lane >> 3)) * 8), r0, r1, r2, r3);
+        mma_bf16(sacc[nt], qhi[ks][0], 0u, qhi[ks][1], 0u, r0, r1);
+        mma_bf16(sacc[nt], qlo[ks][0], 0u, qlo[ks][1], 0u, r0, r1);
+        mma_bf16(sacc[nt], qhi[ks + 1][0], 0u, qhi[ks + 1][1], 0u, r2, r3);
+        mma_bf16(sacc[nt], qlo[ks + 1][0], 0u, qlo[ks + 1][1], 0u, r2, r3);
+      }
+    }
+    // this lane's scores: rows t0 + j*kMB + warp*16 + nt*8 + qc + {0, 1}
+    const int tb = t0 + j * kMB + warp * 16 + qc;
+    float sv[4];
+    float mx = -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float v = tb + nt * 8 + e < tend ? sacc[nt][e] : -INFINITY;
+        sv[nt * 2 + e] = v;
+        mx = fmaxf(mx, v);
+      }
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    const float mnew = fmaxf(m_run, mx);
+    float pr[4] = {0.f, 0.f, 0.f, 0.f};
+    if (mnew != -INFINITY) {
+      const float a = expf(m_run - mnew);  // 0 while m_run is still -inf
+      l_run *= a;
+#pragma unroll
+      for (int dn = 0; dn < D / 8; ++dn) {
+        o[dn][0] *= a;
+        o[dn][1] *= a;
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) pr[i] = expf(sv[i] - mnew);  // masked rows: 0
+      l_run += (pr[0] + pr[1]) + (pr[2] + pr[3]);
+      m_run = mnew;
+    }
+    // O += P V: P's A fragment is the score layout (columns qc + {0,1} of
+    // n-tile 0, then of n-tile 1); ldmatrix.trans of V rows gives the B
+    // fragment (k = row, n = column of the head)
+    const float h0 = bf16r(pr[0]), h1 = bf16r(pr[1]), h2 = bf16r(pr[2]), h3 = bf16r(pr[3]);
+    const uint32_t pa_h = pack_bf16(h0, h1), pb_h = pack_bf16(h2, h3);
+    const uint32_t pa_l = pack_bf16(pr[0] - h0, pr[1] - h1), pb_l = pack_bf16(pr[2] - h2, pr[3] - h3);
+#pragma unroll
+    for (int dn = 0; dn < D / 8; dn += 2) {
+      const int row = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+      uint32_t r0, r1, r2, r3;
+      ldsm_x4_t(vb + swz<D>(row, (dn + (lane >> 4)) * 8), r0, r1, r2, r3);
+      mma_bf16(o[dn], pa_h, 0u, pb_h, 0u, r0, r1);
+      mma_bf16(o[dn], pa_l, 0u, pb_l, 0u, r0, r1);
+      mma_bf16(o[dn + 1], pa_h, 0u, pb_h, 0u, r2, r3);
+      mma_bf16(o[dn + 1], pa_l, 0u, pb_l, 0u, r2, r3);
+    }
+  }
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+
+  // ---- the warps' states to shared memory; wo [kMW][kMG][D] reuses the
+  // staging buffers once every copy has landed and every warp is done
+  cp_async_wait<0>();
+  __syncthreads();
+  float* wo = reinterpret_cast<float*>(stage);
+  if (qr < g) {
+#pragma unroll
+    for (int dn = 0; dn < D / 8; ++dn) {
+      wo[(warp * kMG + qr) * D + dn * 8 + qc] = o[dn][0];
+      wo[(warp * kMG + qr) * D + dn * 8 + qc + 1] = o[dn][1];
+    }
+    if ((lane & 3) == 0) {
+      wm[warp][qr] = m_run;
+      wl[warp][qr] = l_run;
+    }
+  }
+  __syncthreads();
+
+  // ---- this CTA's partial: its warps in order, then row p
+  for (int i = tid; i < g * D; i += kMThreads) {
+    const int h = i / D, d = i % D;
+    float M = owner ? sp[h] : -INFINITY;
+    for (int w = 0; w < kMW; ++w) M = fmaxf(M, wm[w][h]);
+    float Ls = 0.f, O = 0.f;
+    if (M != -INFINITY) {
+      for (int w = 0; w < kMW; ++w) {
+        const float e = wm[w][h] == -INFINITY ? 0.f : expf(wm[w][h] - M);
+        Ls = fmaf(wl[w][h], e, Ls);
+        O = fmaf(wo[(w * kMG + h) * D + d], e, O);
+      }
+      if (owner) {
+        const float e = expf(sp[h] - M);
+        Ls += e;
+        O = fmaf(vp[d], e, O);
+      }
+    }
+    co[h][d] = O;
+    if (d == 0) {
+      cm[h] = M;
+      cl[h] = Ls;
+    }
+  }
+  cluster_sync();  // every CTA's partial is in its shared memory
+
+  // ---- rank 0 merges the cluster's partials in rank order
+  if (s == 0) {
+    for (int i = tid; i < g * D; i += kMThreads) {
+      const int h = i / D, d = i % D;
+      float M = -INFINITY;
+      for (unsigned r = 0; r < cs; ++r) M = fmaxf(M, ld_cluster(&cm[h], r));
+      float Ls = 0.f, O = 0.f;
+      if (M != -INFINITY) {
+        for (unsigned r = 0; r < cs; ++r) {
+          const float mr = ld_cluster(&cm[h], r);
+          if (mr == -INFINITY) continue;
+          const float e = expf(mr - M);
+          Ls = fmaf(ld_cluster(&cl[h], r), e, Ls);
+          O = fmaf(ld_cluster(&co[h][d], r), e, O);
+        }
+      }
+      const float res = (valid && Ls > 0.f) ? O / Ls : 0.f;
+      const size_t oi = ((size_t)b * H + kv * g + h) * D + d;
+      if (out_bf16)
+        reinterpret_cast<uint16_t*>(out)[oi] = f32_to_bf16_bits(res);
+      else
+        reinterpret_cast<float*>(out)[oi] = res;
+    }
+  }
+  cluster_sync();  // no CTA leaves while rank 0 still reads its shared memory
+  tl_exit(fz.tl);
+}
+
+// Whether the tensor-core kernel takes the shape: head_dim 64 or 128, at
+// most 8 query heads per KV head, and at least 2^16 cached rows over all
+// (sequence, kv head) pairs (below that the cluster kernel's lighter
+// prologue wins).
+constexpr long long kMmaMinRows = 1LL << 16;
+inline bool mma_ok(int B, int H, int Hkv, int D, int cap) {
+  if (!(D == 64 || D == 128) || Hkv < 1 || H % Hkv != 0) return false;
+  const int g = H / Hkv;
+  if (g < 1 || g > kMG) return false;
+  return (long long)B * Hkv * cap >= kMmaMinRows;
+}
+
+// CTAs per (sequence, kv head) for the tensor-core kernel: as many as fit
+// in one wave of two CTAs per SM (at most 8, a portable cluster), each a
+// whole number of 64-row blocks; `ch` = rows per CTA.
+inline void mma_plan(int B, int Hkv, int cap, int& cs, int& ch) {
+  const long long pairs = (long long)B * Hkv;
+  long long c = (2LL * num_sms()) / pairs;
+  c = std::max<long long>(1, std::min<long long>(c, kMaxCluster));
+  const int blocks = (cap + kMB - 1) / kMB;
+  c = std::min<long long>(c, blocks);
+  ch = (int)((blocks + c - 1) / c) * kMB;
+  cs = (cap + ch - 1) / ch;
+}
+
+template <int D>
+cudaError_t launch_mma(const float* q, const uint16_t* kc, const uint16_t* vc,
+                       const int32_t* kv_len, const int32_t* pos_for_len, void* out,
+                       bool out_bf16, int B, int H, int Hkv, int cap, float scale,
+                       cudaStream_t st, bool pdl, const AttnFuse& fz) {
+  int cs = 1, ch = cap;
+  mma_plan(B, Hkv, cap, cs, ch);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(cs, Hkv, B);
+  cfg.blockDim = dim3(kMThreads);
+  cfg.dynamicSmemBytes = mma_smem_bytes<D>();
+  ensure_smem((const void*)attention_mma_kernel<D>, (int)cfg.dynamicSmemBytes);
+  cfg.stream = st;
+  cudaLaunchAttribute a[2];
+  a[0].id = cudaLaunchAttributeClusterDimension;
+  a[0].val.clusterDim.x = cs;
+  a[0].val.clusterDim.y = 1;
+  a[0].val.clusterDim.z = 1;
+  a[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  a[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = a;
+  cfg.numAttrs = pdl ? 2 : 1;
+  count_launch();
+  return cudaLaunchKernelEx(&cfg, attention_mma_kernel<D>, q, kc, vc, kv_len, pos_for_len, out,
+                            (int)out_bf16, H, Hkv, cap, scale, ch, fz);
+}
+
 // Whether the cluster kernel takes the shape.
 inline bool cluster_ok(int H, int Hkv, int D) {
   const int g = H / Hkv;
@@ -585,6 +957,13 @@ static cudaError_t attention_launch_any(const float* q, const uint16_t* kc, cons
                                         void* out, bool out_bf16, int B, int H, int Hkv, int D,
                                         int cap, float scale, void* ws, cudaStream_t st, bool pdl,
                                         const AttnFuse& fz) {
+  if (!fz.ow && ac::mma_ok(B, H, Hkv, D, cap)) {
+    if (D == 64)
+      return ac::launch_mma<64>(q, kc, vc, kv_len, pos_for_len, out, out_bf16, B, H, Hkv, cap,
+                                scale, st, pdl, fz);
+    return ac::launch_mma<128>(q, kc, vc, kv_len, pos_for_len, out, out_bf16, B, H, Hkv, cap,
+                               scale, st, pdl, fz);
+  }
   if (ac::cluster_ok(H, Hkv, D)) {
     switch (D) {
       case 32:
@@ -670,7 +1049,7 @@ cudaError_t attention_launch_step(const float* q, const float* k, const float* v
 }
 
 bool attention_oproj_fusable(int B, int H, int Hkv, int D, int cap, int hidden) {
-  if (!ac::cluster_ok(H, Hkv, D)) return false;
+  if (!ac::cluster_ok(H, Hkv, D) || ac::mma_ok(B, H, Hkv, D, cap)) return false;
   return ac::oproj_ok(hidden, ac::cluster_size(B, Hkv, cap), (H / Hkv) * D);
 }
 
@@ -787,9 +1166,10 @@ extern "C" qg_status qg_decode_attention_static_scratch(const float* q, const ui
   clear_error();
   qg_status st = validate_attention(q, k_cache, v_cache, kv_len, out, out_dtype, B, H, Hkv, D, cap);
   if (st != QG_OK || B == 0) return st;
-  // Only the split kernel touches scratch; the cluster kernel merges through
-  // distributed shared memory, so its shapes are not limited by the array.
-  const bool split = !ac::cluster_ok(H, Hkv, D);
+  // Only the split kernel touches scratch; the cluster and tensor-core
+  // kernels merge through distributed shared memory, so their shapes are not
+  // limited by the array.
+  const bool split = !ac::cluster_ok(H, Hkv, D) && !ac::mma_ok(B, H, Hkv, D, cap);
   if (split) {
     const size_t need = attention_ws_bytes(B, H, Hkv, D, cap);
     QG_REQUIRE(need <= kAttnStaticScratchBytes, QG_ERR_WORKSPACE_TOO_SMALL,
