@@ -160,7 +160,12 @@ __device__ __forceinline__ void gemv_tc_body(const Params& P, uint8_t* smem, Wai
   constexpr int kWarps = W, kThreads = W * 32;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
-  const int K = P.K, Kg = K / 64, nsc = K / kSC, S = P.S;
+  const int K = P.K, Kg = K / 64, nsc = K / kSC;
+  // S <= nsc gives every warp of a team at least one super-chunk, so all S
+  // warps of the team meet at its named barrier once per block (a warp with
+  // none would skip the loop and leave the others waiting)
+  int S = P.S;
+  while (S > 1 && S > nsc) S >>= 1;
   // batch tile of this CTA: rows [b0, b0 + Bt) of the launch's P.B
   const int b0 = blockIdx.y * 4 * NT, Bt = min(4 * NT, P.B - b0);
   const int xs = K + 8;  // fp16 row stride of x (pad: batch rows on other banks)
@@ -510,7 +515,7 @@ inline size_t gtc_smem(int K, int NT, int W) {
 __host__ __device__ inline int gtc_split(int nblocks, int K, int W, int sms) {
   const int nsc = K / gtc::kSC;
   int S = 1;
-  while (S < W && S < nsc && (long long)nblocks * 2 * S <= (long long)sms * W) S *= 2;
+  while (2 * S <= W && 2 * S <= nsc && (long long)nblocks * 2 * S <= (long long)sms * W) S *= 2;
   return S;
 }
 
