@@ -612,7 +612,7 @@ qg_status qg_layernorm(const float* x, const float* gamma, const float* beta, fl
  * rounded to bf16 for the weighted sum of V (and summed as rounded), out is
  * rounded to bf16. All pointers 16-byte aligned.
  * Shape rules: D = 64 or 128, H % Hkv == 0, causal needs T <= S; S = 0
- * gives zero rows.
+ * gives zero rows (k and v are then not read and may be NULL).
  * ---------------------------------------------------------------------- */
 qg_status qg_attention_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                             uint16_t* out, int B, int T, int S, int H, int Hkv, int D,

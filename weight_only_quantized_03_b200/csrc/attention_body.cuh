@@ -50,7 +50,9 @@ __device__ __forceinline__ void attn_issue_prefetch(const AttnFuse& fz) {
 // RMSNorm of one head row src[0..D) with weight w, then the NeoX rotation
 // with the (cos, sin) pairs cs[0..D/2); lane owns the pairs (i, i + D/2) for
 // i = lane + 32 j. Writes the rotated fp32 values through `put(i, value)`.
-template <typename Put>
+// The table is read through L2 (it is written by an earlier kernel) unless
+// kSharedCs, when it sits in this CTA's shared memory.
+template <bool kSharedCs = false, typename Put>
 __device__ __forceinline__ void norm_rope_head(const float* src, const uint16_t* w, int D, float eps,
                                                const float2* cs, int lane, Put put) {
   const int half = D >> 1;
@@ -71,7 +73,7 @@ __device__ __forceinline__ void norm_rope_head(const float* src, const uint16_t*
     if (i >= half) break;
     const float a = x1[j] * inv * bf16_bits_to_f32(w[i]);
     const float c2 = x2[j] * inv * bf16_bits_to_f32(w[i + half]);
-    const float2 r = __ldcg(cs + i);
+    const float2 r = kSharedCs ? cs[i] : __ldcg(cs + i);
     put(i, a * r.x - c2 * r.y);
     put(i + half, c2 * r.x + a * r.y);
   }

@@ -242,7 +242,9 @@ extern "C" qg_status qg_attention_rows(const uint16_t* q, const uint16_t* k, con
   QG_REQUIRE((long long)B * S * Hkv * D < (1LL << 40) && (long long)B * T * H * D < (1LL << 40),
              QG_ERR_UNSUPPORTED_SHAPE, "qg_attention_rows: too large");
   if (B == 0 || T == 0) return QG_OK;
-  QG_REQUIRE(q && k && v && out, QG_ERR_INVALID_ARGUMENT, "qg_attention_rows: null pointer");
+  // with no keys (S = 0) k and v are never read and may be NULL
+  QG_REQUIRE(q && out && (S == 0 || (k && v)), QG_ERR_INVALID_ARGUMENT,
+             "qg_attention_rows: null pointer");
   QG_REQUIRE(aligned(q, 16) && aligned(k, 16) && aligned(v, 16) && aligned(out, 16),
              QG_ERR_MISALIGNED, "qg_attention_rows: q, k, v and out must be 16-byte aligned");
   ar::Params P = {};

@@ -48,12 +48,12 @@ __global__ void __launch_bounds__(256)
   const bool write = tk >= 0 && tk < vocab;
   if (j < H) {
     uint16_t* dst = qb + ((size_t)t * H + j) * D;
-    norm_rope_head(q + ((size_t)t * H + j) * D, qn, D, eps, cs, lane,
+    norm_rope_head<true>(q + ((size_t)t * H + j) * D, qn, D, eps, cs, lane,
                    [&](int i, float r) { dst[i] = f32_to_bf16_bits(r); });
   } else if (j < H + Hkv) {
     const int h = j - H;
     uint16_t* dst = kc + ((size_t)h * cap + pos) * D;
-    norm_rope_head(k + ((size_t)t * Hkv + h) * D, kn, D, eps, cs, lane, [&](int i, float r) {
+    norm_rope_head<true>(k + ((size_t)t * Hkv + h) * D, kn, D, eps, cs, lane, [&](int i, float r) {
       if (write) dst[i] = f32_to_bf16_bits(r);
     });
   } else if (j < H + 2 * Hkv) {

@@ -110,7 +110,11 @@ __device__ __forceinline__ void l2_prefetch_range(const void* p, unsigned long l
 
 // Issued by one thread of each CTA (part = its CTA index among `parts`).
 // The positions are inputs of the step, final before its first kernel runs.
+// QG_NO_L2_PREFETCH builds the library without these hints.
 __device__ __forceinline__ void issue_prefetch(const Prefetch& pf, unsigned part, unsigned parts) {
+#ifdef QG_NO_L2_PREFETCH
+  return;
+#endif
   for (int r = 0; r < pf.n; ++r) l2_prefetch_range(pf.r[r].p, pf.r[r].bytes, part, parts);
   if (pf.kv.kc) {
     const int ranges = 2 * pf.kv.B * pf.kv.Hkv;  // (sequence, kv head) x (K, V)
