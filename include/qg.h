@@ -680,7 +680,7 @@ qg_status qg_whisper_encoder_layer_inspect(const qg_whisper_config* cfg, int M,
  * four uint64 per launch -- the bitwise complement of the earliest CTA
  * entry, the latest return from the wait for the previous kernel, the
  * latest CTA exit (all %globaltimer nanoseconds, maxima over the launch's
- * CTAs), and a reserved zero. qg_timeline_end stops recording, copies the
+ * CTAs), and the latest CTA entry. qg_timeline_end stops recording, copies the
  * launch kinds (1 embedding, 2 q/k/v GEMV, 3 attention, 4 o_proj, 5 gate/up,
  * 6 down, 7 output head, 8 other) of the first max_kinds launches to kinds
  * (host, may be NULL) and returns the number of launches recorded.

@@ -280,15 +280,12 @@ def test_invalid_token_or_position_gives_nan_and_leaves_cache():
 
 
 @pytest.mark.parametrize("shape,B,cap,per_layer", [("small", 1, 16, 5), ("0.6b", 4, 16, 5),
-                                                   ("0.6b", 1, 520, 4), ("0.6b", 8, 520, 4)])
+                                                   ("0.6b", 1, 520, 5), ("0.6b", 8, 520, 5)])
 def test_step_launch_count(shape, B, cap, per_layer):
     """One step is the embedding, the LM head and per layer: 5 launches
     (the fused stages; no separate norm or SiLU-mul kernels where the
-    tensor-core GEMV takes the shapes); 4 where o_proj folds into the
-    attention kernel (a cluster of 8 CTAs per KV head, 128 rows of W_o
-    each: a cache of 128 rows or more and up to about 20 sequences); past 4
-    sequences the LM head is a norm plus a tensor-core matmul (one launch
-    more)."""
+    tensor-core GEMV takes the shapes); past 4 sequences the LM head is a
+    norm plus a tensor-core matmul (one launch more)."""
     cfg = dict(SMALL) if shape == "small" else dict(qg_synth.QWEN3_0_6B)
     cfg["layers"] = min(cfg["layers"], 2)
     model = qg.Qwen3Model(cfg, qg_synth.qwen3_weights(cfg, 23))

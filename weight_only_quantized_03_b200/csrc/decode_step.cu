@@ -222,11 +222,14 @@ static Prefetch pf_kv(const qg_qwen3_config& c, const uint16_t* kc, const uint16
 constexpr int kStepGemmBatch = 5;
 
 // o_proj folded into the attention kernel (one launch fewer per layer) where
-// the shapes allow it; QG_NO_FUSE_OPROJ keeps it a GEMV launch of its own.
-#ifdef QG_NO_FUSE_OPROJ
-constexpr bool kStepFuseOProj = false;
-#else
+// the shapes allow it: built only with QG_FUSE_OPROJ. Measured on the B200
+// (0.6B shape, batch 1, KV 512) the folded attention launch took 21 us
+// against 8.5 us for attention plus 4.8 us for the o_proj GEMV, so by
+// default o_proj stays a GEMV launch of its own.
+#ifdef QG_FUSE_OPROJ
 constexpr bool kStepFuseOProj = true;
+#else
+constexpr bool kStepFuseOProj = false;
 #endif
 
 static bool head_uses_gemm(const qg_qwen3_config& c, int N, int B) {

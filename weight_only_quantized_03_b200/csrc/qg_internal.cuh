@@ -110,9 +110,13 @@ __device__ __forceinline__ void l2_prefetch_range(const void* p, unsigned long l
 
 // Issued by one thread of each CTA (part = its CTA index among `parts`).
 // The positions are inputs of the step, final before its first kernel runs.
-// QG_NO_L2_PREFETCH builds the library without these hints.
+// Issued only in a library built with QG_L2_PREFETCH: measured on the B200
+// (0.6B decode step, batch 1) the hints made no kernel of the chain faster,
+// since each kernel already issues its first weight loads before its
+// programmatic-dependent-launch wait, and the embedding kernel's share
+// (layer 0's q/k/v, 4 MB from a few SMs) cost 25 us.
 __device__ __forceinline__ void issue_prefetch(const Prefetch& pf, unsigned part, unsigned parts) {
-#ifdef QG_NO_L2_PREFETCH
+#ifndef QG_L2_PREFETCH
   return;
 #endif
   for (int r = 0; r < pf.n; ++r) l2_prefetch_range(pf.r[r].p, pf.r[r].bytes, part, parts);
@@ -135,9 +139,10 @@ __device__ __forceinline__ void issue_prefetch(const Prefetch& pf, unsigned part
 // records; otherwise the hooks compile to nothing. Each record is filled
 // with atomic maxima over the launch's CTAs (zero-initialised by the
 // caller): the earliest CTA entry (stored as its bitwise complement), the
-// latest return from the wait for the previous kernel, the latest exit.
+// latest return from the wait for the previous kernel, the latest exit, the
+// latest CTA entry.
 struct TlRec {
-  unsigned long long neg_entry, wait, exit, reserved;
+  unsigned long long neg_entry, wait, exit, last_entry;
 };
 
 // Host side: the record for the next launch (nullptr when not recording).
@@ -153,7 +158,11 @@ __device__ __forceinline__ unsigned long long global_ns() {
 }
 #ifdef QG_TIMELINE
 __device__ __forceinline__ void tl_entry(TlRec* r) {
-  if (r && threadIdx.x == 0) atomicMax(&r->neg_entry, ~global_ns());
+  if (r && threadIdx.x == 0) {
+    const unsigned long long t = global_ns();
+    atomicMax(&r->neg_entry, ~t);
+    atomicMax(&r->last_entry, t);
+  }
 }
 __device__ __forceinline__ void tl_wait(TlRec* r) {
   if (r && threadIdx.x == 0) atomicMax(&r->wait, global_ns());
