@@ -49,7 +49,7 @@ namespace qg {
 namespace gtc {
 
 template <int NT, int W>
-__global__ void __launch_bounds__(W * 32, NT == 1 ? 512 / (W * 32) : 1)
+__global__ void __launch_bounds__(W * 32, 1)
     gemv_tc_kernel(const __grid_constant__ Params P) {
   extern __shared__ __align__(16) uint8_t smem[];
   tl_entry(P.tl);
@@ -101,10 +101,13 @@ static cudaError_t gtc_launch(const GemvSeg* segs, int nseg, gtc::Params& P, int
   P.nblocks = blk;
   if (blk == 0) return cudaSuccess;
   // One batch tile (B <= 4): 16 warps for matrices that stream (more
-  // 16-row blocks than warp slots at 8 warps a CTA), 8 warps for the
-  // matrices of a decode layer, whose weights then all go out before the
-  // wait and whose CTAs leave room on each SM for the next kernel's CTA.
-  // Two batch tiles: 8 warps (about 255 registers a thread). Batch tiles of
+  // 16-row blocks than warp slots at 8 warps a CTA; 128 registers a thread),
+  // 8 warps for the matrices of a decode layer, whose weights then all go
+  // out before the wait. The 8-warp kernel takes the registers it needs
+  // (about 234, no spills) at one CTA per SM: measured on the B200 in the
+  // 0.6B step at batch 1, 813 us a step against 937 us when capped at 128
+  // registers (two CTAs per SM, 136 bytes of spills a thread). Two batch
+  // tiles: 8 warps (about 255 registers a thread). Batch tiles of
   // 8 rows along gridDim.y past B = 8: the tiles stream the same weights at
   // about the same time, so all but the first mostly hit L2.
   const int NT = B > 4 ? 2 : 1;

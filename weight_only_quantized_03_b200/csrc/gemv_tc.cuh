@@ -7,9 +7,10 @@
 namespace qg {
 namespace gtc {
 
-// Warps per CTA (template W): 16 with one batch tile (128 registers a
-// thread, the whole register file: the most loads in flight), 8 with two
-// batch tiles (about 255 registers a thread).
+// Warps per CTA (template W): 16 with one batch tile for streaming matrices
+// (128 registers a thread, the whole register file: the most loads in
+// flight); 8 for decode-layer matrices (one batch tile, about 234 registers)
+// and with two batch tiles (about 255).
 constexpr int kRB = 16;        // rows per block (mma M)
 constexpr int kSC = 512;       // columns per super-chunk
 constexpr int kMaxSegs = 4;
