@@ -153,6 +153,39 @@ __device__ __forceinline__ void merge_state(float& m, float& l, float* o, float 
   m = M;
 }
 
+// One output element from the cluster's partials, merged in rank order:
+// every rank's (max, sum, weighted value) is loaded first, so the reads of
+// distributed shared memory overlap in one round trip, then combined. An
+// empty rank has max -inf.
+__device__ __forceinline__ float merge_cluster(const float* m, const float* l, const float* o,
+                                               unsigned cs, bool valid) {
+  float mv[kMaxCluster], lv[kMaxCluster], ov[kMaxCluster];
+#pragma unroll
+  for (int j = 0; j < kMaxCluster; ++j) {
+    mv[j] = -INFINITY;
+    lv[j] = ov[j] = 0.f;
+    if (j < (int)cs) {
+      mv[j] = ld_cluster(m, j);
+      lv[j] = ld_cluster(l, j);
+      ov[j] = ld_cluster(o, j);
+    }
+  }
+  float M = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < kMaxCluster; ++j) M = fmaxf(M, mv[j]);
+  float Ls = 0.f, O = 0.f;
+  if (M != -INFINITY) {
+#pragma unroll
+    for (int j = 0; j < kMaxCluster; ++j) {
+      if (mv[j] == -INFINITY) continue;
+      const float e = expf(mv[j] - M);
+      Ls = fmaf(lv[j], e, Ls);
+      O = fmaf(ov[j], e, O);
+    }
+  }
+  return (valid && Ls > 0.f) ? O / Ls : 0.f;
+}
+
 // 4-byte cp.async granule helpers for the fused o_proj slice
 __device__ __forceinline__ void cp_async_16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
@@ -435,19 +468,7 @@ attention_cluster_kernel(const float* q, const uint16_t* kc, const uint16_t* vc,
   if (s == 0) {
     for (int i = threadIdx.x; i < g * D; i += kThreads) {
       const int h = i / D, d = i % D;
-      float M = -INFINITY;
-      for (unsigned j = 0; j < cs; ++j) M = fmaxf(M, ld_cluster(&cm[h], j));
-      float Ls = 0.f, O = 0.f;
-      if (M != -INFINITY) {
-        for (unsigned j = 0; j < cs; ++j) {
-          const float mj = ld_cluster(&cm[h], j);
-          if (mj == -INFINITY) continue;
-          const float e = expf(mj - M);
-          Ls = fmaf(ld_cluster(&cl[h], j), e, Ls);
-          O = fmaf(ld_cluster(&co[h][d], j), e, O);
-        }
-      }
-      const float res = (valid && Ls > 0.f) ? O / Ls : 0.f;
+      const float res = merge_cluster(&cm[h], &cl[h], &co[h][d], cs, valid);
       const size_t oi = ((size_t)b * H + kv * g + h) * D + d;
       if (out_bf16)
         reinterpret_cast<uint16_t*>(out)[oi] = f32_to_bf16_bits(res);
@@ -788,19 +809,7 @@ attention_mma_kernel(const float* q, const uint16_t* kc, const uint16_t* vc,
   if (s == 0) {
     for (int i = tid; i < g * D; i += kMThreads) {
       const int h = i / D, d = i % D;
-      float M = -INFINITY;
-      for (unsigned r = 0; r < cs; ++r) M = fmaxf(M, ld_cluster(&cm[h], r));
-      float Ls = 0.f, O = 0.f;
-      if (M != -INFINITY) {
-        for (unsigned r = 0; r < cs; ++r) {
-          const float mr = ld_cluster(&cm[h], r);
-          if (mr == -INFINITY) continue;
-          const float e = expf(mr - M);
-          Ls = fmaf(ld_cluster(&cl[h], r), e, Ls);
-          O = fmaf(ld_cluster(&co[h][d], r), e, O);
-        }
-      }
-      const float res = (valid && Ls > 0.f) ? O / Ls : 0.f;
+      const float res = merge_cluster(&cm[h], &cl[h], &co[h][d], cs, valid);
       const size_t oi = ((size_t)b * H + kv * g + h) * D + d;
       if (out_bf16)
         reinterpret_cast<uint16_t*>(out)[oi] = f32_to_bf16_bits(res);

@@ -56,26 +56,32 @@ template <bool kSharedCs = false, typename Put>
 __device__ __forceinline__ void norm_rope_head(const float* src, const uint16_t* w, int D, float eps,
                                                const float2* cs, int lane, Put put) {
   const int half = D >> 1;
-  float x1[4], x2[4];
-  float ss = 0.f;
+  // the row, its norm weights and its (cos, sin) pairs in one round of loads
+  float x1[4], x2[4], w1[4], w2[4];
+  float2 r[4];
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const int i = lane + 32 * j;
-    x1[j] = i < half ? __ldcg(src + i) : 0.f;
-    x2[j] = i < half ? __ldcg(src + i + half) : 0.f;
-    ss = fmaf(x1[j], x1[j], fmaf(x2[j], x2[j], ss));
+    const bool in = i < half;
+    x1[j] = in ? __ldcg(src + i) : 0.f;
+    x2[j] = in ? __ldcg(src + i + half) : 0.f;
+    w1[j] = in ? bf16_bits_to_f32(w[i]) : 0.f;
+    w2[j] = in ? bf16_bits_to_f32(w[i + half]) : 0.f;
+    r[j] = in ? (kSharedCs ? cs[i] : __ldcg(cs + i)) : make_float2(0.f, 0.f);
   }
+  float ss = 0.f;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) ss = fmaf(x1[j], x1[j], fmaf(x2[j], x2[j], ss));
   ss = warp_sum(ss);
   const float inv = 1.0f / sqrtf(ss / (float)D + eps);
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const int i = lane + 32 * j;
     if (i >= half) break;
-    const float a = x1[j] * inv * bf16_bits_to_f32(w[i]);
-    const float c2 = x2[j] * inv * bf16_bits_to_f32(w[i + half]);
-    const float2 r = kSharedCs ? cs[i] : __ldcg(cs + i);
-    put(i, a * r.x - c2 * r.y);
-    put(i + half, c2 * r.x + a * r.y);
+    const float a = x1[j] * inv * w1[j];
+    const float c2 = x2[j] * inv * w2[j];
+    put(i, a * r[j].x - c2 * r[j].y);
+    put(i + half, c2 * r[j].x + a * r[j].y);
   }
 }
 

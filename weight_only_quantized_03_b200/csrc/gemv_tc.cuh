@@ -170,8 +170,11 @@ __device__ __forceinline__ void gemv_tc_body(const Params& P, uint8_t* smem, Wai
   // batch tile of this CTA: rows [b0, b0 + Bt) of the launch's P.B
   const int b0 = blockIdx.y * 4 * NT, Bt = min(4 * NT, P.B - b0);
   const int xs = K + 8;  // fp16 row stride of x (pad: batch rows on other banks)
+  // regions in floats, each a multiple of 4 (16 bytes): xh is read with
+  // 16-byte loads, so it must start on a 16-byte boundary for any W
+  constexpr int kRed = ((4 * NT + 1) * kWarps + 3) & ~3;
   float* red = reinterpret_cast<float*>(smem);                      // [4 NT + 1][kWarps]
-  float* part = red + (4 * NT + 1) * kWarps;                         // [2][kWarps][32][2 NT]
+  float* part = red + kRed;                                          // [2][kWarps][32][2 NT]
   float* gsum = part + 2 * kWarps * 32 * 2 * NT;                    // [4 NT][Kg]
   uint16_t* xh = reinterpret_cast<uint16_t*>(gsum + 4 * NT * Kg);   // [4 NT][xs]
 
@@ -504,7 +507,7 @@ __device__ __forceinline__ void gemv_tc_body(const Params& P, uint8_t* smem, Wai
 
 // dynamic shared memory of gemv_tc_body
 inline size_t gtc_smem(int K, int NT, int W) {
-  return (size_t)(4 * NT + 1) * W * 4 + (size_t)2 * W * 32 * 2 * NT * 4 +
+  return (size_t)(((4 * NT + 1) * W + 3) & ~3) * 4 + (size_t)2 * W * 32 * 2 * NT * 4 +
          (size_t)4 * NT * (K / 64) * 4 + (size_t)4 * NT * (K + 8) * 2;
 }
 
