@@ -42,7 +42,9 @@ def _cuda():
                                             (5, 300, 128, True, False),
                                             (17, 384, 1024, False, True),
                                             (1, 1024, 3072, False, False),
-                                            (32, 3072, 1024, True, False)])
+                                            (32, 3072, 1024, True, False),
+                                            (16, 1000, 2048, True, False),
+                                            (1, 300, 64, False, True)])
 def test_gemm_affine8(T, N, K, res, bf16):
     w, s, b = qg_synth.affine8_packed(N, K, 60)
     xb = qg_synth.gaussian_bf16_bits((T, K), 1.0, 61)

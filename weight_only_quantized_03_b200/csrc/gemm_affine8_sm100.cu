@@ -374,6 +374,12 @@ cudaError_t gemm_affine8_launch(const A8Seg* segs, int nseg, const uint16_t* X, 
     tiles += (segs[i].N + ga8::kBM - 1) / ga8::kBM;
   }
   if (tiles == 0 || T == 0) return cudaSuccess;
+  // a few rows of X: the codes go to the tensor core as they are and each
+  // group's scale and bias apply to its partial sums (no dequantised tile)
+  if (gemm_affine8_skinny_ok(T, K) && nseg <= 3) {
+    if (nt_used) *nt_used = T <= 16 ? 16 : 32;
+    return gemm_affine8_skinny_launch(segs, nseg, X, T, K, err, st, pdl);
+  }
   const int NT = gemm_affine8_tile_rows(tiles, T);
   if (nt_used) *nt_used = NT;
   CUtensorMap map;

@@ -337,6 +337,11 @@ struct A8Seg {
 };
 cudaError_t gemm_affine8_launch(const A8Seg* segs, int nseg, const uint16_t* X, int T, int K,
                                 unsigned* err, cudaStream_t st, bool pdl, int* nt_used);
+// The skinny variant (gemm_affine8_skinny.cu) for T <= 32 and K <= 2048,
+// which gemm_affine8_launch takes by itself for those shapes.
+bool gemm_affine8_skinny_ok(int T, int K);
+cudaError_t gemm_affine8_skinny_launch(const A8Seg* segs, int nseg, const uint16_t* X, int T,
+                                       int K, unsigned* err, cudaStream_t st, bool pdl);
 
 // greedy token per row (argmax.cu); ws of argmax_ws_bytes(B, V) bytes
 size_t argmax_ws_bytes(int B, int V);

@@ -11,6 +11,10 @@ namespace qg {
 // 64 columns x box_rows rows with 128-byte swizzle (rows past the end read as
 // zero); false when the driver's encoder is unavailable or refuses it.
 bool make_bf16_map(CUtensorMap* map, const void* base, int rows, int cols, int box_rows);
+// Host: a TMA descriptor of a byte [rows][cols] row-major tensor (cols a
+// multiple of 16) in boxes of box_cols x box_rows, no swizzle.
+bool make_u8_map(CUtensorMap* map, const void* base, int rows, int cols, int box_cols,
+                 int box_rows);
 
 namespace tc {
 
