@@ -7,8 +7,9 @@
 // the affine factorisation of w = q * s + beta over each group g of 64
 // columns (turbospark-runtime 0.3.0, src/qwen3_asr_metal.rs, PackedLinear /
 // load_packed_linear; the same arithmetic as the GEMV). The centred codes
-// q - 128 lie in [-128, 127] and are exact in bf16, and so are their
-// products with the bf16 activations in fp32, so the MMA operands carry no
+// q - 128 lie in [-128, 127] and are exact in fp16, and so is x * 2^-e in
+// fp16's normal range (x bf16, e a power-of-two prescale chosen from
+// max|x| so that nothing overflows), so the MMA operands carry no
 // dequantisation at all: the codes go to the tensor core as they are, and
 // each group's scale and bias are applied to its partial sums afterwards.
 //
@@ -16,21 +17,22 @@
 // + gridDim.x, ..., each over all K, for NT = 16 or 32 rows of X; its groups
 // in order, tile after tile, are the stages of one ring, so nothing drains
 // between tiles. Roles of a CTA:
-//   * warp 9 (one lane) streams each group's raw code bytes [128][64] and
+//   * the last warp (one lane) streams each group's raw code bytes [128][64] and
 //     X's [NT][64] tile by TMA into a ring of stages (the codes of the first
 //     stages before the programmatic-dependent-launch wait);
-//   * warps 0-3 turn the codes into bf16 (q - 128) in the K-major 128-byte
+//   * warps 0-7 turn the codes into fp16 (q - 128) in the K-major 128-byte
 //     swizzled layout the tensor core reads (16-byte chunk c of row r at
-//     chunk c ^ (r % 8)): one byte permute and one add per code, one packing
-//     permute per two;
-//   * warp 8 owns tensor memory; its lane 0 issues, per group, four
+//     chunk c ^ (r % 8)): one byte permute and one packed subtract per two
+//     codes; and X's tile, in place, into fp16 x * 2^-e;
+//   * warp 12 owns tensor memory; its lane 0 issues, per group, four
 //     tcgen05.mma (M = 128, N = NT, K = 16) into one of four accumulators
 //     (groups take them in turn), commits the stage back to the ring and the
 //     accumulator to the drain;
-//   * warps 4-7 (thread = row of the tile = tensor-memory lane) drain each
-//     group's accumulator with tcgen05.ld and fold it into fp32 registers
-//     with the group's scale and bias (the sums of x per group and row are
-//     formed once, from X in global memory), and store each tile's Y (+ R).
+//   * warps 8-11 (thread = row of the tile = tensor-memory lane) first form,
+//     once per CTA from X in global memory, the sums of x per group and row
+//     and max|x| (hence e); then they drain each group's accumulator with
+//     tcgen05.ld and fold it into fp32 registers with the group's scale
+//     (times 2^e) and bias, and store each tile's Y (+ R).
 // Every wait is bounded (1 s); a wait that gives up sets a CTA-wide abort
 // flag and the caller's error word, and tensor memory is freed only after
 // the last commit has landed.
@@ -48,14 +50,17 @@ constexpr int kBM = 128;
 constexpr int kBK = 64;                  // one quantization group per stage
 constexpr int kMaxGroups = 32;           // K <= 2048 (scales kept in registers)
 constexpr int kMaxSegs = 3;
-constexpr int kThreads = 320;            // 0-3 convert, 4-7 drain, 8 MMA, 9 TMA
-constexpr int kStages = 6;
+constexpr int kConv = 8;                 // converter warps
+constexpr int kThreads = 32 * (kConv + 6);  // converters, 4 drains, MMA, TMA
+constexpr int kRing = 12;              // slots of raw codes and X tiles in flight
+constexpr int kARing = 3;              // converted code tiles
 constexpr int kAcc = 4;                // accumulators in tensor memory (groups in flight)
-constexpr int kStageA = kBM * kBK * 2;   // bf16 codes, 16 KB
-constexpr int kStageX = 32 * kBK * 2;    // room for NT <= 32 rows of X
-constexpr int kStageRaw = kBM * kBK;     // raw code bytes, 8 KB
-constexpr int kStage = kStageA + kStageX + kStageRaw;  // 28 KB, a multiple of 1024
-constexpr int kSmem = 1024 + kStages * kStage + kMaxGroups * 32 * 4 + 512;
+constexpr int kTileA = kBM * kBK * 2;  // fp16 codes, 16 KB
+constexpr int kSlotX = 32 * kBK * 2;   // room for NT <= 32 rows of X (4 KB)
+constexpr int kSlotRaw = kBM * kBK;    // raw code bytes, 8 KB
+constexpr int kSlot = kSlotX + kSlotRaw;  // 12 KB, a multiple of 1024
+constexpr int kSmem = 1024 + kRing * kSlot + kARing * kTileA + kMaxGroups * 32 * 4 +
+                      2 * kMaxGroups * 128 * 2 + 512;
 
 struct Seg {
   const uint16_t* s;   // bf16 [N][K/64]
@@ -83,14 +88,6 @@ __device__ __forceinline__ int seg_of(const Params& P, int tile) {
   for (int i = 1; i < kMaxSegs; ++i)
     if (i < P.nseg && tile >= P.seg[i].tile0) si = i;
   return si;
-}
-
-// two codes (bytes j0, j0 + 1 of w) as a bf16 pair (q - 128): 2^23 + q in
-// fp32 minus 2^23 + 128 is exact, and its upper half is the exact bf16
-__device__ __forceinline__ uint32_t codes_bf16(uint32_t w, int j0) {
-  const float f0 = __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7540u + j0)) - 8388736.0f;
-  const float f1 = __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7541u + j0)) - 8388736.0f;
-  return __byte_perm(__float_as_uint(f0), __float_as_uint(f1), 0x7632u);
 }
 
 template <int NT>
@@ -134,16 +131,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                                int tiles, unsigned* __restrict__ err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t* stages = smem;
-  float* sx = reinterpret_cast<float*>(smem + kStages * kStage);  // [K/64][NT]
-  uint64_t* full_raw = reinterpret_cast<uint64_t*>(sx + kMaxGroups * 32);  // codes landed
-  uint64_t* full_x = full_raw + kStages;                                     // X landed
-  uint64_t* full_a = full_x + kStages;                                       // codes converted
-  uint64_t* empty = full_a + kStages;
-  uint64_t* acc_full = empty + kStages;     // [kAcc]
+  uint8_t* slots = smem;                          // [kRing][X | raw codes]
+  uint8_t* atiles = smem + kRing * kSlot;         // [kARing][fp16 codes]
+  float* sx = reinterpret_cast<float*>(atiles + kARing * kTileA);  // [K/64][NT]
+  uint16_t* tsc = reinterpret_cast<uint16_t*>(sx + kMaxGroups * 32);  // [K/64][128] scales
+  uint16_t* tbi = tsc + kMaxGroups * 128;                             // [K/64][128] biases
+  uint64_t* r_raw = reinterpret_cast<uint64_t*>(tbi + kMaxGroups * 128);  // codes landed
+  uint64_t* r_x = r_raw + kRing;                  // X landed
+  uint64_t* r_empty = r_x + kRing;                // slot free (its MMAs done)
+  // code tile a of group j is free once the MMAs of group j - kARing are
+  // done, which r_empty of that group's slot also tells
+  uint64_t* a_full = r_empty + kRing;             // code tile converted, X tile converted
+  uint64_t* acc_full = a_full + kARing;           // [kAcc]
   uint64_t* acc_empty = acc_full + kAcc;    // [kAcc]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + kAcc);
+  uint64_t* xready = acc_empty + kAcc;     // e is known
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xready + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* xe = const_cast<int*>(abort + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int K = P.K, nk = K / kBK;
@@ -154,20 +158,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr uint32_t kTmemCols = kAcc * NT < 32 ? 32 : kAcc * NT;
 
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full_raw[s], 1);
-      mbar_init(&full_x[s], 1);
-      mbar_init(&full_a[s], 128);
-      mbar_init(&empty[s], 1);
+    for (int s = 0; s < kRing; ++s) {
+      mbar_init(&r_raw[s], 1);
+      mbar_init(&r_x[s], 1);
+      mbar_init(&r_empty[s], 1);
     }
+    for (int a = 0; a < kARing; ++a) mbar_init(&a_full[a], 32 * kConv);
     for (int b = 0; b < kAcc; ++b) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], 128);
     }
+    mbar_init(xready, 1);
     *abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 8) {
+  if (warp == kConv + 4) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(tmem_slot)),
                  "r"(kTmemCols));
@@ -181,7 +186,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_trigger();
 
   bool ok = true;
-  if (warp == 9) {
+  if (warp == kConv + 5) {
     // ------------------------------------------------------------ TMA
     if (lane == 0) {
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmX)) : "memory");
@@ -189,25 +194,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int tile = (int)blockIdx.x + (j / nk) * (int)gridDim.x, kb = j % nk;
         const int si = seg_of(P, tile);
         const int row0 = (tile - P.seg[si].tile0) * kBM;
-        mbar_expect_tx(&full_raw[s], (uint32_t)kStageRaw);
-        tma_load_2d(smem_u32(stages + (size_t)s * kStage + kStageA + kStageX), &maps.w[si],
-                    kb * kBK, row0, &full_raw[s]);
+        mbar_expect_tx(&r_raw[s], (uint32_t)kSlotRaw);
+        tma_load_2d(smem_u32(slots + (size_t)s * kSlot + kSlotX), &maps.w[si], kb * kBK, row0,
+                    &r_raw[s]);
       };
       auto load_x = [&](int j, int s) {
-        mbar_expect_tx(&full_x[s], (uint32_t)(NT * kBK * 2));
-        tma_load_2d(smem_u32(stages + (size_t)s * kStage + kStageA), &tmX, (j % nk) * kBK, 0,
-                    &full_x[s]);
+        mbar_expect_tx(&r_x[s], (uint32_t)(NT * kBK * 2));
+        tma_load_2d(smem_u32(slots + (size_t)s * kSlot), &tmX, (j % nk) * kBK, 0, &r_x[s]);
       };
-      // the codes of the first stages go out before the wait (weights never
+      // the codes of the first slots go out before the wait (weights never
       // depend on the previous kernel), X's tiles after it
-      const int pre = total < kStages ? total : kStages;
+      const int pre = total < kRing ? total : kRing;
       for (int j = 0; j < pre; ++j) load_codes(j, j);
       pdl_wait();  // X is written by the previous kernel
       for (int j = 0; j < pre; ++j) load_x(j, j);
       int issued = pre;
       for (int j = pre; j < total; ++j) {
-        const int s = j % kStages;
-        if (!wait_bar(&empty[s], (uint32_t)((j / kStages) + 1) & 1u, abort)) {
+        const int s = j % kRing;
+        if (!wait_bar(&r_empty[s], (uint32_t)((j / kRing) + 1) & 1u, abort)) {
           ok = false;
           *abort = 1;
           break;
@@ -217,11 +221,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++issued;
       }
       // no copy may land after the CTA is gone: wait (bounded) for the last
-      // fill of every stage used
-      for (int j = issued - kStages > 0 ? issued - kStages : 0; j < issued; ++j) {
-        const int s = j % kStages;
-        const uint32_t par = (uint32_t)(j / kStages) & 1u;
-        for (uint64_t* bar : {&full_raw[s], &full_x[s]}) {
+      // fill of every slot used
+      for (int j = issued - kRing > 0 ? issued - kRing : 0; j < issued; ++j) {
+        const int s = j % kRing;
+        const uint32_t par = (uint32_t)(j / kRing) & 1u;
+        for (uint64_t* bar : {&r_raw[s], &r_x[s]}) {
           if (!mbar_try_wait(bar, par)) {
             const unsigned long long t0 = now_ns();
             while (!mbar_try_wait(bar, par))
@@ -230,51 +234,78 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (warp < 4) {
+  } else if (warp < kConv) {
     // ------------------------------------------------------ converters
+    float down = 1.f;
     for (int j = 0; j < total; ++j) {
-      const int s = j % kStages;
-      if (!wait_bar(&full_raw[s], (uint32_t)(j / kStages) & 1u, abort)) {
+      const int s = j % kRing, a = j % kARing;
+      const uint32_t par = (uint32_t)(j / kRing) & 1u;
+      if (!wait_bar(&r_raw[s], par, abort) ||
+          (j >= kARing && !wait_bar(&r_empty[(j - kARing) % kRing],
+                                    (uint32_t)((j - kARing) / kRing) & 1u, abort))) {
         ok = false;
         *abort = 1;
         break;
       }
-      uint8_t* st = stages + (size_t)s * kStage;
-      const uint8_t* raw = st + kStageA + kStageX;
+      uint8_t* st = atiles + (size_t)a * kTileA;
+      const uint8_t* raw = slots + (size_t)s * kSlot + kSlotX;
 #pragma unroll
-      for (int it = 0; it < 4; ++it) {
-        const int flat = it * 128 + tid;  // 16-byte piece: row flat / 4, columns 16 (flat % 4) ..
+      for (int it = 0; it < 512 / (32 * kConv); ++it) {
+        const int flat = it * 32 * kConv + tid;  // 16-byte piece: row flat / 4, columns 16 (flat % 4) ..
         const int r = flat >> 2, p = flat & 3;
         const uint4 c = *reinterpret_cast<const uint4*>(raw + r * kBK + p * 16);
-        const uint4 lo = make_uint4(codes_bf16(c.x, 0), codes_bf16(c.x, 2), codes_bf16(c.y, 0),
-                                    codes_bf16(c.y, 2));
-        const uint4 hi = make_uint4(codes_bf16(c.z, 0), codes_bf16(c.z, 2), codes_bf16(c.w, 0),
-                                    codes_bf16(c.w, 2));
+        const uint4 lo = make_uint4(codes01(c.x), codes23(c.x), codes01(c.y), codes23(c.y));
+        const uint4 hi = make_uint4(codes01(c.z), codes23(c.z), codes01(c.w), codes23(c.w));
         const int c0 = 2 * p;
         *reinterpret_cast<uint4*>(st + r * 128 + ((c0 ^ (r & 7)) << 4)) = lo;
         *reinterpret_cast<uint4*>(st + r * 128 + (((c0 + 1) ^ (r & 7)) << 4)) = hi;
       }
+      // X's tile of this group, in place: bf16 -> fp16 x * 2^-e (the
+      // element positions of the swizzled tile do not change)
+      if (j == 0) {
+        if (!wait_bar(xready, 0u, abort)) {
+          ok = false;
+          *abort = 1;
+          break;
+        }
+        down = exp2f((float)-*xe);
+      }
+      if (!wait_bar(&r_x[s], par, abort)) {
+        ok = false;
+        *abort = 1;
+        break;
+      }
+      uint8_t* xt = slots + (size_t)s * kSlot;
+      for (int i = tid; i < NT * kBK / 8; i += 32 * kConv) {
+        uint4 v = *reinterpret_cast<const uint4*>(xt + i * 16);
+        uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const __half2 h = __floats2half2_rn(bf16_lo(w[e]) * down, bf16_hi(w[e]) * down);
+          w[e] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+        *reinterpret_cast<uint4*>(xt + i * 16) = v;
+      }
       // make the generic-proxy stores visible to the tensor core
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      mbar_arrive(&full_a[s]);
+      mbar_arrive(&a_full[a]);
     }
     if (!ok) *abort = 1;
-  } else if (warp == 8) {
+  } else if (warp == kConv + 4) {
     // ------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = instr_desc<NT>();
+      const uint32_t idesc = instr_desc_f16<NT>();
       for (int j = 0; j < total; ++j) {
-        const int s = j % kStages, b = j % kAcc;
-        const uint32_t par = (uint32_t)(j / kStages) & 1u;
-        if (!wait_bar(&full_x[s], par, abort) || !wait_bar(&full_a[s], par, abort) ||
+        const int s = j % kRing, a = j % kARing, b = j % kAcc;
+        if (!wait_bar(&a_full[a], (uint32_t)(j / kARing) & 1u, abort) ||
             (j >= kAcc && !wait_bar(&acc_empty[b], (uint32_t)((j / kAcc) + 1) & 1u, abort))) {
           ok = false;
           *abort = 1;
           break;
         }
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        const uint32_t sa = smem_u32(stages + (size_t)s * kStage);
-        const uint32_t sb = sa + kStageA;
+        const uint32_t sa = smem_u32(atiles + (size_t)a * kTileA);
+        const uint32_t sb = smem_u32(slots + (size_t)s * kSlot);
         const uint32_t d = tmem + (uint32_t)(b * NT);
 #pragma unroll
         for (int k = 0; k < kBK / 16; ++k) {
@@ -288,7 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         asm volatile(
             "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                smem_u32(&empty[s]))
+                smem_u32(&r_empty[s]))
             : "memory");
         asm volatile(
             "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -303,7 +334,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the sum of each group of x per row (rows past T are zero), in order:
     // X is the same for every tile, so once per CTA
     pdl_wait();  // x is written by the previous kernel
-    for (int i = tid - 128; i < Kg * NT; i += 128) {
+    float mx = 0.f;
+    const int col = tid - 32 * kConv;  // this drain thread's row of the tile
+    for (int i = col; i < Kg * NT; i += 128) {
       const int g = i / NT, n = i % NT;
       float a = 0.f;
       if (n < P.T) {
@@ -311,16 +344,31 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int jj = 0; jj < 8; ++jj) {
           const uint4 v = __ldcg(xp + jj);
-          a += ((bf16_lo(v.x) + bf16_hi(v.x)) + (bf16_lo(v.y) + bf16_hi(v.y))) +
-               ((bf16_lo(v.z) + bf16_hi(v.z)) + (bf16_lo(v.w) + bf16_hi(v.w)));
+          const float f[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
+                              bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+          a += ((f[0] + f[1]) + (f[2] + f[3])) + ((f[4] + f[5]) + (f[6] + f[7]));
+#pragma unroll
+          for (int e = 0; e < 8; ++e) mx = fmaxf(mx, fabsf(f[e]));
         }
       }
       sx[i] = a;
     }
+    // the prescale 2^-e: max|x| * 2^-e < 2^15 (NaN or inf in x propagate
+    // to y without one)
+    mx = warp_max(mx);
+    float* red = reinterpret_cast<float*>(tsc);  // scratch until the first tile's scales
+    if (lane == 0) red[q] = mx;
     asm volatile("bar.sync 1, 128;" ::: "memory");
-    // per tile: this row's scales and biases as bf16 pairs (group 2 m in
-    // the low half of word m), the fp32 accumulators of the NT rows of X
-    uint32_t sp[kMaxGroups / 2], bp[kMaxGroups / 2];
+    mx = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    const int e = (mx >= 32768.f && mx <= 3.0e38f) ? (int)ceilf(log2f(mx / 16384.f)) : 0;
+    const float up = exp2f((float)e);
+    asm volatile("bar.sync 1, 128;" ::: "memory");  // red is read by all before reuse
+    if (col == 0) {
+      *xe = e;
+      mbar_arrive(xready);
+    }
+    // per tile: this row's bf16 scale and bias per group in its own column
+    // of tsc / tbi; the fp32 accumulators of the NT rows
     float acc[NT];
     int r = 0;
     const Seg* Sg = &P.seg[0];
@@ -331,15 +379,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         Sg = &P.seg[seg_of(P, tile)];
         r = (tile - Sg->tile0) * kBM + 32 * q + lane;  // rows past N are never stored
         const int rc = min(r, Sg->N - 1);
-#pragma unroll
-        for (int m = 0; m < kMaxGroups / 2; ++m) {
-          sp[m] = bp[m] = 0u;
-          if (2 * m < Kg) {
-            const uint16_t* s2 = Sg->s + (size_t)rc * Kg + 2 * m;
-            const uint16_t* b2 = Sg->b + (size_t)rc * Kg + 2 * m;
-            sp[m] = (uint32_t)__ldg(s2) | (2 * m + 1 < Kg ? (uint32_t)__ldg(s2 + 1) << 16 : 0u);
-            bp[m] = (uint32_t)__ldg(b2) | (2 * m + 1 < Kg ? (uint32_t)__ldg(b2 + 1) << 16 : 0u);
-          }
+        for (int g = 0; g < Kg; ++g) {
+          tsc[g * 128 + col] = __ldg(Sg->s + (size_t)rc * Kg + g);
+          tbi[g * 128 + col] = __ldg(Sg->b + (size_t)rc * Kg + g);
         }
 #pragma unroll
         for (int n = 0; n < NT; ++n) acc[n] = 0.f;
@@ -355,15 +397,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
       asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
       mbar_arrive(&acc_empty[b]);
-      uint32_t s2 = 0u, b2 = 0u;
-#pragma unroll
-      for (int m = 0; m < kMaxGroups / 2; ++m)
-        if (m == (kb >> 1)) {
-          s2 = sp[m];
-          b2 = bp[m];
-        }
-      const float s = (kb & 1) ? bf16_hi(s2) : bf16_lo(s2);
-      const float c = fmaf(128.f, s, (kb & 1) ? bf16_hi(b2) : bf16_lo(b2));
+      const float sv = bf16_bits_to_f32(tsc[kb * 128 + col]);
+      const float s = sv * up, c = fmaf(128.f, sv, bf16_bits_to_f32(tbi[kb * 128 + col]));
       const float* sxg = sx + kb * NT;
 #pragma unroll
       for (int n = 0; n < NT; ++n) acc[n] = fmaf(s, __uint_as_float(v[n]), fmaf(c, sxg[n], acc[n]));
@@ -388,7 +423,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // last accumulator (or gave up, in which case the issuer also stopped)
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
-  if (warp == 8) {
+  if (warp == kConv + 4) {
     __syncwarp();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),

@@ -114,8 +114,12 @@ static cudaError_t gtc_launch(const GemvSeg* segs, int nseg, gtc::Params& P, int
   const int sms = num_sms();
   const bool stream16 = NT == 1 && (long long)blk > 8LL * sms;
   const int W = stream16 ? 16 : 8;
-  P.S = gtc_split(blk, K, W, sms);
-  const dim3 grid(std::min(sms, blk), (B + 4 * NT - 1) / (4 * NT));
+  // batch tiles along gridDim.y share one wave of CTAs (one CTA per SM at
+  // these register counts): each tile gets sms / tiles of them
+  const int ny = (B + 4 * NT - 1) / (4 * NT);
+  const int gx = std::max(1, std::min(blk, sms / ny));
+  P.S = gtc_split(blk, K, W, gx);
+  const dim3 grid(gx, ny);
   if (NT == 2) return gtc_launch_nt<2, 8>(P, grid, st, pdl);
   if (W == 16) return gtc_launch_nt<1, 16>(P, grid, st, pdl);
   return gtc_launch_nt<1, 8>(P, grid, st, pdl);

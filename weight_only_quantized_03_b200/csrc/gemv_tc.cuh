@@ -74,22 +74,6 @@ __device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1,
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
-// codes (0,1) and (2,3) of a word as fp16 pairs of q - 128: the byte
-// permute makes 1024 + q (fp16 0x6400 | q), one packed subtract of 1152
-// (0x6480) centres it; both steps are exact. Centred codes keep the fp32
-// partial sums of a group near sum (q - 128) x instead of carrying a
-// 1024 * sum(x) term, so their rounding error is that much smaller.
-__device__ __forceinline__ uint32_t centre(uint32_t h2) {
-  const __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&h2),
-                            __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480)));
-  return *reinterpret_cast<const uint32_t*>(&r);
-}
-__device__ __forceinline__ uint32_t codes01(uint32_t w) {
-  return centre(__byte_perm(w, 0x64646464u, 0x4140u));
-}
-__device__ __forceinline__ uint32_t codes23(uint32_t w) {
-  return centre(__byte_perm(w, 0x64646464u, 0x4342u));
-}
 
 // which segment a global block index belongs to
 __device__ __forceinline__ int seg_of(const Params& P, int blk) {

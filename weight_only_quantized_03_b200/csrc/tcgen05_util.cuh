@@ -49,12 +49,25 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
                "r"(bytes)
                : "memory");
 }
+// try_wait that may suspend the thread up to hint_ns (it resumes as soon as
+// the phase completes), so a waiting role sleeps instead of spinning
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity,
+                                                   uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
 // bounded wait (limit_ns); gives up early once another role has aborted
 __device__ __forceinline__ bool wait_bar_ns(uint64_t* bar, uint32_t parity, volatile int* abort,
                                             unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = now_ns();
-  while (!mbar_try_wait(bar, parity)) {
+  while (!mbar_try_wait_hint(bar, parity, 20000u)) {
     if (*abort) return false;
     if (now_ns() - t0 > limit_ns) return false;
   }
@@ -74,6 +87,14 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr) {
   d |= (uint64_t)1u << 46;             // version
   d |= (uint64_t)2u << 61;             // SWIZZLE_128B
   return d;
+}
+
+// instruction descriptor: fp16 x fp16 -> fp32, both K-major, M = 128
+template <int BN>
+__host__ __device__ constexpr uint32_t instr_desc_f16() {
+  return (1u << 4)                 // D fp32 (A, B fp16: format 0)
+         | ((uint32_t)(BN >> 3) << 17)
+         | ((uint32_t)(128 >> 4) << 24);
 }
 
 // instruction descriptor: bf16 x bf16 -> fp32, both K-major, M = 128
