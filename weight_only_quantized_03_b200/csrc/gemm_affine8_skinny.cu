@@ -17,22 +17,24 @@
 // + gridDim.x, ..., each over all K, for NT = 16 or 32 rows of X; its groups
 // in order, tile after tile, are the stages of one ring, so nothing drains
 // between tiles. Roles of a CTA:
-//   * the last warp (one lane) streams each group's raw code bytes [128][64] and
-//     X's [NT][64] tile by TMA into a ring of stages (the codes of the first
-//     stages before the programmatic-dependent-launch wait);
+//   * the last warp (one lane) streams each group's raw code bytes [128][64]
+//     by TMA into a ring of slots (those of the first slots before the
+//     programmatic-dependent-launch wait);
 //   * warps 0-7 turn the codes into fp16 (q - 128) in the K-major 128-byte
 //     swizzled layout the tensor core reads (16-byte chunk c of row r at
 //     chunk c ^ (r % 8)): one byte permute and one packed subtract per two
-//     codes; and X's tile, in place, into fp16 x * 2^-e;
+//     codes;
 //   * warp 12 owns tensor memory; its lane 0 issues, per group, four
 //     tcgen05.mma (M = 128, N = NT, K = 16) into one of four accumulators
 //     (groups take them in turn), commits the stage back to the ring and the
 //     accumulator to the drain;
 //   * warps 8-11 (thread = row of the tile = tensor-memory lane) first form,
 //     once per CTA from X in global memory, the sums of x per group and row
-//     and max|x| (hence e); then they drain each group's accumulator with
-//     tcgen05.ld and fold it into fp32 registers with the group's scale
-//     (times 2^e) and bias, and store each tile's Y (+ R).
+//     and max|x| (hence e), and write all of X as fp16 x * 2^-e in the same
+//     swizzled layout, where it stays for every tile (NT K 2 <= 64 KB); then
+//     they drain each group's accumulator with tcgen05.ld and fold it into
+//     fp32 registers with the group's scale (times 2^e) and bias, and store
+//     each tile's Y (+ R).
 // Every wait is bounded (1 s); a wait that gives up sets a CTA-wide abort
 // flag and the caller's error word, and tensor memory is freed only after
 // the last commit has landed.
@@ -47,19 +49,20 @@ namespace gas {
 using namespace tc;
 
 constexpr int kBM = 128;
-constexpr int kBK = 64;                  // one quantization group per stage
+constexpr int kBK = 64;                  // columns of a quantization group
 constexpr int kMaxGroups = 32;           // K <= 2048 (scales kept in registers)
 constexpr int kMaxSegs = 3;
 constexpr int kConv = 8;                 // converter warps
 constexpr int kThreads = 32 * (kConv + 6);  // converters, 4 drains, MMA, TMA
-constexpr int kRing = 12;              // slots of raw codes and X tiles in flight
-constexpr int kARing = 3;              // converted code tiles
-constexpr int kAcc = 4;                // accumulators in tensor memory (groups in flight)
-constexpr int kTileA = kBM * kBK * 2;  // fp16 codes, 16 KB
-constexpr int kSlotX = 32 * kBK * 2;   // room for NT <= 32 rows of X (4 KB)
-constexpr int kSlotRaw = kBM * kBK;    // raw code bytes, 8 KB
-constexpr int kSlot = kSlotX + kSlotRaw;  // 12 KB, a multiple of 1024
-constexpr int kSmem = 1024 + kRing * kSlot + kARing * kTileA + kMaxGroups * 32 * 4 +
+// A stage is two groups (128 columns of K): one TMA of codes, one round of
+// waits and commits for two groups' MMAs.
+constexpr int kRing = 4;                   // stages of raw codes in flight
+constexpr int kARing = 2;                  // converted code tiles (two groups each)
+constexpr int kAcc = 4;                    // accumulator pairs in tensor memory
+constexpr int kTileA = 2 * kBM * kBK * 2;  // fp16 codes of two groups, 32 KB
+constexpr int kSlot = kBM * 2 * kBK;       // raw code bytes of two groups, 16 KB
+constexpr int kXBytes = 64 * 1024;     // resident X: NT * K * 2 <= 64 KB
+constexpr int kSmem = 1024 + kXBytes + kRing * kSlot + kARing * kTileA + kMaxGroups * 32 * 4 +
                       2 * kMaxGroups * 128 * 2 + 512;
 
 struct Seg {
@@ -126,41 +129,38 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
 
 template <int NT>
 __global__ void __launch_bounds__(kThreads, 1)
-    gemm_affine8_skinny_kernel(const __grid_constant__ CUtensorMap tmX,
-                               const __grid_constant__ Maps maps, const __grid_constant__ Params P,
+    gemm_affine8_skinny_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params P,
                                int tiles, unsigned* __restrict__ err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t* slots = smem;                          // [kRing][X | raw codes]
-  uint8_t* atiles = smem + kRing * kSlot;         // [kARing][fp16 codes]
+  uint8_t* xres = smem;                           // [K/64][NT][64] fp16, swizzled
+  uint8_t* slots = smem + kXBytes;                // [kRing][128][128] raw codes
+  uint8_t* atiles = slots + kRing * kSlot;        // [kARing][2][128][64] fp16 codes, swizzled
   float* sx = reinterpret_cast<float*>(atiles + kARing * kTileA);  // [K/64][NT]
   uint16_t* tsc = reinterpret_cast<uint16_t*>(sx + kMaxGroups * 32);  // [K/64][128] scales
   uint16_t* tbi = tsc + kMaxGroups * 128;                             // [K/64][128] biases
   uint64_t* r_raw = reinterpret_cast<uint64_t*>(tbi + kMaxGroups * 128);  // codes landed
-  uint64_t* r_x = r_raw + kRing;                  // X landed
-  uint64_t* r_empty = r_x + kRing;                // slot free (its MMAs done)
-  // code tile a of group j is free once the MMAs of group j - kARing are
-  // done, which r_empty of that group's slot also tells
-  uint64_t* a_full = r_empty + kRing;             // code tile converted, X tile converted
+  uint64_t* r_empty = r_raw + kRing;              // slot free (its MMAs done)
+  // code tiles a of stage j are free once the MMAs of stage j - kARing are
+  // done, which r_empty of that stage's slot also tells
+  uint64_t* a_full = r_empty + kRing;             // code tiles converted
   uint64_t* acc_full = a_full + kARing;           // [kAcc]
-  uint64_t* acc_empty = acc_full + kAcc;    // [kAcc]
-  uint64_t* xready = acc_empty + kAcc;     // e is known
+  uint64_t* acc_empty = acc_full + kAcc;          // [kAcc]
+  uint64_t* xready = acc_empty + kAcc;            // X resident (fp16, swizzled)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xready + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int* xe = const_cast<int*>(abort + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int K = P.K, nk = K / kBK;
-  // this CTA's tiles: blockIdx.x, + gridDim.x, ...; its groups in order,
-  // tile after tile, are the stages j = i * nk + kb of one ring
+  const int K = P.K, nk = K / kBK, ns = nk / 2;  // groups, stages (two groups each) per tile
+  // this CTA's tiles: blockIdx.x, + gridDim.x, ...; their stages in order,
+  // tile after tile, are the stages j = i * ns + ks of one ring
   const int ntl = ((int)blockIdx.x < tiles) ? (tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
-  const int total = ntl * nk;
-  constexpr uint32_t kTmemCols = kAcc * NT < 32 ? 32 : kAcc * NT;
+  const int total = ntl * ns;
+  constexpr uint32_t kTmemCols = 2 * kAcc * NT < 32 ? 32 : 2 * kAcc * NT;
 
   if (tid == 0) {
     for (int s = 0; s < kRing; ++s) {
       mbar_init(&r_raw[s], 1);
-      mbar_init(&r_x[s], 1);
       mbar_init(&r_empty[s], 1);
     }
     for (int a = 0; a < kARing; ++a) mbar_init(&a_full[a], 32 * kConv);
@@ -168,7 +168,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], 128);
     }
-    mbar_init(xready, 1);
+    mbar_init(xready, 128);
     *abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -189,25 +189,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kConv + 5) {
     // ------------------------------------------------------------ TMA
     if (lane == 0) {
-      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmX)) : "memory");
       auto load_codes = [&](int j, int s) {
-        const int tile = (int)blockIdx.x + (j / nk) * (int)gridDim.x, kb = j % nk;
+        const int tile = (int)blockIdx.x + (j / ns) * (int)gridDim.x, ks = j % ns;
         const int si = seg_of(P, tile);
         const int row0 = (tile - P.seg[si].tile0) * kBM;
-        mbar_expect_tx(&r_raw[s], (uint32_t)kSlotRaw);
-        tma_load_2d(smem_u32(slots + (size_t)s * kSlot + kSlotX), &maps.w[si], kb * kBK, row0,
+        mbar_expect_tx(&r_raw[s], (uint32_t)kSlot);
+        tma_load_2d(smem_u32(slots + (size_t)s * kSlot), &maps.w[si], ks * 2 * kBK, row0,
                     &r_raw[s]);
       };
-      auto load_x = [&](int j, int s) {
-        mbar_expect_tx(&r_x[s], (uint32_t)(NT * kBK * 2));
-        tma_load_2d(smem_u32(slots + (size_t)s * kSlot), &tmX, (j % nk) * kBK, 0, &r_x[s]);
-      };
-      // the codes of the first slots go out before the wait (weights never
-      // depend on the previous kernel), X's tiles after it
+      // weights never depend on the previous kernel: no wait here
       const int pre = total < kRing ? total : kRing;
       for (int j = 0; j < pre; ++j) load_codes(j, j);
-      pdl_wait();  // X is written by the previous kernel
-      for (int j = 0; j < pre; ++j) load_x(j, j);
       int issued = pre;
       for (int j = pre; j < total; ++j) {
         const int s = j % kRing;
@@ -217,7 +209,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         load_codes(j, s);
-        load_x(j, s);
         ++issued;
       }
       // no copy may land after the CTA is gone: wait (bounded) for the last
@@ -225,18 +216,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = issued - kRing > 0 ? issued - kRing : 0; j < issued; ++j) {
         const int s = j % kRing;
         const uint32_t par = (uint32_t)(j / kRing) & 1u;
-        for (uint64_t* bar : {&r_raw[s], &r_x[s]}) {
-          if (!mbar_try_wait(bar, par)) {
-            const unsigned long long t0 = now_ns();
-            while (!mbar_try_wait(bar, par))
-              if (now_ns() - t0 > kWaitNs) break;
-          }
+        if (!mbar_try_wait(&r_raw[s], par)) {
+          const unsigned long long t0 = now_ns();
+          while (!mbar_try_wait(&r_raw[s], par))
+            if (now_ns() - t0 > kWaitNs) break;
         }
       }
     }
   } else if (warp < kConv) {
     // ------------------------------------------------------ converters
-    float down = 1.f;
     for (int j = 0; j < total; ++j) {
       const int s = j % kRing, a = j % kARing;
       const uint32_t par = (uint32_t)(j / kRing) & 1u;
@@ -247,44 +235,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         *abort = 1;
         break;
       }
-      uint8_t* st = atiles + (size_t)a * kTileA;
-      const uint8_t* raw = slots + (size_t)s * kSlot + kSlotX;
+      uint8_t* at = atiles + (size_t)a * kTileA;
+      const uint8_t* raw = slots + (size_t)s * kSlot;
 #pragma unroll
-      for (int it = 0; it < 512 / (32 * kConv); ++it) {
-        const int flat = it * 32 * kConv + tid;  // 16-byte piece: row flat / 4, columns 16 (flat % 4) ..
-        const int r = flat >> 2, p = flat & 3;
-        const uint4 c = *reinterpret_cast<const uint4*>(raw + r * kBK + p * 16);
+      for (int it = 0; it < 1024 / (32 * kConv); ++it) {
+        // 16-byte piece: row flat / 8, columns 16 (flat % 8) .. of the
+        // stage's 128; group h = piece / 4 of the two
+        const int flat = it * 32 * kConv + tid;
+        const int r = flat >> 3, p = flat & 7, h = p >> 2, c0 = 2 * (p & 3);
+        const uint4 c = *reinterpret_cast<const uint4*>(raw + r * (2 * kBK) + p * 16);
         const uint4 lo = make_uint4(codes01(c.x), codes23(c.x), codes01(c.y), codes23(c.y));
         const uint4 hi = make_uint4(codes01(c.z), codes23(c.z), codes01(c.w), codes23(c.w));
-        const int c0 = 2 * p;
-        *reinterpret_cast<uint4*>(st + r * 128 + ((c0 ^ (r & 7)) << 4)) = lo;
-        *reinterpret_cast<uint4*>(st + r * 128 + (((c0 + 1) ^ (r & 7)) << 4)) = hi;
-      }
-      // X's tile of this group, in place: bf16 -> fp16 x * 2^-e (the
-      // element positions of the swizzled tile do not change)
-      if (j == 0) {
-        if (!wait_bar(xready, 0u, abort)) {
-          ok = false;
-          *abort = 1;
-          break;
-        }
-        down = exp2f((float)-*xe);
-      }
-      if (!wait_bar(&r_x[s], par, abort)) {
-        ok = false;
-        *abort = 1;
-        break;
-      }
-      uint8_t* xt = slots + (size_t)s * kSlot;
-      for (int i = tid; i < NT * kBK / 8; i += 32 * kConv) {
-        uint4 v = *reinterpret_cast<const uint4*>(xt + i * 16);
-        uint32_t* w = reinterpret_cast<uint32_t*>(&v);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const __half2 h = __floats2half2_rn(bf16_lo(w[e]) * down, bf16_hi(w[e]) * down);
-          w[e] = *reinterpret_cast<const uint32_t*>(&h);
-        }
-        *reinterpret_cast<uint4*>(xt + i * 16) = v;
+        uint8_t* t = at + h * (kBM * kBK * 2) + r * 128;
+        *reinterpret_cast<uint4*>(t + ((c0 ^ (r & 7)) << 4)) = lo;
+        *reinterpret_cast<uint4*>(t + (((c0 + 1) ^ (r & 7)) << 4)) = hi;
       }
       // make the generic-proxy stores visible to the tensor core
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -295,7 +259,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc = instr_desc_f16<NT>();
-      for (int j = 0; j < total; ++j) {
+      if (total > 0 && !wait_bar(xready, 0u, abort)) {
+        ok = false;
+        *abort = 1;
+      }
+      for (int j = 0; j < total && ok; ++j) {
         const int s = j % kRing, a = j % kARing, b = j % kAcc;
         if (!wait_bar(&a_full[a], (uint32_t)(j / kARing) & 1u, abort) ||
             (j >= kAcc && !wait_bar(&acc_empty[b], (uint32_t)((j / kAcc) + 1) & 1u, abort))) {
@@ -304,18 +272,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        const uint32_t sa = smem_u32(atiles + (size_t)a * kTileA);
-        const uint32_t sb = smem_u32(slots + (size_t)s * kSlot);
-        const uint32_t d = tmem + (uint32_t)(b * NT);
+        const int g0 = (j % ns) * 2;  // the stage's first group
 #pragma unroll
-        for (int k = 0; k < kBK / 16; ++k) {
-          const uint64_t da = smem_desc(sa + k * 32), db = smem_desc(sb + k * 32);
-          const uint32_t acc = k > 0 ? 1u : 0u;
-          asm volatile(
-              "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-              " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d),
-              "l"(da), "l"(db), "r"(idesc), "r"(acc)
-              : "memory");
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t sa = smem_u32(atiles + (size_t)a * kTileA + h * (kBM * kBK * 2));
+          const uint32_t sb = smem_u32(xres + (size_t)(g0 + h) * (NT * kBK * 2));
+          const uint32_t d = tmem + (uint32_t)((2 * b + h) * NT);
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) {
+            const uint64_t da = smem_desc(sa + k * 32), db = smem_desc(sb + k * 32);
+            const uint32_t acc = k > 0 ? 1u : 0u;
+            asm volatile(
+                "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+                " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d),
+                "l"(da), "l"(db), "r"(idesc), "r"(acc)
+                : "memory");
+          }
         }
         asm volatile(
             "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -331,11 +303,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // --------------------------------------------------------- drains
     const int q = warp & 3;  // tensor-memory lanes 32 q .. 32 q + 31
     const int Kg = K / 64;
+    const int col = tid - 32 * kConv;  // this drain thread's row of the tile
     // the sum of each group of x per row (rows past T are zero), in order:
     // X is the same for every tile, so once per CTA
     pdl_wait();  // x is written by the previous kernel
     float mx = 0.f;
-    const int col = tid - 32 * kConv;  // this drain thread's row of the tile
     for (int i = col; i < Kg * NT; i += 128) {
       const int g = i / NT, n = i % NT;
       float a = 0.f;
@@ -363,19 +335,37 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int e = (mx >= 32768.f && mx <= 3.0e38f) ? (int)ceilf(log2f(mx / 16384.f)) : 0;
     const float up = exp2f((float)e);
     asm volatile("bar.sync 1, 128;" ::: "memory");  // red is read by all before reuse
-    if (col == 0) {
-      *xe = e;
-      mbar_arrive(xready);
+    // all of X as fp16 x * 2^-e, group g's [NT][64] tile at g * NT * 128
+    // bytes, 16-byte chunk c of row n at chunk c ^ (n % 8) (rows past T zero)
+    const float down = exp2f((float)-e);
+    for (int i = col; i < Kg * NT * 8; i += 128) {
+      const int g = i / (NT * 8), n = (i / 8) % NT, c = i % 8;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (n < P.T) {
+        const uint4 xv = __ldcg(reinterpret_cast<const uint4*>(P.x + (size_t)n * K + g * 64 + c * 8));
+        const uint32_t w4[4] = {xv.x, xv.y, xv.z, xv.w};
+        uint32_t h4[4];
+#pragma unroll
+        for (int e2 = 0; e2 < 4; ++e2) {
+          const __half2 h = __floats2half2_rn(bf16_lo(w4[e2]) * down, bf16_hi(w4[e2]) * down);
+          h4[e2] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+        v = make_uint4(h4[0], h4[1], h4[2], h4[3]);
+      }
+      *reinterpret_cast<uint4*>(xres + (size_t)g * NT * 128 + n * 128 + ((c ^ (n & 7)) << 4)) = v;
     }
+    // make the generic-proxy stores visible to the tensor core
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    mbar_arrive(xready);
     // per tile: this row's bf16 scale and bias per group in its own column
     // of tsc / tbi; the fp32 accumulators of the NT rows
     float acc[NT];
     int r = 0;
     const Seg* Sg = &P.seg[0];
     for (int j = 0; j < total; ++j) {
-      const int kb = j % nk, b = j % kAcc;
-      if (kb == 0) {
-        const int tile = (int)blockIdx.x + (j / nk) * (int)gridDim.x;
+      const int ks = j % ns, b = j % kAcc;
+      if (ks == 0) {
+        const int tile = (int)blockIdx.x + (j / ns) * (int)gridDim.x;
         Sg = &P.seg[seg_of(P, tile)];
         r = (tile - Sg->tile0) * kBM + 32 * q + lane;  // rows past N are never stored
         const int rc = min(r, Sg->N - 1);
@@ -392,17 +382,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      uint32_t v[NT];
-      tmem_ld<NT>(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * NT), v);
+      uint32_t v0[NT], v1[NT];
+      tmem_ld<NT>(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(2 * b * NT), v0);
+      tmem_ld<NT>(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)((2 * b + 1) * NT), v1);
       asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
       asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
       mbar_arrive(&acc_empty[b]);
-      const float sv = bf16_bits_to_f32(tsc[kb * 128 + col]);
-      const float s = sv * up, c = fmaf(128.f, sv, bf16_bits_to_f32(tbi[kb * 128 + col]));
-      const float* sxg = sx + kb * NT;
+      const int g0 = 2 * ks;
+      const float s0 = bf16_bits_to_f32(tsc[g0 * 128 + col]);
+      const float s1 = bf16_bits_to_f32(tsc[(g0 + 1) * 128 + col]);
+      const float c0 = fmaf(128.f, s0, bf16_bits_to_f32(tbi[g0 * 128 + col]));
+      const float c1 = fmaf(128.f, s1, bf16_bits_to_f32(tbi[(g0 + 1) * 128 + col]));
+      const float u0 = s0 * up, u1 = s1 * up;
+      const float* sx0 = sx + g0 * NT;
+      const float* sx1 = sx0 + NT;
 #pragma unroll
-      for (int n = 0; n < NT; ++n) acc[n] = fmaf(s, __uint_as_float(v[n]), fmaf(c, sxg[n], acc[n]));
-      if (kb == nk - 1 && r < Sg->N) {
+      for (int n = 0; n < NT; ++n)
+        acc[n] = fmaf(u1, __uint_as_float(v1[n]),
+                      fmaf(c1, sx1[n], fmaf(u0, __uint_as_float(v0[n]), fmaf(c0, sx0[n], acc[n]))));
+      if (ks == ns - 1 && r < Sg->N) {
 #pragma unroll
         for (int n = 0; n < NT; ++n) {
           if (n >= P.T) break;
@@ -433,18 +431,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace gas
 
-// Whether the skinny matmul takes the launch: T <= 32 rows of X and K a
-// multiple of 64 up to 2048 (the groups' scales stay in registers).
-bool gemm_affine8_skinny_ok(int T, int K) { return T >= 1 && T <= 32 && K % 64 == 0 && K <= 2048; }
+// Whether the skinny matmul takes the launch: T <= 32 rows of X, K a
+// multiple of 128 up to 2048, and X resident in shared memory as fp16 (its
+// NT = 16 or 32 rows times K times 2 bytes within 64 KB).
+bool gemm_affine8_skinny_ok(int T, int K) {
+  const int NT = T <= 16 ? 16 : 32;
+  return T >= 1 && T <= 32 && K % 128 == 0 && K <= 2048 && NT * K * 2 <= 64 * 1024;
+}
 
 template <int NT>
-static cudaError_t gas_launch(const CUtensorMap& tmX, const gas::Maps& maps, const gas::Params& P,
-                              int tiles, unsigned* err, cudaStream_t st, bool pdl) {
+static cudaError_t gas_launch(const gas::Maps& maps, const gas::Params& P, int tiles,
+                              unsigned* err, cudaStream_t st, bool pdl) {
   ensure_smem((const void*)gas::gemm_affine8_skinny_kernel<NT>, gas::kSmem);
   // persistent: one CTA per SM walks its tiles
   const int grid = tiles < num_sms() ? tiles : num_sms();
   return launch_pdl(gas::gemm_affine8_skinny_kernel<NT>, dim3(grid), dim3(gas::kThreads),
-                    (size_t)gas::kSmem, st, pdl, tmX, maps, P, tiles, err);
+                    (size_t)gas::kSmem, st, pdl, maps, P, tiles, err);
 }
 
 cudaError_t gemm_affine8_skinny_launch(const A8Seg* segs, int nseg, const uint16_t* X, int T,
@@ -461,16 +463,13 @@ cudaError_t gemm_affine8_skinny_launch(const A8Seg* segs, int nseg, const uint16
   for (int i = 0; i < nseg; ++i) {
     P.seg[i] = gas::Seg{segs[i].s, segs[i].b, segs[i].y, segs[i].res, segs[i].N, segs[i].y_bf16,
                         tiles};
-    if (!make_u8_map(&maps.w[i], segs[i].w, segs[i].N, K, gas::kBK, gas::kBM))
+    if (!make_u8_map(&maps.w[i], segs[i].w, segs[i].N, K, 2 * gas::kBK, gas::kBM))
       return cudaErrorInvalidValue;
     tiles += (segs[i].N + gas::kBM - 1) / gas::kBM;
   }
   if (tiles == 0) return cudaSuccess;
-  const int NT = T <= 16 ? 16 : 32;
-  CUtensorMap tmX;
-  if (!make_bf16_map(&tmX, X, T, K, NT)) return cudaErrorInvalidValue;
-  if (NT == 16) return gas_launch<16>(tmX, maps, P, tiles, err, st, pdl);
-  return gas_launch<32>(tmX, maps, P, tiles, err, st, pdl);
+  if (T <= 16) return gas_launch<16>(maps, P, tiles, err, st, pdl);
+  return gas_launch<32>(maps, P, tiles, err, st, pdl);
 }
 
 }  // namespace qg
