@@ -75,7 +75,8 @@ bool gemv_tc_eligible(const GemvSeg* segs, int nseg, int K, int B, bool x_f32) {
     return false;
   for (int i = 0; i < nseg; ++i)
     if (!aligned(segs[i].w, 32) || !aligned(segs[i].s, 4) || !aligned(segs[i].b, 4)) return false;
-  return gtc_smem(K, B > 4 ? 2 : 1, 16) <= 200 * 1024;
+  const int NT = B > 4 ? 2 : 1;
+  return std::max(gtc_smem(K, NT, 16), gtc_smem(K, NT, 8)) <= 200 * 1024;
 }
 
 template <int NT, int W>

@@ -161,6 +161,11 @@ __device__ __forceinline__ void gemv_tc_body(const Params& P, uint8_t* smem, Wai
   float* part = red + kRed;                                          // [2][kWarps][32][2 NT]
   float* gsum = part + 2 * kWarps * 32 * 2 * NT;                    // [4 NT][Kg]
   uint16_t* xh = reinterpret_cast<uint16_t*>(gsum + 4 * NT * Kg);   // [4 NT][xs]
+  // one batch tile of 8 warps: each warp's second unit of work (a 16-row
+  // block's super-chunk) is staged here before the wait, 16-byte piece q of
+  // chunk p of lane l at ((p * 4 + q) * 32 + l) * 16 (conflict-free)
+  constexpr bool kStage2 = NT == 1 && W == 8;
+  uint8_t* stage2 = reinterpret_cast<uint8_t*>(xh + 4 * NT * xs) + (size_t)warp * 8192;
 
   // L2 prefetch for a later kernel of the chain (one thread per CTA)
   if (tid == 0 && blockIdx.y == 0 && (P.pf.n > 0 || P.pf.kv.kc))
@@ -188,6 +193,34 @@ __device__ __forceinline__ void gemv_tc_body(const Params& P, uint8_t* smem, Wai
     load_scales(lr, Kg, lsc, sv);
 #pragma unroll
     for (int p = 0; p < 4; ++p) load_chunk(lr, K, lsc, p, pol, wb[p]);
+  }
+  // the second unit's codes go to shared memory and its scales to registers,
+  // also before the wait, so that no weight load is left after it for a warp
+  // with two units (K = 3072 split over teams of 4: the down projection)
+  bool staged = false;
+  uint32_t sv1[4] = {0u, 0u, 0u, 0u};
+  if constexpr (kStage2) {
+    if (total >= 2) {
+      int sc1 = lsc + 1, blk1 = lblk;
+      if (sc1 == sc_hi) {
+        sc1 = sc_lo;
+        blk1 += T;
+      }
+      const Rows r1 = rows_of(P, blk1, g, t);
+      load_scales(r1, Kg, sc1, sv1);
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        const uint8_t* a = r1.w + sc1 * kSC + p * 128;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint8_t* src = a + (q >> 1) * (size_t)r1.dr * K + (q & 1) * 16;
+          const uint32_t dst = (uint32_t)__cvta_generic_to_shared(stage2 + ((p * 4 + q) * 32 + lane) * 16);
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+        }
+      }
+      asm volatile("cp.async.commit_group;" ::: "memory");
+      staged = true;
+    }
   }
 
   // The input is formed in items of 128 columns of one batch row (lane l
@@ -393,7 +426,13 @@ __device__ __forceinline__ void gemv_tc_body(const Params& P, uint8_t* smem, Wai
       }
     }
     uint32_t svn[4] = {0u, 0u, 0u, 0u};
-    if (more) load_scales(lr, Kg, lsc, svn);
+    const bool from_stage = staged && it == 0;  // the next unit is already in shared memory
+    if (from_stage) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) svn[i] = sv1[i];
+    } else if (more) {
+      load_scales(lr, Kg, lsc, svn);
+    }
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
       const int src = (lane & ~3) | p;
@@ -426,7 +465,20 @@ __device__ __forceinline__ void gemv_tc_body(const Params& P, uint8_t* smem, Wai
         acc[nt][1] = fmaf(sA1, d0[2] + d1[2], fmaf(cA1, gs.x, fmaf(sB1, d0[3] + d1[3],
                                                                    fmaf(cB1, gs.y, acc[nt][1]))));
       }
-      if (more) load_chunk(lr, K, lsc, p, pol, wb[p]);
+      if (more && !from_stage) load_chunk(lr, K, lsc, p, pol, wb[p]);
+    }
+    if (from_stage) {
+      asm volatile("cp.async.wait_all;" ::: "memory");
+#pragma unroll
+      for (int p = 0; p < 4; ++p)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint4 v = *reinterpret_cast<const uint4*>(stage2 + ((p * 4 + q) * 32 + lane) * 16);
+          wb[p][q * 4 + 0] = v.x;
+          wb[p][q * 4 + 1] = v.y;
+          wb[p][q * 4 + 2] = v.z;
+          wb[p][q * 4 + 3] = v.w;
+        }
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i) sv[i] = svn[i];
@@ -492,7 +544,8 @@ __device__ __forceinline__ void gemv_tc_body(const Params& P, uint8_t* smem, Wai
 // dynamic shared memory of gemv_tc_body
 inline size_t gtc_smem(int K, int NT, int W) {
   return (size_t)(((4 * NT + 1) * W + 3) & ~3) * 4 + (size_t)2 * W * 32 * 2 * NT * 4 +
-         (size_t)4 * NT * (K / 64) * 4 + (size_t)4 * NT * (K + 8) * 2;
+         (size_t)4 * NT * (K / 64) * 4 + (size_t)4 * NT * (K + 8) * 2 +
+         (NT == 1 && W == 8 ? (size_t)W * 8192 : 0);  // the second unit's staging
 }
 
 // Columns of each 16-row block are split over S warps (1, 2, 4, ... <= W,
