@@ -55,14 +55,14 @@ constexpr int kMaxSegs = 3;
 constexpr int kConv = 8;                 // converter warps
 constexpr int kThreads = 32 * (kConv + 6);  // converters, 4 drains, MMA, TMA
 // A stage is two groups (128 columns of K): one TMA of codes, one round of
-// waits and commits for two groups' MMAs.
-constexpr int kRing = 4;                   // stages of raw codes in flight
-constexpr int kARing = 2;                  // converted code tiles (two groups each)
+// waits and commits for two groups' MMAs. The converted codes live in
+// tensor memory, as the MMA's A operand.
+constexpr int kRing = 8;                   // stages of raw codes in flight
+constexpr int kMaxARing = 6;               // code tiles in tensor memory (two groups each)
 constexpr int kAcc = 4;                    // accumulator pairs in tensor memory
-constexpr int kTileA = 2 * kBM * kBK * 2;  // fp16 codes of two groups, 32 KB
 constexpr int kSlot = kBM * 2 * kBK;       // raw code bytes of two groups, 16 KB
 constexpr int kXBytes = 64 * 1024;     // resident X: NT * K * 2 <= 64 KB
-constexpr int kSmem = 1024 + kXBytes + kRing * kSlot + kARing * kTileA + kMaxGroups * 32 * 4 +
+constexpr int kSmem = 1024 + kXBytes + kRing * kSlot + kMaxGroups * 32 * 4 +
                       2 * kMaxGroups * 128 * 2 + 512;
 
 struct Seg {
@@ -131,20 +131,22 @@ template <int NT>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_affine8_skinny_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params P,
                                int tiles, unsigned* __restrict__ err) {
+  // tensor memory: kAcc accumulator pairs (2 NT columns each), then the ring
+  // of converted code tiles (two groups of 32 columns each)
+  constexpr int kAccCols = 2 * kAcc * NT;
+  constexpr int kARing = (512 - kAccCols) / 64;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* xres = smem;                           // [K/64][NT][64] fp16, swizzled
-  uint8_t* slots = smem + kXBytes;                // [kRing][128][128] raw codes
-  uint8_t* atiles = slots + kRing * kSlot;        // [kARing][2][128][64] fp16 codes, swizzled
-  float* sx = reinterpret_cast<float*>(atiles + kARing * kTileA);  // [K/64][NT]
+  uint8_t* slots = smem + kXBytes;                // [kRing][128][128] raw codes, swizzled
+  float* sx = reinterpret_cast<float*>(slots + kRing * kSlot);  // [K/64][NT]
   uint16_t* tsc = reinterpret_cast<uint16_t*>(sx + kMaxGroups * 32);  // [K/64][128] scales
   uint16_t* tbi = tsc + kMaxGroups * 128;                             // [K/64][128] biases
   uint64_t* r_raw = reinterpret_cast<uint64_t*>(tbi + kMaxGroups * 128);  // codes landed
-  uint64_t* r_empty = r_raw + kRing;              // slot free (its MMAs done)
-  // code tiles a of stage j are free once the MMAs of stage j - kARing are
-  // done, which r_empty of that stage's slot also tells
-  uint64_t* a_full = r_empty + kRing;             // code tiles converted
-  uint64_t* acc_full = a_full + kARing;           // [kAcc]
+  uint64_t* r_free = r_raw + kRing;               // codes read by the converters
+  uint64_t* a_full = r_free + kRing;              // [kMaxARing] code tiles in tensor memory
+  uint64_t* a_empty = a_full + kMaxARing;         // [kMaxARing] their MMAs done
+  uint64_t* acc_full = a_empty + kMaxARing;       // [kAcc]
   uint64_t* acc_empty = acc_full + kAcc;          // [kAcc]
   uint64_t* xready = acc_empty + kAcc;            // X resident (fp16, swizzled)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xready + 1);
@@ -156,14 +158,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   // tile after tile, are the stages j = i * ns + ks of one ring
   const int ntl = ((int)blockIdx.x < tiles) ? (tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
   const int total = ntl * ns;
-  constexpr uint32_t kTmemCols = 2 * kAcc * NT < 32 ? 32 : 2 * kAcc * NT;
 
   if (tid == 0) {
     for (int s = 0; s < kRing; ++s) {
       mbar_init(&r_raw[s], 1);
-      mbar_init(&r_empty[s], 1);
+      mbar_init(&r_free[s], 32 * kConv);
     }
-    for (int a = 0; a < kARing; ++a) mbar_init(&a_full[a], 32 * kConv);
+    for (int a = 0; a < kARing; ++a) {
+      mbar_init(&a_full[a], 32 * kConv);
+      mbar_init(&a_empty[a], 1);
+    }
     for (int b = 0; b < kAcc; ++b) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], 128);
@@ -175,7 +179,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kConv + 4) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(tmem_slot)),
-                 "r"(kTmemCols));
+                 "r"(512));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -203,7 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int issued = pre;
       for (int j = pre; j < total; ++j) {
         const int s = j % kRing;
-        if (!wait_bar(&r_empty[s], (uint32_t)((j / kRing) + 1) & 1u, abort)) {
+        if (!wait_bar(&r_free[s], (uint32_t)((j / kRing) + 1) & 1u, abort)) {
           ok = false;
           *abort = 1;
           break;
@@ -225,33 +229,50 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < kConv) {
     // ------------------------------------------------------ converters
+    // warp w: rows 32 (w % 4) + lane (its tensor-memory lanes) of group
+    // w / 4 of each stage; a thread converts its row's 64 codes and stores
+    // them with one tcgen05.st (32 columns of fp16 pairs)
+    const int q = warp & 3, h = warp >> 2;
+    const int r = 32 * q + lane;
     for (int j = 0; j < total; ++j) {
       const int s = j % kRing, a = j % kARing;
       const uint32_t par = (uint32_t)(j / kRing) & 1u;
       if (!wait_bar(&r_raw[s], par, abort) ||
-          (j >= kARing && !wait_bar(&r_empty[(j - kARing) % kRing],
-                                    (uint32_t)((j - kARing) / kRing) & 1u, abort))) {
+          (j >= kARing && !wait_bar(&a_empty[a], (uint32_t)((j / kARing) + 1) & 1u, abort))) {
         ok = false;
         *abort = 1;
         break;
       }
-      uint8_t* at = atiles + (size_t)a * kTileA;
-      const uint8_t* raw = slots + (size_t)s * kSlot;
+      const uint8_t* row = slots + (size_t)s * kSlot + r * 128;
+      uint32_t v[32];
 #pragma unroll
-      for (int it = 0; it < 1024 / (32 * kConv); ++it) {
-        // 16-byte piece: row flat / 8, columns 16 (flat % 8) .. of the
-        // stage's 128; group h = piece / 4 of the two
-        const int flat = it * 32 * kConv + tid;
-        const int r = flat >> 3, p = flat & 7, h = p >> 2, c0 = 2 * (p & 3);
-        const uint4 c = *reinterpret_cast<const uint4*>(raw + r * (2 * kBK) + p * 16);
-        const uint4 lo = make_uint4(codes01(c.x), codes23(c.x), codes01(c.y), codes23(c.y));
-        const uint4 hi = make_uint4(codes01(c.z), codes23(c.z), codes01(c.w), codes23(c.w));
-        uint8_t* t = at + h * (kBM * kBK * 2) + r * 128;
-        *reinterpret_cast<uint4*>(t + ((c0 ^ (r & 7)) << 4)) = lo;
-        *reinterpret_cast<uint4*>(t + (((c0 + 1) ^ (r & 7)) << 4)) = hi;
+      for (int c = 0; c < 4; ++c) {  // 16-byte chunk 4 h + c of the row, swizzled by TMA
+        const uint4 w = *reinterpret_cast<const uint4*>(row + (((4 * h + c) ^ (r & 7)) << 4));
+        v[8 * c + 0] = codes01(w.x);
+        v[8 * c + 1] = codes23(w.x);
+        v[8 * c + 2] = codes01(w.y);
+        v[8 * c + 3] = codes23(w.y);
+        v[8 * c + 4] = codes01(w.z);
+        v[8 * c + 5] = codes23(w.z);
+        v[8 * c + 6] = codes01(w.w);
+        v[8 * c + 7] = codes23(w.w);
       }
-      // make the generic-proxy stores visible to the tensor core
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      const uint32_t ta = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(kAccCols + a * 64 + h * 32);
+      asm volatile(
+          "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+          "%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(ta),
+          "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+          "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+          "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
+          "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
+          "r"(v[29]), "r"(v[30]), "r"(v[31])
+          : "memory");
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+      // the slot's raw codes are consumed only here: the store above used
+      // every value loaded from it (arriving earlier would let the next TMA
+      // overwrite the slot under loads still in flight)
+      mbar_arrive(&r_free[s]);
       mbar_arrive(&a_full[a]);
     }
     if (!ok) *abort = 1;
@@ -264,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         *abort = 1;
       }
       for (int j = 0; j < total && ok; ++j) {
-        const int s = j % kRing, a = j % kARing, b = j % kAcc;
+        const int a = j % kARing, b = j % kAcc;
         if (!wait_bar(&a_full[a], (uint32_t)(j / kARing) & 1u, abort) ||
             (j >= kAcc && !wait_bar(&acc_empty[b], (uint32_t)((j / kAcc) + 1) & 1u, abort))) {
           ok = false;
@@ -274,24 +295,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         const int g0 = (j % ns) * 2;  // the stage's first group
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const uint32_t sa = smem_u32(atiles + (size_t)a * kTileA + h * (kBM * kBK * 2));
-          const uint32_t sb = smem_u32(xres + (size_t)(g0 + h) * (NT * kBK * 2));
-          const uint32_t d = tmem + (uint32_t)((2 * b + h) * NT);
+        for (int hh = 0; hh < 2; ++hh) {
+          const uint32_t ta = tmem + (uint32_t)(kAccCols + a * 64 + hh * 32);
+          const uint32_t sb = smem_u32(xres + (size_t)(g0 + hh) * (NT * kBK * 2));
+          const uint32_t d = tmem + (uint32_t)((2 * b + hh) * NT);
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k) {
-            const uint64_t da = smem_desc(sa + k * 32), db = smem_desc(sb + k * 32);
+            const uint64_t db = smem_desc(sb + k * 32);
             const uint32_t acc = k > 0 ? 1u : 0u;
             asm volatile(
                 "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-                " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d),
-                "l"(da), "l"(db), "r"(idesc), "r"(acc)
+                " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d),
+                "r"(ta + (uint32_t)(k * 8)), "l"(db), "r"(idesc), "r"(acc)
                 : "memory");
           }
         }
         asm volatile(
             "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                smem_u32(&r_empty[s]))
+                smem_u32(&a_empty[a]))
             : "memory");
         asm volatile(
             "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -424,8 +445,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kConv + 4) {
     __syncwarp();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
-                 "r"(kTmemCols));
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
   }
 }
 
@@ -463,7 +483,7 @@ cudaError_t gemm_affine8_skinny_launch(const A8Seg* segs, int nseg, const uint16
   for (int i = 0; i < nseg; ++i) {
     P.seg[i] = gas::Seg{segs[i].s, segs[i].b, segs[i].y, segs[i].res, segs[i].N, segs[i].y_bf16,
                         tiles};
-    if (!make_u8_map(&maps.w[i], segs[i].w, segs[i].N, K, 2 * gas::kBK, gas::kBM))
+    if (!make_u8_map(&maps.w[i], segs[i].w, segs[i].N, K, 2 * gas::kBK, gas::kBM, true))
       return cudaErrorInvalidValue;
     tiles += (segs[i].N + gas::kBM - 1) / gas::kBM;
   }

@@ -659,10 +659,11 @@ bool make_bf16_map(CUtensorMap* map, const void* base, int rows, int cols, int b
 }
 
 // A byte [rows][cols] row-major tensor (row stride cols bytes, a multiple
-// of 16) in boxes of box_cols x box_rows, no swizzle; bytes past the end
-// read as zero.
+// of 16) in boxes of box_cols x box_rows, with no swizzle or the 128-byte
+// one (box_cols = 128: 16-byte chunk c of a box row r lands at chunk
+// c ^ (r % 8)); bytes past the end read as zero.
 bool make_u8_map(CUtensorMap* map, const void* base, int rows, int cols, int box_cols,
-                 int box_rows) {
+                 int box_rows, bool swizzle128) {
   EncodeTiledFn enc = encode_tiled();
   if (!enc) return false;
   const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
@@ -670,7 +671,8 @@ bool make_u8_map(CUtensorMap* map, const void* base, int rows, int cols, int box
   const cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 

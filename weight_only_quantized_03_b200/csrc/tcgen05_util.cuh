@@ -12,9 +12,10 @@ namespace qg {
 // zero); false when the driver's encoder is unavailable or refuses it.
 bool make_bf16_map(CUtensorMap* map, const void* base, int rows, int cols, int box_rows);
 // Host: a TMA descriptor of a byte [rows][cols] row-major tensor (cols a
-// multiple of 16) in boxes of box_cols x box_rows, no swizzle.
+// multiple of 16) in boxes of box_cols x box_rows, no swizzle or (with
+// swizzle128 and box_cols = 128) the 128-byte swizzle.
 bool make_u8_map(CUtensorMap* map, const void* base, int rows, int cols, int box_cols,
-                 int box_rows);
+                 int box_rows, bool swizzle128 = false);
 
 namespace tc {
 
