@@ -178,6 +178,7 @@ GEMM_CASES = [
     (130, 256, 128, True, True),       # ragged M, one 256-column tile
     (200, 384, 192, True, False),      # 128-column tiles, three K stages
     (257, 512, 1280, False, False),    # K ring wraps (20 stages over 4)
+    (5, 128, 256, True, True),         # one raw chunk of W (K = 256), a 5-row A tile
     # the Whisper-large-v3 encoder projections at M = 1500 frames
     (1500, 1280, 1280, True, False),
     (1500, 5120, 1280, True, False),

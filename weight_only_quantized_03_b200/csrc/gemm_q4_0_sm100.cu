@@ -11,7 +11,10 @@
 // Structure
 //   1. a_to_bf16_kernel: A fp32 -> bf16 into the workspace (once per call;
 //      every N tile then reads half the bytes).
-//   2. gemm_q4_0_tc_kernel, one CTA per 128 x BN output tile, over a ring of
+//   2. K % 256 == 0 (every Whisper projection): gemm_q4_0_t_kernel, the
+//      transposed form described at its definition (W dequantized into
+//      tensor memory as the MMA's A operand, A's rows as its B operand).
+//      Otherwise gemm_q4_0_tc_kernel, one CTA per 128 x BN output tile, over a ring of
 //      shared-memory stages of 64 columns of K, both operands in the K-major
 //      128-byte-swizzled layout the tensor core reads (16-byte chunk c of
 //      row r at chunk c ^ (r % 8) of its 1024-byte atom):
@@ -409,72 +412,221 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 
-// ---------------------------------------------------------------------------
-// The same matmul with W's raw bytes staged by TMA (K % 256 == 0, so every
-// row's byte length is a multiple of 16): warp 9 also copies, per four MMA
-// stages, a BN x 144-byte box of raw Q4_0 rows (two blocks a stage) into a
-// two-slot ring; the W producers then read their 36 bytes from shared memory
-// instead of issuing nine scattered global loads per stage. Everything else
-// (the stage ring, the MMA issue, the epilogue, the bounded waits) is as in
-// gemm_q4_0_tc_kernel.
-// ---------------------------------------------------------------------------
+// W's raw Q4_0 rows staged by TMA (K % 256 == 0, so every row's byte length
+// is a multiple of 16): a box of kRawRow bytes a row covers four MMA stages
+// (two Q4_0 blocks a stage).
 constexpr int kRawStages = 4;                 // MMA stages per raw chunk
 constexpr int kRawRow = kRawStages * 36;      // 144 bytes of a row per chunk
-constexpr int kRawSlots = 2;
 
-template <int BN, int MT>
-struct Cfg2 {
-  static constexpr int kStageA = MT * kBM * kBK * 2;
-  static constexpr int kStageB = BN * kBK * 2;
-  static constexpr int kStage = kStageA + kStageB;
-  static constexpr int kRawSlot = ((BN * kRawRow) + 1023) / 1024 * 1024;
-  static constexpr int kBudget = 220 * 1024 - kRawSlots * kRawSlot;
-  static constexpr int kStages = kBudget / kStage < 4 ? kBudget / kStage : 4;
-  static constexpr int kSmem = 1024 + kStages * kStage + kRawSlots * kRawSlot + 1024;
-  static constexpr int kTmemCols = MT * BN;
+// ---------------------------------------------------------------------------
+// Transposed form (K % 256 == 0). The tile is 128 rows of W by TN rows of A:
+// D[n][m] = sum_k W[n][k] A[m][k], so W is the MMA's A operand and comes from
+// tensor memory. The converter warps dequantize each stage's 128 x 64 block
+// of W straight into a ring of tensor-memory stages with tcgen05.st (thread
+// = W row = tensor-memory lane): no swizzled shared-memory stores, no proxy
+// fence, and shared memory left for a deep ring of A's TN x 64 tiles, the B
+// operand, staged by TMA with the 128-byte swizzle. Roles:
+//   warps 0 .. kTConv-1  converters, then the epilogue. They form
+//              kTGroups groups of 8 warps that take the stages in turn
+//              (group g: stages k = g mod kTGroups), since one stage's
+//              conversion is a chain of latencies (shared-memory loads, the
+//              arithmetic, the tensor-memory store) rather than work; in a
+//              group, warp w holds W rows 32 (w % 4) + lane of Q4_0 block
+//              (w / 4) % 2. A converter issues stage k's store, converts its
+//              next stage, and only then waits for the store and publishes
+//              stage k;
+//   warp kTConv  lane 0: TMA for A's stages and for W's raw rows (144 bytes
+//              a row = four stages per chunk, a ring of kTRaw chunks);
+//   warp kTConv+1  tensor-memory allocation; lane 0 issues four MMAs a
+//              stage (M = 128, N = TN, K = 16, bf16 -> fp32) and commits.
+// ---------------------------------------------------------------------------
+constexpr int kTConv = 16;                 // converter (and epilogue) warps
+constexpr int kTGroups = kTConv / 8;       // converter groups, stages taken in turn
+constexpr int kTThreads = 32 * (kTConv + 2);
+constexpr int kTCols = 16;                 // tensor-memory columns a converter thread stores a stage
+constexpr int kTARing = 8;                 // tensor-memory W stages, 32 columns each
+constexpr int kTRaw = 3;                   // raw W chunks in flight
+
+template <int TN>
+struct CfgT {
+  static constexpr int kStageB = TN * kBK * 2;  // A's rows of a stage, bf16
+  static constexpr int kRawSlot = kBM * kRawRow;  // 18 KB
+  static constexpr int kRoom = 216 * 1024 - kTRaw * kRawSlot;
+  static constexpr int kStages = kRoom / kStageB > 8 ? 8 : kRoom / kStageB;
+  static constexpr int kSmem = 1024 + kStages * kStageB + kTRaw * kRawSlot + 512;
+  static constexpr int kAccCols = TN;           // accumulator: columns [0, TN)
+  static_assert(TN + kTARing * 32 <= 512, "tensor memory");
 };
 
-template <int BN, int MT>
-__global__ void __launch_bounds__(kThreads, 1)
-    gemm_q4_0_tc2_kernel(const __grid_constant__ CUtensorMap tmA,
-                         const __grid_constant__ CUtensorMap tmW, const Epi ep, int M, int N,
-                         int K, unsigned* __restrict__ err) {
-  using G = Cfg2<BN, MT>;
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Q4_0 block H of a stage (halfwords 9H .. 9H + 8 of its 36 raw bytes: the
+// fp16 d, then 16 code bytes) as bf16 pairs in k order, pair j = values
+// 2j, 2j + 1: values 0-15 are the low nibbles of code bytes 0-15 (pairs
+// 0-7), values 16-31 the high ones (pairs 8-15). Each value (n - 8) d is
+// exact in fp32 and rounds once to bf16, as in store_w_row.
+template <int H>
+__device__ __forceinline__ void w_block_pairs(const uint32_t (&raw)[9], uint32_t (&v)[16]) {
+  auto hw = [&](int i) -> uint32_t {
+    const int k = 9 * H + i;
+    return (raw[k >> 1] >> (16 * (k & 1))) & 0xFFFFu;
+  };
+  const float d = __half2float(__ushort_as_half((unsigned short)hw(0)));
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const uint32_t b2 = hw(1 + q);  // code bytes 2q, 2q + 1
+    v[q] = bf16x2(nib_m8(b2, 0) * d, nib_m8(b2, 8) * d);
+    v[q + 8] = bf16x2(nib_m8(b2, 4) * d, nib_m8(b2, 12) * d);
+  }
+}
+// a converter's 16 pairs of a stage: Q4_0 block p (columns 16 p .. 16 p + 15)
+__device__ __forceinline__ void w_stage_pairs(const uint32_t (&raw)[9], int p, uint32_t (&v)[16]) {
+  if (p == 0) w_block_pairs<0>(raw, v);
+  else w_block_pairs<1>(raw, v);
+}
+__device__ __forceinline__ void tmem_st_pairs(uint32_t ta, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+      "%13,%14,%15,%16};" ::"r"(ta),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15])
+      : "memory");
+}
+
+// The epilogue of the transposed tile: warp w reads tensor-memory lanes
+// 32 (w % 4) .. +31 (W rows n, columns of C) and half of the TN columns
+// (A rows m); each value goes through the Epi rules to C[m][n] (a warp's
+// stores for one m are 32 consecutive n).
+template <int TN>
+__device__ __forceinline__ void epilogue_t(uint32_t tmem, uint64_t* done, volatile int* abort,
+                                           const Epi& ep, int M, int N, int m0, int n0, int warp,
+                                           int lane, bool ok, unsigned* err) {
+  bool landed = true;
+  if (warp < kTConv) {
+    int st = 0;
+    if (lane == 0) {
+      bool l = mbar_try_wait(done, 0);
+      if (!l) {
+        const unsigned long long t0 = now_ns();
+        while (!(l = mbar_try_wait(done, 0)))
+          if (now_ns() - t0 > kWaitNs) break;
+      }
+      st = (l ? 1 : 0) | (*abort ? 2 : 0);
+    }
+    st = __shfl_sync(0xffffffffu, st, 0);
+    landed = (st & 1) != 0;
+    const bool aborted = (st & 2) != 0;
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    if (landed && !aborted) {
+      const int q = warp & 3, part = warp >> 2;
+      const int n = n0 + 32 * q + lane;
+      const float bias = ep.bias ? ep.bias[n] : 0.f;
+      // this warp's kCols columns in rounds of 64: both 32-column loads of a
+      // round are in flight before the one wait
+      constexpr int kCols = TN / (kTConv / 4);
+      constexpr int kRound = kCols < 64 ? kCols : 64;
+#pragma unroll 1
+      for (int c0 = part * kCols; c0 < (part + 1) * kCols; c0 += kRound) {
+        if (m0 + c0 >= M) break;
+        uint32_t v[kRound];
+#pragma unroll
+        for (int hb = 0; hb < kRound / 32; ++hb) {
+          const uint32_t ta = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(c0 + 32 * hb);
+          uint32_t* w = v + 32 * hb;
+          asm volatile(
+              "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+              "%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+              : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]),
+                "=r"(w[6]), "=r"(w[7]), "=r"(w[8]), "=r"(w[9]), "=r"(w[10]), "=r"(w[11]),
+                "=r"(w[12]), "=r"(w[13]), "=r"(w[14]), "=r"(w[15]), "=r"(w[16]), "=r"(w[17]),
+                "=r"(w[18]), "=r"(w[19]), "=r"(w[20]), "=r"(w[21]), "=r"(w[22]), "=r"(w[23]),
+                "=r"(w[24]), "=r"(w[25]), "=r"(w[26]), "=r"(w[27]), "=r"(w[28]), "=r"(w[29]),
+                "=r"(w[30]), "=r"(w[31])
+              : "r"(ta));
+        }
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+        for (int j = 0; j < kRound; ++j) {
+          const int m = m0 + c0 + j;
+          if (m < M) {
+            const size_t ci = (size_t)m * N + n;
+            float o = __uint_as_float(v[j]);
+            if (ep.bias) o += bias;
+            if (ep.res) o += ep.res[ci];
+            if (ep.gelu) o = gelu_tanh_f(o);
+            if (ep.c_bf16)
+              reinterpret_cast<uint16_t*>(ep.C)[ci] = f32_to_bf16_bits(o);
+            else
+              reinterpret_cast<float*>(ep.C)[ci] = o;
+          }
+        }
+      }
+    }
+    if (!landed || aborted) ok = false;
+  }
+  if (!ok && err) atomicOr(err, 1u);
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (warp == kTConv + 1) {
+    __syncwarp();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+  }
+}
+
+template <int TN>
+__global__ void __launch_bounds__(kTThreads, 1)
+    gemm_q4_0_t_kernel(const __grid_constant__ CUtensorMap tmA,
+                       const __grid_constant__ CUtensorMap tmW, const Epi ep, int M, int N, int K,
+                       unsigned* __restrict__ err) {
+  using G = CfgT<TN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t* stages = smem;
-  uint8_t* raws = smem + G::kStages * G::kStage;
-  uint64_t* full = reinterpret_cast<uint64_t*>(raws + kRawSlots * G::kRawSlot);
-  uint64_t* tfull = full + G::kStages;
-  uint64_t* empty = tfull + G::kStages;
-  uint64_t* rfull = empty + G::kStages;
-  uint64_t* rempty = rfull + kRawSlots;
-  uint64_t* done = rempty + kRawSlots;
+  uint8_t* bst = smem;                                 // A's stages (the MMA's B operand)
+  uint8_t* raws = smem + G::kStages * G::kStageB;      // W's raw chunks
+  uint64_t* bfull = reinterpret_cast<uint64_t*>(raws + kTRaw * G::kRawSlot);
+  uint64_t* bempty = bfull + G::kStages;
+  uint64_t* rfull = bempty + G::kStages;
+  uint64_t* rempty = rfull + kTRaw;
+  uint64_t* afull = rempty + kTRaw;
+  uint64_t* aempty = afull + kTARing;
+  uint64_t* done = aempty + kTARing;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * (MT * kBM);
-  const int nk = K / kBK, nchunk = (nk + kRawStages - 1) / kRawStages;
+  const int n0 = blockIdx.x * kBM, m0 = blockIdx.y * TN;
+  const int nk = K / kBK, nchunk = nk / kRawStages;  // K % 256 == 0
 
   if (tid == 0) {
     for (int s = 0; s < G::kStages; ++s) {
-      mbar_init(&full[s], kProducers);
-      mbar_init(&tfull[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&bfull[s], 1);
+      mbar_init(&bempty[s], 1);
     }
-    for (int r = 0; r < kRawSlots; ++r) {
+    for (int r = 0; r < kTRaw; ++r) {
       mbar_init(&rfull[r], 1);
-      mbar_init(&rempty[r], kProducers);
+      mbar_init(&rempty[r], 32 * kTConv);  // every group reads every chunk
+    }
+    for (int a = 0; a < kTARing; ++a) {
+      mbar_init(&afull[a], 32 * 8);        // the group that converts the stage
+      mbar_init(&aempty[a], 1);
     }
     mbar_init(done, 1);
     *abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 8) {
+  if (warp == kTConv + 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(tmem_slot)),
-                 "r"(G::kTmemCols));
+                 "r"(512));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -483,85 +635,82 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   bool ok = true;
-  if (warp < 8) {
-    // ------------------------------------------------------ W producers
-    const bool has_row = tid < BN;
-    for (int kb = 0; kb < nk && ok; ++kb) {
-      const int c = kb / kRawStages, sub = kb % kRawStages, slot = c % kRawSlots;
-      if (sub == 0 && !wait_bar(&rfull[slot], (uint32_t)(c / kRawSlots) & 1u, abort)) {
+  if (warp < kTConv) {
+    // ------------------------------------------------------ converters
+    const int q = warp & 3, p = (warp >> 2) & 1, grp = warp >> 3, r = 32 * q + lane;
+    // stage k is published (its store waited for, the ring slots released)
+    // once the group's next stage has been converted
+    auto publish = [&](int k) {
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+      // the raw chunk is consumed once the stores have used its last
+      // stage's values
+      if (k % kRawStages + kTGroups >= kRawStages)  // this group's last stage of the chunk
+        mbar_arrive(&rempty[(k / kRawStages) % kTRaw]);
+      mbar_arrive(&afull[k % kTARing]);
+    };
+    int pend = -1;  // stage whose store is issued but not yet published
+    for (int kb = grp; kb < nk; kb += kTGroups) {
+      const int c = kb / kRawStages, sub = kb % kRawStages, slot = c % kTRaw, a = kb % kTARing;
+      // (sub < kTGroups: this group's first stage of the chunk)
+      if ((sub < kTGroups && !wait_bar(&rfull[slot], (uint32_t)(c / kTRaw) & 1u, abort)) ||
+          (kb >= kTARing &&
+           !wait_bar(&aempty[a], (uint32_t)((kb / kTARing) + 1) & 1u, abort))) {
         ok = false;
         break;
       }
-      const int s = kb % G::kStages;
-      if (kb >= G::kStages &&
-          !wait_bar(&empty[s], (uint32_t)((kb / G::kStages) + 1) & 1u, abort)) {
-        ok = false;
-        break;
-      }
-      if (has_row) {
-        const uint32_t* rw =
-            reinterpret_cast<const uint32_t*>(raws + slot * G::kRawSlot + tid * kRawRow + sub * 36);
-        uint32_t raw[9];
+      const uint32_t* rw =
+          reinterpret_cast<const uint32_t*>(raws + slot * G::kRawSlot + r * kRawRow + sub * 36);
+      uint32_t raw[9];
 #pragma unroll
-        for (int i = 0; i < 9; ++i) raw[i] = rw[i];
-        store_w_row(stages + (size_t)s * G::kStage + G::kStageA, tid, raw);
-      }
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      mbar_arrive(&full[s]);
-      if (sub == kRawStages - 1 || kb == nk - 1) mbar_arrive(&rempty[slot]);
+      for (int i = 0; i < 9; ++i) raw[i] = rw[i];
+      uint32_t v[kTCols];
+      w_stage_pairs(raw, p, v);
+      if (pend >= 0) publish(pend);
+      tmem_st_pairs(tmem + ((uint32_t)(32 * q) << 16) +
+                        (uint32_t)(G::kAccCols + a * 32 + p * kTCols),
+                    v);
+      pend = kb;
     }
+    if (ok && pend >= 0) publish(pend);
     if (!ok) *abort = 1;
-  } else if (warp == 9) {
-    // ------------------------------ A and W's raw chunks by TMA (lane 0)
+  } else if (warp == kTConv) {
+    // ------------------------------ A's stages and W's raw chunks by TMA
     if (lane == 0) {
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmW)) : "memory");
       int issued = 0, rissued = 0;
       auto issue_raw = [&](int c) -> bool {
-        const int slot = c % kRawSlots;
-        if (c >= kRawSlots &&
-            !wait_bar(&rempty[slot], (uint32_t)((c / kRawSlots) + 1) & 1u, abort))
+        const int slot = c % kTRaw;
+        if (c >= kTRaw && !wait_bar(&rempty[slot], (uint32_t)((c / kTRaw) + 1) & 1u, abort))
           return false;
-        mbar_expect_tx(&rfull[slot], (uint32_t)(BN * kRawRow));
-        asm volatile(
-            "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-            " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(raws + slot * G::kRawSlot)),
-            "l"(reinterpret_cast<uint64_t>(&tmW)), "r"(c * kRawRow), "r"(n0),
-            "r"(smem_u32(&rfull[slot]))
-            : "memory");
+        mbar_expect_tx(&rfull[slot], (uint32_t)G::kRawSlot);
+        tma_load_2d(smem_u32(raws + slot * G::kRawSlot), &tmW, c * kRawRow, n0, &rfull[slot]);
         ++rissued;
         return true;
       };
-      if (!issue_raw(0)) {
-        ok = false;
-        *abort = 1;
-      }
+      for (int c = 0; c < kTRaw && c < nchunk && ok; ++c)
+        if (!issue_raw(c)) ok = false;
       for (int kb = 0; kb < nk && ok; ++kb) {
-        if (kb % kRawStages == 0 && kb / kRawStages + 1 < nchunk &&
-            !issue_raw(kb / kRawStages + 1)) {
-          ok = false;
-          *abort = 1;
-          break;
+        // the raw chunks run kTRaw - 1 chunks ahead of the stage in progress
+        if (kb > 0 && kb % kRawStages == 0) {
+          const int c = kb / kRawStages + kTRaw - 1;
+          if (c < nchunk && !issue_raw(c)) {
+            ok = false;
+            break;
+          }
         }
         const int s = kb % G::kStages;
         if (kb >= G::kStages &&
-            !wait_bar(&empty[s], (uint32_t)((kb / G::kStages) + 1) & 1u, abort)) {
+            !wait_bar(&bempty[s], (uint32_t)((kb / G::kStages) + 1) & 1u, abort)) {
           ok = false;
-          *abort = 1;
           break;
         }
-        mbar_expect_tx(&tfull[s], (uint32_t)G::kStageA);
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt)
-          asm volatile(
-              "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-              " [%0], [%1, {%2, %3}], [%4];" ::"r"(
-                  smem_u32(stages + (size_t)s * G::kStage + mt * kBM * kBK * 2)),
-              "l"(reinterpret_cast<uint64_t>(&tmA)), "r"(kb * kBK), "r"(m0 + mt * kBM),
-              "r"(smem_u32(&tfull[s]))
-              : "memory");
+        mbar_expect_tx(&bfull[s], (uint32_t)G::kStageB);
+        tma_load_2d(smem_u32(bst + (size_t)s * G::kStageB), &tmA, kb * kBK, m0, &bfull[s]);
         ++issued;
       }
+      if (!ok) *abort = 1;
       // no copy may land after the CTA is gone: wait (bounded) for the last
       // fill of every stage and raw slot used
       auto drain = [&](uint64_t* bars, int nslots, int count) {
@@ -575,41 +724,40 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       };
-      drain(tfull, G::kStages, issued);
-      drain(rfull, kRawSlots, rissued);
+      drain(bfull, G::kStages, issued);
+      drain(rfull, kTRaw, rissued);
     }
   } else if (lane == 0) {
     // ------------------------------------------------------- MMA issuer
-    const uint32_t idesc = instr_desc<BN>();
+    const uint32_t idesc = instr_desc<TN>();
     for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % G::kStages;
-      const uint32_t par = (uint32_t)(kb / G::kStages) & 1u;
-      if (!wait_bar(&tfull[s], par, abort) || !wait_bar(&full[s], par, abort)) {
+      const int s = kb % G::kStages, a = kb % kTARing;
+      if (!wait_bar(&bfull[s], (uint32_t)(kb / G::kStages) & 1u, abort) ||
+          !wait_bar(&afull[a], (uint32_t)(kb / kTARing) & 1u, abort)) {
         ok = false;
         *abort = 1;
         break;
       }
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      const uint32_t sa = smem_u32(stages + (size_t)s * G::kStage);
-      const uint32_t sb = sa + G::kStageA;
+      const uint32_t sb = smem_u32(bst + (size_t)s * G::kStageB);
+      const uint32_t ta = tmem + (uint32_t)(G::kAccCols + a * 32);
 #pragma unroll
       for (int k = 0; k < kBK / 16; ++k) {
         const uint64_t db = smem_desc(sb + k * 32);
         const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-          const uint64_t da = smem_desc(sa + mt * kBM * kBK * 2 + k * 32);
-          asm volatile(
-              "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-              " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
-                  tmem + (uint32_t)(mt * BN)),
-              "l"(da), "l"(db), "r"(idesc), "r"(acc)
-              : "memory");
-        }
+        asm volatile(
+            "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+            " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(tmem),
+            "r"(ta + (uint32_t)(k * 8)), "l"(db), "r"(idesc), "r"(acc)
+            : "memory");
       }
       asm volatile(
           "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-              smem_u32(&empty[s]))
+              smem_u32(&bempty[s]))
+          : "memory");
+      asm volatile(
+          "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+              smem_u32(&aempty[a]))
           : "memory");
     }
     asm volatile(
@@ -617,7 +765,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             smem_u32(done))
         : "memory");
   }
-  epilogue<BN, MT>(tmem, done, abort, ep, M, N, m0, n0, warp, lane, ok, err);
+  epilogue_t<TN>(tmem, done, abort, ep, M, N, m0, n0, warp, lane, ok, err);
 }
 }  // namespace gq4
 
@@ -718,45 +866,38 @@ static bool make_w_raw_map(CUtensorMap* map, const uint8_t* blocks, int N, int K
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, int MT>
-static cudaError_t gq4_launch2(const CUtensorMap& tmA, const CUtensorMap& tmW, const gq4::Epi& ep,
-                               int M, int N, int K, unsigned* err, cudaStream_t st) {
-  using G = gq4::Cfg2<BN, MT>;
-  ensure_smem((const void*)gq4::gemm_q4_0_tc2_kernel<BN, MT>, G::kSmem);
-  dim3 grid(N / BN, (M + MT * gq4::kBM - 1) / (MT * gq4::kBM));
-  return launch_pdl(gq4::gemm_q4_0_tc2_kernel<BN, MT>, grid, dim3(gq4::kThreads),
-                    (size_t)G::kSmem, st, false, tmA, tmW, ep, M, N, K, err);
-}
-
-template <int BN>
-static cudaError_t gq4_launch2_mt(const CUtensorMap& tmA, const CUtensorMap& tmW,
-                                  const gq4::Epi& ep, int M, int N, int K, unsigned* err,
-                                  cudaStream_t st) {
-  const long long tiles2 = (long long)(N / BN) * ((M + 255) / 256);
-  if (2 * tiles2 >= num_sms()) return gq4_launch2<BN, 2>(tmA, tmW, ep, M, N, K, err, st);
-  return gq4_launch2<BN, 1>(tmA, tmW, ep, M, N, K, err, st);
+template <int TN>
+static cudaError_t gq4_launch_t(const CUtensorMap& tmA, const CUtensorMap& tmW, const gq4::Epi& ep,
+                                int M, int N, int K, unsigned* err, cudaStream_t st) {
+  using G = gq4::CfgT<TN>;
+  ensure_smem((const void*)gq4::gemm_q4_0_t_kernel<TN>, G::kSmem);
+  dim3 grid(N / gq4::kBM, (M + TN - 1) / TN);
+  return launch_pdl(gq4::gemm_q4_0_t_kernel<TN>, grid, dim3(gq4::kTThreads), (size_t)G::kSmem, st,
+                    false, tmA, tmW, ep, M, N, K, err);
 }
 
 // The GEMM on a bf16 A already in device memory (`Ab`, [M][K]); `err` is the
 // workspace error word.
 static qg_status gq4_run(const uint8_t* blocks, const uint16_t* Ab, const gq4::Epi& ep, int M,
                          int N, int K, unsigned* err, cudaStream_t s, const char* what) {
+  if (K % 256 == 0 && aligned(blocks, 16)) {
+    // the transposed form: W's raw rows and A's tiles staged by TMA, W
+    // dequantized into tensor memory; 256 rows of A a tile while that still
+    // fills the SMs, else 128
+    const int TN = (long long)(N / gq4::kBM) * ((M + 255) / 256) >= num_sms() ? 256 : 128;
+    CUtensorMap tmA, tmW;
+    if (!make_bf16_map(&tmA, Ab, M, K, TN) || !make_w_raw_map(&tmW, blocks, N, K, gq4::kBM)) {
+      set_error("%s: could not encode a TMA descriptor", what);
+      return QG_ERR_CUDA;
+    }
+    if (TN == 256) gq4_launch_t<256>(tmA, tmW, ep, M, N, K, err, s);
+    else gq4_launch_t<128>(tmA, tmW, ep, M, N, K, err, s);
+    return check_launch(what);
+  }
   CUtensorMap tmA;
   if (!make_a_map(&tmA, Ab, M, K)) {
     set_error("%s: could not encode the TMA descriptor of A", what);
     return QG_ERR_CUDA;
-  }
-  if (K % 256 == 0 && aligned(blocks, 16)) {
-    // W's raw bytes staged by TMA
-    const int BN = N % 256 == 0 ? 256 : 128;
-    CUtensorMap tmW;
-    if (!make_w_raw_map(&tmW, blocks, N, K, BN)) {
-      set_error("%s: could not encode the TMA descriptor of W", what);
-      return QG_ERR_CUDA;
-    }
-    if (BN == 256) gq4_launch2_mt<256>(tmA, tmW, ep, M, N, K, err, s);
-    else gq4_launch2_mt<128>(tmA, tmW, ep, M, N, K, err, s);
-    return check_launch(what);
   }
   const bool w32 = aligned(blocks, 4);
   if (N % 256 == 0) {
