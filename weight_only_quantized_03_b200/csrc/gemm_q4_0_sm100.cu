@@ -435,16 +435,21 @@ constexpr int kRawRow = kRawStages * 36;      // 144 bytes of a row per chunk
 //              (w / 4) % 2. A converter issues stage k's store, converts its
 //              next stage, and only then waits for the store and publishes
 //              stage k;
-//   warp kTConv  lane 0: TMA for A's stages and for W's raw rows (144 bytes
-//              a row = four stages per chunk, a ring of kTRaw chunks);
+//   warp kTConv  lane 0: TMA for A's stages;
 //   warp kTConv+1  tensor-memory allocation; lane 0 issues four MMAs a
-//              stage (M = 128, N = TN, K = 16, bf16 -> fp32) and commits.
+//              stage (M = 128, N = TN, K = 16, bf16 -> fp32) and commits;
+//   warp kTConv+2  lane 0: TMA for W's raw rows (144 bytes a row = four
+//              stages per chunk, a ring of kTRaw chunks), apart from A's
+//              loads so that neither waits behind the other.
+// A stage's A tile and W columns share one full/empty barrier pair, so the
+// MMA thread has one wait and one commit a stage.
 // ---------------------------------------------------------------------------
-constexpr int kTConv = 16;                 // converter (and epilogue) warps
+constexpr int kTConv = 16;                 // converter warps (16 or 24)
 constexpr int kTGroups = kTConv / 8;       // converter groups, stages taken in turn
-constexpr int kTThreads = 32 * (kTConv + 2);
+constexpr int kTEpi = 16;                  // the first kTEpi converter warps then run the epilogue
+constexpr int kTThreads = 32 * (kTConv + 3);
+constexpr bool kTPipe = false;             // publish a stage only after converting the next (measured slower)
 constexpr int kTCols = 16;                 // tensor-memory columns a converter thread stores a stage
-constexpr int kTARing = 8;                 // tensor-memory W stages, 32 columns each
 constexpr int kTRaw = 3;                   // raw W chunks in flight
 
 template <int TN>
@@ -455,7 +460,9 @@ struct CfgT {
   static constexpr int kStages = kRoom / kStageB > 8 ? 8 : kRoom / kStageB;
   static constexpr int kSmem = 1024 + kStages * kStageB + kTRaw * kRawSlot + 512;
   static constexpr int kAccCols = TN;           // accumulator: columns [0, TN)
-  static_assert(TN + kTARing * 32 <= 512, "tensor memory");
+  // stage s of the ring: A's tile in shared memory and W's 32 tensor-memory
+  // columns from kAccCols + 32 s, filled and freed together
+  static_assert(TN + kStages * 32 <= 512, "tensor memory");
 };
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
@@ -510,7 +517,7 @@ __device__ __forceinline__ void epilogue_t(uint32_t tmem, uint64_t* done, volati
                                            const Epi& ep, int M, int N, int m0, int n0, int warp,
                                            int lane, bool ok, unsigned* err) {
   bool landed = true;
-  if (warp < kTConv) {
+  if (warp < kTEpi) {
     int st = 0;
     if (lane == 0) {
       bool l = mbar_try_wait(done, 0);
@@ -531,8 +538,8 @@ __device__ __forceinline__ void epilogue_t(uint32_t tmem, uint64_t* done, volati
       const float bias = ep.bias ? ep.bias[n] : 0.f;
       // this warp's kCols columns in rounds of 64: both 32-column loads of a
       // round are in flight before the one wait
-      constexpr int kCols = TN / (kTConv / 4);
-      constexpr int kRound = kCols < 64 ? kCols : 64;
+      constexpr int kCols = TN / (kTEpi / 4);
+      constexpr int kRound = kCols < 64 && kTConv <= 16 ? kCols : (kTConv <= 16 ? 64 : 32);
 #pragma unroll 1
       for (int c0 = part * kCols; c0 < (part + 1) * kCols; c0 += kRound) {
         if (m0 + c0 >= M) break;
@@ -582,6 +589,20 @@ __device__ __forceinline__ void epilogue_t(uint32_t tmem, uint64_t* done, volati
   }
 }
 
+// no copy may land after the CTA is gone: wait (bounded) for the last fill of
+// every slot of a ring (count fills issued over nslots slots)
+__device__ __forceinline__ void tma_drain(uint64_t* bars, int nslots, int count) {
+  for (int j = count - nslots > 0 ? count - nslots : 0; j < count; ++j) {
+    const int s = j % nslots;
+    const uint32_t par = (uint32_t)(j / nslots) & 1u;
+    if (!mbar_try_wait(&bars[s], par)) {
+      const unsigned long long t0 = now_ns();
+      while (!mbar_try_wait(&bars[s], par))
+        if (now_ns() - t0 > kWaitNs) break;
+    }
+  }
+}
+
 template <int TN>
 __global__ void __launch_bounds__(kTThreads, 1)
     gemm_q4_0_t_kernel(const __grid_constant__ CUtensorMap tmA,
@@ -592,13 +613,13 @@ __global__ void __launch_bounds__(kTThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* bst = smem;                                 // A's stages (the MMA's B operand)
   uint8_t* raws = smem + G::kStages * G::kStageB;      // W's raw chunks
-  uint64_t* bfull = reinterpret_cast<uint64_t*>(raws + kTRaw * G::kRawSlot);
-  uint64_t* bempty = bfull + G::kStages;
-  uint64_t* rfull = bempty + G::kStages;
+  // full[s]: A's tile landed (TMA bytes) and W's stage converted; empty[s]:
+  // the MMAs reading both are done (one commit)
+  uint64_t* full = reinterpret_cast<uint64_t*>(raws + kTRaw * G::kRawSlot);
+  uint64_t* empty = full + G::kStages;
+  uint64_t* rfull = empty + G::kStages;
   uint64_t* rempty = rfull + kTRaw;
-  uint64_t* afull = rempty + kTRaw;
-  uint64_t* aempty = afull + kTARing;
-  uint64_t* done = aempty + kTARing;
+  uint64_t* done = rempty + kTRaw;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -608,16 +629,12 @@ __global__ void __launch_bounds__(kTThreads, 1)
 
   if (tid == 0) {
     for (int s = 0; s < G::kStages; ++s) {
-      mbar_init(&bfull[s], 1);
-      mbar_init(&bempty[s], 1);
+      mbar_init(&full[s], 32 * 8 + 1);  // the converting group and the TMA's arrival
+      mbar_init(&empty[s], 1);
     }
     for (int r = 0; r < kTRaw; ++r) {
       mbar_init(&rfull[r], 1);
       mbar_init(&rempty[r], 32 * kTConv);  // every group reads every chunk
-    }
-    for (int a = 0; a < kTARing; ++a) {
-      mbar_init(&afull[a], 32 * 8);        // the group that converts the stage
-      mbar_init(&aempty[a], 1);
     }
     mbar_init(done, 1);
     *abort = 0;
@@ -645,17 +662,17 @@ __global__ void __launch_bounds__(kTThreads, 1)
       asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
       // the raw chunk is consumed once the stores have used its last
       // stage's values
-      if (k % kRawStages + kTGroups >= kRawStages)  // this group's last stage of the chunk
-        mbar_arrive(&rempty[(k / kRawStages) % kTRaw]);
-      mbar_arrive(&afull[k % kTARing]);
+      if (k % kRawStages + kTGroups >= kRawStages)  // the group's last stage of the chunk
+        mbar_arrive(&rempty[(k / kRawStages) % kTRaw]);  // (every group has one: 4 >= groups)
+      mbar_arrive(&full[k % G::kStages]);
     };
     int pend = -1;  // stage whose store is issued but not yet published
     for (int kb = grp; kb < nk; kb += kTGroups) {
-      const int c = kb / kRawStages, sub = kb % kRawStages, slot = c % kTRaw, a = kb % kTARing;
-      // (sub < kTGroups: this group's first stage of the chunk)
+      const int c = kb / kRawStages, sub = kb % kRawStages, slot = c % kTRaw, a = kb % G::kStages;
+      // (sub < kTGroups: the group's first stage of the chunk)
       if ((sub < kTGroups && !wait_bar(&rfull[slot], (uint32_t)(c / kTRaw) & 1u, abort)) ||
-          (kb >= kTARing &&
-           !wait_bar(&aempty[a], (uint32_t)((kb / kTARing) + 1) & 1u, abort))) {
+          (kb >= G::kStages &&
+           !wait_bar(&empty[a], (uint32_t)((kb / G::kStages) + 1) & 1u, abort))) {
         ok = false;
         break;
       }
@@ -671,79 +688,68 @@ __global__ void __launch_bounds__(kTThreads, 1)
                         (uint32_t)(G::kAccCols + a * 32 + p * kTCols),
                     v);
       pend = kb;
+      // the first stage goes out at once: the MMA has nothing else to do yet
+      if (!kTPipe || kb < kTGroups) {
+        publish(kb);
+        pend = -1;
+      }
     }
     if (ok && pend >= 0) publish(pend);
     if (!ok) *abort = 1;
   } else if (warp == kTConv) {
-    // ------------------------------ A's stages and W's raw chunks by TMA
+    // ----------------------- A's stages by TMA (lane 0), as far ahead as the ring allows
     if (lane == 0) {
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
-      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmW)) : "memory");
-      int issued = 0, rissued = 0;
-      auto issue_raw = [&](int c) -> bool {
-        const int slot = c % kTRaw;
-        if (c >= kTRaw && !wait_bar(&rempty[slot], (uint32_t)((c / kTRaw) + 1) & 1u, abort))
-          return false;
-        mbar_expect_tx(&rfull[slot], (uint32_t)G::kRawSlot);
-        tma_load_2d(smem_u32(raws + slot * G::kRawSlot), &tmW, c * kRawRow, n0, &rfull[slot]);
-        ++rissued;
-        return true;
-      };
-      for (int c = 0; c < kTRaw && c < nchunk && ok; ++c)
-        if (!issue_raw(c)) ok = false;
+      int issued = 0;
       for (int kb = 0; kb < nk && ok; ++kb) {
-        // the raw chunks run kTRaw - 1 chunks ahead of the stage in progress
-        if (kb > 0 && kb % kRawStages == 0) {
-          const int c = kb / kRawStages + kTRaw - 1;
-          if (c < nchunk && !issue_raw(c)) {
-            ok = false;
-            break;
-          }
-        }
         const int s = kb % G::kStages;
         if (kb >= G::kStages &&
-            !wait_bar(&bempty[s], (uint32_t)((kb / G::kStages) + 1) & 1u, abort)) {
+            !wait_bar(&empty[s], (uint32_t)((kb / G::kStages) + 1) & 1u, abort)) {
           ok = false;
           break;
         }
-        mbar_expect_tx(&bfull[s], (uint32_t)G::kStageB);
-        tma_load_2d(smem_u32(bst + (size_t)s * G::kStageB), &tmA, kb * kBK, m0, &bfull[s]);
+        mbar_expect_tx(&full[s], (uint32_t)G::kStageB);  // (the TMA's arrival)
+        tma_load_2d(smem_u32(bst + (size_t)s * G::kStageB), &tmA, kb * kBK, m0, &full[s]);
         ++issued;
       }
       if (!ok) *abort = 1;
-      // no copy may land after the CTA is gone: wait (bounded) for the last
-      // fill of every stage and raw slot used
-      auto drain = [&](uint64_t* bars, int nslots, int count) {
-        for (int j = count - nslots > 0 ? count - nslots : 0; j < count; ++j) {
-          const int s = j % nslots;
-          const uint32_t par = (uint32_t)(j / nslots) & 1u;
-          if (!mbar_try_wait(&bars[s], par)) {
-            const unsigned long long t0 = now_ns();
-            while (!mbar_try_wait(&bars[s], par))
-              if (now_ns() - t0 > kWaitNs) break;
-          }
-        }
-      };
-      drain(bfull, G::kStages, issued);
-      drain(rfull, kTRaw, rissued);
+      tma_drain(full, G::kStages, issued);
     }
-  } else if (lane == 0) {
+  } else if (warp == kTConv + 2) {
+    // ------------------------------------ W's raw chunks by TMA (lane 0)
+    if (lane == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmW)) : "memory");
+      int rissued = 0;
+      for (int c = 0; c < nchunk && ok; ++c) {
+        const int slot = c % kTRaw;
+        if (c >= kTRaw && !wait_bar(&rempty[slot], (uint32_t)((c / kTRaw) + 1) & 1u, abort)) {
+          ok = false;
+          break;
+        }
+        mbar_expect_tx(&rfull[slot], (uint32_t)G::kRawSlot);
+        tma_load_2d(smem_u32(raws + slot * G::kRawSlot), &tmW, c * kRawRow, n0, &rfull[slot]);
+        ++rissued;
+      }
+      if (!ok) *abort = 1;
+      tma_drain(rfull, kTRaw, rissued);
+    }
+  } else if (warp == kTConv + 1 && lane == 0) {
     // ------------------------------------------------------- MMA issuer
     const uint32_t idesc = instr_desc<TN>();
     for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % G::kStages, a = kb % kTARing;
-      if (!wait_bar(&bfull[s], (uint32_t)(kb / G::kStages) & 1u, abort) ||
-          !wait_bar(&afull[a], (uint32_t)(kb / kTARing) & 1u, abort)) {
+      const int s = kb % G::kStages;
+      if (!wait_bar(&full[s], (uint32_t)(kb / G::kStages) & 1u, abort)) {
         ok = false;
         *abort = 1;
         break;
       }
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      const uint32_t sb = smem_u32(bst + (size_t)s * G::kStageB);
-      const uint32_t ta = tmem + (uint32_t)(G::kAccCols + a * 32);
+      // K step k starts 32 bytes further: 2 in the descriptor's address field
+      const uint64_t db0 = smem_desc(smem_u32(bst + (size_t)s * G::kStageB));
+      const uint32_t ta = tmem + (uint32_t)(G::kAccCols + s * 32);
 #pragma unroll
       for (int k = 0; k < kBK / 16; ++k) {
-        const uint64_t db = smem_desc(sb + k * 32);
+        const uint64_t db = db0 + (uint64_t)(2 * k);
         const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
         asm volatile(
             "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
@@ -753,11 +759,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
       }
       asm volatile(
           "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-              smem_u32(&bempty[s]))
-          : "memory");
-      asm volatile(
-          "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-              smem_u32(&aempty[a]))
+              smem_u32(&empty[s]))
           : "memory");
     }
     asm volatile(
