@@ -58,8 +58,8 @@ constexpr int kThreads = 32 * (kConv + 6);  // converters, 4 drains, MMA, TMA
 // waits and commits for two groups' MMAs. The converted codes live in
 // tensor memory, as the MMA's A operand.
 constexpr int kRing = 8;                   // stages of raw codes in flight
-constexpr int kMaxARing = 6;               // code tiles in tensor memory (two groups each)
-constexpr int kAcc = 4;                    // accumulator pairs in tensor memory
+constexpr int kAcc = 4;                    // stages in tensor memory: a code tile (two
+                                           // groups) and an accumulator pair each
 constexpr int kSlot = kBM * 2 * kBK;       // raw code bytes of two groups, 16 KB
 constexpr int kXBytes = 64 * 1024;     // resident X: NT * K * 2 <= 64 KB
 constexpr int kSmem = 1024 + kXBytes + kRing * kSlot + kMaxGroups * 32 * 4 +
@@ -132,9 +132,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     gemm_affine8_skinny_kernel(const __grid_constant__ Maps maps, const __grid_constant__ Params P,
                                int tiles, unsigned* __restrict__ err) {
   // tensor memory: kAcc accumulator pairs (2 NT columns each), then the ring
-  // of converted code tiles (two groups of 32 columns each)
+  // of converted code tiles (two groups of 32 columns each). Stage j uses
+  // pair and tile j % kAcc; one barrier pair per slot serves both:
+  // ready[b] completes when the converters have filled the tile and the
+  // drains have read the pair's previous accumulators, done[b] (one commit)
+  // when the stage's MMAs are done.
   constexpr int kAccCols = 2 * kAcc * NT;
-  constexpr int kARing = (512 - kAccCols) / 64;
+  static_assert(kAccCols + kAcc * 64 <= 512, "tensor memory");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* xres = smem;                           // [K/64][NT][64] fp16, swizzled
@@ -144,11 +148,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint16_t* tbi = tsc + kMaxGroups * 128;                             // [K/64][128] biases
   uint64_t* r_raw = reinterpret_cast<uint64_t*>(tbi + kMaxGroups * 128);  // codes landed
   uint64_t* r_free = r_raw + kRing;               // codes read by the converters
-  uint64_t* a_full = r_free + kRing;              // [kMaxARing] code tiles in tensor memory
-  uint64_t* a_empty = a_full + kMaxARing;         // [kMaxARing] their MMAs done
-  uint64_t* acc_full = a_empty + kMaxARing;       // [kAcc]
-  uint64_t* acc_empty = acc_full + kAcc;          // [kAcc]
-  uint64_t* xready = acc_empty + kAcc;            // X resident (fp16, swizzled)
+  uint64_t* ready = r_free + kRing;               // [kAcc] tile converted, pair free
+  uint64_t* done = ready + kAcc;                  // [kAcc] the stage's MMAs done
+  uint64_t* xready = done + kAcc;                 // X resident (fp16, swizzled)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xready + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -164,13 +166,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&r_raw[s], 1);
       mbar_init(&r_free[s], 32 * kConv);
     }
-    for (int a = 0; a < kARing; ++a) {
-      mbar_init(&a_full[a], 32 * kConv);
-      mbar_init(&a_empty[a], 1);
-    }
     for (int b = 0; b < kAcc; ++b) {
-      mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 128);
+      mbar_init(&ready[b], 32 * kConv + 128);  // the converters and the drains
+      mbar_init(&done[b], 1);
     }
     mbar_init(xready, 128);
     *abort = 0;
@@ -235,10 +233,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3, h = warp >> 2;
     const int r = 32 * q + lane;
     for (int j = 0; j < total; ++j) {
-      const int s = j % kRing, a = j % kARing;
+      const int s = j % kRing, a = j % kAcc;
       const uint32_t par = (uint32_t)(j / kRing) & 1u;
       if (!wait_bar(&r_raw[s], par, abort) ||
-          (j >= kARing && !wait_bar(&a_empty[a], (uint32_t)((j / kARing) + 1) & 1u, abort))) {
+          (j >= kAcc && !wait_bar(&done[a], (uint32_t)((j / kAcc) + 1) & 1u, abort))) {
         ok = false;
         *abort = 1;
         break;
@@ -273,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // every value loaded from it (arriving earlier would let the next TMA
       // overwrite the slot under loads still in flight)
       mbar_arrive(&r_free[s]);
-      mbar_arrive(&a_full[a]);
+      mbar_arrive(&ready[a]);
     }
     if (!ok) *abort = 1;
   } else if (warp == kConv + 4) {
@@ -285,9 +283,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         *abort = 1;
       }
       for (int j = 0; j < total && ok; ++j) {
-        const int a = j % kARing, b = j % kAcc;
-        if (!wait_bar(&a_full[a], (uint32_t)(j / kARing) & 1u, abort) ||
-            (j >= kAcc && !wait_bar(&acc_empty[b], (uint32_t)((j / kAcc) + 1) & 1u, abort))) {
+        const int a = j % kAcc, b = a;
+        if (!wait_bar(&ready[b], (uint32_t)(j / kAcc) & 1u, abort)) {
           ok = false;
           *abort = 1;
           break;
@@ -312,11 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         asm volatile(
             "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                smem_u32(&a_empty[a]))
-            : "memory");
-        asm volatile(
-            "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                smem_u32(&acc_full[b]))
+                smem_u32(&done[b]))
             : "memory");
       }
     }
@@ -327,6 +320,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int col = tid - 32 * kConv;  // this drain thread's row of the tile
     // the sum of each group of x per row (rows past T are zero), in order:
     // X is the same for every tile, so once per CTA
+    // every accumulator pair starts free
+    for (int b = 0; b < kAcc; ++b) mbar_arrive(&ready[b]);
     pdl_wait();  // x is written by the previous kernel
     float mx = 0.f;
     for (int i = col; i < Kg * NT; i += 128) {
@@ -397,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int n = 0; n < NT; ++n) acc[n] = 0.f;
       }
-      if (!wait_bar(&acc_full[b], (uint32_t)(j / kAcc) & 1u, abort)) {
+      if (!wait_bar(&done[b], (uint32_t)(j / kAcc) & 1u, abort)) {
         ok = false;
         *abort = 1;
         break;
@@ -408,7 +403,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld<NT>(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)((2 * b + 1) * NT), v1);
       asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
       asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-      mbar_arrive(&acc_empty[b]);
+      mbar_arrive(&ready[b]);  // the pair is free for stage j + kAcc
       const int g0 = 2 * ks;
       const float s0 = bf16_bits_to_f32(tsc[g0 * 128 + col]);
       const float s1 = bf16_bits_to_f32(tsc[(g0 + 1) * 128 + col]);
