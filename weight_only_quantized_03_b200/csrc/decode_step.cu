@@ -232,6 +232,15 @@ constexpr bool kStepFuseOProj = true;
 constexpr bool kStepFuseOProj = false;
 #endif
 
+// The tensor-core GEMV can form its input in its prologue (RMSNorm of the
+// residual stream, SiLU(gate) * up), which saves a launch per layer at batch
+// 1. But every CTA forms all B x K values: measured on the B200 in the
+// 1.7B-shaped step at batch 8 (K = 6144 for down), the down GEMV spent 43 us
+// after its wait doing so. Past this many values the input is formed once by
+// its own kernel (RMSNorm or SiLU-mul, bf16 out) and the GEMV reads it as is.
+constexpr long long kFusePrologueMaxBK = 8192;
+static bool fuse_prologue(int B, int K) { return (long long)B * K <= kFusePrologueMaxBK; }
+
 static bool head_uses_gemm(const qg_qwen3_config& c, int N, int B) {
   return B >= kStepGemmBatch && c.hidden % 64 == 0 && (N + 127) / 128 >= num_sms();
 }
@@ -295,7 +304,7 @@ static void enqueue_layers(const qg_qwen3_config& c, const qg_qwen3_layer* layer
     // RMSNorm and SiLU-mul run in the next GEMV's prologue where the
     // tensor-core GEMV takes the shape, as separate kernels otherwise
     tl_set_kind(kTlQkv);
-    if (gemv_tc_eligible(qkv, 3, c.hidden, B, false)) {
+    if (fuse_prologue(B, c.hidden) && gemv_tc_eligible(qkv, 3, c.hidden, B, false)) {
       gemv_tc_launch_rmsnorm(qkv, 3, x, L.input_norm, c.eps, c.hidden, B, s, true, sb.xn, &pf_o);
     } else {
       rmsnorm_launch(x, L.input_norm, c.eps, sb.xn, true, B, c.hidden, s, true);
@@ -316,7 +325,7 @@ static void enqueue_layers(const qg_qwen3_config& c, const qg_qwen3_layer* layer
     GemvSeg gu[2] = {{L.gate.w, L.gate.scales, L.gate.biases, sb.gate, nullptr, c.ffn, 0},
                      {L.up.w, L.up.scales, L.up.biases, sb.up, nullptr, c.ffn, 0}};
     tl_set_kind(kTlGateUp);
-    if (gemv_tc_eligible(gu, 2, c.hidden, B, false)) {
+    if (fuse_prologue(B, c.hidden) && gemv_tc_eligible(gu, 2, c.hidden, B, false)) {
       gemv_tc_launch_rmsnorm(gu, 2, sb.xa, L.post_norm, c.eps, c.hidden, B, s, true, sb.xn2,
                              &pf_next_qkv);
     } else {
@@ -325,7 +334,7 @@ static void enqueue_layers(const qg_qwen3_config& c, const qg_qwen3_layer* layer
     }
     GemvSeg dn = {L.down.w, L.down.scales, L.down.biases, x, sb.xa, c.hidden, 0};
     tl_set_kind(kTlDown);
-    if (gemv_tc_eligible(&dn, 1, c.ffn, B, false)) {
+    if (fuse_prologue(B, c.ffn) && gemv_tc_eligible(&dn, 1, c.ffn, B, false)) {
       gemv_tc_launch_silu_mul(&dn, 1, sb.gate, sb.up, c.ffn, B, s, true, sb.hm, &pf_next_kv);
     } else {
       const int n = B * c.ffn;
@@ -354,7 +363,7 @@ static void enqueue_head(const qg_qwen3_config& c, const qg_affine8_matrix& head
     rmsnorm_launch(sb.x, final_norm, c.eps, sb.xnf, true, B, c.hidden, s, true);
     const A8Seg m = {head.w, head.scales, head.biases, logits, nullptr, N, 0};
     gemm_affine8_launch(&m, 1, sb.xnf, B, c.hidden, sb.err, s, true, nullptr);
-  } else if (gemv_tc_eligible(&h, 1, c.hidden, B, false)) {
+  } else if (fuse_prologue(B, c.hidden) && gemv_tc_eligible(&h, 1, c.hidden, B, false)) {
     gemv_tc_launch_rmsnorm(&h, 1, sb.x, final_norm, c.eps, c.hidden, B, s, true);
   } else {
     rmsnorm_launch(sb.x, final_norm, c.eps, sb.xnf, true, B, c.hidden, s, true);
