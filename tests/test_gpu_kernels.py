@@ -120,14 +120,16 @@ def test_gemv_affine8(N, K, B, xd, yd, res, quant):
     assert_parity(host64(y), ref, bf16_out=(yd == "bf16"), what=f"gemv {N}x{K} B={B}")
 
 
-def test_gemv_affine8_large_activations_prescaled():
+@pytest.mark.parametrize("B,K", [(2, 1024), (8, 2048)])
+def test_gemv_affine8_large_activations_prescaled(B, K):
     # |x| far beyond fp16's range: the tensor-core path prescales x by a
-    # power of two, so the products stay exact and nothing overflows
-    N, K = 300, 1024
+    # power of two, so the products stay exact and nothing overflows (B x K
+    # = 8 x 2048 takes the bulk copy of x into shared memory)
+    N = 300
     w, s, b = qg_synth.affine8_packed(N, K, 77)
-    xf = (qg_synth.gaussian((2, K), 1.0, 78) * 2.0 ** 20).astype(np.float32)
+    xf = (qg_synth.gaussian((B, K), 1.0, 78) * 2.0 ** 20).astype(np.float32)
     xbits = qg_synth.f32_to_bf16_bits(xf)
-    y = torch.empty((2, N), dtype=torch.float32, device="cuda")
+    y = torch.empty((B, N), dtype=torch.float32, device="cuda")
     qg.qg_gemv_affine8_g64(dev(w), dev(s), dev(b), bf16_dev(xbits), y)
     ref = O.gemv_affine8(w, s, b, O.bf16_bits_to_f64(xbits))
     assert_parity(host64(y), ref, what="prescaled x")

@@ -48,14 +48,14 @@
 namespace qg {
 namespace gtc {
 
-template <int NT, int W>
+template <int NT, int W, bool BULK>
 __global__ void __launch_bounds__(W * 32, 1)
     gemv_tc_kernel(const __grid_constant__ Params P) {
   extern __shared__ __align__(16) uint8_t smem[];
   tl_entry(P.tl);
   // the next kernel may be scheduled as soon as the weight loads are out (its
   // own wait still covers all of this one)
-  gemv_tc_body<NT, W>(P, smem, [&] {
+  gemv_tc_body<NT, W, BULK>(P, smem, [&] {
     pdl_trigger();
     pdl_wait();
     tl_wait(P.tl);
@@ -79,11 +79,21 @@ bool gemv_tc_eligible(const GemvSeg* segs, int nseg, int K, int B, bool x_f32) {
   return std::max(gtc_smem(K, NT, 16), gtc_smem(K, NT, 8)) <= 200 * 1024;
 }
 
+template <int NT, int W, bool BULK>
+static cudaError_t gtc_launch_k(const gtc::Params& P, dim3 grid, cudaStream_t st, bool pdl) {
+  const size_t smem = gtc_smem(P.K, NT, W);
+  if (smem > 48 * 1024) ensure_smem((const void*)gtc::gemv_tc_kernel<NT, W, BULK>, 200 * 1024);
+  return launch_pdl(gtc::gemv_tc_kernel<NT, W, BULK>, grid, dim3(W * 32), smem, st, pdl, P);
+}
+// the bulk instantiation for a bf16 x with more 128-column items per CTA
+// (its first batch tile's rows times K / 128) than its warps keep in
+// registers (three each)
 template <int NT, int W>
 static cudaError_t gtc_launch_nt(const gtc::Params& P, dim3 grid, cudaStream_t st, bool pdl) {
-  const size_t smem = gtc_smem(P.K, NT, W);
-  if (smem > 48 * 1024) ensure_smem((const void*)gtc::gemv_tc_kernel<NT, W>, 200 * 1024);
-  return launch_pdl(gtc::gemv_tc_kernel<NT, W>, grid, dim3(W * 32), smem, st, pdl, P);
+  const int bt = std::min(P.B, 4 * NT);
+  const bool bulk = P.xmode == gtc::kXBf16 && bt * (P.K / 128) > 3 * W && aligned(P.x, 16);
+  return bulk ? gtc_launch_k<NT, W, true>(P, grid, st, pdl)
+              : gtc_launch_k<NT, W, false>(P, grid, st, pdl);
 }
 
 static cudaError_t gtc_launch(const GemvSeg* segs, int nseg, gtc::Params& P, int K, int B,

@@ -140,7 +140,10 @@ __device__ __forceinline__ void chunk_mma(const uint32_t (&w)[16], const uint4& 
 // flight and before anything written upstream is read (the
 // programmatic-dependent-launch trigger and wait). smem: gtc_smem(K, NT, W)
 // bytes.
-template <int NT, int W, class Wait>
+// BULK: the instantiation with the bulk copy of a bf16 x (below); without
+// it the kernel carries none of that code (the batch-1 decode chain is
+// sensitive to the kernel's size: instruction fetch stalls lead its profile)
+template <int NT, int W, bool BULK, class Wait>
 __device__ __forceinline__ void gemv_tc_body(const Params& P, uint8_t* smem, Wait&& wait) {
   constexpr int kWarps = W, kThreads = W * 32;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -275,10 +278,16 @@ __device__ __forceinline__ void gemv_tc_body(const Params& P, uint8_t* smem, Wai
     }
     return va;
   };
+  // A bf16 x with more items than the warps keep in registers (large B x
+  // K) goes to shared memory in bulk instead: 16-byte copies, four in flight
+  // a thread, then an in-place conversion to fp16 (the item path would load
+  // and form those items one dependent round at a time)
+  const bool bulk = BULK && P.xmode == kXBf16 && nitems > kItems * kWarps &&
+                    (reinterpret_cast<uintptr_t>(P.x) & 15) == 0;
   float4 xv[kItems];
 #pragma unroll
   for (int j = 0; j < kItems; ++j)
-    xv[j] = j < my_items ? load_item(warp + j * kWarps) : make_float4(0.f, 0.f, 0.f, 0.f);
+    xv[j] = !bulk && j < my_items ? load_item(warp + j * kWarps) : make_float4(0.f, 0.f, 0.f, 0.f);
   // residual of the first block this warp stores (lane (g, t): rows g, g + 8
   // of batch row 4 nt + t)
   float resv[NT][2];
@@ -384,7 +393,59 @@ __device__ __forceinline__ void gemv_tc_body(const Params& P, uint8_t* smem, Wai
     }
     return mloc;
   };
-  float mx = form(1.0f);
+  // bulk: x's bf16 rows copied as they are into xh; returns this thread's max|x|
+  auto bulk_copy = [&]() -> float {
+    const int vpr = K / 8, nvec = Bt * vpr;
+    float m = 0.f;
+    for (int i0 = tid; i0 < nvec; i0 += kThreads * 4) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * kThreads;
+        v[u] = make_uint4(0u, 0u, 0u, 0u);
+        if (i < nvec)
+          v[u] = __ldcg(reinterpret_cast<const uint4*>(P.x + (size_t)(b0 + i / vpr) * K) + i % vpr);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * kThreads;
+        if (i < nvec) {
+          *reinterpret_cast<uint4*>(xh + (i / vpr) * xs + (i % vpr) * 8) = v[u];
+          const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) m = fmaxf(m, fmaxf(fabsf(bf16_lo(w[k])), fabsf(bf16_hi(w[k]))));
+        }
+      }
+    }
+    return m;
+  };
+  // bulk: xh converted in place to fp16 x * down, and each 64-column
+  // group's fp16 sum to gsum; eight lanes a group (lane & 7: its 16-byte
+  // chunk), the sum over them in a fixed order
+  auto bulk_convert = [&](float down) {
+    const int ng = Bt * Kg;
+    for (int gi0 = warp * 4; gi0 < ng; gi0 += kWarps * 4) {
+      const int gi = gi0 + (lane >> 3), c8 = lane & 7;
+      float sum = 0.f;
+      if (gi < ng) {
+        uint4* p = reinterpret_cast<uint4*>(xh + (gi / Kg) * xs + (gi % Kg) * 64 + c8 * 8);
+        const uint4 w = *p;
+        uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const __half2 h = __floats2half2_rn(bf16_lo(ww[k]) * down, bf16_hi(ww[k]) * down);
+          ww[k] = *reinterpret_cast<const uint32_t*>(&h);
+          sum += __low2float(h) + __high2float(h);
+        }
+        *p = make_uint4(ww[0], ww[1], ww[2], ww[3]);
+      }
+      sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+      sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+      sum += __shfl_xor_sync(0xffffffffu, sum, 4);
+      if (c8 == 0 && gi < ng) gsum[gi] = sum;  // gsum [4 NT][Kg]: row b at b Kg
+    }
+  };
+  float mx = bulk ? bulk_copy() : form(1.0f);
   for (int i = Bt * Kg + tid; i < 4 * NT * Kg; i += kThreads) gsum[i] = 0.f;
   // 3) max|x| over the CTA; prescale 2^-e so that max|x| * 2^-e < 2^15
   mx = warp_max(mx);
@@ -397,7 +458,10 @@ __device__ __forceinline__ void gemv_tc_body(const Params& P, uint8_t* smem, Wai
   int e = 0;  // NaN or inf in x propagate to y without a prescale
   if (mx >= 32768.f && mx <= 3.0e38f) e = (int)ceilf(log2f(mx / 16384.f));
   const float up = exp2f((float)e);
-  if (e != 0) {  // uniform over the CTA
+  if (bulk) {  // (uniform over the CTA) xh holds the raw copy until here
+    bulk_convert(exp2f((float)-e));
+    __syncthreads();
+  } else if (e != 0) {  // uniform over the CTA
     form(exp2f((float)-e));
     __syncthreads();
   }
