@@ -305,6 +305,7 @@ ATTN_CASES = [
     (1, 4, 4, 256, 40, [40]),
     (10, 16, 8, 128, 513, [512, 1, 100, 511, 256, 2, 3, 400, 512, 77]),
     (1, 16, 8, 128, 2048, [2048]),
+    (1, 16, 8, 128, 2049, [1500]),     # clusters of 16 (chunks of 129 rows), the last ones empty
     (2, 8, 1, 32, 5, [0, 6]),          # invalid lengths -> zero rows
     (4, 16, 4, 128, 300, [300, 1, 150, 299]),   # 4 query heads per kv head
     (2, 6, 2, 64, 100, [100, 37]),              # 3 query heads per kv head

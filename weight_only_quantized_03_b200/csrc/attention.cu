@@ -101,7 +101,8 @@ namespace ac {
 
 constexpr int kNW = 8;                 // warps per CTA
 constexpr int kThreads = kNW * 32;
-constexpr int kMaxCluster = 8;         // portable cluster size
+constexpr int kPortableCluster = 8;    // portable cluster size
+constexpr int kMaxCluster = 16;        // non-portable, for long caches at few (sequence, kv head) pairs
 
 template <int D>
 struct Geo {
@@ -157,11 +158,15 @@ __device__ __forceinline__ void merge_state(float& m, float& l, float* o, float 
 // every rank's (max, sum, weighted value) is loaded first, so the reads of
 // distributed shared memory overlap in one round trip, then combined. An
 // empty rank has max -inf.
+// MC: the largest cluster the instantiation serves (8, or 16 for the
+// non-portable clusters of long caches; only those launches carry the wider
+// merge).
+template <int MC>
 __device__ __forceinline__ float merge_cluster(const float* m, const float* l, const float* o,
                                                unsigned cs, bool valid) {
-  float mv[kMaxCluster], lv[kMaxCluster], ov[kMaxCluster];
+  float mv[MC], lv[MC], ov[MC];
 #pragma unroll
-  for (int j = 0; j < kMaxCluster; ++j) {
+  for (int j = 0; j < MC; ++j) {
     mv[j] = -INFINITY;
     lv[j] = ov[j] = 0.f;
     if (j < (int)cs) {
@@ -172,11 +177,11 @@ __device__ __forceinline__ float merge_cluster(const float* m, const float* l, c
   }
   float M = -INFINITY;
 #pragma unroll
-  for (int j = 0; j < kMaxCluster; ++j) M = fmaxf(M, mv[j]);
+  for (int j = 0; j < MC; ++j) M = fmaxf(M, mv[j]);
   float Ls = 0.f, O = 0.f;
   if (M != -INFINITY) {
 #pragma unroll
-    for (int j = 0; j < kMaxCluster; ++j) {
+    for (int j = 0; j < MC; ++j) {
       if (mv[j] == -INFINITY) continue;
       const float e = expf(mv[j] - M);
       Ls = fmaf(lv[j], e, Ls);
@@ -200,7 +205,7 @@ __device__ __forceinline__ void cp_async_8(void* dst, const void* src) {
                : "memory");
 }
 
-template <int D, int GM, bool OPROJ>
+template <int D, int GM, bool OPROJ, int MC = kPortableCluster>
 __global__ void __launch_bounds__(kThreads, GM <= 2 ? 2 : 1)
 attention_cluster_kernel(const float* q, const uint16_t* kc, const uint16_t* vc,
                          const int32_t* __restrict__ kv_len, const int32_t* __restrict__ pos_for_len,
@@ -468,7 +473,7 @@ attention_cluster_kernel(const float* q, const uint16_t* kc, const uint16_t* vc,
   if (s == 0) {
     for (int i = threadIdx.x; i < g * D; i += kThreads) {
       const int h = i / D, d = i % D;
-      const float res = merge_cluster(&cm[h], &cl[h], &co[h][d], cs, valid);
+      const float res = merge_cluster<MC>(&cm[h], &cl[h], &co[h][d], cs, valid);
       const size_t oi = ((size_t)b * H + kv * g + h) * D + d;
       if (out_bf16)
         reinterpret_cast<uint16_t*>(out)[oi] = f32_to_bf16_bits(res);
@@ -809,7 +814,7 @@ attention_mma_kernel(const float* q, const uint16_t* kc, const uint16_t* vc,
   if (s == 0) {
     for (int i = tid; i < g * D; i += kMThreads) {
       const int h = i / D, d = i % D;
-      const float res = merge_cluster(&cm[h], &cl[h], &co[h][d], cs, valid);
+      const float res = merge_cluster<kPortableCluster>(&cm[h], &cl[h], &co[h][d], cs, valid);
       const size_t oi = ((size_t)b * H + kv * g + h) * D + d;
       if (out_bf16)
         reinterpret_cast<uint16_t*>(out)[oi] = f32_to_bf16_bits(res);
@@ -839,7 +844,7 @@ inline bool mma_ok(int B, int H, int Hkv, int D, int cap) {
 inline void mma_plan(int B, int Hkv, int cap, int& cs, int& ch) {
   const long long pairs = (long long)B * Hkv;
   long long c = (2LL * num_sms()) / pairs;
-  c = std::max<long long>(1, std::min<long long>(c, kMaxCluster));
+  c = std::max<long long>(1, std::min<long long>(c, kPortableCluster));
   const int blocks = (cap + kMB - 1) / kMB;
   c = std::min<long long>(c, blocks);
   ch = (int)((blocks + c - 1) / c) * kMB;
@@ -880,12 +885,17 @@ inline bool cluster_ok(int H, int Hkv, int D) {
 }
 
 // CTAs per (sequence, kv head): enough CTAs for about four waves of two
-// CTAs per SM, at most 8 (a portable cluster), and chunks of at least 16 rows.
+// CTAs per SM, chunks of at least 16 rows, and at most 8 (a portable
+// cluster) unless the chunks stay at least 128 rows long, up to 16. Measured
+// on the B200: clusters of 16 made the 0.6B step (KV 512, 32-row chunks)
+// slower, while a batch-1 cache of 2048 rows leaves 8 kv heads x 8 CTAs =
+// 64 CTAs, each with 256 rows to score.
 inline int cluster_size(int B, int Hkv, int cap) {
   const long long pairs = (long long)B * Hkv;
   long long cs = (8LL * num_sms() + pairs - 1) / pairs;
   cs = std::min<long long>(cs, (cap + 15) / 16);
-  cs = std::max<long long>(1, std::min<long long>(cs, kMaxCluster));
+  const long long most = std::max<long long>(kPortableCluster, std::min<long long>(kMaxCluster, cap / 128));
+  cs = std::max<long long>(1, std::min<long long>(cs, most));
   return (int)cs;
 }
 
@@ -919,6 +929,14 @@ cudaError_t launch(const float* q, const uint16_t* kc, const uint16_t* vc, const
   cfg.dynamicSmemBytes = OPROJ ? oproj_smem(fz.hidden, cs, (H / Hkv) * D) : 0;
   if (OPROJ)
     ensure_smem((const void*)attention_cluster_kernel<D, GM, true>, (int)cfg.dynamicSmemBytes);
+  const bool wide = !OPROJ && cs > kPortableCluster;  // (the fused o_proj keeps portable clusters)
+  if (wide) {
+    static std::once_flag once;
+    std::call_once(once, [] {
+      cudaFuncSetAttribute((const void*)attention_cluster_kernel<D, GM, false, kMaxCluster>,
+                           cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    });
+  }
   cfg.stream = st;
   cudaLaunchAttribute a[2];
   a[0].id = cudaLaunchAttributeClusterDimension;
@@ -930,6 +948,9 @@ cudaError_t launch(const float* q, const uint16_t* kc, const uint16_t* vc, const
   cfg.attrs = a;
   cfg.numAttrs = pdl ? 2 : 1;
   count_launch();
+  if (wide)
+    return cudaLaunchKernelEx(&cfg, attention_cluster_kernel<D, GM, false, kMaxCluster>, q, kc, vc,
+                              kv_len, pos_for_len, out, (int)out_bf16, H, Hkv, cap, scale, ch, fz);
   return cudaLaunchKernelEx(&cfg, attention_cluster_kernel<D, GM, OPROJ>, q, kc, vc, kv_len,
                             pos_for_len, out, (int)out_bf16, H, Hkv, cap, scale, ch, fz);
 }
@@ -1059,7 +1080,9 @@ cudaError_t attention_launch_step(const float* q, const float* k, const float* v
 
 bool attention_oproj_fusable(int B, int H, int Hkv, int D, int cap, int hidden) {
   if (!ac::cluster_ok(H, Hkv, D) || ac::mma_ok(B, H, Hkv, D, cap)) return false;
-  return ac::oproj_ok(hidden, ac::cluster_size(B, Hkv, cap), (H / Hkv) * D);
+  const int cs = ac::cluster_size(B, Hkv, cap);
+  // (the fused o_proj is built for portable clusters only)
+  return cs <= ac::kPortableCluster && ac::oproj_ok(hidden, cs, (H / Hkv) * D);
 }
 
 // Offset of the ticket counters inside an attention workspace.
