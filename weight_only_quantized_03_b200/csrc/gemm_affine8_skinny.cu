@@ -58,8 +58,9 @@ constexpr int kThreads = 32 * (kConv + 6);  // converters, 4 drains, MMA, TMA
 // waits and commits for two groups' MMAs. The converted codes live in
 // tensor memory, as the MMA's A operand.
 constexpr int kRing = 8;                   // stages of raw codes in flight
-constexpr int kAcc = 4;                    // stages in tensor memory: a code tile (two
-                                           // groups) and an accumulator pair each
+// stages in tensor memory (a code tile of two groups and an accumulator
+// pair each): 5 at NT = 16 (160 + 320 of the 512 columns), 4 at NT = 32
+constexpr int acc_slots(int NT) { return 2 * 5 * NT + 5 * 64 <= 512 ? 5 : 4; }
 constexpr int kSlot = kBM * 2 * kBK;       // raw code bytes of two groups, 16 KB
 constexpr int kXBytes = 64 * 1024;     // resident X: NT * K * 2 <= 64 KB
 constexpr int kSmem = 1024 + kXBytes + kRing * kSlot + kMaxGroups * 32 * 4 +
@@ -137,6 +138,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ready[b] completes when the converters have filled the tile and the
   // drains have read the pair's previous accumulators, done[b] (one commit)
   // when the stage's MMAs are done.
+  constexpr int kAcc = acc_slots(NT);
   constexpr int kAccCols = 2 * kAcc * NT;
   static_assert(kAccCols + kAcc * 64 <= 512, "tensor memory");
   extern __shared__ uint8_t smem_raw[];
