@@ -14,27 +14,30 @@
 // each group's scale and bias are applied to its partial sums afterwards.
 //
 // Persistent: one CTA per SM walks the 128-row tiles of W blockIdx.x,
-// + gridDim.x, ..., each over all K, for NT = 16 or 32 rows of X; its groups
-// in order, tile after tile, are the stages of one ring, so nothing drains
-// between tiles. Roles of a CTA:
-//   * the last warp (one lane) streams each group's raw code bytes [128][64]
-//     by TMA into a ring of slots (those of the first slots before the
-//     programmatic-dependent-launch wait);
-//   * warps 0-7 turn the codes into fp16 (q - 128) in the K-major 128-byte
-//     swizzled layout the tensor core reads (16-byte chunk c of row r at
-//     chunk c ^ (r % 8)): one byte permute and one packed subtract per two
-//     codes;
+// + gridDim.x, ..., each over all K, for NT = 16 or 32 rows of X. A stage is
+// two groups (128 columns); a CTA's stages in order, tile after tile, run
+// through one ring, so nothing drains between tiles. Roles of a CTA:
+//   * the last warp (one lane) streams each stage's raw code bytes [128][128]
+//     by TMA (128-byte swizzle) into a ring of shared-memory slots (those of
+//     the first slots before the programmatic-dependent-launch wait);
+//   * warps 0-7 (thread = row = tensor-memory lane; warp w: lane quadrant
+//     w % 4, group w / 4) turn a stage's codes into fp16 pairs q - 128 (one
+//     byte permute and one packed subtract per two codes) and store them
+//     into tensor memory with tcgen05.st, where the MMA reads them as its A
+//     operand;
 //   * warp 12 owns tensor memory; its lane 0 issues, per group, four
-//     tcgen05.mma (M = 128, N = NT, K = 16) into one of four accumulators
-//     (groups take them in turn), commits the stage back to the ring and the
-//     accumulator to the drain;
+//     tcgen05.mma (M = 128, N = NT, K = 16, A from tensor memory, B = X from
+//     shared memory) into the group's accumulator;
 //   * warps 8-11 (thread = row of the tile = tensor-memory lane) first form,
 //     once per CTA from X in global memory, the sums of x per group and row
-//     and max|x| (hence e), and write all of X as fp16 x * 2^-e in the same
-//     swizzled layout, where it stays for every tile (NT K 2 <= 64 KB); then
-//     they drain each group's accumulator with tcgen05.ld and fold it into
-//     fp32 registers with the group's scale (times 2^e) and bias, and store
-//     each tile's Y (+ R).
+//     and max|x| (hence e), and write all of X as fp16 x * 2^-e in the K-major
+//     128-byte swizzled layout the tensor core reads, where it stays for
+//     every tile (NT K 2 <= 64 KB); then they drain each group's accumulator
+//     with tcgen05.ld and fold it into fp32 registers with the group's scale
+//     (times 2^e) and bias, and store each tile's Y (+ R).
+// Tensor memory holds a ring of stage slots (5 at NT = 16, 4 at NT = 32):
+// a code tile and an accumulator pair each, with one barrier pair per slot
+// (filled: converters and drains; done: one MMA commit).
 // Every wait is bounded (1 s); a wait that gives up sets a CTA-wide abort
 // flag and the caller's error word, and tensor memory is freed only after
 // the last commit has landed.
