@@ -142,6 +142,15 @@ __device__ __forceinline__ float ld_cluster(const float* p, unsigned rank) {
   return v;
 }
 
+// fp32 v to the shared memory of CTA `rank` of the cluster, at the address
+// `p` has in this CTA's shared memory.
+__device__ __forceinline__ void st_cluster(float* p, float v, unsigned rank) {
+  const uint32_t local = (uint32_t)__cvta_generic_to_shared(p);
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(rank));
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote), "f"(v) : "memory");
+}
+
 // Merge (m2, l2, o2) into (m, l, o): the larger max wins, the other side is
 // scaled by exp(its max - new max). An empty side has max -inf, sum 0.
 __device__ __forceinline__ void merge_state(float& m, float& l, float* o, float m2, float l2,
@@ -221,6 +230,12 @@ attention_cluster_kernel(const float* q, const uint16_t* kc, const uint16_t* vc,
   __shared__ float wo[kNW][GM][D];
   __shared__ float cm[GM], cl[GM];     // this CTA's partial, read by rank 0
   __shared__ float co[GM][D];
+  // kPush: every CTA stores its partial into rank 0's slots instead (one
+  // cluster barrier, then rank 0 merges from its own shared memory) where
+  // the slots fit a small static budget
+  constexpr bool kPush = !OPROJ && MC * GM * (D + 2) * 4 <= 16384;
+  __shared__ float pm[kPush ? MC : 1][GM], pl[kPush ? MC : 1][GM];
+  __shared__ float po[kPush ? MC : 1][GM][D];
 
   tl_entry(fz.tl);
   attn_issue_prefetch(fz);
@@ -461,13 +476,50 @@ attention_cluster_kernel(const float* q, const uint16_t* kc, const uint16_t* vc,
         O = fmaf(vp[d], e, O);
       }
     }
-    co[h][d] = O;
-    if (d == 0) {
-      cm[h] = M;
-      cl[h] = Ls;
+    if constexpr (kPush) {
+      st_cluster(&po[s][h][d], O, 0);
+      if (d == 0) {
+        st_cluster(&pm[s][h], M, 0);
+        st_cluster(&pl[s][h], Ls, 0);
+      }
+    } else {
+      co[h][d] = O;
+      if (d == 0) {
+        cm[h] = M;
+        cl[h] = Ls;
+      }
     }
   }
-  cluster_sync();  // every CTA's partial is in its shared memory
+  cluster_sync();  // every CTA's partial is in place (kPush: in rank 0's slots)
+
+  if constexpr (kPush) {
+    // ---- rank 0 merges its slots in rank order (the same arithmetic as
+    // merge_cluster); the other CTAs are done
+    if (s == 0) {
+      for (int i = threadIdx.x; i < g * D; i += kThreads) {
+        const int h = i / D, d = i % D;
+        float M = -INFINITY;
+        for (unsigned j = 0; j < cs; ++j) M = fmaxf(M, pm[j][h]);
+        float Ls = 0.f, O = 0.f;
+        if (M != -INFINITY) {
+          for (unsigned j = 0; j < cs; ++j) {
+            if (pm[j][h] == -INFINITY) continue;
+            const float e = expf(pm[j][h] - M);
+            Ls = fmaf(pl[j][h], e, Ls);
+            O = fmaf(po[j][h][d], e, O);
+          }
+        }
+        const float res = (valid && Ls > 0.f) ? O / Ls : 0.f;
+        const size_t oi = ((size_t)b * H + kv * g + h) * D + d;
+        if (out_bf16)
+          reinterpret_cast<uint16_t*>(out)[oi] = f32_to_bf16_bits(res);
+        else
+          reinterpret_cast<float*>(out)[oi] = res;
+      }
+    }
+    tl_exit(fz.tl);
+    return;
+  }
 
   // ---- rank 0 merges the cluster's partials in rank order
   if (s == 0) {
