@@ -233,7 +233,7 @@ attention_cluster_kernel(const float* q, const uint16_t* kc, const uint16_t* vc,
   // kPush: every CTA stores its partial into rank 0's slots instead (one
   // cluster barrier, then rank 0 merges from its own shared memory) where
   // the slots fit a small static budget
-  constexpr bool kPush = !OPROJ && MC * GM * (D + 2) * 4 <= 16384;
+  constexpr bool kPush = !OPROJ && MC * GM * (D + 2) * 4 <= 20480;
   __shared__ float pm[kPush ? MC : 1][GM], pl[kPush ? MC : 1][GM];
   __shared__ float po[kPush ? MC : 1][GM][D];
 
