@@ -237,7 +237,7 @@ def test_qwen3_0_6b_step_whole_depth_bf16_cascade_bound():
     """Untethered 28-layer step against the oracle. The bf16 stores make
     the two sides take different roundings where a value sits within fp32
     noise of a bf16 midpoint, and those one-ulp differences compound from
-    layer to layer, so the per-element spec bound applies per layer
+    layer to layer, so the per-element bound (2e-3 + 1e-3 |ref|) applies per layer
     (test above); across the whole depth the logits must agree to a relative
     RMS error of 2e-2 (a few bf16 ulps, 2^-8 = 3.9e-3 each)."""
     cfg = dict(qg_synth.QWEN3_0_6B)
